@@ -1,0 +1,507 @@
+#!/usr/bin/env python
+"""Throughput of the KDA layer hot path on B200, one JSON line on rank 0.
+
+Headline workload (one step): prep + chunked prefill of one packed batch,
+B = 1, H = 32, T = 8192, d = 128, chunk 64, bf16 activations, fp32 state,
+A_log and dt_bias, seeded synthetic inputs resident in HBM.  Metric: prefill
+tokens/s.  At N = 1 the same line also carries the batched decode workload
+(B = 64, H = 32, d = 128, 1,024 steps after a 512-token prefill, CUDA graph)
+and the speculative verify + rollback workload (B = 16, blocks of 8 drafts
+after a 4,096-token context, 256 rounds, CUDA graph).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kda|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch of the
+same workload (weak scaling, no collective in the data path); the timing is
+the max over ranks.  ``--impl reference`` times the float64 CPU oracle.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+METRIC = 'KDA prefill tokens/s & decode tokens/s (1 B200) + % of TC / HBM roofline'
+SMI_FIELDS = ('index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,'
+              'clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,'
+              'clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap')
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument('--gpus', type=int, default=1)
+    ap.add_argument('--steps', type=int, default=200)
+    ap.add_argument('--warmup', type=int, default=5)
+    ap.add_argument('--impl', default='kda', choices=['kda', 'reference'])
+    ap.add_argument('--tokens', type=int, default=8192, help='prefill length (8192 = headline)')
+    ap.add_argument('--no-extras', action='store_true', help='skip decode / verify workloads')
+    ap.add_argument('--no-cpu', action='store_true', help='skip the CPU oracle baseline')
+    ap.add_argument('--only', default='', help='prefill|decode|verify: run one workload only')
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; no data-path collective)
+# ---------------------------------------------------------------------------
+class Dist:
+    def __init__(self):
+        import torch
+        self.world = int(os.environ.get('WORLD_SIZE', '1'))
+        self.rank = int(os.environ.get('RANK', '0'))
+        self.local = int(os.environ.get('LOCAL_RANK', '0'))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            backend = 'nccl' if torch.cuda.is_available() else 'gloo'
+            if backend == 'nccl':
+                torch.cuda.set_device(self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        import torch
+        dev = 'cuda' if torch.cuda.is_available() else 'cpu'
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.path = os.path.join(ROOT, 'gpurun_out', f'clocks_rank{gpu_index}.csv')
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, 'w')
+            self.proc = subprocess.Popen(
+                ['nvidia-smi', '-i', str(gpu_index), f'--query-gpu={SMI_FIELDS}',
+                 '--format=csv,noheader,nounits', '-lms', '50'],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(',')]
+            if len(parts) >= 9:
+                rows.append(parts)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace('.', '').isdigit()]
+        loaded = [float(r[3]) for r in rows if r[3].replace('.', '').isdigit()]
+        names = ['hw_slowdown', 'hw_thermal_slowdown', 'sw_thermal_slowdown', 'sw_power_cap']
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == 'Active'})
+        return {'sm_mhz': statistics.median(sm) if sm else None,
+                'sm_max_mhz': float(rows[0][2]) if rows[0][2].replace('.', '').isdigit() else None,
+                'reasons': reasons, 'samples': len(rows),
+                'power_w_max': max(loaded) if loaded else None}
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, 'MEASURED_PEAKS.json')) as fh:
+            p = json.load(fh)
+        return p['hbm_gbs'], p['bf16_tflops'], 'measured'
+    except Exception:
+        return 6650.0, 1590.0, 'fallback'
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+def prefill_workload(torch, kda, synth, T, seed, dev):
+    H, d, K = 32, 128, 4
+    cfg = kda.Config(num_heads=H, head_dim=d, conv_size=K, dtype=torch.bfloat16, chunk_size=64)
+    P = {k: v.to(dev) for k, v in synth.layer_params(seed, H, d, K).items()}
+    A_cpu = synth.layer_activations(seed, [T], H, d, torch.bfloat16)
+    A = {k: v.to(dev) for k, v in A_cpu.items()}
+    N = 1
+    out = {'q': torch.empty(T, H, d, dtype=cfg.dtype, device=dev),
+           'k': torch.empty(T, H, d, dtype=cfg.dtype, device=dev),
+           'v': torch.empty(T, H, d, dtype=cfg.dtype, device=dev),
+           'log_a': torch.empty(T, H, d, device=dev), 'beta': torch.empty(T, H, device=dev)}
+    y = torch.empty(T, H, d, dtype=cfg.dtype, device=dev)
+    state = torch.empty(N, H, d, d, device=dev)
+    ws = kda.prefill_workspace(cfg, N, T, dev)
+    return dict(cfg=cfg, P=P, A=A, A_cpu=A_cpu, out=out, y=y, state=state, ws=ws, T=T, H=H, d=d)
+
+
+def prefill_bytes(T, H, d):
+    """Algorithmic HBM bytes of prep and of prefill (bf16 activations, fp32 gates/state)."""
+    th = T * H
+    prep = th * (3 * d * 2 + d * 2 + 2) + th * (3 * d * 2 + d * 4 + 4)
+    prefill = th * (3 * d * 2 + d * 4 + 4 + d * 2) + th * d * 2 + H * d * d * 4
+    return prep, prefill
+
+
+def run_prefill(args, dist, torch, kda, synth, dev):
+    W = prefill_workload(torch, kda, synth, args.tokens, 1 + 1000 * dist.rank, dev)
+    cfg, P, A, out, y, state, ws = (W[k] for k in ('cfg', 'P', 'A', 'out', 'y', 'state', 'ws'))
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step(e=None):
+        if e:
+            e[0].record(stream)
+        kda.kda_prep(cfg, A['cu_seqlens'], A['x'], A['f'], A['beta_logit'], P['conv_w'],
+                     P['A_log'], P['dt_bias'], out=out)
+        if e:
+            e[1].record(stream)
+        kda.kda_prefill(cfg, A['cu_seqlens'], out['q'], out['k'], out['v'], out['log_a'],
+                        out['beta'], A['g'], P['norm_w'], state_out=state, y=y, workspace=ws)
+        if e:
+            e[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    sampler = ClockSampler(torch.cuda.current_device()) if dist.rank == 0 else None
+    torch.cuda.synchronize()
+    per = [[ev(), ev(), ev()] for _ in range(args.steps)]
+    t_start, t_end = ev(), ev()
+    wall0 = time.perf_counter()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(per[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms = t_start.elapsed_time(t_end)
+    # keep the GPU loaded (untimed) so the clock sampler sees at least ~1 s under load
+    while time.perf_counter() - wall0 < 1.0:
+        step()
+        torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    ms_prep = statistics.mean(p[0].elapsed_time(p[1]) for p in per)
+    ms_pref = statistics.mean(p[1].elapsed_time(p[2]) for p in per)
+    ms_max = dist.max(ms)
+    ms_step = ms_max / args.steps
+    T, H, d = W['T'], W['H'], W['d']
+    value = dist.world * T / (ms_step / 1e3)
+
+    # end to end through the same entry points with host buffers (pinned)
+    hx = {k: W['A_cpu'][k].pin_memory() for k in ('x', 'f', 'beta_logit', 'g')}
+    hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    hs = torch.empty(state.shape, dtype=state.dtype).pin_memory()
+    n_e2e = max(3, min(20, args.steps))
+
+    def e2e_step():
+        for k, h in hx.items():
+            A[k].copy_(h, non_blocking=True)
+        step()
+        hy.copy_(y, non_blocking=True)
+        hs.copy_(state, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = dist.max(e0.elapsed_time(e1)) / n_e2e
+    h2d = sum(t.numel() * t.element_size() for t in hx.values())
+    d2h = hy.numel() * hy.element_size() + hs.numel() * hs.element_size()
+
+    hbm, tc, peak_kind = measured_peaks()
+    b_prep, b_pref = prefill_bytes(T, H, d)
+    dominant = ('kda_prefill', b_pref, ms_pref) if ms_pref >= ms_prep else ('kda_prep', b_prep, ms_prep)
+    achieved = dominant[1] / (dominant[2] / 1e3) / 1e9
+    res = {
+        'metric': METRIC, 'value': value, 'unit': 'tokens/s', 'n_gpus': dist.world,
+        'steps': args.steps, 'warmup': args.warmup, 'ms_per_step': ms_step,
+        'higher_is_better': True, 'scaling': 'weak', 'vs_baseline': None, 'dtype': 'bf16',
+        'data': 'synthetic (seeded N(0,1) activations, random-init layer parameters)',
+        'config': {'workload': f'prefill B=1 H=32 T={T} d=128 chunk=64 (prep + chunked prefill)',
+                   'global_batch': dist.world, 'seq_len': T, 'heads': H, 'head_dim': d,
+                   'parallelism': f'replicas x{dist.world} (independent batches per GPU)',
+                   'l2': 'inputs larger than L2 (x alone is %.0f MB)' % (A['x'].numel() * 2 / 1e6)},
+        'e2e': {'value': dist.world * T / (e2e_ms / 1e3), 'unit': 'tokens/s',
+                'h2d_bytes_per_step': h2d, 'd2h_bytes_per_step': d2h,
+                'ms_per_step': e2e_ms},
+        'gpu_launches': 4 * args.steps,
+        'roofline': {'bound': 'hbm', 'kernel': dominant[0], 'achieved': achieved, 'peak': hbm,
+                     'unit': 'GB/s', 'frac': achieved / hbm, 'traffic': None,
+                     'peak_kind': peak_kind, 'algorithmic_bytes_per_launch': dominant[1]},
+        'breakdown_ms': {'kda_prep': ms_prep, 'kda_prefill': ms_pref},
+        'step_roofline': {'algorithmic_bytes': b_prep + b_pref,
+                          'achieved_gbs': (b_prep + b_pref) / (ms_step / 1e3) / 1e9,
+                          'frac': (b_prep + b_pref) / (ms_step / 1e3) / 1e9 / hbm},
+        'clocks': clocks,
+    }
+    del W
+    return res
+
+
+def run_decode(torch, kda, synth, dev, steps=1024):
+    """Batched decode: B=64, H=32, d=128, 512-token prefill then `steps` single-token steps."""
+    B, H, d, K, T0 = 64, 32, 128, 4, 512
+    cfg = kda.Config(num_heads=H, head_dim=d, conv_size=K, dtype=torch.bfloat16, chunk_size=64)
+    P = {k: v.to(dev) for k, v in synth.layer_params(2, H, d, K).items()}
+    A = {k: v.to(dev) for k, v in synth.layer_activations(2, [T0] * B, H, d, torch.bfloat16).items()}
+    state = torch.zeros(B, H, d, d, device=dev)
+    conv = torch.zeros(B, K - 1, H, 3 * d, dtype=cfg.dtype, device=dev)
+    kda.layer_prefill(cfg, P, A, state_in=state, state_out=state, conv_state=conv)
+    # step inputs: sequence b's `steps` tokens drawn as one sequence, laid out [step, b]
+    S = synth.layer_activations(2, [steps] * B, H, d, torch.bfloat16, tag='decode_steps')
+    X = {k: S[k].view(B, steps, *S[k].shape[1:]).transpose(0, 1).contiguous().to(dev)
+         for k in ('x', 'f', 'beta_logit', 'g')}
+    cu = torch.arange(B + 1, dtype=torch.int32, device=dev)
+    o = {'q': torch.empty(B, H, d, dtype=cfg.dtype, device=dev),
+         'k': torch.empty(B, H, d, dtype=cfg.dtype, device=dev),
+         'v': torch.empty(B, H, d, dtype=cfg.dtype, device=dev),
+         'log_a': torch.empty(B, H, d, device=dev), 'beta': torch.empty(B, H, device=dev)}
+    y = torch.empty(steps, B, H, d, dtype=cfg.dtype, device=dev)
+
+    def one(i):
+        kda.kda_prep(cfg, cu, X['x'][i], X['f'][i], X['beta_logit'][i], P['conv_w'], P['A_log'],
+                     P['dt_bias'], conv_state=conv, max_seqlen=1, out=o)
+        kda.kda_decode(cfg, o['q'], o['k'], o['v'], o['log_a'], o['beta'], X['g'][i],
+                       P['norm_w'], state, y=y[i])
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        one(0)                      # warm (also loads the kernels)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(steps):
+            one(i)
+    g.replay()                      # warm
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    # decode kernel alone: back-to-back launches on resident inputs
+    n = 200
+    for _ in range(3):
+        kda.kda_decode(cfg, o['q'], o['k'], o['v'], o['log_a'], o['beta'], X['g'][0],
+                       P['norm_w'], state, y=y[0])
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(n):
+        kda.kda_decode(cfg, o['q'], o['k'], o['v'], o['log_a'], o['beta'], X['g'][0],
+                       P['norm_w'], state, y=y[0])
+    e1.record()
+    torch.cuda.synchronize()
+    ms_k = e0.elapsed_time(e1) / n
+    bytes_k = B * H * (2 * d * d * 4 + 4 * d * 2 + d * 4 + 4 + d * 2)
+    hbm, _, peak_kind = measured_peaks()
+    ach = bytes_k / (ms_k / 1e3) / 1e9
+    del g
+    return {'value': B * steps / (ms / 1e3), 'unit': 'tokens/s',
+            'workload': f'decode B={B} H={H} d={d}, {steps} steps after a {T0}-token prefill '
+                        '(prep + decode per step, CUDA graph)',
+            'ms_per_step': ms / steps, 'gpu_launches': 2 * steps,
+            'roofline': {'bound': 'hbm', 'kernel': 'kda_decode', 'achieved': ach, 'peak': hbm,
+                         'unit': 'GB/s', 'frac': ach / hbm, 'traffic': None,
+                         'peak_kind': peak_kind, 'algorithmic_bytes_per_launch': bytes_k,
+                         'ms_per_launch': ms_k,
+                         'l2_note': 'state 134 MB is just above L2 (126 MB)'}}
+
+
+def run_verify(torch, kda, synth, dev, rounds=256):
+    """Speculative verify: B=16, H=32, d=128, 4,096-token context, blocks of 8, `rounds` rounds."""
+    B, H, d, K, T0, Tb = 16, 32, 128, 4, 4096, 8
+    cfg = kda.Config(num_heads=H, head_dim=d, conv_size=K, dtype=torch.bfloat16, chunk_size=64)
+    P = {k: v.to(dev) for k, v in synth.layer_params(3, H, d, K).items()}
+    A = {k: v.to(dev) for k, v in synth.layer_activations(3, [T0] * B, H, d, torch.bfloat16).items()}
+    state = torch.zeros(B, H, d, d, device=dev)
+    conv = torch.zeros(B, K - 1, H, 3 * d, dtype=cfg.dtype, device=dev)
+    kda.layer_prefill(cfg, P, A, state_in=state, state_out=state, conv_state=conv)
+    D = synth.layer_activations(3, [rounds * Tb] * B, H, d, torch.bfloat16, tag='drafts')
+    X = {k: D[k].view(B, rounds, Tb, *D[k].shape[1:]).transpose(0, 1).contiguous().to(dev)
+         for k in ('x', 'f', 'beta_logit', 'g')}
+    acc = synth.accepted_lengths(3, rounds, B, Tb).to(dev)
+    cu = (torch.arange(B + 1, dtype=torch.int32, device=dev) * Tb)
+    o = {'q': torch.empty(B * Tb, H, d, dtype=cfg.dtype, device=dev),
+         'k': torch.empty(B * Tb, H, d, dtype=cfg.dtype, device=dev),
+         'v': torch.empty(B * Tb, H, d, dtype=cfg.dtype, device=dev),
+         'log_a': torch.empty(B * Tb, H, d, device=dev), 'beta': torch.empty(B * Tb, H, device=dev)}
+    win = torch.empty(B * (Tb + K - 1), H, 3 * d, dtype=cfg.dtype, device=dev)
+    tape = torch.empty(B, Tb, H, d, d, device=dev)
+    y = torch.empty(B, Tb, H, d, dtype=cfg.dtype, device=dev)
+    v4 = lambda t, *tail: t.view(B, Tb, *tail)
+
+    def one(r):
+        kda.kda_prep(cfg, cu, X['x'][r].view(B * Tb, H, 3 * d), X['f'][r].view(B * Tb, H, d),
+                     X['beta_logit'][r].view(B * Tb, H), P['conv_w'], P['A_log'], P['dt_bias'],
+                     conv_state=conv, conv_mode=kda.KDA_CONV_TAPE, conv_window=win,
+                     max_seqlen=Tb, out=o)
+        kda.kda_verify(cfg, v4(o['q'], H, d), v4(o['k'], H, d), v4(o['v'], H, d),
+                       v4(o['log_a'], H, d), v4(o['beta'], H), X['g'][r], P['norm_w'], state,
+                       tape=tape, y=y)
+        kda.kda_rollback(cfg, acc[r], tape, state, conv_window=win, conv_state=conv)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        one(0)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for r in range(rounds):
+            one(r)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    n = 100
+    e0.record()
+    for _ in range(n):
+        kda.kda_verify(cfg, v4(o['q'], H, d), v4(o['k'], H, d), v4(o['v'], H, d),
+                       v4(o['log_a'], H, d), v4(o['beta'], H), X['g'][0], P['norm_w'], state,
+                       tape=tape, y=y)
+    e1.record()
+    torch.cuda.synchronize()
+    ms_k = e0.elapsed_time(e1) / n
+    bytes_k = B * H * (d * d * 4 + Tb * d * d * 4 + Tb * (4 * d * 2 + d * 4 + 4 + d * 2))
+    hbm, _, peak_kind = measured_peaks()
+    ach = bytes_k / (ms_k / 1e3) / 1e9
+    del g
+    return {'value': B * Tb * rounds / (ms / 1e3), 'unit': 'verified draft tokens/s',
+            'workload': f'verify+rollback B={B} H={H} d={d}, blocks of {Tb} after a {T0}-token '
+                        f'context, {rounds} rounds, accepted ~ U{{0..{Tb}}} (CUDA graph)',
+            'ms_per_round': ms / rounds, 'gpu_launches': 3 * rounds,
+            'roofline': {'bound': 'hbm', 'kernel': 'kda_verify', 'achieved': ach, 'peak': hbm,
+                         'unit': 'GB/s', 'frac': ach / hbm, 'traffic': None,
+                         'peak_kind': peak_kind, 'algorithmic_bytes_per_launch': bytes_k,
+                         'ms_per_launch': ms_k}}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline and reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(torch, synth, heads=32, tokens=2048, seed=1):
+    """Units for the oracle: each head of the headline workload over a token prefix."""
+    H, d, K = 32, 128, 4
+    P = synth.layer_params(seed, H, d, K)
+    A = synth.layer_activations(seed, [tokens], H, d, torch.bfloat16)
+    np64 = lambda t: t.to(torch.float64).numpy()
+    units = []
+    for h in range(heads):
+        units.append((np64(A['x'][:, h:h + 1]), np64(A['f'][:, h:h + 1]),
+                      np64(A['beta_logit'][:, h:h + 1]), np64(A['g'][:, h:h + 1]),
+                      np64(P['conv_w'][h:h + 1]), np64(P['A_log'][h:h + 1]),
+                      np64(P['dt_bias'][h:h + 1]), np64(P['norm_w']),
+                      A['cu_seqlens'].numpy()))
+    return units
+
+
+def cpu_baseline(torch, synth, heads=32, tokens=2048):
+    from oracle import baseline
+    units = oracle_sample(torch, synth, heads, tokens)
+    wall, workers = baseline.time_units(units)
+    token_heads = heads * tokens
+    return {'value': token_heads / 32 / wall, 'unit': 'tokens/s', 'cores': workers,
+            'kind': 'oracle',
+            'sample': f'float64 oracle layer (prep + token loop + gated RMSNorm) on {heads} of 32 '
+                      f'heads x the first {tokens} tokens of the headline workload, one head per '
+                      f'process; value scaled to whole tokens (all 32 heads)',
+            'wall_s': wall}
+
+
+def run_reference(args, dist):
+    if dist.rank != 0:
+        return None
+    import torch
+    from linear_attention_recurrence_09_b200 import synth
+    from oracle import baseline
+    units = oracle_sample(torch, synth, heads=32, tokens=256)
+    wall, workers = baseline.time_units(units[:1])          # warm
+    walls = []
+    for i in range(args.warmup + args.steps):
+        w, workers = baseline.time_units(units)
+        if i >= args.warmup:
+            walls.append(w)
+    tps = 256 / statistics.mean(walls)
+    cb = {'value': tps, 'unit': 'tokens/s', 'cores': workers, 'kind': 'oracle',
+          'sample': 'float64 oracle on all 32 heads x the first 256 tokens of the headline '
+                    'workload per step, one head per process'}
+    return {'impl': 'reference', 'metric': METRIC, 'value': tps, 'unit': 'tokens/s',
+            'n_gpus': dist.world, 'steps': args.steps, 'warmup': args.warmup,
+            'ms_per_step': statistics.mean(walls) * 1e3, 'higher_is_better': True,
+            'scaling': 'weak', 'vs_baseline': None, 'dtype': 'f64', 'data': 'synthetic',
+            'config': {'workload': 'prefill B=1 H=32 T=8192 d=128 (sampled: 256-token prefix)'},
+            'cpu_baseline': cb,
+            'e2e': {'value': tps, 'unit': 'tokens/s', 'h2d_bytes_per_step': 0,
+                    'd2h_bytes_per_step': 0}}
+
+
+def main():
+    args = parse_args()
+    dist = Dist()
+    try:
+        if args.impl == 'reference':
+            res = run_reference(args, dist)
+            if res is not None:
+                print(json.dumps(res))
+            return
+        import torch
+        from linear_attention_recurrence_09_b200 import kda, synth
+        if not torch.cuda.is_available():
+            raise SystemExit('bench.py needs a CUDA GPU (there is no CPU fallback)')
+        dev = torch.device('cuda', dist.local)
+        torch.cuda.set_device(dev)
+        kda.lib()
+        res = {}
+        if args.only in ('', 'prefill'):
+            res = run_prefill(args, dist, torch, kda, synth, dev)
+        if dist.world == 1 and not args.no_extras:
+            if args.only in ('', 'decode'):
+                res['decode'] = run_decode(torch, kda, synth, dev)
+            if args.only in ('', 'verify'):
+                res['verify'] = run_verify(torch, kda, synth, dev)
+        if dist.rank == 0 and dist.world == 1 and not args.no_cpu and args.only in ('', 'prefill'):
+            res['cpu_baseline'] = cpu_baseline(torch, synth)
+        if dist.rank == 0:
+            print(json.dumps(res))
+    finally:
+        dist.close()
+
+
+if __name__ == '__main__':
+    main()

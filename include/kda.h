@@ -1,0 +1,236 @@
+/*
+ * kda.h - C ABI of libkda.so: the Kimi Delta Attention (KDA) layer hot path on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (llama.cpp PR #27754 "model: add GLM-5-Next", KDA commit) is, per
+ * head h of width d (d_k = d_v = d), for each token t of a sequence:
+ *
+ *   prep   x~ = depthwise causal conv over q|k|v (one kernel, K taps), then SiLU
+ *          q = q~ / max(||q~||, l2_eps),  k = k~ / max(||k~||, l2_eps),  v = v~
+ *          log a_t = lb * sigmoid(exp(A_log[h]) * (f_t + dt_bias[h]))   (per key channel)
+ *          b_t = sigmoid(beta_logit_t)
+ *   state  S_t = (I - b_t k_t k_t^T) Diag(a_t) S_{t-1} + b_t k_t v_t^T   (S is d_k x d_v,
+ *          decay on the key axis; order: decay, delta update, read)
+ *   out    o_t = q_scale * S_t^T q_t
+ *          y_t = o_t / sqrt(mean(o_t^2) + norm_eps) * w * sigmoid(g_t)
+ *
+ * plus speculative verify (a block of draft tokens run from one state, with a
+ * per-step state tape) and rollback to any accepted prefix (dflash-mlx issue
+ * #63, "What the backend needs": rollback for the KDA recurrent state; PR
+ * #27754: the conv state is one contiguous block so it can be snapshotted).
+ *
+ * Conventions for every entry point
+ *  - Returns KDA_OK (0) or a kda_status code.  Every argument is checked on the
+ *    host BEFORE anything is launched; on an error nothing is launched and no
+ *    output is touched.
+ *  - Every pointer is caller-owned DEVICE memory (any allocator), except `cfg`
+ *    which is host memory.  The library allocates nothing, frees nothing and
+ *    keeps no state between calls.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *    stream) and the call returns without synchronising.  Launch failures are
+ *    reported as KDA_ERR_CUDA.
+ *  - Tensors are dense, row-major (last index fastest), with the shapes given
+ *    below.  Activations (x, f, beta_logit, g, q, k, v, y, conv state/window)
+ *    have the element type cfg->dtype; parameters, log decay, beta, recurrent
+ *    states and tapes are fp32.
+ *  - Every pointer must be 16-byte aligned (KDA_ERR_MISALIGNED otherwise).
+ *  - Packed (varlen) batches use cu_seqlens: int32 [n_seqs + 1], device,
+ *    non-decreasing, cu_seqlens[0] = 0, cu_seqlens[n_seqs] = total_tokens.
+ *    Sequence s owns token rows [cu_seqlens[s], cu_seqlens[s+1]).  The kernels
+ *    clamp every index they derive from it to [0, total_tokens], so a
+ *    malformed array cannot make them access memory out of bounds (its results
+ *    are then undefined).
+ *  - state_slots (optional, int32 [n_seqs], device) maps sequence s to row
+ *    state_slots[s] of a state pool of pool_size rows; NULL means row s.
+ *    Sequences whose slot lies outside [0, pool_size) are skipped.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+typedef struct CUstream_st* kda_stream_t; /* == cudaStream_t */
+
+enum kda_status {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad enum */
+  KDA_ERR_MISALIGNED = 2,   /* a pointer is not 16-byte aligned */
+  KDA_ERR_UNSUPPORTED = 3,  /* valid but not built: e.g. head_dim not in {16,32,64,128} */
+  KDA_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
+  KDA_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up (see kda_workspace_status) */
+  KDA_ERR_WORKSPACE = 6     /* workspace missing or smaller than kda_prefill_workspace_size */
+};
+
+enum kda_dtype { KDA_F32 = 0, KDA_BF16 = 1 };
+
+enum kda_conv_mode {
+  KDA_CONV_COMMIT = 0, /* conv_state <- last K-1 pre-conv rows of [conv_state; x] */
+  KDA_CONV_TAPE = 1    /* conv_state read only; conv_window <- [conv_state; x] */
+};
+
+/* Layer configuration (host memory, read during the call only). */
+typedef struct kda_config {
+  int32_t num_heads;      /* H >= 1 */
+  int32_t head_dim;       /* d = d_k = d_v in {16, 32, 64, 128} */
+  int32_t conv_size;      /* K taps of the short conv, 1..8 (4 in GLM-5.3-Flash) */
+  int32_t dtype;          /* enum kda_dtype of the activations */
+  int32_t chunk_size;     /* prefill chunk length in {16, 32, 64} */
+  float gate_lower_bound; /* lb of the bounded-sigmoid decay, in [-5, 0): PR #27754
+                             makes gate_lower_bound a required key; GLM-5.3-Flash uses -5 */
+  float l2_eps;           /* q/k L2 eps, 1e-6 ("a literal 1e-6", PR #27754) */
+  float norm_eps;         /* output RMSNorm eps, 1e-5 (rms_norm_eps, glm53-flash-mlx README) */
+  float q_scale;          /* multiplies o = S^T q; 1.0 */
+} kda_config;
+
+/* Human-readable name of a kda_status code (static string, never NULL). */
+KDA_API const char* kda_status_string(int status);
+
+/* ABI version of this header; bumped on any incompatible change. */
+KDA_API int kda_abi_version(void);
+
+/*
+ * kda_prep - fused short conv + SiLU + q/k L2 norm + decay gate + beta.
+ * PR #27754, KDA commit: q|k|v convolved as ONE depthwise kernel, SiLU after
+ * the conv, L2 eps a literal 1e-6 with max(sqrt(sum), eps), bounded-sigmoid
+ * decay with dt_bias per channel and per-head A broadcast; f and beta come
+ * from the pre-conv hidden states (separate inputs here).
+ *
+ *  max_seqlen  host hint: an upper bound on every sequence length, or 0 if
+ *              unknown.  When 1 <= max_seqlen <= 16 (decode, verify blocks) the
+ *              conv-state commit happens inside the main kernel; otherwise a
+ *              second small kernel does it.  A wrong non-zero hint leaves the
+ *              conv state of longer sequences undefined (never out of bounds).
+ *  x           [total_tokens, H, 3d]  pre-conv q|k|v, per head q(d) k(d) v(d)
+ *  f           [total_tokens, H, d]   decay-gate input
+ *  beta_logit  [total_tokens, H]
+ *  conv_w      fp32 [H, 3d, K]        tap K-1 multiplies the current token
+ *  A_log       fp32 [H]
+ *  dt_bias     fp32 [H, d]
+ *  conv_state  [pool_size, K-1, H, 3d] pre-conv history, oldest row first, or
+ *              NULL (history = zeros; then nothing is written back).  Rows of
+ *              sequence s are at state_slots[s] (or s).  In COMMIT mode it is
+ *              updated to the last K-1 rows of [history; x_s].
+ *  conv_mode   enum kda_conv_mode
+ *  conv_window TAPE mode only: [total_tokens + n_seqs*(K-1), H, 3d]; sequence s
+ *              occupies rows [cu[s] + s*(K-1), cu[s+1] + (s+1)*(K-1)) and gets
+ *              [history; x_s].  Ignored (may be NULL) in COMMIT mode.
+ *  q, k, v     out [total_tokens, H, d]  normalised q, k and SiLU'd v
+ *  log_a       out fp32 [total_tokens, H, d]
+ *  beta        out fp32 [total_tokens, H]
+ */
+KDA_API int kda_prep(const kda_config* cfg, int32_t n_seqs, int32_t total_tokens,
+             const int32_t* cu_seqlens, int32_t max_seqlen, const void* x, const void* f,
+             const void* beta_logit, const float* conv_w, const float* A_log,
+             const float* dt_bias, void* conv_state, const int32_t* state_slots,
+             int32_t pool_size, int32_t conv_mode, void* conv_window, void* q,
+             void* k, void* v, float* log_a, float* beta, kda_stream_t stream);
+
+/*
+ * Workspace bytes kda_prefill needs for this problem (0 on invalid arguments).
+ * The workspace holds the intra-chunk products handed from the chunk-parallel
+ * pass to the serial inter-chunk pass.
+ */
+KDA_API size_t kda_prefill_workspace_size(const kda_config* cfg, int32_t n_seqs,
+                                  int32_t total_tokens);
+
+/*
+ * kda_prefill - chunkwise-parallel prefill of packed sequences (chunk length
+ * cfg->chunk_size): an intra-chunk pass, parallel over (sequence, head,
+ * chunk), builds the UT/WY form of each chunk with a triangular solve; a
+ * serial inter-chunk pass carries the fp32 state on chip through the chunks
+ * of each sequence and applies the gated RMSNorm epilogue.  The result equals
+ * the token-by-token recurrence up to rounding.
+ *
+ *  q, k, v, log_a, beta   prep outputs (layouts as in kda_prep)
+ *  g          [total_tokens, H, d]   output-gate input (post projection)
+ *  norm_w     fp32 [d]               RMSNorm weight, shared by the heads
+ *  state_in   fp32 [pool_size, H, d, d] initial states (key axis = rows), or
+ *             NULL for zeros.  Row of sequence s: state_slots[s] (or s).
+ *  state_out  fp32 [pool_size, H, d, d] final states, or NULL to skip; may
+ *             equal state_in (updated in place).
+ *  y          out [total_tokens, H, d]
+ *  workspace  device scratch of at least kda_prefill_workspace_size() bytes,
+ *             256-byte aligned; its contents on entry do not matter.
+ */
+KDA_API int kda_prefill(const kda_config* cfg, int32_t n_seqs, int32_t total_tokens,
+                const int32_t* cu_seqlens, const void* q, const void* k,
+                const void* v, const float* log_a, const float* beta,
+                const void* g, const float* norm_w, const float* state_in,
+                float* state_out, const int32_t* state_slots, int32_t pool_size,
+                void* y, void* workspace, size_t workspace_bytes,
+                kda_stream_t stream);
+
+/*
+ * kda_decode - one token for each of `batch` sequences (the "fused operator"
+ * path of PR #27754: no chunking).  Streams each head's d x d fp32 state once:
+ * decay, both column reductions S^T k and S^T q in one pass, rank-1 update,
+ * one store, gated RMSNorm.
+ *
+ *  q, k, v, g [batch, H, d]; log_a fp32 [batch, H, d]; beta fp32 [batch, H]
+ *  state      fp32 [pool_size, H, d, d], updated in place (row state_slots[b] or b)
+ *  y          out [batch, H, d]
+ */
+KDA_API int kda_decode(const kda_config* cfg, int32_t batch, const void* q,
+               const void* k, const void* v, const float* log_a,
+               const float* beta, const void* g, const float* norm_w,
+               float* state, const int32_t* state_slots, int32_t pool_size,
+               void* y, kda_stream_t stream);
+
+/*
+ * kda_verify - speculative verify of a block of `block_len` draft tokens per
+ * sequence (1..16; the DFlash2 drafter of dflash-mlx issue #63 uses 8).  Runs
+ * the decode step block_len times from one load of each state, keeps the live
+ * state untouched, and writes the state after every step to the tape, so that
+ * rollback to any accepted prefix is a copy.
+ *
+ *  q, k, v, g [batch, block_len, H, d]; log_a fp32 [batch, block_len, H, d];
+ *  beta fp32 [batch, block_len, H]
+ *  state      fp32 [pool_size, H, d, d], read only
+ *  tape       out fp32 [batch, block_len, H, d, d]: tape[b, j] = state after draft j
+ *  y          out [batch, block_len, H, d]
+ */
+KDA_API int kda_verify(const kda_config* cfg, int32_t batch, int32_t block_len,
+               const void* q, const void* k, const void* v, const float* log_a,
+               const float* beta, const void* g, const float* norm_w,
+               const float* state, const int32_t* state_slots, int32_t pool_size,
+               float* tape, void* y, kda_stream_t stream);
+
+/*
+ * kda_rollback - commit the accepted prefix of a verified block.
+ * For sequence b with L = accepted[b] (device int32 [batch], clamped to
+ * [0, block_len]): L = 0 leaves state and conv state untouched; otherwise
+ * state <- tape[b, L-1] and conv_state <- conv_window rows [L, L+K-1) of
+ * sequence b.  Bit-exact copies.  conv_window is kda_prep's TAPE output for
+ * the block ([batch, K-1+block_len, H, 3d]); conv_state / conv_window may be
+ * NULL together to roll back only the recurrent state.
+ */
+KDA_API int kda_rollback(const kda_config* cfg, int32_t batch, int32_t block_len,
+                 const int32_t* accepted, const float* tape,
+                 const void* conv_window, float* state, void* conv_state,
+                 const int32_t* state_slots, int32_t pool_size,
+                 kda_stream_t stream);
+
+/*
+ * kda_workspace_status - synchronises `stream`, then reads the status word
+ * the prefill kernels keep at the start of `workspace`.  Returns KDA_OK, or
+ * KDA_ERR_TIMEOUT when a bounded device wait of the last kda_prefill on this
+ * workspace gave up (its outputs are then invalid).
+ */
+KDA_API int kda_workspace_status(const void* workspace, kda_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

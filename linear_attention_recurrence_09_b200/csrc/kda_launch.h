@@ -1,0 +1,101 @@
+// Internal launch interface between the C ABI (kda_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kda {
+
+struct PrepArgs {
+  const int32_t* cu;
+  int n_seqs, total, H, D, K;
+  bool bf16;
+  const void* x;
+  const void* f;
+  const void* beta_logit;
+  const float* conv_w;
+  const float* A_log;
+  const float* dt_bias;
+  void* conv_state;
+  const int32_t* slots;
+  int pool_size;
+  int mode;  // 0 commit, 1 tape
+  int commit_in_kernel;
+  void* window;
+  void* q;
+  void* k;
+  void* v;
+  float* loga;
+  float* beta;
+  float lb, l2_eps;
+};
+
+struct StepArgs {  // decode (T = 1) and verify (T = block_len)
+  int B, T, H, D;
+  bool bf16;
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* loga;
+  const float* beta;
+  const void* g;
+  const float* norm_w;
+  const float* state_in;
+  float* state_out;  // decode: == state_in; verify: nullptr
+  float* tape;       // verify only
+  const int32_t* slots;
+  int pool_size;
+  void* y;
+  float norm_eps, q_scale;
+};
+
+struct RollbackArgs {
+  int B, T, H, D, K;
+  bool bf16;
+  const int32_t* accepted;
+  const float* tape;
+  const void* window;
+  float* state;
+  void* conv_state;
+  const int32_t* slots;
+  int pool_size;
+};
+
+// Workspace of the chunked prefill (byte offsets from its base, 256-aligned).
+struct PrefillLayout {
+  size_t status, W, Ut, Qt, Kp, o, M, gC, total;
+  int nslots;
+  size_t wsize;  // bytes per workspace element (4 fp32 / 2 bf16)
+};
+PrefillLayout prefill_layout(int n_seqs, int total, int H, int D, int C, bool bf16);
+
+struct PrefillArgs {
+  const int32_t* cu;
+  int n_seqs, total, H, D, C;
+  bool bf16;
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* loga;
+  const float* beta;
+  const void* g;
+  const float* norm_w;
+  const float* state_in;
+  float* state_out;
+  const int32_t* slots;
+  int pool_size;
+  void* y;
+  char* ws;
+  PrefillLayout L;
+  float norm_eps, q_scale, lb;
+};
+
+cudaError_t launch_prep(const PrepArgs& a, cudaStream_t st);
+cudaError_t launch_step(const StepArgs& a, cudaStream_t st);
+cudaError_t launch_rollback(const RollbackArgs& a, cudaStream_t st);
+cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st);
+int prep_tile();
+int prep_kmax();
+
+}  // namespace kda

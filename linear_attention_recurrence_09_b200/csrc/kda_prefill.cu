@@ -1,0 +1,393 @@
+// kda_prefill, generic path (SIMT fp32 arithmetic, any supported d and chunk).
+//
+// Chunkwise form of the KDA recurrence (the "chunked fallback" class of
+// llama.cpp PR #27754, written here from the delta-rule UT/WY transform of
+// DeltaNet's chunkwise algorithm with the per-channel decay of gated linear
+// attention).  For a chunk of C tokens starting from state S, with
+// G_r = sum_{i<=r} log a_i per key channel:
+//   A[r,i] = b_r sum_c k_r k_i e^{G_r - G_i}  (i < r),  M[r,i] = q_scale sum_c q_r k_i e^{G_r - G_i}  (i <= r)
+//   W = (I + A)^{-1} diag(b) (K * e^G),  U~ = (I + A)^{-1} diag(b) V
+//   U = U~ - W S,   O = (q_scale Q * e^G) S + M U,   S <- Diag(e^{G_C}) S + (K * e^{G_C - G})^T U
+//
+// Pass 1 (intra_chunk_kernel) is parallel over (chunk, head): it writes W, U~,
+// Q~ = q_scale Q e^G, K' = K e^{G_C - G}, M and e^{G_C} to the workspace.
+// Pass 2 (inter_chunk_kernel) is serial over the chunks of each sequence and
+// parallel over (value-column slice, head, sequence); it keeps its slice of the
+// fp32 state in shared memory and writes o.  Pass 3 applies the gated RMSNorm.
+//
+// Range of the exponentials.  The gate keeps each log a in [lb, 0] with
+// lb >= -5, so over a sub-chunk of 16 tokens a cumulative decay spans at most
+// 80 < 88 (the fp32 exp overflow bound).  The gram terms e^{G_r - G_i} are
+// therefore split at the start of the row's sub-chunk:
+//   e^{G_r - G_i} = e^{G_r - G_ref} * e^{G_ref - G_i},  G_ref = G at the row before it,
+// where the first factor is <= 1 and the second is <= e^80.  Every other
+// exponential in the chunk form has a non-positive argument and may only
+// underflow, which is exact to within fp32.
+#include "kda_common.cuh"
+#include "kda_launch.h"
+
+namespace kda {
+
+constexpr int SUB = 16;      // sub-chunk length bounding the exponent span
+constexpr int P2_J = 16;     // value columns per inter-chunk CTA
+
+static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+PrefillLayout prefill_layout(int n_seqs, int total, int H, int D, int C, bool bf16) {
+  PrefillLayout L;
+  L.wsize = bf16 ? 2 : 4;
+  const size_t per_tok = (size_t)total * H * D;
+  L.nslots = num_slots(total, n_seqs, C);
+  size_t off = 0;
+  L.status = off; off += 256;
+  L.W = off; off += align256(per_tok * L.wsize);
+  L.Ut = off; off += align256(per_tok * L.wsize);
+  L.Qt = off; off += align256(per_tok * L.wsize);
+  L.Kp = off; off += align256(per_tok * L.wsize);
+  L.o = off; off += align256(per_tok * 4);
+  L.M = off; off += align256((size_t)L.nslots * H * C * C * L.wsize);
+  L.gC = off; off += align256((size_t)L.nslots * H * D * 4);
+  L.total = off;
+  return L;
+}
+
+// ---------------------------------------------------------------------------
+// pass 1: intra-chunk (parallel over chunk x head)
+// ---------------------------------------------------------------------------
+template <int D, int C>
+struct P1Smem {
+  static constexpr int KC_LD = D + 1;  // padded row stride: conflict-free column walks
+  static constexpr int A_LD = C + 1;
+  static constexpr size_t bytes =
+      sizeof(float) * (4 * C * D + C * KC_LD + C * A_LD + C);
+};
+
+template <typename T, typename WT, int D, int C>
+__global__ void __launch_bounds__(256) intra_chunk_kernel(const PrefillArgs a) {
+  using SM = P1Smem<D, C>;
+  extern __shared__ __align__(16) float smem[];
+  float* G = smem;                 // [C][D] cumulative log decay
+  float* Kr = G + C * D;           // [C][D] k
+  float* Kb = Kr + C * D;          // [C][D] k_r e^{G_r - G_ref(r)}
+  float* Qb = Kb + C * D;          // [C][D] q_scale q_r e^{G_r - G_ref(r)}
+  float* Kc = Qb + C * D;          // [C][KC_LD] k_i e^{G_ref(R) - G_i} for the current R
+  float* A = Kc + C * SM::KC_LD;   // [C][A_LD]
+  float* bs = A + C * SM::A_LD;    // [C]
+
+  const int h = blockIdx.y, H = a.H;
+  const int slot = blockIdx.x;
+  const TileRange tr = slot_to_tile(a.cu, a.n_seqs, a.total, C, slot);
+  if (tr.len == 0) return;
+  if (pool_row(a.slots, tr.seq, a.pool_size) < 0) return;
+  const int L = tr.len, t0 = tr.t0, tid = threadIdx.x;
+  const T* __restrict__ qg = static_cast<const T*>(a.q);
+  const T* __restrict__ kg = static_cast<const T*>(a.k);
+  const T* __restrict__ vg = static_cast<const T*>(a.v);
+  WT* Wo = reinterpret_cast<WT*>(a.ws + a.L.W);
+  WT* Uo = reinterpret_cast<WT*>(a.ws + a.L.Ut);
+  WT* Qo = reinterpret_cast<WT*>(a.ws + a.L.Qt);
+  WT* Ko = reinterpret_cast<WT*>(a.ws + a.L.Kp);
+  WT* Mo = reinterpret_cast<WT*>(a.ws + a.L.M) + ((size_t)slot * H + h) * C * C;
+  float* gCo = reinterpret_cast<float*>(a.ws + a.L.gC) + ((size_t)slot * H + h) * D;
+
+  for (int e = tid; e < C * D; e += blockDim.x) {
+    const int r = e / D, c = e - (e / D) * D;
+    float la = 0.f, kk = 0.f, qq = 0.f;
+    if (r < L) {
+      const size_t idx = ((size_t)(t0 + r) * H + h) * D + c;
+      la = __ldg(a.loga + idx);
+      kk = ld1(kg + idx);
+      qq = ld1(qg + idx);
+    }
+    G[e] = la; Kr[e] = kk; Qb[e] = qq;
+  }
+  for (int r = tid; r < C; r += blockDim.x)
+    bs[r] = (r < L) ? __ldg(a.beta + (size_t)(t0 + r) * H + h) : 0.f;
+  __syncthreads();
+
+  // cumulative log decay per key channel (padded rows add 0)
+  for (int c = tid; c < D; c += blockDim.x) {
+    float acc = 0.f;
+    for (int r = 0; r < C; ++r) { acc += G[r * D + c]; G[r * D + c] = acc; }
+  }
+  __syncthreads();
+
+  // row-scaled operands and the per-token outputs Q~, K'
+  for (int e = tid; e < C * D; e += blockDim.x) {
+    const int r = e / D, c = e - (e / D) * D;
+    const float g = G[e];
+    const int R = r / SUB;
+    const float ref = (R == 0) ? 0.f : G[(R * SUB - 1) * D + c];
+    const float er = __expf(g - ref);
+    const float kk = Kr[e], qq = Qb[e];
+    Kb[e] = kk * er;
+    Qb[e] = a.q_scale * qq * er;
+    if (r < L) {
+      const size_t idx = ((size_t)(t0 + r) * H + h) * D + c;
+      st1(Qo + idx, a.q_scale * qq * __expf(g));
+      st1(Ko + idx, kk * __expf(G[(C - 1) * D + c] - g));
+    }
+  }
+  for (int c = tid; c < D; c += blockDim.x) gCo[c] = __expf(G[(C - 1) * D + c]);
+  __syncthreads();
+
+  // gram blocks, one row sub-chunk R at a time
+  for (int R = 0; R < C / SUB; ++R) {
+    const int ncol = (R + 1) * SUB;
+    for (int e = tid; e < ncol * D; e += blockDim.x) {
+      const int i = e / D, c = e - (e / D) * D;
+      const float ref = (R == 0) ? 0.f : G[(R * SUB - 1) * D + c];
+      Kc[i * SM::KC_LD + c] = Kr[i * D + c] * __expf(ref - G[i * D + c]);
+    }
+    __syncthreads();
+    for (int p = tid; p < SUB * ncol; p += blockDim.x) {
+      const int r = R * SUB + p / ncol, i = p - (p / ncol) * ncol;
+      float am = 0.f, mm = 0.f;
+      if (i <= r) {
+        const float* kb = Kb + r * D;
+        const float* qb = Qb + r * D;
+        const float* kc = Kc + i * SM::KC_LD;
+#pragma unroll 8
+        for (int c = 0; c < D; ++c) {
+          am = fmaf(kb[c], kc[c], am);
+          mm = fmaf(qb[c], kc[c], mm);
+        }
+      }
+      A[r * SM::A_LD + i] = (i < r) ? bs[r] * am : 0.f;
+      st1(Mo + r * C + i, mm);
+    }
+    for (int p = tid; p < SUB * (C - ncol); p += blockDim.x) {
+      const int r = R * SUB + p / (C - ncol), i = ncol + p % (C - ncol);
+      A[r * SM::A_LD + i] = 0.f;
+      st1(Mo + r * C + i, 0.f);
+    }
+    __syncthreads();
+  }
+
+  // forward substitution (I + A) X = diag(b) B for B = K e^G (m = 0) and V (m = 1);
+  // each thread owns one column of one right-hand side, so no barrier is needed
+  if (tid < 2 * D) {
+    const int m = tid / D, c = tid - (tid / D) * D;
+    WT* out = (m == 0) ? Wo : Uo;
+    float xcol[C];
+#pragma unroll
+    for (int r = 0; r < C; ++r) {
+      float brc;
+      if (m == 0) {
+        brc = Kr[r * D + c] * __expf(G[r * D + c]);
+      } else {
+        brc = (r < L) ? ld1(vg + ((size_t)(t0 + r) * H + h) * D + c) : 0.f;
+      }
+      float acc = bs[r] * brc;
+#pragma unroll
+      for (int i = 0; i < r; ++i) acc = fmaf(-A[r * SM::A_LD + i], xcol[i], acc);
+      xcol[r] = acc;
+      if (r < L) st1(out + ((size_t)(t0 + r) * H + h) * D + c, acc);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// pass 2: inter-chunk (serial over chunks; parallel over value slice x head x sequence)
+// ---------------------------------------------------------------------------
+template <typename WT, int D, int C>
+struct P2Smem {
+  static constexpr size_t tiles = sizeof(WT) * (3 * C * D + C * C);
+  static constexpr size_t floats = sizeof(float) * (2 * C * P2_J + D * P2_J + D);
+  static constexpr size_t bytes = ((tiles + 15) / 16) * 16 + floats;
+};
+
+template <typename WT>
+__device__ __forceinline__ void copy_rows(WT* dst, const WT* src, int rows, int valid, int D,
+                                          size_t row_stride) {
+  // rows x D elements, row r at src + r * row_stride; rows >= valid are zero
+  constexpr int V = 16 / sizeof(WT);
+  const int per_row = D / V;
+  for (int e = threadIdx.x; e < rows * per_row; e += blockDim.x) {
+    const int r = e / per_row, c = (e - r * per_row) * V;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (r < valid) val = *reinterpret_cast<const uint4*>(src + r * row_stride + c);
+    *reinterpret_cast<uint4*>(dst + r * D + c) = val;
+  }
+}
+
+template <typename WT, int D, int C>
+__global__ void __launch_bounds__(256) inter_chunk_kernel(const PrefillArgs a) {
+  using SM = P2Smem<WT, D, C>;
+  constexpr int J = P2_J;
+  constexpr int RPT = C / 16;   // rows of U / O per thread
+  constexpr int SPT = D / 16;   // state rows per thread
+  extern __shared__ __align__(16) unsigned char smraw[];
+  WT* Wt = reinterpret_cast<WT*>(smraw);   // [C][D]
+  WT* Qt = Wt + C * D;                     // [C][D]
+  WT* Kp = Qt + C * D;                     // [C][D]
+  WT* Mt = Kp + C * D;                     // [C][C]
+  float* Ut = reinterpret_cast<float*>(smraw + ((SM::tiles + 15) / 16) * 16);  // [C][J]
+  float* U = Ut + C * J;                   // [C][J]
+  float* S = U + C * J;                    // [D][J]
+  float* gC = S + D * J;                   // [D]
+
+  const int j0 = blockIdx.x * J, h = blockIdx.y, s = blockIdx.z, H = a.H;
+  const int row = pool_row(a.slots, s, a.pool_size);
+  if (row < 0) return;
+  const int tid = threadIdx.x, j = tid % 16, rg = tid / 16;
+  int start, end;
+  seq_range(a.cu, a.total, s, start, end);
+
+  const WT* Wg = reinterpret_cast<const WT*>(a.ws + a.L.W);
+  const WT* Ug = reinterpret_cast<const WT*>(a.ws + a.L.Ut);
+  const WT* Qg = reinterpret_cast<const WT*>(a.ws + a.L.Qt);
+  const WT* Kg = reinterpret_cast<const WT*>(a.ws + a.L.Kp);
+  const WT* Mg = reinterpret_cast<const WT*>(a.ws + a.L.M);
+  const float* gCg = reinterpret_cast<const float*>(a.ws + a.L.gC);
+  float* og = reinterpret_cast<float*>(a.ws + a.L.o);
+
+  const size_t sbase = ((size_t)row * H + h) * D * D;
+  for (int e = tid; e < D * J; e += blockDim.x) {
+    const int c = e / J, jj = e - (e / J) * J;
+    S[e] = a.state_in ? a.state_in[sbase + (size_t)c * D + j0 + jj] : 0.f;
+  }
+
+  const int nch = (end - start + C - 1) / C;
+  for (int ci = 0; ci < nch; ++ci) {
+    const int slot = start / C + s + ci;
+    const int t0 = start + ci * C;
+    const int L = min(C, end - t0);
+    const size_t rstride = (size_t)H * D;
+    const size_t tok0 = ((size_t)t0 * H + h) * D;
+    copy_rows(Wt, Wg + tok0, C, L, D, rstride);
+    copy_rows(Qt, Qg + tok0, C, L, D, rstride);
+    copy_rows(Kp, Kg + tok0, C, L, D, rstride);
+    copy_rows(Mt, Mg + ((size_t)slot * H + h) * C * C, C, C, C, (size_t)C);
+    for (int e = tid; e < C * J; e += blockDim.x) {
+      const int r = e / J, jj = e - (e / J) * J;
+      Ut[e] = (r < L) ? ld1(Ug + tok0 + (size_t)r * rstride + j0 + jj) : 0.f;
+    }
+    for (int c = tid; c < D; c += blockDim.x) gC[c] = gCg[((size_t)slot * H + h) * D + c];
+    __syncthreads();
+
+    // U = U~ - W S
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) {
+      const int r = rg + 16 * m;
+      float acc = Ut[r * J + j];
+      for (int c = 0; c < D; ++c) acc = fmaf(-ld1(Wt + r * D + c), S[c * J + j], acc);
+      U[r * J + j] = acc;
+    }
+    __syncthreads();
+
+    // O = Q~ S + M U
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) {
+      const int r = rg + 16 * m;
+      float acc = 0.f;
+      for (int c = 0; c < D; ++c) acc = fmaf(ld1(Qt + r * D + c), S[c * J + j], acc);
+      for (int i = 0; i <= r; ++i) acc = fmaf(ld1(Mt + r * C + i), U[i * J + j], acc);
+      if (r < L) og[tok0 + (size_t)r * rstride + j0 + j] = acc;
+    }
+    // S <- Diag(e^{G_C}) S + K'^T U
+    float snew[SPT];
+#pragma unroll
+    for (int m = 0; m < SPT; ++m) {
+      const int c = rg + 16 * m;
+      float acc = gC[c] * S[c * J + j];
+      for (int r = 0; r < C; ++r) acc = fmaf(ld1(Kp + r * D + c), U[r * J + j], acc);
+      snew[m] = acc;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < SPT; ++m) S[(rg + 16 * m) * J + j] = snew[m];
+    __syncthreads();
+  }
+
+  if (a.state_out) {
+    for (int e = tid; e < D * J; e += blockDim.x) {
+      const int c = e / J, jj = e - (e / J) * J;
+      a.state_out[sbase + (size_t)c * D + j0 + jj] = S[e];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// pass 3: y = o / sqrt(mean(o^2) + eps) * w * sigmoid(g), one warp per (token, head)
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(256) gated_norm_kernel(const PrefillArgs a) {
+  const size_t rowi = (size_t)blockIdx.x * 8 + threadIdx.x / 32;
+  if (rowi >= (size_t)a.total * a.H) return;
+  const int lane = threadIdx.x & 31;
+  const float* o = reinterpret_cast<const float*>(a.ws + a.L.o) + rowi * D;
+  const T* g = static_cast<const T*>(a.g) + rowi * D;
+  T* y = static_cast<T*>(a.y) + rowi * D;
+  constexpr int PER = (D + 31) / 32;
+  float ov[PER];
+  float ss = 0.f;
+#pragma unroll
+  for (int m = 0; m < PER; ++m) {
+    const int c = lane + 32 * m;
+    ov[m] = (c < D) ? o[c] : 0.f;
+    ss = fmaf(ov[m], ov[m], ss);
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  const float rstd = rsqrtf(ss / (float)D + a.norm_eps);
+#pragma unroll
+  for (int m = 0; m < PER; ++m) {
+    const int c = lane + 32 * m;
+    if (c < D) st1(y + c, ov[m] * rstd * __ldg(a.norm_w + c) * sigmoid(ld1(g + c)));
+  }
+}
+
+template <typename T, int D, int C>
+static cudaError_t launch_prefill_dc(const PrefillArgs& a, cudaStream_t st) {
+  cudaError_t e;
+  {
+    auto k1 = intra_chunk_kernel<T, T, D, C>;
+    const size_t sm = P1Smem<D, C>::bytes;
+    e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    k1<<<dim3(a.L.nslots, a.H), 256, sm, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  {
+    auto k2 = inter_chunk_kernel<T, D, C>;
+    const size_t sm = P2Smem<T, D, C>::bytes;
+    e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    k2<<<dim3(D / P2_J, a.H, a.n_seqs), 256, sm, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (a.total > 0) {
+    const size_t rows = (size_t)a.total * a.H;
+    gated_norm_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+template <typename T, int D>
+static cudaError_t launch_prefill_d(const PrefillArgs& a, cudaStream_t st) {
+  switch (a.C) {
+    case 16: return launch_prefill_dc<T, D, 16>(a, st);
+    case 32: return launch_prefill_dc<T, D, 32>(a, st);
+    case 64: return launch_prefill_dc<T, D, 64>(a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <typename T>
+static cudaError_t launch_prefill_t(const PrefillArgs& a, cudaStream_t st) {
+  switch (a.D) {
+    case 16: return launch_prefill_d<T, 16>(a, st);
+    case 32: return launch_prefill_d<T, 32>(a, st);
+    case 64: return launch_prefill_d<T, 64>(a, st);
+    case 128: return launch_prefill_d<T, 128>(a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st) {
+  return a.bf16 ? launch_prefill_t<__nv_bfloat16>(a, st) : launch_prefill_t<float>(a, st);
+}
+
+}  // namespace kda

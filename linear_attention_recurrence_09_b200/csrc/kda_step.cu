@@ -1,0 +1,196 @@
+// kda_decode / kda_verify / kda_rollback: the token-at-a-time path.
+//
+// The "fused operator" for the delta net of llama.cpp PR #27754 (backends that
+// have it skip the chunked graph for generation): per (sequence, head) the
+// d x d fp32 state is read once, decayed along the key axis, reduced twice in
+// the same pass (S^T k and S^T q), updated by a rank-1 write and stored once.
+// Verify runs that step block_len times from one load of the state and writes
+// the state after every step to a tape (speculative verify of a DFlash2 block,
+// dflash-mlx issue #63); rollback is a copy out of that tape.
+//
+// HBM-bound: the state is 64 KB per head at d = 128, so one CTA per
+// (head, sequence) keeps its whole state in registers (16 float4 per thread
+// at 256 threads) with 16-byte coalesced loads and stores, and the two column
+// reductions go through shared memory across the 8 row groups.
+#include "kda_common.cuh"
+#include "kda_launch.h"
+
+namespace kda {
+
+template <int D>
+struct StepShape {
+  static constexpr int CG = D / 4;                                // column groups of 4
+  static constexpr int RG = (256 / CG < D) ? 256 / CG : D;        // row groups
+  static constexpr int ROWS = D / RG;                             // rows per thread
+  static constexpr int THREADS = CG * RG;
+  static constexpr int NW = (THREADS + 31) / 32;
+};
+
+__device__ __forceinline__ float4 f4_scale(float4 a, float s) {
+  return make_float4(a.x * s, a.y * s, a.z * s, a.w * s);
+}
+__device__ __forceinline__ float4 f4_fma(float s, float4 a, float4 acc) {
+  return make_float4(fmaf(s, a.x, acc.x), fmaf(s, a.y, acc.y), fmaf(s, a.z, acc.z),
+                     fmaf(s, a.w, acc.w));
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(StepShape<D>::THREADS)
+step_kernel(const StepArgs a) {
+  using SH = StepShape<D>;
+  constexpr int CG = SH::CG, RG = SH::RG, ROWS = SH::ROWS, THREADS = SH::THREADS;
+  __shared__ __align__(16) float ks[D];
+  __shared__ __align__(16) float qs[D];
+  __shared__ __align__(16) float as_[D];
+  __shared__ __align__(16) float us[D];
+  __shared__ __align__(16) float redk[RG][D];
+  __shared__ __align__(16) float redq[RG][D];
+  __shared__ float ssq[SH::NW];
+  __shared__ float kq_s;
+
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int H = a.H;
+  const int row = pool_row(a.slots, b, a.pool_size);
+  if (row < 0) return;
+  const int tid = threadIdx.x, cg = tid % CG, rg = tid / CG;
+  const int lane = tid & 31, warp = tid >> 5;
+  const T* __restrict__ qg = static_cast<const T*>(a.q);
+  const T* __restrict__ kg = static_cast<const T*>(a.k);
+  const T* __restrict__ vg = static_cast<const T*>(a.v);
+  const T* __restrict__ gg = static_cast<const T*>(a.g);
+  T* __restrict__ yg = static_cast<T*>(a.y);
+
+  const float* Sg = a.state_in + ((size_t)row * H + h) * D * D;
+  float4 S[ROWS];
+#pragma unroll
+  for (int i = 0; i < ROWS; ++i) S[i] = ld4(Sg + (size_t)(rg + i * RG) * D + 4 * cg);
+
+  for (int t = 0; t < a.T; ++t) {
+    const size_t tok = (size_t)b * a.T + t;
+    const size_t base = (tok * H + h) * D;
+    for (int c = tid; c < D; c += THREADS) {
+      ks[c] = ld1(kg + base + c);
+      qs[c] = ld1(qg + base + c);
+      as_[c] = expf(__ldg(a.loga + base + c));
+    }
+    __syncthreads();
+
+    // decay along the key axis, then both column reductions in one pass
+    float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+#pragma unroll
+    for (int i = 0; i < ROWS; ++i) {
+      const int r = rg + i * RG;
+      S[i] = f4_scale(S[i], as_[r]);
+      pk = f4_fma(ks[r], S[i], pk);
+      pq = f4_fma(qs[r], S[i], pq);
+    }
+    *reinterpret_cast<float4*>(&redk[rg][4 * cg]) = pk;
+    *reinterpret_cast<float4*>(&redq[rg][4 * cg]) = pq;
+    if (warp == 0) {
+      float p = 0.f;
+      for (int c = lane; c < D; c += 32) p = fmaf(ks[c], qs[c], p);
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
+      if (lane == 0) kq_s = p;
+    }
+    __syncthreads();
+
+    // per value column: u = b (v - S^T k), o = S^T q + u (k.q), RMSNorm partials
+    float o = 0.f;
+    if (tid < D) {
+      float rk = 0.f, rq = 0.f;
+#pragma unroll
+      for (int j = 0; j < RG; ++j) { rk += redk[j][tid]; rq += redq[j][tid]; }
+      const float bt = __ldg(a.beta + tok * H + h);
+      const float u = bt * (ld1(vg + base + tid) - rk);
+      o = a.q_scale * fmaf(u, kq_s, rq);
+      us[tid] = u;
+    }
+    if (warp < (D + 31) / 32) {
+      float p = o * o;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
+      if (lane == 0) ssq[warp] = p;
+    }
+    __syncthreads();
+
+    // rank-1 write and the gated RMSNorm epilogue
+#pragma unroll
+    for (int i = 0; i < ROWS; ++i) {
+      const int r = rg + i * RG;
+      S[i] = f4_fma(ks[r], *reinterpret_cast<const float4*>(&us[4 * cg]), S[i]);
+    }
+    if (tid < D) {
+      float ss = 0.f;
+#pragma unroll
+      for (int w = 0; w < (D + 31) / 32; ++w) ss += ssq[w];
+      const float rstd = rsqrtf(ss / (float)D + a.norm_eps);
+      const float gt = ld1(gg + base + tid);
+      st1(yg + base + tid, o * rstd * __ldg(a.norm_w + tid) * sigmoid(gt));
+    }
+    if (a.tape != nullptr) {
+      float* tp = a.tape + (tok * H + h) * D * D;
+#pragma unroll
+      for (int i = 0; i < ROWS; ++i) st4(tp + (size_t)(rg + i * RG) * D + 4 * cg, S[i]);
+    }
+    __syncthreads();
+  }
+
+  if (a.state_out != nullptr) {
+    float* So = a.state_out + ((size_t)row * H + h) * D * D;
+#pragma unroll
+    for (int i = 0; i < ROWS; ++i) st4(So + (size_t)(rg + i * RG) * D + 4 * cg, S[i]);
+  }
+}
+
+template <typename T>
+static cudaError_t launch_step_t(const StepArgs& a, cudaStream_t st) {
+  dim3 grid(a.H, a.B);
+  switch (a.D) {
+    case 16: step_kernel<T, 16><<<grid, StepShape<16>::THREADS, 0, st>>>(a); break;
+    case 32: step_kernel<T, 32><<<grid, StepShape<32>::THREADS, 0, st>>>(a); break;
+    case 64: step_kernel<T, 64><<<grid, StepShape<64>::THREADS, 0, st>>>(a); break;
+    case 128: step_kernel<T, 128><<<grid, StepShape<128>::THREADS, 0, st>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_step(const StepArgs& a, cudaStream_t st) {
+  return a.bf16 ? launch_step_t<__nv_bfloat16>(a, st) : launch_step_t<float>(a, st);
+}
+
+// ---------------------------------------------------------------------------
+// rollback: state <- tape[L-1], conv state <- window rows [L, L+K-1)
+// ---------------------------------------------------------------------------
+template <typename E>
+__global__ void __launch_bounds__(256) rollback_kernel(const RollbackArgs a) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int L = clampi(__ldg(a.accepted + b), 0, a.T);
+  if (L == 0) return;
+  const int row = pool_row(a.slots, b, a.pool_size);
+  if (row < 0) return;
+  const int D = a.D, H = a.H;
+  const float4* src = reinterpret_cast<const float4*>(a.tape + (((size_t)b * a.T + (L - 1)) * H + h) * D * D);
+  float4* dst = reinterpret_cast<float4*>(a.state + ((size_t)row * H + h) * D * D);
+  for (int i = threadIdx.x; i < D * D / 4; i += blockDim.x) dst[i] = src[i];
+  if (a.conv_state != nullptr && a.window != nullptr) {
+    const int Km1 = a.K - 1, C3 = 3 * D;
+    const E* win = static_cast<const E*>(a.window);
+    E* cs = static_cast<E*>(a.conv_state);
+    for (int e = threadIdx.x; e < Km1 * C3; e += blockDim.x) {
+      const int j = e / C3, c = e - (e / C3) * C3;
+      cs[(((size_t)row * Km1 + j) * H + h) * C3 + c] =
+          win[(((size_t)b * (Km1 + a.T) + L + j) * H + h) * C3 + c];
+    }
+  }
+}
+
+cudaError_t launch_rollback(const RollbackArgs& a, cudaStream_t st) {
+  dim3 grid(a.H, a.B);
+  if (a.bf16) rollback_kernel<uint16_t><<<grid, 256, 0, st>>>(a);
+  else rollback_kernel<uint32_t><<<grid, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace kda

@@ -1,0 +1,312 @@
+"""Thin ctypes binding over libkda.so (C ABI in include/kda.h).
+
+Argument marshalling only: every step of the layer runs in the CUDA library.
+Tensors must be contiguous CUDA tensors of the documented dtype; outputs left
+as ``None`` are allocated here with torch (PyTorch supplies device memory and
+the current stream, nothing else).  A missing library raises at first use:
+there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, 'libkda.so')
+
+KDA_OK = 0
+KDA_ERR_INVALID_ARG = 1
+KDA_ERR_MISALIGNED = 2
+KDA_ERR_UNSUPPORTED = 3
+KDA_ERR_CUDA = 4
+KDA_ERR_TIMEOUT = 5
+KDA_ERR_WORKSPACE = 6
+KDA_F32 = 0
+KDA_BF16 = 1
+KDA_CONV_COMMIT = 0
+KDA_CONV_TAPE = 1
+
+ENTRY_POINTS = ('kda_status_string', 'kda_abi_version', 'kda_prep',
+                'kda_prefill_workspace_size', 'kda_prefill', 'kda_decode', 'kda_verify',
+                'kda_rollback', 'kda_workspace_status')
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f'{where}: {kda_status_string(status)} ({status})')
+
+
+class CConfig(ctypes.Structure):
+    _fields_ = [('num_heads', ctypes.c_int32), ('head_dim', ctypes.c_int32),
+                ('conv_size', ctypes.c_int32), ('dtype', ctypes.c_int32),
+                ('chunk_size', ctypes.c_int32), ('gate_lower_bound', ctypes.c_float),
+                ('l2_eps', ctypes.c_float), ('norm_eps', ctypes.c_float),
+                ('q_scale', ctypes.c_float)]
+
+
+@dataclass
+class Config:
+    """Layer configuration; mirrors ``kda_config``."""
+    num_heads: int
+    head_dim: int
+    conv_size: int = 4
+    dtype: torch.dtype = torch.bfloat16
+    chunk_size: int = 64
+    gate_lower_bound: float = -5.0
+    l2_eps: float = 1e-6
+    norm_eps: float = 1e-5
+    q_scale: float = 1.0
+
+    def c(self) -> CConfig:
+        if self.dtype not in (torch.float32, torch.bfloat16):
+            raise ValueError('activation dtype must be float32 or bfloat16')
+        return CConfig(self.num_heads, self.head_dim, self.conv_size,
+                       KDA_BF16 if self.dtype == torch.bfloat16 else KDA_F32,
+                       self.chunk_size, self.gate_lower_bound, self.l2_eps, self.norm_eps,
+                       self.q_scale)
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+
+
+def lib() -> ctypes.CDLL:
+    """Load libkda.so from this package directory (raises if it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f'{LIB_PATH} is missing: build it with '
+                               '`python -m linear_attention_recurrence_09_b200.build`')
+        L = ctypes.CDLL(LIB_PATH)
+        L.kda_status_string.restype = ctypes.c_char_p
+        L.kda_status_string.argtypes = [ctypes.c_int]
+        L.kda_abi_version.restype = ctypes.c_int
+        L.kda_abi_version.argtypes = []
+        L.kda_prep.restype = ctypes.c_int
+        L.kda_prep.argtypes = [ctypes.POINTER(CConfig), _I, _I, _P, _I, _P, _P, _P, _P, _P, _P,
+                               _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _P]
+        L.kda_prefill_workspace_size.restype = ctypes.c_size_t
+        L.kda_prefill_workspace_size.argtypes = [ctypes.POINTER(CConfig), _I, _I]
+        L.kda_prefill.restype = ctypes.c_int
+        L.kda_prefill.argtypes = [ctypes.POINTER(CConfig), _I, _I, _P, _P, _P, _P, _P, _P, _P,
+                                  _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t, _P]
+        L.kda_decode.restype = ctypes.c_int
+        L.kda_decode.argtypes = [ctypes.POINTER(CConfig), _I, _P, _P, _P, _P, _P, _P, _P, _P,
+                                 _P, _I, _P, _P]
+        L.kda_verify.restype = ctypes.c_int
+        L.kda_verify.argtypes = [ctypes.POINTER(CConfig), _I, _I, _P, _P, _P, _P, _P, _P, _P,
+                                 _P, _P, _I, _P, _P, _P]
+        L.kda_rollback.restype = ctypes.c_int
+        L.kda_rollback.argtypes = [ctypes.POINTER(CConfig), _I, _I, _P, _P, _P, _P, _P, _P,
+                                   _I, _P]
+        L.kda_workspace_status.restype = ctypes.c_int
+        L.kda_workspace_status.argtypes = [_P, _P]
+        _lib = L
+    return _lib
+
+
+def kda_status_string(status: int) -> str:
+    return lib().kda_status_string(int(status)).decode()
+
+
+def kda_abi_version() -> int:
+    return lib().kda_abi_version()
+
+
+def _check(status, where):
+    if status != KDA_OK:
+        raise KdaError(status, where)
+
+
+def _ptr(t, dtype=None, name='tensor', shape=None):
+    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f'{name} must be a CUDA tensor')
+    if not t.is_contiguous():
+        raise ValueError(f'{name} must be contiguous')
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f'{name} must be {dtype}, got {t.dtype}')
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f'{name} must have shape {tuple(shape)}, got {tuple(t.shape)}')
+    return t.data_ptr() if t.numel() > 0 else None
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _empty(shape, dtype, device):
+    return torch.empty(shape, dtype=dtype, device=device)
+
+
+# ---------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+# ---------------------------------------------------------------------------
+def kda_prep(cfg: Config, cu_seqlens, x, f, beta_logit, conv_w, A_log, dt_bias,
+             conv_state=None, state_slots=None, pool_size=None, conv_mode=KDA_CONV_COMMIT,
+             conv_window=None, max_seqlen=0, out=None, stream=None):
+    """Conv + SiLU + L2 + decay gate + beta.  Returns dict q, k, v, log_a, beta (+ window)."""
+    H, d, K = cfg.num_heads, cfg.head_dim, cfg.conv_size
+    T = x.shape[0]
+    N = cu_seqlens.numel() - 1
+    dev = x.device
+    o = dict(out or {})
+    for name in ('q', 'k', 'v'):
+        if o.get(name) is None:
+            o[name] = _empty((T, H, d), cfg.dtype, dev)
+    if o.get('log_a') is None:
+        o['log_a'] = _empty((T, H, d), torch.float32, dev)
+    if o.get('beta') is None:
+        o['beta'] = _empty((T, H), torch.float32, dev)
+    if conv_mode == KDA_CONV_TAPE and conv_window is None:
+        conv_window = _empty((T + N * (K - 1), H, 3 * d), cfg.dtype, dev)
+    if pool_size is None:
+        pool_size = conv_state.shape[0] if conv_state is not None else N
+    c = cfg.c()
+    st = lib().kda_prep(
+        ctypes.byref(c), N, T, _ptr(cu_seqlens, torch.int32, 'cu_seqlens'), int(max_seqlen),
+        _ptr(x, cfg.dtype, 'x', (T, H, 3 * d)), _ptr(f, cfg.dtype, 'f', (T, H, d)),
+        _ptr(beta_logit, cfg.dtype, 'beta_logit', (T, H)),
+        _ptr(conv_w, torch.float32, 'conv_w', (H, 3 * d, K)),
+        _ptr(A_log, torch.float32, 'A_log', (H,)),
+        _ptr(dt_bias, torch.float32, 'dt_bias', (H, d)),
+        _ptr(conv_state, cfg.dtype, 'conv_state'), _ptr(state_slots, torch.int32, 'state_slots'),
+        int(pool_size), int(conv_mode), _ptr(conv_window, cfg.dtype, 'conv_window'),
+        _ptr(o['q'], cfg.dtype, 'q'), _ptr(o['k'], cfg.dtype, 'k'), _ptr(o['v'], cfg.dtype, 'v'),
+        _ptr(o['log_a'], torch.float32, 'log_a'), _ptr(o['beta'], torch.float32, 'beta'),
+        _stream(stream))
+    _check(st, 'kda_prep')
+    if conv_mode == KDA_CONV_TAPE:
+        o['window'] = conv_window
+    return o
+
+
+def kda_prefill_workspace_size(cfg: Config, n_seqs: int, total_tokens: int) -> int:
+    c = cfg.c()
+    return int(lib().kda_prefill_workspace_size(ctypes.byref(c), int(n_seqs), int(total_tokens)))
+
+
+def prefill_workspace(cfg: Config, n_seqs: int, total_tokens: int, device='cuda'):
+    """A uint8 device buffer of kda_prefill_workspace_size bytes (256-aligned by torch)."""
+    return torch.empty(kda_prefill_workspace_size(cfg, n_seqs, total_tokens), dtype=torch.uint8,
+                       device=device)
+
+
+def kda_prefill(cfg: Config, cu_seqlens, q, k, v, log_a, beta, g, norm_w, state_in=None,
+                state_out=None, state_slots=None, pool_size=None, y=None, workspace=None,
+                stream=None):
+    """Chunked prefill.  Returns y; the final states go to ``state_out``."""
+    H, d = cfg.num_heads, cfg.head_dim
+    T = q.shape[0]
+    N = cu_seqlens.numel() - 1
+    if y is None:
+        y = _empty((T, H, d), cfg.dtype, q.device)
+    if workspace is None:
+        workspace = prefill_workspace(cfg, N, T, q.device)
+    if pool_size is None:
+        ref = state_in if state_in is not None else state_out
+        pool_size = ref.shape[0] if ref is not None else N
+    c = cfg.c()
+    st = lib().kda_prefill(
+        ctypes.byref(c), N, T, _ptr(cu_seqlens, torch.int32, 'cu_seqlens'),
+        _ptr(q, cfg.dtype, 'q', (T, H, d)), _ptr(k, cfg.dtype, 'k', (T, H, d)),
+        _ptr(v, cfg.dtype, 'v', (T, H, d)), _ptr(log_a, torch.float32, 'log_a', (T, H, d)),
+        _ptr(beta, torch.float32, 'beta', (T, H)), _ptr(g, cfg.dtype, 'g', (T, H, d)),
+        _ptr(norm_w, torch.float32, 'norm_w', (d,)),
+        _ptr(state_in, torch.float32, 'state_in'), _ptr(state_out, torch.float32, 'state_out'),
+        _ptr(state_slots, torch.int32, 'state_slots'), int(pool_size),
+        _ptr(y, cfg.dtype, 'y', (T, H, d)), _ptr(workspace, None, 'workspace'),
+        int(workspace.numel() * workspace.element_size()), _stream(stream))
+    _check(st, 'kda_prefill')
+    return y
+
+
+def kda_decode(cfg: Config, q, k, v, log_a, beta, g, norm_w, state, state_slots=None,
+               pool_size=None, y=None, stream=None):
+    """One token per sequence; ``state`` [pool, H, d, d] is updated in place.  Returns y."""
+    H, d = cfg.num_heads, cfg.head_dim
+    B = q.shape[0]
+    if y is None:
+        y = _empty((B, H, d), cfg.dtype, q.device)
+    if pool_size is None:
+        pool_size = state.shape[0]
+    c = cfg.c()
+    st = lib().kda_decode(
+        ctypes.byref(c), B, _ptr(q, cfg.dtype, 'q', (B, H, d)), _ptr(k, cfg.dtype, 'k', (B, H, d)),
+        _ptr(v, cfg.dtype, 'v', (B, H, d)), _ptr(log_a, torch.float32, 'log_a', (B, H, d)),
+        _ptr(beta, torch.float32, 'beta', (B, H)), _ptr(g, cfg.dtype, 'g', (B, H, d)),
+        _ptr(norm_w, torch.float32, 'norm_w', (d,)), _ptr(state, torch.float32, 'state'),
+        _ptr(state_slots, torch.int32, 'state_slots'), int(pool_size),
+        _ptr(y, cfg.dtype, 'y', (B, H, d)), _stream(stream))
+    _check(st, 'kda_decode')
+    return y
+
+
+def kda_verify(cfg: Config, q, k, v, log_a, beta, g, norm_w, state, state_slots=None,
+               pool_size=None, tape=None, y=None, stream=None):
+    """Verify [B, Tb] draft tokens from ``state`` (unchanged).  Returns (y, tape)."""
+    H, d = cfg.num_heads, cfg.head_dim
+    B, Tb = q.shape[0], q.shape[1]
+    if y is None:
+        y = _empty((B, Tb, H, d), cfg.dtype, q.device)
+    if tape is None:
+        tape = _empty((B, Tb, H, d, d), torch.float32, q.device)
+    if pool_size is None:
+        pool_size = state.shape[0]
+    c = cfg.c()
+    st = lib().kda_verify(
+        ctypes.byref(c), B, Tb, _ptr(q, cfg.dtype, 'q', (B, Tb, H, d)),
+        _ptr(k, cfg.dtype, 'k', (B, Tb, H, d)), _ptr(v, cfg.dtype, 'v', (B, Tb, H, d)),
+        _ptr(log_a, torch.float32, 'log_a', (B, Tb, H, d)),
+        _ptr(beta, torch.float32, 'beta', (B, Tb, H)), _ptr(g, cfg.dtype, 'g', (B, Tb, H, d)),
+        _ptr(norm_w, torch.float32, 'norm_w', (d,)), _ptr(state, torch.float32, 'state'),
+        _ptr(state_slots, torch.int32, 'state_slots'), int(pool_size),
+        _ptr(tape, torch.float32, 'tape', (B, Tb, H, d, d)),
+        _ptr(y, cfg.dtype, 'y', (B, Tb, H, d)), _stream(stream))
+    _check(st, 'kda_verify')
+    return y, tape
+
+
+def kda_rollback(cfg: Config, accepted, tape, state, conv_window=None, conv_state=None,
+                 state_slots=None, pool_size=None, stream=None):
+    """Commit accepted prefixes: state <- tape[L-1], conv state <- window[L:L+K-1]."""
+    H, d = cfg.num_heads, cfg.head_dim
+    B, Tb = tape.shape[0], tape.shape[1]
+    if pool_size is None:
+        pool_size = state.shape[0]
+    c = cfg.c()
+    st = lib().kda_rollback(
+        ctypes.byref(c), B, Tb, _ptr(accepted, torch.int32, 'accepted', (B,)),
+        _ptr(tape, torch.float32, 'tape', (B, Tb, H, d, d)),
+        _ptr(conv_window, cfg.dtype, 'conv_window'), _ptr(state, torch.float32, 'state'),
+        _ptr(conv_state, cfg.dtype, 'conv_state'), _ptr(state_slots, torch.int32, 'state_slots'),
+        int(pool_size), _stream(stream))
+    _check(st, 'kda_rollback')
+
+
+def kda_workspace_status(workspace, stream=None) -> int:
+    """Synchronise the stream and return the prefill workspace status code."""
+    return int(lib().kda_workspace_status(_ptr(workspace, None, 'workspace'), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# compositions of the entry points
+# ---------------------------------------------------------------------------
+def layer_prefill(cfg: Config, params, acts, state_in=None, state_out=None, conv_state=None,
+                  workspace=None, prep_out=None, y=None, stream=None):
+    """prep + prefill over packed sequences; returns (y, prep outputs)."""
+    p = kda_prep(cfg, acts['cu_seqlens'], acts['x'], acts['f'], acts['beta_logit'],
+                 params['conv_w'], params['A_log'], params['dt_bias'], conv_state=conv_state,
+                 out=prep_out, stream=stream)
+    y = kda_prefill(cfg, acts['cu_seqlens'], p['q'], p['k'], p['v'], p['log_a'], p['beta'],
+                    acts['g'], params['norm_w'], state_in=state_in, state_out=state_out,
+                    y=y, workspace=workspace, stream=stream)
+    return y, p

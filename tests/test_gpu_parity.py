@@ -1,0 +1,261 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Bar: max|GPU - oracle| / max|oracle| <= 1e-4 for fp32 inputs and <= 1e-2 for
+bf16 inputs with an fp32 state; rollback and the verify tape are bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_recurrence_09_b200 import kda, synth
+from oracle import kda_oracle as ko
+from tests.kda_cases import (TOL, compare_layer, gpu_layer, make_case, np64, oracle_layer,
+                             rel_err)
+
+pytestmark = pytest.mark.gpu
+
+
+def _assert(errs, tol):
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, f'errors above {tol}: {errs}'
+
+
+def test_tiny_fp32_layer():
+    """Tiny fp32 workload: B=1, H=2, T=64, d=16, chunk 16, conv 4, zero state."""
+    w = synth.WORKLOADS['tiny_fp32']
+    cfg, P, A, S0, hist = make_case(w['seed'], [w['seqlen']], w['heads'], w['head_dim'],
+                                    w['conv'], torch.float32, chunk=w['chunk'])
+    _assert(compare_layer(cfg, P, A, S0, hist), 1e-4)
+
+
+@pytest.mark.parametrize('dtype', [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize('d,K', [(16, 4), (64, 2), (128, 4), (32, 8)])
+def test_prep_matches_oracle(dtype, d, K):
+    seqlens = [0, 1, 5, 17, 40]
+    cfg, P, A, _, hist = make_case(3, seqlens, 3, d, K, dtype, conv_hist=True)
+    _, _, cs, p = gpu_layer(cfg, P, A, None, hist)
+    ref = oracle_layer(cfg, P, A, None, hist)
+    tol = 1e-5 if dtype == torch.float32 else 8e-3
+    for name, rname in [('q', 'q'), ('k', 'k'), ('v', 'v'), ('log_a', 'loga'), ('beta', 'beta')]:
+        assert rel_err(np64(p[name]), ref[rname]) <= tol, name
+    assert np.array_equal(np64(cs), ref['conv_hist'])
+
+
+@pytest.mark.parametrize('dtype', [torch.float32, torch.bfloat16])
+def test_prep_tape_window(dtype):
+    cfg, P, A, _, hist = make_case(4, [8, 8, 8], 2, 32, 4, dtype, conv_hist=True)
+    dev = 'cuda'
+    cs = hist.to(dev)
+    before = cs.clone()
+    p = kda.kda_prep(cfg, A['cu_seqlens'].to(dev), A['x'].to(dev), A['f'].to(dev),
+                     A['beta_logit'].to(dev), P['conv_w'].to(dev), P['A_log'].to(dev),
+                     P['dt_bias'].to(dev), conv_state=cs, conv_mode=kda.KDA_CONV_TAPE,
+                     max_seqlen=8)
+    torch.cuda.synchronize()
+    assert torch.equal(cs, before)          # TAPE mode never writes the conv state
+    win = p['window'].cpu().view(3, 3 + 8, 2, 96)
+    x = A['x'].view(3, 8, 2, 96)
+    for s in range(3):
+        assert torch.equal(win[s, :3], hist[s])
+        assert torch.equal(win[s, 3:], x[s])
+
+
+@pytest.mark.parametrize('d,chunk', [(32, 16), (64, 32), (128, 64), (128, 16)])
+def test_prefill_varlen_ragged_bf16(d, chunk):
+    seqlens = [0, 1, chunk - 1, chunk, chunk + 1, 3 * chunk + 7]
+    cfg, P, A, S0, hist = make_case(5, seqlens, 4, d, 4, torch.bfloat16, state_var=0.01,
+                                    conv_hist=True, chunk=chunk)
+    _assert(compare_layer(cfg, P, A, S0, hist), 1e-2)
+
+
+@pytest.mark.parametrize('d,chunk', [(16, 16), (64, 32), (128, 64)])
+def test_prefill_fp32(d, chunk):
+    cfg, P, A, S0, hist = make_case(6, [37, 2 * chunk + 3], 2, d, 4, torch.float32,
+                                    state_var=0.01, conv_hist=True, chunk=chunk)
+    _assert(compare_layer(cfg, P, A, S0, hist), 1e-4)
+
+
+def test_prefill_no_tokens_copies_state():
+    cfg, P, A, S0, _ = make_case(7, [0, 0], 2, 64, 4, torch.bfloat16, state_var=0.01)
+    y, s_out, _, _ = gpu_layer(cfg, P, A, S0, None)
+    assert torch.equal(s_out.cpu(), S0)
+
+
+def test_beta_zero_no_decay_keeps_state_bit_exact():
+    """b = 0 and a = 1 (logits at -1e4): prefill and decode leave S bit-unchanged."""
+    cfg, P, A, S0, _ = make_case(8, [70], 2, 64, 4, torch.bfloat16, state_var=0.01)
+    A['beta_logit'][:] = -1e4
+    A['f'][:] = -1e4
+    _, s_out, _, p = gpu_layer(cfg, P, A, S0, None)
+    assert torch.equal(s_out.cpu(), S0)
+    st = S0.cuda().clone()
+    kda.kda_decode(cfg, p['q'][:1].contiguous(), p['k'][:1].contiguous(), p['v'][:1].contiguous(),
+                   p['log_a'][:1].contiguous(), p['beta'][:1].contiguous(),
+                   A['g'][:1].cuda().contiguous(), P['norm_w'].cuda(), st, pool_size=1)
+    torch.cuda.synchronize()
+    assert torch.equal(st.cpu()[:1], S0[:1])
+
+
+def test_split_invariance_5_plus_7():
+    """glm53-flash-mlx README test [5]: prefill 5 then 7 equals prefill 12."""
+    cfg, P, A, S0, hist = make_case(9, [12], 2, 128, 4, torch.bfloat16, state_var=0.01,
+                                    conv_hist=True, chunk=64)
+    y_full, s_full, c_full, _ = gpu_layer(cfg, P, A, S0, hist)
+    a1 = {k: v[:5] for k, v in A.items() if k != 'cu_seqlens'}
+    a1['cu_seqlens'] = torch.tensor([0, 5], dtype=torch.int32)
+    a2 = {k: v[5:] for k, v in A.items() if k != 'cu_seqlens'}
+    a2['cu_seqlens'] = torch.tensor([0, 7], dtype=torch.int32)
+    y1, s1, c1, _ = gpu_layer(cfg, P, a1, S0, hist)
+    y2, s2, c2, _ = gpu_layer(cfg, P, a2, s1.cpu(), c1.cpu())
+    y_split = torch.cat([y1, y2]).cpu()
+    assert rel_err(np64(y_split), np64(y_full)) <= 1e-2
+    assert rel_err(np64(s2), np64(s_full)) <= 1e-2
+    assert torch.equal(c2.cpu(), c_full.cpu())
+
+
+def _decode_run(cfg, P, steps_acts, state, conv_state, dev='cuda'):
+    """T decode steps: prep (T=1, COMMIT) + decode.  Returns y [T, B, H, d]."""
+    ys = []
+    for a in steps_acts:
+        p = kda.kda_prep(cfg, a['cu_seqlens'].to(dev), a['x'].to(dev), a['f'].to(dev),
+                         a['beta_logit'].to(dev), P['conv_w'].to(dev), P['A_log'].to(dev),
+                         P['dt_bias'].to(dev), conv_state=conv_state, max_seqlen=1)
+        ys.append(kda.kda_decode(cfg, p['q'], p['k'], p['v'], p['log_a'], p['beta'],
+                                 a['g'].to(dev), P['norm_w'].to(dev), state))
+    torch.cuda.synchronize()
+    return torch.stack(ys)
+
+
+def _step_acts(seed, B, H, d, dtype, n):
+    return [synth.layer_activations(seed, [1] * B, H, d, dtype, tag=('step', i)) for i in range(n)]
+
+
+def _cat_seq(parts, b):
+    """Token rows of sequence b across a list of activation dicts (one token per seq each)."""
+    out = {}
+    for key in ('x', 'f', 'beta_logit', 'g'):
+        out[key] = torch.cat([p[key][p['cu_seqlens'][b]:p['cu_seqlens'][b + 1]] for p in parts])
+    out['cu_seqlens'] = torch.tensor([0, out['x'].shape[0]], dtype=torch.int32)
+    return out
+
+
+def test_decode_matches_oracle():
+    B, H, d, T0, steps = 3, 4, 128, 40, 6
+    cfg, P, A, S0, hist = make_case(10, [T0] * B, H, d, 4, torch.bfloat16, state_var=0.01,
+                                    conv_hist=True)
+    _, s_out, cs, _ = gpu_layer(cfg, P, A, S0, hist)
+    sa = _step_acts(10, B, H, d, torch.bfloat16, steps)
+    ys = _decode_run(cfg, P, sa, s_out, cs).cpu()
+    for b in range(B):
+        seq = _cat_seq([A] + sa, b)
+        ref = oracle_layer(cfg, P, seq, S0[b:b + 1], hist[b:b + 1])
+        assert rel_err(np64(ys[:, b]), ref['y'][T0:]) <= 1e-2
+        assert rel_err(np64(s_out[b]), ref['state'][0]) <= 1e-2
+        assert np.array_equal(np64(cs[b]), ref['conv_hist'][0])
+
+
+def test_decode_equals_prefill_on_gpu():
+    """glm53-flash-mlx README test [5]: token-by-token decode equals one forward."""
+    B, H, d, T = 2, 2, 128, 20
+    cfg, P, A, S0, hist = make_case(11, [1] * B, H, d, 4, torch.bfloat16, state_var=0.01,
+                                    conv_hist=True)
+    sa = _step_acts(11, B, H, d, torch.bfloat16, T)
+    st = S0.cuda().clone()
+    cs = hist.cuda().clone()
+    ys = _decode_run(cfg, P, sa, st, cs).cpu()
+    for b in range(B):
+        seq = _cat_seq(sa, b)
+        y, s_out, c_out, _ = gpu_layer(cfg, P, seq, S0[b:b + 1], hist[b:b + 1])
+        assert rel_err(np64(ys[:, b]), np64(y)) <= 1e-2
+        assert rel_err(np64(st[b]), np64(s_out[0])) <= 1e-2
+        assert torch.equal(cs[b].cpu(), c_out[0].cpu())
+
+
+def test_verify_tape_equals_repeated_decode_bit_exact():
+    B, H, d, Tb = 3, 2, 128, 8
+    cfg, P, A, S0, hist = make_case(12, [Tb] * B, H, d, 4, torch.bfloat16, state_var=0.01,
+                                    conv_hist=True)
+    dev = 'cuda'
+    Pd = {k: v.to(dev) for k, v in P.items()}
+    cs = hist.to(dev)
+    p = kda.kda_prep(cfg, A['cu_seqlens'].to(dev), A['x'].to(dev), A['f'].to(dev),
+                     A['beta_logit'].to(dev), Pd['conv_w'], Pd['A_log'], Pd['dt_bias'],
+                     conv_state=cs, conv_mode=kda.KDA_CONV_TAPE, max_seqlen=Tb)
+    shp = lambda t, *tail: t.view(B, Tb, *tail)
+    st = S0.to(dev)
+    y_v, tape = kda.kda_verify(cfg, shp(p['q'], H, d), shp(p['k'], H, d), shp(p['v'], H, d),
+                               shp(p['log_a'], H, d), shp(p['beta'], H),
+                               shp(A['g'].to(dev), H, d), Pd['norm_w'], st)
+    torch.cuda.synchronize()
+    assert torch.equal(st.cpu(), S0)                    # live state untouched
+    st2 = S0.to(dev)
+    for j in range(Tb):
+        sel = lambda t: t.view(B, Tb, *t.shape[1:])[:, j].contiguous()
+        y_d = kda.kda_decode(cfg, sel(p['q']), sel(p['k']), sel(p['v']), sel(p['log_a']),
+                             sel(p['beta']), sel(A['g'].to(dev)), Pd['norm_w'], st2)
+        torch.cuda.synchronize()
+        assert torch.equal(tape[:, j], st2), j
+        assert torch.equal(y_v[:, j], y_d), j
+    # and against the oracle
+    for b in range(B):
+        seq = {k: v[b * Tb:(b + 1) * Tb] for k, v in A.items() if k != 'cu_seqlens'}
+        seq['cu_seqlens'] = torch.tensor([0, Tb], dtype=torch.int32)
+        ref = oracle_layer(cfg, P, seq, S0[b:b + 1], hist[b:b + 1])
+        assert rel_err(np64(y_v[b]), ref['y']) <= 1e-2
+        assert rel_err(np64(tape[b, -1]), ref['state'][0]) <= 1e-2
+
+
+def test_rollback_bit_exact():
+    B, H, d, Tb, K = 9, 2, 64, 8, 4
+    cfg, P, A, S0, hist = make_case(13, [Tb] * B, H, d, K, torch.bfloat16, state_var=0.01,
+                                    conv_hist=True)
+    dev = 'cuda'
+    Pd = {k: v.to(dev) for k, v in P.items()}
+    cs = hist.to(dev)
+    p = kda.kda_prep(cfg, A['cu_seqlens'].to(dev), A['x'].to(dev), A['f'].to(dev),
+                     A['beta_logit'].to(dev), Pd['conv_w'], Pd['A_log'], Pd['dt_bias'],
+                     conv_state=cs, conv_mode=kda.KDA_CONV_TAPE, max_seqlen=Tb)
+    shp = lambda t, *tail: t.view(B, Tb, *tail)
+    st = S0.to(dev)
+    _, tape = kda.kda_verify(cfg, shp(p['q'], H, d), shp(p['k'], H, d), shp(p['v'], H, d),
+                             shp(p['log_a'], H, d), shp(p['beta'], H),
+                             shp(A['g'].to(dev), H, d), Pd['norm_w'], st)
+    acc = torch.arange(B, dtype=torch.int32) % (Tb + 1)          # 0..8 all present
+    kda.kda_rollback(cfg, acc.to(dev), tape, st, conv_window=p['window'], conv_state=cs)
+    torch.cuda.synchronize()
+    win = p['window'].view(B, K - 1 + Tb, H, 3 * d)
+    for b in range(B):
+        L = int(acc[b])
+        if L == 0:
+            assert torch.equal(st[b].cpu(), S0[b])
+            assert torch.equal(cs[b].cpu(), hist[b])
+        else:
+            assert torch.equal(st[b], tape[b, L - 1])
+            assert torch.equal(cs[b], win[b, L:L + K - 1])
+
+
+def test_state_pool_slots():
+    """decode with state_slots into a larger pool touches only the mapped rows."""
+    B, H, d, pool = 3, 2, 32, 7
+    cfg, P, A, _, _ = make_case(14, [1] * B, H, d, 4, torch.bfloat16)
+    dev = 'cuda'
+    pool_state = synth.initial_state(14, pool, H, d, 0.01).to(dev)
+    before = pool_state.clone()
+    slots = torch.tensor([5, 0, 3], dtype=torch.int32, device=dev)
+    p = kda.kda_prep(cfg, A['cu_seqlens'].to(dev), A['x'].to(dev), A['f'].to(dev),
+                     A['beta_logit'].to(dev), P['conv_w'].to(dev), P['A_log'].to(dev),
+                     P['dt_bias'].to(dev))
+    y = kda.kda_decode(cfg, p['q'], p['k'], p['v'], p['log_a'], p['beta'], A['g'].to(dev),
+                       P['norm_w'].to(dev), pool_state, state_slots=slots)
+    torch.cuda.synchronize()
+    for r in (1, 2, 4, 6):
+        assert torch.equal(pool_state[r], before[r])
+    for b, r in enumerate([5, 0, 3]):
+        st = before[r:r + 1].clone()
+        y1 = kda.kda_decode(cfg, p['q'][b:b + 1].contiguous(), p['k'][b:b + 1].contiguous(),
+                            p['v'][b:b + 1].contiguous(), p['log_a'][b:b + 1].contiguous(),
+                            p['beta'][b:b + 1].contiguous(), A['g'][b:b + 1].to(dev).contiguous(),
+                            P['norm_w'].to(dev), st)
+        torch.cuda.synchronize()
+        assert torch.equal(st[0], pool_state[r])
+        assert torch.equal(y1[0], y[b])
