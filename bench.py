@@ -145,9 +145,8 @@ def prefill_workload(torch, kda, synth, T, seed, dev):
     A_cpu = synth.layer_activations(seed, [T], H, d, torch.bfloat16)
     A = {k: v.to(dev) for k, v in A_cpu.items()}
     N = 1
-    out = {'q': torch.empty(T, H, d, dtype=cfg.dtype, device=dev),
-           'k': torch.empty(T, H, d, dtype=cfg.dtype, device=dev),
-           'v': torch.empty(T, H, d, dtype=cfg.dtype, device=dev),
+    out = {'q': torch.empty(T, H, d, device=dev), 'k': torch.empty(T, H, d, device=dev),
+           'v': torch.empty(T, H, d, device=dev),
            'log_a': torch.empty(T, H, d, device=dev), 'beta': torch.empty(T, H, device=dev)}
     y = torch.empty(T, H, d, dtype=cfg.dtype, device=dev)
     state = torch.empty(N, H, d, d, device=dev)
@@ -158,8 +157,8 @@ def prefill_workload(torch, kda, synth, T, seed, dev):
 def prefill_bytes(T, H, d):
     """Algorithmic HBM bytes of prep and of prefill (bf16 activations, fp32 gates/state)."""
     th = T * H
-    prep = th * (3 * d * 2 + d * 2 + 2) + th * (3 * d * 2 + d * 4 + 4)
-    prefill = th * (3 * d * 2 + d * 4 + 4 + d * 2) + th * d * 2 + H * d * d * 4
+    prep = th * (3 * d * 2 + d * 2 + 2) + th * (3 * d * 4 + d * 4 + 4)
+    prefill = th * (3 * d * 4 + d * 4 + 4 + d * 2) + th * d * 2 + H * d * d * 4
     return prep, prefill
 
 
@@ -280,9 +279,8 @@ def run_decode(torch, kda, synth, dev, steps=1024):
     X = {k: S[k].view(B, steps, *S[k].shape[1:]).transpose(0, 1).contiguous().to(dev)
          for k in ('x', 'f', 'beta_logit', 'g')}
     cu = torch.arange(B + 1, dtype=torch.int32, device=dev)
-    o = {'q': torch.empty(B, H, d, dtype=cfg.dtype, device=dev),
-         'k': torch.empty(B, H, d, dtype=cfg.dtype, device=dev),
-         'v': torch.empty(B, H, d, dtype=cfg.dtype, device=dev),
+    o = {'q': torch.empty(B, H, d, device=dev), 'k': torch.empty(B, H, d, device=dev),
+         'v': torch.empty(B, H, d, device=dev),
          'log_a': torch.empty(B, H, d, device=dev), 'beta': torch.empty(B, H, device=dev)}
     y = torch.empty(steps, B, H, d, dtype=cfg.dtype, device=dev)
 
@@ -323,7 +321,7 @@ def run_decode(torch, kda, synth, dev, steps=1024):
     e1.record()
     torch.cuda.synchronize()
     ms_k = e0.elapsed_time(e1) / n
-    bytes_k = B * H * (2 * d * d * 4 + 4 * d * 2 + d * 4 + 4 + d * 2)
+    bytes_k = B * H * (2 * d * d * 4 + 3 * d * 4 + d * 2 + d * 4 + 4 + d * 2)
     hbm, _, peak_kind = measured_peaks()
     ach = bytes_k / (ms_k / 1e3) / 1e9
     del g
@@ -352,9 +350,8 @@ def run_verify(torch, kda, synth, dev, rounds=256):
          for k in ('x', 'f', 'beta_logit', 'g')}
     acc = synth.accepted_lengths(3, rounds, B, Tb).to(dev)
     cu = (torch.arange(B + 1, dtype=torch.int32, device=dev) * Tb)
-    o = {'q': torch.empty(B * Tb, H, d, dtype=cfg.dtype, device=dev),
-         'k': torch.empty(B * Tb, H, d, dtype=cfg.dtype, device=dev),
-         'v': torch.empty(B * Tb, H, d, dtype=cfg.dtype, device=dev),
+    o = {'q': torch.empty(B * Tb, H, d, device=dev), 'k': torch.empty(B * Tb, H, d, device=dev),
+         'v': torch.empty(B * Tb, H, d, device=dev),
          'log_a': torch.empty(B * Tb, H, d, device=dev), 'beta': torch.empty(B * Tb, H, device=dev)}
     win = torch.empty(B * (Tb + K - 1), H, 3 * d, dtype=cfg.dtype, device=dev)
     tape = torch.empty(B, Tb, H, d, d, device=dev)
@@ -398,7 +395,7 @@ def run_verify(torch, kda, synth, dev, rounds=256):
     e1.record()
     torch.cuda.synchronize()
     ms_k = e0.elapsed_time(e1) / n
-    bytes_k = B * H * (d * d * 4 + Tb * d * d * 4 + Tb * (4 * d * 2 + d * 4 + 4 + d * 2))
+    bytes_k = B * H * (d * d * 4 + Tb * d * d * 4 + Tb * (3 * d * 4 + d * 2 + d * 4 + 4 + d * 2))
     hbm, _, peak_kind = measured_peaks()
     ach = bytes_k / (ms_k / 1e3) / 1e9
     del g

@@ -30,9 +30,11 @@
  *    stream) and the call returns without synchronising.  Launch failures are
  *    reported as KDA_ERR_CUDA.
  *  - Tensors are dense, row-major (last index fastest), with the shapes given
- *    below.  Activations (x, f, beta_logit, g, q, k, v, y, conv state/window)
- *    have the element type cfg->dtype; parameters, log decay, beta, recurrent
- *    states and tapes are fp32.
+ *    below.  Activations (x, f, beta_logit, g, y, conv state/window) have the
+ *    element type cfg->dtype; the prep outputs q, k, v, log decay and beta,
+ *    the parameters, the recurrent states and the tapes are fp32 (rounding the
+ *    normalised q/k/v to bf16 would cost more accuracy than every later bf16
+ *    operand of the chunked prefill together).
  *  - Every pointer must be 16-byte aligned (KDA_ERR_MISALIGNED otherwise).
  *  - Packed (varlen) batches use cu_seqlens: int32 [n_seqs + 1], device,
  *    non-decreasing, cu_seqlens[0] = 0, cu_seqlens[n_seqs] = total_tokens.
@@ -125,7 +127,7 @@ KDA_API int kda_abi_version(void);
  *  conv_window TAPE mode only: [total_tokens + n_seqs*(K-1), H, 3d]; sequence s
  *              occupies rows [cu[s] + s*(K-1), cu[s+1] + (s+1)*(K-1)) and gets
  *              [history; x_s].  Ignored (may be NULL) in COMMIT mode.
- *  q, k, v     out [total_tokens, H, d]  normalised q, k and SiLU'd v
+ *  q, k, v     out fp32 [total_tokens, H, d]  normalised q, k and SiLU'd v
  *  log_a       out fp32 [total_tokens, H, d]
  *  beta        out fp32 [total_tokens, H]
  */
@@ -177,7 +179,8 @@ KDA_API int kda_prefill(const kda_config* cfg, int32_t n_seqs, int32_t total_tok
  * decay, both column reductions S^T k and S^T q in one pass, rank-1 update,
  * one store, gated RMSNorm.
  *
- *  q, k, v, g [batch, H, d]; log_a fp32 [batch, H, d]; beta fp32 [batch, H]
+ *  q, k, v fp32 [batch, H, d]; g [batch, H, d]; log_a fp32 [batch, H, d];
+ *  beta fp32 [batch, H]
  *  state      fp32 [pool_size, H, d, d], updated in place (row state_slots[b] or b)
  *  y          out [batch, H, d]
  */
@@ -194,7 +197,8 @@ KDA_API int kda_decode(const kda_config* cfg, int32_t batch, const void* q,
  * state untouched, and writes the state after every step to the tape, so that
  * rollback to any accepted prefix is a copy.
  *
- *  q, k, v, g [batch, block_len, H, d]; log_a fp32 [batch, block_len, H, d];
+ *  q, k, v fp32 [batch, block_len, H, d]; g [batch, block_len, H, d];
+ *  log_a fp32 [batch, block_len, H, d];
  *  beta fp32 [batch, block_len, H]
  *  state      fp32 [pool_size, H, d, d], read only
  *  tape       out fp32 [batch, block_len, H, d, d]: tape[b, j] = state after draft j

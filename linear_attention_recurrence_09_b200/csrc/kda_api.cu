@@ -100,7 +100,8 @@ int kda_prep(const kda_config* cfg, int32_t n_seqs, int32_t total_tokens,
   a.mode = conv_mode;
   a.commit_in_kernel = (max_seqlen >= 1 && max_seqlen <= kda::prep_tile()) ? 1 : 0;
   a.window = conv_window;
-  a.q = q; a.k = k; a.v = v; a.loga = log_a; a.beta = beta;
+  a.q = static_cast<float*>(q); a.k = static_cast<float*>(k); a.v = static_cast<float*>(v);
+  a.loga = log_a; a.beta = beta;
   a.lb = cfg->gate_lower_bound; a.l2_eps = cfg->l2_eps;
   return cuda_status(kda::launch_prep(a, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -136,7 +137,9 @@ int kda_prefill(const kda_config* cfg, int32_t n_seqs, int32_t total_tokens,
   a.cu = cu_seqlens; a.n_seqs = n_seqs; a.total = total_tokens;
   a.H = cfg->num_heads; a.D = cfg->head_dim; a.C = cfg->chunk_size;
   a.bf16 = cfg->dtype == KDA_BF16;
-  a.q = q; a.k = k; a.v = v; a.loga = log_a; a.beta = beta; a.g = g; a.norm_w = norm_w;
+  a.q = static_cast<const float*>(q); a.k = static_cast<const float*>(k);
+  a.v = static_cast<const float*>(v);
+  a.loga = log_a; a.beta = beta; a.g = g; a.norm_w = norm_w;
   // without states there is no pool to index: every sequence is processed
   const bool pooled = state_in != nullptr || state_out != nullptr;
   a.state_in = state_in; a.state_out = state_out;
@@ -163,7 +166,9 @@ static int step_common(const kda_config* cfg, int32_t batch, int32_t T, const vo
   kda::StepArgs a{};
   a.B = batch; a.T = T; a.H = cfg->num_heads; a.D = cfg->head_dim;
   a.bf16 = cfg->dtype == KDA_BF16;
-  a.q = q; a.k = k; a.v = v; a.loga = log_a; a.beta = beta; a.g = g; a.norm_w = norm_w;
+  a.q = static_cast<const float*>(q); a.k = static_cast<const float*>(k);
+  a.v = static_cast<const float*>(v);
+  a.loga = log_a; a.beta = beta; a.g = g; a.norm_w = norm_w;
   a.state_in = state_in; a.state_out = state_out; a.tape = tape;
   a.slots = slots; a.pool_size = pool_size; a.y = y;
   a.norm_eps = cfg->norm_eps; a.q_scale = cfg->q_scale;

@@ -23,9 +23,9 @@ struct PrepArgs {
   int mode;  // 0 commit, 1 tape
   int commit_in_kernel;
   void* window;
-  void* q;
-  void* k;
-  void* v;
+  float* q;
+  float* k;
+  float* v;
   float* loga;
   float* beta;
   float lb, l2_eps;
@@ -34,9 +34,9 @@ struct PrepArgs {
 struct StepArgs {  // decode (T = 1) and verify (T = block_len)
   int B, T, H, D;
   bool bf16;
-  const void* q;
-  const void* k;
-  const void* v;
+  const float* q;
+  const float* k;
+  const float* v;
   const float* loga;
   const float* beta;
   const void* g;
@@ -74,9 +74,9 @@ struct PrefillArgs {
   const int32_t* cu;
   int n_seqs, total, H, D, C;
   bool bf16;
-  const void* q;
-  const void* k;
-  const void* v;
+  const float* q;
+  const float* k;
+  const float* v;
   const float* loga;
   const float* beta;
   const void* g;

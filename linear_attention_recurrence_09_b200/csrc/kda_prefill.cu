@@ -80,9 +80,9 @@ __global__ void __launch_bounds__(256) intra_chunk_kernel(const PrefillArgs a) {
   if (tr.len == 0) return;
   if (pool_row(a.slots, tr.seq, a.pool_size) < 0) return;
   const int L = tr.len, t0 = tr.t0, tid = threadIdx.x;
-  const T* __restrict__ qg = static_cast<const T*>(a.q);
-  const T* __restrict__ kg = static_cast<const T*>(a.k);
-  const T* __restrict__ vg = static_cast<const T*>(a.v);
+  const float* __restrict__ qg = a.q;
+  const float* __restrict__ kg = a.k;
+  const float* __restrict__ vg = a.v;
   WT* Wo = reinterpret_cast<WT*>(a.ws + a.L.W);
   WT* Uo = reinterpret_cast<WT*>(a.ws + a.L.Ut);
   WT* Qo = reinterpret_cast<WT*>(a.ws + a.L.Qt);
@@ -96,8 +96,8 @@ __global__ void __launch_bounds__(256) intra_chunk_kernel(const PrefillArgs a) {
     if (r < L) {
       const size_t idx = ((size_t)(t0 + r) * H + h) * D + c;
       la = __ldg(a.loga + idx);
-      kk = ld1(kg + idx);
-      qq = ld1(qg + idx);
+      kk = __ldg(kg + idx);
+      qq = __ldg(qg + idx);
     }
     G[e] = la; Kr[e] = kk; Qb[e] = qq;
   }
@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(256) intra_chunk_kernel(const PrefillArgs a) {
       if (m == 0) {
         brc = Kr[r * D + c] * __expf(G[r * D + c]);
       } else {
-        brc = (r < L) ? ld1(vg + ((size_t)(t0 + r) * H + h) * D + c) : 0.f;
+        brc = (r < L) ? __ldg(vg + ((size_t)(t0 + r) * H + h) * D + c) : 0.f;
       }
       float acc = bs[r] * brc;
 #pragma unroll

@@ -106,7 +106,7 @@ prep_kernel(const PrepArgs a) {
   }
 
   if (own) {
-    T* dst = static_cast<T*>(part == 0 ? a.q : (part == 1 ? a.k : a.v));
+    float* dst = part == 0 ? a.q : (part == 1 ? a.k : a.v);
     const int c = ch - part * D;
 #pragma unroll
     for (int i = 0; i < PREP_TILE; ++i) {

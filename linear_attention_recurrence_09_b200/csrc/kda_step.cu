@@ -54,9 +54,9 @@ step_kernel(const StepArgs a) {
   if (row < 0) return;
   const int tid = threadIdx.x, cg = tid % CG, rg = tid / CG;
   const int lane = tid & 31, warp = tid >> 5;
-  const T* __restrict__ qg = static_cast<const T*>(a.q);
-  const T* __restrict__ kg = static_cast<const T*>(a.k);
-  const T* __restrict__ vg = static_cast<const T*>(a.v);
+  const float* __restrict__ qg = a.q;
+  const float* __restrict__ kg = a.k;
+  const float* __restrict__ vg = a.v;
   const T* __restrict__ gg = static_cast<const T*>(a.g);
   T* __restrict__ yg = static_cast<T*>(a.y);
 
@@ -69,8 +69,8 @@ step_kernel(const StepArgs a) {
     const size_t tok = (size_t)b * a.T + t;
     const size_t base = (tok * H + h) * D;
     for (int c = tid; c < D; c += THREADS) {
-      ks[c] = ld1(kg + base + c);
-      qs[c] = ld1(qg + base + c);
+      ks[c] = __ldg(kg + base + c);
+      qs[c] = __ldg(qg + base + c);
       as_[c] = expf(__ldg(a.loga + base + c));
     }
     __syncthreads();
@@ -102,7 +102,7 @@ step_kernel(const StepArgs a) {
 #pragma unroll
       for (int j = 0; j < RG; ++j) { rk += redk[j][tid]; rq += redq[j][tid]; }
       const float bt = __ldg(a.beta + tok * H + h);
-      const float u = bt * (ld1(vg + base + tid) - rk);
+      const float u = bt * (__ldg(vg + base + tid) - rk);
       o = a.q_scale * fmaf(u, kq_s, rq);
       us[tid] = u;
     }

@@ -161,7 +161,7 @@ def kda_prep(cfg: Config, cu_seqlens, x, f, beta_logit, conv_w, A_log, dt_bias,
     o = dict(out or {})
     for name in ('q', 'k', 'v'):
         if o.get(name) is None:
-            o[name] = _empty((T, H, d), cfg.dtype, dev)
+            o[name] = _empty((T, H, d), torch.float32, dev)
     if o.get('log_a') is None:
         o['log_a'] = _empty((T, H, d), torch.float32, dev)
     if o.get('beta') is None:
@@ -180,7 +180,8 @@ def kda_prep(cfg: Config, cu_seqlens, x, f, beta_logit, conv_w, A_log, dt_bias,
         _ptr(dt_bias, torch.float32, 'dt_bias', (H, d)),
         _ptr(conv_state, cfg.dtype, 'conv_state'), _ptr(state_slots, torch.int32, 'state_slots'),
         int(pool_size), int(conv_mode), _ptr(conv_window, cfg.dtype, 'conv_window'),
-        _ptr(o['q'], cfg.dtype, 'q'), _ptr(o['k'], cfg.dtype, 'k'), _ptr(o['v'], cfg.dtype, 'v'),
+        _ptr(o['q'], torch.float32, 'q'), _ptr(o['k'], torch.float32, 'k'),
+        _ptr(o['v'], torch.float32, 'v'),
         _ptr(o['log_a'], torch.float32, 'log_a'), _ptr(o['beta'], torch.float32, 'beta'),
         _stream(stream))
     _check(st, 'kda_prep')
@@ -217,8 +218,8 @@ def kda_prefill(cfg: Config, cu_seqlens, q, k, v, log_a, beta, g, norm_w, state_
     c = cfg.c()
     st = lib().kda_prefill(
         ctypes.byref(c), N, T, _ptr(cu_seqlens, torch.int32, 'cu_seqlens'),
-        _ptr(q, cfg.dtype, 'q', (T, H, d)), _ptr(k, cfg.dtype, 'k', (T, H, d)),
-        _ptr(v, cfg.dtype, 'v', (T, H, d)), _ptr(log_a, torch.float32, 'log_a', (T, H, d)),
+        _ptr(q, torch.float32, 'q', (T, H, d)), _ptr(k, torch.float32, 'k', (T, H, d)),
+        _ptr(v, torch.float32, 'v', (T, H, d)), _ptr(log_a, torch.float32, 'log_a', (T, H, d)),
         _ptr(beta, torch.float32, 'beta', (T, H)), _ptr(g, cfg.dtype, 'g', (T, H, d)),
         _ptr(norm_w, torch.float32, 'norm_w', (d,)),
         _ptr(state_in, torch.float32, 'state_in'), _ptr(state_out, torch.float32, 'state_out'),
@@ -240,8 +241,9 @@ def kda_decode(cfg: Config, q, k, v, log_a, beta, g, norm_w, state, state_slots=
         pool_size = state.shape[0]
     c = cfg.c()
     st = lib().kda_decode(
-        ctypes.byref(c), B, _ptr(q, cfg.dtype, 'q', (B, H, d)), _ptr(k, cfg.dtype, 'k', (B, H, d)),
-        _ptr(v, cfg.dtype, 'v', (B, H, d)), _ptr(log_a, torch.float32, 'log_a', (B, H, d)),
+        ctypes.byref(c), B, _ptr(q, torch.float32, 'q', (B, H, d)),
+        _ptr(k, torch.float32, 'k', (B, H, d)),
+        _ptr(v, torch.float32, 'v', (B, H, d)), _ptr(log_a, torch.float32, 'log_a', (B, H, d)),
         _ptr(beta, torch.float32, 'beta', (B, H)), _ptr(g, cfg.dtype, 'g', (B, H, d)),
         _ptr(norm_w, torch.float32, 'norm_w', (d,)), _ptr(state, torch.float32, 'state'),
         _ptr(state_slots, torch.int32, 'state_slots'), int(pool_size),
@@ -263,8 +265,8 @@ def kda_verify(cfg: Config, q, k, v, log_a, beta, g, norm_w, state, state_slots=
         pool_size = state.shape[0]
     c = cfg.c()
     st = lib().kda_verify(
-        ctypes.byref(c), B, Tb, _ptr(q, cfg.dtype, 'q', (B, Tb, H, d)),
-        _ptr(k, cfg.dtype, 'k', (B, Tb, H, d)), _ptr(v, cfg.dtype, 'v', (B, Tb, H, d)),
+        ctypes.byref(c), B, Tb, _ptr(q, torch.float32, 'q', (B, Tb, H, d)),
+        _ptr(k, torch.float32, 'k', (B, Tb, H, d)), _ptr(v, torch.float32, 'v', (B, Tb, H, d)),
         _ptr(log_a, torch.float32, 'log_a', (B, Tb, H, d)),
         _ptr(beta, torch.float32, 'beta', (B, Tb, H)), _ptr(g, cfg.dtype, 'g', (B, Tb, H, d)),
         _ptr(norm_w, torch.float32, 'norm_w', (d,)), _ptr(state, torch.float32, 'state'),
