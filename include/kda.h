@@ -233,6 +233,17 @@ KDA_API int kda_rollback(const kda_config* cfg, int32_t batch, int32_t block_len
  */
 KDA_API int kda_workspace_status(const void* workspace, kda_stream_t stream);
 
+/*
+ * kda_selftest_wait_timeout - failure-detection self-test.  Enqueues one warp
+ * that waits, with the same bounded wait the prefill pipeline uses, on a
+ * barrier nothing ever completes; after about a quarter of a second it gives up
+ * and records KDA_ERR_TIMEOUT in the status word at the start of `workspace`
+ * (>= 256 bytes, 256-byte aligned, device memory), which it clears first.  A
+ * following kda_workspace_status returns KDA_ERR_TIMEOUT and the context stays
+ * usable.  No trap, no fault, no unbounded wait.
+ */
+KDA_API int kda_selftest_wait_timeout(void* workspace, kda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

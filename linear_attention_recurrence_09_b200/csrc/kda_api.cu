@@ -217,6 +217,14 @@ int kda_rollback(const kda_config* cfg, int32_t batch, int32_t block_len,
   return cuda_status(kda::launch_rollback(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int kda_selftest_wait_timeout(void* workspace, kda_stream_t stream) {
+  if (workspace == nullptr) return KDA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, 256, s) != cudaSuccess) return KDA_ERR_CUDA;
+  return cuda_status(kda::launch_wait_timeout_selftest(workspace, s));
+}
+
 int kda_workspace_status(const void* workspace, kda_stream_t stream) {
   if (workspace == nullptr) return KDA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

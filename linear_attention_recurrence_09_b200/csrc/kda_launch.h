@@ -95,6 +95,9 @@ cudaError_t launch_prep(const PrepArgs& a, cudaStream_t st);
 cudaError_t launch_step(const StepArgs& a, cudaStream_t st);
 cudaError_t launch_rollback(const RollbackArgs& a, cudaStream_t st);
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st);
+bool sm100_interchunk_supported(const PrefillArgs& a);
+cudaError_t launch_interchunk_sm100(const PrefillArgs& a, cudaStream_t st);
+cudaError_t launch_wait_timeout_selftest(void* workspace, cudaStream_t st);
 int prep_tile();
 int prep_kmax();
 

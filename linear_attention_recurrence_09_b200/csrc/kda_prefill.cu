@@ -1,4 +1,4 @@
-// kda_prefill, generic path (SIMT fp32 arithmetic, any supported d and chunk).
+// kda_prefill: chunkwise-parallel prefill.
 //
 // Chunkwise form of the KDA recurrence (the "chunked fallback" class of
 // llama.cpp PR #27754, written here from the delta-rule UT/WY transform of
@@ -9,11 +9,14 @@
 //   W = (I + A)^{-1} diag(b) (K * e^G),  U~ = (I + A)^{-1} diag(b) V
 //   U = U~ - W S,   O = (q_scale Q * e^G) S + M U,   S <- Diag(e^{G_C}) S + (K * e^{G_C - G})^T U
 //
-// Pass 1 (intra_chunk_kernel) is parallel over (chunk, head): it writes W, U~,
-// Q~ = q_scale Q e^G, K' = K e^{G_C - G}, M and e^{G_C} to the workspace.
-// Pass 2 (inter_chunk_kernel) is serial over the chunks of each sequence and
-// parallel over (value-column slice, head, sequence); it keeps its slice of the
-// fp32 state in shared memory and writes o.  Pass 3 applies the gated RMSNorm.
+// Pass 1 (intra_chunk_kernel) is parallel over (chunk, head): it writes, per
+// chunk slot, W, U~, Q~ = q_scale Q e^G (rows = tokens), K'^T = (K e^{G_C - G})^T
+// (rows = key channels), M and e^{G_C} to the workspace, zero-padded past the end
+// of the sequence so every chunk is a full, self-contained tile.
+// Pass 2 is serial over the chunks of each sequence and parallel over (value
+// slice, head, sequence); it carries its slice of the fp32 state on chip and
+// writes o.  It runs as bf16 tcgen05 MMAs for d = 128, chunk 64 (sm100 file) and
+// as SIMT fp32 otherwise (inter_chunk_kernel).  Pass 3 applies the gated RMSNorm.
 //
 // Range of the exponentials.  The gate keeps each log a in [lb, 0] with
 // lb >= -5, so over a sub-chunk of 16 tokens a cumulative decay spans at most
@@ -29,22 +32,22 @@
 namespace kda {
 
 constexpr int SUB = 16;      // sub-chunk length bounding the exponent span
-constexpr int P2_J = 16;     // value columns per inter-chunk CTA
+constexpr int P2_J = 16;     // value columns per SIMT inter-chunk CTA
 
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 PrefillLayout prefill_layout(int n_seqs, int total, int H, int D, int C, bool bf16) {
   PrefillLayout L;
   L.wsize = bf16 ? 2 : 4;
-  const size_t per_tok = (size_t)total * H * D;
   L.nslots = num_slots(total, n_seqs, C);
+  const size_t per_slot = (size_t)L.nslots * H * C * D;   // C x D tile per (slot, head)
   size_t off = 0;
   L.status = off; off += 256;
-  L.W = off; off += align256(per_tok * L.wsize);
-  L.Ut = off; off += align256(per_tok * L.wsize);
-  L.Qt = off; off += align256(per_tok * L.wsize);
-  L.Kp = off; off += align256(per_tok * L.wsize);
-  L.o = off; off += align256(per_tok * 4);
+  L.W = off; off += align256(per_slot * L.wsize);
+  L.Ut = off; off += align256(per_slot * L.wsize);
+  L.Qt = off; off += align256(per_slot * L.wsize);
+  L.Kp = off; off += align256(per_slot * L.wsize);          // K'^T, D x C per (slot, head)
+  L.o = off; off += align256((size_t)total * H * D * 4);
   L.M = off; off += align256((size_t)L.nslots * H * C * C * L.wsize);
   L.gC = off; off += align256((size_t)L.nslots * H * D * 4);
   L.total = off;
@@ -56,22 +59,22 @@ PrefillLayout prefill_layout(int n_seqs, int total, int H, int D, int C, bool bf
 // ---------------------------------------------------------------------------
 template <int D, int C>
 struct P1Smem {
-  static constexpr int KC_LD = D + 1;  // padded row stride: conflict-free column walks
+  static constexpr int LD = D + 1;     // padded row stride: conflict-free column walks
   static constexpr int A_LD = C + 1;
-  static constexpr size_t bytes =
-      sizeof(float) * (4 * C * D + C * KC_LD + C * A_LD + C);
+  static constexpr size_t bytes = sizeof(float) * (5 * C * LD + C * A_LD + C);
 };
 
-template <typename T, typename WT, int D, int C>
+template <typename WT, int D, int C>
 __global__ void __launch_bounds__(256) intra_chunk_kernel(const PrefillArgs a) {
   using SM = P1Smem<D, C>;
+  constexpr int LD = SM::LD;
   extern __shared__ __align__(16) float smem[];
-  float* G = smem;                 // [C][D] cumulative log decay
-  float* Kr = G + C * D;           // [C][D] k
-  float* Kb = Kr + C * D;          // [C][D] k_r e^{G_r - G_ref(r)}
-  float* Qb = Kb + C * D;          // [C][D] q_scale q_r e^{G_r - G_ref(r)}
-  float* Kc = Qb + C * D;          // [C][KC_LD] k_i e^{G_ref(R) - G_i} for the current R
-  float* A = Kc + C * SM::KC_LD;   // [C][A_LD]
+  float* G = smem;                 // [C][LD] cumulative log decay
+  float* Kr = G + C * LD;          // [C][LD] k
+  float* Kb = Kr + C * LD;         // [C][LD] k_r e^{G_r - G_ref(r)}
+  float* Qb = Kb + C * LD;         // [C][LD] q_scale q_r e^{G_r - G_ref(r)}
+  float* Kc = Qb + C * LD;         // [C][LD] k_i e^{G_ref(R) - G_i} for the current R
+  float* A = Kc + C * LD;          // [C][A_LD]
   float* bs = A + C * SM::A_LD;    // [C]
 
   const int h = blockIdx.y, H = a.H;
@@ -80,15 +83,13 @@ __global__ void __launch_bounds__(256) intra_chunk_kernel(const PrefillArgs a) {
   if (tr.len == 0) return;
   if (pool_row(a.slots, tr.seq, a.pool_size) < 0) return;
   const int L = tr.len, t0 = tr.t0, tid = threadIdx.x;
-  const float* __restrict__ qg = a.q;
-  const float* __restrict__ kg = a.k;
-  const float* __restrict__ vg = a.v;
-  WT* Wo = reinterpret_cast<WT*>(a.ws + a.L.W);
-  WT* Uo = reinterpret_cast<WT*>(a.ws + a.L.Ut);
-  WT* Qo = reinterpret_cast<WT*>(a.ws + a.L.Qt);
-  WT* Ko = reinterpret_cast<WT*>(a.ws + a.L.Kp);
-  WT* Mo = reinterpret_cast<WT*>(a.ws + a.L.M) + ((size_t)slot * H + h) * C * C;
-  float* gCo = reinterpret_cast<float*>(a.ws + a.L.gC) + ((size_t)slot * H + h) * D;
+  const size_t tile = (size_t)slot * H + h;
+  WT* Wo = reinterpret_cast<WT*>(a.ws + a.L.W) + tile * C * D;
+  WT* Uo = reinterpret_cast<WT*>(a.ws + a.L.Ut) + tile * C * D;
+  WT* Qo = reinterpret_cast<WT*>(a.ws + a.L.Qt) + tile * C * D;
+  WT* KTo = reinterpret_cast<WT*>(a.ws + a.L.Kp) + tile * D * C;
+  WT* Mo = reinterpret_cast<WT*>(a.ws + a.L.M) + tile * C * C;
+  float* gCo = reinterpret_cast<float*>(a.ws + a.L.gC) + tile * D;
 
   for (int e = tid; e < C * D; e += blockDim.x) {
     const int r = e / D, c = e - (e / D) * D;
@@ -96,10 +97,10 @@ __global__ void __launch_bounds__(256) intra_chunk_kernel(const PrefillArgs a) {
     if (r < L) {
       const size_t idx = ((size_t)(t0 + r) * H + h) * D + c;
       la = __ldg(a.loga + idx);
-      kk = __ldg(kg + idx);
-      qq = __ldg(qg + idx);
+      kk = __ldg(a.k + idx);
+      qq = __ldg(a.q + idx);
     }
-    G[e] = la; Kr[e] = kk; Qb[e] = qq;
+    G[r * LD + c] = la; Kr[r * LD + c] = kk; Qb[r * LD + c] = qq;
   }
   for (int r = tid; r < C; r += blockDim.x)
     bs[r] = (r < L) ? __ldg(a.beta + (size_t)(t0 + r) * H + h) : 0.f;
@@ -108,27 +109,28 @@ __global__ void __launch_bounds__(256) intra_chunk_kernel(const PrefillArgs a) {
   // cumulative log decay per key channel (padded rows add 0)
   for (int c = tid; c < D; c += blockDim.x) {
     float acc = 0.f;
-    for (int r = 0; r < C; ++r) { acc += G[r * D + c]; G[r * D + c] = acc; }
+    for (int r = 0; r < C; ++r) { acc += G[r * LD + c]; G[r * LD + c] = acc; }
   }
   __syncthreads();
 
-  // row-scaled operands and the per-token outputs Q~, K'
+  // row-scaled gram operands and Q~ (rows past the sequence end are zero)
   for (int e = tid; e < C * D; e += blockDim.x) {
     const int r = e / D, c = e - (e / D) * D;
-    const float g = G[e];
+    const float g = G[r * LD + c];
     const int R = r / SUB;
-    const float ref = (R == 0) ? 0.f : G[(R * SUB - 1) * D + c];
+    const float ref = (R == 0) ? 0.f : G[(R * SUB - 1) * LD + c];
     const float er = __expf(g - ref);
-    const float kk = Kr[e], qq = Qb[e];
-    Kb[e] = kk * er;
-    Qb[e] = a.q_scale * qq * er;
-    if (r < L) {
-      const size_t idx = ((size_t)(t0 + r) * H + h) * D + c;
-      st1(Qo + idx, a.q_scale * qq * __expf(g));
-      st1(Ko + idx, kk * __expf(G[(C - 1) * D + c] - g));
-    }
+    const float kk = Kr[r * LD + c], qq = Qb[r * LD + c];
+    Kb[r * LD + c] = kk * er;
+    Qb[r * LD + c] = a.q_scale * qq * er;
+    st1(Qo + (size_t)r * D + c, a.q_scale * qq * __expf(g));
   }
-  for (int c = tid; c < D; c += blockDim.x) gCo[c] = __expf(G[(C - 1) * D + c]);
+  // K'^T[c][r] = k_r[c] e^{G_last[c] - G_r[c]}  (r fastest: coalesced rows of K'^T)
+  for (int e = tid; e < C * D; e += blockDim.x) {
+    const int c = e / C, r = e - (e / C) * C;
+    st1(KTo + (size_t)c * C + r, Kr[r * LD + c] * __expf(G[(C - 1) * LD + c] - G[r * LD + c]));
+  }
+  for (int c = tid; c < D; c += blockDim.x) gCo[c] = __expf(G[(C - 1) * LD + c]);
   __syncthreads();
 
   // gram blocks, one row sub-chunk R at a time
@@ -136,17 +138,17 @@ __global__ void __launch_bounds__(256) intra_chunk_kernel(const PrefillArgs a) {
     const int ncol = (R + 1) * SUB;
     for (int e = tid; e < ncol * D; e += blockDim.x) {
       const int i = e / D, c = e - (e / D) * D;
-      const float ref = (R == 0) ? 0.f : G[(R * SUB - 1) * D + c];
-      Kc[i * SM::KC_LD + c] = Kr[i * D + c] * __expf(ref - G[i * D + c]);
+      const float ref = (R == 0) ? 0.f : G[(R * SUB - 1) * LD + c];
+      Kc[i * LD + c] = Kr[i * LD + c] * __expf(ref - G[i * LD + c]);
     }
     __syncthreads();
     for (int p = tid; p < SUB * ncol; p += blockDim.x) {
       const int r = R * SUB + p / ncol, i = p - (p / ncol) * ncol;
       float am = 0.f, mm = 0.f;
       if (i <= r) {
-        const float* kb = Kb + r * D;
-        const float* qb = Qb + r * D;
-        const float* kc = Kc + i * SM::KC_LD;
+        const float* kb = Kb + r * LD;
+        const float* qb = Qb + r * LD;
+        const float* kc = Kc + i * LD;
 #pragma unroll 8
         for (int c = 0; c < D; ++c) {
           am = fmaf(kb[c], kc[c], am);
@@ -165,7 +167,8 @@ __global__ void __launch_bounds__(256) intra_chunk_kernel(const PrefillArgs a) {
   }
 
   // forward substitution (I + A) X = diag(b) B for B = K e^G (m = 0) and V (m = 1);
-  // each thread owns one column of one right-hand side, so no barrier is needed
+  // each thread owns one column of one right-hand side, so no barrier is needed.
+  // Padded rows have b = 0 and a zero row of A, so their X rows are zero.
   if (tid < 2 * D) {
     const int m = tid / D, c = tid - (tid / D) * D;
     WT* out = (m == 0) ? Wo : Uo;
@@ -174,21 +177,21 @@ __global__ void __launch_bounds__(256) intra_chunk_kernel(const PrefillArgs a) {
     for (int r = 0; r < C; ++r) {
       float brc;
       if (m == 0) {
-        brc = Kr[r * D + c] * __expf(G[r * D + c]);
+        brc = Kr[r * LD + c] * __expf(G[r * LD + c]);
       } else {
-        brc = (r < L) ? __ldg(vg + ((size_t)(t0 + r) * H + h) * D + c) : 0.f;
+        brc = (r < L) ? __ldg(a.v + ((size_t)(t0 + r) * H + h) * D + c) : 0.f;
       }
       float acc = bs[r] * brc;
 #pragma unroll
       for (int i = 0; i < r; ++i) acc = fmaf(-A[r * SM::A_LD + i], xcol[i], acc);
       xcol[r] = acc;
-      if (r < L) st1(out + ((size_t)(t0 + r) * H + h) * D + c, acc);
+      st1(out + (size_t)r * D + c, acc);
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// pass 2: inter-chunk (serial over chunks; parallel over value slice x head x sequence)
+// pass 2, SIMT: inter-chunk (serial over chunks; parallel over slice x head x sequence)
 // ---------------------------------------------------------------------------
 template <typename WT, int D, int C>
 struct P2Smem {
@@ -198,17 +201,11 @@ struct P2Smem {
 };
 
 template <typename WT>
-__device__ __forceinline__ void copy_rows(WT* dst, const WT* src, int rows, int valid, int D,
-                                          size_t row_stride) {
-  // rows x D elements, row r at src + r * row_stride; rows >= valid are zero
+__device__ __forceinline__ void copy_tile(WT* dst, const WT* src, int n) {
+  // n contiguous elements (n * sizeof(WT) a multiple of 16)
   constexpr int V = 16 / sizeof(WT);
-  const int per_row = D / V;
-  for (int e = threadIdx.x; e < rows * per_row; e += blockDim.x) {
-    const int r = e / per_row, c = (e - r * per_row) * V;
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (r < valid) val = *reinterpret_cast<const uint4*>(src + r * row_stride + c);
-    *reinterpret_cast<uint4*>(dst + r * D + c) = val;
-  }
+  for (int e = threadIdx.x; e < n / V; e += blockDim.x)
+    reinterpret_cast<uint4*>(dst)[e] = reinterpret_cast<const uint4*>(src)[e];
 }
 
 template <typename WT, int D, int C>
@@ -220,8 +217,8 @@ __global__ void __launch_bounds__(256) inter_chunk_kernel(const PrefillArgs a) {
   extern __shared__ __align__(16) unsigned char smraw[];
   WT* Wt = reinterpret_cast<WT*>(smraw);   // [C][D]
   WT* Qt = Wt + C * D;                     // [C][D]
-  WT* Kp = Qt + C * D;                     // [C][D]
-  WT* Mt = Kp + C * D;                     // [C][C]
+  WT* KT = Qt + C * D;                     // [D][C]
+  WT* Mt = KT + C * D;                     // [C][C]
   float* Ut = reinterpret_cast<float*>(smraw + ((SM::tiles + 15) / 16) * 16);  // [C][J]
   float* U = Ut + C * J;                   // [C][J]
   float* S = U + C * J;                    // [D][J]
@@ -237,7 +234,7 @@ __global__ void __launch_bounds__(256) inter_chunk_kernel(const PrefillArgs a) {
   const WT* Wg = reinterpret_cast<const WT*>(a.ws + a.L.W);
   const WT* Ug = reinterpret_cast<const WT*>(a.ws + a.L.Ut);
   const WT* Qg = reinterpret_cast<const WT*>(a.ws + a.L.Qt);
-  const WT* Kg = reinterpret_cast<const WT*>(a.ws + a.L.Kp);
+  const WT* KTg = reinterpret_cast<const WT*>(a.ws + a.L.Kp);
   const WT* Mg = reinterpret_cast<const WT*>(a.ws + a.L.M);
   const float* gCg = reinterpret_cast<const float*>(a.ws + a.L.gC);
   float* og = reinterpret_cast<float*>(a.ws + a.L.o);
@@ -250,20 +247,18 @@ __global__ void __launch_bounds__(256) inter_chunk_kernel(const PrefillArgs a) {
 
   const int nch = (end - start + C - 1) / C;
   for (int ci = 0; ci < nch; ++ci) {
-    const int slot = start / C + s + ci;
+    const size_t tile = (size_t)(start / C + s + ci) * H + h;
     const int t0 = start + ci * C;
     const int L = min(C, end - t0);
-    const size_t rstride = (size_t)H * D;
-    const size_t tok0 = ((size_t)t0 * H + h) * D;
-    copy_rows(Wt, Wg + tok0, C, L, D, rstride);
-    copy_rows(Qt, Qg + tok0, C, L, D, rstride);
-    copy_rows(Kp, Kg + tok0, C, L, D, rstride);
-    copy_rows(Mt, Mg + ((size_t)slot * H + h) * C * C, C, C, C, (size_t)C);
+    copy_tile(Wt, Wg + tile * C * D, C * D);
+    copy_tile(Qt, Qg + tile * C * D, C * D);
+    copy_tile(KT, KTg + tile * D * C, C * D);
+    copy_tile(Mt, Mg + tile * C * C, C * C);
     for (int e = tid; e < C * J; e += blockDim.x) {
       const int r = e / J, jj = e - (e / J) * J;
-      Ut[e] = (r < L) ? ld1(Ug + tok0 + (size_t)r * rstride + j0 + jj) : 0.f;
+      Ut[e] = ld1(Ug + (tile * C + r) * D + j0 + jj);
     }
-    for (int c = tid; c < D; c += blockDim.x) gC[c] = gCg[((size_t)slot * H + h) * D + c];
+    for (int c = tid; c < D; c += blockDim.x) gC[c] = gCg[tile * D + c];
     __syncthreads();
 
     // U = U~ - W S
@@ -283,7 +278,7 @@ __global__ void __launch_bounds__(256) inter_chunk_kernel(const PrefillArgs a) {
       float acc = 0.f;
       for (int c = 0; c < D; ++c) acc = fmaf(ld1(Qt + r * D + c), S[c * J + j], acc);
       for (int i = 0; i <= r; ++i) acc = fmaf(ld1(Mt + r * C + i), U[i * J + j], acc);
-      if (r < L) og[tok0 + (size_t)r * rstride + j0 + j] = acc;
+      if (r < L) og[((size_t)(t0 + r) * H + h) * D + j0 + j] = acc;
     }
     // S <- Diag(e^{G_C}) S + K'^T U
     float snew[SPT];
@@ -291,7 +286,7 @@ __global__ void __launch_bounds__(256) inter_chunk_kernel(const PrefillArgs a) {
     for (int m = 0; m < SPT; ++m) {
       const int c = rg + 16 * m;
       float acc = gC[c] * S[c * J + j];
-      for (int r = 0; r < C; ++r) acc = fmaf(ld1(Kp + r * D + c), U[r * J + j], acc);
+      for (int r = 0; r < C; ++r) acc = fmaf(ld1(KT + c * C + r), U[r * J + j], acc);
       snew[m] = acc;
     }
     __syncthreads();
@@ -342,14 +337,17 @@ template <typename T, int D, int C>
 static cudaError_t launch_prefill_dc(const PrefillArgs& a, cudaStream_t st) {
   cudaError_t e;
   {
-    auto k1 = intra_chunk_kernel<T, T, D, C>;
+    auto k1 = intra_chunk_kernel<T, D, C>;
     const size_t sm = P1Smem<D, C>::bytes;
     e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     k1<<<dim3(a.L.nslots, a.H), 256, sm, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  {
+  if (sm100_interchunk_supported(a)) {
+    e = launch_interchunk_sm100(a, st);
+    if (e != cudaSuccess) return e;
+  } else {
     auto k2 = inter_chunk_kernel<T, D, C>;
     const size_t sm = P2Smem<T, D, C>::bytes;
     e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);

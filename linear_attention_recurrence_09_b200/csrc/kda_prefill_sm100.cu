@@ -1,0 +1,494 @@
+// Inter-chunk pass of kda_prefill on the 5th-generation tensor cores (sm_100a):
+// bf16 tcgen05 MMAs fed by TMA, fp32 accumulators in TMEM, the fp32 state carried
+// on chip through the chunks of a sequence.  Used for d = 128, chunk 64, bf16.
+//
+// One CTA per (32-column value slice, head, sequence): the columns of the state
+// evolve independently (each obeys the recurrence with the same k, a, b), so a
+// head's 128 value columns are split over 4 CTAs and the serial chain of a
+// sequence runs on 4 SMs at once.  Per chunk (C = 64 tokens), with S the bf16
+// copy of the state slice (128 x 32):
+//   MMA1   D1[128 x 32]  = [W ; Q~] (128 x 128) . S          -> rows 0-63: W S, rows 64-127: Q~ S
+//   E1     U = U~ - W S  (fp32, rows past the sequence end forced to 0) -> bf16 U^T in smem
+//   MMA2   D2[128 x 32]  = K'^T (128 x 64) . U               (state increment, key rows)
+//   MMA3   D1[64:128]   += M (64 x 64) . U                   (O = Q~ S + M U; A = [0 ; M])
+//   E2     S <- Diag(e^{G_C}) S + D2 in fp32 registers (one key row per thread) -> bf16 S^T
+//   E3     O rows of D1 -> o (fp32, workspace) for the gated RMSNorm pass
+// Warp roles: warp 0 issues TMA (two smem stages, so chunk n+1 loads while n
+// computes), warp 1 allocates TMEM and issues the MMAs (one thread), warps 2-5
+// run the epilogues (TMEM lane quarter = warp % 4).  Every operand is K-major
+// with the 128-byte swizzle: TMA writes the workspace tiles in that layout and
+// the epilogue threads write S^T and U^T in it by hand.
+//
+// Every wait is bounded (about a second): on expiry the CTA records
+// KDA_ERR_TIMEOUT in the workspace status word, drains what it issued, frees
+// its TMEM and exits; the host reads the word with kda_workspace_status.
+#include <cuda.h>
+
+#include "kda_common.cuh"
+#include "kda_launch.h"
+
+namespace kda {
+namespace {
+
+constexpr int D = 128, C = 64, J = 32, NSLICE = D / J;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 128;
+
+// shared memory carve-up (offsets from a 1024-byte aligned base)
+constexpr uint32_t A1_BYTES = 2 * 128 * 128;     // [W;Q~]: 2 K-blocks x 128 rows x 128 B
+constexpr uint32_t A2_BYTES = 128 * 128;         // K'^T : 128 key rows x 64 tokens
+constexpr uint32_t A3_BYTES = 128 * 128;         // [0;M]: 128 rows x 64 (rows 0-63 zero)
+constexpr uint32_t STAGE_BYTES = A1_BYTES + A2_BYTES + A3_BYTES;
+constexpr uint32_t NSTAGE = 2;
+constexpr uint32_t TX_BYTES = 4 * 8192 + 16384 + 8192;   // W x2, Q~ x2, K'^T, M
+constexpr uint32_t OFF_S = NSTAGE * STAGE_BYTES;          // S^T: 2 K-blocks x 32 rows x 128 B
+constexpr uint32_t OFF_U = OFF_S + 2 * J * 128;           // U^T: 32 rows x 128 B
+constexpr uint32_t OFF_BAR = OFF_U + J * 128;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 128 + 1024;     // barriers + alignment slack
+
+// barrier slots (8 bytes each)
+enum { BAR_FULL0 = 0, BAR_FULL1, BAR_EMPTY0, BAR_EMPTY1, BAR_MMA1, BAR_MMA2, BAR_SREADY,
+       BAR_UREADY, BAR_COUNT };
+
+constexpr long long WAIT_LIMIT_CYCLES = 2000000000LL;    // ~1 s at 1.9-2 GHz
+
+struct TmaMaps {
+  CUtensorMap W, Q, KT, M;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// bounded wait: false on timeout or when another role already gave up
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+      *abort_flag = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+// warp-uniform bounded wait: every lane observes the phase (acquire), and the
+// decision to give up is taken by the whole warp together, so the warp stays
+// converged for the .sync.aligned tcgen05 instructions that follow
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
+                                               volatile int* abort_flag) {
+  const long long t0 = clock64();
+  while (true) {
+    const bool done = mbar_try(bar, parity);
+    if (__all_sync(0xffffffffu, done)) return true;
+    const bool give_up = (*abort_flag != 0) || (clock64() - t0 > WAIT_LIMIT_CYCLES);
+    if (__any_sync(0xffffffffu, give_up)) {
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// K-major operand, 128-byte swizzle: 8-row groups 1024 B apart
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;               // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;     // stride byte offset
+  d |= (uint64_t)1 << 46;               // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;               // SWIZZLE_128B
+  return d;
+}
+
+// kind::f16 instruction descriptor: bf16 A and B (K-major), fp32 accumulator
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                     uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// byte offset of element (row n, k) in a K-major, 128B-swizzled tile of 64-wide rows
+__device__ __forceinline__ uint32_t sw128_off(int n, int k) {
+  return (uint32_t)(n * 128 + ((((k >> 3) ^ (n & 7)) & 7) << 4) + (k & 7) * 2);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps maps) {
+  extern __shared__ __align__(1024) unsigned char smraw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(sm);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  __shared__ uint32_t tmem_holder;
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j0 = blockIdx.x * J, h = blockIdx.y, s = blockIdx.z, H = a.H;
+  const int row = pool_row(a.slots, s, a.pool_size);
+  if (row < 0) return;
+  int start, end;
+  seq_range(a.cu, a.total, s, start, end);
+  const int nch = (end - start + C - 1) / C;
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(bar(BAR_FULL0), 1);
+    mbar_init(bar(BAR_FULL1), 1);
+    mbar_init(bar(BAR_EMPTY0), 1);
+    mbar_init(bar(BAR_EMPTY1), 1);
+    mbar_init(bar(BAR_MMA1), 1);
+    mbar_init(bar(BAR_MMA2), 1);
+    mbar_init(bar(BAR_SREADY), 128);
+    mbar_init(bar(BAR_UREADY), 64);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // rows 0-63 of every A3 tile are the zero half of [0 ; M]
+  for (uint32_t st = 0; st < NSTAGE; ++st) {
+    uint4* z = reinterpret_cast<uint4*>(sm + st * STAGE_BYTES + A1_BYTES + A2_BYTES);
+    for (int i = threadIdx.x; i < 8192 / 16; i += THREADS) z[i] = make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async();
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&tmem_holder)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_holder;
+  const uint32_t d1_tmem[2] = {tmem + 0, tmem + 32};
+  const uint32_t d2_tmem = tmem + 64;
+  int* status = reinterpret_cast<int*>(a.ws + a.L.status);
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int n = 0; n < nch && !abort_flag; ++n) {
+        const int st = n & 1;
+        if (n >= 2 && !mbar_wait(bar(BAR_EMPTY0 + st), ((n >> 1) - 1) & 1, &abort_flag)) break;
+        const int tile = (start / C + s + n) * H + h;
+        const uint32_t A1 = sbase + st * STAGE_BYTES, A2 = A1 + A1_BYTES, A3 = A2 + A2_BYTES;
+        mbar_expect_tx(bar(BAR_FULL0 + st), TX_BYTES);
+        tma_load_2d(A1, &maps.W, 0, tile * C, bar(BAR_FULL0 + st));
+        tma_load_2d(A1 + 16384, &maps.W, 64, tile * C, bar(BAR_FULL0 + st));
+        tma_load_2d(A1 + 8192, &maps.Q, 0, tile * C, bar(BAR_FULL0 + st));
+        tma_load_2d(A1 + 16384 + 8192, &maps.Q, 64, tile * C, bar(BAR_FULL0 + st));
+        tma_load_2d(A2, &maps.KT, 0, tile * D, bar(BAR_FULL0 + st));
+        tma_load_2d(A3 + 8192, &maps.M, 0, tile * C, bar(BAR_FULL0 + st));
+        issued = n + 1;
+      }
+      if (abort_flag) {  // let the copies this thread started land before the CTA exits
+        for (int n = (issued >= 2 ? issued - 2 : 0); n < issued; ++n) {
+          const long long t0 = clock64();
+          while (!mbar_try(bar(BAR_FULL0 + (n & 1)), (n >> 1) & 1) &&
+                 clock64() - t0 < WAIT_LIMIT_CYCLES) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t id = idesc_bf16(128, J);
+      int last = -1;
+      for (int n = 0; n < nch; ++n) {
+        const int st = n & 1;
+        if (!mbar_wait(bar(BAR_FULL0 + st), (n >> 1) & 1, &abort_flag)) break;
+        if (!mbar_wait(bar(BAR_SREADY), n & 1, &abort_flag)) break;
+        tc_fence_after();
+        const uint32_t A1 = sbase + st * STAGE_BYTES, A2 = A1 + A1_BYTES, A3 = A2 + A2_BYTES;
+        const uint32_t SB = sbase + OFF_S, UB = sbase + OFF_U;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          umma(d1_tmem[st], sw128_desc(A1 + (k >> 2) * 16384 + (k & 3) * 32),
+               sw128_desc(SB + (k >> 2) * 4096 + (k & 3) * 32), id, k > 0);
+        umma_commit(bar(BAR_MMA1));
+        last = n;
+        if (!mbar_wait(bar(BAR_UREADY), n & 1, &abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma(d2_tmem, sw128_desc(A2 + k * 32), sw128_desc(UB + k * 32), id, k > 0);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma(d1_tmem[st], sw128_desc(A3 + k * 32), sw128_desc(UB + k * 32), id, 1);
+        umma_commit(bar(BAR_MMA2));
+        umma_commit(bar(BAR_EMPTY0 + st));
+      }
+      if (abort_flag && last >= 0) {  // let the issued MMAs retire before TMEM is freed
+        const long long t0 = clock64();
+        while (!mbar_try(bar(BAR_MMA1), last & 1) && clock64() - t0 < WAIT_LIMIT_CYCLES) {
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue warps 2-5 ----------------
+    const int q = warp & 3;                 // TMEM lane quarter
+    const int i = 32 * q + lane;            // key row of the state slice / TMEM lane
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    unsigned char* SB = sm + OFF_S;
+    unsigned char* UB = sm + OFF_U;
+    const float* gCg = reinterpret_cast<const float*>(a.ws + a.L.gC);
+    const __nv_bfloat16* Ug = reinterpret_cast<const __nv_bfloat16*>(a.ws + a.L.Ut);
+    float* og = reinterpret_cast<float*>(a.ws + a.L.o);
+    const size_t sg = (((size_t)row * H + h) * D + i) * D + j0;
+
+    float S[32];
+    if (a.state_in) {
+#pragma unroll
+      for (int c = 0; c < 32; c += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(a.state_in + sg + c);
+        S[c] = v.x; S[c + 1] = v.y; S[c + 2] = v.z; S[c + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) S[c] = 0.f;
+    }
+    auto write_state = [&]() {
+      unsigned char* blk = SB + (i >> 6) * 4096;
+#pragma unroll
+      for (int n = 0; n < 32; ++n)
+        *reinterpret_cast<__nv_bfloat16*>(blk + sw128_off(n, i & 63)) = __float2bfloat16_rn(S[n]);
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(bar(BAR_SREADY));
+    };
+    write_state();
+
+    for (int n = 0; n < nch; ++n) {
+      const int st = n & 1;
+      const int tile = (start / C + s + n) * H + h;
+      const int t0 = start + n * C;
+      const int L = min(C, end - t0);
+      const float gc = __ldg(gCg + (size_t)tile * D + i);
+      if (q < 2) {
+        // E1: U = U~ - W S for token row r = i (0..63)
+        float ut[32];
+        const __nv_bfloat16* up = Ug + ((size_t)tile * C + i) * D + j0;
+#pragma unroll
+        for (int c = 0; c < 32; c += 8) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(up + c);
+          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const float2 f = __bfloat1622float2(p2[m]);
+            ut[c + 2 * m] = f.x; ut[c + 2 * m + 1] = f.y;
+          }
+        }
+        if (!mbar_wait_warp(bar(BAR_MMA1), n & 1, &abort_flag)) break;
+        tc_fence_after();
+        float ws[32];
+        tmem_ld32(d1_tmem[st] + lane_off, ws);
+#pragma unroll
+        for (int m = 0; m < 32; ++m) {
+          const float u = (i < L) ? ut[m] - ws[m] : 0.f;
+          *reinterpret_cast<__nv_bfloat16*>(UB + sw128_off(m, i)) = __float2bfloat16_rn(u);
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(bar(BAR_UREADY));
+      }
+      // E2: state update for key row i
+      if (!mbar_wait_warp(bar(BAR_MMA2), n & 1, &abort_flag)) break;
+      tc_fence_after();
+      {
+        float dv[32];
+        tmem_ld32(d2_tmem + lane_off, dv);
+#pragma unroll
+        for (int m = 0; m < 32; ++m) S[m] = fmaf(gc, S[m], dv[m]);
+      }
+      if (q >= 2) {
+        // E3: O rows (TMEM lanes 64-127) -> o
+        float o[32];
+        tmem_ld32(d1_tmem[st] + lane_off, o);
+        const int r = i - 64;
+        if (r < L) {
+          float* op = og + ((size_t)(t0 + r) * H + h) * D + j0;
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            *reinterpret_cast<float4*>(op + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+        }
+      }
+      write_state();
+    }
+    if (!abort_flag && a.state_out) {
+#pragma unroll
+      for (int c = 0; c < 32; c += 4)
+        *reinterpret_cast<float4*>(a.state_out + sg + c) =
+            make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (abort_flag && threadIdx.x == 0) atomicExch(status, (int)5 /* KDA_ERR_TIMEOUT */);
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// Self-test of the bounded wait: one warp waits on an mbarrier that nothing
+// arrives at, gives up after `limit` cycles and records KDA_ERR_TIMEOUT in the
+// status word, exactly as the prefill kernel does on a stalled pipeline.
+__global__ void __launch_bounds__(32) wait_timeout_selftest_kernel(int* status, long long limit) {
+  __shared__ __align__(8) uint64_t never;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&never), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  const long long t0 = clock64();
+  bool ok = true;
+  while (!mbar_try(smem_u32(&never), 0)) {
+    if (clock64() - t0 > limit) { ok = false; break; }
+  }
+  if (!ok && threadIdx.x == 0) atomicExch(status, 5 /* KDA_ERR_TIMEOUT */);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<EncodeTiledFn>(fn);
+}
+
+// 2D bf16 tensor [rows, cols] (cols contiguous), box [box_rows, 64 cols], 128B swizzle
+bool make_map(EncodeTiledFn enc, CUtensorMap* m, void* base, uint64_t rows, uint64_t cols,
+              uint32_t box_rows) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_wait_timeout_selftest(void* workspace, cudaStream_t st) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(static_cast<int*>(workspace),
+                                                 WAIT_LIMIT_CYCLES / 4);
+  return cudaGetLastError();
+}
+
+bool sm100_interchunk_supported(const PrefillArgs& a) {
+  return a.bf16 && a.D == D && a.C == C;
+}
+
+cudaError_t launch_interchunk_sm100(const PrefillArgs& a, cudaStream_t st) {
+  static_assert(NSLICE * J == D, "slices must cover the value axis");
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  TmaMaps maps;
+  const uint64_t tiles = (uint64_t)a.L.nslots * a.H;
+  if (!make_map(enc, &maps.W, a.ws + a.L.W, tiles * C, D, 64) ||
+      !make_map(enc, &maps.Q, a.ws + a.L.Qt, tiles * C, D, 64) ||
+      !make_map(enc, &maps.KT, a.ws + a.L.Kp, tiles * D, C, 128) ||
+      !make_map(enc, &maps.M, a.ws + a.L.M, tiles * C, C, 64))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(interchunk_sm100_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  interchunk_sm100_kernel<<<dim3(NSLICE, a.H, a.n_seqs), THREADS, SMEM_BYTES, st>>>(a, maps);
+  return cudaGetLastError();
+}
+
+}  // namespace kda

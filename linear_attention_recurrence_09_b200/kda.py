@@ -31,7 +31,7 @@ KDA_CONV_TAPE = 1
 
 ENTRY_POINTS = ('kda_status_string', 'kda_abi_version', 'kda_prep',
                 'kda_prefill_workspace_size', 'kda_prefill', 'kda_decode', 'kda_verify',
-                'kda_rollback', 'kda_workspace_status')
+                'kda_rollback', 'kda_workspace_status', 'kda_selftest_wait_timeout')
 
 
 class KdaError(RuntimeError):
@@ -106,6 +106,8 @@ def lib() -> ctypes.CDLL:
                                    _I, _P]
         L.kda_workspace_status.restype = ctypes.c_int
         L.kda_workspace_status.argtypes = [_P, _P]
+        L.kda_selftest_wait_timeout.restype = ctypes.c_int
+        L.kda_selftest_wait_timeout.argtypes = [_P, _P]
         _lib = L
     return _lib
 
@@ -297,6 +299,12 @@ def kda_rollback(cfg: Config, accepted, tape, state, conv_window=None, conv_stat
 def kda_workspace_status(workspace, stream=None) -> int:
     """Synchronise the stream and return the prefill workspace status code."""
     return int(lib().kda_workspace_status(_ptr(workspace, None, 'workspace'), _stream(stream)))
+
+
+def kda_selftest_wait_timeout(workspace, stream=None):
+    """Run the bounded-wait self-test on ``workspace`` (enqueue only)."""
+    _check(lib().kda_selftest_wait_timeout(_ptr(workspace, None, 'workspace'), _stream(stream)),
+           'kda_selftest_wait_timeout')
 
 
 # ---------------------------------------------------------------------------

@@ -258,3 +258,17 @@ def test_state_pool_slots():
         torch.cuda.synchronize()
         assert torch.equal(st[0], pool_state[r])
         assert torch.equal(y1[0], y[b])
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """A wait that nothing completes gives up, reports KDA_ERR_TIMEOUT, and the
+    context keeps working (failure detection without a GPU fault)."""
+    ws = torch.empty(4096, dtype=torch.uint8, device='cuda')
+    kda.kda_selftest_wait_timeout(ws)
+    assert kda.kda_workspace_status(ws) == kda.KDA_ERR_TIMEOUT
+    cfg, P, A, S0, hist = make_case(15, [20], 2, 64, 4, torch.bfloat16, state_var=0.01)
+    _assert(compare_layer(cfg, P, A, S0, hist), 1e-2)
+    w2 = kda.prefill_workspace(cfg, 1, 20)
+    kda.layer_prefill(cfg, {k: v.cuda() for k, v in P.items()},
+                      {k: v.cuda() for k, v in A.items()}, workspace=w2)
+    assert kda.kda_workspace_status(w2) == kda.KDA_OK
