@@ -71,7 +71,8 @@ enum kda_status {
   KDA_ERR_UNSUPPORTED = 3,  /* valid but not built: e.g. head_dim not in {16,32,64,128} */
   KDA_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
   KDA_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up (see kda_workspace_status) */
-  KDA_ERR_WORKSPACE = 6     /* workspace missing or smaller than kda_prefill_workspace_size */
+  KDA_ERR_WORKSPACE = 6,    /* workspace missing or smaller than kda_prefill_workspace_size */
+  KDA_ERR_SCRATCH_LIMIT = 7 /* problem needs more scratch than kda_prefill_noalloc has */
 };
 
 enum kda_dtype { KDA_F32 = 0, KDA_BF16 = 1 };
@@ -232,6 +233,41 @@ KDA_API int kda_rollback(const kda_config* cfg, int32_t batch, int32_t block_len
  * workspace gave up (its outputs are then invalid).
  */
 KDA_API int kda_workspace_status(const void* workspace, kda_stream_t stream);
+
+/*
+ * kda_prefill_noalloc - kda_prefill for callers that cannot allocate device
+ * memory.  The pages have no counterpart to this entry point.
+ *
+ * Some callers cannot call cudaMalloc: code embedded in a host framework that owns
+ * every byte of device memory (a serving engine that reserves the whole HBM for
+ * its own pools up front), or a path that must not pay cudaMalloc's latency and
+ * device-wide synchronisation.  This entry point takes the same inputs and
+ * outputs as kda_prefill (the caller still passes and owns them) but keeps its
+ * scratch in one fixed array of KDA_NOALLOC_SCRATCH_BYTES (64 MiB) of device
+ * memory inside the library, so it allocates nothing and frees nothing.
+ *
+ *  - Limit: problems whose kda_prefill_workspace_size() exceeds
+ *    KDA_NOALLOC_SCRATCH_BYTES are rejected with KDA_ERR_SCRATCH_LIMIT before
+ *    anything is launched (at H = 32, d = 128, chunk 64, bf16 a single sequence
+ *    of about 1,000 tokens fits).
+ *  - Memory: every GPU that loads the library holds the 64 MiB until the process
+ *    exits.
+ *  - Set-up: the first call on each device (with that device current) looks up
+ *    the array's device address and caches it; make that first call before any
+ *    stream capture.
+ *  - Sharing: every call on a device uses the same array, which keeps the last
+ *    call's contents.  Calls that overlap on the GPU (different streams, or
+ *    different host threads) race on it and give undefined results; order them.
+ *  - Status: kda_workspace_status cannot see this scratch; a bounded-wait
+ *    timeout here leaves the outputs invalid without a readable status word.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+KDA_API int kda_prefill_noalloc(const kda_config* cfg, int32_t n_seqs, int32_t total_tokens,
+                                const int32_t* cu_seqlens, const void* q, const void* k,
+                                const void* v, const float* log_a, const float* beta,
+                                const void* g, const float* norm_w, const float* state_in,
+                                float* state_out, const int32_t* state_slots,
+                                int32_t pool_size, void* y, kda_stream_t stream);
 
 /*
  * kda_selftest_wait_timeout - failure-detection self-test.  Enqueues one warp

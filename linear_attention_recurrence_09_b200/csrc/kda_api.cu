@@ -63,6 +63,8 @@ const char* kda_status_string(int status) {
     case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA launch or runtime call failed";
     case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a bounded device wait gave up";
     case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing or too small";
+    case KDA_ERR_SCRATCH_LIMIT:
+      return "KDA_ERR_SCRATCH_LIMIT: problem exceeds the fixed scratch of kda_prefill_noalloc";
   }
   return "unknown kda status";
 }

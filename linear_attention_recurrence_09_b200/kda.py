@@ -24,6 +24,8 @@ KDA_ERR_UNSUPPORTED = 3
 KDA_ERR_CUDA = 4
 KDA_ERR_TIMEOUT = 5
 KDA_ERR_WORKSPACE = 6
+KDA_ERR_SCRATCH_LIMIT = 7
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 KDA_F32 = 0
 KDA_BF16 = 1
 KDA_CONV_COMMIT = 0
@@ -31,7 +33,8 @@ KDA_CONV_TAPE = 1
 
 ENTRY_POINTS = ('kda_status_string', 'kda_abi_version', 'kda_prep',
                 'kda_prefill_workspace_size', 'kda_prefill', 'kda_decode', 'kda_verify',
-                'kda_rollback', 'kda_workspace_status', 'kda_selftest_wait_timeout')
+                'kda_rollback', 'kda_workspace_status', 'kda_selftest_wait_timeout',
+                'kda_prefill_noalloc')
 
 
 class KdaError(RuntimeError):
@@ -108,6 +111,9 @@ def lib() -> ctypes.CDLL:
         L.kda_workspace_status.argtypes = [_P, _P]
         L.kda_selftest_wait_timeout.restype = ctypes.c_int
         L.kda_selftest_wait_timeout.argtypes = [_P, _P]
+        L.kda_prefill_noalloc.restype = ctypes.c_int
+        L.kda_prefill_noalloc.argtypes = [ctypes.POINTER(CConfig), _I, _I, _P, _P, _P, _P, _P,
+                                          _P, _P, _P, _P, _P, _P, _I, _P, _P]
         _lib = L
     return _lib
 
@@ -229,6 +235,33 @@ def kda_prefill(cfg: Config, cu_seqlens, q, k, v, log_a, beta, g, norm_w, state_
         _ptr(y, cfg.dtype, 'y', (T, H, d)), _ptr(workspace, None, 'workspace'),
         int(workspace.numel() * workspace.element_size()), _stream(stream))
     _check(st, 'kda_prefill')
+    return y
+
+
+def kda_prefill_noalloc(cfg: Config, cu_seqlens, q, k, v, log_a, beta, g, norm_w,
+                        state_in=None, state_out=None, state_slots=None, pool_size=None, y=None,
+                        stream=None):
+    """kda_prefill with the library's fixed device scratch (the entry point itself
+    allocates nothing; pass ``y`` to avoid the one torch allocation made here)."""
+    H, d = cfg.num_heads, cfg.head_dim
+    T = q.shape[0]
+    N = cu_seqlens.numel() - 1
+    if y is None:
+        y = _empty((T, H, d), cfg.dtype, q.device)
+    if pool_size is None:
+        ref = state_in if state_in is not None else state_out
+        pool_size = ref.shape[0] if ref is not None else N
+    c = cfg.c()
+    st = lib().kda_prefill_noalloc(
+        ctypes.byref(c), N, T, _ptr(cu_seqlens, torch.int32, 'cu_seqlens'),
+        _ptr(q, torch.float32, 'q', (T, H, d)), _ptr(k, torch.float32, 'k', (T, H, d)),
+        _ptr(v, torch.float32, 'v', (T, H, d)), _ptr(log_a, torch.float32, 'log_a', (T, H, d)),
+        _ptr(beta, torch.float32, 'beta', (T, H)), _ptr(g, cfg.dtype, 'g', (T, H, d)),
+        _ptr(norm_w, torch.float32, 'norm_w', (d,)),
+        _ptr(state_in, torch.float32, 'state_in'), _ptr(state_out, torch.float32, 'state_out'),
+        _ptr(state_slots, torch.int32, 'state_slots'), int(pool_size),
+        _ptr(y, cfg.dtype, 'y', (T, H, d)), _stream(stream))
+    _check(st, 'kda_prefill_noalloc')
     return y
 
 

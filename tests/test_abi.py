@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported(L):
 
 def test_version_and_status_strings(L):
     assert kda.kda_abi_version() == 1
-    for code in range(7):
+    for code in range(8):
         assert kda.kda_status_string(code).startswith('KDA_')
     assert 'unknown' in kda.kda_status_string(99)
 
