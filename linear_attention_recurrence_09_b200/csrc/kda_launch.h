@@ -96,6 +96,8 @@ cudaError_t launch_step(const StepArgs& a, cudaStream_t st);
 cudaError_t launch_rollback(const RollbackArgs& a, cudaStream_t st);
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st);
 bool sm100_interchunk_supported(const PrefillArgs& a);
+bool sm100_intra_supported(const PrefillArgs& a);
+cudaError_t launch_intra_sm100(const PrefillArgs& a, cudaStream_t st);
 cudaError_t launch_interchunk_sm100(const PrefillArgs& a, cudaStream_t st);
 cudaError_t launch_wait_timeout_selftest(void* workspace, cudaStream_t st);
 int prep_tile();

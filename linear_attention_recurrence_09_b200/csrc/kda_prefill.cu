@@ -336,7 +336,10 @@ __global__ void __launch_bounds__(256) gated_norm_kernel(const PrefillArgs a) {
 template <typename T, int D, int C>
 static cudaError_t launch_prefill_dc(const PrefillArgs& a, cudaStream_t st) {
   cudaError_t e;
-  {
+  if (sm100_intra_supported(a)) {
+    e = launch_intra_sm100(a, st);
+    if (e != cudaSuccess) return e;
+  } else {
     auto k1 = intra_chunk_kernel<T, D, C>;
     const size_t sm = P1Smem<D, C>::bytes;
     e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);

@@ -51,17 +51,28 @@ prep_kernel(const PrepArgs a) {
       wsm[j][ch] = __ldg(a.conv_w + ((size_t)h * C3 + ch) * K + j);
       wsm[j][ch + 1] = __ldg(a.conv_w + ((size_t)h * C3 + ch + 1) * K + j);
     }
-    for (int r = 0; r < nrows; ++r) {
+    // all staged rows are loaded before any is stored, so the loads overlap
+    float2 stage[PREP_TILE + PREP_KMAX - 1];
+#pragma unroll
+    for (int r = 0; r < PREP_TILE + PREP_KMAX - 1; ++r) {
       const int tok = tr.t0 - Km1 + r;
       float2 val = make_float2(0.f, 0.f);
-      if (tok >= tr.start) {
-        val = ld2(x + ((size_t)tok * H + h) * C3 + ch);
-      } else if (cs != nullptr) {
-        const int hr = Km1 + (tok - tr.start);  // history row, 0 = oldest
-        val = ld2(cs + (((size_t)row * Km1 + hr) * H + h) * C3 + ch);
+      if (r < nrows) {
+        if (tok >= tr.start) {
+          val = ld2(x + ((size_t)tok * H + h) * C3 + ch);
+        } else if (cs != nullptr) {
+          const int hr = Km1 + (tok - tr.start);  // history row, 0 = oldest
+          val = ld2(cs + (((size_t)row * Km1 + hr) * H + h) * C3 + ch);
+        }
       }
-      xs[r][ch] = val.x;
-      xs[r][ch + 1] = val.y;
+      stage[r] = val;
+    }
+#pragma unroll
+    for (int r = 0; r < PREP_TILE + PREP_KMAX - 1; ++r) {
+      if (r < nrows) {
+        xs[r][ch] = stage[r].x;
+        xs[r][ch + 1] = stage[r].y;
+      }
     }
   }
 
@@ -134,14 +145,30 @@ prep_kernel(const PrepArgs a) {
     }
   }
 
-  // decay gate and beta
+  // decay gate and beta (loads first, then the arithmetic)
   const T* __restrict__ f = static_cast<const T*>(a.f);
   const float Ah = expf(__ldg(a.A_log + h));
-  for (int e = tid; e < tr.len * D; e += blockDim.x) {
-    const int i = e / D, c = e - (e / D) * D;
-    const size_t idx = ((size_t)(tr.t0 + i) * H + h) * D + c;
-    const float z = Ah * (ld1(f + idx) + __ldg(a.dt_bias + (size_t)h * D + c));
-    a.loga[idx] = a.lb * sigmoid(z);
+  constexpr int NTHR = ((3 * D / 2 + 31) / 32) * 32;      // the launch's block size
+  constexpr int NB = (PREP_TILE * D + NTHR - 1) / NTHR;  // elements per thread
+  const int nthr = NTHR;
+  float fv[NB];
+#pragma unroll
+  for (int m = 0; m < NB; ++m) {
+    const int e = tid + m * nthr;
+    fv[m] = 0.f;
+    if (e < tr.len * D) {
+      const int i = e / D, c = e - (e / D) * D;
+      fv[m] = ld1(f + ((size_t)(tr.t0 + i) * H + h) * D + c);
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < NB; ++m) {
+    const int e = tid + m * nthr;
+    if (e < tr.len * D) {
+      const int i = e / D, c = e - (e / D) * D;
+      const size_t idx = ((size_t)(tr.t0 + i) * H + h) * D + c;
+      a.loga[idx] = a.lb * sigmoid(Ah * (fv[m] + __ldg(a.dt_bias + (size_t)h * D + c)));
+    }
   }
   if (tid < tr.len) {
     const size_t idx = (size_t)(tr.t0 + tid) * H + h;

@@ -97,7 +97,10 @@ def test_beta_zero_no_decay_keeps_state_bit_exact():
 
 
 def test_split_invariance_5_plus_7():
-    """glm53-flash-mlx README test [5]: prefill 5 then 7 equals prefill 12."""
+    """glm53-flash-mlx README test [5]: prefill 5 then 7 equals prefill 12.
+
+    Both spellings are held to the oracle bar (each carries its own bf16
+    rounding); the conv history they leave is bit-identical."""
     cfg, P, A, S0, hist = make_case(9, [12], 2, 128, 4, torch.bfloat16, state_var=0.01,
                                     conv_hist=True, chunk=64)
     y_full, s_full, c_full, _ = gpu_layer(cfg, P, A, S0, hist)
@@ -108,8 +111,11 @@ def test_split_invariance_5_plus_7():
     y1, s1, c1, _ = gpu_layer(cfg, P, a1, S0, hist)
     y2, s2, c2, _ = gpu_layer(cfg, P, a2, s1.cpu(), c1.cpu())
     y_split = torch.cat([y1, y2]).cpu()
-    assert rel_err(np64(y_split), np64(y_full)) <= 1e-2
-    assert rel_err(np64(s2), np64(s_full)) <= 1e-2
+    ref = oracle_layer(cfg, P, A, S0, hist)
+    for y, s in ((y_full, s_full), (y_split, s2)):
+        assert rel_err(np64(y), ref['y']) <= 1e-2
+        assert rel_err(np64(s), ref['state']) <= 1e-2
+    assert rel_err(np64(y_split), np64(y_full)) <= 2e-2
     assert torch.equal(c2.cpu(), c_full.cpu())
 
 
