@@ -88,9 +88,17 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   __nv_bfloat16* KP = reinterpret_cast<__nv_bfloat16*>(sm + OFF_KP);
 
   // ---- log decay -> G (rows past the sequence end add 0), beta ----
-  for (int e = tid; e < C * D; e += THREADS) {
-    const int r = e >> 7, c = e & 127;
-    G[e] = (r < L) ? __ldg(a.loga + ((size_t)(t0 + r) * H + h) * D + c) : 0.f;
+  {
+    float4 lv[8];   // 8 float4 per thread, all in flight before the first store
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const int e4 = tid + m * THREADS;         // float4 index in the [64][128] tile
+      const int r = e4 >> 5, c4 = (e4 & 31) * 4;
+      lv[m] = (r < L) ? ld4(a.loga + ((size_t)(t0 + r) * H + h) * D + c4)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m) reinterpret_cast<float4*>(G)[tid + m * THREADS] = lv[m];
   }
   if (tid < C) bs[tid] = (tid < L) ? __ldg(a.beta + (size_t)(t0 + tid) * H + h) : 0.f;
   if (tid == 0) {
@@ -121,15 +129,27 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
 
   // ---- elementwise operands: 4 consecutive channels of one token row per item ----
   const float qsc = a.q_scale;
-  for (int it = tid; it < C * (D / 4); it += THREADS) {
+  constexpr int BATCH = 4;   // items whose loads are in flight together
+#pragma unroll 1
+  for (int b0 = 0; b0 < (C * (D / 4)) / THREADS; b0 += BATCH) {
+  float4 qa[BATCH], ka[BATCH], va[BATCH];
+#pragma unroll
+  for (int u = 0; u < BATCH; ++u) {
+    const int it = tid + (b0 + u) * THREADS;
     const int r = it >> 5, c4 = (it & 31) * 4;
-    float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), k4 = q4, v4 = q4;
+    qa[u] = ka[u] = va[u] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (r < L) {
       const size_t idx = ((size_t)(t0 + r) * H + h) * D + c4;
-      q4 = ld4(a.q + idx);
-      k4 = ld4(a.k + idx);
-      v4 = ld4(a.v + idx);
+      qa[u] = ld4(a.q + idx);
+      ka[u] = ld4(a.k + idx);
+      va[u] = ld4(a.v + idx);
     }
+  }
+#pragma unroll
+  for (int u = 0; u < BATCH; ++u) {
+    const int it = tid + (b0 + u) * THREADS;
+    const int r = it >> 5, c4 = (it & 31) * 4;
+    const float4 q4 = qa[u], k4 = ka[u], v4 = va[u];
     const float qv[4] = {q4.x, q4.y, q4.z, q4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w};
     float kb[4], qb[4], kc0[4], kc1[4], qt[4], kt[4], kp[4];
     const int rref = (r < 32) ? 15 : 47;
@@ -166,6 +186,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     st4(Qo + (size_t)r * D + c4, make_float4(qt[0], qt[1], qt[2], qt[3]));
 #pragma unroll
     for (int j = 0; j < 4; ++j) KP[(c4 + j) * KP_LD + r] = __float2bfloat16_rn(kp[j]);
+  }
   }
   fence_proxy_async();
   __syncthreads();

@@ -5,174 +5,166 @@
 // the conv; q/k use max(sqrt(sum), eps) with the literal eps 1e-6; the decay is
 // the bounded sigmoid with dt_bias per channel and per-head A broadcast.
 //
-// One CTA per (16-token tile, head).  The tile's K-1+16 pre-conv rows are staged
-// in shared memory (history rows from the conv state or zeros), each thread owns
-// two adjacent channels of the head's 3d, and the per-token L2 sums are reduced
-// across the d/2 threads of the q (resp. k) channel group.  HBM-bound: every
-// input byte is read once (plus a K-1 row halo per tile) and every output byte
-// written once.
+// HBM-bound streaming kernel.  A CTA covers a tile of up to 64 tokens of one
+// sequence for HPB consecutive heads; each thread owns 4 adjacent channels of one
+// head's 3d (8-byte bf16 / 16-byte fp32 accesses, coalesced across the block),
+// walks the tile's tokens in order with 8 rows in flight and keeps the last K-1
+// pre-conv rows of its channels in registers, so every input byte is read once
+// (plus a K-1 row halo per tile).  The per-token L2 sums of q and k reduce by
+// shuffles inside the aligned group of d/4 threads that owns them.  The decay
+// gate and beta follow in a second coalesced pass over the tile.
 #include "kda_common.cuh"
 #include "kda_launch.h"
 
 namespace kda {
 
-constexpr int PREP_TILE = 16;
+constexpr int PREP_TILE = 64;
 constexpr int PREP_KMAX = 8;
+constexpr int PREP_THREADS = 192;
+constexpr int PREP_UNROLL = 8;     // token rows in flight per thread
 
-template <typename T, int D>
-__global__ void __launch_bounds__(((3 * D / 2 + 31) / 32) * 32)
-prep_kernel(const PrepArgs a) {
+__device__ __forceinline__ void unpack4(float4 v, float (&o)[4]) {
+  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+}
+
+template <typename T, int D, int K>
+__global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const PrepArgs a) {
   constexpr int C3 = 3 * D;
-  constexpr int NT = C3 / 2;                       // threads that own a channel pair
-  constexpr int GW = (D / 2 < 32) ? D / 2 : 32;    // shuffle width inside one part
-  constexpr int WPP = (D / 2 > 32) ? (D / 2) / 32 : 1;  // warps per part
-  constexpr int NWARP = ((NT + 31) / 32);
-  __shared__ float xs[PREP_TILE + PREP_KMAX - 1][C3];
-  __shared__ float wsm[PREP_KMAX][C3];
-  __shared__ float part_ss[PREP_TILE][NWARP];
+  constexpr int TPH = C3 / 4;                  // threads per head (4 channels each)
+  constexpr int HPB = PREP_THREADS / TPH;      // heads per CTA
+  constexpr int G = D / 4;                     // threads per q (or k, v) group
+  constexpr int KM1 = K - 1;
+  constexpr int KW = KM1 > 0 ? KM1 : 1;
 
-  const int h = blockIdx.y;
   const TileRange tr = slot_to_tile(a.cu, a.n_seqs, a.total, PREP_TILE, blockIdx.x);
   if (tr.len == 0) return;
   const int row = pool_row(a.slots, tr.seq, a.pool_size);
   if (row < 0) return;
-  const int H = a.H, K = a.K, Km1 = a.K - 1;
-  const int tid = threadIdx.x;
+  const int hs = threadIdx.x / TPH, j = threadIdx.x - hs * TPH;
+  const int h = blockIdx.y * HPB + hs;
+  const bool active = h < a.H;                 // uniform per aligned group of G threads
+  const int H = a.H;
+  const int ch = 4 * j;                        // first channel of this thread in the head's 3d
+  const int part = j / G;                      // 0 = q, 1 = k, 2 = v
   const T* __restrict__ x = static_cast<const T*>(a.x);
   const T* __restrict__ cs = static_cast<const T*>(a.conv_state);
 
-  const bool own = tid < NT;
-  const int ch = 2 * tid;          // channel pair inside the head's 3d
-  const int part = ch / D;         // 0 = q, 1 = k, 2 = v
-  const int nrows = tr.len + Km1;  // staged rows: history then this tile
-
-  if (own) {
-    for (int j = 0; j < K; ++j) {
-      wsm[j][ch] = __ldg(a.conv_w + ((size_t)h * C3 + ch) * K + j);
-      wsm[j][ch + 1] = __ldg(a.conv_w + ((size_t)h * C3 + ch + 1) * K + j);
-    }
-    // all staged rows are loaded before any is stored, so the loads overlap
-    float2 stage[PREP_TILE + PREP_KMAX - 1];
+  float w[K][4];
+  float win[KW][4];
 #pragma unroll
-    for (int r = 0; r < PREP_TILE + PREP_KMAX - 1; ++r) {
-      const int tok = tr.t0 - Km1 + r;
-      float2 val = make_float2(0.f, 0.f);
-      if (r < nrows) {
-        if (tok >= tr.start) {
-          val = ld2(x + ((size_t)tok * H + h) * C3 + ch);
-        } else if (cs != nullptr) {
-          const int hr = Km1 + (tok - tr.start);  // history row, 0 = oldest
-          val = ld2(cs + (((size_t)row * Km1 + hr) * H + h) * C3 + ch);
+  for (int r = 0; r < KW; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) win[r][c] = 0.f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+#pragma unroll
+    for (int t = 0; t < K; ++t)
+      w[t][c] = active ? __ldg(a.conv_w + ((size_t)h * C3 + ch + c) * K + t) : 0.f;
+  if (active) {
+    // history: rows t0-K+1 .. t0-1 (from x inside the sequence, else the conv state)
+#pragma unroll
+    for (int r = 0; r < KM1; ++r) {
+      const int tok = tr.t0 - KM1 + r;
+      if (tok >= tr.start) {
+        unpack4(ld4(x + ((size_t)tok * H + h) * C3 + ch), win[r]);
+      } else if (cs != nullptr) {
+        unpack4(ld4(cs + (((size_t)row * KM1 + (KM1 + tok - tr.start)) * H + h) * C3 + ch),
+                win[r]);
+      }
+    }
+    if (a.mode == 1 && a.window != nullptr && tr.chunk == 0) {
+      T* wp = static_cast<T*>(a.window);
+      const size_t base = (size_t)tr.start + (size_t)tr.seq * KM1;
+#pragma unroll
+      for (int r = 0; r < KM1; ++r)
+        st4(wp + ((base + r) * H + h) * C3 + ch, make_float4(win[r][0], win[r][1], win[r][2], win[r][3]));
+    }
+  }
+  float* dst = part == 0 ? a.q : (part == 1 ? a.k : a.v);
+
+  for (int i0 = 0; i0 < tr.len; i0 += PREP_UNROLL) {
+    float xin[PREP_UNROLL][4];
+#pragma unroll
+    for (int u = 0; u < PREP_UNROLL; ++u) {
+      xin[u][0] = xin[u][1] = xin[u][2] = xin[u][3] = 0.f;
+      if (active && i0 + u < tr.len)
+        unpack4(ld4(x + ((size_t)(tr.t0 + i0 + u) * H + h) * C3 + ch), xin[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < PREP_UNROLL; ++u) {
+      const int i = i0 + u;
+      if (i >= tr.len) break;                  // uniform across the CTA
+      const int tok = tr.t0 + i;
+      float y[4];
+      float ss = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float acc = w[K - 1][c] * xin[u][c];
+#pragma unroll
+        for (int t = 0; t < KM1; ++t) acc = fmaf(w[t][c], win[t][c], acc);
+        y[c] = acc * sigmoid(acc);
+        ss = fmaf(y[c], y[c], ss);
+      }
+      if (KM1 > 0) {
+#pragma unroll
+        for (int t = 0; t + 1 < KM1; ++t)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) win[t][c] = win[t + 1][c];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) win[KW - 1][c] = xin[u][c];
+      }
+#pragma unroll
+      for (int off = G / 2; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      if (active) {
+        const float sc = (part < 2) ? 1.0f / fmaxf(sqrtf(ss), a.l2_eps) : 1.0f;
+        st4(dst + ((size_t)tok * H + h) * D + (ch - part * D),
+            make_float4(y[0] * sc, y[1] * sc, y[2] * sc, y[3] * sc));
+        if (a.mode == 1 && a.window != nullptr) {
+          T* wp = static_cast<T*>(a.window);
+          const size_t wr = (size_t)tr.start + (size_t)tr.seq * KM1 + KM1 + (tok - tr.start);
+          st4(wp + (wr * H + h) * C3 + ch, make_float4(xin[u][0], xin[u][1], xin[u][2], xin[u][3]));
         }
       }
-      stage[r] = val;
     }
+  }
+  // whole sequence in this tile: the register window holds its new conv history
+  if (KM1 > 0 && active && a.mode == 0 && a.commit_in_kernel && cs != nullptr &&
+      tr.chunk == 0 && tr.len == tr.end - tr.start) {
+    T* csw = static_cast<T*>(a.conv_state);
 #pragma unroll
-    for (int r = 0; r < PREP_TILE + PREP_KMAX - 1; ++r) {
-      if (r < nrows) {
-        xs[r][ch] = stage[r].x;
-        xs[r][ch + 1] = stage[r].y;
-      }
-    }
+    for (int r = 0; r < KM1; ++r)
+      st4(csw + (((size_t)row * KM1 + r) * H + h) * C3 + ch,
+          make_float4(win[r][0], win[r][1], win[r][2], win[r][3]));
   }
 
-  // conv + SiLU for the tile (each thread reads only its own columns of xs)
-  float v0[PREP_TILE], v1[PREP_TILE], ss[PREP_TILE];
+  // decay gate (4 channels per item) and beta, coalesced over the tile
+  if (active) {
+    const T* __restrict__ f = static_cast<const T*>(a.f);
+    const float Ah = expf(__ldg(a.A_log + h));
+    constexpr int IPR = D / 4;                 // items per token row
+    for (int e0 = j; e0 < tr.len * IPR; e0 += 4 * TPH) {
+      float4 fv[4];
 #pragma unroll
-  for (int i = 0; i < PREP_TILE; ++i) {
-    v0[i] = 0.f; v1[i] = 0.f;
-    if (own && i < tr.len) {
-      float acc0 = 0.f, acc1 = 0.f;
-      for (int j = 0; j < K; ++j) {
-        acc0 = fmaf(wsm[j][ch], xs[i + j][ch], acc0);
-        acc1 = fmaf(wsm[j][ch + 1], xs[i + j][ch + 1], acc1);
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * TPH;
+        if (e < tr.len * IPR)
+          fv[u] = ld4(f + ((size_t)(tr.t0 + e / IPR) * H + h) * D + (e % IPR) * 4);
       }
-      v0[i] = acc0 * sigmoid(acc0);
-      v1[i] = acc1 * sigmoid(acc1);
-    }
-    ss[i] = (part < 2) ? fmaf(v0[i], v0[i], v1[i] * v1[i]) : 0.f;
-  }
-
-  // L2 sums over the d channels of q and of k
 #pragma unroll
-  for (int i = 0; i < PREP_TILE; ++i) {
-#pragma unroll
-    for (int off = GW / 2; off >= 1; off >>= 1) ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], off);
-  }
-  if (WPP > 1) {
-    if ((tid & 31) == 0 && tid / 32 < NWARP) {
-#pragma unroll
-      for (int i = 0; i < PREP_TILE; ++i) part_ss[i][tid / 32] = ss[i];
-    }
-    __syncthreads();
-    if (own && part < 2) {
-#pragma unroll
-      for (int i = 0; i < PREP_TILE; ++i) {
-        float t = 0.f;
-#pragma unroll
-        for (int w = 0; w < WPP; ++w) t += part_ss[i][part * WPP + w];
-        ss[i] = t;
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * TPH;
+        if (e < tr.len * IPR) {
+          const int c = (e % IPR) * 4;
+          const float4 db = *reinterpret_cast<const float4*>(a.dt_bias + (size_t)h * D + c);
+          st4(a.loga + ((size_t)(tr.t0 + e / IPR) * H + h) * D + c,
+              make_float4(a.lb * sigmoid(Ah * (fv[u].x + db.x)), a.lb * sigmoid(Ah * (fv[u].y + db.y)),
+                          a.lb * sigmoid(Ah * (fv[u].z + db.z)), a.lb * sigmoid(Ah * (fv[u].w + db.w))));
+        }
       }
     }
-  }
-
-  if (own) {
-    float* dst = part == 0 ? a.q : (part == 1 ? a.k : a.v);
-    const int c = ch - part * D;
-#pragma unroll
-    for (int i = 0; i < PREP_TILE; ++i) {
-      if (i < tr.len) {
-        const float sc = (part < 2) ? 1.0f / fmaxf(sqrtf(ss[i]), a.l2_eps) : 1.0f;
-        st2(dst + ((size_t)(tr.t0 + i) * H + h) * D + c, v0[i] * sc, v1[i] * sc);
-      }
-    }
-    if (a.mode == 1 && a.window != nullptr) {  // TAPE: [history; x] per sequence
-      T* win = static_cast<T*>(a.window);
-      const size_t base = (size_t)tr.start + (size_t)tr.seq * Km1;
-      const int r0 = (tr.chunk == 0) ? 0 : Km1;
-      for (int r = r0; r < nrows; ++r) {
-        const size_t wr = base + (size_t)(tr.t0 - tr.start) + r;
-        st2(win + (wr * H + h) * C3 + ch, xs[r][ch], xs[r][ch + 1]);
-      }
-    }
-    if (a.mode == 0 && a.commit_in_kernel && cs != nullptr && tr.chunk == 0 &&
-        tr.len == tr.end - tr.start) {
-      // whole sequence in this tile: the new history is the last K-1 staged rows
-      T* csw = static_cast<T*>(a.conv_state);
-      for (int j = 0; j < Km1; ++j)
-        st2(csw + (((size_t)row * Km1 + j) * H + h) * C3 + ch, xs[tr.len + j][ch],
-            xs[tr.len + j][ch + 1]);
-    }
-  }
-
-  // decay gate and beta (loads first, then the arithmetic)
-  const T* __restrict__ f = static_cast<const T*>(a.f);
-  const float Ah = expf(__ldg(a.A_log + h));
-  constexpr int NTHR = ((3 * D / 2 + 31) / 32) * 32;      // the launch's block size
-  constexpr int NB = (PREP_TILE * D + NTHR - 1) / NTHR;  // elements per thread
-  const int nthr = NTHR;
-  float fv[NB];
-#pragma unroll
-  for (int m = 0; m < NB; ++m) {
-    const int e = tid + m * nthr;
-    fv[m] = 0.f;
-    if (e < tr.len * D) {
-      const int i = e / D, c = e - (e / D) * D;
-      fv[m] = ld1(f + ((size_t)(tr.t0 + i) * H + h) * D + c);
-    }
-  }
-#pragma unroll
-  for (int m = 0; m < NB; ++m) {
-    const int e = tid + m * nthr;
-    if (e < tr.len * D) {
-      const int i = e / D, c = e - (e / D) * D;
-      const size_t idx = ((size_t)(tr.t0 + i) * H + h) * D + c;
-      a.loga[idx] = a.lb * sigmoid(Ah * (fv[m] + __ldg(a.dt_bias + (size_t)h * D + c)));
-    }
-  }
-  if (tid < tr.len) {
-    const size_t idx = (size_t)(tr.t0 + tid) * H + h;
-    a.beta[idx] = sigmoid(ld1(static_cast<const T*>(a.beta_logit) + idx));
+    for (int i = j; i < tr.len; i += TPH)
+      a.beta[(size_t)(tr.t0 + i) * H + h] =
+          sigmoid(ld1(static_cast<const T*>(a.beta_logit) + (size_t)(tr.t0 + i) * H + h));
   }
 }
 
@@ -208,18 +200,33 @@ __global__ void conv_commit_kernel(const PrepArgs a) {
   }
 }
 
-template <typename T, int D>
-static cudaError_t launch_prep_t(const PrepArgs& a, cudaStream_t st) {
-  constexpr int threads = ((3 * D / 2 + 31) / 32) * 32;
-  dim3 grid(num_slots(a.total, a.n_seqs, PREP_TILE), a.H);
-  prep_kernel<T, D><<<grid, threads, 0, st>>>(a);
+template <typename T, int D, int K>
+static cudaError_t launch_prep_k(const PrepArgs& a, cudaStream_t st) {
+  constexpr int HPB = PREP_THREADS / (3 * D / 4);
+  dim3 grid(num_slots(a.total, a.n_seqs, PREP_TILE), (a.H + HPB - 1) / HPB);
+  prep_kernel<T, D, K><<<grid, PREP_THREADS, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (a.mode == 0 && a.conv_state != nullptr && a.K > 1 && !a.commit_in_kernel) {
+  if (a.mode == 0 && a.conv_state != nullptr && K > 1 && !a.commit_in_kernel) {
     conv_commit_kernel<T><<<dim3(a.n_seqs, a.H), 128, 0, st>>>(a);
     e = cudaGetLastError();
   }
   return e;
+}
+
+template <typename T, int D>
+static cudaError_t launch_prep_t(const PrepArgs& a, cudaStream_t st) {
+  switch (a.K) {
+    case 1: return launch_prep_k<T, D, 1>(a, st);
+    case 2: return launch_prep_k<T, D, 2>(a, st);
+    case 3: return launch_prep_k<T, D, 3>(a, st);
+    case 4: return launch_prep_k<T, D, 4>(a, st);
+    case 5: return launch_prep_k<T, D, 5>(a, st);
+    case 6: return launch_prep_k<T, D, 6>(a, st);
+    case 7: return launch_prep_k<T, D, 7>(a, st);
+    case 8: return launch_prep_k<T, D, 8>(a, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 template <typename T>
