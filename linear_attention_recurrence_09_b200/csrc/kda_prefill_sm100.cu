@@ -14,10 +14,13 @@
 //   E2     S <- Diag(e^{G_C}) S + D2 in fp32 registers (one key row per thread) -> bf16 S^T
 //   E3     O rows of D1 -> o (fp32, workspace) for the gated RMSNorm pass
 // Warp roles: warp 0 issues TMA (two smem stages, so chunk n+1 loads while n
-// computes), warp 1 allocates TMEM and issues the MMAs (one thread), warps 2-5
-// run the epilogues (TMEM lane quarter = warp % 4).  Every operand is K-major
-// with the 128-byte swizzle: TMA writes the workspace tiles in that layout and
-// the epilogue threads write S^T and U^T in it by hand.
+// computes; the U~ slice comes with them), warp 1 allocates TMEM and issues the
+// MMAs from one thread with precomputed descriptors, warps 2-9 run the
+// epilogues, two warps per TMEM lane quarter (quarter = warp % 4), each owning
+// 16 of the 32 value columns.  E1 and E2 are on the serial chain; E3 waits for
+// MMA3 after the state is handed back, off the chain.  Every MMA operand is
+// K-major with the 128-byte swizzle: TMA writes the workspace tiles in that
+// layout and the epilogue threads write S^T and U^T in it by hand.
 //
 // Every wait is bounded (about a second): on expiry the CTA records
 // KDA_ERR_TIMEOUT in the workspace status word, drains what it issued, frees
@@ -32,16 +35,19 @@ namespace kda {
 namespace {
 
 constexpr int D = 128, C = 64, J = 32, NSLICE = D / J;
-constexpr int THREADS = 192;
+constexpr int NEPI = 8;                          // epilogue warps (2 per TMEM lane quarter)
+constexpr int THREADS = 64 + 32 * NEPI;
+constexpr int JH = J / 2;                        // value columns per epilogue thread
 constexpr uint32_t TMEM_COLS = 128;
 
 // shared memory carve-up (offsets from a 1024-byte aligned base)
 constexpr uint32_t A1_BYTES = 2 * 128 * 128;     // [W;Q~]: 2 K-blocks x 128 rows x 128 B
 constexpr uint32_t A2_BYTES = 128 * 128;         // K'^T : 128 key rows x 64 tokens
 constexpr uint32_t A3_BYTES = 128 * 128;         // [0;M]: 128 rows x 64 (rows 0-63 zero)
-constexpr uint32_t STAGE_BYTES = A1_BYTES + A2_BYTES + A3_BYTES;
+constexpr uint32_t UT_BYTES = C * J * 2;         // U~ slice: 64 rows x 32 cols bf16, row-major
+constexpr uint32_t STAGE_BYTES = A1_BYTES + A2_BYTES + A3_BYTES + UT_BYTES;
 constexpr uint32_t NSTAGE = 2;
-constexpr uint32_t TX_BYTES = 4 * 8192 + 16384 + 8192;   // W x2, Q~ x2, K'^T, M
+constexpr uint32_t TX_BYTES = 4 * 8192 + 16384 + 8192 + UT_BYTES;   // W x2, Q~ x2, K'^T, M, U~
 constexpr uint32_t OFF_S = NSTAGE * STAGE_BYTES;          // S^T: 2 K-blocks x 32 rows x 128 B
 constexpr uint32_t OFF_U = OFF_S + 2 * J * 128;           // U^T: 32 rows x 128 B
 constexpr uint32_t OFF_BAR = OFF_U + J * 128;
@@ -52,8 +58,11 @@ enum { BAR_FULL0 = 0, BAR_FULL1, BAR_EMPTY0, BAR_EMPTY1, BAR_MMA1, BAR_MMA2, BAR
        BAR_UREADY, BAR_COUNT };
 
 struct TmaMaps {
-  CUtensorMap W, Q, KT, M;
+  CUtensorMap W, Q, KT, M, Ut;
 };
+
+// K-major SW128 descriptor advanced by `bytes` (the 14-bit address field never carries)
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
 __global__ void __launch_bounds__(THREADS, 1)
 interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps maps) {
@@ -82,8 +91,8 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
     mbar_init(bar(BAR_EMPTY1), 1);
     mbar_init(bar(BAR_MMA1), 1);
     mbar_init(bar(BAR_MMA2), 1);
-    mbar_init(bar(BAR_SREADY), 128);
-    mbar_init(bar(BAR_UREADY), 64);
+    mbar_init(bar(BAR_SREADY), 32 * NEPI);
+    mbar_init(bar(BAR_UREADY), 32 * NEPI / 2);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   // rows 0-63 of every A3 tile are the zero half of [0 ; M]
@@ -103,7 +112,7 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
-  const uint32_t d1_tmem[2] = {tmem + 0, tmem + 32};
+  const uint32_t d1_tmem[2] = {tmem + 0, tmem + 32};   // double-buffered [W S ; O]
   const uint32_t d2_tmem = tmem + 64;
   int* status = reinterpret_cast<int*>(a.ws + a.L.status);
 
@@ -116,6 +125,7 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
         if (n >= 2 && !mbar_wait(bar(BAR_EMPTY0 + st), ((n >> 1) - 1) & 1, &abort_flag)) break;
         const int tile = (start / C + s + n) * H + h;
         const uint32_t A1 = sbase + st * STAGE_BYTES, A2 = A1 + A1_BYTES, A3 = A2 + A2_BYTES;
+        const uint32_t UTs = A3 + A3_BYTES;
         mbar_expect_tx(bar(BAR_FULL0 + st), TX_BYTES);
         tma_load_2d(A1, &maps.W, 0, tile * C, bar(BAR_FULL0 + st));
         tma_load_2d(A1 + 16384, &maps.W, 64, tile * C, bar(BAR_FULL0 + st));
@@ -123,6 +133,7 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
         tma_load_2d(A1 + 16384 + 8192, &maps.Q, 64, tile * C, bar(BAR_FULL0 + st));
         tma_load_2d(A2, &maps.KT, 0, tile * D, bar(BAR_FULL0 + st));
         tma_load_2d(A3 + 8192, &maps.M, 0, tile * C, bar(BAR_FULL0 + st));
+        tma_load_2d(UTs, &maps.Ut, j0, tile * C, bar(BAR_FULL0 + st));
         issued = n + 1;
       }
       if (abort_flag) {  // let the copies this thread started land before the CTA exits
@@ -138,29 +149,32 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t id = idesc_bf16(128, J);
+      const uint64_t dA1s0 = sw128_desc(sbase), dA1s1 = sw128_desc(sbase + STAGE_BYTES);
+      const uint64_t dS = sw128_desc(sbase + OFF_S), dU = sw128_desc(sbase + OFF_U);
       int last = -1;
       for (int n = 0; n < nch; ++n) {
         const int st = n & 1;
         if (!mbar_wait(bar(BAR_FULL0 + st), (n >> 1) & 1, &abort_flag)) break;
         if (!mbar_wait(bar(BAR_SREADY), n & 1, &abort_flag)) break;
         tc_fence_after();
-        const uint32_t A1 = sbase + st * STAGE_BYTES, A2 = A1 + A1_BYTES, A3 = A2 + A2_BYTES;
-        const uint32_t SB = sbase + OFF_S, UB = sbase + OFF_U;
+        const uint64_t a1 = st ? dA1s1 : dA1s0;
+        const uint64_t a2 = desc_add(a1, A1_BYTES), a3 = desc_add(a1, A1_BYTES + A2_BYTES);
+        const uint32_t d1 = st ? d1_tmem[1] : d1_tmem[0];
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          umma(d1_tmem[st], sw128_desc(A1 + (k >> 2) * 16384 + (k & 3) * 32),
-               sw128_desc(SB + (k >> 2) * 4096 + (k & 3) * 32), id, k > 0);
+          umma(d1, desc_add(a1, (k >> 2) * 16384 + (k & 3) * 32),
+               desc_add(dS, (k >> 2) * 4096 + (k & 3) * 32), id, k > 0);
         umma_commit(bar(BAR_MMA1));
         last = n;
         if (!mbar_wait(bar(BAR_UREADY), n & 1, &abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          umma(d2_tmem, sw128_desc(A2 + k * 32), sw128_desc(UB + k * 32), id, k > 0);
+          umma(d2_tmem, desc_add(a2, k * 32), desc_add(dU, k * 32), id, k > 0);
+        umma_commit(bar(BAR_MMA2));
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          umma(d1_tmem[st], sw128_desc(A3 + k * 32), sw128_desc(UB + k * 32), id, 1);
-        umma_commit(bar(BAR_MMA2));
+          umma(d1, desc_add(a3, k * 32), desc_add(dU, k * 32), id, 1);
         umma_commit(bar(BAR_EMPTY0 + st));
       }
       if (abort_flag && last >= 0) {  // let the issued MMAs retire before TMEM is freed
@@ -170,33 +184,35 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
       }
     }
   } else {
-    // ---------------- epilogue warps 2-5 ----------------
+    // ---------------- epilogue warps 2..9 ----------------
     const int q = warp & 3;                 // TMEM lane quarter
+    const int half = (warp - 2) / 4;        // which 16 of the slice's 32 value columns
     const int i = 32 * q + lane;            // key row of the state slice / TMEM lane
+    const int cb = JH * half;               // first column of this thread
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     unsigned char* SB = sm + OFF_S;
     unsigned char* UB = sm + OFF_U;
     const float* gCg = reinterpret_cast<const float*>(a.ws + a.L.gC);
-    const __nv_bfloat16* Ug = reinterpret_cast<const __nv_bfloat16*>(a.ws + a.L.Ut);
     float* og = reinterpret_cast<float*>(a.ws + a.L.o);
-    const size_t sg = (((size_t)row * H + h) * D + i) * D + j0;
+    const size_t sg = (((size_t)row * H + h) * D + i) * D + j0 + cb;
 
-    float S[32];
+    float S[JH];
     if (a.state_in) {
 #pragma unroll
-      for (int c = 0; c < 32; c += 4) {
+      for (int c = 0; c < JH; c += 4) {
         const float4 v = *reinterpret_cast<const float4*>(a.state_in + sg + c);
         S[c] = v.x; S[c + 1] = v.y; S[c + 2] = v.z; S[c + 3] = v.w;
       }
     } else {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) S[c] = 0.f;
+      for (int c = 0; c < JH; ++c) S[c] = 0.f;
     }
+    unsigned char* sblk = SB + (i >> 6) * 4096;
     auto write_state = [&]() {
-      unsigned char* blk = SB + (i >> 6) * 4096;
 #pragma unroll
-      for (int n = 0; n < 32; ++n)
-        *reinterpret_cast<__nv_bfloat16*>(blk + sw128_off(n, i & 63)) = __float2bfloat16_rn(S[n]);
+      for (int n = 0; n < JH; ++n)
+        *reinterpret_cast<__nv_bfloat16*>(sblk + sw128_off(cb + n, i & 63)) =
+            __float2bfloat16_rn(S[n]);
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(bar(BAR_SREADY));
@@ -210,58 +226,61 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
       const int L = min(C, end - t0);
       const float gc = __ldg(gCg + (size_t)tile * D + i);
       if (q < 2) {
-        // E1: U = U~ - W S for token row r = i (0..63)
-        float ut[32];
-        const __nv_bfloat16* up = Ug + ((size_t)tile * C + i) * D + j0;
-#pragma unroll
-        for (int c = 0; c < 32; c += 8) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(up + c);
-          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const float2 f = __bfloat1622float2(p2[m]);
-            ut[c + 2 * m] = f.x; ut[c + 2 * m + 1] = f.y;
-          }
-        }
+        // E1: U = U~ - W S for token row r = i (0..63), columns cb..cb+15
         if (!mbar_wait_warp(bar(BAR_MMA1), n & 1, &abort_flag)) break;
         tc_fence_after();
-        float ws[32];
-        tmem_ld32(d1_tmem[st] + lane_off, ws);
+        float ws[JH];
+        tmem_ld16(d1_tmem[st] + lane_off + cb, ws);
+        const __nv_bfloat16* ut =
+            reinterpret_cast<const __nv_bfloat16*>(sm + st * STAGE_BYTES + A1_BYTES + A2_BYTES +
+                                                   A3_BYTES) + i * J + cb;
 #pragma unroll
-        for (int m = 0; m < 32; ++m) {
-          const float u = (i < L) ? ut[m] - ws[m] : 0.f;
-          *reinterpret_cast<__nv_bfloat16*>(UB + sw128_off(m, i)) = __float2bfloat16_rn(u);
+        for (int m = 0; m < JH; m += 8) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(ut + m);
+          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(p2[e]);
+            const float u0 = (i < L) ? f.x - ws[m + 2 * e] : 0.f;
+            const float u1 = (i < L) ? f.y - ws[m + 2 * e + 1] : 0.f;
+            *reinterpret_cast<__nv_bfloat16*>(UB + sw128_off(cb + m + 2 * e, i)) =
+                __float2bfloat16_rn(u0);
+            *reinterpret_cast<__nv_bfloat16*>(UB + sw128_off(cb + m + 2 * e + 1, i)) =
+                __float2bfloat16_rn(u1);
+          }
         }
         fence_proxy_async();
         tc_fence_before();
         mbar_arrive(bar(BAR_UREADY));
       }
-      // E2: state update for key row i
+      // E2: state update for key row i (on the serial chain)
       if (!mbar_wait_warp(bar(BAR_MMA2), n & 1, &abort_flag)) break;
       tc_fence_after();
       {
-        float dv[32];
-        tmem_ld32(d2_tmem + lane_off, dv);
+        float dv[JH];
+        tmem_ld16(d2_tmem + lane_off + cb, dv);
 #pragma unroll
-        for (int m = 0; m < 32; ++m) S[m] = fmaf(gc, S[m], dv[m]);
+        for (int m = 0; m < JH; ++m) S[m] = fmaf(gc, S[m], dv[m]);
       }
+      write_state();
       if (q >= 2) {
-        // E3: O rows (TMEM lanes 64-127) -> o
-        float o[32];
-        tmem_ld32(d1_tmem[st] + lane_off, o);
+        // E3 (off the chain): O rows (TMEM lanes 64-127) once MMA3 has retired
+        if (!mbar_wait_warp(bar(BAR_EMPTY0 + st), (n >> 1) & 1, &abort_flag)) break;
+        tc_fence_after();
+        float o[JH];
+        tmem_ld16(d1_tmem[st] + lane_off + cb, o);
         const int r = i - 64;
         if (r < L) {
-          float* op = og + ((size_t)(t0 + r) * H + h) * D + j0;
+          float* op = og + ((size_t)(t0 + r) * H + h) * D + j0 + cb;
 #pragma unroll
-          for (int c = 0; c < 32; c += 4)
+          for (int c = 0; c < JH; c += 4)
             *reinterpret_cast<float4*>(op + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
         }
       }
-      write_state();
     }
     if (!abort_flag && a.state_out) {
 #pragma unroll
-      for (int c = 0; c < 32; c += 4)
+      for (int c = 0; c < JH; c += 4)
         *reinterpret_cast<float4*>(a.state_out + sg + c) =
             make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
     }
@@ -318,15 +337,15 @@ EncodeTiledFn encode_fn() {
 
 // 2D bf16 tensor [rows, cols] (cols contiguous), box [box_rows, 64 cols], 128B swizzle
 bool make_map(EncodeTiledFn enc, CUtensorMap* m, void* base, uint64_t rows, uint64_t cols,
-              uint32_t box_rows) {
+              uint32_t box_rows, uint32_t box_cols = 64,
+              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -350,7 +369,8 @@ cudaError_t launch_interchunk_sm100(const PrefillArgs& a, cudaStream_t st) {
   if (!make_map(enc, &maps.W, a.ws + a.L.W, tiles * C, D, 64) ||
       !make_map(enc, &maps.Q, a.ws + a.L.Qt, tiles * C, D, 64) ||
       !make_map(enc, &maps.KT, a.ws + a.L.Kp, tiles * D, C, 128) ||
-      !make_map(enc, &maps.M, a.ws + a.L.M, tiles * C, C, 64))
+      !make_map(enc, &maps.M, a.ws + a.L.M, tiles * C, C, 64) ||
+      !make_map(enc, &maps.Ut, a.ws + a.L.Ut, tiles * C, D, 64, J, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(interchunk_sm100_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
