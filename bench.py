@@ -145,40 +145,50 @@ def prefill_workload(torch, kda, synth, T, seed, dev):
     A_cpu = synth.layer_activations(seed, [T], H, d, torch.bfloat16)
     A = {k: v.to(dev) for k, v in A_cpu.items()}
     N = 1
-    out = {'q': torch.empty(T, H, d, device=dev), 'k': torch.empty(T, H, d, device=dev),
-           'v': torch.empty(T, H, d, device=dev),
-           'log_a': torch.empty(T, H, d, device=dev), 'beta': torch.empty(T, H, device=dev)}
     y = torch.empty(T, H, d, dtype=cfg.dtype, device=dev)
     state = torch.empty(N, H, d, d, device=dev)
-    ws = kda.prefill_workspace(cfg, N, T, dev)
-    return dict(cfg=cfg, P=P, A=A, A_cpu=A_cpu, out=out, y=y, state=state, ws=ws, T=T, H=H, d=d)
+    ws = torch.empty(kda.kda_layer_prefill_workspace_size(cfg, N, T), dtype=torch.uint8,
+                     device=dev)
+    return dict(cfg=cfg, P=P, A=A, A_cpu=A_cpu, y=y, state=state, ws=ws, T=T, H=H, d=d)
 
 
-def prefill_bytes(T, H, d):
-    """Algorithmic HBM bytes of prep and of prefill (bf16 activations, fp32 gates/state)."""
+PHASES = ('intra_chunk', 'inter_chunk', 'gated_norm')
+
+
+def prefill_bytes(T, H, d, C=64, K=4):
+    """Algorithmic HBM bytes per launch of each pass of kda_layer_prefill (bf16
+    activations, fp32 state, bf16 chunk tiles, fp32 o), and of the layer as a whole
+    (inputs x, f, beta logit, g read once, y and the final state written once)."""
     th = T * H
-    prep = th * (3 * d * 2 + d * 2 + 2) + th * (3 * d * 4 + d * 4 + 4)
-    prefill = th * (3 * d * 4 + d * 4 + 4 + d * 2) + th * d * 2 + H * d * d * 4
-    return prep, prefill
+    nch = -(-T // C)
+    tiles = th * (4 * d * 2 + C * 2) + nch * H * d * 4          # W, U~, Q~, K', M; e^{G_C}
+    intra = th * (3 * d * 2 + d * 2 + 2) + tiles + H * (3 * d * K + 1 + d) * 4
+    inter = tiles + th * d * 4 + H * d * d * 4                  # tiles in, o and state out
+    norm = th * d * 4 + th * d * 2 + d * 4 + th * d * 2         # o, g, norm_w in; y out
+    layer = th * (3 * d * 2 + d * 2 + 2 + d * 2 + d * 2) + H * d * d * 4
+    return {'intra_chunk': intra, 'inter_chunk': inter, 'gated_norm': norm, 'layer': layer}
 
 
 def run_prefill(args, dist, torch, kda, synth, dev):
     W = prefill_workload(torch, kda, synth, args.tokens, 1 + 1000 * dist.rank, dev)
-    cfg, P, A, out, y, state, ws = (W[k] for k in ('cfg', 'P', 'A', 'out', 'y', 'state', 'ws'))
+    cfg, P, A, y, state, ws = (W[k] for k in ('cfg', 'P', 'A', 'y', 'state', 'ws'))
     stream = torch.cuda.current_stream()
-    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def ev():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)            # torch creates the CUDA event on first record
+        return e
 
     def step(e=None):
+        # one pass of the layer: fused prep + intra-chunk, inter-chunk, gated norm
         if e:
             e[0].record(stream)
-        kda.kda_prep(cfg, A['cu_seqlens'], A['x'], A['f'], A['beta_logit'], P['conv_w'],
-                     P['A_log'], P['dt_bias'], out=out)
+            kda.kda_set_phase_events(e[1:])
+        kda.kda_layer_prefill(cfg, A['cu_seqlens'], A['x'], A['f'], A['beta_logit'], A['g'],
+                              P['conv_w'], P['A_log'], P['dt_bias'], P['norm_w'],
+                              state_out=state, y=y, workspace=ws, max_seqlen=W['T'])
         if e:
-            e[1].record(stream)
-        kda.kda_prefill(cfg, A['cu_seqlens'], out['q'], out['k'], out['v'], out['log_a'],
-                        out['beta'], A['g'], P['norm_w'], state_out=state, y=y, workspace=ws)
-        if e:
-            e[2].record(stream)
+            kda.kda_set_phase_events(())
 
     for _ in range(args.warmup):
         step()
@@ -186,7 +196,7 @@ def run_prefill(args, dist, torch, kda, synth, dev):
     dist.barrier()
     sampler = ClockSampler(torch.cuda.current_device()) if dist.rank == 0 else None
     torch.cuda.synchronize()
-    per = [[ev(), ev(), ev()] for _ in range(args.steps)]
+    per = [[ev() for _ in range(4)] for _ in range(args.steps)]
     t_start, t_end = ev(), ev()
     wall0 = time.perf_counter()
     t_start.record(stream)
@@ -201,8 +211,8 @@ def run_prefill(args, dist, torch, kda, synth, dev):
         step()
         torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
-    ms_prep = statistics.mean(p[0].elapsed_time(p[1]) for p in per)
-    ms_pref = statistics.mean(p[1].elapsed_time(p[2]) for p in per)
+    ms_phase = {ph: statistics.mean(p[i].elapsed_time(p[i + 1]) for p in per)
+                for i, ph in enumerate(PHASES)}
     ms_max = dist.max(ms)
     ms_step = ms_max / args.steps
     T, H, d = W['T'], W['H'], W['d']
@@ -236,29 +246,35 @@ def run_prefill(args, dist, torch, kda, synth, dev):
     d2h = hy.numel() * hy.element_size() + hs.numel() * hs.element_size()
 
     hbm, tc, peak_kind = measured_peaks()
-    b_prep, b_pref = prefill_bytes(T, H, d)
-    dominant = ('kda_prefill', b_pref, ms_pref) if ms_pref >= ms_prep else ('kda_prep', b_prep, ms_prep)
+    nb = prefill_bytes(T, H, d)
+    top = max(PHASES, key=lambda ph: ms_phase[ph])
+    dominant = (top, nb[top], ms_phase[top])
     achieved = dominant[1] / (dominant[2] / 1e3) / 1e9
     res = {
         'metric': METRIC, 'value': value, 'unit': 'tokens/s', 'n_gpus': dist.world,
         'steps': args.steps, 'warmup': args.warmup, 'ms_per_step': ms_step,
         'higher_is_better': True, 'scaling': 'weak', 'vs_baseline': None, 'dtype': 'bf16',
         'data': 'synthetic (seeded N(0,1) activations, random-init layer parameters)',
-        'config': {'workload': f'prefill B=1 H=32 T={T} d=128 chunk=64 (prep + chunked prefill)',
+        'config': {'workload': f'prefill B=1 H=32 T={T} d=128 chunk=64 conv=4 '
+                               '(kda_layer_prefill: prep fused into the intra-chunk pass)',
                    'global_batch': dist.world, 'seq_len': T, 'heads': H, 'head_dim': d,
                    'parallelism': f'replicas x{dist.world} (independent batches per GPU)',
                    'l2': 'inputs larger than L2 (x alone is %.0f MB)' % (A['x'].numel() * 2 / 1e6)},
         'e2e': {'value': dist.world * T / (e2e_ms / 1e3), 'unit': 'tokens/s',
                 'h2d_bytes_per_step': h2d, 'd2h_bytes_per_step': d2h,
                 'ms_per_step': e2e_ms},
-        'gpu_launches': 4 * args.steps,
+        'gpu_launches': len(PHASES) * args.steps,
         'roofline': {'bound': 'hbm', 'kernel': dominant[0], 'achieved': achieved, 'peak': hbm,
                      'unit': 'GB/s', 'frac': achieved / hbm, 'traffic': None,
                      'peak_kind': peak_kind, 'algorithmic_bytes_per_launch': dominant[1]},
-        'breakdown_ms': {'kda_prep': ms_prep, 'kda_prefill': ms_pref},
-        'step_roofline': {'algorithmic_bytes': b_prep + b_pref,
-                          'achieved_gbs': (b_prep + b_pref) / (ms_step / 1e3) / 1e9,
-                          'frac': (b_prep + b_pref) / (ms_step / 1e3) / 1e9 / hbm},
+        'breakdown_ms': ms_phase,
+        'phase_roofline': {ph: {'algorithmic_bytes': nb[ph],
+                                'achieved_gbs': nb[ph] / (ms_phase[ph] / 1e3) / 1e9,
+                                'frac': nb[ph] / (ms_phase[ph] / 1e3) / 1e9 / hbm}
+                           for ph in PHASES},
+        'step_roofline': {'algorithmic_bytes': nb['layer'],
+                          'achieved_gbs': nb['layer'] / (ms_step / 1e3) / 1e9,
+                          'frac': nb['layer'] / (ms_step / 1e3) / 1e9 / hbm},
         'clocks': clocks,
     }
     del W

@@ -175,6 +175,32 @@ KDA_API int kda_prefill(const kda_config* cfg, int32_t n_seqs, int32_t total_tok
                 kda_stream_t stream);
 
 /*
+ * kda_layer_prefill - the whole layer over packed sequences in one call: prep
+ * (conv + SiLU + L2 + gate + beta), chunked prefill and gated RMSNorm, from the
+ * raw inputs.  For bf16, d = 128, chunk 64, K = 4 the prep runs inside the
+ * tensor-core intra-chunk pass (q/k/v stay on chip in fp32); other
+ * configurations run kda_prep into the workspace, then the chunked prefill.
+ * Results equal kda_prep followed by kda_prefill up to rounding.
+ *
+ *  x, f, beta_logit, conv_w, A_log, dt_bias, max_seqlen   as in kda_prep
+ *  g, norm_w, state_in, state_out, y                      as in kda_prefill
+ *  conv_state  [pool_size, K-1, H, 3d] history (NULL = zeros), updated to the
+ *              last K-1 pre-conv rows of each sequence (COMMIT)
+ *  state_slots / pool_size index both the conv state and the recurrent state.
+ *  workspace   at least kda_layer_prefill_workspace_size() bytes, 256-aligned.
+ */
+KDA_API size_t kda_layer_prefill_workspace_size(const kda_config* cfg, int32_t n_seqs,
+                                                int32_t total_tokens);
+KDA_API int kda_layer_prefill(const kda_config* cfg, int32_t n_seqs, int32_t total_tokens,
+                              const int32_t* cu_seqlens, int32_t max_seqlen, const void* x,
+                              const void* f, const void* beta_logit, const void* g,
+                              const float* conv_w, const float* A_log, const float* dt_bias,
+                              const float* norm_w, void* conv_state, const float* state_in,
+                              float* state_out, const int32_t* state_slots, int32_t pool_size,
+                              void* y, void* workspace, size_t workspace_bytes,
+                              kda_stream_t stream);
+
+/*
  * kda_decode - one token for each of `batch` sequences (the "fused operator"
  * path of PR #27754: no chunking).  Streams each head's d x d fp32 state once:
  * decay, both column reductions S^T k and S^T q in one pass, rank-1 update,
@@ -279,6 +305,18 @@ KDA_API int kda_prefill_noalloc(const kda_config* cfg, int32_t n_seqs, int32_t t
  * usable.  No trap, no fault, no unbounded wait.
  */
 KDA_API int kda_selftest_wait_timeout(void* workspace, kda_stream_t stream);
+
+/*
+ * kda_set_phase_events - measurement hook (the paper has no counterpart).
+ * `events` holds n <= 3 cudaEvent_t handles (created by the caller, owned by
+ * the caller, may be NULL entries); while set, every kda_prefill,
+ * kda_prefill_noalloc and kda_layer_prefill issued from THIS host thread
+ * records events[0] after the intra-chunk pass, events[1] after the
+ * inter-chunk pass and events[2] after the output norm, on the call's stream.
+ * The kernels are unchanged.  n = 0 (events may be NULL) clears the hook.
+ * Returns KDA_ERR_INVALID_ARG for n outside [0, 3] or events NULL with n > 0.
+ */
+KDA_API int kda_set_phase_events(void* const* events, int32_t n);
 
 #ifdef __cplusplus
 }

@@ -154,6 +154,105 @@ int kda_prefill(const kda_config* cfg, int32_t n_seqs, int32_t total_tokens,
   return cuda_status(kda::launch_prefill(a, s));
 }
 
+// Bytes the fallback of kda_layer_prefill (separate prep, then the chunked
+// prefill) needs on top of the prefill workspace: fp32 q, k, v, log a and beta.
+static size_t layer_prep_bytes(const kda_config* c, int32_t total) {
+  const size_t th = (size_t)total * c->num_heads;
+  return ((th * c->head_dim * 4 * 4 + th * 4) + 255) & ~(size_t)255;
+}
+
+static bool layer_fused(const kda_config* c) {
+  return c->dtype == KDA_BF16 && c->head_dim == 128 && c->chunk_size == 64 && c->conv_size == 4;
+}
+
+size_t kda_layer_prefill_workspace_size(const kda_config* cfg, int32_t n_seqs,
+                                        int32_t total_tokens) {
+  const size_t base = kda_prefill_workspace_size(cfg, n_seqs, total_tokens);
+  if (base == 0) return 0;
+  return layer_fused(cfg) ? base : base + layer_prep_bytes(cfg, total_tokens);
+}
+
+int kda_layer_prefill(const kda_config* cfg, int32_t n_seqs, int32_t total_tokens,
+                      const int32_t* cu_seqlens, int32_t max_seqlen, const void* x,
+                      const void* f, const void* beta_logit, const void* g,
+                      const float* conv_w, const float* A_log, const float* dt_bias,
+                      const float* norm_w, void* conv_state, const float* state_in,
+                      float* state_out, const int32_t* state_slots, int32_t pool_size, void* y,
+                      void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+  int st = check_cfg(cfg);
+  if (st) return st;
+  if (n_seqs < 0 || total_tokens < 0 || max_seqlen < 0) return KDA_ERR_INVALID_ARG;
+  if (n_seqs == 0) return KDA_OK;
+  if ((st = check_ptrs({cu_seqlens, conv_w, A_log, dt_bias, norm_w},
+                       {conv_state, state_in, state_out, state_slots})))
+    return st;
+  const bool pooled = conv_state != nullptr || state_in != nullptr || state_out != nullptr;
+  if (pooled && (st = check_pool(state_slots, pool_size, n_seqs))) return st;
+  if (total_tokens > 0 && (st = check_ptrs({x, f, beta_logit, g, y}, {}))) return st;
+  const size_t need = kda_layer_prefill_workspace_size(cfg, n_seqs, total_tokens);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < need)
+    return KDA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const kda::PrefillLayout L =
+      kda::prefill_layout(n_seqs, total_tokens, cfg->num_heads, cfg->head_dim,
+                          cfg->chunk_size, cfg->dtype == KDA_BF16);
+  const int32_t* slots = pooled ? state_slots : nullptr;
+  const int32_t pool = pooled ? pool_size : n_seqs;
+
+  // prep arguments: the commit of the conv state (fused path) or the whole prep (fallback)
+  kda::PrepArgs p{};
+  p.cu = cu_seqlens; p.n_seqs = n_seqs; p.total = total_tokens;
+  p.H = cfg->num_heads; p.D = cfg->head_dim; p.K = cfg->conv_size;
+  p.bf16 = cfg->dtype == KDA_BF16;
+  p.x = x; p.f = f; p.beta_logit = beta_logit;
+  p.conv_w = conv_w; p.A_log = A_log; p.dt_bias = dt_bias;
+  p.conv_state = conv_state; p.slots = conv_state ? slots : nullptr;
+  p.pool_size = conv_state ? pool : n_seqs;
+  p.mode = KDA_CONV_COMMIT;
+  p.lb = cfg->gate_lower_bound; p.l2_eps = cfg->l2_eps;
+
+  kda::PrefillArgs a{};
+  a.cu = cu_seqlens; a.n_seqs = n_seqs; a.total = total_tokens;
+  a.H = cfg->num_heads; a.D = cfg->head_dim; a.C = cfg->chunk_size;
+  a.bf16 = cfg->dtype == KDA_BF16;
+  a.g = g; a.norm_w = norm_w;
+  a.state_in = state_in; a.state_out = state_out;
+  a.slots = slots; a.pool_size = pool;
+  a.y = y; a.ws = static_cast<char*>(workspace); a.L = L;
+  a.norm_eps = cfg->norm_eps; a.q_scale = cfg->q_scale; a.lb = cfg->gate_lower_bound;
+  a.l2_eps = cfg->l2_eps; a.K = cfg->conv_size;
+  if (cudaMemsetAsync(a.ws + L.status, 0, 256, s) != cudaSuccess) return KDA_ERR_CUDA;
+
+  if (layer_fused(cfg)) {
+    // prep runs inside the intra-chunk pass; the conv state is committed afterwards
+    a.x = x; a.f = f; a.beta_logit = beta_logit;
+    a.conv_w = conv_w; a.A_log = A_log; a.dt_bias = dt_bias; a.conv_state = conv_state;
+    if ((st = cuda_status(kda::launch_prefill(a, s)))) return st;
+    p.commit_in_kernel = 0;
+    return cuda_status(kda::launch_conv_commit(p, s));
+  }
+  // fallback: prep into the tail of the workspace, then the chunked prefill
+  const size_t th = (size_t)total_tokens * cfg->num_heads;
+  float* q = reinterpret_cast<float*>(a.ws + L.total);
+  float* k = q + th * cfg->head_dim;
+  float* v = k + th * cfg->head_dim;
+  float* la = v + th * cfg->head_dim;
+  float* be = la + th * cfg->head_dim;
+  p.q = q; p.k = k; p.v = v; p.loga = la; p.beta = be;
+  p.commit_in_kernel = (max_seqlen >= 1 && max_seqlen <= kda::prep_tile()) ? 1 : 0;
+  if ((st = cuda_status(kda::launch_prep(p, s)))) return st;
+  a.q = q; a.k = k; a.v = v; a.loga = la; a.beta = be;
+  return cuda_status(kda::launch_prefill(a, s));
+}
+
+int kda_set_phase_events(void* const* events, int32_t n) {
+  if (n < 0 || n > 3 || (n > 0 && events == nullptr)) return KDA_ERR_INVALID_ARG;
+  kda::PhaseEvents& pe = kda::phase_events();
+  for (int i = 0; i < 3; ++i) pe.ev[i] = (i < n) ? static_cast<cudaEvent_t>(events[i]) : nullptr;
+  return KDA_OK;
+}
+
 static int step_common(const kda_config* cfg, int32_t batch, int32_t T, const void* q,
                        const void* k, const void* v, const float* log_a, const float* beta,
                        const void* g, const float* norm_w, const float* state_in,

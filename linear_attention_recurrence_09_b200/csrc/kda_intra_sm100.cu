@@ -1,6 +1,13 @@
-// Intra-chunk pass of kda_prefill on the 5th-generation tensor cores (sm_100a).
-// Used for d = 128, chunk 64, bf16 activations; writes the same per-slot
-// workspace tiles as the SIMT intra_chunk_kernel (W, U~, Q~, K'^T, M, e^{G_C}).
+// Intra-chunk pass of the prefill on the 5th-generation tensor cores (sm_100a).
+// Used for d = 128, chunk 64, bf16 activations; writes the per-slot workspace
+// tiles W, U~, Q~ (token rows), K' (token rows), M and e^{G_C}.
+//
+// Two input modes share one kernel:
+//   * kda_prefill: the prep outputs q, k, v, log a, beta (fp32) are read;
+//   * kda_layer_prefill (FUSED): the raw pre-conv x, f and beta logit are read
+//     and the prep of llama.cpp PR #27754's KDA commit (one depthwise causal
+//     conv over q|k|v, SiLU, q/k L2 norm with max(||x||, eps), bounded-sigmoid
+//     decay, sigmoid beta) runs here in fp32, so q/k/v never round-trip HBM.
 //
 // One CTA per (chunk slot, head).  With G the cumulative log decay of the chunk:
 //   * Gram: A'[r,i] = sum_c k_r k_i e^{G_r - G_i} and M[r,i] = q_scale sum_c q_r k_i e^{G_r - G_i}.
@@ -18,7 +25,10 @@
 //     into a bf16 high part and the bf16 rounding of the remainder (hi + lo), and
 //     W accumulates hi.hi + hi.lo + lo.hi, U~ accumulates V.hi + V.lo: the
 //     rounding of T and K e^G was the largest term left in the error budget.
-// Q~ = q_scale Q e^G, K'^T = (K e^{G_C - G})^T and e^{G_C} are elementwise.
+// Q~ = q_scale Q e^G, K' = K e^{G_C - G} and e^{G_C} are elementwise.  Each warp
+// walks 8 consecutive token rows with lane l owning channels 4l..4l+3 of q, k
+// and v, so the per-token L2 norms are full-warp shuffles and the conv keeps its
+// window of K-1 previous rows in registers.
 #include "kda_common.cuh"
 #include "kda_launch.h"
 #include "kda_sm100.cuh"
@@ -28,8 +38,8 @@ namespace {
 
 constexpr int D = 128, C = 64;
 constexpr int THREADS = 256;
+constexpr int KC = 4;         // conv taps of the fused path
 constexpr uint32_t TMEM_COLS = 128;
-constexpr int KP_LD = 66;     // K'^T staging row stride (elements): odd word stride
 
 // shared memory carve-up (offsets from a 1024-byte aligned base)
 constexpr uint32_t OFF_GA = 0;          // gram A: tf32, 4 K-blocks x 128 rows x 128 B (64 KB)
@@ -38,10 +48,15 @@ constexpr uint32_t OFF_KT = 131072;     // K e^G, high bf16 part: MN-major [64 t
 constexpr uint32_t OFF_KL = 147456;     // K e^G, low bf16 part (the rounding remainder)
 constexpr uint32_t OFF_VT = 163840;     // V:     bf16 MN-major [64 t][128 c] (16 KB)
 constexpr uint32_t OFF_G = 180224;      // G fp32 [64][128] (32 KB); later A fp32 [64][65]
-constexpr uint32_t OFF_KP = 212992;     // K'^T staging bf16 [128][KP_LD]
 constexpr uint32_t OFF_T = OFF_GA;      // T high part, bf16 K-major [64 r][64 i] (8 KB), after the gram
 constexpr uint32_t OFF_TL = OFF_GA + 8192;  // T low part
-constexpr uint32_t SMEM_BYTES = OFF_KP + 128 * KP_LD * 2 + 1024;
+constexpr int AF_LD = 68;                   // row stride (floats) of the fp32 tiles of the solve
+constexpr uint32_t TILE32 = 64 * AF_LD * 4;
+constexpr uint32_t OFF_XS = OFF_GA + 16384;  // X = (I + A)^{-1}, fp32 [64][68], after the gram
+constexpr uint32_t OFF_ZS = OFF_XS + TILE32; // block products of the solve, fp32 [64][68]
+constexpr uint32_t SMEM_BYTES = OFF_G + 32768 + 1024;
+static_assert(OFF_ZS + TILE32 <= OFF_GB, "solve tiles must fit in the gram A area");
+static_assert(TILE32 <= 32768, "A must fit in the G area");
 
 __device__ __forceinline__ uint32_t gram_off(int n, int c) {   // tf32 K-major, K = 128
   return (uint32_t)((c >> 5) * 16384) + sw128_off32(n, c & 31);
@@ -58,13 +73,31 @@ __device__ __forceinline__ void st_tf32x4(unsigned char* p, float a, float b, fl
 __device__ __forceinline__ void st_bf16x4(unsigned char* p, float a, float b, float c, float d) {
   st4(reinterpret_cast<__nv_bfloat16*>(p), make_float4(a, b, c, d));
 }
+// sigmoid and SiLU on the special-function unit (approximate exp and reciprocal);
+// 1 / (1 + inf) = 0 keeps the saturated ends exact
+__device__ __forceinline__ float fsigmoid(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
+__device__ __forceinline__ float fsilu(float z) { return z * fsigmoid(z); }
+__device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void sts4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+// start pulling `bytes` (a multiple of 16, 16-byte aligned) at p into L2
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+template <bool FUSED>
 __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const PrefillArgs a) {
   extern __shared__ __align__(1024) unsigned char smraw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sb = smem_u32(sm);
   __shared__ float bs[C];
+  __shared__ float qsum[4][D];   // per-quarter totals of the log decay
   __shared__ uint32_t tmem_holder;
   __shared__ __align__(8) uint64_t bar_mma;
   __shared__ volatile int abort_flag;
@@ -72,35 +105,35 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   const int h = blockIdx.y, H = a.H, slot = blockIdx.x;
   const TileRange tr = slot_to_tile(a.cu, a.n_seqs, a.total, C, slot);
   if (tr.len == 0) return;
-  if (pool_row(a.slots, tr.seq, a.pool_size) < 0) return;
+  const int prow = pool_row(a.slots, tr.seq, a.pool_size);
+  if (prow < 0) return;
   const int L = tr.len, t0 = tr.t0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t tile = (size_t)slot * H + h;
   __nv_bfloat16* Wo = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.W) + tile * C * D;
   __nv_bfloat16* Uo = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.Ut) + tile * C * D;
   __nv_bfloat16* Qo = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.Qt) + tile * C * D;
-  __nv_bfloat16* KTo = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.Kp) + tile * D * C;
+  __nv_bfloat16* Ko = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.Kp) + tile * C * D;
   __nv_bfloat16* Mo = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.M) + tile * C * C;
   float* gCo = reinterpret_cast<float*>(a.ws + a.L.gC) + tile * D;
   int* status = reinterpret_cast<int*>(a.ws + a.L.status);
   float* G = reinterpret_cast<float*>(sm + OFF_G);
-  float* Af = G;                                  // [64][65], after the gram
-  __nv_bfloat16* KP = reinterpret_cast<__nv_bfloat16*>(sm + OFF_KP);
+  float* Af = G;                                  // [64][AF_LD], after the gram
+  float* Xs = reinterpret_cast<float*>(sm + OFF_XS);
+  float* Zs = reinterpret_cast<float*>(sm + OFF_ZS);
 
-  // ---- log decay -> G (rows past the sequence end add 0), beta ----
-  {
-    float4 lv[8];   // 8 float4 per thread, all in flight before the first store
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      const int e4 = tid + m * THREADS;         // float4 index in the [64][128] tile
-      const int r = e4 >> 5, c4 = (e4 & 31) * 4;
-      lv[m] = (r < L) ? ld4(a.loga + ((size_t)(t0 + r) * H + h) * D + c4)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
+  // this tile's rows start streaming into L2 while the gates are computed
+  if (tid < L) {
+    const size_t row = (size_t)(t0 + tid) * H + h;
+    if (FUSED) {
+      prefetch_l2(static_cast<const __nv_bfloat16*>(a.x) + row * 3 * D, 3 * D * 2);
+    } else {
+      prefetch_l2(a.q + row * D, D * 4);
+      prefetch_l2(a.k + row * D, D * 4);
+      prefetch_l2(a.v + row * D, D * 4);
     }
-#pragma unroll
-    for (int m = 0; m < 8; ++m) reinterpret_cast<float4*>(G)[tid + m * THREADS] = lv[m];
   }
-  if (tid < C) bs[tid] = (tid < L) ? __ldg(a.beta + (size_t)(t0 + tid) * H + h) : 0.f;
+
   if (tid == 0) {
     abort_flag = 0;
     mbar_init(smem_u32(&bar_mma), 1);
@@ -113,80 +146,219 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  __syncthreads();
-  if (tid < D) {
-    float acc = 0.f;
-    for (int r = 0; r < C; ++r) {
-      acc += G[r * D + tid];
-      G[r * D + tid] = acc;
+
+  // ---- log decay and its running sum G over the chunk: channels 2p, 2p+1, rows 16q.. ----
+  {
+    const int cp = 2 * (tid & 63), qr = tid >> 6;
+    float g0[16], g1[16];
+    if (FUSED) {
+      const __nv_bfloat16* f = static_cast<const __nv_bfloat16*>(a.f);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = 16 * qr + i;
+        float2 v = make_float2(0.f, 0.f);
+        if (r < L) v = ld2(f + ((size_t)(t0 + r) * H + h) * D + cp);
+        g0[i] = v.x;
+        g1[i] = v.y;
+      }
+      const float Ah = expf(__ldg(a.A_log + h));
+      const float2 db = *reinterpret_cast<const float2*>(a.dt_bias + (size_t)h * D + cp);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const bool live = 16 * qr + i < L;
+        g0[i] = live ? a.lb * fsigmoid(Ah * (g0[i] + db.x)) : 0.f;
+        g1[i] = live ? a.lb * fsigmoid(Ah * (g1[i] + db.y)) : 0.f;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = 16 * qr + i;
+        float2 v = make_float2(0.f, 0.f);
+        if (r < L) v = ld2(a.loga + ((size_t)(t0 + r) * H + h) * D + cp);
+        g0[i] = v.x;
+        g1[i] = v.y;
+      }
     }
-    gCo[tid] = __expf(acc);
+#pragma unroll
+    for (int i = 1; i < 16; ++i) {
+      g0[i] += g0[i - 1];
+      g1[i] += g1[i - 1];
+    }
+    qsum[qr][cp] = g0[15];
+    qsum[qr][cp + 1] = g1[15];
+    if (tid < C) {
+      float bv = 0.f;
+      if (tid < L) {
+        const size_t bi = (size_t)(t0 + tid) * H + h;
+        bv = FUSED ? fsigmoid(ld1(static_cast<const __nv_bfloat16*>(a.beta_logit) + bi))
+                   : __ldg(a.beta + bi);
+      }
+      bs[tid] = bv;
+    }
+    __syncthreads();
+    float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+    for (int q = 0; q < 3; ++q)
+      if (q < qr) {
+        o0 += qsum[q][cp];
+        o1 += qsum[q][cp + 1];
+      }
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      *reinterpret_cast<float2*>(G + (16 * qr + i) * D + cp) = make_float2(g0[i] + o0, g1[i] + o1);
+    if (qr == 3)
+      *reinterpret_cast<float2*>(gCo + cp) = make_float2(__expf(g0[15] + o0), __expf(g1[15] + o1));
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
 
-  // ---- elementwise operands: 4 consecutive channels of one token row per item ----
-  const float qsc = a.q_scale;
-  constexpr int BATCH = 4;   // items whose loads are in flight together
+  // ---- token rows 8w..8w+7: (prep), operands for the MMAs, Q~ and K' ----
+  {
+    const int c4 = 4 * lane;
+    const float qsc = a.q_scale, inv_eps = 1.0f / a.l2_eps;
+    const float4 g15 = lds4(G + 15 * D + c4), g47 = lds4(G + 47 * D + c4),
+                 g63 = lds4(G + 63 * D + c4);
+    const float r15[4] = {g15.x, g15.y, g15.z, g15.w}, r47[4] = {g47.x, g47.y, g47.z, g47.w},
+                r63[4] = {g63.x, g63.y, g63.z, g63.w};
+    const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x);
+    const __nv_bfloat16* cs = static_cast<const __nv_bfloat16*>(a.conv_state);
+    // fused prep state: conv taps (one float4 per channel) and the K-1 previous pre-conv rows
+    float4 cw[3][4];
+    float win[KC - 1][12];
+    if (FUSED) {
+#pragma unroll
+      for (int sgm = 0; sgm < 3; ++sgm)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          cw[sgm][j] = __ldg(reinterpret_cast<const float4*>(
+              a.conv_w + ((size_t)h * 3 * D + sgm * D + c4 + j) * KC));
+#pragma unroll
+      for (int m = 0; m < KC - 1; ++m) {
+        const int tok = t0 + 8 * warp - (KC - 1) + m;
+        float4 vq = make_float4(0.f, 0.f, 0.f, 0.f), vk = vq, vv = vq;
+        if (tok >= tr.start && tok < tr.end) {   // rows past the end only feed padded rows
+          const __nv_bfloat16* xp = x + ((size_t)tok * H + h) * 3 * D;
+          vq = ld4(xp + c4); vk = ld4(xp + D + c4); vv = ld4(xp + 2 * D + c4);
+        } else if (tok < tr.start && cs != nullptr) {
+          const __nv_bfloat16* hp =
+              cs + (((size_t)prow * (KC - 1) + (KC - 1 + tok - tr.start)) * H + h) * 3 * D;
+          vq = ld4(hp + c4); vk = ld4(hp + D + c4); vv = ld4(hp + 2 * D + c4);
+        }
+        win[m][0] = vq.x; win[m][1] = vq.y; win[m][2] = vq.z; win[m][3] = vq.w;
+        win[m][4] = vk.x; win[m][5] = vk.y; win[m][6] = vk.z; win[m][7] = vk.w;
+        win[m][8] = vv.x; win[m][9] = vv.y; win[m][10] = vv.z; win[m][11] = vv.w;
+      }
+    }
+    // row r's q, k, v channels c4..c4+3 (pre-conv x when fused); zero past the sequence end
+    auto load_row = [&](int r, float4& iq, float4& ik, float4& iv) {
+      iq = ik = iv = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < L) {
+        if (FUSED) {
+          const __nv_bfloat16* xp = x + ((size_t)(t0 + r) * H + h) * 3 * D;
+          iq = ld4(xp + c4); ik = ld4(xp + D + c4); iv = ld4(xp + 2 * D + c4);
+        } else {
+          const size_t idx = ((size_t)(t0 + r) * H + h) * D + c4;
+          iq = ld4(a.q + idx); ik = ld4(a.k + idx); iv = ld4(a.v + idx);
+        }
+      }
+    };
+    // two rows in flight ahead of the one being computed
+    float4 cq, ck, cv, n1q, n1k, n1v;
+    load_row(8 * warp, cq, ck, cv);
+    load_row(8 * warp + 1, n1q, n1k, n1v);
 #pragma unroll 1
-  for (int b0 = 0; b0 < (C * (D / 4)) / THREADS; b0 += BATCH) {
-  float4 qa[BATCH], ka[BATCH], va[BATCH];
+    for (int i = 0; i < 8; ++i) {
+      const int r = 8 * warp + i;
+      float4 n2q, n2k, n2v;
+      load_row(i + 2 < 8 ? r + 2 : C, n2q, n2k, n2v);
+      float qv[4], kv[4], vv[4];
+      if (FUSED) {
+        const float xq[4] = {cq.x, cq.y, cq.z, cq.w};
+        const float xk[4] = {ck.x, ck.y, ck.z, ck.w};
+        const float xv[4] = {cv.x, cv.y, cv.z, cv.w};
+        float sq = 0.f, sk = 0.f;
 #pragma unroll
-  for (int u = 0; u < BATCH; ++u) {
-    const int it = tid + (b0 + u) * THREADS;
-    const int r = it >> 5, c4 = (it & 31) * 4;
-    qa[u] = ka[u] = va[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r < L) {
-      const size_t idx = ((size_t)(t0 + r) * H + h) * D + c4;
-      qa[u] = ld4(a.q + idx);
-      ka[u] = ld4(a.k + idx);
-      va[u] = ld4(a.v + idx);
-    }
-  }
+        for (int j = 0; j < 4; ++j) {
+          // taps 0..K-2 on the window (oldest first), tap K-1 on the current row
+          const float4 wq = cw[0][j], wk = cw[1][j], wv = cw[2][j];
+          float aq = wq.w * xq[j], ak = wk.w * xk[j], av = wv.w * xv[j];
+          aq = fmaf(wq.x, win[0][j], aq); aq = fmaf(wq.y, win[1][j], aq); aq = fmaf(wq.z, win[2][j], aq);
+          ak = fmaf(wk.x, win[0][4 + j], ak); ak = fmaf(wk.y, win[1][4 + j], ak);
+          ak = fmaf(wk.z, win[2][4 + j], ak);
+          av = fmaf(wv.x, win[0][8 + j], av); av = fmaf(wv.y, win[1][8 + j], av);
+          av = fmaf(wv.z, win[2][8 + j], av);
+          qv[j] = fsilu(aq);
+          kv[j] = fsilu(ak);
+          vv[j] = fsilu(av);
+          sq = fmaf(qv[j], qv[j], sq);
+          sk = fmaf(kv[j], kv[j], sk);
+        }
 #pragma unroll
-  for (int u = 0; u < BATCH; ++u) {
-    const int it = tid + (b0 + u) * THREADS;
-    const int r = it >> 5, c4 = (it & 31) * 4;
-    const float4 q4 = qa[u], k4 = ka[u], v4 = va[u];
-    const float qv[4] = {q4.x, q4.y, q4.z, q4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w};
-    float kb[4], qb[4], kc0[4], kc1[4], qt[4], kt[4], kp[4];
-    const int rref = (r < 32) ? 15 : 47;
+        for (int e = 0; e < 12; ++e) {
+          win[0][e] = win[1][e];
+          win[1][e] = win[2][e];
+        }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = c4 + j;
-      const float g = G[r * D + c];
-      const float er = __expf(g - G[rref * D + c]);
-      kb[j] = kv[j] * er;
-      qb[j] = qsc * qv[j] * er;
-      kc0[j] = (r < 32) ? kv[j] * __expf(G[15 * D + c] - g) : 0.f;
-      kc1[j] = kv[j] * __expf(G[47 * D + c] - g);
-      const float eg = __expf(g);
-      qt[j] = qsc * qv[j] * eg;
-      kt[j] = kv[j] * eg;
-      kp[j] = kv[j] * __expf(G[63 * D + c] - g);
-    }
-    const int nk = (r < 32) ? r : 64 + (r - 32);
-    st_tf32x4(sm + OFF_GB + gram_off(nk, c4), kb[0], kb[1], kb[2], kb[3]);
-    st_tf32x4(sm + OFF_GB + gram_off(nk + 32, c4), qb[0], qb[1], qb[2], qb[3]);
-    if (r < 32) st_tf32x4(sm + OFF_GA + gram_off(r, c4), kc0[0], kc0[1], kc0[2], kc0[3]);
-    st_tf32x4(sm + OFF_GA + gram_off(32 + r, c4), kc1[0], kc1[1], kc1[2], kc1[3]);
-    {
-      float hi[4], lo[4];
+        for (int j = 0; j < 4; ++j) {
+          win[2][j] = xq[j]; win[2][4 + j] = xk[j]; win[2][8 + j] = xv[j];
+        }
+        sq = warp_sum(sq);
+        sk = warp_sum(sk);
+        const bool live = r < L;   // rows past the sequence end stay zero
+        // 1 / max(||x||, eps) = min(rsqrt(||x||^2), 1 / eps), rsqrt(0) = inf
+        const float iq = live ? fminf(rsqrtf(sq), inv_eps) : 0.f;
+        const float ik = live ? fminf(rsqrtf(sk), inv_eps) : 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          qv[j] *= iq;
+          kv[j] *= ik;
+          vv[j] = live ? vv[j] : 0.f;
+        }
+      } else {
+        qv[0] = cq.x; qv[1] = cq.y; qv[2] = cq.z; qv[3] = cq.w;
+        kv[0] = ck.x; kv[1] = ck.y; kv[2] = ck.z; kv[3] = ck.w;
+        vv[0] = cv.x; vv[1] = cv.y; vv[2] = cv.z; vv[3] = cv.w;
+      }
+      const float4 gr4 = lds4(G + r * D + c4);
+      const float gr[4] = {gr4.x, gr4.y, gr4.z, gr4.w};
+      const bool lowhalf = r < 32;
+      float kb[4], qb[4], kc0[4], kc1[4], qt[4], kt[4], kp[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        hi[j] = __bfloat162float(__float2bfloat16_rn(kt[j]));
-        lo[j] = kt[j] - hi[j];
+        const float g = gr[j];
+        const float er = __expf(g - (lowhalf ? r15[j] : r47[j]));
+        kb[j] = kv[j] * er;
+        qb[j] = qsc * qv[j] * er;
+        kc0[j] = lowhalf ? kv[j] * __expf(r15[j] - g) : 0.f;
+        kc1[j] = kv[j] * __expf(r47[j] - g);
+        const float eg = __expf(g);
+        qt[j] = qsc * qv[j] * eg;
+        kt[j] = kv[j] * eg;
+        kp[j] = kv[j] * __expf(r63[j] - g);
       }
-      st_bf16x4(sm + OFF_KT + mn_off(r, c4), hi[0], hi[1], hi[2], hi[3]);
-      st_bf16x4(sm + OFF_KL + mn_off(r, c4), lo[0], lo[1], lo[2], lo[3]);
-    }
-    st_bf16x4(sm + OFF_VT + mn_off(r, c4), v4.x, v4.y, v4.z, v4.w);
-    st4(Qo + (size_t)r * D + c4, make_float4(qt[0], qt[1], qt[2], qt[3]));
+      const int nk = lowhalf ? r : 64 + (r - 32);
+      st_tf32x4(sm + OFF_GB + gram_off(nk, c4), kb[0], kb[1], kb[2], kb[3]);
+      st_tf32x4(sm + OFF_GB + gram_off(nk + 32, c4), qb[0], qb[1], qb[2], qb[3]);
+      if (lowhalf) st_tf32x4(sm + OFF_GA + gram_off(r, c4), kc0[0], kc0[1], kc0[2], kc0[3]);
+      st_tf32x4(sm + OFF_GA + gram_off(32 + r, c4), kc1[0], kc1[1], kc1[2], kc1[3]);
+      {
+        float hi[4], lo[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) KP[(c4 + j) * KP_LD + r] = __float2bfloat16_rn(kp[j]);
-  }
+        for (int j = 0; j < 4; ++j) {
+          hi[j] = __bfloat162float(__float2bfloat16_rn(kt[j]));
+          lo[j] = kt[j] - hi[j];
+        }
+        st_bf16x4(sm + OFF_KT + mn_off(r, c4), hi[0], hi[1], hi[2], hi[3]);
+        st_bf16x4(sm + OFF_KL + mn_off(r, c4), lo[0], lo[1], lo[2], lo[3]);
+      }
+      st_bf16x4(sm + OFF_VT + mn_off(r, c4), vv[0], vv[1], vv[2], vv[3]);
+      st4(Qo + (size_t)r * D + c4, make_float4(qt[0], qt[1], qt[2], qt[3]));
+      st4(Ko + (size_t)r * D + c4, make_float4(kp[0], kp[1], kp[2], kp[3]));
+      cq = n1q; ck = n1k; cv = n1v;
+      n1q = n2q; n1k = n2k; n1v = n2v;
+    }
   }
   fence_proxy_async();
   __syncthreads();
@@ -205,13 +377,12 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   }
   bool ok = mbar_wait_warp(smem_u32(&bar_mma), 0, &abort_flag);
   tc_fence_after();
-  for (int e = tid; e < C * (C + 1); e += THREADS) Af[e] = 0.f;   // G is dead now
-  __syncthreads();
+  __syncthreads();   // G is dead now: A takes its place (only entries i < r are ever read)
   // D[m][n]: rows 0-31 = keys 0-31 vs cols 0-31 (keys) / 32-63 (queries) of rows 0-31;
   // rows 32-95 = keys 0-63 vs cols 64-95 (keys) / 96-127 (queries) of rows 32-63
   if (ok && (warp == 0 || warp == 5 || warp == 6)) {
     const int q = warp & 3;
-    const int i = (warp == 0) ? lane : (warp == 5 ? lane : 32 + lane);
+    const int i = (warp == 6) ? 32 + lane : lane;
     const int rbase = (warp == 0) ? 0 : 32;
     const uint32_t col = (warp == 0) ? 0u : 64u;
     float av[32], mv[32];
@@ -220,7 +391,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       const int r = rbase + j;
-      if (i < r) Af[r * (C + 1) + i] = bs[r] * av[j];
+      if (i < r) Af[r * AF_LD + i] = bs[r] * av[j];
       Mo[r * C + i] = __float2bfloat16_rn(i <= r ? mv[j] : 0.f);
     }
   } else if (warp == 7) {
@@ -230,32 +401,80 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   tc_fence_before();
   __syncthreads();
 
-  // ---- T = (I + A)^{-1} diag(b): column j, rows r = 4m + t owned by lane t ----
+  // ---- T = (I + A)^{-1} diag(b), with A strictly lower triangular, by 16 x 16 blocks ----
+  // X = (I + A)^{-1}: the four diagonal blocks by forward substitution (one thread per
+  // column), then the blocks below, one block diagonal at a time:
+  //   X_ab = -X_aa sum_{k=b}^{a-1} A_ak X_kb      (a > b)
+  if (tid < 64) {
+    const int b = tid >> 4, jj = tid & 15;
+    const float* Ab = Af + (16 * b) * AF_LD + 16 * b;
+    float xc[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      float acc = (r == jj) ? 1.f : 0.f;
+#pragma unroll
+      for (int i = 0; i < r; ++i) acc = fmaf(-Ab[r * AF_LD + i], xc[i], acc);
+      xc[r] = acc;
+    }
+#pragma unroll
+    for (int r = 0; r < 16; ++r) Xs[(16 * b + r) * AF_LD + 16 * b + jj] = xc[r];
+  }
+  __syncthreads();
   {
-    const int j = tid >> 2, t = tid & 3;
-    float x[16];
+    const int q = tid >> 6, rho = (tid >> 2) & 15, k4 = 4 * (tid & 3);
+#pragma unroll 1
+    for (int dg = 1; dg < 4; ++dg) {
+      const bool act = q < 4 - dg;
+      const int ab = q + dg, bb = q;   // block (ab, bb) of this block diagonal
+      if (act) {
+        float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+        for (int kb = bb; kb < ab; ++kb) {
+          const float* Ar = Af + (16 * ab + rho) * AF_LD + 16 * kb;
+          const float* Xk = Xs + (16 * kb) * AF_LD + 16 * bb + k4;
 #pragma unroll
-    for (int m = 0; m < 16; ++m) x[m] = 0.f;
+          for (int m = 0; m < 16; ++m) {
+            const float l = Ar[m];
+            const float4 xv = lds4(Xk + m * AF_LD);
+            z.x = fmaf(l, xv.x, z.x); z.y = fmaf(l, xv.y, z.y);
+            z.z = fmaf(l, xv.z, z.z); z.w = fmaf(l, xv.w, z.w);
+          }
+        }
+        sts4(Zs + (16 * ab + rho) * AF_LD + 16 * bb + k4, z);
+      }
+      __syncthreads();
+      if (act) {
+        float4 xo = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float* Xa = Xs + (16 * ab + rho) * AF_LD + 16 * ab;
+        const float* Zb = Zs + (16 * ab) * AF_LD + 16 * bb + k4;
 #pragma unroll
-    for (int r = 0; r < C; ++r) {
-      float p = 0.f;
-#pragma unroll
-      for (int m = 0; m < 16; ++m)
-        if (4 * m + t < r) p = fmaf(Af[r * (C + 1) + 4 * m + t], x[m], p);
-      p += __shfl_xor_sync(0xffffffffu, p, 1);
-      p += __shfl_xor_sync(0xffffffffu, p, 2);
-      if ((r & 3) == t) x[r >> 2] = ((r == j) ? 1.f : 0.f) - p;
+        for (int m = 0; m < 16; ++m) {
+          const float xa = Xa[m];
+          const float4 zv = lds4(Zb + m * AF_LD);
+          xo.x = fmaf(-xa, zv.x, xo.x); xo.y = fmaf(-xa, zv.y, xo.y);
+          xo.z = fmaf(-xa, zv.z, xo.z); xo.w = fmaf(-xa, zv.w, xo.w);
+        }
+        sts4(Xs + (16 * ab + rho) * AF_LD + 16 * bb + k4, xo);
+      }
+      __syncthreads();
     }
-    const float bj = bs[j];
+  }
+  // T[r][j] = X[r][j] b_j for j <= r (else 0), as bf16 high and low parts, K-major [r][j]
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const int r = 4 * m + t;
-      const float tv = x[m] * bj;
-      const __nv_bfloat16 hi = __float2bfloat16_rn(tv);
-      *reinterpret_cast<__nv_bfloat16*>(sm + OFF_T + sw128_off(r, j)) = hi;
-      *reinterpret_cast<__nv_bfloat16*>(sm + OFF_TL + sw128_off(r, j)) =
-          __float2bfloat16_rn(tv - __bfloat162float(hi));
+  for (int e = tid; e < C * 8; e += THREADS) {
+    const int r = e >> 3, j0 = 8 * (e & 7);
+    float hi[8], lo[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u;
+      const float tv = (j <= r) ? Xs[r * AF_LD + j] * bs[j] : 0.f;
+      hi[u] = __bfloat162float(__float2bfloat16_rn(tv));
+      lo[u] = tv - hi[u];
     }
+    st_bf16x4(sm + OFF_T + sw128_off(r, j0), hi[0], hi[1], hi[2], hi[3]);
+    st_bf16x4(sm + OFF_T + sw128_off(r, j0) + 8, hi[4], hi[5], hi[6], hi[7]);
+    st_bf16x4(sm + OFF_TL + sw128_off(r, j0), lo[0], lo[1], lo[2], lo[3]);
+    st_bf16x4(sm + OFF_TL + sw128_off(r, j0) + 8, lo[4], lo[5], lo[6], lo[7]);
   }
   fence_proxy_async();
   __syncthreads();
@@ -289,14 +508,6 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     umma_commit(smem_u32(&bar_mma));
     issued = 2;
   }
-  // K'^T out while the MMAs run (rows of 64 tokens, 16-byte stores)
-  for (int e = tid; e < D * (C / 8); e += THREADS) {
-    const int c = e >> 3, part = (e & 7) * 8;
-    const uint32_t* src = reinterpret_cast<const uint32_t*>(KP + c * KP_LD + part);
-    uint4 v;
-    v.x = src[0]; v.y = src[1]; v.z = src[2]; v.w = src[3];
-    *reinterpret_cast<uint4*>(KTo + (size_t)c * C + part) = v;
-  }
   if (ok) ok = mbar_wait_warp(smem_u32(&bar_mma), 1, &abort_flag);
   tc_fence_after();
   if (ok) {
@@ -305,12 +516,12 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     __nv_bfloat16* dst = (warp < 4) ? Wo : Uo;
     const uint32_t col = (warp < 4) ? 0u : 64u;
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
+    for (int hf = 0; hf < 2; ++hf) {
       float v[32];
-      tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + col + 32 * half, v);
+      tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + col + 32 * hf, v);
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        dst[(size_t)(32 * half + j) * D + c] = __float2bfloat16_rn(v[j]);
+        dst[(size_t)(32 * hf + j) * D + c] = __float2bfloat16_rn(v[j]);
     }
   }
 
@@ -335,16 +546,22 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   }
 }
 
+template <bool FUSED>
+cudaError_t launch_intra_t(const PrefillArgs& a, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(intra_chunk_sm100_kernel<FUSED>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  intra_chunk_sm100_kernel<FUSED><<<dim3(a.L.nslots, a.H), THREADS, SMEM_BYTES, st>>>(a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool sm100_intra_supported(const PrefillArgs& a) { return a.bf16 && a.D == D && a.C == C; }
+bool sm100_fused_supported(const PrefillArgs& a) { return sm100_intra_supported(a) && a.K == KC; }
 
 cudaError_t launch_intra_sm100(const PrefillArgs& a, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(intra_chunk_sm100_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  intra_chunk_sm100_kernel<<<dim3(a.L.nslots, a.H), THREADS, SMEM_BYTES, st>>>(a);
-  return cudaGetLastError();
+  return a.x ? launch_intra_t<true>(a, st) : launch_intra_t<false>(a, st);
 }
 
 }  // namespace kda

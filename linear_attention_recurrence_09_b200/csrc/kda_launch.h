@@ -88,15 +88,33 @@ struct PrefillArgs {
   void* y;
   char* ws;
   PrefillLayout L;
-  float norm_eps, q_scale, lb;
+  float norm_eps, q_scale, lb, l2_eps;
+  // raw inputs of the fused prep path (kda_layer_prefill); x == nullptr otherwise
+  const void* x;
+  const void* f;
+  const void* beta_logit;
+  const float* conv_w;
+  const float* A_log;
+  const float* dt_bias;
+  const void* conv_state;   // [pool, K-1, H, 3d] history, or nullptr for zeros
+  int K;
 };
 
 cudaError_t launch_prep(const PrepArgs& a, cudaStream_t st);
 cudaError_t launch_step(const StepArgs& a, cudaStream_t st);
 cudaError_t launch_rollback(const RollbackArgs& a, cudaStream_t st);
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st);
+
+// Caller-owned events recorded on the prefill's stream after the intra-chunk,
+// inter-chunk and output-norm passes (null entries are skipped); per host thread.
+struct PhaseEvents {
+  cudaEvent_t ev[3];
+};
+PhaseEvents& phase_events();
 bool sm100_interchunk_supported(const PrefillArgs& a);
 bool sm100_intra_supported(const PrefillArgs& a);
+bool sm100_fused_supported(const PrefillArgs& a);
+cudaError_t launch_conv_commit(const PrepArgs& a, cudaStream_t st);
 cudaError_t launch_intra_sm100(const PrefillArgs& a, cudaStream_t st);
 cudaError_t launch_interchunk_sm100(const PrefillArgs& a, cudaStream_t st);
 cudaError_t launch_wait_timeout_selftest(void* workspace, cudaStream_t st);

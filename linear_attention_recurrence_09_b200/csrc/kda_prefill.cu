@@ -336,6 +336,11 @@ __global__ void __launch_bounds__(256) gated_norm_kernel(const PrefillArgs a) {
 template <typename T, int D, int C>
 static cudaError_t launch_prefill_dc(const PrefillArgs& a, cudaStream_t st) {
   cudaError_t e;
+  const PhaseEvents& pe = phase_events();
+  // the tcgen05 passes exchange K' token-major, the SIMT passes K'^T: they pair only
+  // with each other, and raw (pre-conv) inputs are only read by the tcgen05 pass
+  if (sm100_intra_supported(a) != sm100_interchunk_supported(a)) return cudaErrorInvalidValue;
+  if (a.x != nullptr && !sm100_fused_supported(a)) return cudaErrorInvalidValue;
   if (sm100_intra_supported(a)) {
     e = launch_intra_sm100(a, st);
     if (e != cudaSuccess) return e;
@@ -347,6 +352,7 @@ static cudaError_t launch_prefill_dc(const PrefillArgs& a, cudaStream_t st) {
     k1<<<dim3(a.L.nslots, a.H), 256, sm, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  if (pe.ev[0] && (e = cudaEventRecord(pe.ev[0], st)) != cudaSuccess) return e;
   if (sm100_interchunk_supported(a)) {
     e = launch_interchunk_sm100(a, st);
     if (e != cudaSuccess) return e;
@@ -358,12 +364,19 @@ static cudaError_t launch_prefill_dc(const PrefillArgs& a, cudaStream_t st) {
     k2<<<dim3(D / P2_J, a.H, a.n_seqs), 256, sm, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  if (pe.ev[1] && (e = cudaEventRecord(pe.ev[1], st)) != cudaSuccess) return e;
   if (a.total > 0) {
     const size_t rows = (size_t)a.total * a.H;
     gated_norm_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  if (pe.ev[2] && (e = cudaEventRecord(pe.ev[2], st)) != cudaSuccess) return e;
   return cudaSuccess;
+}
+
+PhaseEvents& phase_events() {
+  static thread_local PhaseEvents pe{};
+  return pe;
 }
 
 template <typename T, int D>

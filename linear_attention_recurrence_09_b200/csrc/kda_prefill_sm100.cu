@@ -9,7 +9,8 @@
 // copy of the state slice (128 x 32):
 //   MMA1   D1[128 x 32]  = [W ; Q~] (128 x 128) . S          -> rows 0-63: W S, rows 64-127: Q~ S
 //   E1     U = U~ - W S  (fp32, rows past the sequence end forced to 0) -> bf16 U^T in smem
-//   MMA2   D2[128 x 32]  = K'^T (128 x 64) . U               (state increment, key rows)
+//   MMA2   D2[128 x 32]  = K'^T (128 x 64) . U               (state increment, key rows;
+//                                                               K' stored token-major, read MN-major)
 //   MMA3   D1[64:128]   += M (64 x 64) . U                   (O = Q~ S + M U; A = [0 ; M])
 //   E2     S <- Diag(e^{G_C}) S + D2 in fp32 registers (one key row per thread) -> bf16 S^T
 //   E3     O rows of D1 -> o (fp32, workspace) for the gated RMSNorm pass
@@ -42,12 +43,12 @@ constexpr uint32_t TMEM_COLS = 128;
 
 // shared memory carve-up (offsets from a 1024-byte aligned base)
 constexpr uint32_t A1_BYTES = 2 * 128 * 128;     // [W;Q~]: 2 K-blocks x 128 rows x 128 B
-constexpr uint32_t A2_BYTES = 128 * 128;         // K'^T : 128 key rows x 64 tokens
+constexpr uint32_t A2_BYTES = 128 * 128;         // K'   : 64 tokens x 128 key channels, read MN-major
 constexpr uint32_t A3_BYTES = 128 * 128;         // [0;M]: 128 rows x 64 (rows 0-63 zero)
 constexpr uint32_t UT_BYTES = C * J * 2;         // U~ slice: 64 rows x 32 cols bf16, row-major
 constexpr uint32_t STAGE_BYTES = A1_BYTES + A2_BYTES + A3_BYTES + UT_BYTES;
 constexpr uint32_t NSTAGE = 2;
-constexpr uint32_t TX_BYTES = 4 * 8192 + 16384 + 8192 + UT_BYTES;   // W x2, Q~ x2, K'^T, M, U~
+constexpr uint32_t TX_BYTES = 4 * 8192 + 2 * 8192 + 8192 + UT_BYTES;   // W x2, Q~ x2, K' x2, M, U~
 constexpr uint32_t OFF_S = NSTAGE * STAGE_BYTES;          // S^T: 2 K-blocks x 32 rows x 128 B
 constexpr uint32_t OFF_U = OFF_S + 2 * J * 128;           // U^T: 32 rows x 128 B
 constexpr uint32_t OFF_BAR = OFF_U + J * 128;
@@ -131,7 +132,8 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
         tma_load_2d(A1 + 16384, &maps.W, 64, tile * C, bar(BAR_FULL0 + st));
         tma_load_2d(A1 + 8192, &maps.Q, 0, tile * C, bar(BAR_FULL0 + st));
         tma_load_2d(A1 + 16384 + 8192, &maps.Q, 64, tile * C, bar(BAR_FULL0 + st));
-        tma_load_2d(A2, &maps.KT, 0, tile * D, bar(BAR_FULL0 + st));
+        tma_load_2d(A2, &maps.KT, 0, tile * C, bar(BAR_FULL0 + st));
+        tma_load_2d(A2 + 8192, &maps.KT, 64, tile * C, bar(BAR_FULL0 + st));
         tma_load_2d(A3 + 8192, &maps.M, 0, tile * C, bar(BAR_FULL0 + st));
         tma_load_2d(UTs, &maps.Ut, j0, tile * C, bar(BAR_FULL0 + st));
         issued = n + 1;
@@ -149,6 +151,7 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t id = idesc_bf16(128, J);
+      const uint32_t id_amn = idesc_bf16_amn(128, J);   // K' is read MN-major
       const uint64_t dA1s0 = sw128_desc(sbase), dA1s1 = sw128_desc(sbase + STAGE_BYTES);
       const uint64_t dS = sw128_desc(sbase + OFF_S), dU = sw128_desc(sbase + OFF_U);
       int last = -1;
@@ -158,7 +161,8 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
         if (!mbar_wait(bar(BAR_SREADY), n & 1, &abort_flag)) break;
         tc_fence_after();
         const uint64_t a1 = st ? dA1s1 : dA1s0;
-        const uint64_t a2 = desc_add(a1, A1_BYTES), a3 = desc_add(a1, A1_BYTES + A2_BYTES);
+        const uint32_t a2s = sbase + st * STAGE_BYTES + A1_BYTES;
+        const uint64_t a3 = desc_add(a1, A1_BYTES + A2_BYTES);
         const uint32_t d1 = st ? d1_tmem[1] : d1_tmem[0];
 #pragma unroll
         for (int k = 0; k < 8; ++k)
@@ -170,7 +174,7 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          umma(d2_tmem, desc_add(a2, k * 32), desc_add(dU, k * 32), id, k > 0);
+          umma(d2_tmem, sw128_mn_desc(a2s + k * 2048, 8192), desc_add(dU, k * 32), id_amn, k > 0);
         umma_commit(bar(BAR_MMA2));
 #pragma unroll
         for (int k = 0; k < 4; ++k)
@@ -368,7 +372,7 @@ cudaError_t launch_interchunk_sm100(const PrefillArgs& a, cudaStream_t st) {
   const uint64_t tiles = (uint64_t)a.L.nslots * a.H;
   if (!make_map(enc, &maps.W, a.ws + a.L.W, tiles * C, D, 64) ||
       !make_map(enc, &maps.Q, a.ws + a.L.Qt, tiles * C, D, 64) ||
-      !make_map(enc, &maps.KT, a.ws + a.L.Kp, tiles * D, C, 128) ||
+      !make_map(enc, &maps.KT, a.ws + a.L.Kp, tiles * C, D, 64) ||
       !make_map(enc, &maps.M, a.ws + a.L.M, tiles * C, C, 64) ||
       !make_map(enc, &maps.Ut, a.ws + a.L.Ut, tiles * C, D, 64, J, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;

@@ -240,6 +240,13 @@ static cudaError_t launch_prep_d(const PrepArgs& a, cudaStream_t st) {
   return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_conv_commit(const PrepArgs& a, cudaStream_t st) {
+  if (a.conv_state == nullptr || a.K < 2 || a.n_seqs == 0) return cudaSuccess;
+  if (a.bf16) conv_commit_kernel<__nv_bfloat16><<<dim3(a.n_seqs, a.H), 128, 0, st>>>(a);
+  else conv_commit_kernel<float><<<dim3(a.n_seqs, a.H), 128, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_prep(const PrepArgs& a, cudaStream_t st) {
   return a.bf16 ? launch_prep_d<__nv_bfloat16>(a, st) : launch_prep_d<float>(a, st);
 }

@@ -34,7 +34,8 @@ KDA_CONV_TAPE = 1
 ENTRY_POINTS = ('kda_status_string', 'kda_abi_version', 'kda_prep',
                 'kda_prefill_workspace_size', 'kda_prefill', 'kda_decode', 'kda_verify',
                 'kda_rollback', 'kda_workspace_status', 'kda_selftest_wait_timeout',
-                'kda_prefill_noalloc')
+                'kda_prefill_noalloc', 'kda_layer_prefill_workspace_size', 'kda_layer_prefill',
+                'kda_set_phase_events')
 
 
 class KdaError(RuntimeError):
@@ -111,6 +112,14 @@ def lib() -> ctypes.CDLL:
         L.kda_workspace_status.argtypes = [_P, _P]
         L.kda_selftest_wait_timeout.restype = ctypes.c_int
         L.kda_selftest_wait_timeout.argtypes = [_P, _P]
+        L.kda_layer_prefill_workspace_size.restype = ctypes.c_size_t
+        L.kda_layer_prefill_workspace_size.argtypes = [ctypes.POINTER(CConfig), _I, _I]
+        L.kda_layer_prefill.restype = ctypes.c_int
+        L.kda_layer_prefill.argtypes = [ctypes.POINTER(CConfig), _I, _I, _P, _I, _P, _P, _P, _P,
+                                        _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
+                                        ctypes.c_size_t, _P]
+        L.kda_set_phase_events.restype = ctypes.c_int
+        L.kda_set_phase_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), _I]
         L.kda_prefill_noalloc.restype = ctypes.c_int
         L.kda_prefill_noalloc.argtypes = [ctypes.POINTER(CConfig), _I, _I, _P, _P, _P, _P, _P,
                                           _P, _P, _P, _P, _P, _P, _I, _P, _P]
@@ -340,12 +349,67 @@ def kda_selftest_wait_timeout(workspace, stream=None):
            'kda_selftest_wait_timeout')
 
 
+def kda_set_phase_events(events=()):
+    """Record up to three ``torch.cuda.Event`` after the intra-chunk, inter-chunk and
+    output-norm passes of the following prefills on this thread; ``()`` clears.
+    Each event must already have been recorded once (torch creates it lazily)."""
+    events = list(events)
+    if len(events) > 3:
+        raise ValueError('at most three phase events')
+    handles = []
+    for e in events:
+        h = 0 if e is None else int(e.cuda_event)
+        if e is not None and h == 0:
+            raise ValueError('record the event once before passing it (created lazily)')
+        handles.append(h)
+    arr = (ctypes.c_void_p * max(1, len(handles)))(*handles)
+    _check(lib().kda_set_phase_events(arr if handles else None, len(handles)),
+           'kda_set_phase_events')
+
+
 # ---------------------------------------------------------------------------
 # compositions of the entry points
 # ---------------------------------------------------------------------------
-def layer_prefill(cfg: Config, params, acts, state_in=None, state_out=None, conv_state=None,
-                  workspace=None, prep_out=None, y=None, stream=None):
-    """prep + prefill over packed sequences; returns (y, prep outputs)."""
+def kda_layer_prefill_workspace_size(cfg: Config, n_seqs: int, total_tokens: int) -> int:
+    c = cfg.c()
+    return int(lib().kda_layer_prefill_workspace_size(ctypes.byref(c), int(n_seqs),
+                                                      int(total_tokens)))
+
+
+def kda_layer_prefill(cfg: Config, cu_seqlens, x, f, beta_logit, g, conv_w, A_log, dt_bias,
+                      norm_w, conv_state=None, state_in=None, state_out=None, state_slots=None,
+                      pool_size=None, y=None, workspace=None, max_seqlen=0, stream=None):
+    """The whole layer from raw inputs (prep fused where supported).  Returns y."""
+    H, d, K = cfg.num_heads, cfg.head_dim, cfg.conv_size
+    T = x.shape[0]
+    N = cu_seqlens.numel() - 1
+    if y is None:
+        y = _empty((T, H, d), cfg.dtype, x.device)
+    if workspace is None:
+        workspace = torch.empty(kda_layer_prefill_workspace_size(cfg, N, T), dtype=torch.uint8,
+                                device=x.device)
+    if pool_size is None:
+        ref = next((t for t in (state_in, state_out, conv_state) if t is not None), None)
+        pool_size = ref.shape[0] if ref is not None else N
+    c = cfg.c()
+    st = lib().kda_layer_prefill(
+        ctypes.byref(c), N, T, _ptr(cu_seqlens, torch.int32, 'cu_seqlens'), int(max_seqlen),
+        _ptr(x, cfg.dtype, 'x', (T, H, 3 * d)), _ptr(f, cfg.dtype, 'f', (T, H, d)),
+        _ptr(beta_logit, cfg.dtype, 'beta_logit', (T, H)), _ptr(g, cfg.dtype, 'g', (T, H, d)),
+        _ptr(conv_w, torch.float32, 'conv_w', (H, 3 * d, K)),
+        _ptr(A_log, torch.float32, 'A_log', (H,)), _ptr(dt_bias, torch.float32, 'dt_bias', (H, d)),
+        _ptr(norm_w, torch.float32, 'norm_w', (d,)), _ptr(conv_state, cfg.dtype, 'conv_state'),
+        _ptr(state_in, torch.float32, 'state_in'), _ptr(state_out, torch.float32, 'state_out'),
+        _ptr(state_slots, torch.int32, 'state_slots'), int(pool_size),
+        _ptr(y, cfg.dtype, 'y', (T, H, d)), _ptr(workspace, None, 'workspace'),
+        int(workspace.numel() * workspace.element_size()), _stream(stream))
+    _check(st, 'kda_layer_prefill')
+    return y
+
+
+def prep_then_prefill(cfg: Config, params, acts, state_in=None, state_out=None, conv_state=None,
+                      workspace=None, prep_out=None, y=None, stream=None):
+    """kda_prep + kda_prefill as two calls; returns (y, prep outputs)."""
     p = kda_prep(cfg, acts['cu_seqlens'], acts['x'], acts['f'], acts['beta_logit'],
                  params['conv_w'], params['A_log'], params['dt_bias'], conv_state=conv_state,
                  out=prep_out, stream=stream)
@@ -353,3 +417,12 @@ def layer_prefill(cfg: Config, params, acts, state_in=None, state_out=None, conv
                     acts['g'], params['norm_w'], state_in=state_in, state_out=state_out,
                     y=y, workspace=workspace, stream=stream)
     return y, p
+
+
+def layer_prefill(cfg: Config, params, acts, state_in=None, state_out=None, conv_state=None,
+                  workspace=None, y=None, stream=None):
+    """kda_layer_prefill on dicts of parameters and activations; returns y."""
+    return kda_layer_prefill(cfg, acts['cu_seqlens'], acts['x'], acts['f'], acts['beta_logit'],
+                             acts['g'], params['conv_w'], params['A_log'], params['dt_bias'],
+                             params['norm_w'], conv_state=conv_state, state_in=state_in,
+                             state_out=state_out, y=y, workspace=workspace, stream=stream)

@@ -38,8 +38,9 @@ def make_case(seed, seqlens, H, d, K=4, dtype=torch.bfloat16, state_var=0.0, con
     return cfg, params, acts, S0, hist
 
 
-def gpu_layer(cfg, params, acts, S0=None, hist=None, dev='cuda'):
-    """prep (COMMIT) + prefill on the GPU.  Returns y, final states, conv history, prep outputs."""
+def gpu_layer(cfg, params, acts, S0=None, hist=None, dev='cuda', fused=True):
+    """The layer on the GPU: kda_layer_prefill (fused=True) or kda_prep + kda_prefill.
+    Returns y, final states, conv history, prep outputs (None when fused)."""
     N = acts['cu_seqlens'].numel() - 1
     H, d, K = cfg.num_heads, cfg.head_dim, cfg.conv_size
     P = {k: v.to(dev) for k, v in params.items()}
@@ -48,7 +49,11 @@ def gpu_layer(cfg, params, acts, S0=None, hist=None, dev='cuda'):
     s_out = torch.empty(N, H, d, d, device=dev)
     cs = (hist.clone() if hist is not None else
           torch.zeros(N, K - 1, H, 3 * d, dtype=cfg.dtype)).to(dev)
-    y, p = kda.layer_prefill(cfg, P, Ad, state_in=s_in, state_out=s_out, conv_state=cs)
+    if fused:
+        y = kda.layer_prefill(cfg, P, Ad, state_in=s_in, state_out=s_out, conv_state=cs)
+        p = None
+    else:
+        y, p = kda.prep_then_prefill(cfg, P, Ad, state_in=s_in, state_out=s_out, conv_state=cs)
     torch.cuda.synchronize()
     return y, s_out, cs, p
 
@@ -64,9 +69,9 @@ def oracle_layer(cfg, params, acts, S0=None, hist=None, heads=None):
         q_scale=cfg.q_scale, heads=heads)
 
 
-def compare_layer(cfg, params, acts, S0=None, hist=None, heads=None):
+def compare_layer(cfg, params, acts, S0=None, hist=None, heads=None, fused=True):
     """Run both sides; return dict of relative errors (y, state, conv history)."""
-    y, s_out, cs, _ = gpu_layer(cfg, params, acts, S0, hist)
+    y, s_out, cs, _ = gpu_layer(cfg, params, acts, S0, hist, fused=fused)
     ref = oracle_layer(cfg, params, acts, S0, hist, heads)
     hs = slice(None) if heads is None else list(heads)
     errs = {

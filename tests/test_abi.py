@@ -103,6 +103,37 @@ def test_prefill_rejects_bad_workspace(L):
     assert call(A, need, cu=None) == kda.KDA_ERR_INVALID_ARG
 
 
+def test_layer_prefill_validates_and_sizes_workspace(L):
+    fused = _cfg(head_dim=128, chunk_size=64, dtype=torch.bfloat16, num_heads=4)
+    plain = _cfg(head_dim=64, chunk_size=64, dtype=torch.bfloat16, num_heads=4)
+    for cfg in (fused, plain):
+        c = ctypes.byref(cfg)
+        base = L.kda_prefill_workspace_size(c, 1, 100)
+        lay = L.kda_layer_prefill_workspace_size(c, 1, 100)
+        # the fallback adds fp32 q, k, v, log a (4 x T H d) and beta (T H) for the separate prep
+        extra = 0 if cfg is fused else 100 * 4 * (4 * 64 * 4 + 4)
+        assert lay >= base + extra and lay - base - extra < 256
+    cfg = fused
+    need = L.kda_layer_prefill_workspace_size(ctypes.byref(cfg), 1, 64)
+
+    def call(ws, nbytes, **kw):
+        a = dict(x=A, y=A, cu=A, cw=A)
+        a.update(kw)
+        return L.kda_layer_prefill(ctypes.byref(cfg), 1, 64, a['cu'], 64, a['x'], A, A, A,
+                                   a['cw'], A, A, A, None, None, None, None, 1, a['y'], ws,
+                                   nbytes, None)
+
+    assert call(None, need) == kda.KDA_ERR_WORKSPACE
+    assert call(A, need - 1) == kda.KDA_ERR_WORKSPACE
+    assert call(A + 16, need) == kda.KDA_ERR_WORKSPACE
+    assert call(A, need, x=MIS) == kda.KDA_ERR_MISALIGNED
+    assert call(A, need, y=None) == kda.KDA_ERR_INVALID_ARG
+    assert call(A, need, cw=None) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_layer_prefill(ctypes.byref(cfg), 0, 0, None, 0, None, None, None, None, None,
+                               None, None, None, None, None, None, None, 0, None, None, 0,
+                               None) == kda.KDA_OK      # nothing to do, nothing launched
+
+
 def test_step_entry_points_reject_bad_arguments(L):
     cfg = _cfg()
     c = ctypes.byref(cfg)

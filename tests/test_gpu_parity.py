@@ -33,7 +33,7 @@ def test_tiny_fp32_layer():
 def test_prep_matches_oracle(dtype, d, K):
     seqlens = [0, 1, 5, 17, 40]
     cfg, P, A, _, hist = make_case(3, seqlens, 3, d, K, dtype, conv_hist=True)
-    _, _, cs, p = gpu_layer(cfg, P, A, None, hist)
+    _, _, cs, p = gpu_layer(cfg, P, A, None, hist, fused=False)
     ref = oracle_layer(cfg, P, A, None, hist)
     tol = 1e-5
     for name, rname in [('q', 'q'), ('k', 'k'), ('v', 'v'), ('log_a', 'loga'), ('beta', 'beta')]:
@@ -60,11 +60,21 @@ def test_prep_tape_window(dtype):
         assert torch.equal(win[s, 3:], x[s])
 
 
+@pytest.mark.parametrize('fused', [True, False])
 @pytest.mark.parametrize('d,chunk', [(32, 16), (64, 32), (128, 64), (128, 16)])
-def test_prefill_varlen_ragged_bf16(d, chunk):
+def test_prefill_varlen_ragged_bf16(d, chunk, fused):
+    """kda_layer_prefill (fused prep at d=128, chunk 64) and kda_prep + kda_prefill."""
     seqlens = [0, 1, chunk - 1, chunk, chunk + 1, 3 * chunk + 7]
     cfg, P, A, S0, hist = make_case(5, seqlens, 4, d, 4, torch.bfloat16, state_var=0.01,
                                     conv_hist=True, chunk=chunk)
+    _assert(compare_layer(cfg, P, A, S0, hist, fused=fused), 1e-2)
+
+
+@pytest.mark.parametrize('K', [2, 4])
+def test_layer_prefill_conv_sizes(K):
+    """Fused (K = 4) and fallback (K = 2) layer prefill, conv history carried."""
+    cfg, P, A, S0, hist = make_case(16, [3, 130], 2, 128, K, torch.bfloat16, state_var=0.01,
+                                    conv_hist=True, chunk=64)
     _assert(compare_layer(cfg, P, A, S0, hist), 1e-2)
 
 
@@ -86,8 +96,10 @@ def test_beta_zero_no_decay_keeps_state_bit_exact():
     cfg, P, A, S0, _ = make_case(8, [70], 2, 64, 4, torch.bfloat16, state_var=0.01)
     A['beta_logit'][:] = -1e4
     A['f'][:] = -1e4
-    _, s_out, _, p = gpu_layer(cfg, P, A, S0, None)
+    _, s_out, _, p = gpu_layer(cfg, P, A, S0, None, fused=False)
     assert torch.equal(s_out.cpu(), S0)
+    _, s_f, _, _ = gpu_layer(cfg, P, A, S0, None, fused=True)
+    assert torch.equal(s_f.cpu(), S0)
     st = S0.cuda().clone()
     one = lambda t: t[:1].clone()
     kda.kda_decode(cfg, one(p['q']), one(p['k']), one(p['v']), one(p['log_a']), one(p['beta']),
@@ -274,7 +286,8 @@ def test_bounded_wait_times_out_and_context_survives():
     assert kda.kda_workspace_status(ws) == kda.KDA_ERR_TIMEOUT
     cfg, P, A, S0, hist = make_case(15, [20], 2, 64, 4, torch.bfloat16, state_var=0.01)
     _assert(compare_layer(cfg, P, A, S0, hist), 1e-2)
-    w2 = kda.prefill_workspace(cfg, 1, 20)
+    w2 = torch.empty(kda.kda_layer_prefill_workspace_size(cfg, 1, 20), dtype=torch.uint8,
+                     device='cuda')
     kda.layer_prefill(cfg, {k: v.cuda() for k, v in P.items()},
                       {k: v.cuda() for k, v in A.items()}, workspace=w2)
     assert kda.kda_workspace_status(w2) == kda.KDA_OK

@@ -37,7 +37,7 @@ def test_prefill_8k_full_size():
     P = synth.layer_params(1, H, D, K)
     A = synth.layer_activations(1, [8192], H, D, torch.bfloat16)
     state = torch.empty(1, H, D, D, device='cuda')
-    y, _ = kda.layer_prefill(cfg, _dev(P), _dev(A), state_out=state)
+    y = kda.layer_prefill(cfg, _dev(P), _dev(A), state_out=state)
     torch.cuda.synchronize()
     heads = [0, 17, 31]
     ref = oracle_layer(cfg, P, A, heads=heads)
@@ -135,7 +135,7 @@ def test_varlen_and_131k_full_size():
     A = synth.layer_activations(4, lens, H, D, torch.bfloat16)
     S0 = synth.initial_state(4, len(lens), H, D, 0.01)
     state = S0.cuda()
-    y, _ = kda.layer_prefill(cfg, Pd, _dev(A), state_in=state, state_out=state)
+    y = kda.layer_prefill(cfg, Pd, _dev(A), state_in=state, state_out=state)
     torch.cuda.synchronize()
     y = y.cpu()
     cu = A['cu_seqlens'].tolist()
@@ -151,7 +151,7 @@ def test_varlen_and_131k_full_size():
     L1 = synth.layer_activations(4, [T], H, D, torch.bfloat16, tag='long')
     S1 = synth.initial_state(5, 1, H, D, 0.01)
     st1 = S1.cuda()
-    y1, _ = kda.layer_prefill(cfg, Pd, _dev(L1), state_in=st1, state_out=st1)
+    y1 = kda.layer_prefill(cfg, Pd, _dev(L1), state_in=st1, state_out=st1)
     torch.cuda.synchronize()
     h = 7
     ref = oracle_layer(cfg, P, L1, S0=S1, heads=[h])
