@@ -29,6 +29,8 @@
 // walks 8 consecutive token rows with lane l owning channels 4l..4l+3 of q, k
 // and v, so the per-token L2 norms are full-warp shuffles and the conv keeps its
 // window of K-1 previous rows in registers.
+#include <type_traits>
+
 #include "kda_common.cuh"
 #include "kda_launch.h"
 #include "kda_sm100.cuh"
@@ -73,15 +75,57 @@ __device__ __forceinline__ void st_tf32x4(unsigned char* p, float a, float b, fl
 __device__ __forceinline__ void st_bf16x4(unsigned char* p, float a, float b, float c, float d) {
   st4(reinterpret_cast<__nv_bfloat16*>(p), make_float4(a, b, c, d));
 }
-// sigmoid and SiLU on the special-function unit (approximate exp and reciprocal);
-// 1 / (1 + inf) = 0 keeps the saturated ends exact
-__device__ __forceinline__ float fsigmoid(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
-__device__ __forceinline__ float fsilu(float z) { return z * fsigmoid(z); }
+// Special-function-unit approximations (flush-to-zero: the values they would keep as
+// subnormals, below 2^-126, are negligible next to the bf16 tiles the pass writes).
+// Exponents are carried in log2 units, so an exponential is one ex2.
+constexpr float LOG2E = 1.4426950408889634f, LN2 = 0.6931471805599453f;
+__device__ __forceinline__ float ex2a(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcpa(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rsqrta(float x) {
+  float y;
+  asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// sigmoid of z given z2 = z log2(e); 1 / (1 + inf) = 0 keeps the saturated end exact
+__device__ __forceinline__ float sigmoid2(float z2) { return rcpa(1.f + ex2a(-z2)); }
 __device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 __device__ __forceinline__ void sts4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 // start pulling `bytes` (a multiple of 16, 16-byte aligned) at p into L2
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// acc += sum_m a[m] * b[m * AF_LD .. +3] over m < 16 (fp32 smem tiles), all loads issued first
+__device__ __forceinline__ void mac16(const float* a, const float* b, float4& acc) {
+  float av[16];
+  float4 bv[16];
+#pragma unroll
+  for (int m = 0; m < 16; m += 4) {
+    const float4 t = lds4(a + m);
+    av[m] = t.x; av[m + 1] = t.y; av[m + 2] = t.z; av[m + 3] = t.w;
+  }
+#pragma unroll
+  for (int m = 0; m < 16; ++m) bv[m] = lds4(b + m * AF_LD);
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    acc.x = fmaf(av[m], bv[m].x, acc.x); acc.y = fmaf(av[m], bv[m].y, acc.y);
+    acc.z = fmaf(av[m], bv[m].z, acc.z); acc.w = fmaf(av[m], bv[m].w, acc.w);
+  }
+}
+
+// four channels as loaded -> fp32 (bf16 widens by a 16-bit shift)
+__device__ __forceinline__ float4 to_f4(float4 v) { return v; }
+__device__ __forceinline__ float4 to_f4(uint2 v) {
+  return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                     __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -147,7 +191,60 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
 
-  // ---- log decay and its running sum G over the chunk: channels 2p, 2p+1, rows 16q.. ----
+  // ---- inputs of the token-row pass, issued now so their latency overlaps the gates
+  // (kept as loaded, converted after): lane l owns channels 4l..4l+3 of q, k and v in
+  // rows 8w..8w+7 of warp w ----
+  const int c4 = 4 * lane;
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x);
+  const __nv_bfloat16* cs = static_cast<const __nv_bfloat16*>(a.conv_state);
+  using RawT = typename std::conditional<FUSED, uint2, float4>::type;   // 4 channels as loaded
+  // fused prep state: conv taps (one float4 per channel) and the K-1 previous pre-conv rows
+  float4 cw[3][4];
+  RawT winr[KC - 1][3];
+  if (FUSED) {
+#pragma unroll
+    for (int sgm = 0; sgm < 3; ++sgm)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        cw[sgm][j] = __ldg(reinterpret_cast<const float4*>(
+            a.conv_w + ((size_t)h * 3 * D + sgm * D + c4 + j) * KC));
+#pragma unroll
+    for (int m = 0; m < KC - 1; ++m) {
+      const int tok = t0 + 8 * warp - (KC - 1) + m;
+      const __nv_bfloat16* src = nullptr;
+      if (tok >= tr.start && tok < tr.end)   // rows past the end only feed padded rows
+        src = x + ((size_t)tok * H + h) * 3 * D;
+      else if (tok < tr.start && cs != nullptr)
+        src = cs + (((size_t)prow * (KC - 1) + (KC - 1 + tok - tr.start)) * H + h) * 3 * D;
+#pragma unroll
+      for (int sgm = 0; sgm < 3; ++sgm)
+        winr[m][sgm] = src ? *reinterpret_cast<const RawT*>(src + sgm * D + c4) : RawT{};
+    }
+  }
+  // row r's q, k, v channels c4..c4+3 (pre-conv x when fused); zero past the sequence end
+  auto load_row = [&](int r, RawT& iq, RawT& ik, RawT& iv) {
+    iq = ik = iv = RawT{};
+    if (r < L) {
+      if (FUSED) {
+        const __nv_bfloat16* xp = x + ((size_t)(t0 + r) * H + h) * 3 * D;
+        iq = *reinterpret_cast<const RawT*>(xp + c4);
+        ik = *reinterpret_cast<const RawT*>(xp + D + c4);
+        iv = *reinterpret_cast<const RawT*>(xp + 2 * D + c4);
+      } else {
+        const size_t idx = ((size_t)(t0 + r) * H + h) * D + c4;
+        iq = *reinterpret_cast<const RawT*>(a.q + idx);
+        ik = *reinterpret_cast<const RawT*>(a.k + idx);
+        iv = *reinterpret_cast<const RawT*>(a.v + idx);
+      }
+    }
+  };
+  // the first two rows in flight too (two rows ahead of the one being computed)
+  RawT cq, ck, cv, n1q, n1k, n1v;
+  load_row(8 * warp, cq, ck, cv);
+  load_row(8 * warp + 1, n1q, n1k, n1v);
+
+  // ---- log decay and its running sum G over the chunk, in log2 units (G log2 e):
+  // channels 2p, 2p+1, rows 16q..16q+15 per thread ----
   {
     const int cp = 2 * (tid & 63), qr = tid >> 6;
     float g0[16], g1[16];
@@ -161,13 +258,14 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
         g0[i] = v.x;
         g1[i] = v.y;
       }
-      const float Ah = expf(__ldg(a.A_log + h));
+      // log2 a = lb log2(e) sigmoid(exp(A_log) (f + dt_bias))
+      const float Ah2 = expf(__ldg(a.A_log + h)) * LOG2E, lb2 = a.lb * LOG2E;
       const float2 db = *reinterpret_cast<const float2*>(a.dt_bias + (size_t)h * D + cp);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const bool live = 16 * qr + i < L;
-        g0[i] = live ? a.lb * fsigmoid(Ah * (g0[i] + db.x)) : 0.f;
-        g1[i] = live ? a.lb * fsigmoid(Ah * (g1[i] + db.y)) : 0.f;
+        g0[i] = live ? lb2 * sigmoid2(Ah2 * (g0[i] + db.x)) : 0.f;
+        g1[i] = live ? lb2 * sigmoid2(Ah2 * (g1[i] + db.y)) : 0.f;
       }
     } else {
 #pragma unroll
@@ -175,8 +273,45 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
         const int r = 16 * qr + i;
         float2 v = make_float2(0.f, 0.f);
         if (r < L) v = ld2(a.loga + ((size_t)(t0 + r) * H + h) * D + cp);
-        g0[i] = v.x;
-        g1[i] = v.y;
+        g0[i] = v.x * LOG2E;
+        g1[i] = v.y * LOG2E;
+      }
+    }
+    // while those loads are in flight: pull into L2 the inputs of the tile one wave of
+    // CTAs ahead in the grid (it will run after this one), 128-byte lines spread over threads
+    if (a.pf_stride > 0) {
+      const long long nid = (long long)blockIdx.y * gridDim.x + blockIdx.x + a.pf_stride;
+      if (nid < (long long)gridDim.x * gridDim.y) {
+        const int nh = (int)(nid / gridDim.x), ns = (int)(nid % gridDim.x);
+        // same sequence (slots of a sequence are consecutive): no search
+        const int nc = tr.chunk + (ns - slot);
+        TileRange nt;
+        if (nc >= 0 && (long long)nc * C < tr.end - tr.start) {
+          nt = tr;
+          nt.chunk = nc;
+          nt.t0 = tr.start + nc * C;
+          nt.len = min(C, tr.end - nt.t0);
+        } else {
+          nt = slot_to_tile(a.cu, a.n_seqs, a.total, C, ns);
+        }
+        const int w0 = max(nt.start, nt.t0 - (KC - 1));      // window rows inside the sequence
+        const int nrow = nt.t0 + nt.len - w0;
+        // per row: x (FUSED: 6 lines) or q, k, v (12 lines), then f or log a (2 or 4 lines)
+        const int lx = FUSED ? 6 : 12, lg = FUSED ? 2 : 4, per = lx + lg;
+        for (int e = tid; e < nrow * per; e += THREADS) {
+          const int tok = w0 + e / per, l = e % per;
+          const size_t row = (size_t)tok * H + nh;
+          const char* p;
+          if (l < lx) {
+            if (FUSED) p = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.x) + row * 3 * D) + 128 * l;
+            else p = reinterpret_cast<const char*>((l < 4 ? a.q : l < 8 ? a.k : a.v) + row * D) + 128 * (l & 3);
+          } else {
+            if (tok < nt.t0) continue;                         // no gates for window rows
+            p = FUSED ? reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.f) + row * D) + 128 * (l - lx)
+                      : reinterpret_cast<const char*>(a.loga + row * D) + 128 * (l - lx);
+          }
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+        }
       }
     }
 #pragma unroll
@@ -190,7 +325,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
       float bv = 0.f;
       if (tid < L) {
         const size_t bi = (size_t)(t0 + tid) * H + h;
-        bv = FUSED ? fsigmoid(ld1(static_cast<const __nv_bfloat16*>(a.beta_logit) + bi))
+        bv = FUSED ? sigmoid2(LOG2E * ld1(static_cast<const __nv_bfloat16*>(a.beta_logit) + bi))
                    : __ldg(a.beta + bi);
       }
       bs[tid] = bv;
@@ -207,7 +342,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     for (int i = 0; i < 16; ++i)
       *reinterpret_cast<float2*>(G + (16 * qr + i) * D + cp) = make_float2(g0[i] + o0, g1[i] + o1);
     if (qr == 3)
-      *reinterpret_cast<float2*>(gCo + cp) = make_float2(__expf(g0[15] + o0), __expf(g1[15] + o1));
+      *reinterpret_cast<float2*>(gCo + cp) = make_float2(ex2a(g0[15] + o0), ex2a(g1[15] + o1));
   }
   tc_fence_before();
   __syncthreads();
@@ -216,68 +351,41 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
 
   // ---- token rows 8w..8w+7: (prep), operands for the MMAs, Q~ and K' ----
   {
-    const int c4 = 4 * lane;
-    const float qsc = a.q_scale, inv_eps = 1.0f / a.l2_eps;
-    const float4 g15 = lds4(G + 15 * D + c4), g47 = lds4(G + 47 * D + c4),
-                 g63 = lds4(G + 63 * D + c4);
-    const float r15[4] = {g15.x, g15.y, g15.z, g15.w}, r47[4] = {g47.x, g47.y, g47.z, g47.w},
-                r63[4] = {g63.x, g63.y, g63.z, g63.w};
-    const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x);
-    const __nv_bfloat16* cs = static_cast<const __nv_bfloat16*>(a.conv_state);
-    // fused prep state: conv taps (one float4 per channel) and the K-1 previous pre-conv rows
-    float4 cw[3][4];
     float win[KC - 1][12];
     if (FUSED) {
 #pragma unroll
       for (int sgm = 0; sgm < 3; ++sgm)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          cw[sgm][j] = __ldg(reinterpret_cast<const float4*>(
-              a.conv_w + ((size_t)h * 3 * D + sgm * D + c4 + j) * KC));
+          cw[sgm][j] = make_float4(cw[sgm][j].x * LOG2E, cw[sgm][j].y * LOG2E,
+                                   cw[sgm][j].z * LOG2E, cw[sgm][j].w * LOG2E);
 #pragma unroll
-      for (int m = 0; m < KC - 1; ++m) {
-        const int tok = t0 + 8 * warp - (KC - 1) + m;
-        float4 vq = make_float4(0.f, 0.f, 0.f, 0.f), vk = vq, vv = vq;
-        if (tok >= tr.start && tok < tr.end) {   // rows past the end only feed padded rows
-          const __nv_bfloat16* xp = x + ((size_t)tok * H + h) * 3 * D;
-          vq = ld4(xp + c4); vk = ld4(xp + D + c4); vv = ld4(xp + 2 * D + c4);
-        } else if (tok < tr.start && cs != nullptr) {
-          const __nv_bfloat16* hp =
-              cs + (((size_t)prow * (KC - 1) + (KC - 1 + tok - tr.start)) * H + h) * 3 * D;
-          vq = ld4(hp + c4); vk = ld4(hp + D + c4); vv = ld4(hp + 2 * D + c4);
+      for (int m = 0; m < KC - 1; ++m)
+#pragma unroll
+        for (int sgm = 0; sgm < 3; ++sgm) {
+          const float4 t = to_f4(winr[m][sgm]);
+          win[m][4 * sgm] = t.x; win[m][4 * sgm + 1] = t.y;
+          win[m][4 * sgm + 2] = t.z; win[m][4 * sgm + 3] = t.w;
         }
-        win[m][0] = vq.x; win[m][1] = vq.y; win[m][2] = vq.z; win[m][3] = vq.w;
-        win[m][4] = vk.x; win[m][5] = vk.y; win[m][6] = vk.z; win[m][7] = vk.w;
-        win[m][8] = vv.x; win[m][9] = vv.y; win[m][10] = vv.z; win[m][11] = vv.w;
-      }
     }
-    // row r's q, k, v channels c4..c4+3 (pre-conv x when fused); zero past the sequence end
-    auto load_row = [&](int r, float4& iq, float4& ik, float4& iv) {
-      iq = ik = iv = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < L) {
-        if (FUSED) {
-          const __nv_bfloat16* xp = x + ((size_t)(t0 + r) * H + h) * 3 * D;
-          iq = ld4(xp + c4); ik = ld4(xp + D + c4); iv = ld4(xp + 2 * D + c4);
-        } else {
-          const size_t idx = ((size_t)(t0 + r) * H + h) * D + c4;
-          iq = ld4(a.q + idx); ik = ld4(a.k + idx); iv = ld4(a.v + idx);
-        }
-      }
-    };
-    // two rows in flight ahead of the one being computed
-    float4 cq, ck, cv, n1q, n1k, n1v;
-    load_row(8 * warp, cq, ck, cv);
-    load_row(8 * warp + 1, n1q, n1k, n1v);
+    // q, k and v leave the conv scaled by log2 e (taps pre-scaled): the L2 norm of q and k
+    // cancels the factor (with eps scaled alike) and v takes ln 2 back
+    const float qsc = a.q_scale, inv_eps = 1.0f / (a.l2_eps * LOG2E);
+    const float4 g15 = lds4(G + 15 * D + c4), g47 = lds4(G + 47 * D + c4),
+                 g63 = lds4(G + 63 * D + c4);
+    const float r15[4] = {g15.x, g15.y, g15.z, g15.w}, r47[4] = {g47.x, g47.y, g47.z, g47.w},
+                r63[4] = {g63.x, g63.y, g63.z, g63.w};
 #pragma unroll 1
     for (int i = 0; i < 8; ++i) {
       const int r = 8 * warp + i;
-      float4 n2q, n2k, n2v;
+      RawT n2q, n2k, n2v;
       load_row(i + 2 < 8 ? r + 2 : C, n2q, n2k, n2v);
+      const float4 fq = to_f4(cq), fk = to_f4(ck), fv = to_f4(cv);
       float qv[4], kv[4], vv[4];
       if (FUSED) {
-        const float xq[4] = {cq.x, cq.y, cq.z, cq.w};
-        const float xk[4] = {ck.x, ck.y, ck.z, ck.w};
-        const float xv[4] = {cv.x, cv.y, cv.z, cv.w};
+        const float xq[4] = {fq.x, fq.y, fq.z, fq.w};
+        const float xk[4] = {fk.x, fk.y, fk.z, fk.w};
+        const float xv[4] = {fv.x, fv.y, fv.z, fv.w};
         float sq = 0.f, sk = 0.f;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -289,9 +397,9 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
           ak = fmaf(wk.z, win[2][4 + j], ak);
           av = fmaf(wv.x, win[0][8 + j], av); av = fmaf(wv.y, win[1][8 + j], av);
           av = fmaf(wv.z, win[2][8 + j], av);
-          qv[j] = fsilu(aq);
-          kv[j] = fsilu(ak);
-          vv[j] = fsilu(av);
+          qv[j] = aq * sigmoid2(aq);
+          kv[j] = ak * sigmoid2(ak);
+          vv[j] = LN2 * av * sigmoid2(av);
           sq = fmaf(qv[j], qv[j], sq);
           sk = fmaf(kv[j], kv[j], sk);
         }
@@ -308,8 +416,8 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
         sk = warp_sum(sk);
         const bool live = r < L;   // rows past the sequence end stay zero
         // 1 / max(||x||, eps) = min(rsqrt(||x||^2), 1 / eps), rsqrt(0) = inf
-        const float iq = live ? fminf(rsqrtf(sq), inv_eps) : 0.f;
-        const float ik = live ? fminf(rsqrtf(sk), inv_eps) : 0.f;
+        const float iq = live ? qsc * fminf(rsqrta(sq), inv_eps) : 0.f;   // q_scale folded in
+        const float ik = live ? fminf(rsqrta(sk), inv_eps) : 0.f;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           qv[j] *= iq;
@@ -317,9 +425,9 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
           vv[j] = live ? vv[j] : 0.f;
         }
       } else {
-        qv[0] = cq.x; qv[1] = cq.y; qv[2] = cq.z; qv[3] = cq.w;
-        kv[0] = ck.x; kv[1] = ck.y; kv[2] = ck.z; kv[3] = ck.w;
-        vv[0] = cv.x; vv[1] = cv.y; vv[2] = cv.z; vv[3] = cv.w;
+        qv[0] = qsc * fq.x; qv[1] = qsc * fq.y; qv[2] = qsc * fq.z; qv[3] = qsc * fq.w;
+        kv[0] = fk.x; kv[1] = fk.y; kv[2] = fk.z; kv[3] = fk.w;
+        vv[0] = fv.x; vv[1] = fv.y; vv[2] = fv.z; vv[3] = fv.w;
       }
       const float4 gr4 = lds4(G + r * D + c4);
       const float gr[4] = {gr4.x, gr4.y, gr4.z, gr4.w};
@@ -328,15 +436,15 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float g = gr[j];
-        const float er = __expf(g - (lowhalf ? r15[j] : r47[j]));
+        const float er = ex2a(g - (lowhalf ? r15[j] : r47[j]));
         kb[j] = kv[j] * er;
-        qb[j] = qsc * qv[j] * er;
-        kc0[j] = lowhalf ? kv[j] * __expf(r15[j] - g) : 0.f;
-        kc1[j] = kv[j] * __expf(r47[j] - g);
-        const float eg = __expf(g);
-        qt[j] = qsc * qv[j] * eg;
+        qb[j] = qv[j] * er;                       // qv carries q_scale
+        kc0[j] = lowhalf ? kv[j] * ex2a(r15[j] - g) : 0.f;
+        kc1[j] = kv[j] * ex2a(r47[j] - g);
+        const float eg = ex2a(g);
+        qt[j] = qv[j] * eg;
         kt[j] = kv[j] * eg;
-        kp[j] = kv[j] * __expf(r63[j] - g);
+        kp[j] = kv[j] * ex2a(r63[j] - g);
       }
       const int nk = lowhalf ? r : 64 + (r - 32);
       st_tf32x4(sm + OFF_GB + gram_off(nk, c4), kb[0], kb[1], kb[2], kb[3]);
@@ -429,32 +537,16 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
       if (act) {
         float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 1
-        for (int kb = bb; kb < ab; ++kb) {
-          const float* Ar = Af + (16 * ab + rho) * AF_LD + 16 * kb;
-          const float* Xk = Xs + (16 * kb) * AF_LD + 16 * bb + k4;
-#pragma unroll
-          for (int m = 0; m < 16; ++m) {
-            const float l = Ar[m];
-            const float4 xv = lds4(Xk + m * AF_LD);
-            z.x = fmaf(l, xv.x, z.x); z.y = fmaf(l, xv.y, z.y);
-            z.z = fmaf(l, xv.z, z.z); z.w = fmaf(l, xv.w, z.w);
-          }
-        }
+        for (int kb = bb; kb < ab; ++kb)
+          mac16(Af + (16 * ab + rho) * AF_LD + 16 * kb, Xs + (16 * kb) * AF_LD + 16 * bb + k4, z);
         sts4(Zs + (16 * ab + rho) * AF_LD + 16 * bb + k4, z);
       }
       __syncthreads();
       if (act) {
         float4 xo = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float* Xa = Xs + (16 * ab + rho) * AF_LD + 16 * ab;
-        const float* Zb = Zs + (16 * ab) * AF_LD + 16 * bb + k4;
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          const float xa = Xa[m];
-          const float4 zv = lds4(Zb + m * AF_LD);
-          xo.x = fmaf(-xa, zv.x, xo.x); xo.y = fmaf(-xa, zv.y, xo.y);
-          xo.z = fmaf(-xa, zv.z, xo.z); xo.w = fmaf(-xa, zv.w, xo.w);
-        }
-        sts4(Xs + (16 * ab + rho) * AF_LD + 16 * bb + k4, xo);
+        mac16(Xs + (16 * ab + rho) * AF_LD + 16 * ab, Zs + (16 * ab) * AF_LD + 16 * bb + k4, xo);
+        sts4(Xs + (16 * ab + rho) * AF_LD + 16 * bb + k4,
+             make_float4(-xo.x, -xo.y, -xo.z, -xo.w));
       }
       __syncthreads();
     }
@@ -551,7 +643,13 @@ cudaError_t launch_intra_t(const PrefillArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(intra_chunk_sm100_kernel<FUSED>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  intra_chunk_sm100_kernel<FUSED><<<dim3(a.L.nslots, a.H), THREADS, SMEM_BYTES, st>>>(a);
+  int dev = 0, nsm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  PrefillArgs b = a;
+  b.pf_stride = nsm;   // one CTA per SM (shared memory bound): the next wave is nsm ahead
+  intra_chunk_sm100_kernel<FUSED><<<dim3(a.L.nslots, a.H), THREADS, SMEM_BYTES, st>>>(b);
   return cudaGetLastError();
 }
 
