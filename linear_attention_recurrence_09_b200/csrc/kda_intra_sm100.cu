@@ -55,9 +55,10 @@ constexpr uint32_t OFF_TL = OFF_GA + 8192;  // T low part
 constexpr int AF_LD = 68;                   // row stride (floats) of the fp32 tiles of the solve
 constexpr uint32_t TILE32 = 64 * AF_LD * 4;
 constexpr uint32_t OFF_XS = OFF_GA + 16384;  // X = (I + A)^{-1}, fp32 [64][68], after the gram
-constexpr uint32_t OFF_ZS = OFF_XS + TILE32; // block products of the solve, fp32 [64][68]
+constexpr uint32_t OFF_ZS = OFF_XS + TILE32; // per-warp block products of the solve
+constexpr int ZW_LD = 72;                    // their row stride (floats): fragment reads spread banks
 constexpr uint32_t SMEM_BYTES = OFF_G + 32768 + 1024;
-static_assert(OFF_ZS + TILE32 <= OFF_GB, "solve tiles must fit in the gram A area");
+static_assert(OFF_ZS + 6 * 16 * ZW_LD * 4 <= OFF_GB, "solve tiles must fit in the gram A area");
 static_assert(TILE32 <= 32768, "A must fit in the G area");
 
 __device__ __forceinline__ uint32_t gram_off(int n, int c) {   // tf32 K-major, K = 128
@@ -97,28 +98,39 @@ __device__ __forceinline__ float rsqrta(float x) {
 // sigmoid of z given z2 = z log2(e); 1 / (1 + inf) = 0 keeps the saturated end exact
 __device__ __forceinline__ float sigmoid2(float z2) { return rcpa(1.f + ex2a(-z2)); }
 __device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
-__device__ __forceinline__ void sts4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 // start pulling `bytes` (a multiple of 16, 16-byte aligned) at p into L2
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-// acc += sum_m a[m] * b[m * AF_LD .. +3] over m < 16 (fp32 smem tiles), all loads issued first
-__device__ __forceinline__ void mac16(const float* a, const float* b, float4& acc) {
-  float av[16];
-  float4 bv[16];
+// x = hi + lo with hi, lo tf32 (round to nearest)
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(x - __uint_as_float(hi)));
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4],
+                                         const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// d (16 x 8, fragment layout) += A (16 x 8, row-major, stride lda) . B (8 x 8 [k][n], stride
+// ldb), fp32 smem operands, as three tf32 products (the lo.lo term, ~2^-22, dropped)
+__device__ __forceinline__ void mma3_tf32(float (&d)[4], const float* A, int lda, const float* B,
+                                          int ldb, int g, int t) {
+  const float av[4] = {A[g * lda + t], A[(g + 8) * lda + t], A[g * lda + t + 4],
+                       A[(g + 8) * lda + t + 4]};
+  const float bv[2] = {B[t * ldb + g], B[(t + 4) * ldb + g]};
+  uint32_t ah[4], al[4], bh[2], bl[2];
 #pragma unroll
-  for (int m = 0; m < 16; m += 4) {
-    const float4 t = lds4(a + m);
-    av[m] = t.x; av[m + 1] = t.y; av[m + 2] = t.z; av[m + 3] = t.w;
-  }
+  for (int i = 0; i < 4; ++i) split_tf32(av[i], ah[i], al[i]);
 #pragma unroll
-  for (int m = 0; m < 16; ++m) bv[m] = lds4(b + m * AF_LD);
-#pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    acc.x = fmaf(av[m], bv[m].x, acc.x); acc.y = fmaf(av[m], bv[m].y, acc.y);
-    acc.z = fmaf(av[m], bv[m].z, acc.z); acc.w = fmaf(av[m], bv[m].w, acc.w);
-  }
+  for (int i = 0; i < 2; ++i) split_tf32(bv[i], bh[i], bl[i]);
+  mma_tf32(d, al, bh);
+  mma_tf32(d, ah, bl);
+  mma_tf32(d, ah, bh);
 }
 
 // four channels as loaded -> fp32 (bf16 widens by a 16-bit shift)
@@ -164,7 +176,27 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   float* G = reinterpret_cast<float*>(sm + OFF_G);
   float* Af = G;                                  // [64][AF_LD], after the gram
   float* Xs = reinterpret_cast<float*>(sm + OFF_XS);
-  float* Zs = reinterpret_cast<float*>(sm + OFF_ZS);
+
+  // gate inputs first (the gate pass waits on them): channels 2p, 2p+1 of rows 16q..16q+15
+  const int cp = 2 * (tid & 63), qr = tid >> 6;
+  float g0[16], g1[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int r = 16 * qr + i;
+    float2 v = make_float2(0.f, 0.f);
+    if (r < L) {
+      const size_t idx = ((size_t)(t0 + r) * H + h) * D + cp;
+      v = FUSED ? ld2(static_cast<const __nv_bfloat16*>(a.f) + idx) : ld2(a.loga + idx);
+    }
+    g0[i] = v.x;
+    g1[i] = v.y;
+  }
+  float A_log_h = 0.f;
+  float2 dtb = make_float2(0.f, 0.f);
+  if (FUSED) {
+    A_log_h = __ldg(a.A_log + h);
+    dtb = *reinterpret_cast<const float2*>(a.dt_bias + (size_t)h * D + cp);
+  }
 
   // this tile's rows start streaming into L2 while the gates are computed
   if (tid < L) {
@@ -246,38 +278,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   // ---- log decay and its running sum G over the chunk, in log2 units (G log2 e):
   // channels 2p, 2p+1, rows 16q..16q+15 per thread ----
   {
-    const int cp = 2 * (tid & 63), qr = tid >> 6;
-    float g0[16], g1[16];
-    if (FUSED) {
-      const __nv_bfloat16* f = static_cast<const __nv_bfloat16*>(a.f);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = 16 * qr + i;
-        float2 v = make_float2(0.f, 0.f);
-        if (r < L) v = ld2(f + ((size_t)(t0 + r) * H + h) * D + cp);
-        g0[i] = v.x;
-        g1[i] = v.y;
-      }
-      // log2 a = lb log2(e) sigmoid(exp(A_log) (f + dt_bias))
-      const float Ah2 = expf(__ldg(a.A_log + h)) * LOG2E, lb2 = a.lb * LOG2E;
-      const float2 db = *reinterpret_cast<const float2*>(a.dt_bias + (size_t)h * D + cp);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const bool live = 16 * qr + i < L;
-        g0[i] = live ? lb2 * sigmoid2(Ah2 * (g0[i] + db.x)) : 0.f;
-        g1[i] = live ? lb2 * sigmoid2(Ah2 * (g1[i] + db.y)) : 0.f;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = 16 * qr + i;
-        float2 v = make_float2(0.f, 0.f);
-        if (r < L) v = ld2(a.loga + ((size_t)(t0 + r) * H + h) * D + cp);
-        g0[i] = v.x * LOG2E;
-        g1[i] = v.y * LOG2E;
-      }
-    }
-    // while those loads are in flight: pull into L2 the inputs of the tile one wave of
+    // while the gate loads are in flight: pull into L2 the inputs of the tile one wave of
     // CTAs ahead in the grid (it will run after this one), 128-byte lines spread over threads
     if (a.pf_stride > 0) {
       const long long nid = (long long)blockIdx.y * gridDim.x + blockIdx.x + a.pf_stride;
@@ -312,6 +313,22 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
           }
           asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
         }
+      }
+    }
+    if (FUSED) {
+      // log2 a = lb log2(e) sigmoid(exp(A_log) (f + dt_bias))
+      const float Ah2 = expf(A_log_h) * LOG2E, lb2 = a.lb * LOG2E;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const bool live = 16 * qr + i < L;
+        g0[i] = live ? lb2 * sigmoid2(Ah2 * (g0[i] + dtb.x)) : 0.f;
+        g1[i] = live ? lb2 * sigmoid2(Ah2 * (g1[i] + dtb.y)) : 0.f;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        g0[i] *= LOG2E;
+        g1[i] *= LOG2E;
       }
     }
 #pragma unroll
@@ -529,24 +546,37 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   }
   __syncthreads();
   {
-    const int q = tid >> 6, rho = (tid >> 2) & 15, k4 = 4 * (tid & 3);
+    // one warp per (block, 8-column half): Z = sum_k A_ak X_kb, then X_ab = -X_aa Z, as
+    // m16n8k8 tf32 tensor-core products split 3 ways (hi.hi + hi.lo + lo.hi ~ fp32)
+    const int g = lane >> 2, t = lane & 3;
+    float* Zw = reinterpret_cast<float*>(sm + OFF_ZS) + warp * 16 * ZW_LD;
 #pragma unroll 1
     for (int dg = 1; dg < 4; ++dg) {
-      const bool act = q < 4 - dg;
-      const int ab = q + dg, bb = q;   // block (ab, bb) of this block diagonal
-      if (act) {
-        float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (warp < 2 * (4 - dg)) {
+        const int ab = (warp >> 1) + dg, bb = warp >> 1, n0 = 16 * bb + 8 * (warp & 1);
+        float z[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
         for (int kb = bb; kb < ab; ++kb)
-          mac16(Af + (16 * ab + rho) * AF_LD + 16 * kb, Xs + (16 * kb) * AF_LD + 16 * bb + k4, z);
-        sts4(Zs + (16 * ab + rho) * AF_LD + 16 * bb + k4, z);
-      }
-      __syncthreads();
-      if (act) {
-        float4 xo = make_float4(0.f, 0.f, 0.f, 0.f);
-        mac16(Xs + (16 * ab + rho) * AF_LD + 16 * ab, Zs + (16 * ab) * AF_LD + 16 * bb + k4, xo);
-        sts4(Xs + (16 * ab + rho) * AF_LD + 16 * bb + k4,
-             make_float4(-xo.x, -xo.y, -xo.z, -xo.w));
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks)
+            mma3_tf32(z, Af + (16 * ab) * AF_LD + 16 * kb + 8 * ks, AF_LD,
+                      Xs + (16 * kb + 8 * ks) * AF_LD + n0, AF_LD, g, t);
+        Zw[g * ZW_LD + 2 * t] = z[0];
+        Zw[g * ZW_LD + 2 * t + 1] = z[1];
+        Zw[(g + 8) * ZW_LD + 2 * t] = z[2];
+        Zw[(g + 8) * ZW_LD + 2 * t + 1] = z[3];
+        __syncwarp();
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+          mma3_tf32(y, Xs + (16 * ab) * AF_LD + 16 * ab + 8 * ks, AF_LD, Zw + (8 * ks) * ZW_LD,
+                    ZW_LD, g, t);
+        float* xo = Xs + (16 * ab + g) * AF_LD + n0 + 2 * t;
+        xo[0] = -y[0];
+        xo[1] = -y[1];
+        xo[8 * AF_LD] = -y[2];
+        xo[8 * AF_LD + 1] = -y[3];
+        __syncwarp();
       }
       __syncthreads();
     }
