@@ -117,9 +117,10 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4],
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 // d (16 x 8, fragment layout) += A (16 x 8, row-major, stride lda) . B (8 x 8 [k][n], stride
-// ldb), fp32 smem operands, as three tf32 products (the lo.lo term, ~2^-22, dropped)
-__device__ __forceinline__ void mma3_tf32(float (&d)[4], const float* A, int lda, const float* B,
-                                          int ldb, int g, int t) {
+// ldb), fp32 smem operands, as three tf32 products (the lo.lo term, ~2^-22, dropped), each
+// into its own accumulator so consecutive calls form three short dependency chains
+__device__ __forceinline__ void mma3_tf32(float (&d)[3][4], const float* A, int lda,
+                                          const float* B, int ldb, int g, int t) {
   const float av[4] = {A[g * lda + t], A[(g + 8) * lda + t], A[g * lda + t + 4],
                        A[(g + 8) * lda + t + 4]};
   const float bv[2] = {B[t * ldb + g], B[(t + 4) * ldb + g]};
@@ -128,9 +129,12 @@ __device__ __forceinline__ void mma3_tf32(float (&d)[4], const float* A, int lda
   for (int i = 0; i < 4; ++i) split_tf32(av[i], ah[i], al[i]);
 #pragma unroll
   for (int i = 0; i < 2; ++i) split_tf32(bv[i], bh[i], bl[i]);
-  mma_tf32(d, al, bh);
-  mma_tf32(d, ah, bl);
-  mma_tf32(d, ah, bh);
+  mma_tf32(d[0], ah, bh);
+  mma_tf32(d[1], al, bh);
+  mma_tf32(d[2], ah, bl);
+}
+__device__ __forceinline__ float sum3(const float (&d)[3][4], int i) {
+  return d[0][i] + (d[1][i] + d[2][i]);
 }
 
 // four channels as loaded -> fp32 (bf16 widens by a 16-bit shift)
@@ -554,28 +558,31 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     for (int dg = 1; dg < 4; ++dg) {
       if (warp < 2 * (4 - dg)) {
         const int ab = (warp >> 1) + dg, bb = warp >> 1, n0 = 16 * bb + 8 * (warp & 1);
-        float z[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-        for (int kb = bb; kb < ab; ++kb)
+        float z[3][4] = {};
 #pragma unroll
-          for (int ks = 0; ks < 2; ++ks)
-            mma3_tf32(z, Af + (16 * ab) * AF_LD + 16 * kb + 8 * ks, AF_LD,
-                      Xs + (16 * kb + 8 * ks) * AF_LD + n0, AF_LD, g, t);
-        Zw[g * ZW_LD + 2 * t] = z[0];
-        Zw[g * ZW_LD + 2 * t + 1] = z[1];
-        Zw[(g + 8) * ZW_LD + 2 * t] = z[2];
-        Zw[(g + 8) * ZW_LD + 2 * t + 1] = z[3];
+        for (int kk = 0; kk < 3; ++kk)
+          if (kk < dg) {
+            const int kb = bb + kk;
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks)
+              mma3_tf32(z, Af + (16 * ab) * AF_LD + 16 * kb + 8 * ks, AF_LD,
+                        Xs + (16 * kb + 8 * ks) * AF_LD + n0, AF_LD, g, t);
+          }
+        Zw[g * ZW_LD + 2 * t] = sum3(z, 0);
+        Zw[g * ZW_LD + 2 * t + 1] = sum3(z, 1);
+        Zw[(g + 8) * ZW_LD + 2 * t] = sum3(z, 2);
+        Zw[(g + 8) * ZW_LD + 2 * t + 1] = sum3(z, 3);
         __syncwarp();
-        float y[4] = {0.f, 0.f, 0.f, 0.f};
+        float y[3][4] = {};
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks)
           mma3_tf32(y, Xs + (16 * ab) * AF_LD + 16 * ab + 8 * ks, AF_LD, Zw + (8 * ks) * ZW_LD,
                     ZW_LD, g, t);
         float* xo = Xs + (16 * ab + g) * AF_LD + n0 + 2 * t;
-        xo[0] = -y[0];
-        xo[1] = -y[1];
-        xo[8 * AF_LD] = -y[2];
-        xo[8 * AF_LD + 1] = -y[3];
+        xo[0] = -sum3(y, 0);
+        xo[1] = -sum3(y, 1);
+        xo[8 * AF_LD] = -sum3(y, 2);
+        xo[8 * AF_LD + 1] = -sum3(y, 3);
         __syncwarp();
       }
       __syncthreads();

@@ -304,32 +304,45 @@ __global__ void __launch_bounds__(256) inter_chunk_kernel(const PrefillArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// pass 3: y = o / sqrt(mean(o^2) + eps) * w * sigmoid(g), one warp per (token, head)
+// pass 3: y = o / sqrt(mean(o^2) + eps) * w * sigmoid(g) per (token, head) row.
+// Streaming: lane owns 4 consecutive channels, D/4 lanes per row, and each warp keeps
+// NORM_PASSES groups of rows' loads in flight before reducing any of them.
 // ---------------------------------------------------------------------------
+constexpr int NORM_PASSES = 4;
+template <int D>
+constexpr int norm_rows_per_cta() { return 8 * (128 / D) * NORM_PASSES; }
+
 template <typename T, int D>
 __global__ void __launch_bounds__(256) gated_norm_kernel(const PrefillArgs a) {
-  const size_t rowi = (size_t)blockIdx.x * 8 + threadIdx.x / 32;
-  if (rowi >= (size_t)a.total * a.H) return;
-  const int lane = threadIdx.x & 31;
-  const float* o = reinterpret_cast<const float*>(a.ws + a.L.o) + rowi * D;
-  const T* g = static_cast<const T*>(a.g) + rowi * D;
-  T* y = static_cast<T*>(a.y) + rowi * D;
-  constexpr int PER = (D + 31) / 32;
-  float ov[PER];
-  float ss = 0.f;
+  constexpr int LPR = D / 4, RPW = 32 / LPR;   // lanes per row, rows per warp and pass
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane / LPR, c = 4 * (lane % LPR);
+  const size_t nrows = (size_t)a.total * a.H;
+  const size_t base = (size_t)blockIdx.x * norm_rows_per_cta<D>() + (size_t)warp * RPW * NORM_PASSES;
+  const float* o = reinterpret_cast<const float*>(a.ws + a.L.o);
+  const T* g = static_cast<const T*>(a.g);
+  float4 ov[NORM_PASSES], gv[NORM_PASSES];
 #pragma unroll
-  for (int m = 0; m < PER; ++m) {
-    const int c = lane + 32 * m;
-    ov[m] = (c < D) ? o[c] : 0.f;
-    ss = fmaf(ov[m], ov[m], ss);
+  for (int p = 0; p < NORM_PASSES; ++p) {
+    const size_t row = base + (size_t)p * RPW + sub;
+    ov[p] = gv[p] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (row < nrows) {
+      ov[p] = ld4(o + row * D + c);
+      gv[p] = ld4(g + row * D + c);
+    }
   }
+  const float4 w = ld4(a.norm_w + c);
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-  const float rstd = rsqrtf(ss / (float)D + a.norm_eps);
+  for (int p = 0; p < NORM_PASSES; ++p) {
+    float ss = ov[p].x * ov[p].x + ov[p].y * ov[p].y + ov[p].z * ov[p].z + ov[p].w * ov[p].w;
 #pragma unroll
-  for (int m = 0; m < PER; ++m) {
-    const int c = lane + 32 * m;
-    if (c < D) st1(y + c, ov[m] * rstd * __ldg(a.norm_w + c) * sigmoid(ld1(g + c)));
+    for (int off = LPR / 2; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float rstd = rsqrtf(ss / (float)D + a.norm_eps);
+    const size_t row = base + (size_t)p * RPW + sub;
+    if (row < nrows)
+      st4(static_cast<T*>(a.y) + row * D + c,
+          make_float4(ov[p].x * rstd * w.x * sigmoid(gv[p].x), ov[p].y * rstd * w.y * sigmoid(gv[p].y),
+                      ov[p].z * rstd * w.z * sigmoid(gv[p].z), ov[p].w * rstd * w.w * sigmoid(gv[p].w)));
   }
 }
 
@@ -367,7 +380,8 @@ static cudaError_t launch_prefill_dc(const PrefillArgs& a, cudaStream_t st) {
   if (pe.ev[1] && (e = cudaEventRecord(pe.ev[1], st)) != cudaSuccess) return e;
   if (a.total > 0) {
     const size_t rows = (size_t)a.total * a.H;
-    gated_norm_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(a);
+    constexpr int RPC = norm_rows_per_cta<D>();
+    gated_norm_kernel<T, D><<<(unsigned)((rows + RPC - 1) / RPC), 256, 0, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (pe.ev[2] && (e = cudaEventRecord(pe.ev[2], st)) != cudaSuccess) return e;
