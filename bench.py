@@ -135,6 +135,41 @@ def measured_peaks():
         return 6650.0, 1590.0, 'fallback'
 
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) comes from the
+# committed ncu summaries; a summary records the sha256 of the kernel's source file at
+# capture time and counts only while that file is unchanged.
+PROFILED = {
+    'intra_chunk': ('profiles/intra_chunk_sm100_prefill_8k.md',
+                    'linear_attention_recurrence_09_b200/csrc/kda_intra_sm100.cu'),
+    'inter_chunk': ('profiles/interchunk_sm100_prefill_8k.md',
+                    'linear_attention_recurrence_09_b200/csrc/kda_prefill_sm100.cu'),
+    'gated_norm': ('profiles/gated_norm_prefill_8k.md',
+                   'linear_attention_recurrence_09_b200/csrc/kda_prefill.cu'),
+    'kda_decode': ('profiles/step_decode_b64.md',
+                   'linear_attention_recurrence_09_b200/csrc/kda_step.cu'),
+    'kda_verify': ('profiles/step_verify_b16.md',
+                   'linear_attention_recurrence_09_b200/csrc/kda_step.cu'),
+}
+
+
+def profiled_traffic(kernel):
+    import hashlib
+    import re
+    if kernel not in PROFILED:
+        return None
+    summary, source = (os.path.join(ROOT, f) for f in PROFILED[kernel])
+    try:
+        text = open(summary).read()
+        digest = hashlib.sha256(open(source, 'rb').read()).hexdigest()
+    except OSError:
+        return None
+    m_hash = re.search(r'source_sha256:\s*([0-9a-f]{64})', text)
+    m_traffic = re.search(r'traffic_bytes_per_launch:\s*([0-9]+)', text)
+    if not (m_hash and m_traffic) or m_hash.group(1) != digest:
+        return None
+    return int(m_traffic.group(1))
+
+
 # ---------------------------------------------------------------------------
 # workloads
 # ---------------------------------------------------------------------------
@@ -265,7 +300,8 @@ def run_prefill(args, dist, torch, kda, synth, dev):
                 'ms_per_step': e2e_ms},
         'gpu_launches': len(PHASES) * args.steps,
         'roofline': {'bound': 'hbm', 'kernel': dominant[0], 'achieved': achieved, 'peak': hbm,
-                     'unit': 'GB/s', 'frac': achieved / hbm, 'traffic': None,
+                     'unit': 'GB/s', 'frac': achieved / hbm,
+                     'traffic': profiled_traffic(dominant[0]),
                      'peak_kind': peak_kind, 'algorithmic_bytes_per_launch': dominant[1]},
         'breakdown_ms': ms_phase,
         'phase_roofline': {ph: {'algorithmic_bytes': nb[ph],
@@ -346,7 +382,8 @@ def run_decode(torch, kda, synth, dev, steps=1024):
                         '(prep + decode per step, CUDA graph)',
             'ms_per_step': ms / steps, 'gpu_launches': 2 * steps,
             'roofline': {'bound': 'hbm', 'kernel': 'kda_decode', 'achieved': ach, 'peak': hbm,
-                         'unit': 'GB/s', 'frac': ach / hbm, 'traffic': None,
+                         'unit': 'GB/s', 'frac': ach / hbm,
+                         'traffic': profiled_traffic('kda_decode'),
                          'peak_kind': peak_kind, 'algorithmic_bytes_per_launch': bytes_k,
                          'ms_per_launch': ms_k,
                          'l2_note': 'state 134 MB is just above L2 (126 MB)'}}
@@ -420,7 +457,8 @@ def run_verify(torch, kda, synth, dev, rounds=256):
                         f'context, {rounds} rounds, accepted ~ U{{0..{Tb}}} (CUDA graph)',
             'ms_per_round': ms / rounds, 'gpu_launches': 3 * rounds,
             'roofline': {'bound': 'hbm', 'kernel': 'kda_verify', 'achieved': ach, 'peak': hbm,
-                         'unit': 'GB/s', 'frac': ach / hbm, 'traffic': None,
+                         'unit': 'GB/s', 'frac': ach / hbm,
+                         'traffic': profiled_traffic('kda_verify'),
                          'peak_kind': peak_kind, 'algorithmic_bytes_per_launch': bytes_k,
                          'ms_per_launch': ms_k}}
 
