@@ -190,17 +190,22 @@ def prefill_workload(torch, kda, synth, T, seed, dev):
 PHASES = ('intra_chunk', 'inter_chunk', 'gated_norm')
 
 
-def prefill_bytes(T, H, d, C=64, K=4):
+def prefill_bytes(T, H, d, C=64, K=4, fused_norm=True):
     """Algorithmic HBM bytes per launch of each pass of kda_layer_prefill (bf16
-    activations, fp32 state, bf16 chunk tiles, fp32 o), and of the layer as a whole
-    (inputs x, f, beta logit, g read once, y and the final state written once)."""
+    activations, fp32 state, bf16 chunk tiles), and of the layer as a whole (inputs x,
+    f, beta logit, g read once, y and the final state written once).  With the norm
+    fused into the inter-chunk pass that pass reads g and writes y; otherwise it writes
+    o (fp32) and the gated-norm pass reads o and g and writes y."""
     th = T * H
     nch = -(-T // C)
     tiles = th * (4 * d * 2 + C * 2) + nch * H * d * 4          # W, U~, Q~, K', M; e^{G_C}
     intra = th * (3 * d * 2 + d * 2 + 2) + tiles + H * (3 * d * K + 1 + d) * 4
+    layer = th * (3 * d * 2 + d * 2 + 2 + d * 2 + d * 2) + H * d * d * 4
+    if fused_norm:
+        inter = tiles + th * d * 2 + d * 4 + th * d * 2 + H * d * d * 4   # + g, norm_w in; y out
+        return {'intra_chunk': intra, 'inter_chunk': inter, 'layer': layer}
     inter = tiles + th * d * 4 + H * d * d * 4                  # tiles in, o and state out
     norm = th * d * 4 + th * d * 2 + d * 4 + th * d * 2         # o, g, norm_w in; y out
-    layer = th * (3 * d * 2 + d * 2 + 2 + d * 2 + d * 2) + H * d * d * 4
     return {'intra_chunk': intra, 'inter_chunk': inter, 'gated_norm': norm, 'layer': layer}
 
 
@@ -234,10 +239,12 @@ def run_prefill(args, dist, torch, kda, synth, dev):
     per = [[ev() for _ in range(4)] for _ in range(args.steps)]
     t_start, t_end = ev(), ev()
     wall0 = time.perf_counter()
+    n_launch0 = kda.kda_launch_count()
     t_start.record(stream)
     for i in range(args.steps):
         step(per[i])
     t_end.record(stream)
+    launches = kda.kda_launch_count() - n_launch0
     torch.cuda.synchronize()
     dist.barrier()
     ms = t_start.elapsed_time(t_end)
@@ -246,8 +253,10 @@ def run_prefill(args, dist, torch, kda, synth, dev):
         step()
         torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
+    fused_norm = launches == 2 * args.steps      # intra + inter (norm inside the inter pass)
+    phases = PHASES[:2] if fused_norm else PHASES
     ms_phase = {ph: statistics.mean(p[i].elapsed_time(p[i + 1]) for p in per)
-                for i, ph in enumerate(PHASES)}
+                for i, ph in enumerate(phases)}
     ms_max = dist.max(ms)
     ms_step = ms_max / args.steps
     T, H, d = W['T'], W['H'], W['d']
@@ -281,8 +290,8 @@ def run_prefill(args, dist, torch, kda, synth, dev):
     d2h = hy.numel() * hy.element_size() + hs.numel() * hs.element_size()
 
     hbm, tc, peak_kind = measured_peaks()
-    nb = prefill_bytes(T, H, d)
-    top = max(PHASES, key=lambda ph: ms_phase[ph])
+    nb = prefill_bytes(T, H, d, fused_norm=fused_norm)
+    top = max(phases, key=lambda ph: ms_phase[ph])
     dominant = (top, nb[top], ms_phase[top])
     achieved = dominant[1] / (dominant[2] / 1e3) / 1e9
     res = {
@@ -298,7 +307,7 @@ def run_prefill(args, dist, torch, kda, synth, dev):
         'e2e': {'value': dist.world * T / (e2e_ms / 1e3), 'unit': 'tokens/s',
                 'h2d_bytes_per_step': h2d, 'd2h_bytes_per_step': d2h,
                 'ms_per_step': e2e_ms},
-        'gpu_launches': len(PHASES) * args.steps,
+        'gpu_launches': launches,
         'roofline': {'bound': 'hbm', 'kernel': dominant[0], 'achieved': achieved, 'peak': hbm,
                      'unit': 'GB/s', 'frac': achieved / hbm,
                      'traffic': profiled_traffic(dominant[0]),
@@ -307,7 +316,7 @@ def run_prefill(args, dist, torch, kda, synth, dev):
         'phase_roofline': {ph: {'algorithmic_bytes': nb[ph],
                                 'achieved_gbs': nb[ph] / (ms_phase[ph] / 1e3) / 1e9,
                                 'frac': nb[ph] / (ms_phase[ph] / 1e3) / 1e9 / hbm}
-                           for ph in PHASES},
+                           for ph in phases},
         'step_roofline': {'algorithmic_bytes': nb['layer'],
                           'achieved_gbs': nb['layer'] / (ms_step / 1e3) / 1e9,
                           'frac': nb['layer'] / (ms_step / 1e3) / 1e9 / hbm},

@@ -318,6 +318,14 @@ KDA_API int kda_selftest_wait_timeout(void* workspace, kda_stream_t stream);
  */
 KDA_API int kda_set_phase_events(void* const* events, int32_t n);
 
+/*
+ * kda_launch_count - measurement hook (the paper has no counterpart): the number
+ * of kernels the library has launched from THIS host thread since it was loaded
+ * (cumulative; take differences around the calls of interest).  Launches only:
+ * cudaMemsetAsync and other runtime calls are not counted.
+ */
+KDA_API long long kda_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

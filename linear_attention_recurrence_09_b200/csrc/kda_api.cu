@@ -246,6 +246,8 @@ int kda_layer_prefill(const kda_config* cfg, int32_t n_seqs, int32_t total_token
   return cuda_status(kda::launch_prefill(a, s));
 }
 
+long long kda_launch_count(void) { return kda::launch_counter(); }
+
 int kda_set_phase_events(void* const* events, int32_t n) {
   if (n < 0 || n > 3 || (n > 0 && events == nullptr)) return KDA_ERR_INVALID_ARG;
   kda::PhaseEvents& pe = kda::phase_events();

@@ -687,6 +687,7 @@ cudaError_t launch_intra_t(const PrefillArgs& a, cudaStream_t st) {
   PrefillArgs b = a;
   b.pf_stride = nsm;   // one CTA per SM (shared memory bound): the next wave is nsm ahead
   intra_chunk_sm100_kernel<FUSED><<<dim3(a.L.nslots, a.H), THREADS, SMEM_BYTES, st>>>(b);
+  ++launch_counter();
   return cudaGetLastError();
 }
 

@@ -106,6 +106,12 @@ cudaError_t launch_step(const StepArgs& a, cudaStream_t st);
 cudaError_t launch_rollback(const RollbackArgs& a, cudaStream_t st);
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st);
 
+// Kernels this host thread has launched through the library (cumulative).
+inline long long& launch_counter() {
+  static thread_local long long n = 0;
+  return n;
+}
+
 // Caller-owned events recorded on the prefill's stream after the intra-chunk,
 // inter-chunk and output-norm passes (null entries are skipped); per host thread.
 struct PhaseEvents {
@@ -117,7 +123,8 @@ bool sm100_intra_supported(const PrefillArgs& a);
 bool sm100_fused_supported(const PrefillArgs& a);
 cudaError_t launch_conv_commit(const PrepArgs& a, cudaStream_t st);
 cudaError_t launch_intra_sm100(const PrefillArgs& a, cudaStream_t st);
-cudaError_t launch_interchunk_sm100(const PrefillArgs& a, cudaStream_t st);
+// fused_norm: set when the pass also applied the gated RMSNorm and wrote y
+cudaError_t launch_interchunk_sm100(const PrefillArgs& a, cudaStream_t st, bool* fused_norm);
 cudaError_t launch_wait_timeout_selftest(void* workspace, cudaStream_t st);
 int prep_tile();
 int prep_kmax();

@@ -363,11 +363,13 @@ static cudaError_t launch_prefill_dc(const PrefillArgs& a, cudaStream_t st) {
     e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     k1<<<dim3(a.L.nslots, a.H), 256, sm, st>>>(a);
+    ++launch_counter();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (pe.ev[0] && (e = cudaEventRecord(pe.ev[0], st)) != cudaSuccess) return e;
+  bool fused_norm = false;
   if (sm100_interchunk_supported(a)) {
-    e = launch_interchunk_sm100(a, st);
+    e = launch_interchunk_sm100(a, st, &fused_norm);
     if (e != cudaSuccess) return e;
   } else {
     auto k2 = inter_chunk_kernel<T, D, C>;
@@ -375,13 +377,15 @@ static cudaError_t launch_prefill_dc(const PrefillArgs& a, cudaStream_t st) {
     e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     k2<<<dim3(D / P2_J, a.H, a.n_seqs), 256, sm, st>>>(a);
+    ++launch_counter();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (pe.ev[1] && (e = cudaEventRecord(pe.ev[1], st)) != cudaSuccess) return e;
-  if (a.total > 0) {
+  if (a.total > 0 && !fused_norm) {
     const size_t rows = (size_t)a.total * a.H;
     constexpr int RPC = norm_rows_per_cta<D>();
     gated_norm_kernel<T, D><<<(unsigned)((rows + RPC - 1) / RPC), 256, 0, st>>>(a);
+    ++launch_counter();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (pe.ev[2] && (e = cudaEventRecord(pe.ev[2], st)) != cudaSuccess) return e;

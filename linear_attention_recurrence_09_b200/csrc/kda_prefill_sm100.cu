@@ -13,7 +13,13 @@
 //                                                               K' stored token-major, read MN-major)
 //   MMA3   D1[64:128]   += M (64 x 64) . U                   (O = Q~ S + M U; A = [0 ; M])
 //   E2     S <- Diag(e^{G_C}) S + D2 in fp32 registers (one key row per thread) -> bf16 S^T
-//   E3     O rows of D1 -> o (fp32, workspace) for the gated RMSNorm pass
+//   E3     O rows of D1 -> y = O / rms(O) * w * sigmoid(g) (FUSE_NORM), else o (fp32,
+//          workspace) for the separate gated RMSNorm pass
+// With FUSE_NORM the 4 slice CTAs of a head form a thread-block cluster and two extra
+// warps per CTA run E3 off the chain: every token's sum of squares over its 128 value
+// columns is assembled from the 4 slices' partials, which each CTA sends into every
+// peer's shared memory with asynchronous remote stores that complete on the peer's
+// mbarrier (a 2-slot ring indexed by chunk parity).
 // Warp roles: warp 0 issues TMA (two smem stages, so chunk n+1 loads while n
 // computes; the U~ slice comes with them), warp 1 allocates TMEM and issues the
 // MMAs from one thread with precomputed descriptors, warps 2-9 run the
@@ -37,7 +43,10 @@ namespace {
 
 constexpr int D = 128, C = 64, J = 32, NSLICE = D / J;
 constexpr int NEPI = 8;                          // epilogue warps (2 per TMEM lane quarter)
-constexpr int THREADS = 64 + 32 * NEPI;
+constexpr int THREADS = 64 + 32 * NEPI;          // TMA, MMA and epilogue warps
+constexpr int NOUT = 2;                          // fused norm: O warps (TMEM lanes 64-127)
+template <bool FUSE_NORM>
+constexpr int threads_of() { return THREADS + (FUSE_NORM ? 32 * NOUT : 0); }
 constexpr int JH = J / 2;                        // value columns per epilogue thread
 constexpr uint32_t TMEM_COLS = 128;
 
@@ -52,20 +61,28 @@ constexpr uint32_t TX_BYTES = 4 * 8192 + 2 * 8192 + 8192 + UT_BYTES;   // W x2, 
 constexpr uint32_t OFF_S = NSTAGE * STAGE_BYTES;          // S^T: 2 K-blocks x 32 rows x 128 B
 constexpr uint32_t OFF_U = OFF_S + 2 * J * 128;           // U^T: 32 rows x 128 B
 constexpr uint32_t OFF_BAR = OFF_U + J * 128;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 128 + 1024;     // barriers + alignment slack
+constexpr uint32_t OFF_SSQ = OFF_BAR + 128;   // fused norm: [2 parities][4 slices][64 tokens] fp32
+constexpr uint32_t SMEM_BYTES = OFF_SSQ + 2 * NSLICE * C * 4 + 1024;   // + alignment slack
 
 // barrier slots (8 bytes each)
 enum { BAR_FULL0 = 0, BAR_FULL1, BAR_EMPTY0, BAR_EMPTY1, BAR_MMA1, BAR_MMA2, BAR_SREADY,
-       BAR_UREADY, BAR_COUNT };
+       BAR_UREADY, BAR_NFULL0, BAR_NFULL1, BAR_OFREE0, BAR_OFREE1, BAR_COUNT };
+static_assert(BAR_COUNT * 8 <= 128, "barrier slots");
+// norm partial exchange: every token's partial from every slice CTA, 4 bytes each
+constexpr uint32_t NORM_TX_BYTES = NSLICE * C * 4;
 
 struct TmaMaps {
   CUtensorMap W, Q, KT, M, Ut;
 };
 
+// sigmoid on the special-function unit (bf16 output: approximate exp and divide suffice)
+__device__ __forceinline__ float fast_sigmoid(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
+
 // K-major SW128 descriptor advanced by `bytes` (the 14-bit address field never carries)
 __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
-__global__ void __launch_bounds__(THREADS, 1)
+template <bool FUSE_NORM>
+__global__ void __launch_bounds__(threads_of<FUSE_NORM>(), 1)
 interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps maps) {
   extern __shared__ __align__(1024) unsigned char smraw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
@@ -94,12 +111,16 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
     mbar_init(bar(BAR_MMA2), 1);
     mbar_init(bar(BAR_SREADY), 32 * NEPI);
     mbar_init(bar(BAR_UREADY), 32 * NEPI / 2);
+    mbar_init(bar(BAR_NFULL0), 1);   // armed by one O thread per phase, filled by st.async
+    mbar_init(bar(BAR_NFULL1), 1);
+    mbar_init(bar(BAR_OFREE0), NOUT);
+    mbar_init(bar(BAR_OFREE1), NOUT);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   // rows 0-63 of every A3 tile are the zero half of [0 ; M]
   for (uint32_t st = 0; st < NSTAGE; ++st) {
     uint4* z = reinterpret_cast<uint4*>(sm + st * STAGE_BYTES + A1_BYTES + A2_BYTES);
-    for (int i = threadIdx.x; i < 8192 / 16; i += THREADS) z[i] = make_uint4(0, 0, 0, 0);
+    for (int i = threadIdx.x; i < 8192 / 16; i += threads_of<FUSE_NORM>()) z[i] = make_uint4(0, 0, 0, 0);
   }
   fence_proxy_async();
   if (warp == 1) {
@@ -111,6 +132,7 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
   }
   tc_fence_before();
   __syncthreads();
+  if (FUSE_NORM) cluster_sync_all();   // every peer's barriers exist before any remote arrival
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
   const uint32_t d1_tmem[2] = {tmem + 0, tmem + 32};   // double-buffered [W S ; O]
@@ -159,6 +181,10 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
         const int st = n & 1;
         if (!mbar_wait(bar(BAR_FULL0 + st), (n >> 1) & 1, &abort_flag)) break;
         if (!mbar_wait(bar(BAR_SREADY), n & 1, &abort_flag)) break;
+        // fused norm: the O warps have copied chunk n-2's O out of this D1 buffer
+        if (FUSE_NORM && n >= 2 &&
+            !mbar_wait(bar(BAR_OFREE0 + st), ((n >> 1) - 1) & 1, &abort_flag))
+          break;
         tc_fence_after();
         const uint64_t a1 = st ? dA1s1 : dA1s0;
         const uint32_t a2s = sbase + st * STAGE_BYTES + A1_BYTES;
@@ -187,7 +213,82 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
         }
       }
     }
-  } else {
+  } else if (FUSE_NORM && warp >= 2 + NEPI) {
+    // ---------------- O warps (fused norm), off the serial chain ----------------
+    // warp 10 / 11: TMEM lanes 64-95 / 96-127 = token rows r of the chunk, all 32 columns.
+    // Per chunk: copy O out of D1 and release the buffer to the MMA issuer, then
+    // y = O / sqrt(mean over the head's 128 columns of O^2 + eps) * w * sigmoid(g).
+    const int q = warp & 3;                 // 2 or 3
+    const int r = 32 * (q - 2) + lane;      // token row within the chunk
+    const int ow = q - 2;                   // which O warp
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    float* ssq = reinterpret_cast<float*>(sm + OFF_SSQ);
+    float nw[J];
+#pragma unroll
+    for (int c = 0; c < J; ++c) nw[c] = __ldg(a.norm_w + j0 + c);
+    // gate row of chunk n (token t0 + r, this slice's 32 columns), zero past the end
+    auto load_g = [&](int n, uint4 (&gv)[4]) {
+      const int t0 = start + n * C;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) gv[k] = make_uint4(0, 0, 0, 0);
+      if (n < nch && r < min(C, end - t0)) {
+        const uint4* gp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.g) +
+                                                         ((size_t)(t0 + r) * H + h) * D + j0);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) gv[k] = gp[k];
+      }
+    };
+    uint4 graw[4], gnext[4];
+    load_g(0, graw);
+    for (int n = 0; n < nch; ++n) {
+      const int st = n & 1, p = n & 1;
+      const int t0 = start + n * C;
+      const int L = min(C, end - t0);
+      const size_t yo = ((size_t)(t0 + r) * H + h) * D + j0;
+      load_g(n + 1, gnext);   // one chunk ahead: in flight through this chunk's work
+      if (!mbar_wait_warp(bar(BAR_EMPTY0 + st), (n >> 1) & 1, &abort_flag)) break;
+      tc_fence_after();
+      float o[J];
+      tmem_ld16(d1_tmem[st] + lane_off, *reinterpret_cast<float(*)[16]>(o));
+      tmem_ld16(d1_tmem[st] + lane_off + 16, *reinterpret_cast<float(*)[16]>(o + 16));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_OFREE0 + st));
+      float part = 0.f;
+#pragma unroll
+      for (int c = 0; c < J; ++c) part = fmaf(o[c], o[c], part);
+      // Token r's partial from slice CTA `rank` lands in slot [p][rank][r] of every CTA.  A
+      // slot of parity p is rewritten (chunk n) only after this warp's producer passed the
+      // full barrier of chunk n-1, which every consumer warp reaches only after reading
+      // chunk n-2: two slots need no separate "free" handshake.
+      if (ow == 0 && lane == 0) mbar_expect_tx(bar(BAR_NFULL0 + p), NORM_TX_BYTES);
+      const uint32_t slot = smem_u32(ssq + (p * NSLICE + blockIdx.x) * C + r);
+#pragma unroll
+      for (int dst = 0; dst < NSLICE; ++dst)
+        st_async_cluster(cluster_map(slot, dst), part, cluster_map(bar(BAR_NFULL0 + p), dst));
+      if (!mbar_wait_warp(bar(BAR_NFULL0 + p), (n >> 1) & 1, &abort_flag)) break;
+      float tot = 0.f;
+#pragma unroll
+      for (int k = 0; k < NSLICE; ++k) tot += ssq[(p * NSLICE + k) * C + r];
+      if (r < L) {
+        const float rstd = rsqrtf(tot * (1.0f / D) + a.norm_eps);
+        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(graw);
+        uint4 out[4];
+        __nv_bfloat162* y2 = reinterpret_cast<__nv_bfloat162*>(out);
+#pragma unroll
+        for (int c = 0; c < J; c += 2) {
+          const float2 gv = __bfloat1622float2(g2[c / 2]);
+          y2[c / 2] = __floats2bfloat162_rn(o[c] * rstd * nw[c] * fast_sigmoid(gv.x),
+                                            o[c + 1] * rstd * nw[c + 1] * fast_sigmoid(gv.y));
+        }
+        uint4* yp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.y) + yo);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) yp[k] = out[k];
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) graw[k] = gnext[k];
+    }
+  } else if (warp < 2 + NEPI) {
     // ---------------- epilogue warps 2..9 ----------------
     const int q = warp & 3;                 // TMEM lane quarter
     const int half = (warp - 2) / 4;        // which 16 of the slice's 32 value columns
@@ -267,7 +368,7 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
         for (int m = 0; m < JH; ++m) S[m] = fmaf(gc, S[m], dv[m]);
       }
       write_state();
-      if (q >= 2) {
+      if (!FUSE_NORM && q >= 2) {
         // E3 (off the chain): O rows (TMEM lanes 64-127) once MMA3 has retired
         if (!mbar_wait_warp(bar(BAR_EMPTY0 + st), (n >> 1) & 1, &abort_flag)) break;
         tc_fence_after();
@@ -299,6 +400,8 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
                  "r"(TMEM_COLS)
                  : "memory");
   }
+  // no CTA leaves while a peer may still write its shared memory or arrive at its barriers
+  if (FUSE_NORM) cluster_sync_all();
 }
 
 // Self-test of the bounded wait: one warp waits on an mbarrier that nothing
@@ -364,8 +467,43 @@ bool sm100_interchunk_supported(const PrefillArgs& a) {
   return a.bf16 && a.D == D && a.C == C;
 }
 
-cudaError_t launch_interchunk_sm100(const PrefillArgs& a, cudaStream_t st) {
+// the fused norm needs the 4-CTA clusters of all heads (and sequences) resident in one
+// wave whenever the plain launch would be; decided once per device
+static bool fuse_norm_fits(int clusters) {
+  static int max_clusters[64];
+  static bool known[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!known[dev]) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(NSLICE, 64, 1);
+    cfg.blockDim = dim3(threads_of<true>(), 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = NSLICE;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaFuncSetAttribute(interchunk_sm100_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&n, interchunk_sm100_kernel<true>, &cfg) != cudaSuccess)
+      n = 0;
+    cudaGetLastError();
+    max_clusters[dev] = n;
+    known[dev] = true;
+  }
+  int nsm = 0;
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int plain_wave = nsm / NSLICE;   // heads x sequences one plain wave holds
+  return max_clusters[dev] >= (clusters < plain_wave ? clusters : plain_wave);
+}
+
+cudaError_t launch_interchunk_sm100(const PrefillArgs& a, cudaStream_t st, bool* fused_norm) {
   static_assert(NSLICE * J == D, "slices must cover the value axis");
+  *fused_norm = false;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   TmaMaps maps;
@@ -376,10 +514,35 @@ cudaError_t launch_interchunk_sm100(const PrefillArgs& a, cudaStream_t st) {
       !make_map(enc, &maps.M, a.ws + a.L.M, tiles * C, C, 64) ||
       !make_map(enc, &maps.Ut, a.ws + a.L.Ut, tiles * C, D, 64, J, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(interchunk_sm100_kernel,
+  const dim3 grid(NSLICE, a.H, a.n_seqs);
+  if (a.y != nullptr && a.total > 0 && fuse_norm_fits(a.H * a.n_seqs)) {
+    cudaError_t e = cudaFuncSetAttribute(interchunk_sm100_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads_of<true>(), 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = NSLICE;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, interchunk_sm100_kernel<true>, a, maps);
+    if (e == cudaSuccess) {
+      *fused_norm = true;
+      ++launch_counter();
+    }
+    return e;
+  }
+  cudaError_t e = cudaFuncSetAttribute(interchunk_sm100_kernel<false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  interchunk_sm100_kernel<<<dim3(NSLICE, a.H, a.n_seqs), THREADS, SMEM_BYTES, st>>>(a, maps);
+  interchunk_sm100_kernel<false><<<grid, threads_of<false>(), SMEM_BYTES, st>>>(a, maps);
+  ++launch_counter();
   return cudaGetLastError();
 }
 

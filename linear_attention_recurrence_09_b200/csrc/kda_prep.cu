@@ -205,10 +205,12 @@ static cudaError_t launch_prep_k(const PrepArgs& a, cudaStream_t st) {
   constexpr int HPB = PREP_THREADS / (3 * D / 4);
   dim3 grid(num_slots(a.total, a.n_seqs, PREP_TILE), (a.H + HPB - 1) / HPB);
   prep_kernel<T, D, K><<<grid, PREP_THREADS, 0, st>>>(a);
+  ++launch_counter();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.mode == 0 && a.conv_state != nullptr && K > 1 && !a.commit_in_kernel) {
     conv_commit_kernel<T><<<dim3(a.n_seqs, a.H), 128, 0, st>>>(a);
+    ++launch_counter();
     e = cudaGetLastError();
   }
   return e;
@@ -244,6 +246,7 @@ cudaError_t launch_conv_commit(const PrepArgs& a, cudaStream_t st) {
   if (a.conv_state == nullptr || a.K < 2 || a.n_seqs == 0) return cudaSuccess;
   if (a.bf16) conv_commit_kernel<__nv_bfloat16><<<dim3(a.n_seqs, a.H), 128, 0, st>>>(a);
   else conv_commit_kernel<float><<<dim3(a.n_seqs, a.H), 128, 0, st>>>(a);
+  ++launch_counter();
   return cudaGetLastError();
 }
 

@@ -65,6 +65,59 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
   }
 }
 
+// ---- thread-block clusters: distributed shared memory and remote mbarrier arrivals ----
+// shared::cluster address of the variable at CTA-local shared address `saddr` in CTA `rank`
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster(uint32_t caddr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(caddr), "f"(v) : "memory");
+}
+// asynchronous 4-byte store into CTA-shared memory of any CTA of the cluster; on arrival it
+// counts 4 bytes off the transaction count of the mbarrier at `cbar` in that CTA
+__device__ __forceinline__ void st_async_cluster(uint32_t caddr, float v, uint32_t cbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];" ::"r"(
+                   caddr),
+               "f"(v), "r"(cbar)
+               : "memory");
+}
+// arrive (release, cluster scope) on an mbarrier of any CTA of the cluster
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// warp-uniform bounded wait on a local mbarrier that other CTAs of the cluster arrive at
+__device__ __forceinline__ bool mbar_wait_cluster_warp(uint32_t bar, uint32_t parity,
+                                                       volatile int* abort_flag) {
+  const long long t0 = clock64();
+  while (true) {
+    const bool done = mbar_try_cluster(bar, parity);
+    if (__all_sync(0xffffffffu, done)) return true;
+    const bool give_up = (*abort_flag != 0) || (clock64() - t0 > WAIT_LIMIT_CYCLES);
+    if (__any_sync(0xffffffffu, give_up)) {
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+// every thread of every CTA of the cluster (used once after set-up and once before exit)
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

@@ -153,6 +153,7 @@ static cudaError_t launch_step_t(const StepArgs& a, cudaStream_t st) {
     case 128: step_kernel<T, 128><<<grid, StepShape<128>::THREADS, 0, st>>>(a); break;
     default: return cudaErrorInvalidValue;
   }
+  ++launch_counter();
   return cudaGetLastError();
 }
 
@@ -190,6 +191,7 @@ cudaError_t launch_rollback(const RollbackArgs& a, cudaStream_t st) {
   dim3 grid(a.H, a.B);
   if (a.bf16) rollback_kernel<uint16_t><<<grid, 256, 0, st>>>(a);
   else rollback_kernel<uint32_t><<<grid, 256, 0, st>>>(a);
+  ++launch_counter();
   return cudaGetLastError();
 }
 

@@ -35,7 +35,7 @@ ENTRY_POINTS = ('kda_status_string', 'kda_abi_version', 'kda_prep',
                 'kda_prefill_workspace_size', 'kda_prefill', 'kda_decode', 'kda_verify',
                 'kda_rollback', 'kda_workspace_status', 'kda_selftest_wait_timeout',
                 'kda_prefill_noalloc', 'kda_layer_prefill_workspace_size', 'kda_layer_prefill',
-                'kda_set_phase_events')
+                'kda_set_phase_events', 'kda_launch_count')
 
 
 class KdaError(RuntimeError):
@@ -118,6 +118,8 @@ def lib() -> ctypes.CDLL:
         L.kda_layer_prefill.argtypes = [ctypes.POINTER(CConfig), _I, _I, _P, _I, _P, _P, _P, _P,
                                         _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
                                         ctypes.c_size_t, _P]
+        L.kda_launch_count.restype = ctypes.c_longlong
+        L.kda_launch_count.argtypes = []
         L.kda_set_phase_events.restype = ctypes.c_int
         L.kda_set_phase_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), _I]
         L.kda_prefill_noalloc.restype = ctypes.c_int
@@ -347,6 +349,11 @@ def kda_selftest_wait_timeout(workspace, stream=None):
     """Run the bounded-wait self-test on ``workspace`` (enqueue only)."""
     _check(lib().kda_selftest_wait_timeout(_ptr(workspace, None, 'workspace'), _stream(stream)),
            'kda_selftest_wait_timeout')
+
+
+def kda_launch_count() -> int:
+    """Kernels the library launched from this thread so far (cumulative)."""
+    return int(lib().kda_launch_count())
 
 
 def kda_set_phase_events(events=()):

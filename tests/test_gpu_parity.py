@@ -291,3 +291,22 @@ def test_bounded_wait_times_out_and_context_survives():
     kda.layer_prefill(cfg, {k: v.cuda() for k, v in P.items()},
                       {k: v.cuda() for k, v in A.items()}, workspace=w2)
     assert kda.kda_workspace_status(w2) == kda.KDA_OK
+
+
+def test_layer_prefill_launches_and_fused_norm():
+    """bf16, d = 128, chunk 64, conv 4: prep runs inside the intra-chunk pass and the gated
+    norm inside the inter-chunk pass, so one layer call is two kernels (plus the conv-state
+    commit when a conv state is given); the result is the oracle's either way."""
+    cfg, P, A, S0, hist = make_case(21, [300, 64], 4, 128, 4, torch.bfloat16, state_var=0.01,
+                                    conv_hist=True, chunk=64)
+    Pd = {k: v.cuda() for k, v in P.items()}
+    Ad = {k: v.cuda() for k, v in A.items()}
+    n0 = kda.kda_launch_count()
+    kda.layer_prefill(cfg, Pd, Ad, state_out=torch.empty(2, 4, 128, 128, device='cuda'))
+    assert kda.kda_launch_count() - n0 == 2
+    n0 = kda.kda_launch_count()
+    y, s_out, cs, _ = gpu_layer(cfg, P, A, S0, hist, fused=True)
+    assert kda.kda_launch_count() - n0 == 3
+    ref = oracle_layer(cfg, P, A, S0, hist)
+    assert rel_err(np64(y), ref['y']) <= 1e-2
+    assert rel_err(np64(s_out), ref['state']) <= 1e-2
