@@ -326,6 +326,13 @@ KDA_API int kda_set_phase_events(void* const* events, int32_t n);
  */
 KDA_API long long kda_launch_count(void);
 
+/*
+ * kda_last_cuda_error - the CUDA runtime's message for the error behind the most
+ * recent KDA_ERR_CUDA returned to THIS host thread ("no error" if there was none).
+ * Static string; do not free.
+ */
+KDA_API const char* kda_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif

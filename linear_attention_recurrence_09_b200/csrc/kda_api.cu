@@ -48,7 +48,15 @@ int check_pool(const int32_t* slots, int32_t pool_size, int32_t n) {
   return KDA_OK;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+cudaError_t& last_cuda_error() {
+  static thread_local cudaError_t e = cudaSuccess;
+  return e;
+}
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return KDA_OK;
+  last_cuda_error() = e;
+  return KDA_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -247,6 +255,8 @@ int kda_layer_prefill(const kda_config* cfg, int32_t n_seqs, int32_t total_token
 }
 
 long long kda_launch_count(void) { return kda::launch_counter(); }
+
+const char* kda_last_cuda_error(void) { return cudaGetErrorString(last_cuda_error()); }
 
 int kda_set_phase_events(void* const* events, int32_t n) {
   if (n < 0 || n > 3 || (n > 0 && events == nullptr)) return KDA_ERR_INVALID_ARG;

@@ -98,10 +98,6 @@ __device__ __forceinline__ float rsqrta(float x) {
 // sigmoid of z given z2 = z log2(e); 1 / (1 + inf) = 0 keeps the saturated end exact
 __device__ __forceinline__ float sigmoid2(float z2) { return rcpa(1.f + ex2a(-z2)); }
 __device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
-// start pulling `bytes` (a multiple of 16, 16-byte aligned) at p into L2
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
 
 // x = hi + lo with hi, lo tf32 (round to nearest)
 __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
@@ -200,18 +196,6 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   if (FUSED) {
     A_log_h = __ldg(a.A_log + h);
     dtb = *reinterpret_cast<const float2*>(a.dt_bias + (size_t)h * D + cp);
-  }
-
-  // this tile's rows start streaming into L2 while the gates are computed
-  if (tid < L) {
-    const size_t row = (size_t)(t0 + tid) * H + h;
-    if (FUSED) {
-      prefetch_l2(static_cast<const __nv_bfloat16*>(a.x) + row * 3 * D, 3 * D * 2);
-    } else {
-      prefetch_l2(a.q + row * D, D * 4);
-      prefetch_l2(a.k + row * D, D * 4);
-      prefetch_l2(a.v + row * D, D * 4);
-    }
   }
 
   if (tid == 0) {
@@ -509,21 +493,31 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   __syncthreads();   // G is dead now: A takes its place (only entries i < r are ever read)
   // D[m][n]: rows 0-31 = keys 0-31 vs cols 0-31 (keys) / 32-63 (queries) of rows 0-31;
   // rows 32-95 = keys 0-63 vs cols 64-95 (keys) / 96-127 (queries) of rows 32-63
-  if (ok && (warp == 0 || warp == 5 || warp == 6)) {
+  // Warps of lane quarters 0-2 each read one 32-column group: warp w < 4 the keys (A),
+  // warp w + 4 the queries (M); quarter 3 (rows 96-127 of D) holds nothing and writes the
+  // zero upper-right block of M.
+  if (ok && (warp & 3) < 3) {
     const int q = warp & 3;
-    const int i = (warp == 6) ? 32 + lane : lane;
-    const int rbase = (warp == 0) ? 0 : 32;
-    const uint32_t col = (warp == 0) ? 0u : 64u;
-    float av[32], mv[32];
-    tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + col, av);
-    tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + col + 32, mv);
+    const int i = (q == 2) ? 32 + lane : lane;          // key index of this TMEM lane
+    const int rbase = (q == 0) ? 0 : 32;                 // first row r of the group
+    const bool keys = warp < 4;
+    const uint32_t col = ((q == 0) ? 0u : 64u) + (keys ? 0u : 32u);
+    float v[32];
+    tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + col, v);
+    if (keys) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int r = rbase + j;
-      if (i < r) Af[r * AF_LD + i] = bs[r] * av[j];
-      Mo[r * C + i] = __float2bfloat16_rn(i <= r ? mv[j] : 0.f);
+      for (int j = 0; j < 32; ++j) {
+        const int r = rbase + j;
+        if (i < r) Af[r * AF_LD + i] = bs[r] * v[j];
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int r = rbase + j;
+        Mo[r * C + i] = __float2bfloat16_rn(i <= r ? v[j] : 0.f);
+      }
     }
-  } else if (warp == 7) {
+  } else if (warp == 3) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) Mo[j * C + 32 + lane] = __float2bfloat16_rn(0.f);
   }

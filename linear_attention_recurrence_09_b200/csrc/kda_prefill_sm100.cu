@@ -61,13 +61,14 @@ constexpr uint32_t TX_BYTES = 4 * 8192 + 2 * 8192 + 8192 + UT_BYTES;   // W x2, 
 constexpr uint32_t OFF_S = NSTAGE * STAGE_BYTES;          // S^T: 2 K-blocks x 32 rows x 128 B
 constexpr uint32_t OFF_U = OFF_S + 2 * J * 128;           // U^T: 32 rows x 128 B
 constexpr uint32_t OFF_BAR = OFF_U + J * 128;
-constexpr uint32_t OFF_SSQ = OFF_BAR + 128;   // fused norm: [2 parities][4 slices][64 tokens] fp32
+constexpr uint32_t OFF_SSQ = OFF_BAR + 256;   // fused norm: [2 parities][4 slices][64 tokens] fp32
 constexpr uint32_t SMEM_BYTES = OFF_SSQ + 2 * NSLICE * C * 4 + 1024;   // + alignment slack
 
 // barrier slots (8 bytes each)
 enum { BAR_FULL0 = 0, BAR_FULL1, BAR_EMPTY0, BAR_EMPTY1, BAR_MMA1, BAR_MMA2, BAR_SREADY,
-       BAR_UREADY, BAR_NFULL0, BAR_NFULL1, BAR_OFREE0, BAR_OFREE1, BAR_COUNT };
-static_assert(BAR_COUNT * 8 <= 128, "barrier slots");
+       BAR_UREADY, BAR_NFULL0, BAR_NFULL1, BAR_OFREE0, BAR_OFREE1, BAR_OFREE2, BAR_ODONE0,
+       BAR_ODONE1, BAR_ODONE2, BAR_COUNT };
+static_assert(BAR_COUNT * 8 <= 256, "barrier slots");
 // norm partial exchange: every token's partial from every slice CTA, 4 bytes each
 constexpr uint32_t NORM_TX_BYTES = NSLICE * C * 4;
 
@@ -115,6 +116,10 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
     mbar_init(bar(BAR_NFULL1), 1);
     mbar_init(bar(BAR_OFREE0), NOUT);
     mbar_init(bar(BAR_OFREE1), NOUT);
+    mbar_init(bar(BAR_OFREE2), NOUT);
+    mbar_init(bar(BAR_ODONE0), 1);
+    mbar_init(bar(BAR_ODONE1), 1);
+    mbar_init(bar(BAR_ODONE2), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   // rows 0-63 of every A3 tile are the zero half of [0 ; M]
@@ -135,7 +140,11 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
   if (FUSE_NORM) cluster_sync_all();   // every peer's barriers exist before any remote arrival
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
-  const uint32_t d1_tmem[2] = {tmem + 0, tmem + 32};   // double-buffered [W S ; O]
+  // [W S ; O] of chunk n in D1 buffer n % 3 (three, so the O readers have slack); K'^T U in D2
+  auto d1_of = [&](int n) -> uint32_t {
+    const int b = n % 3;
+    return tmem + (b == 2 ? 96u : 32u * (uint32_t)b);
+  };
   const uint32_t d2_tmem = tmem + 64;
   int* status = reinterpret_cast<int*>(a.ws + a.L.status);
 
@@ -181,15 +190,16 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
         const int st = n & 1;
         if (!mbar_wait(bar(BAR_FULL0 + st), (n >> 1) & 1, &abort_flag)) break;
         if (!mbar_wait(bar(BAR_SREADY), n & 1, &abort_flag)) break;
-        // fused norm: the O warps have copied chunk n-2's O out of this D1 buffer
-        if (FUSE_NORM && n >= 2 &&
-            !mbar_wait(bar(BAR_OFREE0 + st), ((n >> 1) - 1) & 1, &abort_flag))
+        const int db = n % 3;
+        // fused norm: the O warps have copied chunk n-3's O out of this D1 buffer
+        if (FUSE_NORM && n >= 3 &&
+            !mbar_wait(bar(BAR_OFREE0 + db), ((n / 3) - 1) & 1, &abort_flag))
           break;
         tc_fence_after();
         const uint64_t a1 = st ? dA1s1 : dA1s0;
         const uint32_t a2s = sbase + st * STAGE_BYTES + A1_BYTES;
         const uint64_t a3 = desc_add(a1, A1_BYTES + A2_BYTES);
-        const uint32_t d1 = st ? d1_tmem[1] : d1_tmem[0];
+        const uint32_t d1 = d1_of(n);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           umma(d1, desc_add(a1, (k >> 2) * 16384 + (k & 3) * 32),
@@ -206,6 +216,9 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
         for (int k = 0; k < 4; ++k)
           umma(d1, desc_add(a3, k * 32), desc_add(dU, k * 32), id, 1);
         umma_commit(bar(BAR_EMPTY0 + st));
+        // O of chunk n complete in D1 buffer n % 3 (its own barrier: the O warps may lag
+        // behind the stage barrier by more than one phase, never behind this one)
+        if (FUSE_NORM) umma_commit(bar(BAR_ODONE0 + db));
       }
       if (abort_flag && last >= 0) {  // let the issued MMAs retire before TMEM is freed
         const long long t0 = clock64();
@@ -241,19 +254,19 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
     uint4 graw[4], gnext[4];
     load_g(0, graw);
     for (int n = 0; n < nch; ++n) {
-      const int st = n & 1, p = n & 1;
+      const int p = n & 1;
       const int t0 = start + n * C;
       const int L = min(C, end - t0);
       const size_t yo = ((size_t)(t0 + r) * H + h) * D + j0;
       load_g(n + 1, gnext);   // one chunk ahead: in flight through this chunk's work
-      if (!mbar_wait_warp(bar(BAR_EMPTY0 + st), (n >> 1) & 1, &abort_flag)) break;
+      if (!mbar_wait_warp(bar(BAR_ODONE0 + n % 3), (n / 3) & 1, &abort_flag)) break;
       tc_fence_after();
       float o[J];
-      tmem_ld16(d1_tmem[st] + lane_off, *reinterpret_cast<float(*)[16]>(o));
-      tmem_ld16(d1_tmem[st] + lane_off + 16, *reinterpret_cast<float(*)[16]>(o + 16));
+      tmem_ld16(d1_of(n) + lane_off, *reinterpret_cast<float(*)[16]>(o));
+      tmem_ld16(d1_of(n) + lane_off + 16, *reinterpret_cast<float(*)[16]>(o + 16));
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_OFREE0 + st));
+      if (lane == 0) mbar_arrive(bar(BAR_OFREE0 + n % 3));
       float part = 0.f;
 #pragma unroll
       for (int c = 0; c < J; ++c) part = fmaf(o[c], o[c], part);
@@ -335,7 +348,7 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
         if (!mbar_wait_warp(bar(BAR_MMA1), n & 1, &abort_flag)) break;
         tc_fence_after();
         float ws[JH];
-        tmem_ld16(d1_tmem[st] + lane_off + cb, ws);
+        tmem_ld16(d1_of(n) + lane_off + cb, ws);
         const __nv_bfloat16* ut =
             reinterpret_cast<const __nv_bfloat16*>(sm + st * STAGE_BYTES + A1_BYTES + A2_BYTES +
                                                    A3_BYTES) + i * J + cb;
@@ -373,7 +386,7 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
         if (!mbar_wait_warp(bar(BAR_EMPTY0 + st), (n >> 1) & 1, &abort_flag)) break;
         tc_fence_after();
         float o[JH];
-        tmem_ld16(d1_tmem[st] + lane_off + cb, o);
+        tmem_ld16(d1_of(n) + lane_off + cb, o);
         const int r = i - 64;
         if (r < L) {
           float* op = og + ((size_t)(t0 + r) * H + h) * D + j0 + cb;

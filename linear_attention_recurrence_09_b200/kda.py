@@ -35,13 +35,16 @@ ENTRY_POINTS = ('kda_status_string', 'kda_abi_version', 'kda_prep',
                 'kda_prefill_workspace_size', 'kda_prefill', 'kda_decode', 'kda_verify',
                 'kda_rollback', 'kda_workspace_status', 'kda_selftest_wait_timeout',
                 'kda_prefill_noalloc', 'kda_layer_prefill_workspace_size', 'kda_layer_prefill',
-                'kda_set_phase_events', 'kda_launch_count')
+                'kda_set_phase_events', 'kda_launch_count', 'kda_last_cuda_error')
 
 
 class KdaError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
-        super().__init__(f'{where}: {kda_status_string(status)} ({status})')
+        msg = f'{where}: {kda_status_string(status)} ({status})'
+        if status == KDA_ERR_CUDA:
+            msg += ': ' + lib().kda_last_cuda_error().decode()
+        super().__init__(msg)
 
 
 class CConfig(ctypes.Structure):
@@ -118,6 +121,8 @@ def lib() -> ctypes.CDLL:
         L.kda_layer_prefill.argtypes = [ctypes.POINTER(CConfig), _I, _I, _P, _I, _P, _P, _P, _P,
                                         _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
                                         ctypes.c_size_t, _P]
+        L.kda_last_cuda_error.restype = ctypes.c_char_p
+        L.kda_last_cuda_error.argtypes = []
         L.kda_launch_count.restype = ctypes.c_longlong
         L.kda_launch_count.argtypes = []
         L.kda_set_phase_events.restype = ctypes.c_int
