@@ -25,10 +25,11 @@
 //     into a bf16 high part and the bf16 rounding of the remainder (hi + lo), and
 //     W accumulates hi.hi + hi.lo + lo.hi, U~ accumulates V.hi + V.lo: the
 //     rounding of T and K e^G was the largest term left in the error budget.
-// Q~ = q_scale Q e^G, K' = K e^{G_C - G} and e^{G_C} are elementwise.  Each warp
-// walks 8 consecutive token rows with lane l owning channels 4l..4l+3 of q, k
-// and v, so the per-token L2 norms are full-warp shuffles and the conv keeps its
-// window of K-1 previous rows in registers.
+// Q~ = q_scale Q e^G, K' = K e^{G_C - G} and e^{G_C} are elementwise.  16 warps: warps
+// w and w + 8 walk token rows 8(w%8)..8(w%8)+7 in pairs, each owning 64 of the 128
+// channels of q, k and v (two per lane); the per-token L2 norms are warp shuffles plus
+// one exchange with the partner warp per row pair, and the conv keeps its window of
+// K-1 previous rows in registers.
 #include <type_traits>
 
 #include "kda_common.cuh"
@@ -39,7 +40,7 @@ namespace kda {
 namespace {
 
 constexpr int D = 128, C = 64;
-constexpr int THREADS = 256;
+constexpr int THREADS = 512;   // 16 warps: two per group of 8 token rows (one per channel half)
 constexpr int KC = 4;         // conv taps of the fused path
 constexpr uint32_t TMEM_COLS = 128;
 
@@ -70,8 +71,16 @@ __device__ __forceinline__ uint32_t mn_off(int t, int c) {     // bf16 MN-major 
                     (((((c & 63) >> 3) ^ row) & 7) << 4) + (c & 7) * 2);
 }
 
-__device__ __forceinline__ void st_tf32x4(unsigned char* p, float a, float b, float c, float d) {
-  *reinterpret_cast<float4*>(p) = make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
+// fp32 -> nearest tf32 (10 mantissa bits, ties away from zero: the rounding of
+// cvt.rna.tf32.f32) with two integer operations on the bit pattern; finite inputs only
+__device__ __forceinline__ float tf32_rna(float x) {
+  return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xffffe000u);
+}
+__device__ __forceinline__ void st_tf32x2(unsigned char* p, float a, float b) {
+  *reinterpret_cast<float2*>(p) = make_float2(tf32_rna(a), tf32_rna(b));
+}
+__device__ __forceinline__ void st_bf16x2(void* p, float a, float b) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
 }
 __device__ __forceinline__ void st_bf16x4(unsigned char* p, float a, float b, float c, float d) {
   st4(reinterpret_cast<__nv_bfloat16*>(p), make_float4(a, b, c, d));
@@ -97,7 +106,6 @@ __device__ __forceinline__ float rsqrta(float x) {
 }
 // sigmoid of z given z2 = z log2(e); 1 / (1 + inf) = 0 keeps the saturated end exact
 __device__ __forceinline__ float sigmoid2(float z2) { return rcpa(1.f + ex2a(-z2)); }
-__device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
 // x = hi + lo with hi, lo tf32 (round to nearest)
 __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
@@ -133,11 +141,10 @@ __device__ __forceinline__ float sum3(const float (&d)[3][4], int i) {
   return d[0][i] + (d[1][i] + d[2][i]);
 }
 
-// four channels as loaded -> fp32 (bf16 widens by a 16-bit shift)
-__device__ __forceinline__ float4 to_f4(float4 v) { return v; }
-__device__ __forceinline__ float4 to_f4(uint2 v) {
-  return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
-                     __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+// two channels as loaded -> fp32 (bf16 widens by a 16-bit shift)
+__device__ __forceinline__ float2 to_f2(float2 v) { return v; }
+__device__ __forceinline__ float2 to_f2(uint32_t v) {
+  return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -153,7 +160,8 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sb = smem_u32(sm);
   __shared__ float bs[C];
-  __shared__ float qsum[4][D];   // per-quarter totals of the log decay
+  __shared__ float qsum[8][D];   // per-row-group totals of the log decay
+  __shared__ float4 pnorm[8][2][2];   // q/k sums of squares of a row pair: [group][parity][half]
   __shared__ uint32_t tmem_holder;
   __shared__ __align__(8) uint64_t bar_mma;
   __shared__ volatile int abort_flag;
@@ -177,12 +185,12 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   float* Af = G;                                  // [64][AF_LD], after the gram
   float* Xs = reinterpret_cast<float*>(sm + OFF_XS);
 
-  // gate inputs first (the gate pass waits on them): channels 2p, 2p+1 of rows 16q..16q+15
+  // gate inputs first (the gate pass waits on them): channels 2p, 2p+1 of rows 8q..8q+7
   const int cp = 2 * (tid & 63), qr = tid >> 6;
-  float g0[16], g1[16];
+  float g0[8], g1[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int r = 16 * qr + i;
+  for (int i = 0; i < 8; ++i) {
+    const int r = 8 * qr + i;
     float2 v = make_float2(0.f, 0.f);
     if (r < L) {
       const size_t idx = ((size_t)(t0 + r) * H + h) * D + cp;
@@ -212,25 +220,26 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   }
 
   // ---- inputs of the token-row pass, issued now so their latency overlaps the gates
-  // (kept as loaded, converted after): lane l owns channels 4l..4l+3 of q, k and v in
-  // rows 8w..8w+7 of warp w ----
-  const int c4 = 4 * lane;
+  // (kept as loaded, converted after).  Warps w and w + 8 share token rows 8(w%8)..+7;
+  // warp w < 8 holds channels 0-63 and w >= 8 channels 64-127 of q, k and v, two per lane.
+  const int pr = warp & 7, hh = warp >> 3;
+  const int c2 = 64 * hh + 2 * lane;
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x);
   const __nv_bfloat16* cs = static_cast<const __nv_bfloat16*>(a.conv_state);
-  using RawT = typename std::conditional<FUSED, uint2, float4>::type;   // 4 channels as loaded
+  using RawT = typename std::conditional<FUSED, uint32_t, float2>::type;   // 2 channels as loaded
   // fused prep state: conv taps (one float4 per channel) and the K-1 previous pre-conv rows
-  float4 cw[3][4];
+  float4 cw[3][2];
   RawT winr[KC - 1][3];
   if (FUSED) {
 #pragma unroll
     for (int sgm = 0; sgm < 3; ++sgm)
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+      for (int j = 0; j < 2; ++j)
         cw[sgm][j] = __ldg(reinterpret_cast<const float4*>(
-            a.conv_w + ((size_t)h * 3 * D + sgm * D + c4 + j) * KC));
+            a.conv_w + ((size_t)h * 3 * D + sgm * D + c2 + j) * KC));
 #pragma unroll
     for (int m = 0; m < KC - 1; ++m) {
-      const int tok = t0 + 8 * warp - (KC - 1) + m;
+      const int tok = t0 + 8 * pr - (KC - 1) + m;
       const __nv_bfloat16* src = nullptr;
       if (tok >= tr.start && tok < tr.end)   // rows past the end only feed padded rows
         src = x + ((size_t)tok * H + h) * 3 * D;
@@ -238,33 +247,33 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
         src = cs + (((size_t)prow * (KC - 1) + (KC - 1 + tok - tr.start)) * H + h) * 3 * D;
 #pragma unroll
       for (int sgm = 0; sgm < 3; ++sgm)
-        winr[m][sgm] = src ? *reinterpret_cast<const RawT*>(src + sgm * D + c4) : RawT{};
+        winr[m][sgm] = src ? *reinterpret_cast<const RawT*>(src + sgm * D + c2) : RawT{};
     }
   }
-  // row r's q, k, v channels c4..c4+3 (pre-conv x when fused); zero past the sequence end
+  // row r's q, k, v channels c2, c2+1 (pre-conv x when fused); zero past the sequence end
   auto load_row = [&](int r, RawT& iq, RawT& ik, RawT& iv) {
     iq = ik = iv = RawT{};
     if (r < L) {
       if (FUSED) {
         const __nv_bfloat16* xp = x + ((size_t)(t0 + r) * H + h) * 3 * D;
-        iq = *reinterpret_cast<const RawT*>(xp + c4);
-        ik = *reinterpret_cast<const RawT*>(xp + D + c4);
-        iv = *reinterpret_cast<const RawT*>(xp + 2 * D + c4);
+        iq = *reinterpret_cast<const RawT*>(xp + c2);
+        ik = *reinterpret_cast<const RawT*>(xp + D + c2);
+        iv = *reinterpret_cast<const RawT*>(xp + 2 * D + c2);
       } else {
-        const size_t idx = ((size_t)(t0 + r) * H + h) * D + c4;
+        const size_t idx = ((size_t)(t0 + r) * H + h) * D + c2;
         iq = *reinterpret_cast<const RawT*>(a.q + idx);
         ik = *reinterpret_cast<const RawT*>(a.k + idx);
         iv = *reinterpret_cast<const RawT*>(a.v + idx);
       }
     }
   };
-  // the first two rows in flight too (two rows ahead of the one being computed)
-  RawT cq, ck, cv, n1q, n1k, n1v;
-  load_row(8 * warp, cq, ck, cv);
-  load_row(8 * warp + 1, n1q, n1k, n1v);
+  // the first row pair in flight too (rows are processed in pairs, one pair ahead)
+  RawT aq, ak, av, bq, bk, bv;
+  load_row(8 * pr, aq, ak, av);
+  load_row(8 * pr + 1, bq, bk, bv);
 
   // ---- log decay and its running sum G over the chunk, in log2 units (G log2 e):
-  // channels 2p, 2p+1, rows 16q..16q+15 per thread ----
+  // channels 2p, 2p+1, rows 8q..8q+7 per thread ----
   {
     // while the gate loads are in flight: pull into L2 the inputs of the tile one wave of
     // CTAs ahead in the grid (it will run after this one), 128-byte lines spread over threads
@@ -307,25 +316,25 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
       // log2 a = lb log2(e) sigmoid(exp(A_log) (f + dt_bias))
       const float Ah2 = expf(A_log_h) * LOG2E, lb2 = a.lb * LOG2E;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const bool live = 16 * qr + i < L;
+      for (int i = 0; i < 8; ++i) {
+        const bool live = 8 * qr + i < L;
         g0[i] = live ? lb2 * sigmoid2(Ah2 * (g0[i] + dtb.x)) : 0.f;
         g1[i] = live ? lb2 * sigmoid2(Ah2 * (g1[i] + dtb.y)) : 0.f;
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < 8; ++i) {
         g0[i] *= LOG2E;
         g1[i] *= LOG2E;
       }
     }
 #pragma unroll
-    for (int i = 1; i < 16; ++i) {
+    for (int i = 1; i < 8; ++i) {
       g0[i] += g0[i - 1];
       g1[i] += g1[i - 1];
     }
-    qsum[qr][cp] = g0[15];
-    qsum[qr][cp + 1] = g1[15];
+    qsum[qr][cp] = g0[7];
+    qsum[qr][cp + 1] = g1[7];
     if (tid < C) {
       float bv = 0.f;
       if (tid < L) {
@@ -338,108 +347,87 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     __syncthreads();
     float o0 = 0.f, o1 = 0.f;
 #pragma unroll
-    for (int q = 0; q < 3; ++q)
+    for (int q = 0; q < 7; ++q)
       if (q < qr) {
         o0 += qsum[q][cp];
         o1 += qsum[q][cp + 1];
       }
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-      *reinterpret_cast<float2*>(G + (16 * qr + i) * D + cp) = make_float2(g0[i] + o0, g1[i] + o1);
-    if (qr == 3)
-      *reinterpret_cast<float2*>(gCo + cp) = make_float2(ex2a(g0[15] + o0), ex2a(g1[15] + o1));
+    for (int i = 0; i < 8; ++i)
+      *reinterpret_cast<float2*>(G + (8 * qr + i) * D + cp) = make_float2(g0[i] + o0, g1[i] + o1);
+    if (qr == 7)
+      *reinterpret_cast<float2*>(gCo + cp) = make_float2(ex2a(g0[7] + o0), ex2a(g1[7] + o1));
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
 
-  // ---- token rows 8w..8w+7: (prep), operands for the MMAs, Q~ and K' ----
+  // ---- token rows, in pairs: (prep), operands for the MMAs, Q~ and K' ----
   {
-    float win[KC - 1][12];
+    // q, k and v leave the conv scaled by log2 e (taps pre-scaled): the L2 norm of q and k
+    // cancels the factor (with eps scaled alike) and v takes ln 2 back
+    const float qsc = a.q_scale, inv_eps = 1.0f / (a.l2_eps * LOG2E);
+    float win[KC - 1][6];   // previous pre-conv rows, oldest first: q0 q1 k0 k1 v0 v1
     if (FUSED) {
 #pragma unroll
       for (int sgm = 0; sgm < 3; ++sgm)
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 2; ++j)
           cw[sgm][j] = make_float4(cw[sgm][j].x * LOG2E, cw[sgm][j].y * LOG2E,
                                    cw[sgm][j].z * LOG2E, cw[sgm][j].w * LOG2E);
 #pragma unroll
       for (int m = 0; m < KC - 1; ++m)
 #pragma unroll
         for (int sgm = 0; sgm < 3; ++sgm) {
-          const float4 t = to_f4(winr[m][sgm]);
-          win[m][4 * sgm] = t.x; win[m][4 * sgm + 1] = t.y;
-          win[m][4 * sgm + 2] = t.z; win[m][4 * sgm + 3] = t.w;
+          const float2 t = to_f2(winr[m][sgm]);
+          win[m][2 * sgm] = t.x;
+          win[m][2 * sgm + 1] = t.y;
         }
     }
-    // q, k and v leave the conv scaled by log2 e (taps pre-scaled): the L2 norm of q and k
-    // cancels the factor (with eps scaled alike) and v takes ln 2 back
-    const float qsc = a.q_scale, inv_eps = 1.0f / (a.l2_eps * LOG2E);
-    const float4 g15 = lds4(G + 15 * D + c4), g47 = lds4(G + 47 * D + c4),
-                 g63 = lds4(G + 63 * D + c4);
-    const float r15[4] = {g15.x, g15.y, g15.z, g15.w}, r47[4] = {g47.x, g47.y, g47.z, g47.w},
-                r63[4] = {g63.x, g63.y, g63.z, g63.w};
-#pragma unroll 1
-    for (int i = 0; i < 8; ++i) {
-      const int r = 8 * warp + i;
-      RawT n2q, n2k, n2v;
-      load_row(i + 2 < 8 ? r + 2 : C, n2q, n2k, n2v);
-      const float4 fq = to_f4(cq), fk = to_f4(ck), fv = to_f4(cv);
-      float qv[4], kv[4], vv[4];
-      if (FUSED) {
-        const float xq[4] = {fq.x, fq.y, fq.z, fq.w};
-        const float xk[4] = {fk.x, fk.y, fk.z, fk.w};
-        const float xv[4] = {fv.x, fv.y, fv.z, fv.w};
-        float sq = 0.f, sk = 0.f;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          // taps 0..K-2 on the window (oldest first), tap K-1 on the current row
-          const float4 wq = cw[0][j], wk = cw[1][j], wv = cw[2][j];
-          float aq = wq.w * xq[j], ak = wk.w * xk[j], av = wv.w * xv[j];
-          aq = fmaf(wq.x, win[0][j], aq); aq = fmaf(wq.y, win[1][j], aq); aq = fmaf(wq.z, win[2][j], aq);
-          ak = fmaf(wk.x, win[0][4 + j], ak); ak = fmaf(wk.y, win[1][4 + j], ak);
-          ak = fmaf(wk.z, win[2][4 + j], ak);
-          av = fmaf(wv.x, win[0][8 + j], av); av = fmaf(wv.y, win[1][8 + j], av);
-          av = fmaf(wv.z, win[2][8 + j], av);
-          qv[j] = aq * sigmoid2(aq);
-          kv[j] = ak * sigmoid2(ak);
-          vv[j] = LN2 * av * sigmoid2(av);
-          sq = fmaf(qv[j], qv[j], sq);
-          sk = fmaf(kv[j], kv[j], sk);
-        }
-#pragma unroll
-        for (int e = 0; e < 12; ++e) {
-          win[0][e] = win[1][e];
-          win[1][e] = win[2][e];
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          win[2][j] = xq[j]; win[2][4 + j] = xk[j]; win[2][8 + j] = xv[j];
-        }
-        sq = warp_sum(sq);
-        sk = warp_sum(sk);
-        const bool live = r < L;   // rows past the sequence end stay zero
-        // 1 / max(||x||, eps) = min(rsqrt(||x||^2), 1 / eps), rsqrt(0) = inf
-        const float iq = live ? qsc * fminf(rsqrta(sq), inv_eps) : 0.f;   // q_scale folded in
-        const float ik = live ? fminf(rsqrta(sk), inv_eps) : 0.f;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          qv[j] *= iq;
-          kv[j] *= ik;
-          vv[j] = live ? vv[j] : 0.f;
-        }
-      } else {
-        qv[0] = qsc * fq.x; qv[1] = qsc * fq.y; qv[2] = qsc * fq.z; qv[3] = qsc * fq.w;
-        kv[0] = fk.x; kv[1] = fk.y; kv[2] = fk.z; kv[3] = fk.w;
-        vv[0] = fv.x; vv[1] = fv.y; vv[2] = fv.z; vv[3] = fv.w;
+    const float2 g15 = *reinterpret_cast<const float2*>(G + 15 * D + c2);
+    const float2 g47 = *reinterpret_cast<const float2*>(G + 47 * D + c2);
+    const float2 g63 = *reinterpret_cast<const float2*>(G + 63 * D + c2);
+    const float r15[2] = {g15.x, g15.y}, r47[2] = {g47.x, g47.y}, r63[2] = {g63.x, g63.y};
+
+    // depthwise conv (taps 0..K-2 on the window, K-1 on the row) and SiLU of one row;
+    // the row then enters the window.  Returns the partial sums of squares of q and k.
+    auto conv_row = [&](RawT iq, RawT ik, RawT iv, float (&qv)[2], float (&kv)[2],
+                        float (&vv)[2]) -> float2 {
+      const float2 fq = to_f2(iq), fk = to_f2(ik), fv = to_f2(iv);
+      if (!FUSED) {
+        qv[0] = qsc * fq.x; qv[1] = qsc * fq.y;
+        kv[0] = fk.x; kv[1] = fk.y;
+        vv[0] = fv.x; vv[1] = fv.y;
+        return make_float2(0.f, 0.f);
       }
-      const float4 gr4 = lds4(G + r * D + c4);
-      const float gr[4] = {gr4.x, gr4.y, gr4.z, gr4.w};
-      const bool lowhalf = r < 32;
-      float kb[4], qb[4], kc0[4], kc1[4], qt[4], kt[4], kp[4];
+      const float xr[6] = {fq.x, fq.y, fk.x, fk.y, fv.x, fv.y};
+      float z[6];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int e = 0; e < 6; ++e) {
+        const float4 w = cw[e >> 1][e & 1];
+        float acc = w.w * xr[e];
+        acc = fmaf(w.x, win[0][e], acc);
+        acc = fmaf(w.y, win[1][e], acc);
+        acc = fmaf(w.z, win[2][e], acc);
+        z[e] = acc * sigmoid2(acc);
+        win[0][e] = win[1][e];
+        win[1][e] = win[2][e];
+        win[2][e] = xr[e];
+      }
+      qv[0] = z[0]; qv[1] = z[1];
+      kv[0] = z[2]; kv[1] = z[3];
+      vv[0] = LN2 * z[4]; vv[1] = LN2 * z[5];
+      return make_float2(fmaf(z[0], z[0], z[1] * z[1]), fmaf(z[2], z[2], z[3] * z[3]));
+    };
+    // every operand of one token row r for this lane's two channels
+    auto operands = [&](int r, const float (&qv)[2], const float (&kv)[2], const float (&vv)[2]) {
+      const float2 gr2 = *reinterpret_cast<const float2*>(G + r * D + c2);
+      const float gr[2] = {gr2.x, gr2.y};
+      const bool lowhalf = r < 32;
+      float kb[2], qb[2], kc0[2], kc1[2], qt[2], kt[2], kp[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
         const float g = gr[j];
         const float er = ex2a(g - (lowhalf ? r15[j] : r47[j]));
         kb[j] = kv[j] * er;
@@ -452,25 +440,50 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
         kp[j] = kv[j] * ex2a(r63[j] - g);
       }
       const int nk = lowhalf ? r : 64 + (r - 32);
-      st_tf32x4(sm + OFF_GB + gram_off(nk, c4), kb[0], kb[1], kb[2], kb[3]);
-      st_tf32x4(sm + OFF_GB + gram_off(nk + 32, c4), qb[0], qb[1], qb[2], qb[3]);
-      if (lowhalf) st_tf32x4(sm + OFF_GA + gram_off(r, c4), kc0[0], kc0[1], kc0[2], kc0[3]);
-      st_tf32x4(sm + OFF_GA + gram_off(32 + r, c4), kc1[0], kc1[1], kc1[2], kc1[3]);
-      {
-        float hi[4], lo[4];
+      st_tf32x2(sm + OFF_GB + gram_off(nk, c2), kb[0], kb[1]);
+      st_tf32x2(sm + OFF_GB + gram_off(nk + 32, c2), qb[0], qb[1]);
+      if (lowhalf) st_tf32x2(sm + OFF_GA + gram_off(r, c2), kc0[0], kc0[1]);
+      st_tf32x2(sm + OFF_GA + gram_off(32 + r, c2), kc1[0], kc1[1]);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(kt[0], kt[1]);
+      const float2 hf = __bfloat1622float2(hi);
+      *reinterpret_cast<__nv_bfloat162*>(sm + OFF_KT + mn_off(r, c2)) = hi;
+      st_bf16x2(sm + OFF_KL + mn_off(r, c2), kt[0] - hf.x, kt[1] - hf.y);
+      st_bf16x2(sm + OFF_VT + mn_off(r, c2), vv[0], vv[1]);
+      st_bf16x2(Qo + (size_t)r * D + c2, qt[0], qt[1]);
+      st_bf16x2(Ko + (size_t)r * D + c2, kp[0], kp[1]);
+    };
+
+#pragma unroll 1
+    for (int k = 0; k < 4; ++k) {
+      const int ra = 8 * pr + 2 * k, rb = ra + 1;
+      RawT nq0, nk0, nv0, nq1, nk1, nv1;   // the next pair, in flight through this one
+      load_row(k < 3 ? ra + 2 : C, nq0, nk0, nv0);
+      load_row(k < 3 ? ra + 3 : C, nq1, nk1, nv1);
+      float qa[2], ka[2], va[2], qb2[2], kb2[2], vb2[2];
+      const float2 sa = conv_row(aq, ak, av, qa, ka, va);
+      const float2 sb = conv_row(bq, bk, bv, qb2, kb2, vb2);
+      if (FUSED) {
+        // q and k norms over 128 channels: this warp's 64 (shuffles) + the partner warp's
+        float4 part = make_float4(warp_sum(sa.x), warp_sum(sa.y), warp_sum(sb.x), warp_sum(sb.y));
+        if (lane == 0) pnorm[pr][k & 1][hh] = part;
+        asm volatile("bar.sync %0, 64;" ::"r"(1 + pr) : "memory");
+        const float4 o = pnorm[pr][k & 1][hh ^ 1];
+        part.x += o.x; part.y += o.y; part.z += o.z; part.w += o.w;
+        // 1 / max(||x||, eps) = min(rsqrt(||x||^2), 1 / eps), rsqrt(0) = inf; q_scale folded
+        const float iqa = ra < L ? qsc * fminf(rsqrta(part.x), inv_eps) : 0.f;
+        const float ika = ra < L ? fminf(rsqrta(part.y), inv_eps) : 0.f;
+        const float iqb = rb < L ? qsc * fminf(rsqrta(part.z), inv_eps) : 0.f;
+        const float ikb = rb < L ? fminf(rsqrta(part.w), inv_eps) : 0.f;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          hi[j] = __bfloat162float(__float2bfloat16_rn(kt[j]));
-          lo[j] = kt[j] - hi[j];
+        for (int j = 0; j < 2; ++j) {
+          qa[j] *= iqa; ka[j] *= ika; va[j] = ra < L ? va[j] : 0.f;
+          qb2[j] *= iqb; kb2[j] *= ikb; vb2[j] = rb < L ? vb2[j] : 0.f;
         }
-        st_bf16x4(sm + OFF_KT + mn_off(r, c4), hi[0], hi[1], hi[2], hi[3]);
-        st_bf16x4(sm + OFF_KL + mn_off(r, c4), lo[0], lo[1], lo[2], lo[3]);
       }
-      st_bf16x4(sm + OFF_VT + mn_off(r, c4), vv[0], vv[1], vv[2], vv[3]);
-      st4(Qo + (size_t)r * D + c4, make_float4(qt[0], qt[1], qt[2], qt[3]));
-      st4(Ko + (size_t)r * D + c4, make_float4(kp[0], kp[1], kp[2], kp[3]));
-      cq = n1q; ck = n1k; cv = n1v;
-      n1q = n2q; n1k = n2k; n1v = n2v;
+      operands(ra, qa, ka, va);
+      operands(rb, qb2, kb2, vb2);
+      aq = nq0; ak = nk0; av = nv0;
+      bq = nq1; bk = nk1; bv = nv1;
     }
   }
   fence_proxy_async();
@@ -496,7 +509,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   // Warps of lane quarters 0-2 each read one 32-column group: warp w < 4 the keys (A),
   // warp w + 4 the queries (M); quarter 3 (rows 96-127 of D) holds nothing and writes the
   // zero upper-right block of M.
-  if (ok && (warp & 3) < 3) {
+  if (ok && warp < 8 && (warp & 3) < 3) {
     const int q = warp & 3;
     const int i = (q == 2) ? 32 + lane : lane;          // key index of this TMEM lane
     const int rbase = (q == 0) ? 0 : 32;                 // first row r of the group
@@ -634,18 +647,16 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   if (ok) ok = mbar_wait_warp(smem_u32(&bar_mma), 1, &abort_flag);
   tc_fence_after();
   if (ok) {
+    // warp w: TMEM lane quarter w % 4 (channels), W (w & 4 == 0) or U~, token half w / 8
     const int q = warp & 3;
     const int c = 32 * q + lane;
-    __nv_bfloat16* dst = (warp < 4) ? Wo : Uo;
-    const uint32_t col = (warp < 4) ? 0u : 64u;
+    const bool isW = (warp & 4) == 0;
+    const int hf = warp >> 3;
+    __nv_bfloat16* dst = isW ? Wo : Uo;
+    float v[32];
+    tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (isW ? 0u : 64u) + 32u * hf, v);
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      float v[32];
-      tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + col + 32 * hf, v);
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        dst[(size_t)(32 * hf + j) * D + c] = __float2bfloat16_rn(v[j]);
-    }
+    for (int j = 0; j < 32; ++j) dst[(size_t)(32 * hf + j) * D + c] = __float2bfloat16_rn(v[j]);
   }
 
   tc_fence_before();
