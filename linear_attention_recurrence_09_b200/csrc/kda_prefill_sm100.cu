@@ -25,9 +25,9 @@
 // MMAs from one thread with precomputed descriptors, warps 2-9 run the
 // epilogues, two warps per TMEM lane quarter (quarter = warp % 4), each owning
 // 16 of the 32 value columns.  E1 and E2 are on the serial chain; E3 waits for
-// MMA3 after the state is handed back, off the chain.  Every MMA operand is
-// K-major with the 128-byte swizzle: TMA writes the workspace tiles in that
-// layout and the epilogue threads write S^T and U^T in it by hand.
+// MMA3 after the state is handed back, off the chain.  Every MMA operand uses the
+// 128-byte swizzle: TMA writes the workspace tiles (K-major; K' read MN-major) and the
+// epilogue threads write S and U MN-major, 16 bytes at a time.
 //
 // Every wait is bounded (about a second): on expiry the CTA records
 // KDA_ERR_TIMEOUT in the workspace status word, drains what it issued, frees
@@ -58,9 +58,12 @@ constexpr uint32_t UT_BYTES = C * J * 2;         // U~ slice: 64 rows x 32 cols 
 constexpr uint32_t STAGE_BYTES = A1_BYTES + A2_BYTES + A3_BYTES + UT_BYTES;
 constexpr uint32_t NSTAGE = 2;
 constexpr uint32_t TX_BYTES = 4 * 8192 + 2 * 8192 + 8192 + UT_BYTES;   // W x2, Q~ x2, K' x2, M, U~
-constexpr uint32_t OFF_S = NSTAGE * STAGE_BYTES;          // S^T: 2 K-blocks x 32 rows x 128 B
-constexpr uint32_t OFF_U = OFF_S + 2 * J * 128;           // U^T: 32 rows x 128 B
-constexpr uint32_t OFF_BAR = OFF_U + J * 128;
+// S (128 key rows) and U (64 token rows) as MN-major B operands: one 128-byte swizzled
+// row per key / token with the slice's 32 value columns in its first 64 bytes (the MMAs
+// have N = 32 and never read the rest), so a thread writes its 16 columns as 2 x 16 bytes
+constexpr uint32_t OFF_S = NSTAGE * STAGE_BYTES;          // S: 128 rows x 128 B
+constexpr uint32_t OFF_U = OFF_S + 128 * 128;             // U:  64 rows x 128 B
+constexpr uint32_t OFF_BAR = OFF_U + 64 * 128;
 constexpr uint32_t OFF_SSQ = OFF_BAR + 256;   // fused norm: [2 parities][4 slices][64 tokens] fp32
 constexpr uint32_t SMEM_BYTES = OFF_SSQ + 2 * NSLICE * C * 4 + 1024;   // + alignment slack
 
@@ -78,6 +81,20 @@ struct TmaMaps {
 
 // sigmoid on the special-function unit (bf16 output: approximate exp and divide suffice)
 __device__ __forceinline__ float fast_sigmoid(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
+
+// byte offset of element (row k, column n < 64) of an MN-major, 128B-swizzled bf16 tile
+// (rows of 128 bytes, 8-row groups of 1024 bytes, 16-byte chunks XOR-ed with k mod 8)
+__device__ __forceinline__ uint32_t mn_row_chunk(int k, int chunk) {
+  return (uint32_t)((k >> 3) * 1024 + (k & 7) * 128 + (((chunk ^ k) & 7) << 4));
+}
+// eight fp32 values -> eight bf16 in one 16-byte chunk
+__device__ __forceinline__ uint4 pack8_bf16(const float* v) {
+  uint4 r;
+  __nv_bfloat162* p = reinterpret_cast<__nv_bfloat162*>(&r);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) p[e] = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+  return r;
+}
 
 // K-major SW128 descriptor advanced by `bytes` (the 14-bit address field never carries)
 __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
@@ -181,10 +198,10 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      const uint32_t id = idesc_bf16(128, J);
-      const uint32_t id_amn = idesc_bf16_amn(128, J);   // K' is read MN-major
+      const uint32_t id = idesc_bf16(128, J) | (1u << 16);      // B (S or U) MN-major
+      const uint32_t id_amn = id | (1u << 15);                   // K' is read MN-major too
       const uint64_t dA1s0 = sw128_desc(sbase), dA1s1 = sw128_desc(sbase + STAGE_BYTES);
-      const uint64_t dS = sw128_desc(sbase + OFF_S), dU = sw128_desc(sbase + OFF_U);
+      const uint32_t sS = sbase + OFF_S, sU = sbase + OFF_U;   // K steps of 16 rows = 2 KB
       int last = -1;
       for (int n = 0; n < nch; ++n) {
         const int st = n & 1;
@@ -203,18 +220,19 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           umma(d1, desc_add(a1, (k >> 2) * 16384 + (k & 3) * 32),
-               desc_add(dS, (k >> 2) * 4096 + (k & 3) * 32), id, k > 0);
+               sw128_mn_desc(sS + k * 2048, 8192), id, k > 0);
         umma_commit(bar(BAR_MMA1));
         last = n;
         if (!mbar_wait(bar(BAR_UREADY), n & 1, &abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          umma(d2_tmem, sw128_mn_desc(a2s + k * 2048, 8192), desc_add(dU, k * 32), id_amn, k > 0);
+          umma(d2_tmem, sw128_mn_desc(a2s + k * 2048, 8192), sw128_mn_desc(sU + k * 2048, 8192),
+               id_amn, k > 0);
         umma_commit(bar(BAR_MMA2));
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          umma(d1, desc_add(a3, k * 32), desc_add(dU, k * 32), id, 1);
+          umma(d1, desc_add(a3, k * 32), sw128_mn_desc(sU + k * 2048, 8192), id, 1);
         umma_commit(bar(BAR_EMPTY0 + st));
         // O of chunk n complete in D1 buffer n % 3 (its own barrier: the O warps may lag
         // behind the stage barrier by more than one phase, never behind this one)
@@ -325,12 +343,9 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
 #pragma unroll
       for (int c = 0; c < JH; ++c) S[c] = 0.f;
     }
-    unsigned char* sblk = SB + (i >> 6) * 4096;
-    auto write_state = [&]() {
-#pragma unroll
-      for (int n = 0; n < JH; ++n)
-        *reinterpret_cast<__nv_bfloat16*>(sblk + sw128_off(cb + n, i & 63)) =
-            __float2bfloat16_rn(S[n]);
+    auto write_state = [&]() {   // key row i, columns cb..cb+15: two 16-byte chunks
+      *reinterpret_cast<uint4*>(SB + mn_row_chunk(i, cb / 8)) = pack8_bf16(S);
+      *reinterpret_cast<uint4*>(SB + mn_row_chunk(i, cb / 8 + 1)) = pack8_bf16(S + 8);
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(bar(BAR_SREADY));
@@ -353,19 +368,17 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
             reinterpret_cast<const __nv_bfloat16*>(sm + st * STAGE_BYTES + A1_BYTES + A2_BYTES +
                                                    A3_BYTES) + i * J + cb;
 #pragma unroll
-        for (int m = 0; m < JH; m += 8) {
+        for (int m = 0; m < JH; m += 8) {   // token row i, columns cb+m..cb+m+7
           const uint4 raw = *reinterpret_cast<const uint4*>(ut + m);
           const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+          float u[8];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 f = __bfloat1622float2(p2[e]);
-            const float u0 = (i < L) ? f.x - ws[m + 2 * e] : 0.f;
-            const float u1 = (i < L) ? f.y - ws[m + 2 * e + 1] : 0.f;
-            *reinterpret_cast<__nv_bfloat16*>(UB + sw128_off(cb + m + 2 * e, i)) =
-                __float2bfloat16_rn(u0);
-            *reinterpret_cast<__nv_bfloat16*>(UB + sw128_off(cb + m + 2 * e + 1, i)) =
-                __float2bfloat16_rn(u1);
+            u[2 * e] = (i < L) ? f.x - ws[m + 2 * e] : 0.f;
+            u[2 * e + 1] = (i < L) ? f.y - ws[m + 2 * e + 1] : 0.f;
           }
+          *reinterpret_cast<uint4*>(UB + mn_row_chunk(i, (cb + m) / 8)) = pack8_bf16(u);
         }
         fence_proxy_async();
         tc_fence_before();
