@@ -218,6 +218,47 @@ KDA_API int kda_decode(const kda_config* cfg, int32_t batch, const void* q,
                void* y, kda_stream_t stream);
 
 /*
+ * kda_layer_decode - one token for each of `batch` sequences from the raw layer
+ * inputs: the prep of kda_prep (COMMIT mode: depthwise causal conv against the conv
+ * state, which is advanced in place; SiLU; q, k L2 norms; the decay gate; beta) and
+ * the step of kda_decode, in one kernel.  Same result as kda_prep + kda_decode.
+ *
+ *  x [batch, H, 3d] (pre-conv q|k|v); f, g [batch, H, d]; beta_logit [batch, H]
+ *    (all in cfg->dtype); conv_w fp32 [H, 3d, K]; A_log fp32 [H]; dt_bias fp32 [H, d]
+ *  conv_state [pool_size, K-1, H, 3d] (cfg->dtype), NULL for zeros (then not updated)
+ *  state      fp32 [pool_size, H, d, d], updated in place (row state_slots[b] or b)
+ *  y          out [batch, H, d]
+ */
+KDA_API int kda_layer_decode(const kda_config* cfg, int32_t batch, const void* x,
+                             const void* f, const void* beta_logit, const void* g,
+                             const float* conv_w, const float* A_log, const float* dt_bias,
+                             const float* norm_w, void* conv_state, float* state,
+                             const int32_t* state_slots, int32_t pool_size, void* y,
+                             kda_stream_t stream);
+
+/*
+ * kda_layer_verify - kda_prep in TAPE mode and kda_verify in one kernel: a block of
+ * `block_len` (1..16) draft tokens per sequence from the raw layer inputs.  The conv
+ * state and the recurrent state are only read; the tape and the conv window (history
+ * then the block's x rows, for kda_rollback) are written.  Same result as kda_prep
+ * (TAPE) + kda_verify.
+ *
+ *  x [batch, block_len, H, 3d]; f, g [batch, block_len, H, d];
+ *  beta_logit [batch, block_len, H]; conv_w, A_log, dt_bias, norm_w as kda_layer_decode
+ *  conv_state [pool_size, K-1, H, 3d] or NULL (zeros); state fp32 [pool_size, H, d, d]
+ *  tape       out fp32 [batch, block_len, H, d, d]
+ *  conv_window out [batch, K-1+block_len, H, 3d] (cfg->dtype)
+ *  y          out [batch, block_len, H, d]
+ */
+KDA_API int kda_layer_verify(const kda_config* cfg, int32_t batch, int32_t block_len,
+                             const void* x, const void* f, const void* beta_logit,
+                             const void* g, const float* conv_w, const float* A_log,
+                             const float* dt_bias, const float* norm_w,
+                             const void* conv_state, const float* state,
+                             const int32_t* state_slots, int32_t pool_size, float* tape,
+                             void* conv_window, void* y, kda_stream_t stream);
+
+/*
  * kda_verify - speculative verify of a block of `block_len` draft tokens per
  * sequence (1..16; the DFlash2 drafter of dflash-mlx issue #63 uses 8).  Runs
  * the decode step block_len times from one load of each state, keeps the live

@@ -288,6 +288,61 @@ static int step_common(const kda_config* cfg, int32_t batch, int32_t T, const vo
   return cuda_status(kda::launch_step(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+static int layer_step_common(const kda_config* cfg, int32_t batch, int32_t T, const void* x,
+                             const void* f, const void* beta_logit, const void* g,
+                             const float* conv_w, const float* A_log, const float* dt_bias,
+                             const float* norm_w, void* conv_state, const float* state_in,
+                             float* state_out, float* tape, void* window,
+                             const int32_t* slots, int32_t pool_size, void* y,
+                             kda_stream_t stream) {
+  int st = check_cfg(cfg);
+  if (st) return st;
+  if (batch < 0) return KDA_ERR_INVALID_ARG;
+  if (batch == 0) return KDA_OK;
+  if ((st = check_ptrs({x, f, beta_logit, g, conv_w, A_log, dt_bias, norm_w, state_in, y},
+                       {slots, conv_state, window})))
+    return st;
+  if ((st = check_pool(slots, pool_size, batch))) return st;
+  kda::StepArgs a{};
+  a.B = batch; a.T = T; a.H = cfg->num_heads; a.D = cfg->head_dim;
+  a.bf16 = cfg->dtype == KDA_BF16;
+  a.g = g; a.norm_w = norm_w;
+  a.state_in = state_in; a.state_out = state_out; a.tape = tape;
+  a.slots = slots; a.pool_size = pool_size; a.y = y;
+  a.norm_eps = cfg->norm_eps; a.q_scale = cfg->q_scale;
+  a.x = x; a.f = f; a.beta_logit = beta_logit;
+  a.conv_w = conv_w; a.A_log = A_log; a.dt_bias = dt_bias;
+  a.conv_state = conv_state; a.window = window; a.K = cfg->conv_size;
+  a.lb = cfg->gate_lower_bound; a.l2_eps = cfg->l2_eps;
+  return cuda_status(kda::launch_step(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int kda_layer_decode(const kda_config* cfg, int32_t batch, const void* x, const void* f,
+                     const void* beta_logit, const void* g, const float* conv_w,
+                     const float* A_log, const float* dt_bias, const float* norm_w,
+                     void* conv_state, float* state, const int32_t* state_slots,
+                     int32_t pool_size, void* y, kda_stream_t stream) {
+  return layer_step_common(cfg, batch, 1, x, f, beta_logit, g, conv_w, A_log, dt_bias, norm_w,
+                           conv_state, state, state, nullptr, nullptr, state_slots, pool_size,
+                           y, stream);
+}
+
+int kda_layer_verify(const kda_config* cfg, int32_t batch, int32_t block_len, const void* x,
+                     const void* f, const void* beta_logit, const void* g,
+                     const float* conv_w, const float* A_log, const float* dt_bias,
+                     const float* norm_w, const void* conv_state, const float* state,
+                     const int32_t* state_slots, int32_t pool_size, float* tape,
+                     void* conv_window, void* y, kda_stream_t stream) {
+  if (block_len < 1 || block_len > 16) return KDA_ERR_INVALID_ARG;
+  if (batch > 0) {
+    int st = check_ptrs({tape, conv_window}, {});
+    if (st) return st;
+  }
+  return layer_step_common(cfg, batch, block_len, x, f, beta_logit, g, conv_w, A_log, dt_bias,
+                           norm_w, const_cast<void*>(conv_state), state, nullptr, tape,
+                           conv_window, state_slots, pool_size, y, stream);
+}
+
 int kda_decode(const kda_config* cfg, int32_t batch, const void* q, const void* k,
                const void* v, const float* log_a, const float* beta, const void* g,
                const float* norm_w, float* state, const int32_t* state_slots,

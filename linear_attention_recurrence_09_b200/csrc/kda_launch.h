@@ -48,6 +48,17 @@ struct StepArgs {  // decode (T = 1) and verify (T = block_len)
   int pool_size;
   void* y;
   float norm_eps, q_scale;
+  // raw inputs of the fused prep (kda_layer_decode / kda_layer_verify); x == nullptr otherwise
+  const void* x;            // [B, T, H, 3d] pre-conv q|k|v
+  const void* f;            // [B, T, H, d]
+  const void* beta_logit;   // [B, T, H]
+  const float* conv_w;      // [H, 3d, K]
+  const float* A_log;       // [H]
+  const float* dt_bias;     // [H, d]
+  void* conv_state;         // [pool, K-1, H, 3d]: updated in place (decode) or read (verify)
+  void* window;             // verify: [B, K-1+T, H, 3d] = [history; x] for rollback
+  int K;
+  float lb, l2_eps;
 };
 
 struct RollbackArgs {

@@ -1,4 +1,5 @@
-// kda_decode / kda_verify / kda_rollback: the token-at-a-time path.
+// kda_decode / kda_verify / kda_rollback (and kda_layer_decode / kda_layer_verify, which
+// run the prep of each token in the same kernel): the token-at-a-time path.
 //
 // The "fused operator" for the delta net of llama.cpp PR #27754 (backends that
 // have it skip the chunked graph for generation): per (sequence, head) the
@@ -26,6 +27,10 @@ struct StepShape {
   static constexpr int NW = (THREADS + 31) / 32;
 };
 
+// sigmoid on the special-function unit (approximate exp and reciprocal, relative error
+// ~1e-7); 1 / (1 + inf) = 0 keeps the saturated end exact
+__device__ __forceinline__ float fsig(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
+
 __device__ __forceinline__ float4 f4_scale(float4 a, float s) {
   return make_float4(a.x * s, a.y * s, a.z * s, a.w * s);
 }
@@ -34,7 +39,7 @@ __device__ __forceinline__ float4 f4_fma(float s, float4 a, float4 acc) {
                      fmaf(s, a.w, acc.w));
 }
 
-template <typename T, int D>
+template <typename T, int D, bool PREP>
 __global__ void __launch_bounds__(StepShape<D>::THREADS)
 step_kernel(const StepArgs a) {
   using SH = StepShape<D>;
@@ -47,6 +52,11 @@ step_kernel(const StepArgs a) {
   __shared__ __align__(16) float redq[RG][D];
   __shared__ float ssq[SH::NW];
   __shared__ float kq_s;
+  // fused prep: conv history [K-1][3d] (oldest first), conv + SiLU outputs, v, beta, norms
+  constexpr int KMAX = 8;
+  __shared__ __align__(16) float hist[PREP ? KMAX - 1 : 1][PREP ? 3 * D : 1];
+  __shared__ __align__(16) float pre[PREP ? 3 * D : 1];
+  __shared__ float beta_s, nrm_w[SH::NW];   // per-warp partial sums of squares (q | k)
 
   const int h = blockIdx.x, b = blockIdx.y;
   const int H = a.H;
@@ -60,6 +70,23 @@ step_kernel(const StepArgs a) {
   const T* __restrict__ gg = static_cast<const T*>(a.g);
   T* __restrict__ yg = static_cast<T*>(a.y);
 
+  constexpr int C3 = 3 * D;
+  const int Km1 = PREP ? a.K - 1 : 0;
+  T* csg = PREP ? static_cast<T*>(a.conv_state) : nullptr;
+  T* wing = PREP ? static_cast<T*>(a.window) : nullptr;
+  if (PREP) {
+    // the sequence's conv history for this head (zeros without a conv state); verify
+    // also starts its rollback window with it
+    for (int e = tid; e < Km1 * C3; e += THREADS) {
+      const int j = e / C3, c = e - j * C3;
+      float hv = 0.f;
+      if (csg) hv = ld1(csg + (((size_t)row * Km1 + j) * H + h) * C3 + c);
+      hist[j][c] = hv;
+      if (wing) st1(wing + (((size_t)b * (Km1 + a.T) + j) * H + h) * C3 + c, hv);
+    }
+    __syncthreads();   // loaded by (row, channel) pairs, used per channel below
+  }
+  // the state streams in while the (first token's) prep runs
   const float* Sg = a.state_in + ((size_t)row * H + h) * D * D;
   float4 S[ROWS];
 #pragma unroll
@@ -68,10 +95,71 @@ step_kernel(const StepArgs a) {
   for (int t = 0; t < a.T; ++t) {
     const size_t tok = (size_t)b * a.T + t;
     const size_t base = (tok * H + h) * D;
-    for (int c = tid; c < D; c += THREADS) {
-      ks[c] = __ldg(kg + base + c);
-      qs[c] = __ldg(qg + base + c);
-      as_[c] = expf(__ldg(a.loga + base + c));
+    if (PREP) {
+      // depthwise causal conv (tap K-1 = this token) + SiLU per channel of q|k|v; each
+      // thread owns its channels, so it also shifts their history.  Channel c < 2d (q, k)
+      // of thread c also accumulates its warp's sum of squares.
+      const T* xg = static_cast<const T*>(a.x) + tok * H * C3 + (size_t)h * C3;
+      const T* fg = static_cast<const T*>(a.f) + base;
+      float sq = 0.f;
+      for (int c = tid; c < C3; c += THREADS) {
+        const float xc = ld1(xg + c);
+        const float* w = a.conv_w + ((size_t)h * C3 + c) * a.K;
+        float acc;
+        if (a.K == 4) {   // the common case: one 16-byte load of the taps
+          const float4 w4 = __ldg(reinterpret_cast<const float4*>(w));
+          acc = fmaf(w4.x, hist[0][c], fmaf(w4.y, hist[1][c], fmaf(w4.z, hist[2][c], w4.w * xc)));
+        } else {
+          acc = __ldg(w + Km1) * xc;
+          for (int j = 0; j < Km1; ++j) acc = fmaf(__ldg(w + j), hist[j][c], acc);
+        }
+        const float z = acc * fsig(acc);
+        pre[c] = z;
+        if (c < 2 * D) sq = fmaf(z, z, sq);
+        for (int j = 0; j + 1 < Km1; ++j) hist[j][c] = hist[j + 1][c];
+        if (Km1 > 0) hist[Km1 - 1][c] = xc;
+        if (wing) st1(wing + (((size_t)b * (Km1 + a.T) + Km1 + t) * H + h) * C3 + c, xc);
+      }
+      // warps whose first channels are q (resp. k) hold q (resp. k) partial norms; with
+      // d < 32 a warp spans both, so the d < 32 shapes reduce per half-warp group below
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+      if (lane == 0) nrm_w[warp] = sq;
+      // decay a = exp(lb sigmoid(exp(A_log) (f + dt_bias))) and beta = sigmoid(logit)
+      const float Ah = __expf(__ldg(a.A_log + h));
+      for (int c = tid; c < D; c += THREADS)
+        as_[c] = __expf(a.lb * fsig(Ah * (ld1(fg + c) + __ldg(a.dt_bias + (size_t)h * D + c))));
+      if (tid == 0) beta_s = fsig(ld1(static_cast<const T*>(a.beta_logit) + tok * H + h));
+      __syncthreads();
+      if (D >= 32) {
+        // q channels are those of warps [0, d/32), k channels of warps [d/32, 2d/32)
+        float nq = 0.f, nk = 0.f;
+#pragma unroll
+        for (int w = 0; w < D / 32; ++w) { nq += nrm_w[w]; nk += nrm_w[D / 32 + w]; }
+        const float iq = 1.0f / fmaxf(sqrtf(nq), a.l2_eps), ik = 1.0f / fmaxf(sqrtf(nk), a.l2_eps);
+        for (int c = tid; c < D; c += THREADS) {
+          qs[c] = pre[c] * iq;
+          ks[c] = pre[D + c] * ik;
+        }
+      } else {
+        // d = 16: one warp covers q and k; reduce each half directly
+        float nq = 0.f, nk = 0.f;
+        for (int c = 0; c < D; ++c) {
+          nq = fmaf(pre[c], pre[c], nq);
+          nk = fmaf(pre[D + c], pre[D + c], nk);
+        }
+        const float iq = 1.0f / fmaxf(sqrtf(nq), a.l2_eps), ik = 1.0f / fmaxf(sqrtf(nk), a.l2_eps);
+        for (int c = tid; c < D; c += THREADS) {
+          qs[c] = pre[c] * iq;
+          ks[c] = pre[D + c] * ik;
+        }
+      }
+    } else {
+      for (int c = tid; c < D; c += THREADS) {
+        ks[c] = __ldg(kg + base + c);
+        qs[c] = __ldg(qg + base + c);
+        as_[c] = expf(__ldg(a.loga + base + c));
+      }
     }
     __syncthreads();
 
@@ -101,8 +189,9 @@ step_kernel(const StepArgs a) {
       float rk = 0.f, rq = 0.f;
 #pragma unroll
       for (int j = 0; j < RG; ++j) { rk += redk[j][tid]; rq += redq[j][tid]; }
-      const float bt = __ldg(a.beta + tok * H + h);
-      const float u = bt * (__ldg(vg + base + tid) - rk);
+      const float bt = PREP ? beta_s : __ldg(a.beta + tok * H + h);
+      const float vt = PREP ? pre[2 * D + tid] : __ldg(vg + base + tid);
+      const float u = bt * (vt - rk);
       o = a.q_scale * fmaf(u, kq_s, rq);
       us[tid] = u;
     }
@@ -136,6 +225,12 @@ step_kernel(const StepArgs a) {
     __syncthreads();
   }
 
+  if (PREP && csg != nullptr && wing == nullptr) {
+    // decode: the history now ends with this step's token(s); each thread wrote its own
+    // channels of hist, so no barrier is needed before it stores them
+    for (int c = tid; c < C3; c += THREADS)
+      for (int j = 0; j < Km1; ++j) st1(csg + (((size_t)row * Km1 + j) * H + h) * C3 + c, hist[j][c]);
+  }
   if (a.state_out != nullptr) {
     float* So = a.state_out + ((size_t)row * H + h) * D * D;
 #pragma unroll
@@ -143,18 +238,24 @@ step_kernel(const StepArgs a) {
   }
 }
 
-template <typename T>
-static cudaError_t launch_step_t(const StepArgs& a, cudaStream_t st) {
+template <typename T, bool PREP>
+static cudaError_t launch_step_p(const StepArgs& a, cudaStream_t st) {
   dim3 grid(a.H, a.B);
   switch (a.D) {
-    case 16: step_kernel<T, 16><<<grid, StepShape<16>::THREADS, 0, st>>>(a); break;
-    case 32: step_kernel<T, 32><<<grid, StepShape<32>::THREADS, 0, st>>>(a); break;
-    case 64: step_kernel<T, 64><<<grid, StepShape<64>::THREADS, 0, st>>>(a); break;
-    case 128: step_kernel<T, 128><<<grid, StepShape<128>::THREADS, 0, st>>>(a); break;
+    case 16: step_kernel<T, 16, PREP><<<grid, StepShape<16>::THREADS, 0, st>>>(a); break;
+    case 32: step_kernel<T, 32, PREP><<<grid, StepShape<32>::THREADS, 0, st>>>(a); break;
+    case 64: step_kernel<T, 64, PREP><<<grid, StepShape<64>::THREADS, 0, st>>>(a); break;
+    case 128: step_kernel<T, 128, PREP><<<grid, StepShape<128>::THREADS, 0, st>>>(a); break;
     default: return cudaErrorInvalidValue;
   }
   ++launch_counter();
   return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_step_t(const StepArgs& a, cudaStream_t st) {
+  if (a.x != nullptr && (a.K < 1 || a.K > 8)) return cudaErrorInvalidValue;
+  return a.x ? launch_step_p<T, true>(a, st) : launch_step_p<T, false>(a, st);
 }
 
 cudaError_t launch_step(const StepArgs& a, cudaStream_t st) {

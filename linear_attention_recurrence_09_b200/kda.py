@@ -35,7 +35,8 @@ ENTRY_POINTS = ('kda_status_string', 'kda_abi_version', 'kda_prep',
                 'kda_prefill_workspace_size', 'kda_prefill', 'kda_decode', 'kda_verify',
                 'kda_rollback', 'kda_workspace_status', 'kda_selftest_wait_timeout',
                 'kda_prefill_noalloc', 'kda_layer_prefill_workspace_size', 'kda_layer_prefill',
-                'kda_set_phase_events', 'kda_launch_count', 'kda_last_cuda_error')
+                'kda_set_phase_events', 'kda_launch_count', 'kda_last_cuda_error',
+                'kda_layer_decode', 'kda_layer_verify')
 
 
 class KdaError(RuntimeError):
@@ -121,6 +122,12 @@ def lib() -> ctypes.CDLL:
         L.kda_layer_prefill.argtypes = [ctypes.POINTER(CConfig), _I, _I, _P, _I, _P, _P, _P, _P,
                                         _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
                                         ctypes.c_size_t, _P]
+        L.kda_layer_decode.restype = ctypes.c_int
+        L.kda_layer_decode.argtypes = [ctypes.POINTER(CConfig), _I, _P, _P, _P, _P, _P, _P, _P,
+                                       _P, _P, _P, _P, _I, _P, _P]
+        L.kda_layer_verify.restype = ctypes.c_int
+        L.kda_layer_verify.argtypes = [ctypes.POINTER(CConfig), _I, _I, _P, _P, _P, _P, _P, _P,
+                                       _P, _P, _P, _P, _P, _I, _P, _P, _P, _P]
         L.kda_last_cuda_error.restype = ctypes.c_char_p
         L.kda_last_cuda_error.argtypes = []
         L.kda_launch_count.restype = ctypes.c_longlong
@@ -354,6 +361,57 @@ def kda_selftest_wait_timeout(workspace, stream=None):
     """Run the bounded-wait self-test on ``workspace`` (enqueue only)."""
     _check(lib().kda_selftest_wait_timeout(_ptr(workspace, None, 'workspace'), _stream(stream)),
            'kda_selftest_wait_timeout')
+
+
+def kda_layer_decode(cfg: Config, x, f, beta_logit, g, conv_w, A_log, dt_bias, norm_w, state,
+                     conv_state=None, state_slots=None, pool_size=None, y=None, stream=None):
+    """One token per sequence from the raw layer inputs (prep fused).  Returns y."""
+    H, d, K = cfg.num_heads, cfg.head_dim, cfg.conv_size
+    B = x.shape[0]
+    if y is None:
+        y = _empty((B, H, d), cfg.dtype, x.device)
+    if pool_size is None:
+        pool_size = state.shape[0]
+    c = cfg.c()
+    _check(lib().kda_layer_decode(
+        ctypes.byref(c), B, _ptr(x, cfg.dtype, 'x', (B, H, 3 * d)),
+        _ptr(f, cfg.dtype, 'f', (B, H, d)), _ptr(beta_logit, cfg.dtype, 'beta_logit', (B, H)),
+        _ptr(g, cfg.dtype, 'g', (B, H, d)), _ptr(conv_w, torch.float32, 'conv_w', (H, 3 * d, K)),
+        _ptr(A_log, torch.float32, 'A_log', (H,)), _ptr(dt_bias, torch.float32, 'dt_bias', (H, d)),
+        _ptr(norm_w, torch.float32, 'norm_w', (d,)), _ptr(conv_state, cfg.dtype, 'conv_state'),
+        _ptr(state, torch.float32, 'state'), _ptr(state_slots, torch.int32, 'state_slots'),
+        int(pool_size), _ptr(y, cfg.dtype, 'y', (B, H, d)), _stream(stream)), 'kda_layer_decode')
+    return y
+
+
+def kda_layer_verify(cfg: Config, x, f, beta_logit, g, conv_w, A_log, dt_bias, norm_w, state,
+                     conv_state=None, state_slots=None, pool_size=None, tape=None, window=None,
+                     y=None, stream=None):
+    """A block of draft tokens per sequence from the raw inputs (prep fused).
+    x is [B, T_b, H, 3d].  Returns (y, tape, window)."""
+    H, d, K = cfg.num_heads, cfg.head_dim, cfg.conv_size
+    B, Tb = x.shape[0], x.shape[1]
+    if y is None:
+        y = _empty((B, Tb, H, d), cfg.dtype, x.device)
+    if tape is None:
+        tape = _empty((B, Tb, H, d, d), torch.float32, x.device)
+    if window is None:
+        window = _empty((B, K - 1 + Tb, H, 3 * d), cfg.dtype, x.device)
+    if pool_size is None:
+        pool_size = state.shape[0]
+    c = cfg.c()
+    _check(lib().kda_layer_verify(
+        ctypes.byref(c), B, Tb, _ptr(x, cfg.dtype, 'x', (B, Tb, H, 3 * d)),
+        _ptr(f, cfg.dtype, 'f', (B, Tb, H, d)),
+        _ptr(beta_logit, cfg.dtype, 'beta_logit', (B, Tb, H)),
+        _ptr(g, cfg.dtype, 'g', (B, Tb, H, d)), _ptr(conv_w, torch.float32, 'conv_w', (H, 3 * d, K)),
+        _ptr(A_log, torch.float32, 'A_log', (H,)), _ptr(dt_bias, torch.float32, 'dt_bias', (H, d)),
+        _ptr(norm_w, torch.float32, 'norm_w', (d,)), _ptr(conv_state, cfg.dtype, 'conv_state'),
+        _ptr(state, torch.float32, 'state'), _ptr(state_slots, torch.int32, 'state_slots'),
+        int(pool_size), _ptr(tape, torch.float32, 'tape', (B, Tb, H, d, d)),
+        _ptr(window, cfg.dtype, 'window', (B, K - 1 + Tb, H, 3 * d)),
+        _ptr(y, cfg.dtype, 'y', (B, Tb, H, d)), _stream(stream)), 'kda_layer_verify')
+    return y, tape, window
 
 
 def kda_launch_count() -> int:

@@ -131,10 +131,18 @@ def test_split_invariance_5_plus_7():
     assert torch.equal(c2.cpu(), c_full.cpu())
 
 
-def _decode_run(cfg, P, steps_acts, state, conv_state, dev='cuda'):
-    """T decode steps: prep (T=1, COMMIT) + decode.  Returns y [T, B, H, d]."""
+def _decode_run(cfg, P, steps_acts, state, conv_state, dev='cuda', fused=False):
+    """T decode steps: prep (T=1, COMMIT) + decode, or kda_layer_decode (fused).
+    Returns y [T, B, H, d]."""
     ys = []
     for a in steps_acts:
+        if fused:
+            ys.append(kda.kda_layer_decode(cfg, a['x'].to(dev), a['f'].to(dev),
+                                           a['beta_logit'].to(dev), a['g'].to(dev),
+                                           P['conv_w'].to(dev), P['A_log'].to(dev),
+                                           P['dt_bias'].to(dev), P['norm_w'].to(dev), state,
+                                           conv_state=conv_state))
+            continue
         p = kda.kda_prep(cfg, a['cu_seqlens'].to(dev), a['x'].to(dev), a['f'].to(dev),
                          a['beta_logit'].to(dev), P['conv_w'].to(dev), P['A_log'].to(dev),
                          P['dt_bias'].to(dev), conv_state=conv_state, max_seqlen=1)
@@ -310,3 +318,68 @@ def test_layer_prefill_launches_and_fused_norm():
     ref = oracle_layer(cfg, P, A, S0, hist)
     assert rel_err(np64(y), ref['y']) <= 1e-2
     assert rel_err(np64(s_out), ref['state']) <= 1e-2
+
+
+@pytest.mark.parametrize('dtype,d', [(torch.bfloat16, 128), (torch.bfloat16, 32),
+                                     (torch.float32, 64), (torch.float32, 16)])
+def test_layer_decode_fused_prep(dtype, d):
+    """kda_layer_decode (prep inside the step kernel) against kda_prep + kda_decode and the
+    oracle: same y and state to rounding, the same conv state bit for bit."""
+    B, H, T0, steps = 3, 4, 40, 6
+    cfg, P, A, S0, hist = make_case(12, [T0] * B, H, d, 4, dtype, state_var=0.01,
+                                    conv_hist=True, chunk=16)
+    _, s0, c0, _ = gpu_layer(cfg, P, A, S0, hist)
+    sa = _step_acts(12, B, H, d, dtype, steps)
+    s_a, c_a = s0.clone(), c0.clone()
+    s_b, c_b = s0.clone(), c0.clone()
+    n0 = kda.kda_launch_count()
+    ys_f = _decode_run(cfg, P, sa, s_a, c_a, fused=True).cpu()
+    assert kda.kda_launch_count() - n0 == steps
+    ys_u = _decode_run(cfg, P, sa, s_b, c_b).cpu()
+    assert torch.equal(c_a.cpu(), c_b.cpu())
+    tol = TOL[dtype]
+    assert rel_err(np64(ys_f), np64(ys_u)) <= tol
+    assert rel_err(np64(s_a), np64(s_b)) <= tol
+    for b in range(B):
+        seq = _cat_seq([A] + sa, b)
+        ref = oracle_layer(cfg, P, seq, S0[b:b + 1], hist[b:b + 1])
+        assert rel_err(np64(ys_f[:, b]), ref['y'][T0:]) <= tol
+        assert rel_err(np64(s_a[b]), ref['state'][0]) <= tol
+
+
+@pytest.mark.parametrize('dtype', [torch.bfloat16, torch.float32])
+def test_layer_verify_fused_prep_and_rollback(dtype):
+    """kda_layer_verify against kda_prep (TAPE) + kda_verify: y and tape to rounding, the
+    conv window bit for bit; rolling back with it equals the unfused rollback exactly."""
+    B, H, d, Tb = 3, 4, 64, 8
+    cfg, P, A, S0, hist = make_case(13, [1] * B, H, d, 4, dtype, state_var=0.01,
+                                    conv_hist=True, chunk=16)
+    D = synth.layer_activations(13, [Tb] * B, H, d, dtype, tag='drafts')
+    dev = 'cuda'
+    Pd = {k: v.to(dev) for k, v in P.items()}
+    st = S0.to(dev)
+    cs = hist.to(dev)
+    v4 = lambda t, *tail: t.to(dev).reshape(B, Tb, *tail).contiguous()
+    y_f, tape_f, win_f = kda.kda_layer_verify(
+        cfg, v4(D['x'], H, 3 * d), v4(D['f'], H, d), v4(D['beta_logit'], H), v4(D['g'], H, d),
+        Pd['conv_w'], Pd['A_log'], Pd['dt_bias'], Pd['norm_w'], st, conv_state=cs)
+    p = kda.kda_prep(cfg, D['cu_seqlens'].to(dev), D['x'].to(dev), D['f'].to(dev),
+                     D['beta_logit'].to(dev), Pd['conv_w'], Pd['A_log'], Pd['dt_bias'],
+                     conv_state=cs, conv_mode=kda.KDA_CONV_TAPE, max_seqlen=Tb)
+    y_u, tape_u = kda.kda_verify(cfg, p['q'].view(B, Tb, H, d), p['k'].view(B, Tb, H, d),
+                                 p['v'].view(B, Tb, H, d), p['log_a'].view(B, Tb, H, d),
+                                 p['beta'].view(B, Tb, H), v4(D['g'], H, d), Pd['norm_w'], st)
+    torch.cuda.synchronize()
+    assert torch.equal(win_f.cpu().reshape(p['window'].shape), p['window'].cpu())
+    assert torch.equal(st.cpu(), S0) and torch.equal(cs.cpu(), hist)   # read only
+    tol = TOL[dtype]
+    assert rel_err(np64(y_f), np64(y_u)) <= tol
+    assert rel_err(np64(tape_f), np64(tape_u)) <= tol
+    acc = torch.tensor([0, 3, 8], dtype=torch.int32, device=dev)
+    s1, c1 = st.clone(), cs.clone()
+    kda.kda_rollback(cfg, acc, tape_f, s1, conv_window=win_f, conv_state=c1)
+    torch.cuda.synchronize()
+    assert torch.equal(s1[0].cpu(), S0[0]) and torch.equal(c1[0].cpu(), hist[0])
+    for b, L in ((1, 3), (2, 8)):
+        assert torch.equal(s1[b], tape_f[b, L - 1])
+        assert torch.equal(c1[b], win_f[b, L:L + 3])
