@@ -58,8 +58,10 @@ constexpr uint32_t TILE32 = 64 * AF_LD * 4;
 constexpr uint32_t OFF_XS = OFF_GA + 16384;  // X = (I + A)^{-1}, fp32 [64][68], after the gram
 constexpr uint32_t OFF_ZS = OFF_XS + TILE32; // per-warp block products of the solve
 constexpr int ZW_LD = 72;                    // their row stride (floats): fragment reads spread banks
+constexpr int Z32_LD = 40;                   // the 32 x 32 block product, same bank spread
 constexpr uint32_t SMEM_BYTES = OFF_G + 32768 + 1024;
-static_assert(OFF_ZS + 6 * 16 * ZW_LD * 4 <= OFF_GB, "solve tiles must fit in the gram A area");
+static_assert(OFF_ZS + (4 * 16 * ZW_LD + 32 * Z32_LD) * 4 <= OFF_GB,
+              "solve tiles must fit in the gram A area");
 static_assert(TILE32 <= 32768, "A must fit in the G area");
 
 __device__ __forceinline__ uint32_t gram_off(int n, int c) {   // tf32 K-major, K = 128
@@ -535,12 +537,14 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     for (int j = 0; j < 32; ++j) Mo[j * C + 32 + lane] = __float2bfloat16_rn(0.f);
   }
   tc_fence_before();
-  __syncthreads();
+  // the diagonal blocks of A come from warps 0 and 2: the substitution below (warps 0-1)
+  // starts once warps 0-2 are done, while the M rows are still being written
+  if (warp < 3) asm volatile("bar.sync 9, 96;" ::: "memory");
 
   // ---- T = (I + A)^{-1} diag(b), with A strictly lower triangular, by 16 x 16 blocks ----
   // X = (I + A)^{-1}: the four diagonal blocks by forward substitution (one thread per
-  // column), then the blocks below, one block diagonal at a time:
-  //   X_ab = -X_aa sum_{k=b}^{a-1} A_ak X_kb      (a > b)
+  // column), then the blocks below (X_ab = -X_aa sum_{k=b}^{a-1} A_ak X_kb for a > b),
+  // organised as two levels of 32 x 32 doubling
   if (tid < 64) {
     const int b = tid >> 4, jj = tid & 15;
     const float* Ab = Af + (16 * b) * AF_LD + 16 * b;
@@ -557,43 +561,74 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   }
   __syncthreads();
   {
-    // one warp per (block, 8-column half): Z = sum_k A_ak X_kb, then X_ab = -X_aa Z, as
-    // m16n8k8 tf32 tensor-core products split 3 ways (hi.hi + hi.lo + lo.hi ~ fp32)
+    // Below the diagonal in two levels (m16n8k8 tf32 tensor-core products split three
+    // ways, hi.hi + hi.lo + lo.hi ~ fp32; one warp per 16 x 8 output tile):
+    //  1. inside each 32-row half: X_10 = -X_11 (A_10 X_00), X_32 = -X_33 (A_32 X_22)
+    //  2. the lower-left 32 x 32 block: X_BA = -X_BB (A_BA X_AA), A = rows/cols 0-31,
+    //     B = rows/cols 32-63, through Z = A_BA X_AA
     const int g = lane >> 2, t = lane & 3;
     float* Zw = reinterpret_cast<float*>(sm + OFF_ZS) + warp * 16 * ZW_LD;
-#pragma unroll 1
-    for (int dg = 1; dg < 4; ++dg) {
-      if (warp < 2 * (4 - dg)) {
-        const int ab = (warp >> 1) + dg, bb = warp >> 1, n0 = 16 * bb + 8 * (warp & 1);
-        float z[3][4] = {};
+    float* Z32 = reinterpret_cast<float*>(sm + OFF_ZS) + 4 * 16 * ZW_LD;   // [32][Z32_LD]
+    if (warp < 4) {
+      const int ab = 2 * (warp >> 1) + 1, bb = ab - 1, n0 = 16 * bb + 8 * (warp & 1);
+      float z[3][4] = {};
 #pragma unroll
-        for (int kk = 0; kk < 3; ++kk)
-          if (kk < dg) {
-            const int kb = bb + kk;
+      for (int ks = 0; ks < 2; ++ks)
+        mma3_tf32(z, Af + (16 * ab) * AF_LD + 16 * bb + 8 * ks, AF_LD,
+                  Xs + (16 * bb + 8 * ks) * AF_LD + n0, AF_LD, g, t);
+      Zw[g * ZW_LD + 2 * t] = sum3(z, 0);
+      Zw[g * ZW_LD + 2 * t + 1] = sum3(z, 1);
+      Zw[(g + 8) * ZW_LD + 2 * t] = sum3(z, 2);
+      Zw[(g + 8) * ZW_LD + 2 * t + 1] = sum3(z, 3);
+      __syncwarp();
+      float y[3][4] = {};
 #pragma unroll
-            for (int ks = 0; ks < 2; ++ks)
-              mma3_tf32(z, Af + (16 * ab) * AF_LD + 16 * kb + 8 * ks, AF_LD,
-                        Xs + (16 * kb + 8 * ks) * AF_LD + n0, AF_LD, g, t);
-          }
-        Zw[g * ZW_LD + 2 * t] = sum3(z, 0);
-        Zw[g * ZW_LD + 2 * t + 1] = sum3(z, 1);
-        Zw[(g + 8) * ZW_LD + 2 * t] = sum3(z, 2);
-        Zw[(g + 8) * ZW_LD + 2 * t + 1] = sum3(z, 3);
-        __syncwarp();
-        float y[3][4] = {};
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks)
-          mma3_tf32(y, Xs + (16 * ab) * AF_LD + 16 * ab + 8 * ks, AF_LD, Zw + (8 * ks) * ZW_LD,
-                    ZW_LD, g, t);
-        float* xo = Xs + (16 * ab + g) * AF_LD + n0 + 2 * t;
-        xo[0] = -sum3(y, 0);
-        xo[1] = -sum3(y, 1);
-        xo[8 * AF_LD] = -sum3(y, 2);
-        xo[8 * AF_LD + 1] = -sum3(y, 3);
-        __syncwarp();
-      }
-      __syncthreads();
+      for (int ks = 0; ks < 2; ++ks)
+        mma3_tf32(y, Xs + (16 * ab) * AF_LD + 16 * ab + 8 * ks, AF_LD, Zw + (8 * ks) * ZW_LD,
+                  ZW_LD, g, t);
+      float* xo = Xs + (16 * ab + g) * AF_LD + n0 + 2 * t;
+      xo[0] = -sum3(y, 0);
+      xo[1] = -sum3(y, 1);
+      xo[8 * AF_LD] = -sum3(y, 2);
+      xo[8 * AF_LD + 1] = -sum3(y, 3);
     }
+    __syncthreads();
+    // warp w < 8: 16-row block i = w / 4 of B, 16-column block j of A, 8-column half
+    const int bi = warp >> 2, bj = (warp >> 1) & 1, n0 = 16 * bj + 8 * (warp & 1);
+    if (warp < 8) {   // Z_ij = sum_{k >= j} A_{2+i,k} X_kj
+      float z[3][4] = {};
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        if (k >= bj) {
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks)
+            mma3_tf32(z, Af + (32 + 16 * bi) * AF_LD + 16 * k + 8 * ks, AF_LD,
+                      Xs + (16 * k + 8 * ks) * AF_LD + n0, AF_LD, g, t);
+        }
+      float* zo = Z32 + (16 * bi + g) * Z32_LD + n0 + 2 * t;
+      zo[0] = sum3(z, 0);
+      zo[1] = sum3(z, 1);
+      zo[8 * Z32_LD] = sum3(z, 2);
+      zo[8 * Z32_LD + 1] = sum3(z, 3);
+    }
+    __syncthreads();
+    if (warp < 8) {   // X_{2+i,j} = -sum_{k <= i} X_{2+i,2+k} Z_kj
+      float y[3][4] = {};
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        if (k <= bi) {
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks)
+            mma3_tf32(y, Xs + (32 + 16 * bi) * AF_LD + 32 + 16 * k + 8 * ks, AF_LD,
+                      Z32 + (16 * k + 8 * ks) * Z32_LD + n0, Z32_LD, g, t);
+        }
+      float* xo = Xs + (32 + 16 * bi + g) * AF_LD + n0 + 2 * t;
+      xo[0] = -sum3(y, 0);
+      xo[1] = -sum3(y, 1);
+      xo[8 * AF_LD] = -sum3(y, 2);
+      xo[8 * AF_LD + 1] = -sum3(y, 3);
+    }
+    __syncthreads();
   }
   // T[r][j] = X[r][j] b_j for j <= r (else 0), as bf16 high and low parts, K-major [r][j]
 #pragma unroll
