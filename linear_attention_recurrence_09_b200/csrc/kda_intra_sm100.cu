@@ -168,13 +168,39 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   __shared__ __align__(8) uint64_t bar_mma;
   __shared__ volatile int abort_flag;
 
-  const int h = blockIdx.y, H = a.H, slot = blockIdx.x;
-  const TileRange tr = slot_to_tile(a.cu, a.n_seqs, a.total, C, slot);
-  if (tr.len == 0) return;
-  const int prow = pool_row(a.slots, tr.seq, a.pool_size);
-  if (prow < 0) return;
-  const int L = tr.len, t0 = tr.t0;
+  const int H = a.H, nslots = a.L.nslots;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int* status = reinterpret_cast<int*>(a.ws + a.L.status);
+
+  // once per CTA: the MMA barrier and 128 TMEM columns, kept across tiles
+  if (tid == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar_mma), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&tmem_holder)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_holder;
+  int issued = 0;   // MMA batches committed by thread 0 (two per tile)
+
+  // persistent: tile index = head x slots + slot, strided over the grid
+  const int ntiles = nslots * H;
+#pragma unroll 1
+  for (int tl = blockIdx.x; tl < ntiles; tl += gridDim.x) {
+  const int h = tl / nslots, slot = tl % nslots;
+  const TileRange tr = slot_to_tile(a.cu, a.n_seqs, a.total, C, slot);
+  if (tr.len == 0) continue;
+  const int prow = pool_row(a.slots, tr.seq, a.pool_size);
+  if (prow < 0) continue;
+  const int L = tr.len, t0 = tr.t0;
   const size_t tile = (size_t)slot * H + h;
   __nv_bfloat16* Wo = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.W) + tile * C * D;
   __nv_bfloat16* Uo = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.Ut) + tile * C * D;
@@ -182,7 +208,6 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   __nv_bfloat16* Ko = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.Kp) + tile * C * D;
   __nv_bfloat16* Mo = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.M) + tile * C * C;
   float* gCo = reinterpret_cast<float*>(a.ws + a.L.gC) + tile * D;
-  int* status = reinterpret_cast<int*>(a.ws + a.L.status);
   float* G = reinterpret_cast<float*>(sm + OFF_G);
   float* Af = G;                                  // [64][AF_LD], after the gram
   float* Xs = reinterpret_cast<float*>(sm + OFF_XS);
@@ -206,19 +231,6 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   if (FUSED) {
     A_log_h = __ldg(a.A_log + h);
     dtb = *reinterpret_cast<const float2*>(a.dt_bias + (size_t)h * D + cp);
-  }
-
-  if (tid == 0) {
-    abort_flag = 0;
-    mbar_init(smem_u32(&bar_mma), 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(&tmem_holder)),
-                 "r"(TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
 
   // ---- inputs of the token-row pass, issued now so their latency overlaps the gates
@@ -277,12 +289,12 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   // ---- log decay and its running sum G over the chunk, in log2 units (G log2 e):
   // channels 2p, 2p+1, rows 8q..8q+7 per thread ----
   {
-    // while the gate loads are in flight: pull into L2 the inputs of the tile one wave of
-    // CTAs ahead in the grid (it will run after this one), 128-byte lines spread over threads
-    if (a.pf_stride > 0) {
-      const long long nid = (long long)blockIdx.y * gridDim.x + blockIdx.x + a.pf_stride;
-      if (nid < (long long)gridDim.x * gridDim.y) {
-        const int nh = (int)(nid / gridDim.x), ns = (int)(nid % gridDim.x);
+    // while the gate loads are in flight: pull into L2 the inputs of this CTA's next tile,
+    // 128-byte lines spread over the threads
+    {
+      const int nid = tl + gridDim.x;   // this CTA's next tile
+      if (nid < ntiles) {
+        const int nh = nid / nslots, ns = nid % nslots;
         // same sequence (slots of a sequence are consecutive): no search
         const int nc = tr.chunk + (ns - slot);
         TileRange nt;
@@ -360,10 +372,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     if (qr == 7)
       *reinterpret_cast<float2*>(gCo + cp) = make_float2(ex2a(g0[7] + o0), ex2a(g1[7] + o1));
   }
-  tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_holder;
 
   // ---- token rows, in pairs: (prep), operands for the MMAs, Q~ and K' ----
   {
@@ -492,7 +501,6 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   __syncthreads();
 
   // ---- gram MMA (tf32, 128 x 128 x 128) ----
-  int issued = 0;   // MMA batches committed by thread 0
   if (tid == 0) {
     tc_fence_after();
     const uint32_t id = idesc_tf32(128, 128);
@@ -501,7 +509,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
       umma_tf32(tmem, sw128_desc(sb + OFF_GA + (s >> 2) * 16384 + (s & 3) * 32),
                 sw128_desc(sb + OFF_GB + (s >> 2) * 16384 + (s & 3) * 32), id, s > 0);
     umma_commit(smem_u32(&bar_mma));
-    issued = 1;
+    ++issued;
   }
   bool ok = mbar_wait_warp(smem_u32(&bar_mma), 0, &abort_flag);
   tc_fence_after();
@@ -677,7 +685,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
       umma(tmem + 64, sw128_mn_desc(sb + OFF_VT + s * 2048, 8192),
            sw128_desc(sb + OFF_TL + s * 32), id, 1);
     umma_commit(smem_u32(&bar_mma));
-    issued = 2;
+    ++issued;
   }
   if (ok) ok = mbar_wait_warp(smem_u32(&bar_mma), 1, &abort_flag);
   tc_fence_after();
@@ -695,7 +703,10 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   }
 
   tc_fence_before();
-  __syncthreads();
+  __syncthreads();   // this tile's shared memory and TMEM are free for the next one
+  if (abort_flag) break;
+  }   // tiles
+
   if (abort_flag && tid == 0) {
     // let the last issued MMA batch retire before TMEM is released (bounded), then report
     if (issued > 0) {
@@ -724,9 +735,11 @@ cudaError_t launch_intra_t(const PrefillArgs& a, cudaStream_t st) {
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return e;
-  PrefillArgs b = a;
-  b.pf_stride = nsm;   // one CTA per SM (shared memory bound): the next wave is nsm ahead
-  intra_chunk_sm100_kernel<FUSED><<<dim3(a.L.nslots, a.H), THREADS, SMEM_BYTES, st>>>(b);
+  // persistent: one CTA per SM (shared memory allows one), each looping over tiles
+  const long long ntiles = (long long)a.L.nslots * a.H;
+  const unsigned grid = (unsigned)(ntiles < nsm ? ntiles : nsm);
+  if (grid == 0) return cudaSuccess;
+  intra_chunk_sm100_kernel<FUSED><<<grid, THREADS, SMEM_BYTES, st>>>(a);
   ++launch_counter();
   return cudaGetLastError();
 }

@@ -109,7 +109,6 @@ struct PrefillArgs {
   const float* dt_bias;
   const void* conv_state;   // [pool, K-1, H, 3d] history, or nullptr for zeros
   int K;
-  int pf_stride;            // grid distance of the tile whose inputs a CTA prefetches (0: none)
 };
 
 cudaError_t launch_prep(const PrepArgs& a, cudaStream_t st);
