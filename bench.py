@@ -190,6 +190,15 @@ def prefill_workload(torch, kda, synth, T, seed, dev):
 PHASES = ('intra_chunk', 'inter_chunk', 'gated_norm')
 
 
+def prefill_config(T, H, d, world):
+    """The headline workload's description, shared by both arms."""
+    return {'workload': f'prefill B=1 H={H} T={T} d={d} chunk=64 conv=4 (one KDA layer: prep, '
+                        'chunked recurrence, gated RMSNorm)',
+            'global_batch': world, 'seq_len': T, 'heads': H, 'head_dim': d,
+            'parallelism': f'replicas x{world} (independent batches per GPU)',
+            'l2': f'inputs larger than L2 (x alone is {T * H * 3 * d * 2 / 1e6:.0f} MB)'}
+
+
 def prefill_bytes(T, H, d, C=64, K=4, fused_norm=True):
     """Algorithmic HBM bytes per launch of each pass of kda_layer_prefill (bf16
     activations, fp32 state, bf16 chunk tiles), and of the layer as a whole (inputs x,
@@ -299,11 +308,7 @@ def run_prefill(args, dist, torch, kda, synth, dev):
         'steps': args.steps, 'warmup': args.warmup, 'ms_per_step': ms_step,
         'higher_is_better': True, 'scaling': 'weak', 'vs_baseline': None, 'dtype': 'bf16',
         'data': 'synthetic (seeded N(0,1) activations, random-init layer parameters)',
-        'config': {'workload': f'prefill B=1 H=32 T={T} d=128 chunk=64 conv=4 '
-                               '(kda_layer_prefill: prep fused into the intra-chunk pass)',
-                   'global_batch': dist.world, 'seq_len': T, 'heads': H, 'head_dim': d,
-                   'parallelism': f'replicas x{dist.world} (independent batches per GPU)',
-                   'l2': 'inputs larger than L2 (x alone is %.0f MB)' % (A['x'].numel() * 2 / 1e6)},
+        'config': prefill_config(T, H, d, dist.world),
         'e2e': {'value': dist.world * T / (e2e_ms / 1e3), 'unit': 'tokens/s',
                 'h2d_bytes_per_step': h2d, 'd2h_bytes_per_step': d2h,
                 'ms_per_step': e2e_ms},
@@ -525,7 +530,7 @@ def run_reference(args, dist):
             'n_gpus': dist.world, 'steps': args.steps, 'warmup': args.warmup,
             'ms_per_step': statistics.mean(walls) * 1e3, 'higher_is_better': True,
             'scaling': 'weak', 'vs_baseline': None, 'dtype': 'f64', 'data': 'synthetic',
-            'config': {'workload': 'prefill B=1 H=32 T=8192 d=128 (sampled: 256-token prefix)'},
+            'config': prefill_config(8192, 32, 128, dist.world),
             'cpu_baseline': cb,
             'e2e': {'value': tps, 'unit': 'tokens/s', 'h2d_bytes_per_step': 0,
                     'd2h_bytes_per_step': 0}}
