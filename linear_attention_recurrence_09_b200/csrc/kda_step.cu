@@ -70,6 +70,13 @@ step_kernel(const StepArgs a) {
   const T* __restrict__ gg = static_cast<const T*>(a.g);
   T* __restrict__ yg = static_cast<T*>(a.y);
 
+  // the state streams in first: everything below (the prep of the first token
+  // included) runs while it arrives
+  const float* Sg = a.state_in + ((size_t)row * H + h) * D * D;
+  float4 S[ROWS];
+#pragma unroll
+  for (int i = 0; i < ROWS; ++i) S[i] = ld4(Sg + (size_t)(rg + i * RG) * D + 4 * cg);
+
   constexpr int C3 = 3 * D;
   const int Km1 = PREP ? a.K - 1 : 0;
   T* csg = PREP ? static_cast<T*>(a.conv_state) : nullptr;
@@ -86,11 +93,6 @@ step_kernel(const StepArgs a) {
     }
     __syncthreads();   // loaded by (row, channel) pairs, used per channel below
   }
-  // the state streams in while the (first token's) prep runs
-  const float* Sg = a.state_in + ((size_t)row * H + h) * D * D;
-  float4 S[ROWS];
-#pragma unroll
-  for (int i = 0; i < ROWS; ++i) S[i] = ld4(Sg + (size_t)(rg + i * RG) * D + 4 * cg);
 
   for (int t = 0; t < a.T; ++t) {
     const size_t tok = (size_t)b * a.T + t;
