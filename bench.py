@@ -143,8 +143,6 @@ PROFILED = {
                     'linear_attention_recurrence_09_b200/csrc/kda_intra_sm100.cu'),
     'inter_chunk': ('profiles/interchunk_sm100_prefill_8k.md',
                     'linear_attention_recurrence_09_b200/csrc/kda_prefill_sm100.cu'),
-    'gated_norm': ('profiles/gated_norm_prefill_8k.md',
-                   'linear_attention_recurrence_09_b200/csrc/kda_prefill.cu'),
     'kda_decode': ('profiles/step_decode_b64.md',
                    'linear_attention_recurrence_09_b200/csrc/kda_step.cu'),
     'kda_verify': ('profiles/step_verify_b16.md',
