@@ -494,7 +494,7 @@ def oracle_sample(torch, synth, heads=32, tokens=2048, seed=1):
     return units
 
 
-def cpu_baseline(torch, synth, heads=32, tokens=2048):
+def cpu_baseline(torch, synth, heads=32, tokens=4096):
     from oracle import baseline
     units = oracle_sample(torch, synth, heads, tokens)
     wall, workers = baseline.time_units(units)
@@ -504,7 +504,7 @@ def cpu_baseline(torch, synth, heads=32, tokens=2048):
             'sample': f'float64 oracle layer (prep + token loop + gated RMSNorm) on {heads} of 32 '
                       f'heads x the first {tokens} tokens of the headline workload, one head per '
                       f'process; value scaled to whole tokens (all 32 heads)',
-            'wall_s': wall}
+            'wall_s': wall, 'cpu_s': wall * workers}
 
 
 def run_reference(args, dist):
