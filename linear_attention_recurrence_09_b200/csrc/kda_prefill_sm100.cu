@@ -493,8 +493,8 @@ bool sm100_interchunk_supported(const PrefillArgs& a) {
   return a.bf16 && a.D == D && a.C == C;
 }
 
-// the fused norm needs the 4-CTA clusters of all heads (and sequences) resident in one
-// wave whenever the plain launch would be; decided once per device
+// the fused norm runs 4-CTA clusters; it is used unless it needs more waves of CTAs than
+// the plain launch (the cluster occupancy is queried once per device)
 static bool fuse_norm_fits(int clusters) {
   static int max_clusters[64];
   static bool known[64];
@@ -523,8 +523,11 @@ static bool fuse_norm_fits(int clusters) {
   }
   int nsm = 0;
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  const int plain_wave = nsm / NSLICE;   // heads x sequences one plain wave holds
-  return max_clusters[dev] >= (clusters < plain_wave ? clusters : plain_wave);
+  if (max_clusters[dev] < 1 || nsm < NSLICE) return false;
+  // fuse unless it needs more waves of CTAs than the plain launch (one CTA per SM)
+  const long long plain_waves = ((long long)clusters * NSLICE + nsm - 1) / nsm;
+  const long long fused_waves = ((long long)clusters + max_clusters[dev] - 1) / max_clusters[dev];
+  return fused_waves <= plain_waves;
 }
 
 cudaError_t launch_interchunk_sm100(const PrefillArgs& a, cudaStream_t st, bool* fused_norm) {
