@@ -383,3 +383,34 @@ def test_layer_verify_fused_prep_and_rollback(dtype):
     for b, L in ((1, 3), (2, 8)):
         assert torch.equal(s1[b], tape_f[b, L - 1])
         assert torch.equal(c1[b], win_f[b, L:L + 3])
+
+
+@pytest.mark.parametrize('fused', [True, False])
+def test_maximal_decay_gate_bf16(fused):
+    """Every gate at its lower bound (f large: log a = lb = -5 per token and channel), the
+    widest exponent range inside a chunk (G spans -320 over 64 tokens): the reference-row
+    split of the tcgen05 gram must stay exact, and the state forgets at e^-5 per token."""
+    cfg, P, A, S0, hist = make_case(14, [64, 130, 7], 4, 128, 4, torch.bfloat16, state_var=0.01,
+                                    conv_hist=True, chunk=64)
+    A['f'] = torch.full_like(A['f'], 30.0)
+    _assert(compare_layer(cfg, P, A, S0, hist, fused=fused), 1e-2)
+
+
+def test_mixed_decay_gate_bf16():
+    """Gates alternating between no decay and the lower bound along the chunk and across
+    channels (G jumps by 5 between neighbouring tokens on half the channels)."""
+    cfg, P, A, S0, hist = make_case(15, [200], 4, 128, 4, torch.bfloat16, state_var=0.01,
+                                    conv_hist=True, chunk=64)
+    f = torch.full_like(A['f'], -30.0)
+    f[::2, :, ::2] = 30.0
+    A['f'] = f
+    _assert(compare_layer(cfg, P, A, S0, hist), 1e-2)
+
+
+@pytest.mark.parametrize('fused', [True, False])
+def test_q_scale_bf16(fused):
+    """q_scale != 1 (folded into the q normalisation on the fused path)."""
+    cfg, P, A, S0, hist = make_case(16, [90, 33], 4, 128, 4, torch.bfloat16, state_var=0.01,
+                                    conv_hist=True, chunk=64)
+    cfg.q_scale = 128 ** -0.5
+    _assert(compare_layer(cfg, P, A, S0, hist, fused=fused), 1e-2)
