@@ -27,9 +27,12 @@
 //     rounding of T and K e^G was the largest term left in the error budget.
 // Q~ = q_scale Q e^G, K' = K e^{G_C - G} and e^{G_C} are elementwise.  16 warps: warps
 // w and w + 8 walk token rows 8(w%8)..8(w%8)+7 in pairs, each owning 64 of the 128
-// channels of q, k and v (two per lane); the per-token L2 norms are warp shuffles plus
-// one exchange with the partner warp per row pair, and the conv keeps its window of
-// K-1 previous rows in registers.
+// channels of q, k and v (two per lane, one packed f32x2 pair); the per-token L2 norms are
+// a shuffle reduce-scatter plus one exchange with the partner warp per row pair, and the
+// conv keeps its window of K-1 previous rows in registers.  Per row and channel the row
+// pass takes three exponentials: e^{G_r - G_ref} and its reciprocal give the gram scalings,
+// e^{G_r} is e^{G_15} times the first (rows 0-31) and e^{G_C - G_r} is e^{G_C - G_47} times
+// e^{G_47 - G_r} (both factors stay above 2^-116 with the gate bounded below by -5).
 #include <type_traits>
 
 #include "kda_common.cuh"
@@ -64,22 +67,11 @@ static_assert(OFF_ZS + (4 * 16 * ZW_LD + 32 * Z32_LD) * 4 <= OFF_GB,
               "solve tiles must fit in the gram A area");
 static_assert(TILE32 <= 32768, "A must fit in the G area");
 
-__device__ __forceinline__ uint32_t gram_off(int n, int c) {   // tf32 K-major, K = 128
-  return (uint32_t)((c >> 5) * 16384) + sw128_off32(n, c & 31);
-}
-__device__ __forceinline__ uint32_t mn_off(int t, int c) {     // bf16 MN-major [t][c]
-  const int row = t & 7;
-  return (uint32_t)((c >> 6) * 8192 + (t >> 3) * 1024 + row * 128 +
-                    (((((c & 63) >> 3) ^ row) & 7) << 4) + (c & 7) * 2);
-}
 
 // fp32 -> nearest tf32 (10 mantissa bits, ties away from zero: the rounding of
 // cvt.rna.tf32.f32) with two integer operations on the bit pattern; finite inputs only
 __device__ __forceinline__ float tf32_rna(float x) {
   return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xffffe000u);
-}
-__device__ __forceinline__ void st_tf32x2(unsigned char* p, float a, float b) {
-  *reinterpret_cast<float2*>(p) = make_float2(tf32_rna(a), tf32_rna(b));
 }
 __device__ __forceinline__ void st_bf16x2(void* p, float a, float b) {
   *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
@@ -149,11 +141,61 @@ __device__ __forceinline__ float2 to_f2(uint32_t v) {
   return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+// Two fp32 values in one 64-bit register pair, for the packed f32x2 arithmetic of sm_100
+// (both halves rounded as the scalar instruction would round them)
+typedef unsigned long long f2x;
+__device__ __forceinline__ f2x pk2(float lo, float hi) {
+  f2x r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 up2(f2x v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ f2x fma2(f2x a, f2x b, f2x c) {
+  f2x d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f2x mul2(f2x a, f2x b) {
+  f2x d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2x add2(f2x a, f2x b) {
+  f2x d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2x sub2(f2x a, f2x b) {
+  f2x d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// a pair rounded to tf32 / bf16 and stored (shared memory by 32-bit address, or global)
+__device__ __forceinline__ void st_tf32p(uint32_t saddr, f2x v) {
+  const float2 t = up2(v);
+  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(saddr), "f"(tf32_rna(t.x)),
+               "f"(tf32_rna(t.y))
+               : "memory");
+}
+__device__ __forceinline__ void st_bf16p(uint32_t saddr, f2x v) {
+  const float2 t = up2(v);
+  const __nv_bfloat162 b = __floats2bfloat162_rn(t.x, t.y);
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(saddr), "r"(*reinterpret_cast<const uint32_t*>(&b))
+               : "memory");
+}
+__device__ __forceinline__ void st_shared_b32(uint32_t saddr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(saddr), "r"(v) : "memory");
+}
+__device__ __forceinline__ f2x ld_shared_f2x(uint32_t saddr) {
+  f2x v;
+  asm volatile("ld.shared.b64 %0, [%1];" : "=l"(v) : "r"(saddr) : "memory");
   return v;
 }
+
 
 template <bool FUSED>
 __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const PrefillArgs a) {
@@ -193,13 +235,40 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
 
   // persistent: tile index = head x slots + slot, strided over the grid
   const int ntiles = nslots * H;
+  // The next tile's range and state row are looked up by one thread during the gram MMA
+  // and published here, so that a tile starts without that round trip to memory.
+  __shared__ int next_meta[8];   // seq, start, end, t0, len, chunk, state row, valid
+  using GRawT = typename std::conditional<FUSED, uint32_t, float2>::type;   // 2 gate channels as loaded
+  GRawT graw[8];
+  bool have_meta = false;
+  const int cp = 2 * (tid & 63), qr = tid >> 6;   // gate pass: channels cp, cp+1 of rows 8qr..8qr+7
+  // gate inputs (f, or log a) of tile rows 8qr..8qr+7
+  auto load_gates = [&](const TileRange& r, int hd) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      graw[i] = GRawT{};
+      if (8 * qr + i < r.len) {
+        const size_t idx = ((size_t)(r.t0 + 8 * qr + i) * H + hd) * D + cp;
+        graw[i] = FUSED ? *reinterpret_cast<const GRawT*>(static_cast<const __nv_bfloat16*>(a.f) + idx)
+                        : *reinterpret_cast<const GRawT*>(a.loga + idx);
+      }
+    }
+  };
 #pragma unroll 1
   for (int tl = blockIdx.x; tl < ntiles; tl += gridDim.x) {
   const int h = tl / nslots, slot = tl % nslots;
-  const TileRange tr = slot_to_tile(a.cu, a.n_seqs, a.total, C, slot);
-  if (tr.len == 0) continue;
-  const int prow = pool_row(a.slots, tr.seq, a.pool_size);
-  if (prow < 0) continue;
+  TileRange tr;
+  int prow;
+  if (have_meta) {
+    tr.seq = next_meta[0]; tr.start = next_meta[1]; tr.end = next_meta[2];
+    tr.t0 = next_meta[3]; tr.len = next_meta[4]; tr.chunk = next_meta[5];
+    prow = next_meta[6];
+  } else {
+    tr = slot_to_tile(a.cu, a.n_seqs, a.total, C, slot);
+    prow = tr.len ? pool_row(a.slots, tr.seq, a.pool_size) : -1;
+  }
+  have_meta = false;
+  if (tr.len == 0 || prow < 0) continue;
   const int L = tr.len, t0 = tr.t0;
   const size_t tile = (size_t)slot * H + h;
   __nv_bfloat16* Wo = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.W) + tile * C * D;
@@ -212,20 +281,8 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   float* Af = G;                                  // [64][AF_LD], after the gram
   float* Xs = reinterpret_cast<float*>(sm + OFF_XS);
 
-  // gate inputs first (the gate pass waits on them): channels 2p, 2p+1 of rows 8q..8q+7
-  const int cp = 2 * (tid & 63), qr = tid >> 6;
-  float g0[8], g1[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = 8 * qr + i;
-    float2 v = make_float2(0.f, 0.f);
-    if (r < L) {
-      const size_t idx = ((size_t)(t0 + r) * H + h) * D + cp;
-      v = FUSED ? ld2(static_cast<const __nv_bfloat16*>(a.f) + idx) : ld2(a.loga + idx);
-    }
-    g0[i] = v.x;
-    g1[i] = v.y;
-  }
+  // gate inputs first (the gate pass waits on them)
+  load_gates(tr, h);
   float A_log_h = 0.f;
   float2 dtb = make_float2(0.f, 0.f);
   if (FUSED) {
@@ -326,20 +383,23 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
         }
       }
     }
+    float g0[8], g1[8];
     if (FUSED) {
       // log2 a = lb log2(e) sigmoid(exp(A_log) (f + dt_bias))
       const float Ah2 = expf(A_log_h) * LOG2E, lb2 = a.lb * LOG2E;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const bool live = 8 * qr + i < L;
-        g0[i] = live ? lb2 * sigmoid2(Ah2 * (g0[i] + dtb.x)) : 0.f;
-        g1[i] = live ? lb2 * sigmoid2(Ah2 * (g1[i] + dtb.y)) : 0.f;
+        const float2 v = to_f2(graw[i]);
+        g0[i] = live ? lb2 * sigmoid2(Ah2 * (v.x + dtb.x)) : 0.f;
+        g1[i] = live ? lb2 * sigmoid2(Ah2 * (v.y + dtb.y)) : 0.f;
       }
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        g0[i] *= LOG2E;
-        g1[i] *= LOG2E;
+        const float2 v = to_f2(graw[i]);
+        g0[i] = v.x * LOG2E;
+        g1[i] = v.y * LOG2E;
       }
     }
 #pragma unroll
@@ -375,93 +435,121 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   __syncthreads();
 
   // ---- token rows, in pairs: (prep), operands for the MMAs, Q~ and K' ----
+  // A lane's two channels travel as one packed pair through the f32x2 arithmetic.
   {
     // q, k and v leave the conv scaled by log2 e (taps pre-scaled): the L2 norm of q and k
     // cancels the factor (with eps scaled alike) and v takes ln 2 back
     const float qsc = a.q_scale, inv_eps = 1.0f / (a.l2_eps * LOG2E);
-    float win[KC - 1][6];   // previous pre-conv rows, oldest first: q0 q1 k0 k1 v0 v1
+    f2x cwp[3][KC];       // conv taps of channels c2, c2+1 per segment (q, k, v), oldest tap first
+    f2x win[KC - 1][3];   // previous pre-conv rows, oldest first, per segment
     if (FUSED) {
 #pragma unroll
-      for (int sgm = 0; sgm < 3; ++sgm)
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-          cw[sgm][j] = make_float4(cw[sgm][j].x * LOG2E, cw[sgm][j].y * LOG2E,
-                                   cw[sgm][j].z * LOG2E, cw[sgm][j].w * LOG2E);
+      for (int sgm = 0; sgm < 3; ++sgm) {
+        const float4 w0 = cw[sgm][0], w1 = cw[sgm][1];
+        cwp[sgm][0] = pk2(LOG2E * w0.x, LOG2E * w1.x);
+        cwp[sgm][1] = pk2(LOG2E * w0.y, LOG2E * w1.y);
+        cwp[sgm][2] = pk2(LOG2E * w0.z, LOG2E * w1.z);
+        cwp[sgm][3] = pk2(LOG2E * w0.w, LOG2E * w1.w);
+      }
 #pragma unroll
       for (int m = 0; m < KC - 1; ++m)
 #pragma unroll
         for (int sgm = 0; sgm < 3; ++sgm) {
           const float2 t = to_f2(winr[m][sgm]);
-          win[m][2 * sgm] = t.x;
-          win[m][2 * sgm + 1] = t.y;
+          win[m][sgm] = pk2(t.x, t.y);
         }
     }
-    const float2 g15 = *reinterpret_cast<const float2*>(G + 15 * D + c2);
-    const float2 g47 = *reinterpret_cast<const float2*>(G + 47 * D + c2);
-    const float2 g63 = *reinterpret_cast<const float2*>(G + 63 * D + c2);
-    const float r15[2] = {g15.x, g15.y}, r47[2] = {g47.x, g47.y}, r63[2] = {g63.x, g63.y};
+    // reference rows of the exponent split: row 15 for rows 0-31, row 47 for rows 32-63
+    const f2x R15 = *reinterpret_cast<const f2x*>(G + 15 * D + c2);
+    const f2x R47 = *reinterpret_cast<const f2x*>(G + 47 * D + c2);
+    const float2 r47 = up2(R47), r63 = *reinterpret_cast<const float2*>(G + 63 * D + c2);
+    const bool lowhalf = pr < 4;
+    const f2x RREF = lowhalf ? R15 : R47;
+    // 2^{G_15} and 2^{G_63 - G_47}: each spans at most 16 steps of the decay (lb >= -5), so
+    // both are >= 2^-116, normal fp32 numbers
+    const float2 r15 = up2(R15);
+    const f2x E15 = pk2(ex2a(r15.x), ex2a(r15.y));
+    const f2x C6347 = pk2(ex2a(r63.x - r47.x), ex2a(r63.y - r47.y));
+    const f2x ONE2 = pk2(1.f, 1.f), LN2_2 = pk2(LN2, LN2);
+    // shared-memory addresses: the per-thread part here, a row adds j * 128 and the swizzle
+    // of j = row & 7 (row = 8 pr + j).  Gram rows: a key at B row r (rows 0-31) or r + 32,
+    // its query 32 rows further; the column-scaled key at A row r (rows 0-31) and r + 32.
+    const int gq = (c2 & 31) >> 2, mq = (c2 & 63) >> 3;
+    const uint32_t gA = sb + OFF_GA + (c2 >> 5) * 16384 + (c2 & 3) * 4 + pr * 1024;
+    const uint32_t gB = sb + OFF_GB + (c2 >> 5) * 16384 + (c2 & 3) * 4 + pr * 1024 +
+                        (lowhalf ? 0 : 4096);
+    const uint32_t mB = sb + (c2 >> 6) * 8192 + pr * 1024 + (c2 & 7) * 2;
+    const uint32_t Grow = sb + OFF_G + (uint32_t)(8 * pr * D + c2) * 4;
 
     // depthwise conv (taps 0..K-2 on the window, K-1 on the row) and SiLU of one row;
     // the row then enters the window.  Returns the partial sums of squares of q and k.
-    auto conv_row = [&](RawT iq, RawT ik, RawT iv, float (&qv)[2], float (&kv)[2],
-                        float (&vv)[2]) -> float2 {
-      const float2 fq = to_f2(iq), fk = to_f2(ik), fv = to_f2(iv);
+    auto conv_row = [&](RawT iq, RawT ik, RawT iv, f2x& qv, f2x& kv, f2x& vv) -> float2 {
       if (!FUSED) {
-        qv[0] = qsc * fq.x; qv[1] = qsc * fq.y;
-        kv[0] = fk.x; kv[1] = fk.y;
-        vv[0] = fv.x; vv[1] = fv.y;
+        const float2 fq = to_f2(iq), fk = to_f2(ik), fv = to_f2(iv);
+        qv = pk2(qsc * fq.x, qsc * fq.y);
+        kv = pk2(fk.x, fk.y);
+        vv = pk2(fv.x, fv.y);
         return make_float2(0.f, 0.f);
       }
-      const float xr[6] = {fq.x, fq.y, fk.x, fk.y, fv.x, fv.y};
-      float z[6];
+      const RawT raw[3] = {iq, ik, iv};
+      f2x z[3];
 #pragma unroll
-      for (int e = 0; e < 6; ++e) {
-        const float4 w = cw[e >> 1][e & 1];
-        float acc = w.w * xr[e];
-        acc = fmaf(w.x, win[0][e], acc);
-        acc = fmaf(w.y, win[1][e], acc);
-        acc = fmaf(w.z, win[2][e], acc);
-        z[e] = acc * sigmoid2(acc);
-        win[0][e] = win[1][e];
-        win[1][e] = win[2][e];
-        win[2][e] = xr[e];
+      for (int sgm = 0; sgm < 3; ++sgm) {
+        const float2 xf = to_f2(raw[sgm]);
+        const f2x x = pk2(xf.x, xf.y);
+        f2x acc = mul2(cwp[sgm][KC - 1], x);
+        acc = fma2(cwp[sgm][0], win[0][sgm], acc);
+        acc = fma2(cwp[sgm][1], win[1][sgm], acc);
+        acc = fma2(cwp[sgm][2], win[2][sgm], acc);
+        // SiLU in log2 units: acc / (1 + 2^-acc)
+        const float2 af = up2(acc);
+        const float2 den = up2(add2(pk2(ex2a(-af.x), ex2a(-af.y)), ONE2));
+        z[sgm] = mul2(acc, pk2(rcpa(den.x), rcpa(den.y)));
+        win[0][sgm] = win[1][sgm];
+        win[1][sgm] = win[2][sgm];
+        win[2][sgm] = x;
       }
-      qv[0] = z[0]; qv[1] = z[1];
-      kv[0] = z[2]; kv[1] = z[3];
-      vv[0] = LN2 * z[4]; vv[1] = LN2 * z[5];
-      return make_float2(fmaf(z[0], z[0], z[1] * z[1]), fmaf(z[2], z[2], z[3] * z[3]));
+      qv = z[0];
+      kv = z[1];
+      vv = mul2(z[2], LN2_2);
+      const float2 q2 = up2(z[0]), k2 = up2(z[1]);
+      return make_float2(fmaf(q2.x, q2.x, q2.y * q2.y), fmaf(k2.x, k2.x, k2.y * k2.y));
     };
-    // every operand of one token row r for this lane's two channels
-    auto operands = [&](int r, const float (&qv)[2], const float (&kv)[2], const float (&vv)[2]) {
-      const float2 gr2 = *reinterpret_cast<const float2*>(G + r * D + c2);
-      const float gr[2] = {gr2.x, gr2.y};
-      const bool lowhalf = r < 32;
-      float kb[2], qb[2], kc0[2], kc1[2], qt[2], kt[2], kp[2];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const float g = gr[j];
-        const float er = ex2a(g - (lowhalf ? r15[j] : r47[j]));
-        kb[j] = kv[j] * er;
-        qb[j] = qv[j] * er;                       // qv carries q_scale
-        kc0[j] = lowhalf ? kv[j] * ex2a(r15[j] - g) : 0.f;
-        kc1[j] = kv[j] * ex2a(r47[j] - g);
-        const float eg = ex2a(g);
-        qt[j] = qv[j] * eg;
-        kt[j] = kv[j] * eg;
-        kp[j] = kv[j] * ex2a(r63[j] - g);
+    // every operand of token row 8 pr + j for this lane's two channels
+    auto operands = [&](int j, f2x qv, f2x kv, f2x vv) {
+      const f2x gr = ld_shared_f2x(Grow + j * D * 4);
+      // er = 2^{G_r - G_ref} and its reciprocal: |exponent| <= 80 log2 e, both in range
+      const float2 d = up2(sub2(gr, RREF));
+      const float er0 = ex2a(d.x), er1 = ex2a(d.y);
+      const f2x er = pk2(er0, er1), ei = pk2(rcpa(er0), rcpa(er1));
+      const f2x kb = mul2(kv, er), qb = mul2(qv, er);
+      f2x kc1, eg;   // k 2^{G_47 - G_r} and 2^{G_r}
+      if (lowhalf) {
+        const float2 d1 = up2(sub2(R47, gr));
+        kc1 = mul2(kv, pk2(ex2a(d1.x), ex2a(d1.y)));
+        eg = mul2(E15, er);   // 2^{G_15} 2^{G_r - G_15}; below 2^-126 it flushes to 0
+      } else {
+        kc1 = mul2(kv, ei);
+        const float2 g = up2(gr);
+        eg = pk2(ex2a(g.x), ex2a(g.y));
       }
-      const int nk = lowhalf ? r : 64 + (r - 32);
-      st_tf32x2(sm + OFF_GB + gram_off(nk, c2), kb[0], kb[1]);
-      st_tf32x2(sm + OFF_GB + gram_off(nk + 32, c2), qb[0], qb[1]);
-      if (lowhalf) st_tf32x2(sm + OFF_GA + gram_off(r, c2), kc0[0], kc0[1]);
-      st_tf32x2(sm + OFF_GA + gram_off(32 + r, c2), kc1[0], kc1[1]);
-      const __nv_bfloat162 hi = __floats2bfloat162_rn(kt[0], kt[1]);
+      const f2x qt = mul2(qv, eg), kt = mul2(kv, eg);
+      const f2x kp = mul2(kc1, C6347);   // k 2^{G_63 - G_r}
+      const int jo = j * 128 + (((gq ^ j) & 7) << 4);
+      st_tf32p(gB + jo, kb);
+      st_tf32p(gB + jo + 4096, qb);
+      if (lowhalf) st_tf32p(gA + jo, mul2(kv, ei));   // k 2^{G_15 - G_r}
+      st_tf32p(gA + jo + 4096, kc1);
+      const uint32_t mp = mB + j * 128 + (((mq ^ j) & 7) << 4);
+      const float2 ktf = up2(kt);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(ktf.x, ktf.y);
       const float2 hf = __bfloat1622float2(hi);
-      *reinterpret_cast<__nv_bfloat162*>(sm + OFF_KT + mn_off(r, c2)) = hi;
-      st_bf16x2(sm + OFF_KL + mn_off(r, c2), kt[0] - hf.x, kt[1] - hf.y);
-      st_bf16x2(sm + OFF_VT + mn_off(r, c2), vv[0], vv[1]);
-      st_bf16x2(Qo + (size_t)r * D + c2, qt[0], qt[1]);
-      st_bf16x2(Ko + (size_t)r * D + c2, kp[0], kp[1]);
+      st_shared_b32(mp + OFF_KT, *reinterpret_cast<const uint32_t*>(&hi));
+      st_bf16p(mp + OFF_KL, sub2(kt, pk2(hf.x, hf.y)));
+      st_bf16p(mp + OFF_VT, vv);
+      const float2 qtf = up2(qt), kpf = up2(kp);
+      st_bf16x2(Qo + (size_t)(8 * pr + j) * D + c2, qtf.x, qtf.y);
+      st_bf16x2(Ko + (size_t)(8 * pr + j) * D + c2, kpf.x, kpf.y);
     };
 
 #pragma unroll 1
@@ -470,29 +558,38 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
       RawT nq0, nk0, nv0, nq1, nk1, nv1;   // the next pair, in flight through this one
       load_row(k < 3 ? ra + 2 : C, nq0, nk0, nv0);
       load_row(k < 3 ? ra + 3 : C, nq1, nk1, nv1);
-      float qa[2], ka[2], va[2], qb2[2], kb2[2], vb2[2];
+      f2x qa, ka, va, qb2, kb2, vb2;
       const float2 sa = conv_row(aq, ak, av, qa, ka, va);
       const float2 sb = conv_row(bq, bk, bv, qb2, kb2, vb2);
       if (FUSED) {
-        // q and k norms over 128 channels: this warp's 64 (shuffles) + the partner warp's
-        float4 part = make_float4(warp_sum(sa.x), warp_sum(sa.y), warp_sum(sb.x), warp_sum(sb.y));
-        if (lane == 0) pnorm[pr][k & 1][hh] = part;
+        // q and k norms over 128 channels: the four sums of this warp's 64 channels by a
+        // reduce-scatter over the lanes (lane 8v ends with sum v), then the partner warp's
+        const bool b4 = lane & 16, b3 = lane & 8;
+        float k0 = b4 ? sb.x : sa.x, k1 = b4 ? sb.y : sa.y;
+        k0 += __shfl_xor_sync(0xffffffffu, b4 ? sa.x : sb.x, 16);
+        k1 += __shfl_xor_sync(0xffffffffu, b4 ? sa.y : sb.y, 16);
+        float m = (b3 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, b3 ? k0 : k1, 8);
+        m += __shfl_xor_sync(0xffffffffu, m, 4);
+        m += __shfl_xor_sync(0xffffffffu, m, 2);
+        m += __shfl_xor_sync(0xffffffffu, m, 1);
+        if ((lane & 7) == 0) reinterpret_cast<float*>(&pnorm[pr][k & 1][hh])[lane >> 3] = m;
         asm volatile("bar.sync %0, 64;" ::"r"(1 + pr) : "memory");
-        const float4 o = pnorm[pr][k & 1][hh ^ 1];
-        part.x += o.x; part.y += o.y; part.z += o.z; part.w += o.w;
+        const float4 o0 = pnorm[pr][k & 1][0], o1 = pnorm[pr][k & 1][1];
+        const float4 part = make_float4(o0.x + o1.x, o0.y + o1.y, o0.z + o1.z, o0.w + o1.w);
         // 1 / max(||x||, eps) = min(rsqrt(||x||^2), 1 / eps), rsqrt(0) = inf; q_scale folded
         const float iqa = ra < L ? qsc * fminf(rsqrta(part.x), inv_eps) : 0.f;
         const float ika = ra < L ? fminf(rsqrta(part.y), inv_eps) : 0.f;
         const float iqb = rb < L ? qsc * fminf(rsqrta(part.z), inv_eps) : 0.f;
         const float ikb = rb < L ? fminf(rsqrta(part.w), inv_eps) : 0.f;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          qa[j] *= iqa; ka[j] *= ika; va[j] = ra < L ? va[j] : 0.f;
-          qb2[j] *= iqb; kb2[j] *= ikb; vb2[j] = rb < L ? vb2[j] : 0.f;
-        }
+        qa = mul2(qa, pk2(iqa, iqa));
+        ka = mul2(ka, pk2(ika, ika));
+        qb2 = mul2(qb2, pk2(iqb, iqb));
+        kb2 = mul2(kb2, pk2(ikb, ikb));
+        if (ra >= L) va = 0ull;
+        if (rb >= L) vb2 = 0ull;
       }
-      operands(ra, qa, ka, va);
-      operands(rb, qb2, kb2, vb2);
+      operands(2 * k, qa, ka, va);
+      operands(2 * k + 1, qb2, kb2, vb2);
       aq = nq0; ak = nk0; av = nv0;
       bq = nq1; bk = nk1; bv = nv1;
     }
@@ -510,6 +607,18 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
                 sw128_desc(sb + OFF_GB + (s >> 2) * 16384 + (s & 3) * 32), id, s > 0);
     umma_commit(smem_u32(&bar_mma));
     ++issued;
+  }
+  if (tid == THREADS - 1) {   // the next tile's range, while the gram runs (read after later barriers)
+    const int nid = tl + gridDim.x;
+    TileRange nt{};
+    int np = -1;
+    if (nid < ntiles) {
+      nt = slot_to_tile(a.cu, a.n_seqs, a.total, C, nid % nslots);
+      np = nt.len ? pool_row(a.slots, nt.seq, a.pool_size) : -1;
+    }
+    next_meta[0] = nt.seq; next_meta[1] = nt.start; next_meta[2] = nt.end;
+    next_meta[3] = nt.t0; next_meta[4] = nt.len; next_meta[5] = nt.chunk;
+    next_meta[6] = np; next_meta[7] = nid < ntiles;
   }
   bool ok = mbar_wait_warp(smem_u32(&bar_mma), 0, &abort_flag);
   tc_fence_after();
@@ -687,6 +796,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     umma_commit(smem_u32(&bar_mma));
     ++issued;
   }
+  have_meta = next_meta[7] != 0;   // published before the barriers of the solve
   if (ok) ok = mbar_wait_warp(smem_u32(&bar_mma), 1, &abort_flag);
   tc_fence_after();
   if (ok) {
@@ -696,10 +806,14 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     const bool isW = (warp & 4) == 0;
     const int hf = warp >> 3;
     __nv_bfloat16* dst = isW ? Wo : Uo;
-    float v[32];
-    tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (isW ? 0u : 64u) + 32u * hf, v);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) dst[(size_t)(32 * hf + j) * D + c] = __float2bfloat16_rn(v[j]);
+    for (int part = 0; part < 2; ++part) {   // 16 columns at a time: the next tile's gates are live
+      float v[16];
+      tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (isW ? 0u : 64u) + 32u * hf + 16u * part, v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        dst[(size_t)(32 * hf + 16 * part + j) * D + c] = __float2bfloat16_rn(v[j]);
+    }
   }
 
   tc_fence_before();
