@@ -9,7 +9,8 @@
 //     conv over q|k|v, SiLU, q/k L2 norm with max(||x||, eps), bounded-sigmoid
 //     decay, sigmoid beta) runs here in fp32, so q/k/v never round-trip HBM.
 //
-// One CTA per (chunk slot, head).  With G the cumulative log decay of the chunk:
+// Persistent: one CTA per SM walks the (chunk slot, head) tiles.  With G the cumulative
+// log decay of the chunk:
 //   * Gram: A'[r,i] = sum_c k_r k_i e^{G_r - G_i} and M[r,i] = q_scale sum_c q_r k_i e^{G_r - G_i}.
 //     The exponent is split at a reference row, row 15 for rows 0-31 and row 47
 //     for rows 32-63: with the gate bounded below by -5, every factor is at most
@@ -18,7 +19,8 @@
 //     keys of both halves (32 + 64 rows), B rows the row-scaled keys and queries
 //     (4 x 32 rows); only the two diagonal blocks of the product are read.  tf32
 //     (not bf16) because the gram's rounding dominates the parity error budget.
-//   * T = (I + A)^{-1} diag(b) by forward substitution in fp32 (4 threads per column).
+//   * T = (I + A)^{-1} diag(b): forward substitution on the four 16 x 16 diagonal blocks,
+//     then two levels of 32 x 32 doubling on mma.sync tf32 products split three ways (~fp32).
 //   * W^T = (K e^G)^T T^T and U~^T = V^T T^T as bf16 MMAs, M = 128 (key / value
 //     channels), N = 64, K = 64 tokens, with K e^G and V read MN-major (stored
 //     token-major by the threads that compute them).  T and K e^G are each split
@@ -33,6 +35,8 @@
 // pass takes three exponentials: e^{G_r - G_ref} and its reciprocal give the gram scalings,
 // e^{G_r} is e^{G_15} times the first (rows 0-31) and e^{G_C - G_r} is e^{G_C - G_47} times
 // e^{G_47 - G_r} (both factors stay above 2^-116 with the gate bounded below by -5).
+// After a tile's row pass, warps 0-7 run its serial tail (gram readout, solve, W/U~) while
+// warps 8-15 compute the next tile's gates (G, beta, e^{G_C}): the next row pass starts at once.
 #include <type_traits>
 
 #include "kda_common.cuh"
@@ -53,7 +57,7 @@ constexpr uint32_t OFF_GB = 65536;      // gram B: same shape (64 KB)
 constexpr uint32_t OFF_KT = 131072;     // K e^G, high bf16 part: MN-major [64 t][128 c] (16 KB)
 constexpr uint32_t OFF_KL = 147456;     // K e^G, low bf16 part (the rounding remainder)
 constexpr uint32_t OFF_VT = 163840;     // V:     bf16 MN-major [64 t][128 c] (16 KB)
-constexpr uint32_t OFF_G = 180224;      // G fp32 [64][128] (32 KB); later A fp32 [64][65]
+constexpr uint32_t OFF_G = 180224;      // G fp32 [64][128] (32 KB), written a tile ahead
 constexpr uint32_t OFF_T = OFF_GA;      // T high part, bf16 K-major [64 r][64 i] (8 KB), after the gram
 constexpr uint32_t OFF_TL = OFF_GA + 8192;  // T low part
 constexpr int AF_LD = 68;                   // row stride (floats) of the fp32 tiles of the solve
@@ -65,7 +69,7 @@ constexpr int Z32_LD = 40;                   // the 32 x 32 block product, same 
 constexpr uint32_t SMEM_BYTES = OFF_G + 32768 + 1024;
 static_assert(OFF_ZS + (4 * 16 * ZW_LD + 32 * Z32_LD) * 4 <= OFF_GB,
               "solve tiles must fit in the gram A area");
-static_assert(TILE32 <= 32768, "A must fit in the G area");
+static_assert(TILE32 <= 65536, "A (fp32, after the gram) must fit in the gram B area");
 
 
 // fp32 -> nearest tf32 (10 mantissa bits, ties away from zero: the rounding of
@@ -203,8 +207,8 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sb = smem_u32(sm);
-  __shared__ float bs[C];
-  __shared__ float qsum[8][D];   // per-row-group totals of the log decay
+  __shared__ float bs[2][C];       // beta of the tile in flight and of the next one
+  __shared__ float qsum[4][D];     // gate pass: per-16-row-group totals of the log decay
   __shared__ float4 pnorm[8][2][2];   // q/k sums of squares of a row pair: [group][parity][half]
   __shared__ uint32_t tmem_holder;
   __shared__ __align__(8) uint64_t bar_mma;
@@ -233,68 +237,147 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   const uint32_t tmem = tmem_holder;
   int issued = 0;   // MMA batches committed by thread 0 (two per tile)
 
-  // persistent: tile index = head x slots + slot, strided over the grid
+  // Persistent: tile index = head x slots + slot, strided over the grid.  Each iteration
+  // runs the row pass of the tile in flight on all 16 warps; then warps 0-7 take its serial
+  // tail (gram readout, solve, W/U~) while warps 8-15 look up this CTA's next tile and run
+  // its gate pass, whose G and beta the next row pass and tail read.
   const int ntiles = nslots * H;
-  // The next tile's range and state row are looked up by one thread during the gram MMA
-  // and published here, so that a tile starts without that round trip to memory.
-  __shared__ int next_meta[8];   // seq, start, end, t0, len, chunk, state row, valid
-  using GRawT = typename std::conditional<FUSED, uint32_t, float2>::type;   // 2 gate channels as loaded
-  GRawT graw[8];
-  bool have_meta = false;
-  const int cp = 2 * (tid & 63), qr = tid >> 6;   // gate pass: channels cp, cp+1 of rows 8qr..8qr+7
-  // gate inputs (f, or log a) of tile rows 8qr..8qr+7
-  auto load_gates = [&](const TileRange& r, int hd) {
+  __shared__ int next_meta[8];   // the next tile: index (-1: none), seq, start, end, t0, len, chunk, state row
+  const int pr = warp & 7, hh = warp >> 3;
+  const int c2 = 64 * hh + 2 * lane;   // row pass: warps w and w + 8 share rows 8(w%8)..+7
+  // ---- the log decay of tile n, its running sum G over the chunk (log2 units: G log2 e)
+  // and beta, by warps 8-15 (256 threads: channels gp, gp+1 of rows 16 gq .. 16 gq + 15) ----
+  auto gate_pass = [&](int n, const TileRange& nt, int nbuf) {
+    const int gt = tid - 256, gp = 2 * (gt & 63), gq = gt >> 6;
+    const int nh = n / nslots, ns = n % nslots;
+    using GRawT = typename std::conditional<FUSED, uint32_t, float2>::type;   // 2 channels as loaded
+    GRawT graw[16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 16; ++i) {
       graw[i] = GRawT{};
-      if (8 * qr + i < r.len) {
-        const size_t idx = ((size_t)(r.t0 + 8 * qr + i) * H + hd) * D + cp;
+      if (16 * gq + i < nt.len) {
+        const size_t idx = ((size_t)(nt.t0 + 16 * gq + i) * H + nh) * D + gp;
         graw[i] = FUSED ? *reinterpret_cast<const GRawT*>(static_cast<const __nv_bfloat16*>(a.f) + idx)
                         : *reinterpret_cast<const GRawT*>(a.loga + idx);
       }
     }
+    float A_log_h = 0.f;
+    float2 dtb = make_float2(0.f, 0.f);
+    if (FUSED) {
+      A_log_h = __ldg(a.A_log + nh);
+      dtb = *reinterpret_cast<const float2*>(a.dt_bias + (size_t)nh * D + gp);
+    }
+    // while the loads are in flight: pull into L2 the inputs of the tile after this one,
+    // 128-byte lines spread over the threads
+    {
+      const int nid = n + gridDim.x;
+      if (nid < ntiles) {
+        const int nnh = nid / nslots, nns = nid % nslots;
+        // same sequence (slots of a sequence are consecutive): no search
+        const int nc = nt.chunk + (nns - ns);
+        TileRange ft;
+        if (nc >= 0 && (long long)nc * C < nt.end - nt.start) {
+          ft = nt;
+          ft.chunk = nc;
+          ft.t0 = nt.start + nc * C;
+          ft.len = min(C, nt.end - ft.t0);
+        } else {
+          ft = slot_to_tile(a.cu, a.n_seqs, a.total, C, nns);
+        }
+        const int w0 = max(ft.start, ft.t0 - (KC - 1));      // window rows inside the sequence
+        const int nrow = ft.t0 + ft.len - w0;
+        // per row: x (FUSED: 6 lines) or q, k, v (12 lines), then f or log a (2 or 4 lines)
+        const int lx = FUSED ? 6 : 12, lg = FUSED ? 2 : 4, per = lx + lg;
+        for (int e = gt; e < nrow * per; e += 256) {
+          const int tok = w0 + e / per, l = e % per;
+          const size_t row = (size_t)tok * H + nnh;
+          const char* p;
+          if (l < lx) {
+            if (FUSED) p = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.x) + row * 3 * D) + 128 * l;
+            else p = reinterpret_cast<const char*>((l < 4 ? a.q : l < 8 ? a.k : a.v) + row * D) + 128 * (l & 3);
+          } else {
+            if (tok < ft.t0) continue;                         // no gates for window rows
+            p = FUSED ? reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.f) + row * D) + 128 * (l - lx)
+                      : reinterpret_cast<const char*>(a.loga + row * D) + 128 * (l - lx);
+          }
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+        }
+      }
+    }
+    float g0[16], g1[16];
+    if (FUSED) {
+      // log2 a = lb log2(e) sigmoid(exp(A_log) (f + dt_bias))
+      const float Ah2 = expf(A_log_h) * LOG2E, lb2 = a.lb * LOG2E;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const bool live = 16 * gq + i < nt.len;
+        const float2 v = to_f2(graw[i]);
+        g0[i] = live ? lb2 * sigmoid2(Ah2 * (v.x + dtb.x)) : 0.f;
+        g1[i] = live ? lb2 * sigmoid2(Ah2 * (v.y + dtb.y)) : 0.f;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 v = to_f2(graw[i]);
+        g0[i] = v.x * LOG2E;
+        g1[i] = v.y * LOG2E;
+      }
+    }
+#pragma unroll
+    for (int i = 1; i < 16; ++i) {
+      g0[i] += g0[i - 1];
+      g1[i] += g1[i - 1];
+    }
+    qsum[gq][gp] = g0[15];
+    qsum[gq][gp + 1] = g1[15];
+    if (gt < C) {
+      float bv = 0.f;
+      if (gt < nt.len) {
+        const size_t bi = (size_t)(nt.t0 + gt) * H + nh;
+        bv = FUSED ? sigmoid2(LOG2E * ld1(static_cast<const __nv_bfloat16*>(a.beta_logit) + bi))
+                   : __ldg(a.beta + bi);
+      }
+      bs[nbuf][gt] = bv;
+    }
+    asm volatile("bar.sync 10, 256;" ::: "memory");   // warps 8-15
+    float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+    for (int q = 0; q < 3; ++q)
+      if (q < gq) {
+        o0 += qsum[q][gp];
+        o1 += qsum[q][gp + 1];
+      }
+    float* G = reinterpret_cast<float*>(sm + OFF_G);
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      *reinterpret_cast<float2*>(G + (16 * gq + i) * D + gp) = make_float2(g0[i] + o0, g1[i] + o1);
+    if (gq == 3) {
+      float* gCo = reinterpret_cast<float*>(a.ws + a.L.gC) + ((size_t)ns * H + nh) * D;
+      *reinterpret_cast<float2*>(gCo + gp) = make_float2(ex2a(g0[15] + o0), ex2a(g1[15] + o1));
+    }
   };
+
+  int tl = -1, buf = 0;   // tile in flight (-1: none yet) and its beta buffer
+  TileRange tr{};
+  int prow = -1;
 #pragma unroll 1
-  for (int tl = blockIdx.x; tl < ntiles; tl += gridDim.x) {
-  const int h = tl / nslots, slot = tl % nslots;
-  TileRange tr;
-  int prow;
-  if (have_meta) {
-    tr.seq = next_meta[0]; tr.start = next_meta[1]; tr.end = next_meta[2];
-    tr.t0 = next_meta[3]; tr.len = next_meta[4]; tr.chunk = next_meta[5];
-    prow = next_meta[6];
-  } else {
-    tr = slot_to_tile(a.cu, a.n_seqs, a.total, C, slot);
-    prow = tr.len ? pool_row(a.slots, tr.seq, a.pool_size) : -1;
-  }
-  have_meta = false;
-  if (tr.len == 0 || prow < 0) continue;
-  const int L = tr.len, t0 = tr.t0;
+  while (true) {
+  const int h = tl >= 0 ? tl / nslots : 0, slot = tl >= 0 ? tl % nslots : 0;
   const size_t tile = (size_t)slot * H + h;
   __nv_bfloat16* Wo = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.W) + tile * C * D;
   __nv_bfloat16* Uo = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.Ut) + tile * C * D;
   __nv_bfloat16* Qo = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.Qt) + tile * C * D;
   __nv_bfloat16* Ko = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.Kp) + tile * C * D;
   __nv_bfloat16* Mo = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.M) + tile * C * C;
-  float* gCo = reinterpret_cast<float*>(a.ws + a.L.gC) + tile * D;
   float* G = reinterpret_cast<float*>(sm + OFF_G);
-  float* Af = G;                                  // [64][AF_LD], after the gram
+  float* Af = reinterpret_cast<float*>(sm + OFF_GB);   // [64][AF_LD], once the gram is done
   float* Xs = reinterpret_cast<float*>(sm + OFF_XS);
+  const float* bsb = bs[buf];
+  const int L = tr.len, t0 = tr.t0;
 
-  // gate inputs first (the gate pass waits on them)
-  load_gates(tr, h);
-  float A_log_h = 0.f;
-  float2 dtb = make_float2(0.f, 0.f);
-  if (FUSED) {
-    A_log_h = __ldg(a.A_log + h);
-    dtb = *reinterpret_cast<const float2*>(a.dt_bias + (size_t)h * D + cp);
-  }
-
-  // ---- inputs of the token-row pass, issued now so their latency overlaps the gates
-  // (kept as loaded, converted after).  Warps w and w + 8 share token rows 8(w%8)..+7;
-  // warp w < 8 holds channels 0-63 and w >= 8 channels 64-127 of q, k and v, two per lane.
-  const int pr = warp & 7, hh = warp >> 3;
-  const int c2 = 64 * hh + 2 * lane;
+  if (tl >= 0) {
+  // ---- inputs of the token-row pass (kept as loaded, converted after).  Warp w < 8 holds
+  // channels 0-63 and w >= 8 channels 64-127 of q, k and v, two per lane.
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x);
   const __nv_bfloat16* cs = static_cast<const __nv_bfloat16*>(a.conv_state);
   using RawT = typename std::conditional<FUSED, uint32_t, float2>::type;   // 2 channels as loaded
@@ -342,97 +425,6 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   RawT aq, ak, av, bq, bk, bv;
   load_row(8 * pr, aq, ak, av);
   load_row(8 * pr + 1, bq, bk, bv);
-
-  // ---- log decay and its running sum G over the chunk, in log2 units (G log2 e):
-  // channels 2p, 2p+1, rows 8q..8q+7 per thread ----
-  {
-    // while the gate loads are in flight: pull into L2 the inputs of this CTA's next tile,
-    // 128-byte lines spread over the threads
-    {
-      const int nid = tl + gridDim.x;   // this CTA's next tile
-      if (nid < ntiles) {
-        const int nh = nid / nslots, ns = nid % nslots;
-        // same sequence (slots of a sequence are consecutive): no search
-        const int nc = tr.chunk + (ns - slot);
-        TileRange nt;
-        if (nc >= 0 && (long long)nc * C < tr.end - tr.start) {
-          nt = tr;
-          nt.chunk = nc;
-          nt.t0 = tr.start + nc * C;
-          nt.len = min(C, tr.end - nt.t0);
-        } else {
-          nt = slot_to_tile(a.cu, a.n_seqs, a.total, C, ns);
-        }
-        const int w0 = max(nt.start, nt.t0 - (KC - 1));      // window rows inside the sequence
-        const int nrow = nt.t0 + nt.len - w0;
-        // per row: x (FUSED: 6 lines) or q, k, v (12 lines), then f or log a (2 or 4 lines)
-        const int lx = FUSED ? 6 : 12, lg = FUSED ? 2 : 4, per = lx + lg;
-        for (int e = tid; e < nrow * per; e += THREADS) {
-          const int tok = w0 + e / per, l = e % per;
-          const size_t row = (size_t)tok * H + nh;
-          const char* p;
-          if (l < lx) {
-            if (FUSED) p = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.x) + row * 3 * D) + 128 * l;
-            else p = reinterpret_cast<const char*>((l < 4 ? a.q : l < 8 ? a.k : a.v) + row * D) + 128 * (l & 3);
-          } else {
-            if (tok < nt.t0) continue;                         // no gates for window rows
-            p = FUSED ? reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.f) + row * D) + 128 * (l - lx)
-                      : reinterpret_cast<const char*>(a.loga + row * D) + 128 * (l - lx);
-          }
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-        }
-      }
-    }
-    float g0[8], g1[8];
-    if (FUSED) {
-      // log2 a = lb log2(e) sigmoid(exp(A_log) (f + dt_bias))
-      const float Ah2 = expf(A_log_h) * LOG2E, lb2 = a.lb * LOG2E;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const bool live = 8 * qr + i < L;
-        const float2 v = to_f2(graw[i]);
-        g0[i] = live ? lb2 * sigmoid2(Ah2 * (v.x + dtb.x)) : 0.f;
-        g1[i] = live ? lb2 * sigmoid2(Ah2 * (v.y + dtb.y)) : 0.f;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float2 v = to_f2(graw[i]);
-        g0[i] = v.x * LOG2E;
-        g1[i] = v.y * LOG2E;
-      }
-    }
-#pragma unroll
-    for (int i = 1; i < 8; ++i) {
-      g0[i] += g0[i - 1];
-      g1[i] += g1[i - 1];
-    }
-    qsum[qr][cp] = g0[7];
-    qsum[qr][cp + 1] = g1[7];
-    if (tid < C) {
-      float bv = 0.f;
-      if (tid < L) {
-        const size_t bi = (size_t)(t0 + tid) * H + h;
-        bv = FUSED ? sigmoid2(LOG2E * ld1(static_cast<const __nv_bfloat16*>(a.beta_logit) + bi))
-                   : __ldg(a.beta + bi);
-      }
-      bs[tid] = bv;
-    }
-    __syncthreads();
-    float o0 = 0.f, o1 = 0.f;
-#pragma unroll
-    for (int q = 0; q < 7; ++q)
-      if (q < qr) {
-        o0 += qsum[q][cp];
-        o1 += qsum[q][cp + 1];
-      }
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      *reinterpret_cast<float2*>(G + (8 * qr + i) * D + cp) = make_float2(g0[i] + o0, g1[i] + o1);
-    if (qr == 7)
-      *reinterpret_cast<float2*>(gCo + cp) = make_float2(ex2a(g0[7] + o0), ex2a(g1[7] + o1));
-  }
-  __syncthreads();
 
   // ---- token rows, in pairs: (prep), operands for the MMAs, Q~ and K' ----
   // A lane's two channels travel as one packed pair through the f32x2 arithmetic.
@@ -597,7 +589,6 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   fence_proxy_async();
   __syncthreads();
 
-  // ---- gram MMA (tf32, 128 x 128 x 128) ----
   if (tid == 0) {
     tc_fence_after();
     const uint32_t id = idesc_tf32(128, 128);
@@ -608,21 +599,14 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     umma_commit(smem_u32(&bar_mma));
     ++issued;
   }
-  if (tid == THREADS - 1) {   // the next tile's range, while the gram runs (read after later barriers)
-    const int nid = tl + gridDim.x;
-    TileRange nt{};
-    int np = -1;
-    if (nid < ntiles) {
-      nt = slot_to_tile(a.cu, a.n_seqs, a.total, C, nid % nslots);
-      np = nt.len ? pool_row(a.slots, nt.seq, a.pool_size) : -1;
-    }
-    next_meta[0] = nt.seq; next_meta[1] = nt.start; next_meta[2] = nt.end;
-    next_meta[3] = nt.t0; next_meta[4] = nt.len; next_meta[5] = nt.chunk;
-    next_meta[6] = np; next_meta[7] = nid < ntiles;
-  }
+
+  }   // row pass
+
+  if (warp < 8) {
+  if (tl >= 0) {
   bool ok = mbar_wait_warp(smem_u32(&bar_mma), 0, &abort_flag);
   tc_fence_after();
-  __syncthreads();   // G is dead now: A takes its place (only entries i < r are ever read)
+  asm volatile("bar.sync 11, 256;" ::: "memory");   // warps 0-7
   // D[m][n]: rows 0-31 = keys 0-31 vs cols 0-31 (keys) / 32-63 (queries) of rows 0-31;
   // rows 32-95 = keys 0-63 vs cols 64-95 (keys) / 96-127 (queries) of rows 32-63
   // Warps of lane quarters 0-2 each read one 32-column group: warp w < 4 the keys (A),
@@ -640,7 +624,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const int r = rbase + j;
-        if (i < r) Af[r * AF_LD + i] = bs[r] * v[j];
+        if (i < r) Af[r * AF_LD + i] = bsb[r] * v[j];
       }
     } else {
 #pragma unroll
@@ -676,7 +660,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
 #pragma unroll
     for (int r = 0; r < 16; ++r) Xs[(16 * b + r) * AF_LD + 16 * b + jj] = xc[r];
   }
-  __syncthreads();
+  asm volatile("bar.sync 11, 256;" ::: "memory");
   {
     // Below the diagonal in two levels (m16n8k8 tf32 tensor-core products split three
     // ways, hi.hi + hi.lo + lo.hi ~ fp32; one warp per 16 x 8 output tile):
@@ -709,7 +693,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
       xo[8 * AF_LD] = -sum3(y, 2);
       xo[8 * AF_LD + 1] = -sum3(y, 3);
     }
-    __syncthreads();
+    asm volatile("bar.sync 11, 256;" ::: "memory");
     // warp w < 8: 16-row block i = w / 4 of B, 16-column block j of A, 8-column half
     const int bi = warp >> 2, bj = (warp >> 1) & 1, n0 = 16 * bj + 8 * (warp & 1);
     if (warp < 8) {   // Z_ij = sum_{k >= j} A_{2+i,k} X_kj
@@ -728,7 +712,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
       zo[8 * Z32_LD] = sum3(z, 2);
       zo[8 * Z32_LD + 1] = sum3(z, 3);
     }
-    __syncthreads();
+    asm volatile("bar.sync 11, 256;" ::: "memory");
     if (warp < 8) {   // X_{2+i,j} = -sum_{k <= i} X_{2+i,2+k} Z_kj
       float y[3][4] = {};
 #pragma unroll
@@ -745,17 +729,17 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
       xo[8 * AF_LD] = -sum3(y, 2);
       xo[8 * AF_LD + 1] = -sum3(y, 3);
     }
-    __syncthreads();
+    asm volatile("bar.sync 11, 256;" ::: "memory");
   }
   // T[r][j] = X[r][j] b_j for j <= r (else 0), as bf16 high and low parts, K-major [r][j]
 #pragma unroll
-  for (int e = tid; e < C * 8; e += THREADS) {
+  for (int e = tid; e < C * 8; e += 256) {
     const int r = e >> 3, j0 = 8 * (e & 7);
     float hi[8], lo[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int j = j0 + u;
-      const float tv = (j <= r) ? Xs[r * AF_LD + j] * bs[j] : 0.f;
+      const float tv = (j <= r) ? Xs[r * AF_LD + j] * bsb[j] : 0.f;
       hi[u] = __bfloat162float(__float2bfloat16_rn(tv));
       lo[u] = tv - hi[u];
     }
@@ -765,7 +749,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     st_bf16x4(sm + OFF_TL + sw128_off(r, j0) + 8, lo[4], lo[5], lo[6], lo[7]);
   }
   fence_proxy_async();
-  __syncthreads();
+  asm volatile("bar.sync 11, 256;" ::: "memory");
 
   // ---- W^T = K~^T T^T (cols 0-63), U~^T = V^T T^T (cols 64-127) ----
   if (tid == 0 && ok) {
@@ -796,29 +780,58 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     umma_commit(smem_u32(&bar_mma));
     ++issued;
   }
-  have_meta = next_meta[7] != 0;   // published before the barriers of the solve
   if (ok) ok = mbar_wait_warp(smem_u32(&bar_mma), 1, &abort_flag);
   tc_fence_after();
   if (ok) {
-    // warp w: TMEM lane quarter w % 4 (channels), W (w & 4 == 0) or U~, token half w / 8
+    // warp w: TMEM lane quarter w % 4 (channels), W (w < 4) or U~ (w >= 4), all 64 tokens
     const int q = warp & 3;
     const int c = 32 * q + lane;
-    const bool isW = (warp & 4) == 0;
-    const int hf = warp >> 3;
+    const bool isW = warp < 4;
     __nv_bfloat16* dst = isW ? Wo : Uo;
 #pragma unroll
-    for (int part = 0; part < 2; ++part) {   // 16 columns at a time: the next tile's gates are live
+    for (int part = 0; part < 4; ++part) {   // 16 token columns at a time
       float v[16];
-      tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (isW ? 0u : 64u) + 32u * hf + 16u * part, v);
+      tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (isW ? 0u : 64u) + 16u * part, v);
 #pragma unroll
       for (int j = 0; j < 16; ++j)
-        dst[(size_t)(32 * hf + 16 * part + j) * D + c] = __float2bfloat16_rn(v[j]);
+        dst[(size_t)(16 * part + j) * D + c] = __float2bfloat16_rn(v[j]);
+    }
+  }
+  }   // tail
+  } else {
+    // the next tile with work: one thread walks this CTA's tiles, the group reads the result
+    if (warp == THREADS / 32 - 1 && lane == 0) {
+      int n = tl < 0 ? (int)blockIdx.x : tl + (int)gridDim.x;
+      TileRange nt{};
+      int np = -1;
+      for (; n < ntiles; n += gridDim.x) {
+        nt = slot_to_tile(a.cu, a.n_seqs, a.total, C, n % nslots);
+        np = nt.len ? pool_row(a.slots, nt.seq, a.pool_size) : -1;
+        if (nt.len > 0 && np >= 0) break;
+      }
+      next_meta[0] = n < ntiles ? n : -1;
+      next_meta[1] = nt.seq; next_meta[2] = nt.start; next_meta[3] = nt.end;
+      next_meta[4] = nt.t0; next_meta[5] = nt.len; next_meta[6] = nt.chunk; next_meta[7] = np;
+    }
+    asm volatile("bar.sync 10, 256;" ::: "memory");   // warps 8-15
+    const int n = next_meta[0];
+    if (n >= 0) {
+      TileRange nt;
+      nt.seq = next_meta[1]; nt.start = next_meta[2]; nt.end = next_meta[3];
+      nt.t0 = next_meta[4]; nt.len = next_meta[5]; nt.chunk = next_meta[6];
+      gate_pass(n, nt, buf ^ 1);
     }
   }
 
   tc_fence_before();
-  __syncthreads();   // this tile's shared memory and TMEM are free for the next one
+  __syncthreads();   // the tile's shared memory and TMEM are free; the next tile's G and beta are in place
   if (abort_flag) break;
+  tl = next_meta[0];
+  if (tl < 0) break;
+  tr.seq = next_meta[1]; tr.start = next_meta[2]; tr.end = next_meta[3];
+  tr.t0 = next_meta[4]; tr.len = next_meta[5]; tr.chunk = next_meta[6];
+  prow = next_meta[7];
+  buf ^= 1;
   }   // tiles
 
   if (abort_flag && tid == 0) {
@@ -839,6 +852,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
                  : "memory");
   }
 }
+
 
 template <bool FUSED>
 cudaError_t launch_intra_t(const PrefillArgs& a, cudaStream_t st) {
