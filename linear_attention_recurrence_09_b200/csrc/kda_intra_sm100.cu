@@ -35,8 +35,9 @@
 // pass takes three exponentials: e^{G_r - G_ref} and its reciprocal give the gram scalings,
 // e^{G_r} is e^{G_15} times the first (rows 0-31) and e^{G_C - G_r} is e^{G_C - G_47} times
 // e^{G_47 - G_r} (both factors stay above 2^-116 with the gate bounded below by -5).
-// After a tile's row pass, warps 0-7 run its serial tail (gram readout, solve, W/U~) while
-// warps 8-15 compute the next tile's gates (G, beta, e^{G_C}): the next row pass starts at once.
+// After a tile's row pass, warps 0-7 run its serial tail (key gram readout, solve, W/U~) while
+// warps 8-15 compute the next tile's gates (G, beta, e^{G_C}), so the next row pass starts at
+// once; warps 12-15 then read the query gram M out of TMEM, off the tail's critical path.
 #include <type_traits>
 
 #include "kda_common.cuh"
@@ -239,8 +240,8 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
 
   // Persistent: tile index = head x slots + slot, strided over the grid.  Each iteration
   // runs the row pass of the tile in flight on all 16 warps; then warps 0-7 take its serial
-  // tail (gram readout, solve, W/U~) while warps 8-15 look up this CTA's next tile and run
-  // its gate pass, whose G and beta the next row pass and tail read.
+  // tail (key gram readout, solve, W/U~) while warps 8-15 look up this CTA's next tile and run
+  // its gate pass, whose G and beta the next row pass and tail read, and warps 12-15 read M.
   const int ntiles = nslots * H;
   __shared__ int next_meta[8];   // the next tile: index (-1: none), seq, start, end, t0, len, chunk, state row
   const int pr = warp & 7, hh = warp >> 3;
@@ -612,30 +613,18 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   // Warps of lane quarters 0-2 each read one 32-column group: warp w < 4 the keys (A),
   // warp w + 4 the queries (M); quarter 3 (rows 96-127 of D) holds nothing and writes the
   // zero upper-right block of M.
-  if (ok && warp < 8 && (warp & 3) < 3) {
-    const int q = warp & 3;
+  if (ok && warp < 3) {   // the keys (A); the queries (M) are read by warps 12-15
+    const int q = warp;
     const int i = (q == 2) ? 32 + lane : lane;          // key index of this TMEM lane
     const int rbase = (q == 0) ? 0 : 32;                 // first row r of the group
-    const bool keys = warp < 4;
-    const uint32_t col = ((q == 0) ? 0u : 64u) + (keys ? 0u : 32u);
+    const uint32_t col = (q == 0) ? 0u : 64u;
     float v[32];
     tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + col, v);
-    if (keys) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int r = rbase + j;
-        if (i < r) Af[r * AF_LD + i] = bsb[r] * v[j];
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int r = rbase + j;
-        Mo[r * C + i] = __float2bfloat16_rn(i <= r ? v[j] : 0.f);
-      }
+    for (int j = 0; j < 32; ++j) {
+      const int r = rbase + j;
+      if (i < r) Af[r * AF_LD + i] = bsb[r] * v[j];
     }
-  } else if (warp == 3) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) Mo[j * C + 32 + lane] = __float2bfloat16_rn(0.f);
   }
   tc_fence_before();
   // the diagonal blocks of A come from warps 0 and 2: the substitution below (warps 0-1)
@@ -749,7 +738,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     st_bf16x4(sm + OFF_TL + sw128_off(r, j0) + 8, lo[4], lo[5], lo[6], lo[7]);
   }
   fence_proxy_async();
-  asm volatile("bar.sync 11, 256;" ::: "memory");
+  asm volatile("bar.sync 13, 384;" ::: "memory");   // warps 0-7 and 12-15 (M read from TMEM)
 
   // ---- W^T = K~^T T^T (cols 0-63), U~^T = V^T T^T (cols 64-127) ----
   if (tid == 0 && ok) {
@@ -820,6 +809,30 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
       nt.seq = next_meta[1]; nt.start = next_meta[2]; nt.end = next_meta[3];
       nt.t0 = next_meta[4]; nt.len = next_meta[5]; nt.chunk = next_meta[6];
       gate_pass(n, nt, buf ^ 1);
+    }
+    // M of the tile in flight, before the W/U~ MMA reuses its TMEM columns: warps 12-14 read
+    // the query columns of lane quarters 0-2; quarter 3 holds nothing and warp 15 writes the
+    // zero upper-right block
+    if (tl >= 0 && warp >= 12) {
+      const bool okm = mbar_wait_warp(smem_u32(&bar_mma), 0, &abort_flag);
+      tc_fence_after();
+      const int q = warp & 3;
+      if (okm && q < 3) {
+        const int i = (q == 2) ? 32 + lane : lane;
+        const int rbase = (q == 0) ? 0 : 32;
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + ((q == 0) ? 0u : 64u) + 32u, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int r = rbase + j;
+          Mo[r * C + i] = __float2bfloat16_rn(i <= r ? v[j] : 0.f);
+        }
+      } else if (q == 3) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) Mo[j * C + 32 + lane] = __float2bfloat16_rn(0.f);
+      }
+      tc_fence_before();
+      asm volatile("bar.sync 13, 384;" ::: "memory");   // with warps 0-7, before the W/U~ MMA
     }
   }
 
