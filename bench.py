@@ -137,7 +137,8 @@ def measured_peaks():
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) comes from the
 # committed ncu summaries; a summary records the sha256 of the kernel's source file at
-# capture time and counts only while that file is unchanged.
+# capture time, and the sha256 of its code (comments and blank lines removed), and counts
+# only while that code is unchanged.
 PROFILED = {
     'intra_chunk': ('profiles/intra_chunk_sm100_prefill_8k.md',
                     'linear_attention_recurrence_09_b200/csrc/kda_intra_sm100.cu'),
@@ -150,18 +151,48 @@ PROFILED = {
 }
 
 
-def profiled_traffic(kernel):
+def code_text(src):
+    """C/C++/CUDA source without comments, trailing blanks and blank lines (string and
+    character literals kept as they are)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in '"\'':
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == '\\' else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith('//', i):
+            while i < n and src[i] != '\n':
+                i += 1
+        elif src.startswith('/*', i):
+            j = src.find('*/', i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (line.rstrip() for line in ''.join(out).split('\n'))
+    return '\n'.join(line for line in lines if line)
+
+
+def code_sha256(path):
     import hashlib
+    with open(path, encoding='utf-8') as fh:
+        return hashlib.sha256(code_text(fh.read()).encode()).hexdigest()
+
+
+def profiled_traffic(kernel):
     import re
     if kernel not in PROFILED:
         return None
     summary, source = (os.path.join(ROOT, f) for f in PROFILED[kernel])
     try:
         text = open(summary).read()
-        digest = hashlib.sha256(open(source, 'rb').read()).hexdigest()
+        digest = code_sha256(source)
     except OSError:
         return None
-    m_hash = re.search(r'source_sha256:\s*([0-9a-f]{64})', text)
+    m_hash = re.search(r'code_sha256:\s*([0-9a-f]{64})', text)
     m_traffic = re.search(r'traffic_bytes_per_launch:\s*([0-9]+)', text)
     if not (m_hash and m_traffic) or m_hash.group(1) != digest:
         return None

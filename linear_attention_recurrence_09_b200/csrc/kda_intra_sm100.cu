@@ -609,10 +609,9 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   tc_fence_after();
   asm volatile("bar.sync 11, 256;" ::: "memory");   // warps 0-7
   // D[m][n]: rows 0-31 = keys 0-31 vs cols 0-31 (keys) / 32-63 (queries) of rows 0-31;
-  // rows 32-95 = keys 0-63 vs cols 64-95 (keys) / 96-127 (queries) of rows 32-63
-  // Warps of lane quarters 0-2 each read one 32-column group: warp w < 4 the keys (A),
-  // warp w + 4 the queries (M); quarter 3 (rows 96-127 of D) holds nothing and writes the
-  // zero upper-right block of M.
+  // rows 32-95 = keys 0-63 vs cols 64-95 (keys) / 96-127 (queries) of rows 32-63.
+  // Warps 0-2 (lane quarters 0-2) read the key columns of their quarter into A; warps
+  // 12-14 read the query columns (M) later, and quarter 3 (rows 96-127 of D) holds nothing.
   if (ok && warp < 3) {   // the keys (A); the queries (M) are read by warps 12-15
     const int q = warp;
     const int i = (q == 2) ? 32 + lane : lane;          // key index of this TMEM lane
@@ -628,7 +627,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   }
   tc_fence_before();
   // the diagonal blocks of A come from warps 0 and 2: the substitution below (warps 0-1)
-  // starts once warps 0-2 are done, while the M rows are still being written
+  // starts once warps 0-2 are done
   if (warp < 3) asm volatile("bar.sync 9, 96;" ::: "memory");
 
   // ---- T = (I + A)^{-1} diag(b), with A strictly lower triangular, by 16 x 16 blocks ----

@@ -1,0 +1,39 @@
+"""Host-side logic of bench.py that needs no GPU: the code digest that decides whether a
+committed ncu summary still describes the kernel source, and the summaries themselves."""
+import os
+import re
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_code_text_drops_comments_and_keeps_literals():
+    src = ('int a = 1;  // trailing\n'
+           '/* block\n   comment */ const char* s = "x//y /*z*/";\n'
+           "char q = '\"'; char e = '\\\\';\n"
+           '\n\n   \n'
+           'asm("mov.b64 %0, {%1, %2};" : "=l"(r));  /* tail */\n')
+    assert bench.code_text(src) == ('int a = 1;\n const char* s = "x//y /*z*/";\n'
+                                    "char q = '\"'; char e = '\\\\';\n"
+                                    'asm("mov.b64 %0, {%1, %2};" : "=l"(r));')
+
+
+def test_code_digest_ignores_comments_but_not_code(tmp_path):
+    a = tmp_path / 'a.cu'
+    a.write_text('// header\n__global__ void k(float* p) {\n  p[0] = 1.f;  // one\n}\n')
+    b = tmp_path / 'b.cu'
+    b.write_text('/* another header */\n\n__global__ void k(float* p) {\n  p[0] = 1.f;\n}\n')
+    c = tmp_path / 'c.cu'
+    c.write_text('__global__ void k(float* p) {\n  p[0] = 2.f;\n}\n')
+    assert bench.code_sha256(str(a)) == bench.code_sha256(str(b))
+    assert bench.code_sha256(str(a)) != bench.code_sha256(str(c))
+
+
+def test_profile_summaries_name_their_source_and_traffic():
+    for kernel, (summary, source) in bench.PROFILED.items():
+        text = open(os.path.join(ROOT, summary)).read()
+        assert re.search(r'code_sha256:\s*[0-9a-f]{64}', text), summary
+        assert re.search(r'traffic_bytes_per_launch:\s*[0-9]+', text), summary
+        assert os.path.exists(os.path.join(ROOT, source)), source
+        assert '--clock-control none' in text, summary
