@@ -89,7 +89,10 @@ class Dist:
 class ClockSampler:
     def __init__(self, gpu_index: int):
         self.proc = None
-        self.path = os.path.join(ROOT, 'gpurun_out', f'clocks_rank{gpu_index}.csv')
+        import tempfile
+        # the raw samples go to KDA_CLOCKS_DIR (default: the system temp directory)
+        folder = os.environ.get('KDA_CLOCKS_DIR') or tempfile.gettempdir()
+        self.path = os.path.join(folder, f'kda_bench_clocks_rank{gpu_index}_{os.getpid()}.csv')
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, 'w')
