@@ -250,6 +250,39 @@ def prefill_bytes(T, H, d, C=64, K=4, fused_norm=True):
     return {'intra_chunk': intra, 'inter_chunk': inter, 'gated_norm': norm, 'layer': layer}
 
 
+# nominal dense tensor-core rates on B200 (PFLOP/s): tf32 1.1, bf16 2.25; a tf32 MMA is timed
+# against the measured bf16 peak scaled by this ratio
+TF32_PER_BF16 = 1.1 / 2.25
+
+
+def prefill_mma_flops(T, H, d, C=64):
+    """Tensor-core work the two passes issue per step (flops of the MMAs as issued, padding
+    included), by operand type.  Pass 1 per (chunk, head): the tf32 gram (M = N = 2C,
+    K = d) and the bf16 W/U~ products (three + two MMAs of M = d, N = K = C).  Pass 2 per
+    (chunk, head): [W; Q~] S (M = 2C, K = d), K'^T U (M = d, K = C) and [0; M] U (M = 2C,
+    K = C), each over the d value columns."""
+    tiles = -(-T // C) * H
+    intra_tf32 = tiles * 2 * (2 * C) * (2 * C) * d
+    intra_bf16 = tiles * 5 * 2 * d * C * C
+    inter_bf16 = tiles * (2 * (2 * C) * d * d + 2 * d * d * C + 2 * (2 * C) * d * C)
+    return {'intra_chunk': {'tf32': intra_tf32, 'bf16': intra_bf16},
+            'inter_chunk': {'tf32': 0, 'bf16': inter_bf16}}
+
+
+def tensor_roofline(flops, ms_phase, bf16_tflops):
+    """Per pass: the time the tensor pipe needs for its MMAs at peak (bf16 at the measured
+    peak, tf32 at that times the nominal ratio) as a fraction of the pass's duration."""
+    out = {}
+    for ph, f in flops.items():
+        if ph not in ms_phase:
+            continue
+        t_peak = f['bf16'] / (bf16_tflops * 1e12) + f['tf32'] / (bf16_tflops * TF32_PER_BF16 * 1e12)
+        out[ph] = {'mma_gflop': (f['bf16'] + f['tf32']) / 1e9,
+                   'ms_at_peak': t_peak * 1e3,
+                   'frac': t_peak * 1e3 / ms_phase[ph]}
+    return out
+
+
 def run_prefill(args, dist, torch, kda, synth, dev):
     W = prefill_workload(torch, kda, synth, args.tokens, 1 + 1000 * dist.rank, dev)
     cfg, P, A, y, state, ws = (W[k] for k in ('cfg', 'P', 'A', 'y', 'state', 'ws'))
@@ -357,6 +390,7 @@ def run_prefill(args, dist, torch, kda, synth, dev):
         'step_roofline': {'algorithmic_bytes': nb['layer'],
                           'achieved_gbs': nb['layer'] / (ms_step / 1e3) / 1e9,
                           'frac': nb['layer'] / (ms_step / 1e3) / 1e9 / hbm},
+        'tensor_roofline': tensor_roofline(prefill_mma_flops(T, H, d), ms_phase, tc),
         'clocks': clocks,
     }
     del W

@@ -37,3 +37,24 @@ def test_profile_summaries_name_their_source_and_traffic():
         assert re.search(r'traffic_bytes_per_launch:\s*[0-9]+', text), summary
         assert os.path.exists(os.path.join(ROOT, source)), source
         assert '--clock-control none' in text, summary
+
+
+def test_prefill_mma_flops_by_hand():
+    # T = 64 (one chunk), H = 1, d = 128, C = 64
+    f = bench.prefill_mma_flops(64, 1, 128, 64)
+    assert f['intra_chunk']['tf32'] == 2 * 128 * 128 * 128          # gram, M = N = K = 128
+    assert f['intra_chunk']['bf16'] == 5 * 2 * 128 * 64 * 64        # W: 3 MMAs, U~: 2
+    assert f['inter_chunk']['bf16'] == (2 * 128 * 128 * 128        # [W; Q~] S
+                                        + 2 * 128 * 128 * 64        # K'^T U
+                                        + 2 * 128 * 128 * 64)       # [0; M] U
+    # a ragged tail counts as a whole chunk (the tiles are padded)
+    assert bench.prefill_mma_flops(65, 2, 128, 64)['intra_chunk']['tf32'] == 4 * f['intra_chunk']['tf32']
+
+
+def test_tensor_roofline_fraction():
+    flops = {'intra_chunk': {'tf32': 1.1e9, 'bf16': 2.25e9}, 'inter_chunk': {'tf32': 0, 'bf16': 0}}
+    r = bench.tensor_roofline(flops, {'intra_chunk': 2.0}, 2250.0)
+    # bf16 2.25 GFLOP at 2.25 PFLOP/s = 1 us; tf32 1.1 GFLOP at 1.1 PFLOP/s = 1 us
+    assert abs(r['intra_chunk']['ms_at_peak'] - 2e-3) < 1e-12
+    assert abs(r['intra_chunk']['frac'] - 1e-3) < 1e-12
+    assert 'inter_chunk' not in r
