@@ -24,8 +24,10 @@
  *    host BEFORE anything is launched; on an error nothing is launched and no
  *    output is touched.
  *  - Every pointer is caller-owned DEVICE memory (any allocator), except `cfg`
- *    which is host memory.  The library allocates nothing, frees nothing and
- *    keeps no state between calls.
+ *    which is host memory.  The library allocates nothing and frees nothing;
+ *    between calls it keeps only the per-thread measurement hooks below
+ *    (phase events, launch count, last CUDA error message) and the fixed
+ *    scratch of kda_prefill_noalloc.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
  *    stream) and the call returns without synchronising.  Launch failures are
  *    reported as KDA_ERR_CUDA.
@@ -348,7 +350,7 @@ KDA_API int kda_prefill_noalloc(const kda_config* cfg, int32_t n_seqs, int32_t t
 KDA_API int kda_selftest_wait_timeout(void* workspace, kda_stream_t stream);
 
 /*
- * kda_set_phase_events - measurement hook (the paper has no counterpart).
+ * kda_set_phase_events - measurement hook (the pages have no counterpart).
  * `events` holds n <= 3 cudaEvent_t handles (created by the caller, owned by
  * the caller, may be NULL entries); while set, every kda_prefill,
  * kda_prefill_noalloc and kda_layer_prefill issued from THIS host thread
@@ -360,7 +362,7 @@ KDA_API int kda_selftest_wait_timeout(void* workspace, kda_stream_t stream);
 KDA_API int kda_set_phase_events(void* const* events, int32_t n);
 
 /*
- * kda_launch_count - measurement hook (the paper has no counterpart): the number
+ * kda_launch_count - measurement hook (the pages have no counterpart): the number
  * of kernels the library has launched from THIS host thread since it was loaded
  * (cumulative; take differences around the calls of interest).  Launches only:
  * cudaMemsetAsync and other runtime calls are not counted.
