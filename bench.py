@@ -5,9 +5,10 @@ Headline workload (one step): prep + chunked prefill of one packed batch,
 B = 1, H = 32, T = 8192, d = 128, chunk 64, bf16 activations, fp32 state,
 A_log and dt_bias, seeded synthetic inputs resident in HBM.  Metric: prefill
 tokens/s.  At N = 1 the same line also carries the batched decode workload
-(B = 64, H = 32, d = 128, 1,024 steps after a 512-token prefill, CUDA graph)
-and the speculative verify + rollback workload (B = 16, blocks of 8 drafts
-after a 4,096-token context, 256 rounds, CUDA graph).
+(B = 64, H = 32, d = 128, 1,024 steps after a 512-token prefill, CUDA graph),
+the speculative verify + rollback workload (B = 16, blocks of 8 drafts after a
+4,096-token context, 256 rounds, CUDA graph) and the long / varlen prefill (one
+131,072-token sequence; 8 packed sequences of 1K-32K tokens).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kda|reference]
 
@@ -42,7 +43,8 @@ def parse_args():
     ap.add_argument('--tokens', type=int, default=8192, help='prefill length (8192 = headline)')
     ap.add_argument('--no-extras', action='store_true', help='skip decode / verify workloads')
     ap.add_argument('--no-cpu', action='store_true', help='skip the CPU oracle baseline')
-    ap.add_argument('--only', default='', help='prefill|decode|verify: run one workload only')
+    ap.add_argument('--only', default='', help='prefill|decode|verify|long: run one workload only')
+    ap.add_argument('--no-long', action='store_true', help='skip the long / varlen workload')
     return ap.parse_args()
 
 
@@ -130,12 +132,14 @@ class ClockSampler:
 
 
 def measured_peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, bf16 TFLOP/s sustained, 'measured' | 'fallback')."""
     try:
         with open(os.path.join(ROOT, 'MEASURED_PEAKS.json')) as fh:
             p = json.load(fh)
-        return p['hbm_gbs'], p['bf16_tflops'], 'measured'
+        return (p['hbm_gbs'], p['bf16_tflops'], p.get('bf16_tflops_sustained', p['bf16_tflops']),
+                'measured')
     except Exception:
-        return 6650.0, 1590.0, 'fallback'
+        return 6650.0, 1590.0, 1400.0, 'fallback'
 
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) comes from the
@@ -250,6 +254,25 @@ def prefill_bytes(T, H, d, C=64, K=4, fused_norm=True):
     return {'intra_chunk': intra, 'inter_chunk': inter, 'gated_norm': norm, 'layer': layer}
 
 
+def layer_method_bytes(total_tokens, n_seqs, H, d):
+    """The method's own HBM bytes for one layer call (the per-unit figure of the
+    hot-path measurement: 1,538 B per (token, head) at d = 128 with bf16 activations):
+    x (3d), f (d), g (d) and the beta logit (1) read once, y (d) written once, plus the
+    final fp32 state of every (sequence, head) written once.  Everything else the
+    passes move (the chunk tiles handed from pass 1 to pass 2) is design traffic."""
+    th = total_tokens * H
+    return th * (3 * d * 2 + d * 2 + 2 + d * 2 + d * 2) + n_seqs * H * d * d * 4
+
+
+def prefill_dense_flops(T, H, d, C=64):
+    """Flops of the chunk form's dense tiles per step: per (chunk, head) the grams A and
+    M (2 C^2 d MAC), W = T (K e^G) and U~ = T V (2 C^2 d), U = U~ - W S, Q~ S and the
+    state increment K'^T U (3 C d^2), and M U (C^2 d): 2 (5 C d + 3 d^2) flops per
+    (token, head), 47.2 GFLOP at B = 1, H = 32, T = 8192, d = 128, C = 64.  Issued MMA
+    work (hi/lo splits, padding, the unused part of the 128 x 128 gram) is not counted."""
+    return 2 * (5 * C * d + 3 * d * d) * (-(-T // C) * C) * H
+
+
 # nominal dense tensor-core rates on B200 (PFLOP/s): tf32 1.1, bf16 2.25; a tf32 MMA is timed
 # against the measured bf16 peak scaled by this ratio
 TF32_PER_BF16 = 1.1 / 2.25
@@ -269,18 +292,28 @@ def prefill_mma_flops(T, H, d, C=64):
             'inter_chunk': {'tf32': 0, 'bf16': inter_bf16}}
 
 
-def tensor_roofline(flops, ms_phase, bf16_tflops):
-    """Per pass: the time the tensor pipe needs for its MMAs at peak (bf16 at the measured
-    peak, tf32 at that times the nominal ratio) as a fraction of the pass's duration."""
+def issued_mma_view(flops, ms_phase, bf16_tflops):
+    """Per pass: the time the tensor pipe needs for the MMAs it issues at peak (bf16 at
+    the measured peak, tf32 at that times the nominal ratio) as a fraction of the pass's
+    duration.  A view of the design, not the roofline (see tensor_roofline)."""
     out = {}
     for ph, f in flops.items():
         if ph not in ms_phase:
             continue
         t_peak = f['bf16'] / (bf16_tflops * 1e12) + f['tf32'] / (bf16_tflops * TF32_PER_BF16 * 1e12)
-        out[ph] = {'mma_gflop': (f['bf16'] + f['tf32']) / 1e9,
+        out[ph] = {'issued_mma_gflop': (f['bf16'] + f['tf32']) / 1e9,
                    'ms_at_peak': t_peak * 1e3,
                    'frac': t_peak * 1e3 / ms_phase[ph]}
     return out
+
+
+def tensor_roofline(dense_flops, ms_step, burst_tflops, sustained_tflops):
+    """Dense-tile flops of one step over (step time x bf16 dense peak)."""
+    achieved = dense_flops / (ms_step / 1e3) / 1e12
+    return {'bound': 'tensor', 'dense_tile_gflop': dense_flops / 1e9, 'achieved': achieved,
+            'peak': burst_tflops, 'unit': 'TFLOP/s', 'frac': achieved / burst_tflops,
+            'frac_sustained': achieved / sustained_tflops,
+            'ms_at_peak': dense_flops / (burst_tflops * 1e12) * 1e3}
 
 
 def run_prefill(args, dist, torch, kda, synth, dev):
@@ -329,10 +362,13 @@ def run_prefill(args, dist, torch, kda, synth, dev):
     clocks = sampler.stop() if sampler else None
     fused_norm = launches == 2 * args.steps      # intra + inter (norm inside the inter pass)
     phases = PHASES[:2] if fused_norm else PHASES
-    ms_phase = {ph: statistics.mean(p[i].elapsed_time(p[i + 1]) for p in per)
+    # per-step statistic: the median of the K per-step event durations (the timed region's
+    # mean is kept beside it); per pass likewise
+    step_ms = [p[0].elapsed_time(p[len(phases)]) for p in per]
+    ms_phase = {ph: statistics.median(p[i].elapsed_time(p[i + 1]) for p in per)
                 for i, ph in enumerate(phases)}
-    ms_max = dist.max(ms)
-    ms_step = ms_max / args.steps
+    ms_step = dist.max(statistics.median(step_ms))
+    ms_mean = dist.max(ms) / args.steps
     T, H, d = W['T'], W['H'], W['d']
     value = dist.world * T / (ms_step / 1e3)
 
@@ -363,14 +399,15 @@ def run_prefill(args, dist, torch, kda, synth, dev):
     h2d = sum(t.numel() * t.element_size() for t in hx.values())
     d2h = hy.numel() * hy.element_size() + hs.numel() * hs.element_size()
 
-    hbm, tc, peak_kind = measured_peaks()
+    hbm, tc, tc_sus, peak_kind = measured_peaks()
     nb = prefill_bytes(T, H, d, fused_norm=fused_norm)
-    top = max(phases, key=lambda ph: ms_phase[ph])
-    dominant = (top, nb[top], ms_phase[top])
-    achieved = dominant[1] / (dominant[2] / 1e3) / 1e9
+    method = layer_method_bytes(T, 1, H, d)
+    achieved = method / (ms_step / 1e3) / 1e9
+    pass_traffic = [profiled_traffic(ph) for ph in phases]
     res = {
         'metric': METRIC, 'value': value, 'unit': 'tokens/s', 'n_gpus': dist.world,
         'steps': args.steps, 'warmup': args.warmup, 'ms_per_step': ms_step,
+        'ms_per_step_mean': ms_mean, 'timing': 'median of per-step CUDA-event durations',
         'higher_is_better': True, 'scaling': 'weak', 'vs_baseline': None, 'dtype': 'bf16',
         'data': 'synthetic (seeded N(0,1) activations, random-init layer parameters)',
         'config': prefill_config(T, H, d, dist.world),
@@ -378,23 +415,123 @@ def run_prefill(args, dist, torch, kda, synth, dev):
                 'h2d_bytes_per_step': h2d, 'd2h_bytes_per_step': d2h,
                 'ms_per_step': e2e_ms},
         'gpu_launches': launches,
-        'roofline': {'bound': 'hbm', 'kernel': dominant[0], 'achieved': achieved, 'peak': hbm,
-                     'unit': 'GB/s', 'frac': achieved / hbm,
-                     'traffic': profiled_traffic(dominant[0]),
-                     'peak_kind': peak_kind, 'algorithmic_bytes_per_launch': dominant[1]},
+        # the method's bytes (x, f, g, beta logit in; y, final state out) over the step, i.e.
+        # over the one kda_layer_prefill call whose two launches are the dominant work
+        'roofline': {'bound': 'hbm', 'kernel': 'kda_layer_prefill (intra-chunk + inter-chunk '
+                     'launches)', 'achieved': achieved, 'peak': hbm, 'unit': 'GB/s',
+                     'frac': achieved / hbm,
+                     'traffic': (sum(pass_traffic) if all(t is not None for t in pass_traffic)
+                                 else None),
+                     'peak_kind': peak_kind, 'algorithmic_bytes_per_launch': method,
+                     'per_unit': '1,538 B per (token, head) + 64 KB state per head'},
         'breakdown_ms': ms_phase,
-        'phase_roofline': {ph: {'algorithmic_bytes': nb[ph],
+        # bytes this design moves per pass (incl. the chunk tiles handed from pass 1 to pass
+        # 2, which the method itself does not need), with ncu DRAM traffic where profiled
+        'design_traffic': {ph: {'bytes': nb[ph],
                                 'achieved_gbs': nb[ph] / (ms_phase[ph] / 1e3) / 1e9,
-                                'frac': nb[ph] / (ms_phase[ph] / 1e3) / 1e9 / hbm}
-                           for ph in phases},
-        'step_roofline': {'algorithmic_bytes': nb['layer'],
-                          'achieved_gbs': nb['layer'] / (ms_step / 1e3) / 1e9,
-                          'frac': nb['layer'] / (ms_step / 1e3) / 1e9 / hbm},
-        'tensor_roofline': tensor_roofline(prefill_mma_flops(T, H, d), ms_phase, tc),
+                                'frac': nb[ph] / (ms_phase[ph] / 1e3) / 1e9 / hbm,
+                                'ncu_dram_bytes': tr}
+                           for ph, tr in zip(phases, pass_traffic)},
+        'tensor_roofline': tensor_roofline(prefill_dense_flops(T, H, d), ms_step, tc, tc_sus),
+        'issued_mma': issued_mma_view(prefill_mma_flops(T, H, d), ms_phase, tc),
         'clocks': clocks,
     }
     del W
     return res
+
+
+def run_long(torch, kda, synth, dev, steps=5, warmup=3):
+    """The long / varlen prefill workload: one B = 1, T = 131,072 sequence, and 8 packed
+    sequences of log-uniform lengths in [1,024, 32,768]; H = 32, d = 128, bf16, initial
+    state N(0, 0.01).  Inputs are drawn on the device from a seeded generator with the
+    recipe's distributions (the timing does not depend on the values)."""
+    H, d, K = 32, 128, 4
+    cfg = kda.Config(num_heads=H, head_dim=d, conv_size=K, dtype=torch.bfloat16, chunk_size=64)
+    P = {k: v.to(dev) for k, v in synth.layer_params(4, H, d, K).items()}
+    hbm, _, _, peak_kind = measured_peaks()
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4)
+    out = {}
+    for name, lens in (('single_131k', [131072]), ('packed_8', synth.varlen_lengths(4))):
+        N, T = len(lens), sum(lens)
+        cu = torch.tensor([0] + list(__import__('itertools').accumulate(lens)),
+                          dtype=torch.int32, device=dev)
+        rnd = lambda *shape: torch.randn(*shape, generator=gen, device=dev).to(cfg.dtype)
+        x, f, bl, g = rnd(T, H, 3 * d), rnd(T, H, d), rnd(T, H), rnd(T, H, d)
+        s0 = torch.randn(N, H, d, d, generator=gen, device=dev) * 0.1
+        state = torch.empty_like(s0)
+        y = torch.empty(T, H, d, dtype=cfg.dtype, device=dev)
+        ws = torch.empty(kda.kda_layer_prefill_workspace_size(cfg, N, T), dtype=torch.uint8,
+                         device=dev)
+        stream = torch.cuda.current_stream()
+
+        def ev():
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)            # torch creates the CUDA event on first record
+            return e
+
+        evs = [[ev() for _ in range(4)] for _ in range(steps)]
+
+        def step(e=None):
+            if e:
+                e[0].record(stream)
+                kda.kda_set_phase_events(e[1:])
+            kda.kda_layer_prefill(cfg, cu, x, f, bl, g, P['conv_w'], P['A_log'], P['dt_bias'],
+                                  P['norm_w'], state_in=s0, state_out=state, y=y, workspace=ws,
+                                  max_seqlen=max(lens))
+            if e:
+                kda.kda_set_phase_events(())
+
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        n0 = kda.kda_launch_count()
+        for i in range(steps):
+            step(evs[i])
+        launches = (kda.kda_launch_count() - n0) // steps
+        torch.cuda.synchronize()
+        ms = statistics.median(e[0].elapsed_time(e[3]) for e in evs)
+        ms_inter = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+        method = layer_method_bytes(T, N, H, d)
+        ach = method / (ms / 1e3) / 1e9
+        rec = {'value': T / (ms / 1e3), 'unit': 'tokens/s', 'tokens': T, 'n_seqs': N,
+               'max_seqlen': max(lens), 'ms_per_step': ms,
+               'breakdown_ms': {'intra_chunk': statistics.median(e[0].elapsed_time(e[1])
+                                                                  for e in evs),
+                                'inter_chunk': ms_inter},
+               'launches_per_step': launches,
+               'roofline': {'bound': 'hbm', 'achieved': ach, 'peak': hbm, 'unit': 'GB/s',
+                            'frac': ach / hbm, 'peak_kind': peak_kind,
+                            'algorithmic_bytes_per_launch': method}}
+        if N == 1:
+            # one wave of 128 chain CTAs: the inter-chunk pass time over the serial chunks
+            rec['chain_us_per_chunk'] = ms_inter * 1e3 / (-(-T // 64))
+        out[name] = rec
+        del x, f, bl, g, y, ws, state, s0
+        torch.cuda.empty_cache()
+    out['workload'] = ('long/varlen prefill: one B=1 T=131072 sequence, and 8 packed sequences '
+                       'of log-uniform lengths in [1024, 32768]; H=32 d=128 chunk 64 bf16, '
+                       'initial state N(0, 0.01)')
+    return out
+
+
+def hbm_roofline(kernel, alg_bytes, ms_launch, hbm, peak_kind, note=None):
+    """HBM roofline of a state-streaming kernel.  `frac` uses the ncu DRAM bytes of the
+    committed summary while the kernel's code is unchanged (the state can partly hit in
+    the 126 MB L2 between launches, so bytes / time alone can overstate), otherwise the
+    algorithmic bytes; `frac_basis` says which.  Both figures are given."""
+    traffic = profiled_traffic(kernel)
+    alg = alg_bytes / (ms_launch / 1e3) / 1e9
+    dram = traffic / (ms_launch / 1e3) / 1e9 if traffic else None
+    out = {'bound': 'hbm', 'kernel': kernel, 'achieved': dram if dram else alg, 'peak': hbm,
+           'unit': 'GB/s', 'frac': (dram if dram else alg) / hbm,
+           'frac_basis': 'ncu DRAM bytes' if dram else 'algorithmic bytes',
+           'frac_algorithmic': alg / hbm, 'frac_dram': dram / hbm if dram else None,
+           'traffic': traffic, 'peak_kind': peak_kind,
+           'algorithmic_bytes_per_launch': alg_bytes, 'ms_per_launch': ms_launch}
+    if note:
+        out['note'] = note
+    return out
 
 
 def run_decode(torch, kda, synth, dev, steps=1024):
@@ -454,19 +591,14 @@ def run_decode(torch, kda, synth, dev, steps=1024):
     torch.cuda.synchronize()
     ms_k = e0.elapsed_time(e1) / n
     bytes_k = B * H * (2 * d * d * 4 + 3 * d * 4 + d * 2 + d * 4 + 4 + d * 2)
-    hbm, _, peak_kind = measured_peaks()
-    ach = bytes_k / (ms_k / 1e3) / 1e9
+    hbm, _, _, peak_kind = measured_peaks()
     del g
     return {'value': B * steps / (ms / 1e3), 'unit': 'tokens/s',
             'workload': f'decode B={B} H={H} d={d}, {steps} steps after a {T0}-token prefill '
                         '(prep + decode per step, CUDA graph)',
             'ms_per_step': ms / steps, 'gpu_launches': 2 * steps,
-            'roofline': {'bound': 'hbm', 'kernel': 'kda_decode', 'achieved': ach, 'peak': hbm,
-                         'unit': 'GB/s', 'frac': ach / hbm,
-                         'traffic': profiled_traffic('kda_decode'),
-                         'peak_kind': peak_kind, 'algorithmic_bytes_per_launch': bytes_k,
-                         'ms_per_launch': ms_k,
-                         'l2_note': 'state 134 MB is just above L2 (126 MB)'}}
+            'roofline': hbm_roofline('kda_decode', bytes_k, ms_k, hbm, peak_kind,
+                                     'state 134 MB is just above L2 (126 MB)')}
 
 
 def run_verify(torch, kda, synth, dev, rounds=256):
@@ -529,18 +661,13 @@ def run_verify(torch, kda, synth, dev, rounds=256):
     torch.cuda.synchronize()
     ms_k = e0.elapsed_time(e1) / n
     bytes_k = B * H * (d * d * 4 + Tb * d * d * 4 + Tb * (3 * d * 4 + d * 2 + d * 4 + 4 + d * 2))
-    hbm, _, peak_kind = measured_peaks()
-    ach = bytes_k / (ms_k / 1e3) / 1e9
+    hbm, _, _, peak_kind = measured_peaks()
     del g
     return {'value': B * Tb * rounds / (ms / 1e3), 'unit': 'verified draft tokens/s',
             'workload': f'verify+rollback B={B} H={H} d={d}, blocks of {Tb} after a {T0}-token '
                         f'context, {rounds} rounds, accepted ~ U{{0..{Tb}}} (CUDA graph)',
             'ms_per_round': ms / rounds, 'gpu_launches': 3 * rounds,
-            'roofline': {'bound': 'hbm', 'kernel': 'kda_verify', 'achieved': ach, 'peak': hbm,
-                         'unit': 'GB/s', 'frac': ach / hbm,
-                         'traffic': profiled_traffic('kda_verify'),
-                         'peak_kind': peak_kind, 'algorithmic_bytes_per_launch': bytes_k,
-                         'ms_per_launch': ms_k}}
+            'roofline': hbm_roofline('kda_verify', bytes_k, ms_k, hbm, peak_kind)}
 
 
 # ---------------------------------------------------------------------------
@@ -626,6 +753,8 @@ def main():
                 res['decode'] = run_decode(torch, kda, synth, dev)
             if args.only in ('', 'verify'):
                 res['verify'] = run_verify(torch, kda, synth, dev)
+            if args.only in ('', 'long') and not args.no_long:
+                res['long'] = run_long(torch, kda, synth, dev)
         if dist.rank == 0 and dist.world == 1 and not args.no_cpu and args.only in ('', 'prefill'):
             res['cpu_baseline'] = cpu_baseline(torch, synth)
         if dist.rank == 0:

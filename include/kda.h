@@ -151,8 +151,11 @@ KDA_API size_t kda_prefill_workspace_size(const kda_config* cfg, int32_t n_seqs,
 
 /*
  * kda_prefill - chunkwise-parallel prefill of packed sequences (chunk length
- * cfg->chunk_size): an intra-chunk pass, parallel over (sequence, head,
- * chunk), builds the UT/WY form of each chunk with a triangular solve; a
+ * cfg->chunk_size).  llama.cpp PR #27754, KDA commit: prefill on backends without
+ * the fused delta-net operator runs the layer as a "chunked fallback" graph; this
+ * is that algorithm class, written for sm_100a.  An intra-chunk pass, parallel
+ * over (sequence, head, chunk), builds the UT/WY form of each chunk with a
+ * triangular solve; a
  * serial inter-chunk pass carries the fp32 state on chip through the chunks
  * of each sequence and applies the gated RMSNorm epilogue.  The result equals
  * the token-by-token recurrence up to rounding.
@@ -321,9 +324,10 @@ KDA_API int kda_workspace_status(const void* workspace, kda_stream_t stream);
  *    of about 1,000 tokens fits).
  *  - Memory: every GPU that loads the library holds the 64 MiB until the process
  *    exits.
- *  - Set-up: the first call on each device (with that device current) looks up
- *    the array's device address and caches it; make that first call before any
- *    stream capture.
+ *  - Set-up: every call looks up the array's device address on the current
+ *    device (nothing is cached, so the address stays right after a
+ *    cudaDeviceReset); the first call on a device also loads the library's
+ *    device code there, so make that first call before any stream capture.
  *  - Sharing: every call on a device uses the same array, which keeps the last
  *    call's contents.  Calls that overlap on the GPU (different streams, or
  *    different host threads) race on it and give undefined results; order them.

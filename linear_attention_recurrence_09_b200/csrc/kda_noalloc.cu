@@ -3,11 +3,12 @@
 //
 // The scratch is one file-scope __device__ array of KDA_NOALLOC_SCRATCH_BYTES.
 // Host code may not pass the array's name to a kernel (on the host it is only a
-// stand-in symbol, not a device address), so the first call on each device looks
-// up the real address with cudaGetSymbolAddress while that device is current and
-// caches it; every later call on that device reuses it.
-#include <mutex>
-
+// stand-in symbol, not a device address), so every call looks up the real address
+// with cudaGetSymbolAddress while the caller's device is current.  The lookup is
+// not cached: after a cudaDeviceReset the module is loaded again and the array may
+// sit at another address, which a cached pointer would not follow.  The first call
+// on a device also loads the module there (a set-up step that should not happen
+// inside a stream capture).
 #include "../../include/kda.h"
 #include "kda_launch.h"
 
@@ -16,23 +17,12 @@ namespace {
 constexpr size_t kScratchBytes = (size_t)KDA_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of the scratch on the current device (looked up once per device).
+// Device address of the scratch on the current device.
 int scratch_on_current_device(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return KDA_ERR_CUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+    return KDA_ERR_CUDA;
+  *out = p;
   return KDA_OK;
 }
 

@@ -27,7 +27,8 @@ are the plainest reading consistent with all of them.
 
 Readings taken where the pages are silent:
 
-* log a_t = lb * sigmoid(exp(A_log[h]) * (f_t + dt_bias[h])), lb = -5;
+* log a_t = lb * sigmoid(exp(A_log[h]) * (f_t + dt_bias[h])), lb = -5 (bounded
+  branch); with no lower bound, log a_t = -exp(A_log[h]) * softplus(f_t + dt_bias[h]);
 * S_t = (I - b_t k_t k_t^T) Diag(a_t) S_{t-1} + b_t k_t v_t^T, o_t = S_t^T q_t
   (state S is d_k x d_v, key axis = rows); b_t = sigmoid(beta_logit_t);
 * conv: causal, left padded by the conv state (zeros when absent); tap K-1
@@ -77,19 +78,34 @@ def l2_normalize(x, eps=L2_EPS):
     return x / np.maximum(n, eps)
 
 
+def softplus(x):
+    """log(1 + e^x), evaluated without overflow."""
+    return np.logaddexp(0.0, np.asarray(x, dtype=np.float64))
+
+
 def log_decay(f, A_log, dt_bias, lb=GATE_LOWER_BOUND):
-    """Per-key-channel log decay, bounded sigmoid branch.
+    """Per-key-channel log decay.
 
-    log a = lb * sigmoid(exp(A_log[h]) * (f + dt_bias[h, :])).
+    Bounded-sigmoid branch (``lb`` given):
+        log a = lb * sigmoid(exp(A_log[h]) * (f + dt_bias[h, :])), in [lb, 0].
+    Softplus branch (``lb`` is None):
+        log a = -exp(A_log[h]) * softplus(f + dt_bias[h, :]), in (-inf, 0].
 
-    PR #27754, KDA commit: bounded-sigmoid decay gate selected by the required
-    ``gate_lower_bound`` key; dt_bias added per channel before the reshape;
-    per-head A broadcast over the channels.  f: [..., H, d]; A_log: [H];
-    dt_bias: [H, d].  Result lies in [lb, 0].
+    PR #27754, KDA commit: the bounded-sigmoid gate is selected by the
+    ``gate_lower_bound`` key; dt_bias is added per channel before the reshape and
+    the per-head A is broadcast over the channels.  PR #27754, "Metadata and
+    tensor loading" commit: when that key is absent the softplus branch is
+    selected, a different function rather than a missing clamp.  Its form here
+    (the negative per-head rate exp(A_log) times softplus of the biased gate) is
+    the plainest reading: the pages name the branch but do not write it out.
+    f: [..., H, d]; A_log: [H]; dt_bias: [H, d].
     """
     f = np.asarray(f, dtype=np.float64)
     A = np.exp(np.asarray(A_log, dtype=np.float64))[:, None]
-    return lb * sigmoid(A * (f + np.asarray(dt_bias, dtype=np.float64)))
+    z = f + np.asarray(dt_bias, dtype=np.float64)
+    if lb is None:
+        return -A * softplus(z)
+    return lb * sigmoid(A * z)
 
 
 def apply_key_decay(S, a):
@@ -130,7 +146,8 @@ def prep(x, f, beta_logit, conv_w, A_log, dt_bias, conv_hist=None,
 
     x: [T, H, 3d] pre-conv q|k|v; f: [T, H, d]; beta_logit: [T, H];
     conv_w: [H, 3d, K]; A_log: [H]; dt_bias: [H, d];
-    conv_hist: [K-1, H, 3d] or None (zeros).
+    conv_hist: [K-1, H, 3d] or None (zeros); lb: the gate's lower bound, or
+    None for the softplus branch (see ``log_decay``).
     Returns dict q, k, v [T, H, d], loga [T, H, d], beta [T, H],
     conv_hist [K-1, H, 3d] (new), window [K-1+T, H, 3d] (hist then x).
     """
@@ -217,7 +234,8 @@ def layer(x, f, beta_logit, g, conv_w, A_log, dt_bias, norm_w, cu_seqlens,
 
     x: [Ttot, H, 3d]; f, g: [Ttot, H, d]; beta_logit: [Ttot, H];
     cu_seqlens: [N+1]; S0: [N, H, d, d] or None; conv_hist: [N, K-1, H, 3d]
-    or None.  ``heads`` restricts the computation to a subset of heads (every
+    or None; lb as in ``prep`` (None selects the softplus decay branch).
+    ``heads`` restricts the computation to a subset of heads (every
     head is independent); the returned arrays then hold only those heads.
     Returns dict y [Ttot, Hs, d], o, state [N, Hs, d, d], conv_hist
     [N, K-1, Hs, 3d], and the prep outputs.

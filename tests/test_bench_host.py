@@ -51,10 +51,21 @@ def test_prefill_mma_flops_by_hand():
     assert bench.prefill_mma_flops(65, 2, 128, 64)['intra_chunk']['tf32'] == 4 * f['intra_chunk']['tf32']
 
 
-def test_tensor_roofline_fraction():
+def test_issued_mma_view_fraction():
     flops = {'intra_chunk': {'tf32': 1.1e9, 'bf16': 2.25e9}, 'inter_chunk': {'tf32': 0, 'bf16': 0}}
-    r = bench.tensor_roofline(flops, {'intra_chunk': 2.0}, 2250.0)
+    r = bench.issued_mma_view(flops, {'intra_chunk': 2.0}, 2250.0)
     # bf16 2.25 GFLOP at 2.25 PFLOP/s = 1 us; tf32 1.1 GFLOP at 1.1 PFLOP/s = 1 us
     assert abs(r['intra_chunk']['ms_at_peak'] - 2e-3) < 1e-12
     assert abs(r['intra_chunk']['frac'] - 1e-3) < 1e-12
     assert 'inter_chunk' not in r
+
+
+def test_dense_tile_flops_and_method_bytes_by_hand():
+    # per (token, head): grams 2 C d, W and U~ 2 C d, M U C d -> 5 C d; W S, Q~ S, K'^T U -> 3 d^2
+    assert bench.prefill_dense_flops(64, 1, 128, 64) == 2 * (5 * 64 * 128 + 3 * 128 * 128) * 64
+    # the headline step: 47.2 GFLOP
+    assert abs(bench.prefill_dense_flops(8192, 32, 128) / 1e9 - 47.24) < 0.01
+    # 1,538 B per (token, head) + the final fp32 state (64 KB per head)
+    assert bench.layer_method_bytes(8192, 1, 32, 128) == 8192 * 32 * 1538 + 32 * 128 * 128 * 4
+    r = bench.tensor_roofline(2.25e9, 2.0, 2250.0, 1125.0)
+    assert abs(r['frac'] - 5e-4) < 1e-12 and abs(r['frac_sustained'] - 1e-3) < 1e-12

@@ -64,6 +64,51 @@ def pin_log_decay():
     return max(e1, e2, e3, e4)
 
 
+LN1PE = 1.3132616875182228   # ln(1 + e)
+
+
+def pin_softplus_decay():
+    """Closed forms of the softplus branch, -exp(A_log) * softplus(f + dt_bias), selected
+    when the gate has no lower bound (lb None)."""
+    H, d = 2, 3
+    dtb = np.array([[0.3, -0.2, 0.1], [0.0, 0.5, -0.5]])
+    A_log = np.array([math.log(2.0), 0.0])
+    # f = -dt_bias: softplus(0) = ln 2 -> -exp(A_log) ln 2 per head
+    g0 = ko.log_decay(-dtb, A_log, dtb, None)
+    e1 = max(np.abs(g0[0] + 2 * math.log(2.0)).max(), np.abs(g0[1] + math.log(2.0)).max())
+    # f + dt_bias = 1: softplus(1) = ln(1 + e)
+    g1 = ko.log_decay(1.0 - dtb, A_log, dtb, None)
+    e2 = max(np.abs(g1[0] + 2 * LN1PE).max(), np.abs(g1[1] + LN1PE).max())
+    # large argument: softplus(x) = x + ln(1 + e^-x) -> x; very negative: -> e^x -> 0
+    g2 = ko.log_decay(50.0 - dtb, A_log, dtb, None)
+    e3 = max(np.abs(g2[0] + 100.0).max(), np.abs(g2[1] + 50.0).max())
+    g3 = ko.log_decay(np.full((H, d), -800.0), A_log, dtb, None)
+    e4 = np.abs(g3).max()
+    # no lower bound: log a keeps growing with the gate (past -5 of the bounded branch)
+    e5 = 0.0 if ko.log_decay(np.full((1, 1), 10.0), np.zeros(1), np.zeros((1, 1)), None)[0, 0] < -9.9 else 1.0
+    return max(e1, e2, e3, e4, e5)
+
+
+def pin_q_scale():
+    """o = q_scale S^T q: the hand example's outputs at q_scale = 2 are twice those at
+    1 and the state is unchanged; through the layer with a huge RMSNorm eps (so y is
+    proportional to o) y doubles too."""
+    gv = _read_golden('recurrence_d2_hand.txt')
+    q = np.stack([gv['q1'], gv['q2']])
+    k = np.stack([gv['k1'], gv['k2']])
+    v = np.stack([gv['v1'], gv['v2']])
+    loga = np.log(np.stack([gv['a1'], gv['a2']]))
+    beta = np.array([gv['b1'][0], gv['b2'][0]])
+    o2, S2 = ko.recurrence(q, k, v, loga, beta, q_scale=2.0)
+    e1 = max(np.abs(o2[0] - 2 * gv['o1']).max(), np.abs(o2[1] - 2 * gv['o2']).max(),
+             np.abs(S2.reshape(-1) - gv['S2']).max())
+    inp = _layer_inputs(19, 9)
+    y1 = ko.layer(cu_seqlens=[0, 9], **inp, norm_eps=1e12)['y']
+    y2 = ko.layer(cu_seqlens=[0, 9], **inp, norm_eps=1e12, q_scale=2.0)['y']
+    e2 = np.abs(y2 - 2 * y1).max() / np.abs(y1).max()
+    return max(e1, e2)
+
+
 def pin_conv_library():
     """Conv against numpy.convolve with the kernel reversed (cross-correlation)."""
     rng = _rng(1)
@@ -234,6 +279,14 @@ def test_log_decay_closed_forms():
     assert np.all(np.exp(lo) == 1.0)    # a = 1 exactly
 
 
+def test_softplus_decay_closed_forms():
+    assert pin_softplus_decay() < 1e-12
+
+
+def test_q_scale_doubles_outputs():
+    assert pin_q_scale() < 1e-10
+
+
 def test_conv_matches_numpy_convolve():
     assert pin_conv_library() < 1e-13
 
@@ -383,6 +436,7 @@ def _all_pins():
         'prep': pin_prep_composition, 'l2': pin_l2_library, 'rmsnorm': pin_rmsnorm,
         'hand': pin_hand_example, 'brute_square': lambda: pin_brute_force(8, 8),
         'beta_zero': pin_beta_zero, 'retrieval': pin_retrieval,
+        'softplus': pin_softplus_decay, 'q_scale': pin_q_scale,
     }
     out = {}
     for name, fn in pins.items():
@@ -404,6 +458,30 @@ def _mut_reversed_taps(x, w, hist=None):
 def _mut_softplus_decay(f, A_log, dt_bias, lb=-5.0):
     A = np.exp(np.asarray(A_log))[:, None]
     return -A * np.logaddexp(0.0, np.asarray(f) + dt_bias)
+
+
+def _mut_softplus_bias_sign(f, A_log, dt_bias, lb=-5.0):
+    """Mutation of the softplus branch only: the bias subtracted instead of added."""
+    if lb is not None:
+        return ko.__dict__['_orig_log_decay'](f, A_log, dt_bias, lb)
+    A = np.exp(np.asarray(A_log))[:, None]
+    return -A * np.logaddexp(0.0, np.asarray(f) - dt_bias)
+
+
+def _mut_softplus_no_rate(f, A_log, dt_bias, lb=-5.0):
+    """Mutation of the softplus branch only: the per-head rate exp(A_log) dropped."""
+    if lb is not None:
+        return ko.__dict__['_orig_log_decay'](f, A_log, dt_bias, lb)
+    return -np.logaddexp(0.0, np.asarray(f) + dt_bias)
+
+
+def _mut_q_scale_squared(q, k, v, loga, beta, S0=None, q_scale=1.0, return_states=False):
+    return ko.__dict__['_orig_recurrence'](q, k, v, loga, beta, S0, q_scale * q_scale,
+                                           return_states)
+
+
+def _mut_layer_drops_q_scale(*args, q_scale=1.0, **kw):
+    return ko.__dict__['_orig_layer'](*args, **kw)
 
 
 def _mut_value_axis(S, a):
@@ -445,6 +523,10 @@ MUTATIONS = {
     'value_axis_decay': ('apply_key_decay', _mut_value_axis),
     'missing_output_gate': ('gated_rmsnorm', _mut_no_gate),
     'decay_after_update': ('recurrence', _mut_decay_after_update),
+    'softplus_bias_sign': ('log_decay', _mut_softplus_bias_sign),
+    'softplus_no_rate': ('log_decay', _mut_softplus_no_rate),
+    'q_scale_squared': ('recurrence', _mut_q_scale_squared),
+    'layer_drops_q_scale': ('layer', _mut_layer_drops_q_scale),
 }
 
 
@@ -452,6 +534,9 @@ MUTATIONS = {
 def test_mutation_is_caught(name, monkeypatch):
     attr, fn = MUTATIONS[name]
     monkeypatch.setitem(ko.__dict__, '_orig_conv', ko.causal_depthwise_conv)
+    monkeypatch.setitem(ko.__dict__, '_orig_log_decay', ko.log_decay)
+    monkeypatch.setitem(ko.__dict__, '_orig_recurrence', ko.recurrence)
+    monkeypatch.setitem(ko.__dict__, '_orig_layer', ko.layer)
     monkeypatch.setattr(ko, attr, fn)
     pins = _all_pins()
     failing = [k for k, e in pins.items() if not (e < 1e-10)]

@@ -8,15 +8,12 @@ collected last so that a run stopping at the first failure has already run
 every other test; it passes alone in a fresh process (whose first call does
 the per-device set-up) and after the other tests.
 """
-import numpy as np
 import pytest
 import torch
 
 from linear_attention_recurrence_09_b200 import kda, synth
-from tests.kda_cases import np64, rel_err
 
 pytestmark = pytest.mark.gpu
-TOL = 1e-2
 
 
 def _prep(cfg, P, A):
@@ -46,8 +43,10 @@ def test_noalloc_matches_prefill_on_two_calls_in_a_row(dtype, d, chunk):
                                 p['beta'], A['g'], P['norm_w'], state_in=s_na, state_out=s_na,
                                 y=y_na)
         torch.cuda.synchronize()
-        assert rel_err(np64(y_na), np64(y_ref)) <= TOL, call
-        assert rel_err(np64(s_na), np64(s_ref)) <= TOL, call
+        # the same deterministic kernels on the same inputs: any byte of stale scratch
+        # that leaked into the result would show as a difference
+        assert torch.equal(y_na, y_ref), call
+        assert torch.equal(s_na, s_ref), call
         assert not torch.isnan(y_na.float()).any()
 
 
