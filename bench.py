@@ -43,7 +43,8 @@ def parse_args():
     ap.add_argument('--tokens', type=int, default=8192, help='prefill length (8192 = headline)')
     ap.add_argument('--no-extras', action='store_true', help='skip decode / verify workloads')
     ap.add_argument('--no-cpu', action='store_true', help='skip the CPU oracle baseline')
-    ap.add_argument('--only', default='', help='prefill|decode|verify|long: run one workload only')
+    ap.add_argument('--only', default='',
+                    help='prefill|decode|verify|long|layer_full: run one workload only')
     ap.add_argument('--no-long', action='store_true', help='skip the long / varlen workload')
     return ap.parse_args()
 
@@ -440,6 +441,74 @@ def run_prefill(args, dist, torch, kda, synth, dev):
     return res
 
 
+def run_layer_full(torch, kda, synth, dev, steps=10, warmup=3):
+    """The layer from hidden states (B = 1, T = 8192, H = 32, d = 128, hidden 4096, gate
+    rank 128, random-init weights): the fused input projection and the low-rank gate as
+    two kda_proj_gemm launches, then kda_layer_prefill.  Reports tokens/s for the whole
+    x -> y layer and the projections' tensor-core fraction (GEMM flops over their
+    event-timed duration at the measured bf16 dense peak)."""
+    w = synth.WORKLOADS['layer_8k_projections']
+    T, H, d, hidden, r = w['seqlen'], w['heads'], w['head_dim'], w['hidden'], w['gate_rank']
+    cfg = kda.Config(num_heads=H, head_dim=d, conv_size=4, dtype=torch.bfloat16, chunk_size=64)
+    W = {k: v.to(dev) for k, v in synth.proj_weights(w['seed'], hidden, H, d, r).items()}
+    P = {k: v.to(dev) for k, v in synth.layer_params(w['seed'], H, d, 4).items()}
+    hs = synth.hidden_states(w['seed'], T, hidden).to(dev)
+    cu = torch.tensor([0, T], dtype=torch.int32, device=dev)
+    o = {'x': torch.empty(T, H, 3 * d, dtype=cfg.dtype, device=dev),
+         'f': torch.empty(T, H, d, dtype=cfg.dtype, device=dev),
+         'beta_logit': torch.empty(T, H, dtype=cfg.dtype, device=dev),
+         'g_a': torch.empty(T, r, dtype=cfg.dtype, device=dev),
+         'g': torch.empty(T, H, d, dtype=cfg.dtype, device=dev)}
+    y = torch.empty(T, H, d, dtype=cfg.dtype, device=dev)
+    state = torch.empty(1, H, d, d, device=dev)
+    ws = torch.empty(kda.kda_layer_prefill_workspace_size(cfg, 1, T), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream()
+
+    def ev():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        return e
+
+    def step(e=None):
+        if e:
+            e[0].record(stream)
+        kda.layer_projections(cfg, hs, W['W_in'], W['W_gb'], r, out=o)
+        if e:
+            e[1].record(stream)
+        kda.kda_layer_prefill(cfg, cu, o['x'], o['f'], o['beta_logit'], o['g'], P['conv_w'],
+                              P['A_log'], P['dt_bias'], P['norm_w'], state_out=state, y=y,
+                              workspace=ws, max_seqlen=T)
+        if e:
+            e[2].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[ev() for _ in range(3)] for _ in range(steps)]
+    n0 = kda.kda_launch_count()
+    for i in range(steps):
+        step(evs[i])
+    launches = (kda.kda_launch_count() - n0) // steps
+    torch.cuda.synchronize()
+    ms = statistics.median(e[0].elapsed_time(e[2]) for e in evs)
+    ms_gemm = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    n_in = 4 * H * d + H + r
+    flops = 2 * T * hidden * n_in + 2 * T * r * H * d
+    _, tc, tc_sus, peak_kind = measured_peaks()
+    ach = flops / (ms_gemm / 1e3) / 1e12
+    return {'value': T / (ms / 1e3), 'unit': 'tokens/s',
+            'workload': f'layer from hidden states: B=1 T={T} H={H} d={d} hidden={hidden} gate '
+                        f'rank {r}; fused input projection [{n_in} x {hidden}] + g_b '
+                        f'[{H * d} x {r}] (random-init bf16 weights) + KDA layer',
+            'ms_per_step': ms, 'ms_projections': ms_gemm, 'ms_layer': ms - ms_gemm,
+            'launches_per_step': launches,
+            'tensor_roofline': {'bound': 'tensor', 'kernel': 'kda_proj_gemm (2 launches)',
+                                'achieved': ach, 'peak': tc, 'unit': 'TFLOP/s',
+                                'frac': ach / tc, 'frac_sustained': ach / tc_sus,
+                                'gflop_per_step': flops / 1e9, 'peak_kind': peak_kind}}
+
+
 def run_long(torch, kda, synth, dev, steps=5, warmup=3):
     """The long / varlen prefill workload: one B = 1, T = 131,072 sequence, and 8 packed
     sequences of log-uniform lengths in [1,024, 32,768]; H = 32, d = 128, bf16, initial
@@ -620,54 +689,77 @@ def run_verify(torch, kda, synth, dev, rounds=256):
          'log_a': torch.empty(B * Tb, H, d, device=dev), 'beta': torch.empty(B * Tb, H, device=dev)}
     win = torch.empty(B * (Tb + K - 1), H, 3 * d, dtype=cfg.dtype, device=dev)
     tape = torch.empty(B, Tb, H, d, d, device=dev)
+    kua = torch.empty(B, Tb, H, 3, d, device=dev)
     y = torch.empty(B, Tb, H, d, dtype=cfg.dtype, device=dev)
     v4 = lambda t, *tail: t.view(B, Tb, *tail)
+    vargs = lambda r: (v4(o['q'], H, d), v4(o['k'], H, d), v4(o['v'], H, d),
+                       v4(o['log_a'], H, d), v4(o['beta'], H), X['g'][r], P['norm_w'], state)
 
-    def one(r):
+    def one(r, compact):
+        # prep (conv window for the rollback), verify, rollback to the accepted prefix
         kda.kda_prep(cfg, cu, X['x'][r].view(B * Tb, H, 3 * d), X['f'][r].view(B * Tb, H, d),
                      X['beta_logit'][r].view(B * Tb, H), P['conv_w'], P['A_log'], P['dt_bias'],
                      conv_state=conv, conv_mode=kda.KDA_CONV_TAPE, conv_window=win,
                      max_seqlen=Tb, out=o)
-        kda.kda_verify(cfg, v4(o['q'], H, d), v4(o['k'], H, d), v4(o['v'], H, d),
-                       v4(o['log_a'], H, d), v4(o['beta'], H), X['g'][r], P['norm_w'], state,
-                       tape=tape, y=y)
-        kda.kda_rollback(cfg, acc[r], tape, state, conv_window=win, conv_state=conv)
+        if compact:
+            kda.kda_verify_compact(cfg, *vargs(r), tape_kua=kua, y=y)
+            kda.kda_rollback_replay(cfg, acc[r], kua, state, conv_window=win, conv_state=conv)
+        else:
+            kda.kda_verify(cfg, *vargs(r), tape=tape, y=y)
+            kda.kda_rollback(cfg, acc[r], tape, state, conv_window=win, conv_state=conv)
 
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
-        one(0)
-    torch.cuda.current_stream().wait_stream(s)
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        for r in range(rounds):
-            one(r)
-    g.replay()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    g.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    n = 100
-    e0.record()
-    for _ in range(n):
-        kda.kda_verify(cfg, v4(o['q'], H, d), v4(o['k'], H, d), v4(o['v'], H, d),
-                       v4(o['log_a'], H, d), v4(o['beta'], H), X['g'][0], P['norm_w'], state,
-                       tape=tape, y=y)
-    e1.record()
-    torch.cuda.synchronize()
-    ms_k = e0.elapsed_time(e1) / n
-    bytes_k = B * H * (d * d * 4 + Tb * d * d * 4 + Tb * (3 * d * 4 + d * 2 + d * 4 + 4 + d * 2))
+    def graph_ms(compact):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            one(0, compact)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for r in range(rounds):
+                one(r, compact)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1)
+
+    def launch_ms(fn, n=100):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    ms = graph_ms(True)
+    ms_full = graph_ms(False)
+    ms_k = launch_ms(lambda: kda.kda_verify_compact(cfg, *vargs(0), tape_kua=kua, y=y))
+    ms_r = launch_ms(lambda: kda.kda_rollback_replay(cfg, acc[0], kua, state, conv_window=win,
+                                                     conv_state=conv))
+    io = Tb * (3 * d * 4 + d * 4 + 4 + d * 2 + d * 2)          # q, k, v, log a, beta, g in; y out
+    bytes_k = B * H * (d * d * 4 + io + Tb * 3 * d * 4)         # + the state in, compact tape out
+    n_acc = int((acc[0] > 0).sum())
+    bytes_r = n_acc * H * (2 * d * d * 4) + int(acc[0].sum()) * H * 3 * d * 4
     hbm, _, _, peak_kind = measured_peaks()
-    del g
     return {'value': B * Tb * rounds / (ms / 1e3), 'unit': 'verified draft tokens/s',
             'workload': f'verify+rollback B={B} H={H} d={d}, blocks of {Tb} after a {T0}-token '
-                        f'context, {rounds} rounds, accepted ~ U{{0..{Tb}}} (CUDA graph)',
+                        f'context, {rounds} rounds, accepted ~ U{{0..{Tb}}} (CUDA graph; '
+                        'compact (k, u, a) tape, rollback by replay)',
             'ms_per_round': ms / rounds, 'gpu_launches': 3 * rounds,
-            'roofline': hbm_roofline('kda_verify', bytes_k, ms_k, hbm, peak_kind)}
+            'full_state_tape_ms_per_round': ms_full / rounds,
+            'roofline': hbm_roofline('kda_verify_compact', bytes_k, ms_k, hbm, peak_kind),
+            'rollback_replay': {'ms_per_launch': ms_r, 'algorithmic_bytes_per_launch': bytes_r,
+                                'frac': bytes_r / (ms_r / 1e3) / 1e9 / hbm}}
 
 
 # ---------------------------------------------------------------------------
@@ -755,6 +847,8 @@ def main():
                 res['verify'] = run_verify(torch, kda, synth, dev)
             if args.only in ('', 'long') and not args.no_long:
                 res['long'] = run_long(torch, kda, synth, dev)
+            if args.only in ('', 'layer_full'):
+                res['layer_full'] = run_layer_full(torch, kda, synth, dev)
         if dist.rank == 0 and dist.world == 1 and not args.no_cpu and args.only in ('', 'prefill'):
             res['cpu_baseline'] = cpu_baseline(torch, synth)
         if dist.rank == 0:

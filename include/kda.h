@@ -7,7 +7,8 @@
  *
  *   prep   x~ = depthwise causal conv over q|k|v (one kernel, K taps), then SiLU
  *          q = q~ / max(||q~||, l2_eps),  k = k~ / max(||k~||, l2_eps),  v = v~
- *          log a_t = lb * sigmoid(exp(A_log[h]) * (f_t + dt_bias[h]))   (per key channel)
+ *          log a_t = lb * sigmoid(exp(A_log[h]) * (f_t + dt_bias[h]))   (per key channel;
+ *                    or -exp(A_log[h]) * softplus(f_t + dt_bias[h]), enum kda_gate)
  *          b_t = sigmoid(beta_logit_t)
  *   state  S_t = (I - b_t k_t k_t^T) Diag(a_t) S_{t-1} + b_t k_t v_t^T   (S is d_k x d_v,
  *          decay on the key axis; order: decay, delta update, read)
@@ -84,6 +85,20 @@ enum kda_conv_mode {
   KDA_CONV_TAPE = 1    /* conv_state read only; conv_window <- [conv_state; x] */
 };
 
+/*
+ * Decay gate (per key channel, A = exp(A_log[h])).  PR #27754, "Metadata and tensor
+ * loading" commit: the bounded-sigmoid branch is selected by the gate_lower_bound key
+ * and, when the key is absent, a softplus branch, "a different function":
+ *   KDA_GATE_BOUNDED_SIGMOID  log a = lb * sigmoid(A (f + dt_bias)),  lb in [-5, 0)
+ *   KDA_GATE_SOFTPLUS         log a = -A * softplus(f + dt_bias)      (lb ignored)
+ * The softplus gate has no lower bound, so a chunk's cumulative decay can span far
+ * more than fp32's exponent range; the tensor-core prefill passes rely on the bound
+ * (their exponent split keeps every factor within e^80) and a softplus layer runs on
+ * the SIMT prefill passes, whose gram takes one exponential per (pair, channel)
+ * inside each 16-token block instead of splitting it.
+ */
+enum kda_gate { KDA_GATE_BOUNDED_SIGMOID = 0, KDA_GATE_SOFTPLUS = 1 };
+
 /* Layer configuration (host memory, read during the call only). */
 typedef struct kda_config {
   int32_t num_heads;      /* H >= 1 */
@@ -91,11 +106,12 @@ typedef struct kda_config {
   int32_t conv_size;      /* K taps of the short conv, 1..8 (4 in GLM-5.3-Flash) */
   int32_t dtype;          /* enum kda_dtype of the activations */
   int32_t chunk_size;     /* prefill chunk length in {16, 32, 64} */
-  float gate_lower_bound; /* lb of the bounded-sigmoid decay, in [-5, 0): PR #27754
-                             makes gate_lower_bound a required key; GLM-5.3-Flash uses -5 */
+  float gate_lower_bound; /* lb of the bounded-sigmoid decay, in [-5, 0) (GLM-5.3-Flash:
+                             -5); ignored by the softplus gate */
   float l2_eps;           /* q/k L2 eps, 1e-6 ("a literal 1e-6", PR #27754) */
   float norm_eps;         /* output RMSNorm eps, 1e-5 (rms_norm_eps, glm53-flash-mlx README) */
   float q_scale;          /* multiplies o = S^T q; 1.0 */
+  int32_t gate_kind;      /* enum kda_gate: which decay-gate function (see below) */
 } kda_config;
 
 /* Human-readable name of a kda_status code (static string, never NULL). */
@@ -297,6 +313,77 @@ KDA_API int kda_rollback(const kda_config* cfg, int32_t batch, int32_t block_len
                  const void* conv_window, float* state, void* conv_state,
                  const int32_t* state_slots, int32_t pool_size,
                  kda_stream_t stream);
+
+/*
+ * Compact verify tape and rollback by replay.  dflash-mlx issue #63, "What the backend
+ * needs": the KDA recurrent state is to roll back the way the GatedDeltaNet
+ * tape-replay path does.  Each verify step changes the state by
+ *   S_j = Diag(a_j) S_{j-1} + k_j u_j^T,   u_j = b_j (v_j - (Diag(a_j) S_{j-1})^T k_j),
+ * so the step is recorded as the three d-vectors (k_j, u_j, a_j) instead of the
+ * d x d state (3d floats: 1.5 KB instead of 64 KB per head at d = 128), and rollback
+ * to L accepted drafts replays L such updates from the live state, which verify left
+ * untouched.  The replay performs the step kernel's own operations on each element
+ * (a multiply by a, then one fused multiply-add of k u), so the rolled-back state is
+ * bit-identical to the full tape's entry tape[L-1].
+ *
+ *  tape_kua  fp32 [batch, block_len, H, 3, d]: per step and head k, u, a (a = e^{log a})
+ *
+ * kda_verify_compact       - kda_verify writing tape_kua instead of the full tape.
+ * kda_layer_verify_compact - kda_layer_verify writing tape_kua instead of the full tape.
+ * kda_rollback_replay      - kda_rollback from tape_kua: for L = accepted[b] >= 1 the
+ *                            state row is replaced by L replayed steps (in place) and
+ *                            the conv state by conv_window rows [L, L+K-1); L = 0 leaves
+ *                            both untouched.  Run it on the state verify read, before
+ *                            anything else changes that state.
+ */
+KDA_API int kda_verify_compact(const kda_config* cfg, int32_t batch, int32_t block_len,
+                               const void* q, const void* k, const void* v,
+                               const float* log_a, const float* beta, const void* g,
+                               const float* norm_w, const float* state,
+                               const int32_t* state_slots, int32_t pool_size, float* tape_kua,
+                               void* y, kda_stream_t stream);
+KDA_API int kda_layer_verify_compact(const kda_config* cfg, int32_t batch, int32_t block_len,
+                                     const void* x, const void* f, const void* beta_logit,
+                                     const void* g, const float* conv_w, const float* A_log,
+                                     const float* dt_bias, const float* norm_w,
+                                     const void* conv_state, const float* state,
+                                     const int32_t* state_slots, int32_t pool_size,
+                                     float* tape_kua, void* conv_window, void* y,
+                                     kda_stream_t stream);
+KDA_API int kda_rollback_replay(const kda_config* cfg, int32_t batch, int32_t block_len,
+                                const int32_t* accepted, const float* tape_kua,
+                                const void* conv_window, float* state, void* conv_state,
+                                const int32_t* state_slots, int32_t pool_size,
+                                kda_stream_t stream);
+
+/*
+ * kda_proj_gemm - the layer's projections: C = A B^T on the tensor cores, bf16 operands,
+ * fp32 accumulation, bf16 results.  glm53-flash-mlx README, quantization recipe: the
+ * runtime fuses the six KDA input projections into one matmul; llama.cpp PR #27754, KDA
+ * commit: the output gate is low rank, g_b(g_a(x)).  With A the hidden states and B the
+ * fused input weight, one call produces q|k|v (pre-conv), f, the beta logit and g_a,
+ * each written to its own dense tensor by the output ranges below; a second call with
+ * A = g_a and B = the g_b weight produces g.
+ *
+ *  A       bf16 [M, K] row-major (one row per token)
+ *  B       bf16 [N, K] row-major (the weight, one row per output column)
+ *  outs    host array of n_outs (1..4) ranges: columns [col_begin, col_end) of C go to
+ *          out[row * ld + (col - col_begin)], bf16, device memory.  col_begin, col_end
+ *          and ld are multiples of 8, 0 <= col_begin < col_end <= N, ld >= the range's
+ *          width, and the ranges do not overlap; columns outside every range are dropped.
+ *  status  optional device int32 the caller clears: set to KDA_ERR_TIMEOUT if a bounded
+ *          device wait gave up (read it with kda_workspace_status), or NULL.
+ *  M >= 0, N >= 0 (a multiple of 8), K >= 8 (a multiple of 8); M = 0 or N = 0 launches
+ *  nothing.
+ */
+typedef struct kda_proj_out {
+  void* out;
+  int64_t ld;
+  int32_t col_begin, col_end;
+} kda_proj_out;
+KDA_API int kda_proj_gemm(int32_t M, int32_t N, int32_t K, const void* A, const void* B,
+                          const kda_proj_out* outs, int32_t n_outs, void* status,
+                          kda_stream_t stream);
 
 /*
  * kda_workspace_status - synchronises `stream`, then reads the status word

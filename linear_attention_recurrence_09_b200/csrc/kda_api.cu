@@ -19,9 +19,13 @@ int check_cfg(const kda_config* c) {
     return KDA_ERR_UNSUPPORTED;
   if (c->chunk_size != 16 && c->chunk_size != 32 && c->chunk_size != 64)
     return KDA_ERR_UNSUPPORTED;
-  // lb >= -5 keeps a 16-token sub-chunk's decay span <= 80 (< fp32 exp overflow)
-  if (!std::isfinite(c->gate_lower_bound) || c->gate_lower_bound < -5.0f ||
-      c->gate_lower_bound >= 0.0f)
+  if (c->gate_kind != KDA_GATE_BOUNDED_SIGMOID && c->gate_kind != KDA_GATE_SOFTPLUS)
+    return KDA_ERR_INVALID_ARG;
+  // lb >= -5 keeps a 16-token sub-chunk's decay span <= 80 (< fp32 exp overflow); the
+  // softplus gate ignores lb
+  if (c->gate_kind == KDA_GATE_BOUNDED_SIGMOID &&
+      (!std::isfinite(c->gate_lower_bound) || c->gate_lower_bound < -5.0f ||
+       c->gate_lower_bound >= 0.0f))
     return KDA_ERR_UNSUPPORTED;
   if (!(c->l2_eps > 0.0f) || !std::isfinite(c->l2_eps)) return KDA_ERR_INVALID_ARG;
   if (!(c->norm_eps >= 0.0f) || !std::isfinite(c->norm_eps)) return KDA_ERR_INVALID_ARG;
@@ -77,7 +81,7 @@ const char* kda_status_string(int status) {
   return "unknown kda status";
 }
 
-int kda_abi_version(void) { return 1; }
+int kda_abi_version(void) { return 2; }
 
 int kda_prep(const kda_config* cfg, int32_t n_seqs, int32_t total_tokens,
              const int32_t* cu_seqlens, int32_t max_seqlen, const void* x, const void* f,
@@ -113,6 +117,7 @@ int kda_prep(const kda_config* cfg, int32_t n_seqs, int32_t total_tokens,
   a.q = static_cast<float*>(q); a.k = static_cast<float*>(k); a.v = static_cast<float*>(v);
   a.loga = log_a; a.beta = beta;
   a.lb = cfg->gate_lower_bound; a.l2_eps = cfg->l2_eps;
+  a.gate_softplus = cfg->gate_kind == KDA_GATE_SOFTPLUS;
   return cuda_status(kda::launch_prep(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -157,6 +162,7 @@ int kda_prefill(const kda_config* cfg, int32_t n_seqs, int32_t total_tokens,
   a.pool_size = pooled ? pool_size : n_seqs;
   a.y = y; a.ws = static_cast<char*>(workspace); a.L = L;
   a.norm_eps = cfg->norm_eps; a.q_scale = cfg->q_scale; a.lb = cfg->gate_lower_bound;
+  a.gate_softplus = cfg->gate_kind == KDA_GATE_SOFTPLUS;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(a.ws + L.status, 0, 256, s) != cudaSuccess) return KDA_ERR_CUDA;
   return cuda_status(kda::launch_prefill(a, s));
@@ -169,8 +175,10 @@ static size_t layer_prep_bytes(const kda_config* c, int32_t total) {
   return ((th * c->head_dim * 4 * 4 + th * 4) + 255) & ~(size_t)255;
 }
 
+// prep inside the tcgen05 intra-chunk pass: bf16, d = 128, chunk 64, K = 4, bounded gate
 static bool layer_fused(const kda_config* c) {
-  return c->dtype == KDA_BF16 && c->head_dim == 128 && c->chunk_size == 64 && c->conv_size == 4;
+  return c->dtype == KDA_BF16 && c->head_dim == 128 && c->chunk_size == 64 &&
+         c->conv_size == 4 && c->gate_kind == KDA_GATE_BOUNDED_SIGMOID;
 }
 
 size_t kda_layer_prefill_workspace_size(const kda_config* cfg, int32_t n_seqs,
@@ -219,6 +227,7 @@ int kda_layer_prefill(const kda_config* cfg, int32_t n_seqs, int32_t total_token
   p.pool_size = conv_state ? pool : n_seqs;
   p.mode = KDA_CONV_COMMIT;
   p.lb = cfg->gate_lower_bound; p.l2_eps = cfg->l2_eps;
+  p.gate_softplus = cfg->gate_kind == KDA_GATE_SOFTPLUS;
 
   kda::PrefillArgs a{};
   a.cu = cu_seqlens; a.n_seqs = n_seqs; a.total = total_tokens;
@@ -230,6 +239,7 @@ int kda_layer_prefill(const kda_config* cfg, int32_t n_seqs, int32_t total_token
   a.y = y; a.ws = static_cast<char*>(workspace); a.L = L;
   a.norm_eps = cfg->norm_eps; a.q_scale = cfg->q_scale; a.lb = cfg->gate_lower_bound;
   a.l2_eps = cfg->l2_eps; a.K = cfg->conv_size;
+  a.gate_softplus = cfg->gate_kind == KDA_GATE_SOFTPLUS;
   if (cudaMemsetAsync(a.ws + L.status, 0, 256, s) != cudaSuccess) return KDA_ERR_CUDA;
 
   if (layer_fused(cfg)) {
@@ -268,7 +278,7 @@ int kda_set_phase_events(void* const* events, int32_t n) {
 static int step_common(const kda_config* cfg, int32_t batch, int32_t T, const void* q,
                        const void* k, const void* v, const float* log_a, const float* beta,
                        const void* g, const float* norm_w, const float* state_in,
-                       float* state_out, float* tape, const int32_t* slots,
+                       float* state_out, float* tape, float* tape_kua, const int32_t* slots,
                        int32_t pool_size, void* y, kda_stream_t stream) {
   int st = check_cfg(cfg);
   if (st) return st;
@@ -282,7 +292,7 @@ static int step_common(const kda_config* cfg, int32_t batch, int32_t T, const vo
   a.q = static_cast<const float*>(q); a.k = static_cast<const float*>(k);
   a.v = static_cast<const float*>(v);
   a.loga = log_a; a.beta = beta; a.g = g; a.norm_w = norm_w;
-  a.state_in = state_in; a.state_out = state_out; a.tape = tape;
+  a.state_in = state_in; a.state_out = state_out; a.tape = tape; a.tape_kua = tape_kua;
   a.slots = slots; a.pool_size = pool_size; a.y = y;
   a.norm_eps = cfg->norm_eps; a.q_scale = cfg->q_scale;
   return cuda_status(kda::launch_step(a, reinterpret_cast<cudaStream_t>(stream)));
@@ -292,7 +302,7 @@ static int layer_step_common(const kda_config* cfg, int32_t batch, int32_t T, co
                              const void* f, const void* beta_logit, const void* g,
                              const float* conv_w, const float* A_log, const float* dt_bias,
                              const float* norm_w, void* conv_state, const float* state_in,
-                             float* state_out, float* tape, void* window,
+                             float* state_out, float* tape, float* tape_kua, void* window,
                              const int32_t* slots, int32_t pool_size, void* y,
                              kda_stream_t stream) {
   int st = check_cfg(cfg);
@@ -307,13 +317,14 @@ static int layer_step_common(const kda_config* cfg, int32_t batch, int32_t T, co
   a.B = batch; a.T = T; a.H = cfg->num_heads; a.D = cfg->head_dim;
   a.bf16 = cfg->dtype == KDA_BF16;
   a.g = g; a.norm_w = norm_w;
-  a.state_in = state_in; a.state_out = state_out; a.tape = tape;
+  a.state_in = state_in; a.state_out = state_out; a.tape = tape; a.tape_kua = tape_kua;
   a.slots = slots; a.pool_size = pool_size; a.y = y;
   a.norm_eps = cfg->norm_eps; a.q_scale = cfg->q_scale;
   a.x = x; a.f = f; a.beta_logit = beta_logit;
   a.conv_w = conv_w; a.A_log = A_log; a.dt_bias = dt_bias;
   a.conv_state = conv_state; a.window = window; a.K = cfg->conv_size;
   a.lb = cfg->gate_lower_bound; a.l2_eps = cfg->l2_eps;
+  a.gate_softplus = cfg->gate_kind == KDA_GATE_SOFTPLUS;
   return cuda_status(kda::launch_step(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -323,8 +334,26 @@ int kda_layer_decode(const kda_config* cfg, int32_t batch, const void* x, const 
                      void* conv_state, float* state, const int32_t* state_slots,
                      int32_t pool_size, void* y, kda_stream_t stream) {
   return layer_step_common(cfg, batch, 1, x, f, beta_logit, g, conv_w, A_log, dt_bias, norm_w,
-                           conv_state, state, state, nullptr, nullptr, state_slots, pool_size,
-                           y, stream);
+                           conv_state, state, state, nullptr, nullptr, nullptr, state_slots,
+                           pool_size, y, stream);
+}
+
+static int layer_verify_common(const kda_config* cfg, int32_t batch, int32_t block_len,
+                               const void* x, const void* f, const void* beta_logit,
+                               const void* g, const float* conv_w, const float* A_log,
+                               const float* dt_bias, const float* norm_w,
+                               const void* conv_state, const float* state,
+                               const int32_t* state_slots, int32_t pool_size, float* tape,
+                               float* tape_kua, void* conv_window, void* y,
+                               kda_stream_t stream) {
+  if (block_len < 1 || block_len > 16) return KDA_ERR_INVALID_ARG;
+  if (batch > 0) {
+    int st = check_ptrs({tape ? tape : tape_kua, conv_window}, {});
+    if (st) return st;
+  }
+  return layer_step_common(cfg, batch, block_len, x, f, beta_logit, g, conv_w, A_log, dt_bias,
+                           norm_w, const_cast<void*>(conv_state), state, nullptr, tape,
+                           tape_kua, conv_window, state_slots, pool_size, y, stream);
 }
 
 int kda_layer_verify(const kda_config* cfg, int32_t batch, int32_t block_len, const void* x,
@@ -333,14 +362,23 @@ int kda_layer_verify(const kda_config* cfg, int32_t batch, int32_t block_len, co
                      const float* norm_w, const void* conv_state, const float* state,
                      const int32_t* state_slots, int32_t pool_size, float* tape,
                      void* conv_window, void* y, kda_stream_t stream) {
-  if (block_len < 1 || block_len > 16) return KDA_ERR_INVALID_ARG;
-  if (batch > 0) {
-    int st = check_ptrs({tape, conv_window}, {});
-    if (st) return st;
-  }
-  return layer_step_common(cfg, batch, block_len, x, f, beta_logit, g, conv_w, A_log, dt_bias,
-                           norm_w, const_cast<void*>(conv_state), state, nullptr, tape,
-                           conv_window, state_slots, pool_size, y, stream);
+  if (batch > 0 && tape == nullptr) return KDA_ERR_INVALID_ARG;
+  return layer_verify_common(cfg, batch, block_len, x, f, beta_logit, g, conv_w, A_log,
+                             dt_bias, norm_w, conv_state, state, state_slots, pool_size, tape,
+                             nullptr, conv_window, y, stream);
+}
+
+int kda_layer_verify_compact(const kda_config* cfg, int32_t batch, int32_t block_len,
+                             const void* x, const void* f, const void* beta_logit,
+                             const void* g, const float* conv_w, const float* A_log,
+                             const float* dt_bias, const float* norm_w,
+                             const void* conv_state, const float* state,
+                             const int32_t* state_slots, int32_t pool_size, float* tape_kua,
+                             void* conv_window, void* y, kda_stream_t stream) {
+  if (batch > 0 && tape_kua == nullptr) return KDA_ERR_INVALID_ARG;
+  return layer_verify_common(cfg, batch, block_len, x, f, beta_logit, g, conv_w, A_log,
+                             dt_bias, norm_w, conv_state, state, state_slots, pool_size,
+                             nullptr, tape_kua, conv_window, y, stream);
 }
 
 int kda_decode(const kda_config* cfg, int32_t batch, const void* q, const void* k,
@@ -348,7 +386,7 @@ int kda_decode(const kda_config* cfg, int32_t batch, const void* q, const void* 
                const float* norm_w, float* state, const int32_t* state_slots,
                int32_t pool_size, void* y, kda_stream_t stream) {
   return step_common(cfg, batch, 1, q, k, v, log_a, beta, g, norm_w, state, state, nullptr,
-                     state_slots, pool_size, y, stream);
+                     nullptr, state_slots, pool_size, y, stream);
 }
 
 int kda_verify(const kda_config* cfg, int32_t batch, int32_t block_len, const void* q,
@@ -362,7 +400,21 @@ int kda_verify(const kda_config* cfg, int32_t batch, int32_t block_len, const vo
     if (st) return st;
   }
   return step_common(cfg, batch, block_len, q, k, v, log_a, beta, g, norm_w, state, nullptr,
-                     tape, state_slots, pool_size, y, stream);
+                     tape, nullptr, state_slots, pool_size, y, stream);
+}
+
+int kda_verify_compact(const kda_config* cfg, int32_t batch, int32_t block_len, const void* q,
+                       const void* k, const void* v, const float* log_a, const float* beta,
+                       const void* g, const float* norm_w, const float* state,
+                       const int32_t* state_slots, int32_t pool_size, float* tape_kua,
+                       void* y, kda_stream_t stream) {
+  if (block_len < 1 || block_len > 16) return KDA_ERR_INVALID_ARG;
+  if (batch > 0) {
+    int st = check_ptrs({tape_kua}, {});
+    if (st) return st;
+  }
+  return step_common(cfg, batch, block_len, q, k, v, log_a, beta, g, norm_w, state, nullptr,
+                     nullptr, tape_kua, state_slots, pool_size, y, stream);
 }
 
 int kda_rollback(const kda_config* cfg, int32_t batch, int32_t block_len,
@@ -383,6 +435,54 @@ int kda_rollback(const kda_config* cfg, int32_t batch, int32_t block_len,
   a.accepted = accepted; a.tape = tape; a.window = conv_window; a.state = state;
   a.conv_state = conv_state; a.slots = state_slots; a.pool_size = pool_size;
   return cuda_status(kda::launch_rollback(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int kda_rollback_replay(const kda_config* cfg, int32_t batch, int32_t block_len,
+                        const int32_t* accepted, const float* tape_kua,
+                        const void* conv_window, float* state, void* conv_state,
+                        const int32_t* state_slots, int32_t pool_size, kda_stream_t stream) {
+  int st = check_cfg(cfg);
+  if (st) return st;
+  if (batch < 0 || block_len < 1 || block_len > 16) return KDA_ERR_INVALID_ARG;
+  if (batch == 0) return KDA_OK;
+  if ((conv_window == nullptr) != (conv_state == nullptr)) return KDA_ERR_INVALID_ARG;
+  if ((st = check_ptrs({accepted, tape_kua, state}, {conv_window, conv_state, state_slots})))
+    return st;
+  if ((st = check_pool(state_slots, pool_size, batch))) return st;
+  kda::RollbackArgs a{};
+  a.B = batch; a.T = block_len; a.H = cfg->num_heads; a.D = cfg->head_dim;
+  a.K = cfg->conv_size; a.bf16 = cfg->dtype == KDA_BF16;
+  a.accepted = accepted; a.tape_kua = tape_kua; a.window = conv_window; a.state = state;
+  a.conv_state = conv_state; a.slots = state_slots; a.pool_size = pool_size;
+  return cuda_status(kda::launch_rollback(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int kda_proj_gemm(int32_t M, int32_t N, int32_t K, const void* A, const void* B,
+                  const kda_proj_out* outs, int32_t n_outs, void* status,
+                  kda_stream_t stream) {
+  if (M < 0 || N < 0 || K < 8 || (K % 8) != 0 || (N % 8) != 0) return KDA_ERR_INVALID_ARG;
+  if (outs == nullptr || n_outs < 1 || n_outs > kda::proj_gemm_max_outs())
+    return KDA_ERR_INVALID_ARG;
+  int st;
+  if ((st = check_ptrs({A, B}, {})) != KDA_OK) return st;
+  if (status != nullptr && (reinterpret_cast<uintptr_t>(status) & 3u) != 0)
+    return KDA_ERR_MISALIGNED;
+  kda::ProjOut po[4];
+  for (int i = 0; i < n_outs; ++i) {
+    const kda_proj_out& o = outs[i];
+    if ((st = check_ptrs({o.out}, {})) != KDA_OK) return st;
+    if (o.col_begin < 0 || o.col_end > N || o.col_begin >= o.col_end ||
+        (o.col_begin % 8) != 0 || (o.col_end % 8) != 0 || (o.ld % 8) != 0 ||
+        o.ld < (int64_t)(o.col_end - o.col_begin))
+      return KDA_ERR_INVALID_ARG;
+    for (int j = 0; j < i; ++j)
+      if (o.col_begin < outs[j].col_end && outs[j].col_begin < o.col_end)
+        return KDA_ERR_INVALID_ARG;
+    po[i].out = o.out; po[i].ld = o.ld; po[i].col_begin = o.col_begin; po[i].col_end = o.col_end;
+  }
+  if (M == 0 || N == 0) return KDA_OK;
+  return cuda_status(kda::launch_proj_gemm(M, N, K, A, B, po, n_outs, static_cast<int*>(status),
+                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int kda_selftest_wait_timeout(void* workspace, kda_stream_t stream) {

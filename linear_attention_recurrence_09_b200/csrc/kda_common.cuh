@@ -48,6 +48,15 @@ __device__ __forceinline__ void st4(__nv_bfloat16* p, float4 v) {
 // logistic function; exp overflow to +inf gives exactly 0, never NaN
 __device__ __forceinline__ float sigmoid(float x) { return 1.0f / (1.0f + expf(-x)); }
 
+// log(1 + e^z) = max(z, 0) + log(1 + e^{-|z|}), without overflow
+__device__ __forceinline__ float softplus(float z) { return fmaxf(z, 0.f) + log1pf(expf(-fabsf(z))); }
+
+// log decay of one key channel with A = exp(A_log[h]) and z = f + dt_bias: the bounded
+// sigmoid lb * sigmoid(A z), or -A softplus(z) for the gate without a lower bound
+__device__ __forceinline__ float gate_log_decay(float A, float z, float lb, int softplus_gate) {
+  return softplus_gate ? -A * softplus(z) : lb * sigmoid(A * z);
+}
+
 // ---------------------------------------------------------------------------
 // Packed sequences -> fixed-size tiles.
 //

@@ -886,7 +886,10 @@ cudaError_t launch_intra_t(const PrefillArgs& a, cudaStream_t st) {
 
 }  // namespace
 
-bool sm100_intra_supported(const PrefillArgs& a) { return a.bf16 && a.D == D && a.C == C; }
+// the exponent split of the gram needs the bounded gate (lb >= -5)
+bool sm100_intra_supported(const PrefillArgs& a) {
+  return a.bf16 && a.D == D && a.C == C && !a.gate_softplus;
+}
 bool sm100_fused_supported(const PrefillArgs& a) { return sm100_intra_supported(a) && a.K == KC; }
 
 cudaError_t launch_intra_sm100(const PrefillArgs& a, cudaStream_t st) {

@@ -29,6 +29,7 @@ struct PrepArgs {
   float* loga;
   float* beta;
   float lb, l2_eps;
+  int gate_softplus;   // 1: log a = -A softplus(f + dt_bias); 0: lb sigmoid(A (f + dt_bias))
 };
 
 struct StepArgs {  // decode (T = 1) and verify (T = block_len)
@@ -43,7 +44,8 @@ struct StepArgs {  // decode (T = 1) and verify (T = block_len)
   const float* norm_w;
   const float* state_in;
   float* state_out;  // decode: == state_in; verify: nullptr
-  float* tape;       // verify only
+  float* tape;       // verify only: the state after every step
+  float* tape_kua;   // verify only: k, u and a of every step (the compact tape)
   const int32_t* slots;
   int pool_size;
   void* y;
@@ -59,13 +61,15 @@ struct StepArgs {  // decode (T = 1) and verify (T = block_len)
   void* window;             // verify: [B, K-1+T, H, 3d] = [history; x] for rollback
   int K;
   float lb, l2_eps;
+  int gate_softplus;        // as in PrepArgs
 };
 
 struct RollbackArgs {
   int B, T, H, D, K;
   bool bf16;
   const int32_t* accepted;
-  const float* tape;
+  const float* tape;       // full-state tape, or
+  const float* tape_kua;   // the compact tape, replayed from the live state
   const void* window;
   float* state;
   void* conv_state;
@@ -109,7 +113,19 @@ struct PrefillArgs {
   const float* dt_bias;
   const void* conv_state;   // [pool, K-1, H, 3d] history, or nullptr for zeros
   int K;
+  int gate_softplus;        // unbounded decay: the SIMT passes with exact diagonal gram blocks
 };
+
+// One output range of the projection GEMM: columns [col_begin, col_end) of C = A B^T go
+// to out[row * ld + (col - col_begin)] (bf16).
+struct ProjOut {
+  void* out;
+  long long ld;
+  int col_begin, col_end;
+};
+cudaError_t launch_proj_gemm(int M, int N, int K, const void* A, const void* B,
+                             const ProjOut* outs, int n_outs, int* status, cudaStream_t st);
+int proj_gemm_max_outs();
 
 cudaError_t launch_prep(const PrepArgs& a, cudaStream_t st);
 cudaError_t launch_step(const StepArgs& a, cudaStream_t st);

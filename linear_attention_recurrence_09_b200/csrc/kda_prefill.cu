@@ -25,7 +25,10 @@
 //   e^{G_r - G_i} = e^{G_r - G_ref} * e^{G_ref - G_i},  G_ref = G at the row before it,
 // where the first factor is <= 1 and the second is <= e^80.  Every other
 // exponential in the chunk form has a non-positive argument and may only
-// underflow, which is exact to within fp32.
+// underflow, which is exact to within fp32.  The softplus gate has no lower bound:
+// with it, the pairs inside the row's own sub-chunk take e^{G_r - G_i} directly (one
+// exponential per pair and channel, argument <= 0), and only the pairs across a
+// sub-chunk boundary use the split, whose two factors are then both <= 1.
 #include "kda_common.cuh"
 #include "kda_launch.h"
 
@@ -61,7 +64,7 @@ template <int D, int C>
 struct P1Smem {
   static constexpr int LD = D + 1;     // padded row stride: conflict-free column walks
   static constexpr int A_LD = C + 1;
-  static constexpr size_t bytes = sizeof(float) * (5 * C * LD + C * A_LD + C);
+  static constexpr size_t bytes = sizeof(float) * (6 * C * LD + C * A_LD + C);
 };
 
 template <typename WT, int D, int C>
@@ -74,7 +77,8 @@ __global__ void __launch_bounds__(256) intra_chunk_kernel(const PrefillArgs a) {
   float* Kb = Kr + C * LD;         // [C][LD] k_r e^{G_r - G_ref(r)}
   float* Qb = Kb + C * LD;         // [C][LD] q_scale q_r e^{G_r - G_ref(r)}
   float* Kc = Qb + C * LD;         // [C][LD] k_i e^{G_ref(R) - G_i} for the current R
-  float* A = Kc + C * LD;          // [C][A_LD]
+  float* Qr = Kc + C * LD;         // [C][LD] q_scale q (unscaled by the decay)
+  float* A = Qr + C * LD;          // [C][A_LD]
   float* bs = A + C * SM::A_LD;    // [C]
 
   const int h = blockIdx.y, H = a.H;
@@ -101,6 +105,7 @@ __global__ void __launch_bounds__(256) intra_chunk_kernel(const PrefillArgs a) {
       qq = __ldg(a.q + idx);
     }
     G[r * LD + c] = la; Kr[r * LD + c] = kk; Qb[r * LD + c] = qq;
+    Qr[r * LD + c] = a.q_scale * qq;
   }
   for (int r = tid; r < C; r += blockDim.x)
     bs[r] = (r < L) ? __ldg(a.beta + (size_t)(t0 + r) * H + h) : 0.f;
@@ -145,7 +150,20 @@ __global__ void __launch_bounds__(256) intra_chunk_kernel(const PrefillArgs a) {
     for (int p = tid; p < SUB * ncol; p += blockDim.x) {
       const int r = R * SUB + p / ncol, i = p - (p / ncol) * ncol;
       float am = 0.f, mm = 0.f;
-      if (i <= r) {
+      if (i <= r && a.gate_softplus && i >= R * SUB) {
+        // same sub-chunk, unbounded decay: e^{G_r - G_i} per channel (argument <= 0)
+        const float* kr = Kr + r * LD;
+        const float* qr = Qr + r * LD;
+        const float* ki = Kr + i * LD;
+        const float* gr = G + r * LD;
+        const float* gi = G + i * LD;
+#pragma unroll 4
+        for (int c = 0; c < D; ++c) {
+          const float e = __expf(gr[c] - gi[c]);
+          am = fmaf(kr[c] * ki[c], e, am);
+          mm = fmaf(qr[c] * ki[c], e, mm);
+        }
+      } else if (i <= r) {
         const float* kb = Kb + r * LD;
         const float* qb = Qb + r * LD;
         const float* kc = Kc + i * LD;

@@ -489,8 +489,9 @@ cudaError_t launch_wait_timeout_selftest(void* workspace, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// pairs with the tcgen05 intra-chunk pass (K' token-major), so the same condition
 bool sm100_interchunk_supported(const PrefillArgs& a) {
-  return a.bf16 && a.D == D && a.C == C;
+  return a.bf16 && a.D == D && a.C == C && !a.gate_softplus;
 }
 
 // the fused norm runs 4-CTA clusters; it is used unless it needs more waves of CTAs than

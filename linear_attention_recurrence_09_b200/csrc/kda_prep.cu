@@ -3,7 +3,9 @@
 // llama.cpp PR #27754 "model: add GLM-5-Next", KDA commit: q|k|v are convolved as
 // ONE depthwise kernel so the conv state is one contiguous block; SiLU follows
 // the conv; q/k use max(sqrt(sum), eps) with the literal eps 1e-6; the decay is
-// the bounded sigmoid with dt_bias per channel and per-head A broadcast.
+// the bounded sigmoid with dt_bias per channel and per-head A broadcast (or, when the
+// gate has no lower bound, the softplus branch of the "Metadata and tensor loading"
+// commit).
 //
 // HBM-bound streaming kernel.  A CTA covers a tile of up to 64 tokens of one
 // sequence for HPB consecutive heads; each thread owns 4 adjacent channels of one
@@ -156,9 +158,12 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const PrepArgs a) {
         if (e < tr.len * IPR) {
           const int c = (e % IPR) * 4;
           const float4 db = *reinterpret_cast<const float4*>(a.dt_bias + (size_t)h * D + c);
+          const int sp = a.gate_softplus;
           st4(a.loga + ((size_t)(tr.t0 + e / IPR) * H + h) * D + c,
-              make_float4(a.lb * sigmoid(Ah * (fv[u].x + db.x)), a.lb * sigmoid(Ah * (fv[u].y + db.y)),
-                          a.lb * sigmoid(Ah * (fv[u].z + db.z)), a.lb * sigmoid(Ah * (fv[u].w + db.w))));
+              make_float4(gate_log_decay(Ah, fv[u].x + db.x, a.lb, sp),
+                          gate_log_decay(Ah, fv[u].y + db.y, a.lb, sp),
+                          gate_log_decay(Ah, fv[u].z + db.z, a.lb, sp),
+                          gate_log_decay(Ah, fv[u].w + db.w, a.lb, sp)));
         }
       }
     }

@@ -7,7 +7,13 @@
 // the same pass (S^T k and S^T q), updated by a rank-1 write and stored once.
 // Verify runs that step block_len times from one load of the state and writes
 // the state after every step to a tape (speculative verify of a DFlash2 block,
-// dflash-mlx issue #63); rollback is a copy out of that tape.
+// dflash-mlx issue #63); rollback is a copy out of that tape.  Or, in the manner
+// of the tape-replay path that issue names for the GatedDeltaNet rollback, verify
+// writes only what each step adds to the state: S_j = Diag(a_j) S_{j-1} + k_j u_j^T,
+// so (k_j, u_j, a_j) is 3d floats per step instead of a d x d state, and rollback
+// replays the L accepted steps from the live state with the very operations of the
+// step (a multiply, then one fused multiply-add per element), which makes the
+// replayed state bit-identical to the full tape's.
 //
 // HBM-bound: the state is 64 KB per head at d = 128, so one CTA per
 // (head, sequence) keeps its whole state in registers (16 float4 per thread
@@ -127,10 +133,13 @@ step_kernel(const StepArgs a) {
 #pragma unroll
       for (int off = 16; off >= 1; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
       if (lane == 0) nrm_w[warp] = sq;
-      // decay a = exp(lb sigmoid(exp(A_log) (f + dt_bias))) and beta = sigmoid(logit)
+      // decay a = exp(lb sigmoid(exp(A_log) (f + dt_bias))) (or exp(-exp(A_log) softplus(..))
+      // for the gate without a lower bound) and beta = sigmoid(logit)
       const float Ah = __expf(__ldg(a.A_log + h));
-      for (int c = tid; c < D; c += THREADS)
-        as_[c] = __expf(a.lb * fsig(Ah * (ld1(fg + c) + __ldg(a.dt_bias + (size_t)h * D + c))));
+      for (int c = tid; c < D; c += THREADS) {
+        const float z = ld1(fg + c) + __ldg(a.dt_bias + (size_t)h * D + c);
+        as_[c] = __expf(a.gate_softplus ? -Ah * softplus(z) : a.lb * fsig(Ah * z));
+      }
       if (tid == 0) beta_s = fsig(ld1(static_cast<const T*>(a.beta_logit) + tok * H + h));
       __syncthreads();
       if (D >= 32) {
@@ -196,6 +205,12 @@ step_kernel(const StepArgs a) {
       const float u = bt * (vt - rk);
       o = a.q_scale * fmaf(u, kq_s, rq);
       us[tid] = u;
+      if (a.tape_kua != nullptr) {   // compact tape: this step's k, u and a
+        float* tk = a.tape_kua + (tok * H + h) * 3 * D;
+        tk[tid] = ks[tid];
+        tk[D + tid] = u;
+        tk[2 * D + tid] = as_[tid];
+      }
     }
     if (warp < (D + 31) / 32) {
       float p = o * o;
@@ -290,10 +305,79 @@ __global__ void __launch_bounds__(256) rollback_kernel(const RollbackArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// rollback by replay: state <- the accepted steps of the compact tape applied to the
+// live state, S <- Diag(a_j) S, then S <- S + k_j u_j^T, element by element exactly as
+// step_kernel does it (same layout, same two operations), so the result equals the
+// full tape's entry bit for bit; conv state as in rollback_kernel
+// ---------------------------------------------------------------------------
+template <typename E, int D>
+__global__ void __launch_bounds__(StepShape<D>::THREADS) rollback_replay_kernel(const RollbackArgs a) {
+  using SH = StepShape<D>;
+  constexpr int CG = SH::CG, RG = SH::RG, ROWS = SH::ROWS, THREADS = SH::THREADS;
+  constexpr int TMAX = 16;
+  __shared__ __align__(16) float kua[TMAX][3][D];
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int L = clampi(__ldg(a.accepted + b), 0, a.T);
+  if (L == 0) return;
+  const int row = pool_row(a.slots, b, a.pool_size);
+  if (row < 0) return;
+  const int H = a.H, tid = threadIdx.x, cg = tid % CG, rg = tid / CG;
+  float* Sg = a.state + ((size_t)row * H + h) * D * D;
+  float4 S[ROWS];
+#pragma unroll
+  for (int i = 0; i < ROWS; ++i) S[i] = ld4(Sg + (size_t)(rg + i * RG) * D + 4 * cg);
+  for (int e = tid; e < L * 3 * D; e += THREADS) {
+    const int j = e / (3 * D), w = e - j * 3 * D;
+    (&kua[j][0][0])[w] = __ldg(a.tape_kua + (((size_t)b * a.T + j) * H + h) * 3 * D + w);
+  }
+  __syncthreads();
+  for (int j = 0; j < L; ++j) {
+    const float4 u4 = *reinterpret_cast<const float4*>(&kua[j][1][4 * cg]);
+#pragma unroll
+    for (int i = 0; i < ROWS; ++i) {
+      const int r = rg + i * RG;
+      S[i] = f4_scale(S[i], kua[j][2][r]);
+      S[i] = f4_fma(kua[j][0][r], u4, S[i]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < ROWS; ++i) st4(Sg + (size_t)(rg + i * RG) * D + 4 * cg, S[i]);
+  if (a.conv_state != nullptr && a.window != nullptr) {
+    const int Km1 = a.K - 1, C3 = 3 * D;
+    const E* win = static_cast<const E*>(a.window);
+    E* cs = static_cast<E*>(a.conv_state);
+    for (int e = tid; e < Km1 * C3; e += THREADS) {
+      const int j = e / C3, c = e - (e / C3) * C3;
+      cs[(((size_t)row * Km1 + j) * H + h) * C3 + c] =
+          win[(((size_t)b * (Km1 + a.T) + L + j) * H + h) * C3 + c];
+    }
+  }
+}
+
+template <typename E>
+static cudaError_t launch_replay_e(const RollbackArgs& a, cudaStream_t st) {
+  dim3 grid(a.H, a.B);
+  switch (a.D) {
+    case 16: rollback_replay_kernel<E, 16><<<grid, StepShape<16>::THREADS, 0, st>>>(a); break;
+    case 32: rollback_replay_kernel<E, 32><<<grid, StepShape<32>::THREADS, 0, st>>>(a); break;
+    case 64: rollback_replay_kernel<E, 64><<<grid, StepShape<64>::THREADS, 0, st>>>(a); break;
+    case 128: rollback_replay_kernel<E, 128><<<grid, StepShape<128>::THREADS, 0, st>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaSuccess;
+}
+
 cudaError_t launch_rollback(const RollbackArgs& a, cudaStream_t st) {
   dim3 grid(a.H, a.B);
-  if (a.bf16) rollback_kernel<uint16_t><<<grid, 256, 0, st>>>(a);
-  else rollback_kernel<uint32_t><<<grid, 256, 0, st>>>(a);
+  if (a.tape_kua != nullptr) {
+    const cudaError_t e = a.bf16 ? launch_replay_e<uint16_t>(a, st) : launch_replay_e<uint32_t>(a, st);
+    if (e != cudaSuccess) return e;
+  } else if (a.bf16) {
+    rollback_kernel<uint16_t><<<grid, 256, 0, st>>>(a);
+  } else {
+    rollback_kernel<uint32_t><<<grid, 256, 0, st>>>(a);
+  }
   ++launch_counter();
   return cudaGetLastError();
 }

@@ -11,6 +11,7 @@ from __future__ import annotations
 import ctypes
 import os
 from dataclasses import dataclass
+from typing import Optional
 
 import torch
 
@@ -30,13 +31,17 @@ KDA_F32 = 0
 KDA_BF16 = 1
 KDA_CONV_COMMIT = 0
 KDA_CONV_TAPE = 1
+KDA_GATE_BOUNDED_SIGMOID = 0
+KDA_GATE_SOFTPLUS = 1
+ABI_VERSION = 2
 
 ENTRY_POINTS = ('kda_status_string', 'kda_abi_version', 'kda_prep',
                 'kda_prefill_workspace_size', 'kda_prefill', 'kda_decode', 'kda_verify',
                 'kda_rollback', 'kda_workspace_status', 'kda_selftest_wait_timeout',
                 'kda_prefill_noalloc', 'kda_layer_prefill_workspace_size', 'kda_layer_prefill',
                 'kda_set_phase_events', 'kda_launch_count', 'kda_last_cuda_error',
-                'kda_layer_decode', 'kda_layer_verify')
+                'kda_layer_decode', 'kda_layer_verify', 'kda_verify_compact',
+                'kda_layer_verify_compact', 'kda_rollback_replay', 'kda_proj_gemm')
 
 
 class KdaError(RuntimeError):
@@ -53,18 +58,19 @@ class CConfig(ctypes.Structure):
                 ('conv_size', ctypes.c_int32), ('dtype', ctypes.c_int32),
                 ('chunk_size', ctypes.c_int32), ('gate_lower_bound', ctypes.c_float),
                 ('l2_eps', ctypes.c_float), ('norm_eps', ctypes.c_float),
-                ('q_scale', ctypes.c_float)]
+                ('q_scale', ctypes.c_float), ('gate_kind', ctypes.c_int32)]
 
 
 @dataclass
 class Config:
-    """Layer configuration; mirrors ``kda_config``."""
+    """Layer configuration; mirrors ``kda_config``.  ``gate_lower_bound=None`` selects
+    the softplus decay gate (KDA_GATE_SOFTPLUS), as an absent lower bound does."""
     num_heads: int
     head_dim: int
     conv_size: int = 4
     dtype: torch.dtype = torch.bfloat16
     chunk_size: int = 64
-    gate_lower_bound: float = -5.0
+    gate_lower_bound: Optional[float] = -5.0
     l2_eps: float = 1e-6
     norm_eps: float = 1e-5
     q_scale: float = 1.0
@@ -72,10 +78,17 @@ class Config:
     def c(self) -> CConfig:
         if self.dtype not in (torch.float32, torch.bfloat16):
             raise ValueError('activation dtype must be float32 or bfloat16')
+        softplus = self.gate_lower_bound is None
         return CConfig(self.num_heads, self.head_dim, self.conv_size,
                        KDA_BF16 if self.dtype == torch.bfloat16 else KDA_F32,
-                       self.chunk_size, self.gate_lower_bound, self.l2_eps, self.norm_eps,
-                       self.q_scale)
+                       self.chunk_size, 0.0 if softplus else self.gate_lower_bound,
+                       self.l2_eps, self.norm_eps, self.q_scale,
+                       KDA_GATE_SOFTPLUS if softplus else KDA_GATE_BOUNDED_SIGMOID)
+
+
+class CProjOut(ctypes.Structure):
+    _fields_ = [('out', ctypes.c_void_p), ('ld', ctypes.c_int64), ('col_begin', ctypes.c_int32),
+                ('col_end', ctypes.c_int32)]
 
 
 _lib = None
@@ -128,6 +141,14 @@ def lib() -> ctypes.CDLL:
         L.kda_layer_verify.restype = ctypes.c_int
         L.kda_layer_verify.argtypes = [ctypes.POINTER(CConfig), _I, _I, _P, _P, _P, _P, _P, _P,
                                        _P, _P, _P, _P, _P, _I, _P, _P, _P, _P]
+        L.kda_verify_compact.restype = ctypes.c_int
+        L.kda_verify_compact.argtypes = L.kda_verify.argtypes
+        L.kda_layer_verify_compact.restype = ctypes.c_int
+        L.kda_layer_verify_compact.argtypes = L.kda_layer_verify.argtypes
+        L.kda_rollback_replay.restype = ctypes.c_int
+        L.kda_rollback_replay.argtypes = L.kda_rollback.argtypes
+        L.kda_proj_gemm.restype = ctypes.c_int
+        L.kda_proj_gemm.argtypes = [_I, _I, _I, _P, _P, ctypes.POINTER(CProjOut), _I, _P, _P]
         L.kda_last_cuda_error.restype = ctypes.c_char_p
         L.kda_last_cuda_error.argtypes = []
         L.kda_launch_count.restype = ctypes.c_longlong
@@ -335,6 +356,49 @@ def kda_verify(cfg: Config, q, k, v, log_a, beta, g, norm_w, state, state_slots=
     return y, tape
 
 
+def kda_verify_compact(cfg: Config, q, k, v, log_a, beta, g, norm_w, state, state_slots=None,
+                       pool_size=None, tape_kua=None, y=None, stream=None):
+    """Verify [B, Tb] draft tokens from ``state`` (unchanged), recording each step's
+    (k, u, a) instead of the state.  Returns (y, tape_kua [B, Tb, H, 3, d])."""
+    H, d = cfg.num_heads, cfg.head_dim
+    B, Tb = q.shape[0], q.shape[1]
+    if y is None:
+        y = _empty((B, Tb, H, d), cfg.dtype, q.device)
+    if tape_kua is None:
+        tape_kua = _empty((B, Tb, H, 3, d), torch.float32, q.device)
+    if pool_size is None:
+        pool_size = state.shape[0]
+    c = cfg.c()
+    st = lib().kda_verify_compact(
+        ctypes.byref(c), B, Tb, _ptr(q, torch.float32, 'q', (B, Tb, H, d)),
+        _ptr(k, torch.float32, 'k', (B, Tb, H, d)), _ptr(v, torch.float32, 'v', (B, Tb, H, d)),
+        _ptr(log_a, torch.float32, 'log_a', (B, Tb, H, d)),
+        _ptr(beta, torch.float32, 'beta', (B, Tb, H)), _ptr(g, cfg.dtype, 'g', (B, Tb, H, d)),
+        _ptr(norm_w, torch.float32, 'norm_w', (d,)), _ptr(state, torch.float32, 'state'),
+        _ptr(state_slots, torch.int32, 'state_slots'), int(pool_size),
+        _ptr(tape_kua, torch.float32, 'tape_kua', (B, Tb, H, 3, d)),
+        _ptr(y, cfg.dtype, 'y', (B, Tb, H, d)), _stream(stream))
+    _check(st, 'kda_verify_compact')
+    return y, tape_kua
+
+
+def kda_rollback_replay(cfg: Config, accepted, tape_kua, state, conv_window=None,
+                        conv_state=None, state_slots=None, pool_size=None, stream=None):
+    """Commit accepted prefixes by replaying the compact tape on the live state."""
+    H, d = cfg.num_heads, cfg.head_dim
+    B, Tb = tape_kua.shape[0], tape_kua.shape[1]
+    if pool_size is None:
+        pool_size = state.shape[0]
+    c = cfg.c()
+    st = lib().kda_rollback_replay(
+        ctypes.byref(c), B, Tb, _ptr(accepted, torch.int32, 'accepted', (B,)),
+        _ptr(tape_kua, torch.float32, 'tape_kua', (B, Tb, H, 3, d)),
+        _ptr(conv_window, cfg.dtype, 'conv_window'), _ptr(state, torch.float32, 'state'),
+        _ptr(conv_state, cfg.dtype, 'conv_state'), _ptr(state_slots, torch.int32, 'state_slots'),
+        int(pool_size), _stream(stream))
+    _check(st, 'kda_rollback_replay')
+
+
 def kda_rollback(cfg: Config, accepted, tape, state, conv_window=None, conv_state=None,
                  state_slots=None, pool_size=None, stream=None):
     """Commit accepted prefixes: state <- tape[L-1], conv state <- window[L:L+K-1]."""
@@ -412,6 +476,57 @@ def kda_layer_verify(cfg: Config, x, f, beta_logit, g, conv_w, A_log, dt_bias, n
         _ptr(window, cfg.dtype, 'window', (B, K - 1 + Tb, H, 3 * d)),
         _ptr(y, cfg.dtype, 'y', (B, Tb, H, d)), _stream(stream)), 'kda_layer_verify')
     return y, tape, window
+
+
+def kda_layer_verify_compact(cfg: Config, x, f, beta_logit, g, conv_w, A_log, dt_bias, norm_w,
+                             state, conv_state=None, state_slots=None, pool_size=None,
+                             tape_kua=None, window=None, y=None, stream=None):
+    """kda_layer_verify recording each step's (k, u, a).  Returns (y, tape_kua, window)."""
+    H, d, K = cfg.num_heads, cfg.head_dim, cfg.conv_size
+    B, Tb = x.shape[0], x.shape[1]
+    if y is None:
+        y = _empty((B, Tb, H, d), cfg.dtype, x.device)
+    if tape_kua is None:
+        tape_kua = _empty((B, Tb, H, 3, d), torch.float32, x.device)
+    if window is None:
+        window = _empty((B, K - 1 + Tb, H, 3 * d), cfg.dtype, x.device)
+    if pool_size is None:
+        pool_size = state.shape[0]
+    c = cfg.c()
+    _check(lib().kda_layer_verify_compact(
+        ctypes.byref(c), B, Tb, _ptr(x, cfg.dtype, 'x', (B, Tb, H, 3 * d)),
+        _ptr(f, cfg.dtype, 'f', (B, Tb, H, d)),
+        _ptr(beta_logit, cfg.dtype, 'beta_logit', (B, Tb, H)),
+        _ptr(g, cfg.dtype, 'g', (B, Tb, H, d)), _ptr(conv_w, torch.float32, 'conv_w', (H, 3 * d, K)),
+        _ptr(A_log, torch.float32, 'A_log', (H,)), _ptr(dt_bias, torch.float32, 'dt_bias', (H, d)),
+        _ptr(norm_w, torch.float32, 'norm_w', (d,)), _ptr(conv_state, cfg.dtype, 'conv_state'),
+        _ptr(state, torch.float32, 'state'), _ptr(state_slots, torch.int32, 'state_slots'),
+        int(pool_size), _ptr(tape_kua, torch.float32, 'tape_kua', (B, Tb, H, 3, d)),
+        _ptr(window, cfg.dtype, 'window', (B, K - 1 + Tb, H, 3 * d)),
+        _ptr(y, cfg.dtype, 'y', (B, Tb, H, d)), _stream(stream)), 'kda_layer_verify_compact')
+    return y, tape_kua, window
+
+
+def kda_proj_gemm(A, B, outs, status=None, stream=None):
+    """C = A B^T (bf16 in, fp32 accumulate, bf16 out) with column ranges of C routed to
+    separate tensors.  A [M, K] and B [N, K] are bf16 CUDA tensors; ``outs`` is a list of
+    (tensor, col_begin, col_end): columns [col_begin, col_end) of C go to ``tensor``, a
+    contiguous bf16 CUDA tensor read as M rows of numel / M elements, each row starting
+    with the range."""
+    M, K = A.shape
+    N = B.shape[0]
+    if B.shape[1] != K:
+        raise ValueError('A and B must share K')
+    arr = (CProjOut * max(1, len(outs)))()
+    for i, (t, c0, c1) in enumerate(outs):
+        if t.numel() % max(M, 1):
+            raise ValueError('output tensor size must be a multiple of M rows')
+        ld = t.numel() // max(M, 1)
+        arr[i] = CProjOut(_ptr(t, torch.bfloat16, f'outs[{i}]'), ld, int(c0), int(c1))
+    _check(lib().kda_proj_gemm(int(M), int(N), int(K), _ptr(A, torch.bfloat16, 'A'),
+                               _ptr(B, torch.bfloat16, 'B'), arr, len(outs),
+                               _ptr(status, torch.int32, 'status'), _stream(stream)),
+           'kda_proj_gemm')
 
 
 def kda_launch_count() -> int:
@@ -496,3 +611,27 @@ def layer_prefill(cfg: Config, params, acts, state_in=None, state_out=None, conv
                              acts['g'], params['conv_w'], params['A_log'], params['dt_bias'],
                              params['norm_w'], conv_state=conv_state, state_in=state_in,
                              state_out=state_out, y=y, workspace=workspace, stream=stream)
+
+
+def layer_projections(cfg: Config, hidden, W_in, W_gb, gate_rank, out=None, stream=None):
+    """The layer's inputs from the hidden states: kda_proj_gemm with the fused input
+    weight (x = q|k|v pre-conv, f, beta logit, g_a, each into its own dense tensor),
+    then kda_proj_gemm with the gate's second factor (g = g_a W_gb^T).  bf16 only; the
+    head count and gate rank must be multiples of 8 (the output ranges are 16-byte
+    aligned).  Returns dict x, f, beta_logit, g_a, g."""
+    H, d = cfg.num_heads, cfg.head_dim
+    T = hidden.shape[0]
+    dev = hidden.device
+    nx, nf = 3 * H * d, H * d
+    o = dict(out or {})
+    shapes = {'x': (T, H, 3 * d), 'f': (T, H, d), 'beta_logit': (T, H),
+              'g_a': (T, gate_rank), 'g': (T, H, d)}
+    for name, shp in shapes.items():
+        if o.get(name) is None:
+            o[name] = _empty(shp, torch.bfloat16, dev)
+    kda_proj_gemm(hidden, W_in, [(o['x'], 0, nx), (o['f'], nx, nx + nf),
+                                 (o['beta_logit'], nx + nf, nx + nf + H),
+                                 (o['g_a'], nx + nf + H, nx + nf + H + gate_rank)],
+                  stream=stream)
+    kda_proj_gemm(o['g_a'], W_gb, [(o['g'], 0, H * d)], stream=stream)
+    return o

@@ -77,6 +77,22 @@ def layer_activations(seed, seqlens, H, d, dtype=torch.bfloat16, tag='act'):
     return out
 
 
+def proj_weights(seed, hidden, H, d, gate_rank, dtype=torch.bfloat16):
+    """Random-init projection weights of one layer: the fused input weight W_in
+    [3Hd + Hd + H + gate_rank, hidden] ~ N(0, 1/hidden) (so that x, f, the beta logit and
+    g_a come out ~ N(0, 1) for N(0, 1) hidden states, the activations' recipe) and the
+    gate's second factor W_gb [H d, gate_rank] ~ N(0, 1/gate_rank)."""
+    n = 4 * H * d + H + gate_rank
+    W_in = _normal((n, hidden), 1.0 / math.sqrt(hidden), seed, 'W_in').to(dtype)
+    W_gb = _normal((H * d, gate_rank), 1.0 / math.sqrt(gate_rank), seed, 'W_gb').to(dtype)
+    return dict(W_in=W_in, W_gb=W_gb)
+
+
+def hidden_states(seed, T, hidden, dtype=torch.bfloat16, tag='hidden'):
+    """Hidden states [T, hidden] ~ N(0, 1), drawn per 4096-token block."""
+    return _normal_tokens('hidden', (seed, tag), 0, T, (hidden,), dtype)
+
+
 def initial_state(seed, n, H, d, variance):
     """fp32 recurrent states [n,H,d,d] ~ N(0, variance); zeros if variance is 0."""
     if variance == 0:
@@ -114,4 +130,6 @@ WORKLOADS = {
                        head_dim=128, chunk=64, conv=4, dtype='bf16', state_variance=0.0),
     'varlen_long': dict(seed=4, n_seqs=8, lo=1024, hi=32768, long_seqlen=131072, heads=32,
                         head_dim=128, chunk=64, conv=4, dtype='bf16', state_variance=0.01),
+    'layer_8k_projections': dict(seed=6, batch=1, heads=32, seqlen=8192, head_dim=128,
+                                 hidden=4096, gate_rank=128, chunk=64, conv=4, dtype='bf16'),
 }

@@ -278,6 +278,35 @@ def layer(x, f, beta_logit, g, conv_w, A_log, dt_bias, norm_w, cu_seqlens,
 
 
 # ---------------------------------------------------------------------------
+# the steps either side: the fused input projection and the low-rank output gate
+# ---------------------------------------------------------------------------
+def projections(hidden, W_in, W_gb, H, d, gate_rank):
+    """The layer's inputs from the hidden states, float64.
+
+    glm53-flash-mlx README, quantization recipe: the runtime fuses the six KDA input
+    projections into one matmul (they share the hidden width).  PR #27754, KDA commit:
+    f, g and beta are read from the pre-conv hidden states, and the output gate is low
+    rank, g_b(g_a(x)).  Reading taken (the pages name the pieces, not their layout): the
+    six projections are q, k, v, f, beta and g_a, stacked as the rows of one weight
+    W_in [3Hd + Hd + H + r, hidden] in the order q|k|v per head (the pre-conv x of the
+    layer, [T, H, 3d]), f ([T, H, d]), the beta logit ([T, H]) and g_a ([T, r]); then
+    g = g_a W_gb^T with W_gb [H d, r].  No bias.
+
+    hidden: [T, hidden]; returns dict x, f, beta_logit, g_a, g.
+    """
+    hidden = np.asarray(hidden, np.float64)
+    T = hidden.shape[0]
+    Y = hidden @ np.asarray(W_in, np.float64).T
+    nx, nf = 3 * H * d, H * d
+    x = Y[:, :nx].reshape(T, H, 3 * d)
+    f = Y[:, nx:nx + nf].reshape(T, H, d)
+    beta_logit = Y[:, nx + nf:nx + nf + H]
+    g_a = Y[:, nx + nf + H:nx + nf + H + gate_rank]
+    g = (g_a @ np.asarray(W_gb, np.float64).T).reshape(T, H, d)
+    return dict(x=x, f=f, beta_logit=beta_logit, g_a=g_a, g=g)
+
+
+# ---------------------------------------------------------------------------
 # speculative verify + rollback
 # ---------------------------------------------------------------------------
 def verify(q, k, v, loga, beta, g, norm_w, S0, q_scale=1.0, norm_eps=NORM_EPS):

@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert kda.kda_abi_version() == 1
+    assert kda.kda_abi_version() == kda.ABI_VERSION == 2
     for code in range(8):
         assert kda.kda_status_string(code).startswith('KDA_')
     assert 'unknown' in kda.kda_status_string(99)
@@ -70,6 +70,15 @@ def test_prep_rejects_bad_arguments(L):
     assert _prep(L, _cfg(chunk_size=128)) == kda.KDA_ERR_UNSUPPORTED
     assert _prep(L, _cfg(gate_lower_bound=-6.0)) == kda.KDA_ERR_UNSUPPORTED
     assert _prep(L, _cfg(gate_lower_bound=0.0)) == kda.KDA_ERR_UNSUPPORTED
+    # the softplus gate ignores the lower bound: validation goes on to the pointers
+    sp = _cfg(gate_lower_bound=None)
+    assert sp.gate_kind == kda.KDA_GATE_SOFTPLUS
+    assert _prep(L, sp, cu=None) == kda.KDA_ERR_INVALID_ARG
+    sp.gate_lower_bound = -6.0
+    assert _prep(L, sp, cu=MIS) == kda.KDA_ERR_MISALIGNED
+    bad = _cfg()
+    bad.gate_kind = 2
+    assert _prep(L, bad) == kda.KDA_ERR_INVALID_ARG
     assert _prep(L, _cfg(conv_size=9)) == kda.KDA_ERR_INVALID_ARG
     assert _prep(L, _cfg(num_heads=0)) == kda.KDA_ERR_INVALID_ARG
     assert _prep(L, _cfg(l2_eps=0.0)) == kda.KDA_ERR_INVALID_ARG
@@ -148,6 +157,22 @@ def test_step_entry_points_reject_bad_arguments(L):
     assert L.kda_rollback(c, 2, 0, A, A, None, A, None, None, 2, None) == kda.KDA_ERR_INVALID_ARG
     assert L.kda_rollback(c, 2, 8, A, A, A, A, None, None, 2, None) == kda.KDA_ERR_INVALID_ARG
     assert L.kda_workspace_status(None, None) == kda.KDA_ERR_INVALID_ARG
+    # compact tape: the tape_kua pointer is required, the block length bounded
+    assert L.kda_verify_compact(c, 2, 8, A, A, A, A, A, A, A, A, None, 2, None, A, None) == \
+        kda.KDA_ERR_INVALID_ARG
+    assert L.kda_verify_compact(c, 2, 8, A, A, A, A, A, A, A, A, None, 2, MIS, A, None) == \
+        kda.KDA_ERR_MISALIGNED
+    assert L.kda_verify_compact(c, 2, 0, A, A, A, A, A, A, A, A, None, 2, A, A, None) == \
+        kda.KDA_ERR_INVALID_ARG
+    assert L.kda_rollback_replay(c, 2, 17, A, A, None, A, None, None, 2, None) == \
+        kda.KDA_ERR_INVALID_ARG
+    assert L.kda_rollback_replay(c, 2, 8, A, None, None, A, None, None, 2, None) == \
+        kda.KDA_ERR_INVALID_ARG
+    assert L.kda_rollback_replay(c, 2, 8, A, A, A, A, None, None, 2, None) == \
+        kda.KDA_ERR_INVALID_ARG
+    assert L.kda_rollback_replay(c, 0, 8, None, None, None, None, None, None, 0, None) == kda.KDA_OK
+    lv = [c, 2, 8, A, A, A, A, A, A, A, A, None, A, None, 2, None, A, A, None]
+    assert L.kda_layer_verify_compact(*lv) == kda.KDA_ERR_INVALID_ARG      # tape_kua NULL
 
 
 def test_workspace_size_grows_with_tokens(L):

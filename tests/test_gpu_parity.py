@@ -3,6 +3,8 @@
 Bar: max|GPU - oracle| / max|oracle| <= 1e-4 for fp32 inputs and <= 1e-2 for
 bf16 inputs with an fp32 state; rollback and the verify tape are bit-exact.
 """
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -559,3 +561,140 @@ def test_l2_eps_zero_and_tiny_rows_decode_verify(dtype, d):
     for h, rows in _edge_regions():
         r = slice(max(rows.start, T0) - T0, rows.stop - T0)
         assert rel_err(yv[r, h], ref['y'][T0:][r, h]) <= tol, h
+
+
+# ---------------------------------------------------------------------------
+# the softplus decay gate (no lower bound): PR #27754, "Metadata and tensor loading"
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize('fused', [True, False])
+@pytest.mark.parametrize('dtype,d,chunk', [(torch.bfloat16, 128, 64), (torch.float32, 64, 32),
+                                           (torch.bfloat16, 32, 16), (torch.float32, 16, 16)])
+def test_softplus_gate_prefill(dtype, d, chunk, fused):
+    """kda_layer_prefill and kda_prep + kda_prefill with log a = -exp(A_log) softplus(f +
+    dt_bias): decays far below the bounded gate's -5 per token, so a chunk's cumulative
+    decay spans hundreds of nats (the SIMT passes, exact inside each 16-token block)."""
+    seqlens = [chunk - 3, 2 * chunk + 5, 1]
+    cfg, P, A, S0, hist = make_case(41, seqlens, 3, d, 4, dtype, state_var=0.01,
+                                    conv_hist=True, chunk=chunk)
+    cfg.gate_lower_bound = None
+    P['A_log'][0] = math.log(16.0)            # the recipe's largest rate on one head
+    y, s_out, cs, p = gpu_layer(cfg, P, A, S0, hist, fused=fused)
+    ref = oracle_layer(cfg, P, A, S0, hist)
+    assert ref['loga'].min() < -20.0          # the workload reaches well past -5 per token
+    tol = TOL[dtype]
+    assert rel_err(np64(y), ref['y']) <= tol
+    assert rel_err(np64(s_out), ref['state']) <= tol
+    assert np.array_equal(np64(cs), ref['conv_hist'])
+    if p is not None:
+        assert rel_err(np64(p['log_a']), ref['loga']) <= 1e-5
+
+
+@pytest.mark.parametrize('dtype,d', [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_softplus_gate_decode_verify(dtype, d):
+    """The softplus gate through the step kernel: kda_layer_decode (gate computed in the
+    kernel), kda_prep + kda_decode, and kda_layer_verify + rollback."""
+    B, H, T0, steps = 2, 4, 30, 6
+    cfg, P, A, S0, hist = make_case(42, [T0] * B, H, d, 4, dtype, state_var=0.01,
+                                    conv_hist=True, chunk=16)
+    cfg.gate_lower_bound = None
+    _, s0, c0, _ = gpu_layer(cfg, P, A, S0, hist)
+    sa = _step_acts(42, B, H, d, dtype, steps)
+    tol = TOL[dtype]
+    for fused in (True, False):
+        st, cs = s0.clone(), c0.clone()
+        ys = _decode_run(cfg, P, sa, st, cs, fused=fused).cpu()
+        for b in range(B):
+            ref = oracle_layer(cfg, P, _cat_seq([A] + sa, b), S0[b:b + 1], hist[b:b + 1])
+            assert rel_err(np64(ys[:, b]), ref['y'][T0:]) <= tol, (fused, b)
+            assert rel_err(np64(st[b]), ref['state'][0]) <= tol, (fused, b)
+    Tb = 8
+    D = synth.layer_activations(42, [Tb] * B, H, d, dtype, tag='drafts')
+    v4 = lambda t, *tail: t.cuda().reshape(B, Tb, *tail).contiguous()
+    Pd = {k: v.cuda() for k, v in P.items()}
+    st, cs = s0.clone(), c0.clone()
+    y_v, tape, win = kda.kda_layer_verify(cfg, v4(D['x'], H, 3 * d), v4(D['f'], H, d),
+                                          v4(D['beta_logit'], H), v4(D['g'], H, d),
+                                          Pd['conv_w'], Pd['A_log'], Pd['dt_bias'],
+                                          Pd['norm_w'], st, conv_state=cs)
+    acc = torch.tensor([3, 8], dtype=torch.int32, device='cuda')
+    kda.kda_rollback(cfg, acc, tape, st, conv_window=win, conv_state=cs)
+    torch.cuda.synchronize()
+    for b, L in ((0, 3), (1, 8)):
+        seq = {k: torch.cat([A[k][b * T0:(b + 1) * T0], D[k][b * Tb:b * Tb + L]])
+               for k in ('x', 'f', 'beta_logit', 'g')}
+        seq['cu_seqlens'] = torch.tensor([0, T0 + L], dtype=torch.int32)
+        ref = oracle_layer(cfg, P, seq, S0[b:b + 1], hist[b:b + 1])
+        assert rel_err(np64(y_v[b, :L]), ref['y'][T0:]) <= tol, b
+        assert rel_err(np64(st[b]), ref['state'][0]) <= tol, b
+        assert np.array_equal(np64(cs[b]), ref['conv_hist'][0])
+
+
+# ---------------------------------------------------------------------------
+# compact verify tape (k, u, a per step) and rollback by replay
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize('dtype,d', [(torch.bfloat16, 128), (torch.float32, 64),
+                                     (torch.bfloat16, 32)])
+def test_replay_rollback_equals_full_tape_bit_exact(dtype, d):
+    """dflash-mlx issue #63 (tape-replay rollback): kda_verify_compact + kda_rollback_replay
+    against kda_verify + kda_rollback on the same block, for every accepted length 0..8:
+    the same y, and the replayed state equal to the full tape's entry bit for bit."""
+    B, H, Tb, K = 9, 3, 8, 4
+    cfg, P, A, S0, hist = make_case(43, [Tb] * B, H, d, K, dtype, state_var=0.01,
+                                    conv_hist=True, chunk=16)
+    dev = 'cuda'
+    Pd = {k: v.to(dev) for k, v in P.items()}
+    p = kda.kda_prep(cfg, A['cu_seqlens'].to(dev), A['x'].to(dev), A['f'].to(dev),
+                     A['beta_logit'].to(dev), Pd['conv_w'], Pd['A_log'], Pd['dt_bias'],
+                     conv_state=hist.to(dev), conv_mode=kda.KDA_CONV_TAPE, max_seqlen=Tb)
+    shp = lambda t, *tail: t.view(B, Tb, *tail)
+    args = (shp(p['q'], H, d), shp(p['k'], H, d), shp(p['v'], H, d), shp(p['log_a'], H, d),
+            shp(p['beta'], H), shp(A['g'].to(dev), H, d), Pd['norm_w'])
+    st_full, st_rep = S0.to(dev), S0.to(dev)
+    y_full, tape = kda.kda_verify(cfg, *args, st_full)
+    y_rep, kua = kda.kda_verify_compact(cfg, *args, st_rep)
+    acc = torch.arange(B, dtype=torch.int32, device=dev) % (Tb + 1)     # 0..8
+    cs_full, cs_rep = hist.to(dev), hist.to(dev)
+    kda.kda_rollback(cfg, acc, tape, st_full, conv_window=p['window'], conv_state=cs_full)
+    kda.kda_rollback_replay(cfg, acc, kua, st_rep, conv_window=p['window'], conv_state=cs_rep)
+    torch.cuda.synchronize()
+    assert torch.equal(y_full, y_rep)
+    assert torch.equal(st_rep, st_full)
+    assert torch.equal(cs_rep, cs_full)
+    for b in range(B):
+        L = int(acc[b])
+        assert torch.equal(st_rep[b], tape[b, L - 1] if L else S0[b].to(dev)), b
+    # the compact tape holds the step's k and a as prep produced them
+    assert torch.equal(kua[:, :, :, 0], shp(p['k'], H, d))
+    assert torch.allclose(kua[:, :, :, 2], torch.exp(shp(p['log_a'], H, d)), rtol=1e-6, atol=0)
+
+
+@pytest.mark.parametrize('dtype', [torch.bfloat16, torch.float32])
+def test_layer_verify_compact_and_replay(dtype):
+    """kda_layer_verify_compact (prep in the step kernel) + kda_rollback_replay equals
+    kda_layer_verify + kda_rollback bit for bit, and the oracle's accepted prefix."""
+    B, H, d, Tb = 3, 4, 64, 8
+    cfg, P, A, S0, hist = make_case(44, [1] * B, H, d, 4, dtype, state_var=0.01,
+                                    conv_hist=True, chunk=16)
+    D = synth.layer_activations(44, [Tb] * B, H, d, dtype, tag='drafts')
+    dev = 'cuda'
+    Pd = {k: v.to(dev) for k, v in P.items()}
+    v4 = lambda t, *tail: t.to(dev).reshape(B, Tb, *tail).contiguous()
+    args = (v4(D['x'], H, 3 * d), v4(D['f'], H, d), v4(D['beta_logit'], H), v4(D['g'], H, d),
+            Pd['conv_w'], Pd['A_log'], Pd['dt_bias'], Pd['norm_w'])
+    s1, c1 = S0.to(dev), hist.to(dev)
+    s2, c2 = S0.to(dev), hist.to(dev)
+    y1, tape, w1 = kda.kda_layer_verify(cfg, *args, s1, conv_state=c1)
+    y2, kua, w2 = kda.kda_layer_verify_compact(cfg, *args, s2, conv_state=c2)
+    acc = torch.tensor([0, 5, 8], dtype=torch.int32, device=dev)
+    kda.kda_rollback(cfg, acc, tape, s1, conv_window=w1, conv_state=c1)
+    kda.kda_rollback_replay(cfg, acc, kua, s2, conv_window=w2, conv_state=c2)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2) and torch.equal(w1, w2)
+    assert torch.equal(s1, s2) and torch.equal(c1, c2)
+    for b, L in enumerate([0, 5, 8]):
+        # the block starts from S0 and the conv history: the oracle runs the L accepted drafts
+        blk = {k: D[k][b * Tb:b * Tb + L] for k in ('x', 'f', 'beta_logit', 'g')}
+        blk['cu_seqlens'] = torch.tensor([0, L], dtype=torch.int32)
+        ref = oracle_layer(cfg, P, blk, S0[b:b + 1], hist[b:b + 1])
+        assert rel_err(np64(s2[b]), ref['state'][0]) <= TOL[dtype], b
+        assert np.array_equal(np64(c2[b]), ref['conv_hist'][0]), b

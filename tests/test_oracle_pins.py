@@ -109,6 +109,44 @@ def pin_q_scale():
     return max(e1, e2)
 
 
+def pin_projections():
+    """The fused projection against a brute-force triple loop on a tiny case, and the
+    routing of its rows by hand: with W_in the identity on the first rows, x, f, the
+    beta logit and g_a are consecutive slices of the hidden state."""
+    rng = _rng(20)
+    T, H, d, r = 3, 2, 2, 2
+    n = 3 * H * d + H * d + H + r            # 12 + 4 + 2 + 2 = 20
+    hid = n + 3
+    hidden = rng.standard_normal((T, hid))
+    W_in = rng.standard_normal((n, hid))
+    W_gb = rng.standard_normal((H * d, r))
+    p = ko.projections(hidden, W_in, W_gb, H, d, r)
+    Y = np.zeros((T, n))
+    for t in range(T):
+        for j in range(n):
+            acc = 0.0
+            for c in range(hid):
+                acc += hidden[t, c] * W_in[j, c]
+            Y[t, j] = acc
+    G = np.zeros((T, H * d))
+    for t in range(T):
+        for j in range(H * d):
+            G[t, j] = sum(Y[t, 16 + H + c] * W_gb[j, c] for c in range(r))
+    e1 = max(np.abs(p['x'].reshape(T, -1) - Y[:, :12]).max(),
+             np.abs(p['f'].reshape(T, -1) - Y[:, 12:16]).max(),
+             np.abs(p['beta_logit'] - Y[:, 16:18]).max(), np.abs(p['g_a'] - Y[:, 18:20]).max(),
+             np.abs(p['g'].reshape(T, -1) - G).max())
+    eye = np.zeros((n, hid))
+    eye[:, :n] = np.eye(n)
+    q = ko.projections(hidden, eye, W_gb, H, d, r)
+    # x[t, h, :] = q_h | k_h | v_h: head 1's k is hidden columns 6 + 2 .. 6 + 3
+    e2 = max(np.abs(q['x'][:, 1, 2:4] - hidden[:, 8:10]).max(),
+             np.abs(q['f'][:, 0, :] - hidden[:, 12:14]).max(),
+             np.abs(q['beta_logit'] - hidden[:, 16:18]).max(),
+             np.abs(q['g_a'] - hidden[:, 18:20]).max())
+    return max(e1, e2)
+
+
 def pin_conv_library():
     """Conv against numpy.convolve with the kernel reversed (cross-correlation)."""
     rng = _rng(1)
@@ -287,6 +325,10 @@ def test_q_scale_doubles_outputs():
     assert pin_q_scale() < 1e-10
 
 
+def test_projections_brute_force_and_routing():
+    assert pin_projections() < 1e-12
+
+
 def test_conv_matches_numpy_convolve():
     assert pin_conv_library() < 1e-13
 
@@ -437,6 +479,7 @@ def _all_pins():
         'hand': pin_hand_example, 'brute_square': lambda: pin_brute_force(8, 8),
         'beta_zero': pin_beta_zero, 'retrieval': pin_retrieval,
         'softplus': pin_softplus_decay, 'q_scale': pin_q_scale,
+        'projections': pin_projections,
     }
     out = {}
     for name, fn in pins.items():
@@ -484,6 +527,24 @@ def _mut_layer_drops_q_scale(*args, q_scale=1.0, **kw):
     return ko.__dict__['_orig_layer'](*args, **kw)
 
 
+def _mut_proj_transposed_gate(hidden, W_in, W_gb, H, d, gate_rank):
+    """Mutation: g_b applied with the gate weight's layout transposed (rank-major)."""
+    p = ko.__dict__['_orig_projections'](hidden, W_in, W_gb, H, d, gate_rank)
+    T = p['g_a'].shape[0]
+    W = np.asarray(W_gb, np.float64).reshape(gate_rank, H * d).T
+    p['g'] = (p['g_a'] @ W.T).reshape(T, H, d)
+    return p
+
+
+def _mut_proj_beta_gate_swapped(hidden, W_in, W_gb, H, d, gate_rank):
+    """Mutation: the beta logit taken from the end of the fused rows (after g_a)."""
+    p = ko.__dict__['_orig_projections'](hidden, W_in, W_gb, H, d, gate_rank)
+    Y = np.asarray(hidden, np.float64) @ np.asarray(W_in, np.float64).T
+    nx, nf = 3 * H * d, H * d
+    p['beta_logit'] = Y[:, nx + nf + gate_rank:nx + nf + gate_rank + H]
+    return p
+
+
 def _mut_value_axis(S, a):
     return S * a[..., None, :]
 
@@ -527,6 +588,8 @@ MUTATIONS = {
     'softplus_no_rate': ('log_decay', _mut_softplus_no_rate),
     'q_scale_squared': ('recurrence', _mut_q_scale_squared),
     'layer_drops_q_scale': ('layer', _mut_layer_drops_q_scale),
+    'proj_transposed_gate': ('projections', _mut_proj_transposed_gate),
+    'proj_beta_gate_swapped': ('projections', _mut_proj_beta_gate_swapped),
 }
 
 
@@ -537,6 +600,7 @@ def test_mutation_is_caught(name, monkeypatch):
     monkeypatch.setitem(ko.__dict__, '_orig_log_decay', ko.log_decay)
     monkeypatch.setitem(ko.__dict__, '_orig_recurrence', ko.recurrence)
     monkeypatch.setitem(ko.__dict__, '_orig_layer', ko.layer)
+    monkeypatch.setitem(ko.__dict__, '_orig_projections', ko.projections)
     monkeypatch.setattr(ko, attr, fn)
     pins = _all_pins()
     failing = [k for k, e in pins.items() if not (e < 1e-10)]
