@@ -622,51 +622,64 @@ def run_decode(torch, kda, synth, dev, steps=1024):
          'log_a': torch.empty(B, H, d, device=dev), 'beta': torch.empty(B, H, device=dev)}
     y = torch.empty(steps, B, H, d, dtype=cfg.dtype, device=dev)
 
-    def one(i):
+    def fused(i):
+        # one launch: conv against the conv state (advanced in place), SiLU, norms, gate,
+        # beta and the state step
+        kda.kda_layer_decode(cfg, X['x'][i], X['f'][i], X['beta_logit'][i], X['g'][i],
+                             P['conv_w'], P['A_log'], P['dt_bias'], P['norm_w'], state,
+                             conv_state=conv, y=y[i])
+
+    def two_call(i):
         kda.kda_prep(cfg, cu, X['x'][i], X['f'][i], X['beta_logit'][i], P['conv_w'], P['A_log'],
                      P['dt_bias'], conv_state=conv, max_seqlen=1, out=o)
         kda.kda_decode(cfg, o['q'], o['k'], o['v'], o['log_a'], o['beta'], X['g'][i],
                        P['norm_w'], state, y=y[i])
 
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
-        one(0)                      # warm (also loads the kernels)
-    torch.cuda.current_stream().wait_stream(s)
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        for i in range(steps):
-            one(i)
-    g.replay()                      # warm
-    torch.cuda.synchronize()
+    def graph_ms(one):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            one(0)                  # warm (also loads the kernels)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(steps):
+                one(i)
+        g.replay()                  # warm
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1)
+
+    ms = graph_ms(fused)
+    ms_two = graph_ms(two_call)
+    # the decode kernel alone: back-to-back launches on resident inputs
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    g.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    # decode kernel alone: back-to-back launches on resident inputs
     n = 200
     for _ in range(3):
-        kda.kda_decode(cfg, o['q'], o['k'], o['v'], o['log_a'], o['beta'], X['g'][0],
-                       P['norm_w'], state, y=y[0])
+        fused(0)
     torch.cuda.synchronize()
     e0.record()
     for _ in range(n):
-        kda.kda_decode(cfg, o['q'], o['k'], o['v'], o['log_a'], o['beta'], X['g'][0],
-                       P['norm_w'], state, y=y[0])
+        fused(0)
     e1.record()
     torch.cuda.synchronize()
     ms_k = e0.elapsed_time(e1) / n
-    bytes_k = B * H * (2 * d * d * 4 + 3 * d * 4 + d * 2 + d * 4 + 4 + d * 2)
+    # per (b, h): state read + written, x row, conv history read + written, f, g, beta
+    # logit in, y out (bf16 activations)
+    bytes_k = B * H * (2 * d * d * 4 + 3 * d * 2 + 2 * 3 * 3 * d * 2 + d * 2 + d * 2 + 2 + d * 2)
     hbm, _, _, peak_kind = measured_peaks()
-    del g
     return {'value': B * steps / (ms / 1e3), 'unit': 'tokens/s',
             'workload': f'decode B={B} H={H} d={d}, {steps} steps after a {T0}-token prefill '
-                        '(prep + decode per step, CUDA graph)',
-            'ms_per_step': ms / steps, 'gpu_launches': 2 * steps,
-            'roofline': hbm_roofline('kda_decode', bytes_k, ms_k, hbm, peak_kind,
+                        '(kda_layer_decode: prep fused into the step kernel, CUDA graph)',
+            'ms_per_step': ms / steps, 'gpu_launches': steps,
+            'two_call_ms_per_step': ms_two / steps,
+            'roofline': hbm_roofline('kda_layer_decode', bytes_k, ms_k, hbm, peak_kind,
                                      'state 134 MB is just above L2 (126 MB)')}
 
 

@@ -269,9 +269,221 @@ static cudaError_t launch_step_p(const StepArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Decode at d = 128 as a persistent stream.  One CTA per SM walks the (sequence, head)
+// units; while it computes unit u from the state in its registers, the loads of unit
+// u + grid (its 64 KB state and, with the fused prep, its x row, conv history, f, beta
+// logit and g) are already in flight into a second register set, so every SM keeps a
+// state's worth of reads outstanding the whole time instead of alternating load and
+// compute phases.  The per-unit arithmetic is step_kernel's with the L2 normalisation of
+// q and k folded into the reductions: S^T k = (S^T k~) / max(||k~||, eps) with k~ the
+// un-normalised conv + SiLU output, so one barrier fewer per token.  Shared arrays are
+// double-buffered by unit parity, which leaves three block barriers per unit.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int DS_D = 128, DS_THREADS = 256, DS_ROWS = 16;   // rows rg + 8 i per thread
+
+template <typename T, bool PREP>
+struct DecodeIn {         // one unit's inputs as loaded (one thread's share)
+  float4 S[DS_ROWS];
+  float xc[2], hist[2][3];  // PREP: channels tid, tid + 256 (< 3d): x and 3 history rows
+  float f, g, beta_l;       // f, g at channel tid (< d); the beta logit
+  float q, k, v, la;        // !PREP: prep outputs at channel tid (< d); la = log a
+  int row;                  // state row (-1: skip)
+};
+
+template <typename T, bool PREP>
+__device__ __forceinline__ void ds_load(const StepArgs& a, int u, DecodeIn<T, PREP>& in) {
+  const int tid = threadIdx.x, cg = tid & 31, rg = tid >> 5;
+  const int H = a.H, b = u / H, h = u - b * H;
+  in.row = pool_row(a.slots, b, a.pool_size);
+  if (in.row < 0) return;
+  const float* Sg = a.state_in + ((size_t)in.row * H + h) * DS_D * DS_D;
+#pragma unroll
+  for (int i = 0; i < DS_ROWS; ++i) in.S[i] = ld4(Sg + (size_t)(rg + 8 * i) * DS_D + 4 * cg);
+  const size_t base = ((size_t)b * H + h) * DS_D;
+  if (PREP) {
+    constexpr int C3 = 3 * DS_D;
+    const T* xg = static_cast<const T*>(a.x) + ((size_t)b * H + h) * C3;
+    const T* cs = static_cast<const T*>(a.conv_state);
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int c = tid + 256 * m;
+      in.xc[m] = 0.f;
+      in.hist[m][0] = in.hist[m][1] = in.hist[m][2] = 0.f;
+      if (c < C3) {
+        in.xc[m] = ld1(xg + c);
+        if (cs != nullptr) {
+#pragma unroll
+          for (int j = 0; j < 3; ++j) in.hist[m][j] = ld1(cs + (((size_t)in.row * 3 + j) * H + h) * C3 + c);
+        }
+      }
+    }
+    if (tid < DS_D) {
+      in.f = ld1(static_cast<const T*>(a.f) + base + tid);
+      in.g = ld1(static_cast<const T*>(a.g) + base + tid);
+    }
+    in.beta_l = ld1(static_cast<const T*>(a.beta_logit) + (size_t)b * H + h);
+  } else {
+    if (tid < DS_D) {
+      in.q = __ldg(a.q + base + tid);
+      in.k = __ldg(a.k + base + tid);
+      in.v = __ldg(a.v + base + tid);
+      in.la = __ldg(a.loga + base + tid);
+      in.g = ld1(static_cast<const T*>(a.g) + base + tid);
+    }
+    in.beta_l = __ldg(a.beta + (size_t)b * H + h);
+  }
+}
+}  // namespace
+
+template <typename T, bool PREP>
+__global__ void __launch_bounds__(DS_THREADS, 1) decode_stream_kernel(const StepArgs a) {
+  constexpr int D = DS_D;
+  __shared__ __align__(16) float zq[2][D], zk[2][D], as_[2][D], us[2][D];
+  __shared__ __align__(16) float redk[8][D], redq[8][D];
+  __shared__ float nrm[2][8], kq_s[2], ssq[2][4];
+  const int tid = threadIdx.x, cg = tid & 31, rg = tid >> 5, lane = tid & 31, warp = tid >> 5;
+  const int H = a.H, n_units = a.B * H;
+  DecodeIn<T, PREP> cur, nxt;
+  int u = blockIdx.x, done = 0;
+  if (u < n_units) ds_load<T, PREP>(a, u, nxt);
+  for (; u < n_units; u += gridDim.x) {
+    cur = nxt;
+    if (u + (int)gridDim.x < n_units) ds_load<T, PREP>(a, u + gridDim.x, nxt);
+    if (cur.row < 0) continue;                           // uniform over the CTA
+    // buffer parity of the units this CTA computes (skipped units pass no barrier, so
+    // they must not flip it)
+    const int p = (done++) & 1, b = u / H, h = u - b * H;
+    const size_t base = ((size_t)b * H + h) * D;
+    float vv = 0.f, beta;
+    if (PREP) {
+      // depthwise causal conv (K = 4: three history rows and this token) + SiLU; thread tid
+      // owns channels tid (q or k) and tid + 256 (v, when < 3d)
+      constexpr int C3 = 3 * D;
+      T* cs = static_cast<T*>(a.conv_state);
+      float z[2];
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int c = tid + 256 * m;
+        z[m] = 0.f;
+        if (c < C3) {
+          const float4 w = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((size_t)h * C3 + c) * 4));
+          const float acc = fmaf(w.x, cur.hist[m][0], fmaf(w.y, cur.hist[m][1],
+                                 fmaf(w.z, cur.hist[m][2], w.w * cur.xc[m])));
+          z[m] = acc * fsig(acc);
+          if (cs != nullptr) {
+            st1(cs + (((size_t)cur.row * 3 + 0) * H + h) * C3 + c, cur.hist[m][1]);
+            st1(cs + (((size_t)cur.row * 3 + 1) * H + h) * C3 + c, cur.hist[m][2]);
+            st1(cs + (((size_t)cur.row * 3 + 2) * H + h) * C3 + c, cur.xc[m]);
+          }
+        }
+      }
+      // warps 0-3 hold q (channel tid) and v (tid + 256), warps 4-7 hold k
+      float sq = z[0] * z[0];
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+      if (lane == 0) nrm[p][warp] = sq;
+      if (tid < D) {
+        zq[p][tid] = z[0];
+        vv = z[1];
+        const float Ah = __expf(__ldg(a.A_log + h));
+        const float zf = cur.f + __ldg(a.dt_bias + (size_t)h * D + tid);
+        as_[p][tid] = __expf(a.gate_softplus ? -Ah * softplus(zf) : a.lb * fsig(Ah * zf));
+      } else {
+        zk[p][tid - D] = z[0];
+      }
+      beta = fsig(cur.beta_l);
+    } else {
+      if (tid < D) {
+        zq[p][tid] = cur.q;
+        zk[p][tid] = cur.k;
+        as_[p][tid] = expf(cur.la);
+        vv = cur.v;
+      }
+      beta = cur.beta_l;
+    }
+    __syncthreads();                                     // (1) q~, k~, a in shared memory
+    float iq = 1.f, ik = 1.f;
+    if (PREP) {
+      const float nq = nrm[p][0] + nrm[p][1] + nrm[p][2] + nrm[p][3];
+      const float nk = nrm[p][4] + nrm[p][5] + nrm[p][6] + nrm[p][7];
+      iq = 1.0f / fmaxf(sqrtf(nq), a.l2_eps);
+      ik = 1.0f / fmaxf(sqrtf(nk), a.l2_eps);
+    }
+    // decay along the key axis, then both column reductions (of the un-normalised q~, k~)
+    float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+#pragma unroll
+    for (int i = 0; i < DS_ROWS; ++i) {
+      const int r = rg + 8 * i;
+      cur.S[i] = f4_scale(cur.S[i], as_[p][r]);
+      pk = f4_fma(zk[p][r], cur.S[i], pk);
+      pq = f4_fma(zq[p][r], cur.S[i], pq);
+    }
+    *reinterpret_cast<float4*>(&redk[rg][4 * cg]) = pk;
+    *reinterpret_cast<float4*>(&redq[rg][4 * cg]) = pq;
+    if (warp == 0) {
+      float t = 0.f;
+#pragma unroll
+      for (int c = lane; c < D; c += 32) t = fmaf(zk[p][c], zq[p][c], t);
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+      if (lane == 0) kq_s[p] = t;
+    }
+    __syncthreads();                                     // (2) partial reductions
+    float o = 0.f;
+    if (tid < D) {
+      float rk = 0.f, rq = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { rk += redk[j][tid]; rq += redq[j][tid]; }
+      const float uu = beta * (vv - ik * rk);
+      o = a.q_scale * (iq * fmaf(uu * ik, kq_s[p], rq));
+      us[p][tid] = uu * ik;                              // k u^T = k~ (ik u)^T
+      float t = o * o;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+      if (lane == 0) ssq[p][warp] = t;
+    }
+    __syncthreads();                                     // (3) u and the norm partials
+    // rank-1 write with the un-normalised k~ (its scale moved into u), store the state
+    float* Sg = a.state_out + ((size_t)cur.row * H + h) * D * D;
+    const float4 u4 = *reinterpret_cast<const float4*>(&us[p][4 * cg]);
+#pragma unroll
+    for (int i = 0; i < DS_ROWS; ++i) {
+      const int r = rg + 8 * i;
+      st4(Sg + (size_t)r * D + 4 * cg, f4_fma(zk[p][r], u4, cur.S[i]));
+    }
+    if (tid < D) {
+      const float ss = ssq[p][0] + ssq[p][1] + ssq[p][2] + ssq[p][3];
+      const float rstd = rsqrtf(ss / (float)D + a.norm_eps);
+      st1(static_cast<T*>(a.y) + base + tid, o * rstd * __ldg(a.norm_w + tid) * fsig(cur.g));
+    }
+  }
+}
+
+template <typename T, bool PREP>
+static cudaError_t launch_decode_stream(const StepArgs& a, cudaStream_t st) {
+  int dev = 0, nsm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int units = a.B * a.H;
+  decode_stream_kernel<T, PREP><<<units < nsm ? units : nsm, DS_THREADS, 0, st>>>(a);
+  ++launch_counter();
+  return cudaGetLastError();
+}
+
+// the persistent stream serves one-token decode at d = 128 (K = 4 when the prep is fused)
+static bool decode_stream_applies(const StepArgs& a) {
+  return a.T == 1 && a.D == DS_D && a.tape == nullptr && a.tape_kua == nullptr &&
+         a.window == nullptr && a.state_out == a.state_in && (a.x == nullptr || a.K == 4);
+}
+
 template <typename T>
 static cudaError_t launch_step_t(const StepArgs& a, cudaStream_t st) {
   if (a.x != nullptr && (a.K < 1 || a.K > 8)) return cudaErrorInvalidValue;
+  if (decode_stream_applies(a))
+    return a.x ? launch_decode_stream<T, true>(a, st) : launch_decode_stream<T, false>(a, st);
   return a.x ? launch_step_p<T, true>(a, st) : launch_step_p<T, false>(a, st);
 }
 
