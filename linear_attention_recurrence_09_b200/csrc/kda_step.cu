@@ -37,6 +37,10 @@ struct StepShape {
 // ~1e-7); 1 / (1 + inf) = 0 keeps the saturated end exact
 __device__ __forceinline__ float fsig(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
 
+__device__ __forceinline__ uint32_t smem_u32_(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
 __device__ __forceinline__ float4 f4_scale(float4 a, float s) {
   return make_float4(a.x * s, a.y * s, a.z * s, a.w * s);
 }
@@ -45,24 +49,29 @@ __device__ __forceinline__ float4 f4_fma(float s, float4 a, float4 acc) {
                      fmaf(s, a.w, acc.w));
 }
 
+// One CTA per (head, sequence): the T tokens' inputs are independent of the state, so they
+// are made ready for every step first (loaded, or with the fused prep computed: the conv
+// over the window [history; block] for every (token, channel) at once, SiLU, the gate,
+// then the q / k L2 norms per token), and the recurrence then runs T steps on the state
+// in registers with two block barriers per step.
 template <typename T, int D, bool PREP>
 __global__ void __launch_bounds__(StepShape<D>::THREADS)
 step_kernel(const StepArgs a) {
   using SH = StepShape<D>;
-  constexpr int CG = SH::CG, RG = SH::RG, ROWS = SH::ROWS, THREADS = SH::THREADS;
-  __shared__ __align__(16) float ks[D];
-  __shared__ __align__(16) float qs[D];
-  __shared__ __align__(16) float as_[D];
+  constexpr int CG = SH::CG, RG = SH::RG, ROWS = SH::ROWS, THREADS = SH::THREADS, NW = SH::NW;
+  constexpr int TMAX = 16, C3 = 3 * D;
+  extern __shared__ __align__(16) float dsm[];
+  const int Tn = a.T;
+  float* qs = dsm;                    // [T][D] normalised q
+  float* ks = qs + Tn * D;            // [T][D] normalised k
+  float* vs = ks + Tn * D;            // [T][D] v
+  float* as_ = vs + Tn * D;           // [T][D] a = e^{log a}
+  float* gs = as_ + Tn * D;           // [T][D] g
+  float* xwin = gs + Tn * D;          // fused prep: [K-1+T][3d] pre-conv window
   __shared__ __align__(16) float us[D];
   __shared__ __align__(16) float redk[RG][D];
   __shared__ __align__(16) float redq[RG][D];
-  __shared__ float ssq[SH::NW];
-  __shared__ float kq_s;
-  // fused prep: conv history [K-1][3d] (oldest first), conv + SiLU outputs, v, beta, norms
-  constexpr int KMAX = 8;
-  __shared__ __align__(16) float hist[PREP ? KMAX - 1 : 1][PREP ? 3 * D : 1];
-  __shared__ __align__(16) float pre[PREP ? 3 * D : 1];
-  __shared__ float beta_s, nrm_w[SH::NW];   // per-warp partial sums of squares (q | k)
+  __shared__ float ssq[NW], kq_s[TMAX], beta_s[TMAX];
 
   const int h = blockIdx.x, b = blockIdx.y;
   const int H = a.H;
@@ -70,129 +79,103 @@ step_kernel(const StepArgs a) {
   if (row < 0) return;
   const int tid = threadIdx.x, cg = tid % CG, rg = tid / CG;
   const int lane = tid & 31, warp = tid >> 5;
-  const float* __restrict__ qg = a.q;
-  const float* __restrict__ kg = a.k;
-  const float* __restrict__ vg = a.v;
-  const T* __restrict__ gg = static_cast<const T*>(a.g);
-  T* __restrict__ yg = static_cast<T*>(a.y);
 
-  // the state streams in first: everything below (the prep of the first token
-  // included) runs while it arrives
+  // the state streams in first: the inputs below are made ready while it arrives
   const float* Sg = a.state_in + ((size_t)row * H + h) * D * D;
   float4 S[ROWS];
 #pragma unroll
   for (int i = 0; i < ROWS; ++i) S[i] = ld4(Sg + (size_t)(rg + i * RG) * D + 4 * cg);
 
-  constexpr int C3 = 3 * D;
   const int Km1 = PREP ? a.K - 1 : 0;
   T* csg = PREP ? static_cast<T*>(a.conv_state) : nullptr;
   T* wing = PREP ? static_cast<T*>(a.window) : nullptr;
   if (PREP) {
-    // the sequence's conv history for this head (zeros without a conv state); verify
-    // also starts its rollback window with it
-    for (int e = tid; e < Km1 * C3; e += THREADS) {
+    // the window [history; x of the block] (history zeros without a conv state); verify
+    // also writes it out for the rollback
+    for (int e = tid; e < (Km1 + Tn) * C3; e += THREADS) {
       const int j = e / C3, c = e - j * C3;
-      float hv = 0.f;
-      if (csg) hv = ld1(csg + (((size_t)row * Km1 + j) * H + h) * C3 + c);
-      hist[j][c] = hv;
-      if (wing) st1(wing + (((size_t)b * (Km1 + a.T) + j) * H + h) * C3 + c, hv);
-    }
-    __syncthreads();   // loaded by (row, channel) pairs, used per channel below
-  }
-
-  for (int t = 0; t < a.T; ++t) {
-    const size_t tok = (size_t)b * a.T + t;
-    const size_t base = (tok * H + h) * D;
-    if (PREP) {
-      // depthwise causal conv (tap K-1 = this token) + SiLU per channel of q|k|v; each
-      // thread owns its channels, so it also shifts their history.  Channel c < 2d (q, k)
-      // of thread c also accumulates its warp's sum of squares.
-      const T* xg = static_cast<const T*>(a.x) + tok * H * C3 + (size_t)h * C3;
-      const T* fg = static_cast<const T*>(a.f) + base;
-      float sq = 0.f;
-      for (int c = tid; c < C3; c += THREADS) {
-        const float xc = ld1(xg + c);
-        const float* w = a.conv_w + ((size_t)h * C3 + c) * a.K;
-        float acc;
-        if (a.K == 4) {   // the common case: one 16-byte load of the taps
-          const float4 w4 = __ldg(reinterpret_cast<const float4*>(w));
-          acc = fmaf(w4.x, hist[0][c], fmaf(w4.y, hist[1][c], fmaf(w4.z, hist[2][c], w4.w * xc)));
-        } else {
-          acc = __ldg(w + Km1) * xc;
-          for (int j = 0; j < Km1; ++j) acc = fmaf(__ldg(w + j), hist[j][c], acc);
-        }
-        const float z = acc * fsig(acc);
-        pre[c] = z;
-        if (c < 2 * D) sq = fmaf(z, z, sq);
-        for (int j = 0; j + 1 < Km1; ++j) hist[j][c] = hist[j + 1][c];
-        if (Km1 > 0) hist[Km1 - 1][c] = xc;
-        if (wing) st1(wing + (((size_t)b * (Km1 + a.T) + Km1 + t) * H + h) * C3 + c, xc);
-      }
-      // warps whose first channels are q (resp. k) hold q (resp. k) partial norms; with
-      // d < 32 a warp spans both, so the d < 32 shapes reduce per half-warp group below
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
-      if (lane == 0) nrm_w[warp] = sq;
-      // decay a = exp(lb sigmoid(exp(A_log) (f + dt_bias))) (or exp(-exp(A_log) softplus(..))
-      // for the gate without a lower bound) and beta = sigmoid(logit)
-      const float Ah = __expf(__ldg(a.A_log + h));
-      for (int c = tid; c < D; c += THREADS) {
-        const float z = ld1(fg + c) + __ldg(a.dt_bias + (size_t)h * D + c);
-        as_[c] = __expf(a.gate_softplus ? -Ah * softplus(z) : a.lb * fsig(Ah * z));
-      }
-      if (tid == 0) beta_s = fsig(ld1(static_cast<const T*>(a.beta_logit) + tok * H + h));
-      __syncthreads();
-      if (D >= 32) {
-        // q channels are those of warps [0, d/32), k channels of warps [d/32, 2d/32)
-        float nq = 0.f, nk = 0.f;
-#pragma unroll
-        for (int w = 0; w < D / 32; ++w) { nq += nrm_w[w]; nk += nrm_w[D / 32 + w]; }
-        const float iq = 1.0f / fmaxf(sqrtf(nq), a.l2_eps), ik = 1.0f / fmaxf(sqrtf(nk), a.l2_eps);
-        for (int c = tid; c < D; c += THREADS) {
-          qs[c] = pre[c] * iq;
-          ks[c] = pre[D + c] * ik;
-        }
+      float v = 0.f;
+      if (j < Km1) {
+        if (csg) v = ld1(csg + (((size_t)row * Km1 + j) * H + h) * C3 + c);
       } else {
-        // d = 16: one warp covers q and k; reduce each half directly
-        float nq = 0.f, nk = 0.f;
-        for (int c = 0; c < D; ++c) {
-          nq = fmaf(pre[c], pre[c], nq);
-          nk = fmaf(pre[D + c], pre[D + c], nk);
-        }
-        const float iq = 1.0f / fmaxf(sqrtf(nq), a.l2_eps), ik = 1.0f / fmaxf(sqrtf(nk), a.l2_eps);
-        for (int c = tid; c < D; c += THREADS) {
-          qs[c] = pre[c] * iq;
-          ks[c] = pre[D + c] * ik;
-        }
+        v = ld1(static_cast<const T*>(a.x) + (((size_t)b * Tn + (j - Km1)) * H + h) * C3 + c);
       }
-    } else {
-      for (int c = tid; c < D; c += THREADS) {
-        ks[c] = __ldg(kg + base + c);
-        qs[c] = __ldg(qg + base + c);
-        as_[c] = expf(__ldg(a.loga + base + c));
-      }
+      xwin[e] = v;
+      if (wing) st1(wing + (((size_t)b * (Km1 + Tn) + j) * H + h) * C3 + c, v);
+    }
+    const float Ah = __expf(__ldg(a.A_log + h));
+    for (int e = tid; e < Tn * D; e += THREADS) {
+      const int t = e / D, c = e - t * D;
+      const size_t idx = (((size_t)b * Tn + t) * H + h) * D + c;
+      const float z = ld1(static_cast<const T*>(a.f) + idx) + __ldg(a.dt_bias + (size_t)h * D + c);
+      as_[e] = __expf(a.gate_softplus ? -Ah * softplus(z) : a.lb * fsig(Ah * z));
+      gs[e] = ld1(static_cast<const T*>(a.g) + idx);
+    }
+    for (int t = tid; t < Tn; t += THREADS)
+      beta_s[t] = fsig(ld1(static_cast<const T*>(a.beta_logit) + ((size_t)b * Tn + t) * H + h));
+    __syncthreads();
+    // depthwise causal conv (tap K-1 = the token itself) + SiLU for every (token, channel)
+    for (int e = tid; e < Tn * C3; e += THREADS) {
+      const int t = e / C3, c = e - t * C3;
+      const float* w = a.conv_w + ((size_t)h * C3 + c) * a.K;
+      float acc = __ldg(w + Km1) * xwin[(t + Km1) * C3 + c];
+      for (int j = Km1 - 1; j >= 0; --j) acc = fmaf(__ldg(w + j), xwin[(t + j) * C3 + c], acc);
+      const float z = acc * fsig(acc);
+      const int part = c / D;
+      (part == 0 ? qs : part == 1 ? ks : vs)[t * D + (c - part * D)] = z;
     }
     __syncthreads();
+    // L2 norms of q and k per token: one warp per (token, q | k), scaled in place
+    for (int pidx = warp; pidx < 2 * Tn; pidx += NW) {
+      float* arr = ((pidx & 1) ? ks : qs) + (pidx >> 1) * D;
+      float ss = 0.f;
+      for (int c = lane; c < D; c += 32) ss = fmaf(arr[c], arr[c], ss);
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      const float inv = 1.0f / fmaxf(sqrtf(ss), a.l2_eps);
+      for (int c = lane; c < D; c += 32) arr[c] *= inv;
+    }
+  } else {
+    for (int e = tid; e < Tn * D; e += THREADS) {
+      const int t = e / D, c = e - t * D;
+      const size_t idx = (((size_t)b * Tn + t) * H + h) * D + c;
+      qs[e] = __ldg(a.q + idx);
+      ks[e] = __ldg(a.k + idx);
+      vs[e] = __ldg(a.v + idx);
+      as_[e] = expf(__ldg(a.loga + idx));
+      gs[e] = ld1(static_cast<const T*>(a.g) + idx);
+    }
+    for (int t = tid; t < Tn; t += THREADS)
+      beta_s[t] = __ldg(a.beta + ((size_t)b * Tn + t) * H + h);
+  }
+  __syncthreads();
+  // k . q per token (lane-strided, then a butterfly: the decode kernels' order)
+  for (int t = warp; t < Tn; t += NW) {
+    float p = 0.f;
+    for (int c = lane; c < D; c += 32) p = fmaf(ks[t * D + c], qs[t * D + c], p);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
+    if (lane == 0) kq_s[t] = p;
+  }
+  __syncthreads();
 
+  for (int t = 0; t < Tn; ++t) {
+    const size_t tok = (size_t)b * Tn + t;
+    const float* kt = ks + t * D;
+    const float* qt = qs + t * D;
+    const float* at = as_ + t * D;
     // decay along the key axis, then both column reductions in one pass
     float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
 #pragma unroll
     for (int i = 0; i < ROWS; ++i) {
       const int r = rg + i * RG;
-      S[i] = f4_scale(S[i], as_[r]);
-      pk = f4_fma(ks[r], S[i], pk);
-      pq = f4_fma(qs[r], S[i], pq);
+      S[i] = f4_scale(S[i], at[r]);
+      pk = f4_fma(kt[r], S[i], pk);
+      pq = f4_fma(qt[r], S[i], pq);
     }
     *reinterpret_cast<float4*>(&redk[rg][4 * cg]) = pk;
     *reinterpret_cast<float4*>(&redq[rg][4 * cg]) = pq;
-    if (warp == 0) {
-      float p = 0.f;
-      for (int c = lane; c < D; c += 32) p = fmaf(ks[c], qs[c], p);
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
-      if (lane == 0) kq_s = p;
-    }
-    __syncthreads();
+    __syncthreads();                                       // (A) partial reductions
 
     // per value column: u = b (v - S^T k), o = S^T q + u (k.q), RMSNorm partials
     float o = 0.f;
@@ -200,16 +183,14 @@ step_kernel(const StepArgs a) {
       float rk = 0.f, rq = 0.f;
 #pragma unroll
       for (int j = 0; j < RG; ++j) { rk += redk[j][tid]; rq += redq[j][tid]; }
-      const float bt = PREP ? beta_s : __ldg(a.beta + tok * H + h);
-      const float vt = PREP ? pre[2 * D + tid] : __ldg(vg + base + tid);
-      const float u = bt * (vt - rk);
-      o = a.q_scale * fmaf(u, kq_s, rq);
+      const float u = beta_s[t] * (vs[t * D + tid] - rk);
+      o = a.q_scale * fmaf(u, kq_s[t], rq);
       us[tid] = u;
       if (a.tape_kua != nullptr) {   // compact tape: this step's k, u and a
         float* tk = a.tape_kua + (tok * H + h) * 3 * D;
-        tk[tid] = ks[tid];
+        tk[tid] = kt[tid];
         tk[D + tid] = u;
-        tk[2 * D + tid] = as_[tid];
+        tk[2 * D + tid] = at[tid];
       }
     }
     if (warp < (D + 31) / 32) {
@@ -218,35 +199,36 @@ step_kernel(const StepArgs a) {
       for (int off = 16; off >= 1; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
       if (lane == 0) ssq[warp] = p;
     }
-    __syncthreads();
+    __syncthreads();                                       // (B) u and the norm partials
 
-    // rank-1 write and the gated RMSNorm epilogue
+    // rank-1 write and the gated RMSNorm epilogue.  The next step rewrites redk/redq, us
+    // and ssq only after its barrier (A), which every thread reaches after these reads.
 #pragma unroll
     for (int i = 0; i < ROWS; ++i) {
       const int r = rg + i * RG;
-      S[i] = f4_fma(ks[r], *reinterpret_cast<const float4*>(&us[4 * cg]), S[i]);
+      S[i] = f4_fma(kt[r], *reinterpret_cast<const float4*>(&us[4 * cg]), S[i]);
     }
     if (tid < D) {
       float ss = 0.f;
 #pragma unroll
       for (int w = 0; w < (D + 31) / 32; ++w) ss += ssq[w];
       const float rstd = rsqrtf(ss / (float)D + a.norm_eps);
-      const float gt = ld1(gg + base + tid);
-      st1(yg + base + tid, o * rstd * __ldg(a.norm_w + tid) * sigmoid(gt));
+      st1(static_cast<T*>(a.y) + (tok * H + h) * D + tid,
+          o * rstd * __ldg(a.norm_w + tid) * sigmoid(gs[t * D + tid]));
     }
     if (a.tape != nullptr) {
       float* tp = a.tape + (tok * H + h) * D * D;
 #pragma unroll
       for (int i = 0; i < ROWS; ++i) st4(tp + (size_t)(rg + i * RG) * D + 4 * cg, S[i]);
     }
-    __syncthreads();
   }
 
   if (PREP && csg != nullptr && wing == nullptr) {
-    // decode: the history now ends with this step's token(s); each thread wrote its own
-    // channels of hist, so no barrier is needed before it stores them
-    for (int c = tid; c < C3; c += THREADS)
-      for (int j = 0; j < Km1; ++j) st1(csg + (((size_t)row * Km1 + j) * H + h) * C3 + c, hist[j][c]);
+    // decode: the history now ends with this block's tokens (the last K-1 window rows)
+    for (int e = tid; e < Km1 * C3; e += THREADS) {
+      const int j = e / C3, c = e - j * C3;
+      st1(csg + (((size_t)row * Km1 + j) * H + h) * C3 + c, xwin[(Tn + j) * C3 + c]);
+    }
   }
   if (a.state_out != nullptr) {
     float* So = a.state_out + ((size_t)row * H + h) * D * D;
@@ -258,11 +240,22 @@ step_kernel(const StepArgs a) {
 template <typename T, bool PREP>
 static cudaError_t launch_step_p(const StepArgs& a, cudaStream_t st) {
   dim3 grid(a.H, a.B);
+  const size_t smem =
+      sizeof(float) * ((size_t)5 * a.T * a.D + (PREP ? (size_t)(a.K - 1 + a.T) * 3 * a.D : 0));
+  cudaError_t e = cudaSuccess;
   switch (a.D) {
-    case 16: step_kernel<T, 16, PREP><<<grid, StepShape<16>::THREADS, 0, st>>>(a); break;
-    case 32: step_kernel<T, 32, PREP><<<grid, StepShape<32>::THREADS, 0, st>>>(a); break;
-    case 64: step_kernel<T, 64, PREP><<<grid, StepShape<64>::THREADS, 0, st>>>(a); break;
-    case 128: step_kernel<T, 128, PREP><<<grid, StepShape<128>::THREADS, 0, st>>>(a); break;
+#define KDA_STEP_CASE(DD)                                                                     \
+  case DD:                                                                                    \
+    e = cudaFuncSetAttribute(step_kernel<T, DD, PREP>,                                        \
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);         \
+    if (e != cudaSuccess) return e;                                                           \
+    step_kernel<T, DD, PREP><<<grid, StepShape<DD>::THREADS, smem, st>>>(a);                  \
+    break;
+    KDA_STEP_CASE(16)
+    KDA_STEP_CASE(32)
+    KDA_STEP_CASE(64)
+    KDA_STEP_CASE(128)
+#undef KDA_STEP_CASE
     default: return cudaErrorInvalidValue;
   }
   ++launch_counter();
@@ -270,37 +263,51 @@ static cudaError_t launch_step_p(const StepArgs& a, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------------------
-// Decode at d = 128 as a persistent stream.  One CTA per SM walks the (sequence, head)
-// units; while it computes unit u from the state in its registers, the loads of unit
-// u + grid (its 64 KB state and, with the fused prep, its x row, conv history, f, beta
-// logit and g) are already in flight into a second register set, so every SM keeps a
-// state's worth of reads outstanding the whole time instead of alternating load and
-// compute phases.  The per-unit arithmetic is step_kernel's with the L2 normalisation of
-// q and k folded into the reductions: S^T k = (S^T k~) / max(||k~||, eps) with k~ the
-// un-normalised conv + SiLU output, so one barrier fewer per token.  Shared arrays are
-// double-buffered by unit parity, which leaves three block barriers per unit.
+// Decode at d = 128 as a persistent stream.  Each CTA walks (sequence, head) units; the
+// state of the unit after the current one is copied into shared memory with cp.async
+// (each thread copies exactly the 16 float4 it will later read, so the buffer needs no
+// block barrier) while the current unit is computed from registers, and the small prep
+// inputs of the next unit are loaded into a second register set.  Two CTAs per SM
+// (64 KB of state in flight each), so the SM never waits for a whole state load.  The
+// per-unit arithmetic is step_kernel's with the L2 normalisation of q and k folded into
+// the reductions: S^T k = (S^T k~) / max(||k~||, eps) with k~ the un-normalised conv +
+// SiLU output, so one barrier fewer per token.  Shared arrays are double-buffered by unit
+// parity, which leaves three block barriers per unit.  No spin-waits: the only waits are
+// cp.async.wait_all and block barriers.
 // ---------------------------------------------------------------------------
 namespace {
 constexpr int DS_D = 128, DS_THREADS = 256, DS_ROWS = 16;   // rows rg + 8 i per thread
 
-template <typename T, bool PREP>
-struct DecodeIn {         // one unit's inputs as loaded (one thread's share)
-  float4 S[DS_ROWS];
+template <bool PREP>
+struct DecodeIn {           // one unit's small inputs as loaded (one thread's share)
   float xc[2], hist[2][3];  // PREP: channels tid, tid + 256 (< 3d): x and 3 history rows
-  float f, g, beta_l;       // f, g at channel tid (< d); the beta logit
+  float f, g, beta_l;       // f, g at channel tid (< d); the beta logit (or beta)
   float q, k, v, la;        // !PREP: prep outputs at channel tid (< d); la = log a
-  int row;                  // state row (-1: skip)
 };
 
-template <typename T, bool PREP>
-__device__ __forceinline__ void ds_load(const StepArgs& a, int u, DecodeIn<T, PREP>& in) {
-  const int tid = threadIdx.x, cg = tid & 31, rg = tid >> 5;
-  const int H = a.H, b = u / H, h = u - b * H;
-  in.row = pool_row(a.slots, b, a.pool_size);
-  if (in.row < 0) return;
-  const float* Sg = a.state_in + ((size_t)in.row * H + h) * DS_D * DS_D;
+// the state row of unit u (-1: no unit or skipped)
+__device__ __forceinline__ int ds_row(const StepArgs& a, int u) {
+  if (u >= a.B * a.H) return -1;
+  return pool_row(a.slots, u / a.H, a.pool_size);
+}
+
+// asynchronous copy of this thread's 16 float4 of unit u's state into its shared slots
+__device__ __forceinline__ void ds_copy_state(const StepArgs& a, int u, int row, float4* sbuf) {
+  const int tid = threadIdx.x, cg = tid & 31, rg = tid >> 5, h = u % a.H;
+  const float* Sg = a.state_in + ((size_t)row * a.H + h) * DS_D * DS_D;
 #pragma unroll
-  for (int i = 0; i < DS_ROWS; ++i) in.S[i] = ld4(Sg + (size_t)(rg + 8 * i) * DS_D + 4 * cg);
+  for (int i = 0; i < DS_ROWS; ++i) {
+    const uint32_t dst = smem_u32_(sbuf + i * DS_THREADS + tid);
+    const float* src = Sg + (size_t)(rg + 8 * i) * DS_D + 4 * cg;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <typename T, bool PREP>
+__device__ __forceinline__ void ds_load_small(const StepArgs& a, int u, int row, DecodeIn<PREP>& in) {
+  const int tid = threadIdx.x;
+  const int H = a.H, b = u / H, h = u - b * H;
   const size_t base = ((size_t)b * H + h) * DS_D;
   if (PREP) {
     constexpr int C3 = 3 * DS_D;
@@ -315,7 +322,7 @@ __device__ __forceinline__ void ds_load(const StepArgs& a, int u, DecodeIn<T, PR
         in.xc[m] = ld1(xg + c);
         if (cs != nullptr) {
 #pragma unroll
-          for (int j = 0; j < 3; ++j) in.hist[m][j] = ld1(cs + (((size_t)in.row * 3 + j) * H + h) * C3 + c);
+          for (int j = 0; j < 3; ++j) in.hist[m][j] = ld1(cs + (((size_t)row * 3 + j) * H + h) * C3 + c);
         }
       }
     }
@@ -338,24 +345,37 @@ __device__ __forceinline__ void ds_load(const StepArgs& a, int u, DecodeIn<T, PR
 }  // namespace
 
 template <typename T, bool PREP>
-__global__ void __launch_bounds__(DS_THREADS, 1) decode_stream_kernel(const StepArgs a) {
+__global__ void __launch_bounds__(DS_THREADS, 2) decode_stream_kernel(const StepArgs a) {
   constexpr int D = DS_D;
+  extern __shared__ float4 sbuf[];                      // [DS_ROWS][DS_THREADS]: 64 KB
   __shared__ __align__(16) float zq[2][D], zk[2][D], as_[2][D], us[2][D];
   __shared__ __align__(16) float redk[8][D], redq[8][D];
   __shared__ float nrm[2][8], kq_s[2], ssq[2][4];
   const int tid = threadIdx.x, cg = tid & 31, rg = tid >> 5, lane = tid & 31, warp = tid >> 5;
-  const int H = a.H, n_units = a.B * H;
-  DecodeIn<T, PREP> cur, nxt;
-  int u = blockIdx.x, done = 0;
-  if (u < n_units) ds_load<T, PREP>(a, u, nxt);
-  for (; u < n_units; u += gridDim.x) {
-    cur = nxt;
-    if (u + (int)gridDim.x < n_units) ds_load<T, PREP>(a, u + gridDim.x, nxt);
-    if (cur.row < 0) continue;                           // uniform over the CTA
-    // buffer parity of the units this CTA computes (skipped units pass no barrier, so
-    // they must not flip it)
-    const int p = (done++) & 1, b = u / H, h = u - b * H;
+  const int H = a.H, n_units = a.B * H, G = gridDim.x;
+  // this CTA's units with a state row, in order: u, then the next one after it
+  auto next_unit = [&](int v) {
+    for (; v < n_units; v += G)
+      if (ds_row(a, v) >= 0) return v;
+    return n_units;
+  };
+  int u = next_unit(blockIdx.x);
+  DecodeIn<PREP> cur, nxt;
+  if (u < n_units) {
+    ds_copy_state(a, u, ds_row(a, u), sbuf);
+    ds_load_small<T, PREP>(a, u, ds_row(a, u), nxt);
+  }
+  for (int done = 0; u < n_units; ++done) {
+    const int un = next_unit(u + G);
+    const int row = ds_row(a, u), p = done & 1, b = u / H, h = u - b * H;
     const size_t base = ((size_t)b * H + h) * D;
+    // this unit's state: its copy has landed (each thread waits for its own)
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    float4 S[DS_ROWS];
+#pragma unroll
+    for (int i = 0; i < DS_ROWS; ++i) S[i] = sbuf[i * DS_THREADS + tid];
+    cur = nxt;
+    if (un < n_units) ds_load_small<T, PREP>(a, un, ds_row(a, un), nxt);
     float vv = 0.f, beta;
     if (PREP) {
       // depthwise causal conv (K = 4: three history rows and this token) + SiLU; thread tid
@@ -373,9 +393,9 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_stream_kernel(const Step
                                  fmaf(w.z, cur.hist[m][2], w.w * cur.xc[m])));
           z[m] = acc * fsig(acc);
           if (cs != nullptr) {
-            st1(cs + (((size_t)cur.row * 3 + 0) * H + h) * C3 + c, cur.hist[m][1]);
-            st1(cs + (((size_t)cur.row * 3 + 1) * H + h) * C3 + c, cur.hist[m][2]);
-            st1(cs + (((size_t)cur.row * 3 + 2) * H + h) * C3 + c, cur.xc[m]);
+            st1(cs + (((size_t)row * 3 + 0) * H + h) * C3 + c, cur.hist[m][1]);
+            st1(cs + (((size_t)row * 3 + 1) * H + h) * C3 + c, cur.hist[m][2]);
+            st1(cs + (((size_t)row * 3 + 2) * H + h) * C3 + c, cur.xc[m]);
           }
         }
       }
@@ -416,10 +436,13 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_stream_kernel(const Step
 #pragma unroll
     for (int i = 0; i < DS_ROWS; ++i) {
       const int r = rg + 8 * i;
-      cur.S[i] = f4_scale(cur.S[i], as_[p][r]);
-      pk = f4_fma(zk[p][r], cur.S[i], pk);
-      pq = f4_fma(zq[p][r], cur.S[i], pq);
+      S[i] = f4_scale(S[i], as_[p][r]);
+      pk = f4_fma(zk[p][r], S[i], pk);
+      pq = f4_fma(zq[p][r], S[i], pq);
     }
+    // every read of this thread's shared slots has been consumed: refill them with the
+    // next unit's state while this one finishes
+    if (un < n_units) ds_copy_state(a, un, ds_row(a, un), sbuf);
     *reinterpret_cast<float4*>(&redk[rg][4 * cg]) = pk;
     *reinterpret_cast<float4*>(&redq[rg][4 * cg]) = pq;
     if (warp == 0) {
@@ -446,29 +469,34 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_stream_kernel(const Step
     }
     __syncthreads();                                     // (3) u and the norm partials
     // rank-1 write with the un-normalised k~ (its scale moved into u), store the state
-    float* Sg = a.state_out + ((size_t)cur.row * H + h) * D * D;
+    float* Sg = a.state_out + ((size_t)row * H + h) * D * D;
     const float4 u4 = *reinterpret_cast<const float4*>(&us[p][4 * cg]);
 #pragma unroll
     for (int i = 0; i < DS_ROWS; ++i) {
       const int r = rg + 8 * i;
-      st4(Sg + (size_t)r * D + 4 * cg, f4_fma(zk[p][r], u4, cur.S[i]));
+      st4(Sg + (size_t)r * D + 4 * cg, f4_fma(zk[p][r], u4, S[i]));
     }
     if (tid < D) {
       const float ss = ssq[p][0] + ssq[p][1] + ssq[p][2] + ssq[p][3];
       const float rstd = rsqrtf(ss / (float)D + a.norm_eps);
-      st1(static_cast<T*>(a.y) + base + tid, o * rstd * __ldg(a.norm_w + tid) * fsig(cur.g));
+      st1(static_cast<T*>(a.y) + base + tid, o * rstd * __ldg(a.norm_w + tid) * sigmoid(cur.g));
     }
+    u = un;
   }
 }
 
 template <typename T, bool PREP>
 static cudaError_t launch_decode_stream(const StepArgs& a, cudaStream_t st) {
+  constexpr int SMEM = DS_ROWS * DS_THREADS * 16;      // 64 KB of state per CTA
   int dev = 0, nsm = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(decode_stream_kernel<T, PREP>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
-  const int units = a.B * a.H;
-  decode_stream_kernel<T, PREP><<<units < nsm ? units : nsm, DS_THREADS, 0, st>>>(a);
+  const int units = a.B * a.H, grid = 2 * nsm;          // two resident CTAs per SM
+  decode_stream_kernel<T, PREP><<<units < grid ? units : grid, DS_THREADS, SMEM, st>>>(a);
   ++launch_counter();
   return cudaGetLastError();
 }
