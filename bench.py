@@ -708,30 +708,41 @@ def run_verify(torch, kda, synth, dev, rounds=256):
     vargs = lambda r: (v4(o['q'], H, d), v4(o['k'], H, d), v4(o['v'], H, d),
                        v4(o['log_a'], H, d), v4(o['beta'], H), X['g'][r], P['norm_w'], state)
 
-    def one(r, compact):
+    win4 = win.view(B, Tb + K - 1, H, 3 * d)
+    xb = lambda r, key, *tail: X[key][r].view(B, Tb, *tail)
+
+    def one(r, mode):
+        if mode == 'fused':
+            # one launch for prep + verify (compact tape), then the replay rollback
+            kda.kda_layer_verify_compact(cfg, xb(r, 'x', H, 3 * d), xb(r, 'f', H, d),
+                                         xb(r, 'beta_logit', H), X['g'][r], P['conv_w'],
+                                         P['A_log'], P['dt_bias'], P['norm_w'], state,
+                                         conv_state=conv, tape_kua=kua, window=win4, y=y)
+            kda.kda_rollback_replay(cfg, acc[r], kua, state, conv_window=win4, conv_state=conv)
+            return
         # prep (conv window for the rollback), verify, rollback to the accepted prefix
         kda.kda_prep(cfg, cu, X['x'][r].view(B * Tb, H, 3 * d), X['f'][r].view(B * Tb, H, d),
                      X['beta_logit'][r].view(B * Tb, H), P['conv_w'], P['A_log'], P['dt_bias'],
                      conv_state=conv, conv_mode=kda.KDA_CONV_TAPE, conv_window=win,
                      max_seqlen=Tb, out=o)
-        if compact:
+        if mode == 'compact':
             kda.kda_verify_compact(cfg, *vargs(r), tape_kua=kua, y=y)
             kda.kda_rollback_replay(cfg, acc[r], kua, state, conv_window=win, conv_state=conv)
         else:
             kda.kda_verify(cfg, *vargs(r), tape=tape, y=y)
             kda.kda_rollback(cfg, acc[r], tape, state, conv_window=win, conv_state=conv)
 
-    def graph_ms(compact):
+    def graph_ms(mode):
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
-            one(0, compact)
+            one(0, mode)
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for r in range(rounds):
-                one(r, compact)
+                one(r, mode)
         g.replay()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -754,8 +765,9 @@ def run_verify(torch, kda, synth, dev, rounds=256):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / n
 
-    ms = graph_ms(True)
-    ms_full = graph_ms(False)
+    ms = graph_ms('fused')
+    ms_two = graph_ms('compact')
+    ms_full = graph_ms('full')
     ms_k = launch_ms(lambda: kda.kda_verify_compact(cfg, *vargs(0), tape_kua=kua, y=y))
     ms_r = launch_ms(lambda: kda.kda_rollback_replay(cfg, acc[0], kua, state, conv_window=win,
                                                      conv_state=conv))
@@ -767,8 +779,10 @@ def run_verify(torch, kda, synth, dev, rounds=256):
     return {'value': B * Tb * rounds / (ms / 1e3), 'unit': 'verified draft tokens/s',
             'workload': f'verify+rollback B={B} H={H} d={d}, blocks of {Tb} after a {T0}-token '
                         f'context, {rounds} rounds, accepted ~ U{{0..{Tb}}} (CUDA graph; '
-                        'compact (k, u, a) tape, rollback by replay)',
-            'ms_per_round': ms / rounds, 'gpu_launches': 3 * rounds,
+                        'kda_layer_verify_compact: prep fused, compact (k, u, a) tape; '
+                        'kda_rollback_replay)',
+            'ms_per_round': ms / rounds, 'gpu_launches': 2 * rounds,
+            'prep_then_verify_ms_per_round': ms_two / rounds,
             'full_state_tape_ms_per_round': ms_full / rounds,
             'roofline': hbm_roofline('kda_verify_compact', bytes_k, ms_k, hbm, peak_kind),
             'rollback_replay': {'ms_per_launch': ms_r, 'algorithmic_bytes_per_launch': bytes_r,

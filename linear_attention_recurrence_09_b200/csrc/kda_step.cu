@@ -37,10 +37,6 @@ struct StepShape {
 // ~1e-7); 1 / (1 + inf) = 0 keeps the saturated end exact
 __device__ __forceinline__ float fsig(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
 
-__device__ __forceinline__ uint32_t smem_u32_(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
 __device__ __forceinline__ float4 f4_scale(float4 a, float s) {
   return make_float4(a.x * s, a.y * s, a.z * s, a.w * s);
 }
@@ -49,43 +45,17 @@ __device__ __forceinline__ float4 f4_fma(float s, float4 a, float4 acc) {
                      fmaf(s, a.w, acc.w));
 }
 
-// One CTA per (head, sequence): the T tokens' inputs are independent of the state, so they
-// are made ready for every step first (loaded, or with the fused prep computed: the conv
-// over the window [history; block] for every (token, channel) at once, SiLU, the gate,
-// then the q / k L2 norms per token), and the recurrence then runs T steps on the state
-// in registers with two block barriers per step.
-template <typename T, int D, bool PREP>
-__global__ void __launch_bounds__(StepShape<D>::THREADS)
-step_kernel(const StepArgs a) {
-  using SH = StepShape<D>;
-  constexpr int CG = SH::CG, RG = SH::RG, ROWS = SH::ROWS, THREADS = SH::THREADS, NW = SH::NW;
-  constexpr int TMAX = 16, C3 = 3 * D;
-  extern __shared__ __align__(16) float dsm[];
-  const int Tn = a.T;
-  float* qs = dsm;                    // [T][D] normalised q
-  float* ks = qs + Tn * D;            // [T][D] normalised k
-  float* vs = ks + Tn * D;            // [T][D] v
-  float* as_ = vs + Tn * D;           // [T][D] a = e^{log a}
-  float* gs = as_ + Tn * D;           // [T][D] g
-  float* xwin = gs + Tn * D;          // fused prep: [K-1+T][3d] pre-conv window
-  __shared__ __align__(16) float us[D];
-  __shared__ __align__(16) float redk[RG][D];
-  __shared__ __align__(16) float redq[RG][D];
-  __shared__ float ssq[NW], kq_s[TMAX], beta_s[TMAX];
-
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int H = a.H;
-  const int row = pool_row(a.slots, b, a.pool_size);
-  if (row < 0) return;
-  const int tid = threadIdx.x, cg = tid % CG, rg = tid / CG;
-  const int lane = tid & 31, warp = tid >> 5;
-
-  // the state streams in first: the inputs below are made ready while it arrives
-  const float* Sg = a.state_in + ((size_t)row * H + h) * D * D;
-  float4 S[ROWS];
-#pragma unroll
-  for (int i = 0; i < ROWS; ++i) S[i] = ld4(Sg + (size_t)(rg + i * RG) * D + 4 * cg);
-
+// The T tokens' inputs are independent of the state, so they are made ready for every
+// step first, in shared memory: loaded (kda_verify / kda_decode), or with the fused prep
+// computed (kda_layer_*): the conv over the window [history; block] for every (token,
+// channel) at once, SiLU, the gate, then the q / k L2 norms per token.  Also k . q per
+// token.  Shared by the step kernels below; ends with a block barrier.
+template <typename T, int D, bool PREP, int THREADS>
+__device__ __forceinline__ void stage_inputs(const StepArgs& a, int b, int h, int row, float* qs,
+                                             float* ks, float* vs, float* as_, float* gs,
+                                             float* xwin, float* kq_s, float* beta_s) {
+  constexpr int NW = THREADS / 32, C3 = 3 * D;
+  const int H = a.H, Tn = a.T, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Km1 = PREP ? a.K - 1 : 0;
   T* csg = PREP ? static_cast<T*>(a.conv_state) : nullptr;
   T* wing = PREP ? static_cast<T*>(a.window) : nullptr;
@@ -159,6 +129,56 @@ step_kernel(const StepArgs a) {
   }
   __syncthreads();
 
+}
+
+// The conv-state commit of kda_layer_decode: the history ends with the block's tokens
+// (the last K-1 rows of the window in shared memory)
+template <typename T, int D, int THREADS>
+__device__ __forceinline__ void commit_conv(const StepArgs& a, int h, int row, const float* xwin) {
+  constexpr int C3 = 3 * D;
+  const int Km1 = a.K - 1, H = a.H;
+  T* csg = static_cast<T*>(a.conv_state);
+  for (int e = threadIdx.x; e < Km1 * C3; e += THREADS) {
+    const int j = e / C3, c = e - j * C3;
+    st1(csg + (((size_t)row * Km1 + j) * H + h) * C3 + c, xwin[(a.T + j) * C3 + c]);
+  }
+}
+
+// One CTA per (head, sequence), any d: the inputs of every step staged first, then the
+// recurrence runs T steps on the state in registers with two block barriers per step.
+template <typename T, int D, bool PREP>
+__global__ void __launch_bounds__(StepShape<D>::THREADS)
+step_kernel(const StepArgs a) {
+  using SH = StepShape<D>;
+  constexpr int CG = SH::CG, RG = SH::RG, ROWS = SH::ROWS, THREADS = SH::THREADS, NW = SH::NW;
+  constexpr int TMAX = 16;
+  extern __shared__ __align__(16) float dsm[];
+  const int Tn = a.T;
+  float* qs = dsm;                    // [T][D] normalised q
+  float* ks = qs + Tn * D;            // [T][D] normalised k
+  float* vs = ks + Tn * D;            // [T][D] v
+  float* as_ = vs + Tn * D;           // [T][D] a = e^{log a}
+  float* gs = as_ + Tn * D;           // [T][D] g
+  float* xwin = gs + Tn * D;          // fused prep: [K-1+T][3d] pre-conv window
+  __shared__ __align__(16) float us[D];
+  __shared__ __align__(16) float redk[RG][D];
+  __shared__ __align__(16) float redq[RG][D];
+  __shared__ float ssq[NW], kq_s[TMAX], beta_s[TMAX];
+
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int H = a.H;
+  const int row = pool_row(a.slots, b, a.pool_size);
+  if (row < 0) return;
+  const int tid = threadIdx.x, cg = tid % CG, rg = tid / CG;
+  const int lane = tid & 31, warp = tid >> 5;
+
+  // the state streams in first: the inputs below are made ready while it arrives
+  const float* Sg = a.state_in + ((size_t)row * H + h) * D * D;
+  float4 S[ROWS];
+#pragma unroll
+  for (int i = 0; i < ROWS; ++i) S[i] = ld4(Sg + (size_t)(rg + i * RG) * D + 4 * cg);
+
+  stage_inputs<T, D, PREP, THREADS>(a, b, h, row, qs, ks, vs, as_, gs, xwin, kq_s, beta_s);
   for (int t = 0; t < Tn; ++t) {
     const size_t tok = (size_t)b * Tn + t;
     const float* kt = ks + t * D;
@@ -223,13 +243,8 @@ step_kernel(const StepArgs a) {
     }
   }
 
-  if (PREP && csg != nullptr && wing == nullptr) {
-    // decode: the history now ends with this block's tokens (the last K-1 window rows)
-    for (int e = tid; e < Km1 * C3; e += THREADS) {
-      const int j = e / C3, c = e - j * C3;
-      st1(csg + (((size_t)row * Km1 + j) * H + h) * C3 + c, xwin[(Tn + j) * C3 + c]);
-    }
-  }
+  if (PREP && a.conv_state != nullptr && a.window == nullptr)
+    commit_conv<T, D, THREADS>(a, h, row, xwin);
   if (a.state_out != nullptr) {
     float* So = a.state_out + ((size_t)row * H + h) * D * D;
 #pragma unroll
@@ -262,256 +277,9 @@ static cudaError_t launch_step_p(const StepArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// ---------------------------------------------------------------------------
-// Decode at d = 128 as a persistent stream.  Each CTA walks (sequence, head) units; the
-// state of the unit after the current one is copied into shared memory with cp.async
-// (each thread copies exactly the 16 float4 it will later read, so the buffer needs no
-// block barrier) while the current unit is computed from registers, and the small prep
-// inputs of the next unit are loaded into a second register set.  Two CTAs per SM
-// (64 KB of state in flight each), so the SM never waits for a whole state load.  The
-// per-unit arithmetic is step_kernel's with the L2 normalisation of q and k folded into
-// the reductions: S^T k = (S^T k~) / max(||k~||, eps) with k~ the un-normalised conv +
-// SiLU output, so one barrier fewer per token.  Shared arrays are double-buffered by unit
-// parity, which leaves three block barriers per unit.  No spin-waits: the only waits are
-// cp.async.wait_all and block barriers.
-// ---------------------------------------------------------------------------
-namespace {
-constexpr int DS_D = 128, DS_THREADS = 256, DS_ROWS = 16;   // rows rg + 8 i per thread
-
-template <bool PREP>
-struct DecodeIn {           // one unit's small inputs as loaded (one thread's share)
-  float xc[2], hist[2][3];  // PREP: channels tid, tid + 256 (< 3d): x and 3 history rows
-  float f, g, beta_l;       // f, g at channel tid (< d); the beta logit (or beta)
-  float q, k, v, la;        // !PREP: prep outputs at channel tid (< d); la = log a
-};
-
-// the state row of unit u (-1: no unit or skipped)
-__device__ __forceinline__ int ds_row(const StepArgs& a, int u) {
-  if (u >= a.B * a.H) return -1;
-  return pool_row(a.slots, u / a.H, a.pool_size);
-}
-
-// asynchronous copy of this thread's 16 float4 of unit u's state into its shared slots
-__device__ __forceinline__ void ds_copy_state(const StepArgs& a, int u, int row, float4* sbuf) {
-  const int tid = threadIdx.x, cg = tid & 31, rg = tid >> 5, h = u % a.H;
-  const float* Sg = a.state_in + ((size_t)row * a.H + h) * DS_D * DS_D;
-#pragma unroll
-  for (int i = 0; i < DS_ROWS; ++i) {
-    const uint32_t dst = smem_u32_(sbuf + i * DS_THREADS + tid);
-    const float* src = Sg + (size_t)(rg + 8 * i) * DS_D + 4 * cg;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-  }
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-template <typename T, bool PREP>
-__device__ __forceinline__ void ds_load_small(const StepArgs& a, int u, int row, DecodeIn<PREP>& in) {
-  const int tid = threadIdx.x;
-  const int H = a.H, b = u / H, h = u - b * H;
-  const size_t base = ((size_t)b * H + h) * DS_D;
-  if (PREP) {
-    constexpr int C3 = 3 * DS_D;
-    const T* xg = static_cast<const T*>(a.x) + ((size_t)b * H + h) * C3;
-    const T* cs = static_cast<const T*>(a.conv_state);
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      const int c = tid + 256 * m;
-      in.xc[m] = 0.f;
-      in.hist[m][0] = in.hist[m][1] = in.hist[m][2] = 0.f;
-      if (c < C3) {
-        in.xc[m] = ld1(xg + c);
-        if (cs != nullptr) {
-#pragma unroll
-          for (int j = 0; j < 3; ++j) in.hist[m][j] = ld1(cs + (((size_t)row * 3 + j) * H + h) * C3 + c);
-        }
-      }
-    }
-    if (tid < DS_D) {
-      in.f = ld1(static_cast<const T*>(a.f) + base + tid);
-      in.g = ld1(static_cast<const T*>(a.g) + base + tid);
-    }
-    in.beta_l = ld1(static_cast<const T*>(a.beta_logit) + (size_t)b * H + h);
-  } else {
-    if (tid < DS_D) {
-      in.q = __ldg(a.q + base + tid);
-      in.k = __ldg(a.k + base + tid);
-      in.v = __ldg(a.v + base + tid);
-      in.la = __ldg(a.loga + base + tid);
-      in.g = ld1(static_cast<const T*>(a.g) + base + tid);
-    }
-    in.beta_l = __ldg(a.beta + (size_t)b * H + h);
-  }
-}
-}  // namespace
-
-template <typename T, bool PREP>
-__global__ void __launch_bounds__(DS_THREADS, 2) decode_stream_kernel(const StepArgs a) {
-  constexpr int D = DS_D;
-  extern __shared__ float4 sbuf[];                      // [DS_ROWS][DS_THREADS]: 64 KB
-  __shared__ __align__(16) float zq[2][D], zk[2][D], as_[2][D], us[2][D];
-  __shared__ __align__(16) float redk[8][D], redq[8][D];
-  __shared__ float nrm[2][8], kq_s[2], ssq[2][4];
-  const int tid = threadIdx.x, cg = tid & 31, rg = tid >> 5, lane = tid & 31, warp = tid >> 5;
-  const int H = a.H, n_units = a.B * H, G = gridDim.x;
-  // this CTA's units with a state row, in order: u, then the next one after it
-  auto next_unit = [&](int v) {
-    for (; v < n_units; v += G)
-      if (ds_row(a, v) >= 0) return v;
-    return n_units;
-  };
-  int u = next_unit(blockIdx.x);
-  DecodeIn<PREP> cur, nxt;
-  if (u < n_units) {
-    ds_copy_state(a, u, ds_row(a, u), sbuf);
-    ds_load_small<T, PREP>(a, u, ds_row(a, u), nxt);
-  }
-  for (int done = 0; u < n_units; ++done) {
-    const int un = next_unit(u + G);
-    const int row = ds_row(a, u), p = done & 1, b = u / H, h = u - b * H;
-    const size_t base = ((size_t)b * H + h) * D;
-    // this unit's state: its copy has landed (each thread waits for its own)
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    float4 S[DS_ROWS];
-#pragma unroll
-    for (int i = 0; i < DS_ROWS; ++i) S[i] = sbuf[i * DS_THREADS + tid];
-    cur = nxt;
-    if (un < n_units) ds_load_small<T, PREP>(a, un, ds_row(a, un), nxt);
-    float vv = 0.f, beta;
-    if (PREP) {
-      // depthwise causal conv (K = 4: three history rows and this token) + SiLU; thread tid
-      // owns channels tid (q or k) and tid + 256 (v, when < 3d)
-      constexpr int C3 = 3 * D;
-      T* cs = static_cast<T*>(a.conv_state);
-      float z[2];
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const int c = tid + 256 * m;
-        z[m] = 0.f;
-        if (c < C3) {
-          const float4 w = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((size_t)h * C3 + c) * 4));
-          const float acc = fmaf(w.x, cur.hist[m][0], fmaf(w.y, cur.hist[m][1],
-                                 fmaf(w.z, cur.hist[m][2], w.w * cur.xc[m])));
-          z[m] = acc * fsig(acc);
-          if (cs != nullptr) {
-            st1(cs + (((size_t)row * 3 + 0) * H + h) * C3 + c, cur.hist[m][1]);
-            st1(cs + (((size_t)row * 3 + 1) * H + h) * C3 + c, cur.hist[m][2]);
-            st1(cs + (((size_t)row * 3 + 2) * H + h) * C3 + c, cur.xc[m]);
-          }
-        }
-      }
-      // warps 0-3 hold q (channel tid) and v (tid + 256), warps 4-7 hold k
-      float sq = z[0] * z[0];
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
-      if (lane == 0) nrm[p][warp] = sq;
-      if (tid < D) {
-        zq[p][tid] = z[0];
-        vv = z[1];
-        const float Ah = __expf(__ldg(a.A_log + h));
-        const float zf = cur.f + __ldg(a.dt_bias + (size_t)h * D + tid);
-        as_[p][tid] = __expf(a.gate_softplus ? -Ah * softplus(zf) : a.lb * fsig(Ah * zf));
-      } else {
-        zk[p][tid - D] = z[0];
-      }
-      beta = fsig(cur.beta_l);
-    } else {
-      if (tid < D) {
-        zq[p][tid] = cur.q;
-        zk[p][tid] = cur.k;
-        as_[p][tid] = expf(cur.la);
-        vv = cur.v;
-      }
-      beta = cur.beta_l;
-    }
-    __syncthreads();                                     // (1) q~, k~, a in shared memory
-    float iq = 1.f, ik = 1.f;
-    if (PREP) {
-      const float nq = nrm[p][0] + nrm[p][1] + nrm[p][2] + nrm[p][3];
-      const float nk = nrm[p][4] + nrm[p][5] + nrm[p][6] + nrm[p][7];
-      iq = 1.0f / fmaxf(sqrtf(nq), a.l2_eps);
-      ik = 1.0f / fmaxf(sqrtf(nk), a.l2_eps);
-    }
-    // decay along the key axis, then both column reductions (of the un-normalised q~, k~)
-    float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
-#pragma unroll
-    for (int i = 0; i < DS_ROWS; ++i) {
-      const int r = rg + 8 * i;
-      S[i] = f4_scale(S[i], as_[p][r]);
-      pk = f4_fma(zk[p][r], S[i], pk);
-      pq = f4_fma(zq[p][r], S[i], pq);
-    }
-    // every read of this thread's shared slots has been consumed: refill them with the
-    // next unit's state while this one finishes
-    if (un < n_units) ds_copy_state(a, un, ds_row(a, un), sbuf);
-    *reinterpret_cast<float4*>(&redk[rg][4 * cg]) = pk;
-    *reinterpret_cast<float4*>(&redq[rg][4 * cg]) = pq;
-    if (warp == 0) {
-      float t = 0.f;
-#pragma unroll
-      for (int c = lane; c < D; c += 32) t = fmaf(zk[p][c], zq[p][c], t);
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
-      if (lane == 0) kq_s[p] = t;
-    }
-    __syncthreads();                                     // (2) partial reductions
-    float o = 0.f;
-    if (tid < D) {
-      float rk = 0.f, rq = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) { rk += redk[j][tid]; rq += redq[j][tid]; }
-      const float uu = beta * (vv - ik * rk);
-      o = a.q_scale * (iq * fmaf(uu * ik, kq_s[p], rq));
-      us[p][tid] = uu * ik;                              // k u^T = k~ (ik u)^T
-      float t = o * o;
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
-      if (lane == 0) ssq[p][warp] = t;
-    }
-    __syncthreads();                                     // (3) u and the norm partials
-    // rank-1 write with the un-normalised k~ (its scale moved into u), store the state
-    float* Sg = a.state_out + ((size_t)row * H + h) * D * D;
-    const float4 u4 = *reinterpret_cast<const float4*>(&us[p][4 * cg]);
-#pragma unroll
-    for (int i = 0; i < DS_ROWS; ++i) {
-      const int r = rg + 8 * i;
-      st4(Sg + (size_t)r * D + 4 * cg, f4_fma(zk[p][r], u4, S[i]));
-    }
-    if (tid < D) {
-      const float ss = ssq[p][0] + ssq[p][1] + ssq[p][2] + ssq[p][3];
-      const float rstd = rsqrtf(ss / (float)D + a.norm_eps);
-      st1(static_cast<T*>(a.y) + base + tid, o * rstd * __ldg(a.norm_w + tid) * sigmoid(cur.g));
-    }
-    u = un;
-  }
-}
-
-template <typename T, bool PREP>
-static cudaError_t launch_decode_stream(const StepArgs& a, cudaStream_t st) {
-  constexpr int SMEM = DS_ROWS * DS_THREADS * 16;      // 64 KB of state per CTA
-  int dev = 0, nsm = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(decode_stream_kernel<T, PREP>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-  if (e != cudaSuccess) return e;
-  const int units = a.B * a.H, grid = 2 * nsm;          // two resident CTAs per SM
-  decode_stream_kernel<T, PREP><<<units < grid ? units : grid, DS_THREADS, SMEM, st>>>(a);
-  ++launch_counter();
-  return cudaGetLastError();
-}
-
-// the persistent stream serves one-token decode at d = 128 (K = 4 when the prep is fused)
-static bool decode_stream_applies(const StepArgs& a) {
-  return a.T == 1 && a.D == DS_D && a.tape == nullptr && a.tape_kua == nullptr &&
-         a.window == nullptr && a.state_out == a.state_in && (a.x == nullptr || a.K == 4);
-}
-
 template <typename T>
 static cudaError_t launch_step_t(const StepArgs& a, cudaStream_t st) {
   if (a.x != nullptr && (a.K < 1 || a.K > 8)) return cudaErrorInvalidValue;
-  if (decode_stream_applies(a))
-    return a.x ? launch_decode_stream<T, true>(a, st) : launch_decode_stream<T, false>(a, st);
   return a.x ? launch_step_p<T, true>(a, st) : launch_step_p<T, false>(a, st);
 }
 
