@@ -768,11 +768,16 @@ def run_verify(torch, kda, synth, dev, rounds=256):
     ms = graph_ms('fused')
     ms_two = graph_ms('compact')
     ms_full = graph_ms('full')
-    ms_k = launch_ms(lambda: kda.kda_verify_compact(cfg, *vargs(0), tape_kua=kua, y=y))
+    ms_k = launch_ms(lambda: kda.kda_layer_verify_compact(
+        cfg, xb(0, 'x', H, 3 * d), xb(0, 'f', H, d), xb(0, 'beta_logit', H), X['g'][0],
+        P['conv_w'], P['A_log'], P['dt_bias'], P['norm_w'], state, conv_state=conv,
+        tape_kua=kua, window=win4, y=y))
     ms_r = launch_ms(lambda: kda.kda_rollback_replay(cfg, acc[0], kua, state, conv_window=win,
                                                      conv_state=conv))
-    io = Tb * (3 * d * 4 + d * 4 + 4 + d * 2 + d * 2)          # q, k, v, log a, beta, g in; y out
-    bytes_k = B * H * (d * d * 4 + io + Tb * 3 * d * 4)         # + the state in, compact tape out
+    # per (b, h): the state in; per draft x, f, g, beta logit in, y and the compact tape out;
+    # the conv history in and the rollback window [history; block] out (bf16 activations)
+    io = Tb * (3 * d * 2 + d * 2 + d * 2 + 2 + d * 2 + 3 * d * 4)
+    bytes_k = B * H * (d * d * 4 + io + (K - 1) * 3 * d * 2 + (K - 1 + Tb) * 3 * d * 2)
     n_acc = int((acc[0] > 0).sum())
     bytes_r = n_acc * H * (2 * d * d * 4) + int(acc[0].sum()) * H * 3 * d * 4
     hbm, _, _, peak_kind = measured_peaks()
@@ -784,7 +789,7 @@ def run_verify(torch, kda, synth, dev, rounds=256):
             'ms_per_round': ms / rounds, 'gpu_launches': 2 * rounds,
             'prep_then_verify_ms_per_round': ms_two / rounds,
             'full_state_tape_ms_per_round': ms_full / rounds,
-            'roofline': hbm_roofline('kda_verify_compact', bytes_k, ms_k, hbm, peak_kind),
+            'roofline': hbm_roofline('kda_layer_verify_compact', bytes_k, ms_k, hbm, peak_kind),
             'rollback_replay': {'ms_per_launch': ms_r, 'algorithmic_bytes_per_launch': bytes_r,
                                 'frac': bytes_r / (ms_r / 1e3) / 1e9 / hbm}}
 
