@@ -152,10 +152,8 @@ PROFILED = {
                     'linear_attention_recurrence_09_b200/csrc/kda_intra_sm100.cu'),
     'inter_chunk': ('profiles/interchunk_sm100_prefill_8k.md',
                     'linear_attention_recurrence_09_b200/csrc/kda_prefill_sm100.cu'),
-    'kda_decode': ('profiles/step_decode_b64.md',
-                   'linear_attention_recurrence_09_b200/csrc/kda_step.cu'),
-    'kda_verify': ('profiles/step_verify_b16.md',
-                   'linear_attention_recurrence_09_b200/csrc/kda_step.cu'),
+    'proj_gemm': ('profiles/proj_gemm_layer_8k.md',
+                  'linear_attention_recurrence_09_b200/csrc/kda_gemm_sm100.cu'),
 }
 
 
@@ -506,7 +504,8 @@ def run_layer_full(torch, kda, synth, dev, steps=10, warmup=3):
             'tensor_roofline': {'bound': 'tensor', 'kernel': 'kda_proj_gemm (2 launches)',
                                 'achieved': ach, 'peak': tc, 'unit': 'TFLOP/s',
                                 'frac': ach / tc, 'frac_sustained': ach / tc_sus,
-                                'gflop_per_step': flops / 1e9, 'peak_kind': peak_kind}}
+                                'gflop_per_step': flops / 1e9, 'peak_kind': peak_kind,
+                                'traffic_fused_projection': profiled_traffic('proj_gemm')}}
 
 
 def run_long(torch, kda, synth, dev, steps=5, warmup=3):
@@ -656,30 +655,33 @@ def run_decode(torch, kda, synth, dev, steps=1024):
         del g
         return e0.elapsed_time(e1)
 
-    ms = graph_ms(fused)
-    ms_two = graph_ms(two_call)
+    # the two-call step (kda_prep, then kda_decode) is timed first and is the headline: on
+    # B200 it is faster than the one-launch kda_layer_decode, timed beside it
+    ms = graph_ms(two_call)
+    ms_fused = graph_ms(fused)
     # the decode kernel alone: back-to-back launches on resident inputs
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n = 200
+    dec = lambda: kda.kda_decode(cfg, o['q'], o['k'], o['v'], o['log_a'], o['beta'], X['g'][0],
+                                 P['norm_w'], state, y=y[0])
     for _ in range(3):
-        fused(0)
+        dec()
     torch.cuda.synchronize()
     e0.record()
     for _ in range(n):
-        fused(0)
+        dec()
     e1.record()
     torch.cuda.synchronize()
     ms_k = e0.elapsed_time(e1) / n
-    # per (b, h): state read + written, x row, conv history read + written, f, g, beta
-    # logit in, y out (bf16 activations)
-    bytes_k = B * H * (2 * d * d * 4 + 3 * d * 2 + 2 * 3 * 3 * d * 2 + d * 2 + d * 2 + 2 + d * 2)
+    # per (b, h): state read + written; q, k, v, log a (fp32), beta in; g in, y out (bf16)
+    bytes_k = B * H * (2 * d * d * 4 + 4 * d * 4 + 4 + d * 2 + d * 2)
     hbm, _, _, peak_kind = measured_peaks()
     return {'value': B * steps / (ms / 1e3), 'unit': 'tokens/s',
             'workload': f'decode B={B} H={H} d={d}, {steps} steps after a {T0}-token prefill '
-                        '(kda_layer_decode: prep fused into the step kernel, CUDA graph)',
-            'ms_per_step': ms / steps, 'gpu_launches': steps,
-            'two_call_ms_per_step': ms_two / steps,
-            'roofline': hbm_roofline('kda_layer_decode', bytes_k, ms_k, hbm, peak_kind,
+                        '(kda_prep + kda_decode per step, CUDA graph)',
+            'ms_per_step': ms / steps, 'gpu_launches': 2 * steps,
+            'fused_ms_per_step': ms_fused / steps,
+            'roofline': hbm_roofline('kda_decode', bytes_k, ms_k, hbm, peak_kind,
                                      'state 134 MB is just above L2 (126 MB)')}
 
 
@@ -765,31 +767,31 @@ def run_verify(torch, kda, synth, dev, rounds=256):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / n
 
-    ms = graph_ms('fused')
-    ms_two = graph_ms('compact')
+    # the three-call round (kda_prep, kda_verify_compact, kda_rollback_replay) is timed first
+    # and is the headline: on B200 it is faster than the two-call round with the prep fused
+    # (kda_layer_verify_compact), timed beside it with the full-state tape round
+    ms = graph_ms('compact')
+    ms_fused = graph_ms('fused')
     ms_full = graph_ms('full')
-    ms_k = launch_ms(lambda: kda.kda_layer_verify_compact(
-        cfg, xb(0, 'x', H, 3 * d), xb(0, 'f', H, d), xb(0, 'beta_logit', H), X['g'][0],
-        P['conv_w'], P['A_log'], P['dt_bias'], P['norm_w'], state, conv_state=conv,
-        tape_kua=kua, window=win4, y=y))
+    ms_k = launch_ms(lambda: kda.kda_verify_compact(cfg, *vargs(0), tape_kua=kua, y=y))
     ms_r = launch_ms(lambda: kda.kda_rollback_replay(cfg, acc[0], kua, state, conv_window=win,
                                                      conv_state=conv))
-    # per (b, h): the state in; per draft x, f, g, beta logit in, y and the compact tape out;
-    # the conv history in and the rollback window [history; block] out (bf16 activations)
-    io = Tb * (3 * d * 2 + d * 2 + d * 2 + 2 + d * 2 + 3 * d * 4)
-    bytes_k = B * H * (d * d * 4 + io + (K - 1) * 3 * d * 2 + (K - 1 + Tb) * 3 * d * 2)
+    # per (b, h): the state in; per draft q, k, v, log a (fp32), beta, g in; y and the
+    # compact tape (3 d fp32) out
+    io = Tb * (4 * d * 4 + 4 + d * 2 + d * 2 + 3 * d * 4)
+    bytes_k = B * H * (d * d * 4 + io)
     n_acc = int((acc[0] > 0).sum())
     bytes_r = n_acc * H * (2 * d * d * 4) + int(acc[0].sum()) * H * 3 * d * 4
     hbm, _, _, peak_kind = measured_peaks()
     return {'value': B * Tb * rounds / (ms / 1e3), 'unit': 'verified draft tokens/s',
             'workload': f'verify+rollback B={B} H={H} d={d}, blocks of {Tb} after a {T0}-token '
                         f'context, {rounds} rounds, accepted ~ U{{0..{Tb}}} (CUDA graph; '
-                        'kda_layer_verify_compact: prep fused, compact (k, u, a) tape; '
+                        'kda_prep, kda_verify_compact with the compact (k, u, a) tape, '
                         'kda_rollback_replay)',
-            'ms_per_round': ms / rounds, 'gpu_launches': 2 * rounds,
-            'prep_then_verify_ms_per_round': ms_two / rounds,
+            'ms_per_round': ms / rounds, 'gpu_launches': 3 * rounds,
+            'fused_prep_ms_per_round': ms_fused / rounds,
             'full_state_tape_ms_per_round': ms_full / rounds,
-            'roofline': hbm_roofline('kda_layer_verify_compact', bytes_k, ms_k, hbm, peak_kind),
+            'roofline': hbm_roofline('kda_verify_compact', bytes_k, ms_k, hbm, peak_kind),
             'rollback_replay': {'ms_per_launch': ms_r, 'algorithmic_bytes_per_launch': bytes_r,
                                 'frac': bytes_r / (ms_r / 1e3) / 1e9 / hbm}}
 
