@@ -84,15 +84,29 @@ __device__ __forceinline__ void stage_inputs(const StepArgs& a, int b, int h, in
     for (int t = tid; t < Tn; t += THREADS)
       beta_s[t] = fsig(ld1(static_cast<const T*>(a.beta_logit) + ((size_t)b * Tn + t) * H + h));
     __syncthreads();
-    // depthwise causal conv (tap K-1 = the token itself) + SiLU for every (token, channel)
-    for (int e = tid; e < Tn * C3; e += THREADS) {
-      const int t = e / C3, c = e - t * C3;
-      const float* w = a.conv_w + ((size_t)h * C3 + c) * a.K;
-      float acc = __ldg(w + Km1) * xwin[(t + Km1) * C3 + c];
-      for (int j = Km1 - 1; j >= 0; --j) acc = fmaf(__ldg(w + j), xwin[(t + j) * C3 + c], acc);
-      const float z = acc * fsig(acc);
+    // depthwise causal conv (tap K-1 = the token itself) + SiLU: each thread owns channels
+    // (their taps loaded once, one 16-byte load when K = 4) and walks the block's tokens
+    for (int c = tid; c < C3; c += THREADS) {
+      const float* wp = a.conv_w + ((size_t)h * C3 + c) * a.K;
+      float w[8];
+      if (a.K == 4) {
+        const float4 w4 = __ldg(reinterpret_cast<const float4*>(wp));
+        w[0] = w4.x; w[1] = w4.y; w[2] = w4.z; w[3] = w4.w;
+#pragma unroll
+        for (int j = 4; j < 8; ++j) w[j] = 0.f;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[j] = (j < a.K) ? __ldg(wp + j) : 0.f;
+      }
       const int part = c / D;
-      (part == 0 ? qs : part == 1 ? ks : vs)[t * D + (c - part * D)] = z;
+      float* dst = (part == 0 ? qs : part == 1 ? ks : vs) + (c - part * D);
+      for (int t = 0; t < Tn; ++t) {
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 7; j >= 0; --j)
+          if (j <= Km1) acc = fmaf(w[j], xwin[(t + j) * C3 + c], acc);
+        dst[t * D] = acc * fsig(acc);
+      }
     }
     __syncthreads();
     // L2 norms of q and k per token: one warp per (token, q | k), scaled in place
