@@ -154,6 +154,10 @@ PROFILED = {
                     'linear_attention_recurrence_09_b200/csrc/kda_prefill_sm100.cu'),
     'proj_gemm': ('profiles/proj_gemm_layer_8k.md',
                   'linear_attention_recurrence_09_b200/csrc/kda_gemm_sm100.cu'),
+    'kda_decode': ('profiles/step_decode_b64.md',
+                   'linear_attention_recurrence_09_b200/csrc/kda_step.cu'),
+    'kda_verify_compact': ('profiles/step_verify_compact_b16.md',
+                           'linear_attention_recurrence_09_b200/csrc/kda_step.cu'),
 }
 
 
