@@ -19,6 +19,7 @@ the max over ranks.  ``--impl reference`` times the float64 CPU oracle.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -632,10 +633,13 @@ def run_decode(torch, kda, synth, dev, steps=1024):
                              P['conv_w'], P['A_log'], P['dt_bias'], P['norm_w'], state,
                              conv_state=conv, y=y[i])
 
-    def two_call(i):
+    # the decode kernel streams the state while kda_prep (which never writes it) finishes
+    cfg_early = dataclasses.replace(cfg, launch_flags=kda.KDA_LAUNCH_EARLY_STATE)
+
+    def two_call(i, c_step=cfg_early):
         kda.kda_prep(cfg, cu, X['x'][i], X['f'][i], X['beta_logit'][i], P['conv_w'], P['A_log'],
                      P['dt_bias'], conv_state=conv, max_seqlen=1, out=o)
-        kda.kda_decode(cfg, o['q'], o['k'], o['v'], o['log_a'], o['beta'], X['g'][i],
+        kda.kda_decode(c_step, o['q'], o['k'], o['v'], o['log_a'], o['beta'], X['g'][i],
                        P['norm_w'], state, y=y[i])
 
     def graph_ms(one):
@@ -662,6 +666,7 @@ def run_decode(torch, kda, synth, dev, steps=1024):
     # the two-call step (kda_prep, then kda_decode) is timed first and is the headline: on
     # B200 it is faster than the one-launch kda_layer_decode, timed beside it
     ms = graph_ms(two_call)
+    ms_wait = graph_ms(lambda i: two_call(i, cfg))
     ms_fused = graph_ms(fused)
     # the decode kernel alone: back-to-back launches on resident inputs
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -682,8 +687,10 @@ def run_decode(torch, kda, synth, dev, steps=1024):
     hbm, _, _, peak_kind = measured_peaks()
     return {'value': B * steps / (ms / 1e3), 'unit': 'tokens/s',
             'workload': f'decode B={B} H={H} d={d}, {steps} steps after a {T0}-token prefill '
-                        '(kda_prep + kda_decode per step, CUDA graph)',
+                        '(kda_prep + kda_decode per step, CUDA graph; the decode launch '
+                        'streams the state while kda_prep finishes)',
             'ms_per_step': ms / steps, 'gpu_launches': 2 * steps,
+            'state_after_prep_ms_per_step': ms_wait / steps,
             'fused_ms_per_step': ms_fused / steps,
             'roofline': hbm_roofline('kda_decode', bytes_k, ms_k, hbm, peak_kind,
                                      'state 134 MB is just above L2 (126 MB)')}
@@ -717,25 +724,30 @@ def run_verify(torch, kda, synth, dev, rounds=256):
     win4 = win.view(B, Tb + K - 1, H, 3 * d)
     xb = lambda r, key, *tail: X[key][r].view(B, Tb, *tail)
 
+    # verify and the replay stream the state while the kernel before them (kda_prep,
+    # kda_verify_compact; neither writes it) finishes
+    cfg_early = dataclasses.replace(cfg, launch_flags=kda.KDA_LAUNCH_EARLY_STATE)
+
     def one(r, mode):
+        ce = cfg if mode == 'compact_wait' else cfg_early
         if mode == 'fused':
             # one launch for prep + verify (compact tape), then the replay rollback
             kda.kda_layer_verify_compact(cfg, xb(r, 'x', H, 3 * d), xb(r, 'f', H, d),
                                          xb(r, 'beta_logit', H), X['g'][r], P['conv_w'],
                                          P['A_log'], P['dt_bias'], P['norm_w'], state,
                                          conv_state=conv, tape_kua=kua, window=win4, y=y)
-            kda.kda_rollback_replay(cfg, acc[r], kua, state, conv_window=win4, conv_state=conv)
+            kda.kda_rollback_replay(ce, acc[r], kua, state, conv_window=win4, conv_state=conv)
             return
         # prep (conv window for the rollback), verify, rollback to the accepted prefix
         kda.kda_prep(cfg, cu, X['x'][r].view(B * Tb, H, 3 * d), X['f'][r].view(B * Tb, H, d),
                      X['beta_logit'][r].view(B * Tb, H), P['conv_w'], P['A_log'], P['dt_bias'],
                      conv_state=conv, conv_mode=kda.KDA_CONV_TAPE, conv_window=win,
                      max_seqlen=Tb, out=o)
-        if mode == 'compact':
-            kda.kda_verify_compact(cfg, *vargs(r), tape_kua=kua, y=y)
-            kda.kda_rollback_replay(cfg, acc[r], kua, state, conv_window=win, conv_state=conv)
+        if mode in ('compact', 'compact_wait'):
+            kda.kda_verify_compact(ce, *vargs(r), tape_kua=kua, y=y)
+            kda.kda_rollback_replay(ce, acc[r], kua, state, conv_window=win, conv_state=conv)
         else:
-            kda.kda_verify(cfg, *vargs(r), tape=tape, y=y)
+            kda.kda_verify(ce, *vargs(r), tape=tape, y=y)
             kda.kda_rollback(cfg, acc[r], tape, state, conv_window=win, conv_state=conv)
 
     def graph_ms(mode):
@@ -775,6 +787,7 @@ def run_verify(torch, kda, synth, dev, rounds=256):
     # and is the headline: on B200 it is faster than the two-call round with the prep fused
     # (kda_layer_verify_compact), timed beside it with the full-state tape round
     ms = graph_ms('compact')
+    ms_wait = graph_ms('compact_wait')
     ms_fused = graph_ms('fused')
     ms_full = graph_ms('full')
     ms_k = launch_ms(lambda: kda.kda_verify_compact(cfg, *vargs(0), tape_kua=kua, y=y))
@@ -791,8 +804,10 @@ def run_verify(torch, kda, synth, dev, rounds=256):
             'workload': f'verify+rollback B={B} H={H} d={d}, blocks of {Tb} after a {T0}-token '
                         f'context, {rounds} rounds, accepted ~ U{{0..{Tb}}} (CUDA graph; '
                         'kda_prep, kda_verify_compact with the compact (k, u, a) tape, '
-                        'kda_rollback_replay)',
+                        'kda_rollback_replay; verify and replay stream the state while the '
+                        'kernel before them finishes)',
             'ms_per_round': ms / rounds, 'gpu_launches': 3 * rounds,
+            'state_after_previous_ms_per_round': ms_wait / rounds,
             'fused_prep_ms_per_round': ms_fused / rounds,
             'full_state_tape_ms_per_round': ms_full / rounds,
             'roofline': hbm_roofline('kda_verify_compact', bytes_k, ms_k, hbm, peak_kind),

@@ -99,6 +99,22 @@ enum kda_conv_mode {
  */
 enum kda_gate { KDA_GATE_BOUNDED_SIGMOID = 0, KDA_GATE_SOFTPLUS = 1 };
 
+/*
+ * Launch flags (kda_config.launch_flags).  The token-step kernels (kda_decode,
+ * kda_verify, kda_verify_compact, the kda_layer_* step calls) and
+ * kda_rollback_replay are launched as programmatic dependents of the kernel before
+ * them on the stream: they may be scheduled while that kernel finishes, and wait for
+ * it (its completion and its memory) before they read any input.  With
+ * KDA_LAUNCH_EARLY_STATE they instead start streaming the recurrent state (the rows
+ * named by state_slots) BEFORE that wait, overlapping the state read with the tail of
+ * the previous kernel.  Set it only when the kernel issued just before the call on
+ * the same stream writes neither `state` nor `state_slots` (kda_prep, kda_verify_compact
+ * before kda_rollback_replay, the projection GEMM); everything else the call reads is
+ * read after the wait.  Any other bit is KDA_ERR_INVALID_ARG.  Flags are ignored by
+ * entry points that do not take a recurrent state from a previous call.
+ */
+enum kda_launch_flag { KDA_LAUNCH_EARLY_STATE = 1 };
+
 /* Layer configuration (host memory, read during the call only). */
 typedef struct kda_config {
   int32_t num_heads;      /* H >= 1 */
@@ -112,6 +128,7 @@ typedef struct kda_config {
   float norm_eps;         /* output RMSNorm eps, 1e-5 (rms_norm_eps, glm53-flash-mlx README) */
   float q_scale;          /* multiplies o = S^T q; 1.0 */
   int32_t gate_kind;      /* enum kda_gate: which decay-gate function (see below) */
+  int32_t launch_flags;   /* bitwise OR of enum kda_launch_flag (see below); 0 by default */
 } kda_config;
 
 /* Human-readable name of a kda_status code (static string, never NULL). */

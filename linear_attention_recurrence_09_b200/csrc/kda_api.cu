@@ -30,6 +30,7 @@ int check_cfg(const kda_config* c) {
   if (!(c->l2_eps > 0.0f) || !std::isfinite(c->l2_eps)) return KDA_ERR_INVALID_ARG;
   if (!(c->norm_eps >= 0.0f) || !std::isfinite(c->norm_eps)) return KDA_ERR_INVALID_ARG;
   if (!std::isfinite(c->q_scale)) return KDA_ERR_INVALID_ARG;
+  if ((c->launch_flags & ~KDA_LAUNCH_EARLY_STATE) != 0) return KDA_ERR_INVALID_ARG;
   return KDA_OK;
 }
 
@@ -295,6 +296,7 @@ static int step_common(const kda_config* cfg, int32_t batch, int32_t T, const vo
   a.state_in = state_in; a.state_out = state_out; a.tape = tape; a.tape_kua = tape_kua;
   a.slots = slots; a.pool_size = pool_size; a.y = y;
   a.norm_eps = cfg->norm_eps; a.q_scale = cfg->q_scale;
+  a.early_state = (cfg->launch_flags & KDA_LAUNCH_EARLY_STATE) != 0;
   return cuda_status(kda::launch_step(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -325,6 +327,7 @@ static int layer_step_common(const kda_config* cfg, int32_t batch, int32_t T, co
   a.conv_state = conv_state; a.window = window; a.K = cfg->conv_size;
   a.lb = cfg->gate_lower_bound; a.l2_eps = cfg->l2_eps;
   a.gate_softplus = cfg->gate_kind == KDA_GATE_SOFTPLUS;
+  a.early_state = (cfg->launch_flags & KDA_LAUNCH_EARLY_STATE) != 0;
   return cuda_status(kda::launch_step(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -454,6 +457,7 @@ int kda_rollback_replay(const kda_config* cfg, int32_t batch, int32_t block_len,
   a.K = cfg->conv_size; a.bf16 = cfg->dtype == KDA_BF16;
   a.accepted = accepted; a.tape_kua = tape_kua; a.window = conv_window; a.state = state;
   a.conv_state = conv_state; a.slots = state_slots; a.pool_size = pool_size;
+  a.early_state = (cfg->launch_flags & KDA_LAUNCH_EARLY_STATE) != 0;
   return cuda_status(kda::launch_rollback(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 

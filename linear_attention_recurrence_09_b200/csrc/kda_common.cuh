@@ -8,6 +8,33 @@
 namespace kda {
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch (sm_90+): a kernel launched with the programmatic
+// stream-serialization attribute may start before the kernel ahead of it on the
+// stream has finished; grid_dep_wait() blocks until that kernel has completed and its
+// memory is visible (at once when there is none).  grid_dep_trigger() lets the next
+// such kernel be scheduled once every CTA of this grid has issued it or exited.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_trigger() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+// launch `kernel` on `st` as a programmatic dependent of the previous kernel there
+template <typename Args>
+inline cudaError_t launch_dependent(void (*kernel)(Args), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t st, const Args& args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args);
+}
+
+// ---------------------------------------------------------------------------
 // element I/O: activations are fp32 or bf16, arithmetic is fp32
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float ld1(const float* p) { return *p; }

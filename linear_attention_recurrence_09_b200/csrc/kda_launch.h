@@ -62,6 +62,7 @@ struct StepArgs {  // decode (T = 1) and verify (T = block_len)
   int K;
   float lb, l2_eps;
   int gate_softplus;        // as in PrepArgs
+  bool early_state;         // stream the state before waiting for the previous kernel
 };
 
 struct RollbackArgs {
@@ -75,6 +76,7 @@ struct RollbackArgs {
   void* conv_state;
   const int32_t* slots;
   int pool_size;
+  bool early_state;        // replay: as in StepArgs
 };
 
 // Workspace of the chunked prefill (byte offsets from its base, 256-aligned).

@@ -38,6 +38,9 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const PrepArgs a) {
   constexpr int KM1 = K - 1;
   constexpr int KW = KM1 > 0 ? KM1 : 1;
 
+  // a token-step kernel launched next may be scheduled now (it waits for this grid's
+  // completion before reading what it writes)
+  grid_dep_trigger();
   const TileRange tr = slot_to_tile(a.cu, a.n_seqs, a.total, PREP_TILE, blockIdx.x);
   if (tr.len == 0) return;
   const int row = pool_row(a.slots, tr.seq, a.pool_size);

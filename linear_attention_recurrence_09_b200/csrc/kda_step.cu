@@ -27,22 +27,86 @@ namespace kda {
 template <int D>
 struct StepShape {
   static constexpr int CG = D / 4;                                // column groups of 4
-  static constexpr int RG = (256 / CG < D) ? 256 / CG : D;        // row groups
-  static constexpr int ROWS = D / RG;                             // rows per thread
+  static constexpr int RG = (256 / CG < D / 2) ? 256 / CG : D / 2;  // row groups
+  static constexpr int ROWS = D / RG;                             // rows per thread (even)
+  static constexpr int PAIRS = ROWS / 2;                          // row pairs per thread
+  static constexpr int RV = ROWS % 4 == 0 ? 4 : 2;                // rows per staged load
   static constexpr int THREADS = CG * RG;
   static constexpr int NW = (THREADS + 31) / 32;
+  // Row group rg holds the key rows rg, rg + RG, rg + 2 RG, ... (so the CTA's i-th state
+  // load covers RG consecutive rows); the staged per-row vectors (q, k, a) are stored
+  // permuted so that those ROWS rows sit at consecutive positions rg * ROWS + i.
+  static __device__ __forceinline__ int pos(int r) { return (r % RG) * ROWS + r / RG; }
 };
 
 // sigmoid on the special-function unit (approximate exp and reciprocal, relative error
 // ~1e-7); 1 / (1 + inf) = 0 keeps the saturated end exact
 __device__ __forceinline__ float fsig(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
 
-__device__ __forceinline__ float4 f4_scale(float4 a, float s) {
-  return make_float4(a.x * s, a.y * s, a.z * s, a.w * s);
+// A thread's state tile is held as pairs of its rows: S2[p][c] = (S[r][c], S[r'][c]) for
+// r = rg + 2p RG, r' = r + RG and its four columns c.  The per-row factors of a step (a, k,
+// q) then come in pairs straight from a vector load of the (permuted) staged d-vector, and
+// every multiply and
+// fused multiply-add runs on sm_100's paired fp32 instructions: two lanes per
+// instruction, each rounded to nearest like a scalar fmul / fma, so every state element
+// gets the same value bit for bit as with scalar arithmetic.
+template <int PAIRS>
+struct PairTile {
+  float2 v[PAIRS][4];
+};
+
+// The state arrives as plain rows (every load issued before any of them is used), and is
+// regrouped into row pairs once it is needed
+template <int D, int ROWS>
+__device__ __forceinline__ void rows_ld(float4 (&raw)[ROWS], const float* base, int rg, int c0) {
+  constexpr int RG = D / ROWS;
+#pragma unroll
+  for (int i = 0; i < ROWS; ++i) raw[i] = ld4(base + (size_t)(rg + i * RG) * D + c0);
 }
-__device__ __forceinline__ float4 f4_fma(float s, float4 a, float4 acc) {
-  return make_float4(fmaf(s, a.x, acc.x), fmaf(s, a.y, acc.y), fmaf(s, a.z, acc.z),
-                     fmaf(s, a.w, acc.w));
+
+template <int PAIRS>
+__device__ __forceinline__ void tile_from_rows(PairTile<PAIRS>& S, const float4 (&raw)[2 * PAIRS]) {
+#pragma unroll
+  for (int p = 0; p < PAIRS; ++p) {
+    const float4 x = raw[2 * p], y = raw[2 * p + 1];
+    S.v[p][0] = make_float2(x.x, y.x);
+    S.v[p][1] = make_float2(x.y, y.y);
+    S.v[p][2] = make_float2(x.z, y.z);
+    S.v[p][3] = make_float2(x.w, y.w);
+  }
+}
+
+template <int D, int PAIRS>
+__device__ __forceinline__ void tile_st(const PairTile<PAIRS>& S, float* base, int rg, int c0) {
+  constexpr int RG = D / (2 * PAIRS);
+#pragma unroll
+  for (int p = 0; p < PAIRS; ++p) {
+    st4(base + (size_t)(rg + 2 * p * RG) * D + c0,
+        make_float4(S.v[p][0].x, S.v[p][1].x, S.v[p][2].x, S.v[p][3].x));
+    st4(base + (size_t)(rg + (2 * p + 1) * RG) * D + c0,
+        make_float4(S.v[p][0].y, S.v[p][1].y, S.v[p][2].y, S.v[p][3].y));
+  }
+}
+
+// RV consecutive entries of a staged d-vector in shared memory as RV / 2 row pairs
+template <int RV>
+__device__ __forceinline__ void pairs_ld(const float* p, float2 (&v)[RV / 2]) {
+  if constexpr (RV == 4) {
+    const float4 w = *reinterpret_cast<const float4*>(p);
+    v[0] = make_float2(w.x, w.y);
+    v[1] = make_float2(w.z, w.w);
+  } else {
+    v[0] = *reinterpret_cast<const float2*>(p);
+  }
+}
+
+// four columns of a staged d-vector, each duplicated into both lanes of a pair
+__device__ __forceinline__ void cols_dup(const float* p, float2 (&v)[4]) {
+  const float4 w = *reinterpret_cast<const float4*>(p);
+  v[0] = make_float2(w.x, w.x);
+  v[1] = make_float2(w.y, w.y);
+  v[2] = make_float2(w.z, w.z);
+  v[3] = make_float2(w.w, w.w);
 }
 
 // The T tokens' inputs are independent of the state, so they are made ready for every
@@ -54,6 +118,7 @@ template <typename T, int D, bool PREP, int THREADS>
 __device__ __forceinline__ void stage_inputs(const StepArgs& a, int b, int h, int row, float* qs,
                                              float* ks, float* vs, float* as_, float* gs,
                                              float* xwin, float* kq_s, float* beta_s) {
+  using SH = StepShape<D>;
   constexpr int NW = THREADS / 32, C3 = 3 * D;
   const int H = a.H, Tn = a.T, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Km1 = PREP ? a.K - 1 : 0;
@@ -78,8 +143,8 @@ __device__ __forceinline__ void stage_inputs(const StepArgs& a, int b, int h, in
       const int t = e / D, c = e - t * D;
       const size_t idx = (((size_t)b * Tn + t) * H + h) * D + c;
       const float z = ld1(static_cast<const T*>(a.f) + idx) + __ldg(a.dt_bias + (size_t)h * D + c);
-      as_[e] = __expf(a.gate_softplus ? -Ah * softplus(z) : a.lb * fsig(Ah * z));
-      gs[e] = ld1(static_cast<const T*>(a.g) + idx);
+      as_[t * D + SH::pos(c)] = __expf(a.gate_softplus ? -Ah * softplus(z) : a.lb * fsig(Ah * z));
+      gs[e] = sigmoid(ld1(static_cast<const T*>(a.g) + idx));
     }
     for (int t = tid; t < Tn; t += THREADS)
       beta_s[t] = fsig(ld1(static_cast<const T*>(a.beta_logit) + ((size_t)b * Tn + t) * H + h));
@@ -99,7 +164,8 @@ __device__ __forceinline__ void stage_inputs(const StepArgs& a, int b, int h, in
         for (int j = 0; j < 8; ++j) w[j] = (j < a.K) ? __ldg(wp + j) : 0.f;
       }
       const int part = c / D;
-      float* dst = (part == 0 ? qs : part == 1 ? ks : vs) + (c - part * D);
+      const int cc = c - part * D;
+      float* dst = part == 0 ? qs + SH::pos(cc) : part == 1 ? ks + SH::pos(cc) : vs + cc;
       for (int t = 0; t < Tn; ++t) {
         float acc = 0.f;
 #pragma unroll
@@ -123,11 +189,11 @@ __device__ __forceinline__ void stage_inputs(const StepArgs& a, int b, int h, in
     for (int e = tid; e < Tn * D; e += THREADS) {
       const int t = e / D, c = e - t * D;
       const size_t idx = (((size_t)b * Tn + t) * H + h) * D + c;
-      qs[e] = __ldg(a.q + idx);
-      ks[e] = __ldg(a.k + idx);
+      qs[t * D + SH::pos(c)] = __ldg(a.q + idx);
+      ks[t * D + SH::pos(c)] = __ldg(a.k + idx);
       vs[e] = __ldg(a.v + idx);
-      as_[e] = expf(__ldg(a.loga + idx));
-      gs[e] = ld1(static_cast<const T*>(a.g) + idx);
+      as_[t * D + SH::pos(c)] = expf(__ldg(a.loga + idx));
+      gs[e] = sigmoid(ld1(static_cast<const T*>(a.g) + idx));
     }
     for (int t = tid; t < Tn; t += THREADS)
       beta_s[t] = __ldg(a.beta + ((size_t)b * Tn + t) * H + h);
@@ -161,11 +227,11 @@ __device__ __forceinline__ void commit_conv(const StepArgs& a, int h, int row, c
 // One CTA per (head, sequence), any d: the inputs of every step staged first, then the
 // recurrence runs T steps on the state in registers with two block barriers per step.
 template <typename T, int D, bool PREP>
-__global__ void __launch_bounds__(StepShape<D>::THREADS)
+__global__ void __launch_bounds__(StepShape<D>::THREADS, 2)
 step_kernel(const StepArgs a) {
   using SH = StepShape<D>;
-  constexpr int CG = SH::CG, RG = SH::RG, ROWS = SH::ROWS, THREADS = SH::THREADS, NW = SH::NW;
-  constexpr int TMAX = 16;
+  constexpr int CG = SH::CG, RG = SH::RG, ROWS = SH::ROWS, PAIRS = SH::PAIRS, RV = SH::RV;
+  constexpr int THREADS = SH::THREADS, NW = SH::NW, TMAX = 16;
   extern __shared__ __align__(16) float dsm[];
   const int Tn = a.T;
   float* qs = dsm;                    // [T][D] normalised q
@@ -181,34 +247,56 @@ step_kernel(const StepArgs a) {
 
   const int h = blockIdx.x, b = blockIdx.y;
   const int H = a.H;
+  grid_dep_trigger();
+  if (!a.early_state) grid_dep_wait();
   const int row = pool_row(a.slots, b, a.pool_size);
   if (row < 0) return;
   const int tid = threadIdx.x, cg = tid % CG, rg = tid / CG;
   const int lane = tid & 31, warp = tid >> 5;
 
-  // the state streams in first: the inputs below are made ready while it arrives
+  // the state streams in first: the inputs below are made ready while it arrives.  Row
+  // group rg (a warp at d = 128) owns rows rg + i RG, lane cg the four columns from 4 cg:
+  // every state load and store is a whole 512-byte row per warp, and the CTA's i-th load
+  // covers RG consecutive rows.  s0: the first of the thread's staged positions.
+  const int s0 = rg * ROWS, c0 = 4 * cg;
   const float* Sg = a.state_in + ((size_t)row * H + h) * D * D;
-  float4 S[ROWS];
-#pragma unroll
-  for (int i = 0; i < ROWS; ++i) S[i] = ld4(Sg + (size_t)(rg + i * RG) * D + 4 * cg);
-
-  stage_inputs<T, D, PREP, THREADS>(a, b, h, row, qs, ks, vs, as_, gs, xwin, kq_s, beta_s);
+  PairTile<PAIRS> S;
+  {
+    float4 raw[ROWS];
+    rows_ld<D>(raw, Sg, rg, c0);
+    if (a.early_state) grid_dep_wait();    // the other inputs may come from the kernel before
+    stage_inputs<T, D, PREP, THREADS>(a, b, h, row, qs, ks, vs, as_, gs, xwin, kq_s, beta_s);
+    tile_from_rows(S, raw);
+  }
+  const float nw = tid < D ? __ldg(a.norm_w + tid) : 0.f;
   for (int t = 0; t < Tn; ++t) {
     const size_t tok = (size_t)b * Tn + t;
-    const float* kt = ks + t * D;
-    const float* qt = qs + t * D;
-    const float* at = as_ + t * D;
-    // decay along the key axis, then both column reductions in one pass
-    float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+    // decay along the key axis, then both column reductions in one pass; each column's
+    // partial sums run in two lanes (even and odd rows), added at the end
+    float2 pk[4], pq[4];
 #pragma unroll
-    for (int i = 0; i < ROWS; ++i) {
-      const int r = rg + i * RG;
-      S[i] = f4_scale(S[i], at[r]);
-      pk = f4_fma(kt[r], S[i], pk);
-      pq = f4_fma(qt[r], S[i], pq);
+    for (int c = 0; c < 4; ++c) pk[c] = pq[c] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int i0 = 0; i0 < ROWS; i0 += RV) {
+      float2 k2[RV / 2], q2[RV / 2], a2[RV / 2];
+      pairs_ld<RV>(ks + t * D + s0 + i0, k2);
+      pairs_ld<RV>(qs + t * D + s0 + i0, q2);
+      pairs_ld<RV>(as_ + t * D + s0 + i0, a2);
+#pragma unroll
+      for (int j = 0; j < RV / 2; ++j) {
+        const int p = i0 / 2 + j;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          S.v[p][c] = __fmul2_rn(S.v[p][c], a2[j]);
+          pk[c] = __ffma2_rn(k2[j], S.v[p][c], pk[c]);
+          pq[c] = __ffma2_rn(q2[j], S.v[p][c], pq[c]);
+        }
+      }
     }
-    *reinterpret_cast<float4*>(&redk[rg][4 * cg]) = pk;
-    *reinterpret_cast<float4*>(&redq[rg][4 * cg]) = pq;
+    *reinterpret_cast<float4*>(&redk[rg][c0]) =
+        make_float4(pk[0].x + pk[0].y, pk[1].x + pk[1].y, pk[2].x + pk[2].y, pk[3].x + pk[3].y);
+    *reinterpret_cast<float4*>(&redq[rg][c0]) =
+        make_float4(pq[0].x + pq[0].y, pq[1].x + pq[1].y, pq[2].x + pq[2].y, pq[3].x + pq[3].y);
     __syncthreads();                                       // (A) partial reductions
 
     // per value column: u = b (v - S^T k), o = S^T q + u (k.q), RMSNorm partials
@@ -222,9 +310,9 @@ step_kernel(const StepArgs a) {
       us[tid] = u;
       if (a.tape_kua != nullptr) {   // compact tape: this step's k, u and a
         float* tk = a.tape_kua + (tok * H + h) * 3 * D;
-        tk[tid] = kt[tid];
+        tk[tid] = ks[t * D + SH::pos(tid)];
         tk[D + tid] = u;
-        tk[2 * D + tid] = at[tid];
+        tk[2 * D + tid] = as_[t * D + SH::pos(tid)];
       }
     }
     if (warp < (D + 31) / 32) {
@@ -237,33 +325,31 @@ step_kernel(const StepArgs a) {
 
     // rank-1 write and the gated RMSNorm epilogue.  The next step rewrites redk/redq, us
     // and ssq only after its barrier (A), which every thread reaches after these reads.
+    float2 u2[4];
+    cols_dup(&us[c0], u2);
 #pragma unroll
-    for (int i = 0; i < ROWS; ++i) {
-      const int r = rg + i * RG;
-      S[i] = f4_fma(kt[r], *reinterpret_cast<const float4*>(&us[4 * cg]), S[i]);
+    for (int i0 = 0; i0 < ROWS; i0 += RV) {
+      float2 k2[RV / 2];
+      pairs_ld<RV>(ks + t * D + s0 + i0, k2);
+#pragma unroll
+      for (int j = 0; j < RV / 2; ++j)
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          S.v[i0 / 2 + j][c] = __ffma2_rn(k2[j], u2[c], S.v[i0 / 2 + j][c]);
     }
     if (tid < D) {
       float ss = 0.f;
 #pragma unroll
       for (int w = 0; w < (D + 31) / 32; ++w) ss += ssq[w];
       const float rstd = rsqrtf(ss / (float)D + a.norm_eps);
-      st1(static_cast<T*>(a.y) + (tok * H + h) * D + tid,
-          o * rstd * __ldg(a.norm_w + tid) * sigmoid(gs[t * D + tid]));
+      st1(static_cast<T*>(a.y) + (tok * H + h) * D + tid, o * rstd * nw * gs[t * D + tid]);
     }
-    if (a.tape != nullptr) {
-      float* tp = a.tape + (tok * H + h) * D * D;
-#pragma unroll
-      for (int i = 0; i < ROWS; ++i) st4(tp + (size_t)(rg + i * RG) * D + 4 * cg, S[i]);
-    }
+    if (a.tape != nullptr) tile_st<D>(S, a.tape + (tok * H + h) * D * D, rg, c0);
   }
 
   if (PREP && a.conv_state != nullptr && a.window == nullptr)
     commit_conv<T, D, THREADS>(a, h, row, xwin);
-  if (a.state_out != nullptr) {
-    float* So = a.state_out + ((size_t)row * H + h) * D * D;
-#pragma unroll
-    for (int i = 0; i < ROWS; ++i) st4(So + (size_t)(rg + i * RG) * D + 4 * cg, S[i]);
-  }
+  if (a.state_out != nullptr) tile_st<D>(S, a.state_out + ((size_t)row * H + h) * D * D, rg, c0);
 }
 
 template <typename T, bool PREP>
@@ -278,7 +364,8 @@ static cudaError_t launch_step_p(const StepArgs& a, cudaStream_t st) {
     e = cudaFuncSetAttribute(step_kernel<T, DD, PREP>,                                        \
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);         \
     if (e != cudaSuccess) return e;                                                           \
-    step_kernel<T, DD, PREP><<<grid, StepShape<DD>::THREADS, smem, st>>>(a);                  \
+    e = launch_dependent(step_kernel<T, DD, PREP>, grid, dim3(StepShape<DD>::THREADS), smem,  \
+                         st, a);                                                              \
     break;
     KDA_STEP_CASE(16)
     KDA_STEP_CASE(32)
@@ -287,6 +374,7 @@ static cudaError_t launch_step_p(const StepArgs& a, cudaStream_t st) {
 #undef KDA_STEP_CASE
     default: return cudaErrorInvalidValue;
   }
+  if (e != cudaSuccess) return e;
   ++launch_counter();
   return cudaGetLastError();
 }
@@ -336,35 +424,57 @@ __global__ void __launch_bounds__(256) rollback_kernel(const RollbackArgs a) {
 template <typename E, int D>
 __global__ void __launch_bounds__(StepShape<D>::THREADS) rollback_replay_kernel(const RollbackArgs a) {
   using SH = StepShape<D>;
-  constexpr int CG = SH::CG, RG = SH::RG, ROWS = SH::ROWS, THREADS = SH::THREADS;
-  constexpr int TMAX = 16;
+  constexpr int CG = SH::CG, ROWS = SH::ROWS, PAIRS = SH::PAIRS, RV = SH::RV;
+  constexpr int THREADS = SH::THREADS, TMAX = 16;
   __shared__ __align__(16) float kua[TMAX][3][D];
   const int h = blockIdx.x, b = blockIdx.y;
-  const int L = clampi(__ldg(a.accepted + b), 0, a.T);
-  if (L == 0) return;
+  grid_dep_trigger();
+  if (!a.early_state) grid_dep_wait();
   const int row = pool_row(a.slots, b, a.pool_size);
   if (row < 0) return;
   const int H = a.H, tid = threadIdx.x, cg = tid % CG, rg = tid / CG;
+  const int s0 = rg * ROWS, c0 = 4 * cg;
   float* Sg = a.state + ((size_t)row * H + h) * D * D;
-  float4 S[ROWS];
-#pragma unroll
-  for (int i = 0; i < ROWS; ++i) S[i] = ld4(Sg + (size_t)(rg + i * RG) * D + 4 * cg);
-  for (int e = tid; e < L * 3 * D; e += THREADS) {
-    const int j = e / (3 * D), w = e - j * 3 * D;
-    (&kua[j][0][0])[w] = __ldg(a.tape_kua + (((size_t)b * a.T + j) * H + h) * 3 * D + w);
+  int L = 0;
+  PairTile<PAIRS> S;
+  {
+    float4 raw[ROWS];
+    if (a.early_state) {         // the state streams in while the kernel before finishes
+      rows_ld<D>(raw, Sg, rg, c0);
+      grid_dep_wait();
+      L = clampi(__ldg(a.accepted + b), 0, a.T);
+      if (L == 0) return;
+    } else {
+      L = clampi(__ldg(a.accepted + b), 0, a.T);
+      if (L == 0) return;
+      rows_ld<D>(raw, Sg, rg, c0);
+    }
+    for (int e = tid; e < L * 3 * D; e += THREADS) {   // k and a staged permuted
+      const int j = e / (3 * D), w = e - j * 3 * D, part = w / D, c = w - part * D;
+      kua[j][part][part == 1 ? c : SH::pos(c)] =
+          __ldg(a.tape_kua + (((size_t)b * a.T + j) * H + h) * 3 * D + w);
+    }
+    __syncthreads();
+    tile_from_rows(S, raw);
   }
-  __syncthreads();
   for (int j = 0; j < L; ++j) {
-    const float4 u4 = *reinterpret_cast<const float4*>(&kua[j][1][4 * cg]);
+    float2 u2[4];
+    cols_dup(&kua[j][1][c0], u2);
 #pragma unroll
-    for (int i = 0; i < ROWS; ++i) {
-      const int r = rg + i * RG;
-      S[i] = f4_scale(S[i], kua[j][2][r]);
-      S[i] = f4_fma(kua[j][0][r], u4, S[i]);
+    for (int i0 = 0; i0 < ROWS; i0 += RV) {
+      float2 k2[RV / 2], a2[RV / 2];
+      pairs_ld<RV>(&kua[j][0][s0 + i0], k2);
+      pairs_ld<RV>(&kua[j][2][s0 + i0], a2);
+#pragma unroll
+      for (int q = 0; q < RV / 2; ++q)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float2& x = S.v[i0 / 2 + q][c];
+          x = __ffma2_rn(k2[q], u2[c], __fmul2_rn(x, a2[q]));
+        }
     }
   }
-#pragma unroll
-  for (int i = 0; i < ROWS; ++i) st4(Sg + (size_t)(rg + i * RG) * D + 4 * cg, S[i]);
+  tile_st<D>(S, Sg, rg, c0);
   if (a.conv_state != nullptr && a.window != nullptr) {
     const int Km1 = a.K - 1, C3 = 3 * D;
     const E* win = static_cast<const E*>(a.window);
@@ -381,13 +491,17 @@ template <typename E>
 static cudaError_t launch_replay_e(const RollbackArgs& a, cudaStream_t st) {
   dim3 grid(a.H, a.B);
   switch (a.D) {
-    case 16: rollback_replay_kernel<E, 16><<<grid, StepShape<16>::THREADS, 0, st>>>(a); break;
-    case 32: rollback_replay_kernel<E, 32><<<grid, StepShape<32>::THREADS, 0, st>>>(a); break;
-    case 64: rollback_replay_kernel<E, 64><<<grid, StepShape<64>::THREADS, 0, st>>>(a); break;
-    case 128: rollback_replay_kernel<E, 128><<<grid, StepShape<128>::THREADS, 0, st>>>(a); break;
+#define KDA_REPLAY_CASE(DD)                                                                   \
+  case DD:                                                                                    \
+    return launch_dependent(rollback_replay_kernel<E, DD>, grid, dim3(StepShape<DD>::THREADS), \
+                            0, st, a);
+    KDA_REPLAY_CASE(16)
+    KDA_REPLAY_CASE(32)
+    KDA_REPLAY_CASE(64)
+    KDA_REPLAY_CASE(128)
+#undef KDA_REPLAY_CASE
     default: return cudaErrorInvalidValue;
   }
-  return cudaSuccess;
 }
 
 cudaError_t launch_rollback(const RollbackArgs& a, cudaStream_t st) {

@@ -33,6 +33,7 @@ KDA_CONV_COMMIT = 0
 KDA_CONV_TAPE = 1
 KDA_GATE_BOUNDED_SIGMOID = 0
 KDA_GATE_SOFTPLUS = 1
+KDA_LAUNCH_EARLY_STATE = 1
 ABI_VERSION = 2
 
 ENTRY_POINTS = ('kda_status_string', 'kda_abi_version', 'kda_prep',
@@ -58,13 +59,18 @@ class CConfig(ctypes.Structure):
                 ('conv_size', ctypes.c_int32), ('dtype', ctypes.c_int32),
                 ('chunk_size', ctypes.c_int32), ('gate_lower_bound', ctypes.c_float),
                 ('l2_eps', ctypes.c_float), ('norm_eps', ctypes.c_float),
-                ('q_scale', ctypes.c_float), ('gate_kind', ctypes.c_int32)]
+                ('q_scale', ctypes.c_float), ('gate_kind', ctypes.c_int32),
+                ('launch_flags', ctypes.c_int32)]
 
 
 @dataclass
 class Config:
     """Layer configuration; mirrors ``kda_config``.  ``gate_lower_bound=None`` selects
-    the softplus decay gate (KDA_GATE_SOFTPLUS), as an absent lower bound does."""
+    the softplus decay gate (KDA_GATE_SOFTPLUS), as an absent lower bound does.
+    ``launch_flags``: KDA_LAUNCH_EARLY_STATE lets the token-step calls and the replay
+    rollback stream the recurrent state before the kernel ahead of them on the stream
+    has finished; set it only when that kernel writes neither the state nor the slots
+    (kda_prep, or kda_verify_compact before kda_rollback_replay)."""
     num_heads: int
     head_dim: int
     conv_size: int = 4
@@ -74,6 +80,7 @@ class Config:
     l2_eps: float = 1e-6
     norm_eps: float = 1e-5
     q_scale: float = 1.0
+    launch_flags: int = 0
 
     def c(self) -> CConfig:
         if self.dtype not in (torch.float32, torch.bfloat16):
@@ -83,7 +90,8 @@ class Config:
                        KDA_BF16 if self.dtype == torch.bfloat16 else KDA_F32,
                        self.chunk_size, 0.0 if softplus else self.gate_lower_bound,
                        self.l2_eps, self.norm_eps, self.q_scale,
-                       KDA_GATE_SOFTPLUS if softplus else KDA_GATE_BOUNDED_SIGMOID)
+                       KDA_GATE_SOFTPLUS if softplus else KDA_GATE_BOUNDED_SIGMOID,
+                       self.launch_flags)
 
 
 class CProjOut(ctypes.Structure):

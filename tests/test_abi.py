@@ -79,6 +79,12 @@ def test_prep_rejects_bad_arguments(L):
     bad = _cfg()
     bad.gate_kind = 2
     assert _prep(L, bad) == kda.KDA_ERR_INVALID_ARG
+    bad = _cfg()
+    bad.launch_flags = 2                              # only KDA_LAUNCH_EARLY_STATE is defined
+    assert _prep(L, bad) == kda.KDA_ERR_INVALID_ARG
+    ok = _cfg()
+    ok.launch_flags = kda.KDA_LAUNCH_EARLY_STATE
+    assert _prep(L, ok, cu=None) == kda.KDA_ERR_INVALID_ARG   # accepted: on to the pointers
     assert _prep(L, _cfg(conv_size=9)) == kda.KDA_ERR_INVALID_ARG
     assert _prep(L, _cfg(num_heads=0)) == kda.KDA_ERR_INVALID_ARG
     assert _prep(L, _cfg(l2_eps=0.0)) == kda.KDA_ERR_INVALID_ARG

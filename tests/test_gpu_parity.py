@@ -3,6 +3,7 @@
 Bar: max|GPU - oracle| / max|oracle| <= 1e-4 for fp32 inputs and <= 1e-2 for
 bf16 inputs with an fp32 state; rollback and the verify tape are bit-exact.
 """
+import dataclasses
 import math
 
 import numpy as np
@@ -698,3 +699,63 @@ def test_layer_verify_compact_and_replay(dtype):
         ref = oracle_layer(cfg, P, blk, S0[b:b + 1], hist[b:b + 1])
         assert rel_err(np64(s2[b]), ref['state'][0]) <= TOL[dtype], b
         assert np.array_equal(np64(c2[b]), ref['conv_hist'][0]), b
+
+
+# ---------------------------------------------------------------------------
+# KDA_LAUNCH_EARLY_STATE: the step and replay kernels stream the state before the
+# kernel ahead of them on the stream has finished (programmatic dependent launch)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize('dtype,d', [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_early_state_launch_bit_exact(dtype, d):
+    """Decode steps after kda_prep, and verify rounds (kda_prep, kda_verify_compact,
+    kda_rollback_replay), with KDA_LAUNCH_EARLY_STATE, eager and replayed from a CUDA
+    graph, equal the default launches bit for bit (y, state, conv state)."""
+    B, H, Tb, steps, rounds = 5, 4, 8, 6, 3
+    cfg, P, _, S0, hist = make_case(45, [1] * B, H, d, 4, dtype, state_var=0.01,
+                                    conv_hist=True, chunk=16)
+    early = dataclasses.replace(cfg, launch_flags=kda.KDA_LAUNCH_EARLY_STATE)
+    dev = 'cuda'
+    Pd = {k: v.to(dev) for k, v in P.items()}
+    sa = [{k: v.to(dev) for k, v in a.items()} for a in _step_acts(45, B, H, d, dtype, steps)]
+    blocks = [{k: v.to(dev) for k, v in
+               synth.layer_activations(46, [Tb] * B, H, d, dtype, tag=('round', r)).items()}
+              for r in range(rounds)]
+    acc = [torch.tensor([(3 * r + b) % (Tb + 1) for b in range(B)], dtype=torch.int32,
+                        device=dev) for r in range(rounds)]
+
+    def run(c, st, cs):
+        ys = []
+        for a in sa:
+            p = kda.kda_prep(c, a['cu_seqlens'], a['x'], a['f'], a['beta_logit'], Pd['conv_w'],
+                             Pd['A_log'], Pd['dt_bias'], conv_state=cs, max_seqlen=1)
+            ys.append(kda.kda_decode(c, p['q'], p['k'], p['v'], p['log_a'], p['beta'], a['g'],
+                                     Pd['norm_w'], st))
+        shp = lambda t, *tail: t.view(B, Tb, *tail)
+        for r, a in enumerate(blocks):
+            p = kda.kda_prep(c, a['cu_seqlens'], a['x'], a['f'], a['beta_logit'], Pd['conv_w'],
+                             Pd['A_log'], Pd['dt_bias'], conv_state=cs,
+                             conv_mode=kda.KDA_CONV_TAPE, max_seqlen=Tb)
+            y, kua = kda.kda_verify_compact(c, shp(p['q'], H, d), shp(p['k'], H, d),
+                                            shp(p['v'], H, d), shp(p['log_a'], H, d),
+                                            shp(p['beta'], H), shp(a['g'], H, d), Pd['norm_w'],
+                                            st)
+            kda.kda_rollback_replay(c, acc[r], kua, st, conv_window=p['window'], conv_state=cs)
+            ys.append(y.reshape(B * Tb, H, d)[:B])
+        return torch.stack(ys)
+
+    ref_st, ref_cs = S0.to(dev), hist.to(dev)
+    ref_y = run(cfg, ref_st, ref_cs)
+    st, cs = S0.to(dev), hist.to(dev)
+    y = run(early, st, cs)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref_y) and torch.equal(st, ref_st) and torch.equal(cs, ref_cs)
+
+    g_st, g_cs = S0.to(dev), hist.to(dev)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        g_y = run(early, g_st, g_cs)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(g_y, ref_y) and torch.equal(g_st, ref_st) and torch.equal(g_cs, ref_cs)
+    del g
