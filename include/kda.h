@@ -145,10 +145,13 @@ KDA_API int kda_abi_version(void);
  * from the pre-conv hidden states (separate inputs here).
  *
  *  max_seqlen  host hint: an upper bound on every sequence length, or 0 if
- *              unknown.  When 1 <= max_seqlen <= 16 (decode, verify blocks) the
- *              conv-state commit happens inside the main kernel; otherwise a
- *              second small kernel does it.  A wrong non-zero hint leaves the
- *              conv state of longer sequences undefined (never out of bounds).
+ *              unknown.  When 1 <= max_seqlen <= 16 (decode, verify blocks) a
+ *              kernel for short sequences runs (one CTA per sequence and head,
+ *              every input requested at once; still correct for longer
+ *              sequences).  Otherwise the tiled kernel runs; when max_seqlen <= 64
+ *              it commits the conv state itself, else a second small kernel does.
+ *              There, a wrong non-zero hint leaves the conv state of longer
+ *              sequences undefined (never out of bounds).
  *  x           [total_tokens, H, 3d]  pre-conv q|k|v, per head q(d) k(d) v(d)
  *  f           [total_tokens, H, d]   decay-gate input
  *  beta_logit  [total_tokens, H]

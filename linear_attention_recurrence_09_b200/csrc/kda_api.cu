@@ -114,6 +114,8 @@ int kda_prep(const kda_config* cfg, int32_t n_seqs, int32_t total_tokens,
   a.pool_size = conv_state ? pool_size : n_seqs;
   a.mode = conv_mode;
   a.commit_in_kernel = (max_seqlen >= 1 && max_seqlen <= kda::prep_tile()) ? 1 : 0;
+  a.short_tb = max_seqlen < 1 ? 0 : max_seqlen == 1 ? 1 : max_seqlen <= 8 ? 8
+             : max_seqlen <= 16 ? 16 : 0;
   a.window = conv_window;
   a.q = static_cast<float*>(q); a.k = static_cast<float*>(k); a.v = static_cast<float*>(v);
   a.loga = log_a; a.beta = beta;

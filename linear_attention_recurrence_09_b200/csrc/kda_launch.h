@@ -22,6 +22,7 @@ struct PrepArgs {
   int pool_size;
   int mode;  // 0 commit, 1 tape
   int commit_in_kernel;
+  int short_tb;        // > 0: every sequence has at most about this many tokens (1, 8, 16)
   void* window;
   float* q;
   float* k;

@@ -208,6 +208,152 @@ __global__ void conv_commit_kernel(const PrepArgs a) {
   }
 }
 
+// kda_prep for short sequences (decode steps, verify blocks): one CTA of d threads per
+// (sequence, head).  Thread j < 3d/4 owns channels 4j..4j+3 of the head's q|k|v, thread
+// j >= 3d/4 four channels of the decay gate (the first of them also beta).  Every input of
+// the CTA (taps, conv history, x rows, f, beta logit) is requested at once, so a launch
+// costs about two dependent memory round trips; tokens are taken TB at a time, so a
+// sequence longer than the hint is still processed in full.  The conv runs over a register
+// window of the last KM >= K rows with the taps placed by distance from the token (zero
+// past K), accumulated from the token itself backwards.
+template <typename T, int D, int TB, int KM>
+__global__ void __launch_bounds__(D) prep_short_kernel(const PrepArgs a) {
+  constexpr int C3 = 3 * D, G = D / 4;
+  grid_dep_trigger();
+  const int s = blockIdx.x, h = blockIdx.y, H = a.H, K = a.K, Km1 = K - 1;
+  const int j = threadIdx.x, part = j / G;             // 0 q, 1 k, 2 v, 3 gate
+  int start, end;
+  seq_range(a.cu, a.total, s, start, end);
+  const int row = pool_row(a.slots, s, a.pool_size);
+  if (row < 0) return;
+  const int len = end - start;
+  const T* __restrict__ x = static_cast<const T*>(a.x);
+  const T* __restrict__ cs = static_cast<const T*>(a.conv_state);
+  T* wp = static_cast<T*>(a.window);
+  const size_t wbase = (size_t)start + (size_t)s * Km1;   // window row of this sequence's oldest
+
+  if (part < 3) {
+    const int ch = 4 * j;                                  // channel in the head's 3d
+    // taps by distance m from the token: wa[m] = w[K-1-m] for m < K, else 0
+    float wa[KM][4];
+    const float* wr = a.conv_w + ((size_t)h * C3 + ch) * K;
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int m = 0; m < KM; ++m) wa[m][c] = m < K ? __ldg(wr + (size_t)c * K + (K - 1 - m)) : 0.f;
+    // win[m] = the row m back from the next token (m = 1..KM-1); history rows first
+    float win[KM][4];
+#pragma unroll
+    for (int m = 0; m < KM; ++m) {
+      win[m][0] = win[m][1] = win[m][2] = win[m][3] = 0.f;
+      if (m >= 1 && m <= Km1 && cs != nullptr)
+        unpack4(ld4(cs + (((size_t)row * Km1 + (Km1 - m)) * H + h) * C3 + ch), win[m]);
+    }
+    if (a.mode == 1 && wp != nullptr) {
+#pragma unroll
+      for (int m = 1; m < KM; ++m)
+        if (m <= Km1)
+          st4(wp + ((wbase + (Km1 - m)) * H + h) * C3 + ch,
+              make_float4(win[m][0], win[m][1], win[m][2], win[m][3]));
+    }
+    const unsigned gmask =
+        G >= 32 ? 0xffffffffu : (((1u << G) - 1u) << ((j & 31) & ~(G - 1)));
+    float* dst = (part == 0 ? a.q : part == 1 ? a.k : a.v) + (ch - part * D);
+    for (int t0 = 0; t0 < len; t0 += TB) {
+      const int n = min(TB, len - t0);
+      float xin[TB][4];
+#pragma unroll
+      for (int i = 0; i < TB; ++i) {
+        xin[i][0] = xin[i][1] = xin[i][2] = xin[i][3] = 0.f;
+        if (i < n) unpack4(ld4(x + ((size_t)(start + t0 + i) * H + h) * C3 + ch), xin[i]);
+      }
+#pragma unroll
+      for (int i = 0; i < TB; ++i) {
+        if (i >= n) break;                                 // uniform across the CTA
+        const int tok = start + t0 + i;
+        float y[4], ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float acc = fmaf(wa[0][c], xin[i][c], 0.f);
+#pragma unroll
+          for (int m = 1; m < KM; ++m) acc = fmaf(wa[m][c], win[m][c], acc);
+          y[c] = acc * sigmoid(acc);
+          ss = fmaf(y[c], y[c], ss);
+        }
+#pragma unroll
+        for (int off = G / 2; off >= 1; off >>= 1) ss += __shfl_xor_sync(gmask, ss, off);
+        const float sc = (part < 2) ? 1.0f / fmaxf(sqrtf(ss), a.l2_eps) : 1.0f;
+        st4(dst + ((size_t)tok * H + h) * D, make_float4(y[0] * sc, y[1] * sc, y[2] * sc, y[3] * sc));
+        if (a.mode == 1 && wp != nullptr)
+          st4(wp + ((wbase + Km1 + t0 + i) * H + h) * C3 + ch,
+              make_float4(xin[i][0], xin[i][1], xin[i][2], xin[i][3]));
+#pragma unroll
+        for (int m = KM - 1; m >= 2; --m)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) win[m][c] = win[m - 1][c];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) win[1][c] = xin[i][c];
+      }
+    }
+    // commit: the new history is the last K-1 rows of [history; x]
+    if (a.mode == 0 && a.conv_state != nullptr) {
+      T* csw = static_cast<T*>(a.conv_state);
+#pragma unroll
+      for (int m = 1; m < KM; ++m)
+        if (m <= Km1)
+          st4(csw + (((size_t)row * Km1 + (Km1 - m)) * H + h) * C3 + ch,
+              make_float4(win[m][0], win[m][1], win[m][2], win[m][3]));
+    }
+  } else {
+    // decay gate of four channels, and beta, for every token
+    const int c0 = 4 * (j - 3 * G);
+    const T* __restrict__ f = static_cast<const T*>(a.f);
+    const float Ah = expf(__ldg(a.A_log + h));
+    const float4 db = *reinterpret_cast<const float4*>(a.dt_bias + (size_t)h * D + c0);
+    const int sp = a.gate_softplus;
+    for (int t0 = 0; t0 < len; t0 += TB) {
+      const int n = min(TB, len - t0);
+      float4 fv[TB];
+      float bl[TB];
+#pragma unroll
+      for (int i = 0; i < TB; ++i) {
+        if (i < n) {
+          fv[i] = ld4(f + ((size_t)(start + t0 + i) * H + h) * D + c0);
+          if (c0 == 0) bl[i] = ld1(static_cast<const T*>(a.beta_logit) + (size_t)(start + t0 + i) * H + h);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < TB; ++i) {
+        if (i >= n) break;
+        const size_t tok = (size_t)(start + t0 + i);
+        st4(a.loga + (tok * H + h) * D + c0,
+            make_float4(gate_log_decay(Ah, fv[i].x + db.x, a.lb, sp),
+                        gate_log_decay(Ah, fv[i].y + db.y, a.lb, sp),
+                        gate_log_decay(Ah, fv[i].z + db.z, a.lb, sp),
+                        gate_log_decay(Ah, fv[i].w + db.w, a.lb, sp)));
+        if (c0 == 0) a.beta[tok * H + h] = sigmoid(bl[i]);
+      }
+    }
+  }
+}
+
+template <typename T, int D, int KM>
+static cudaError_t launch_prep_short_k(const PrepArgs& a, cudaStream_t st) {
+  const dim3 grid(a.n_seqs, a.H);
+  switch (a.short_tb) {
+    case 1: prep_short_kernel<T, D, 1, KM><<<grid, D, 0, st>>>(a); break;
+    case 8: prep_short_kernel<T, D, 8, KM><<<grid, D, 0, st>>>(a); break;
+    default: prep_short_kernel<T, D, 16, KM><<<grid, D, 0, st>>>(a); break;
+  }
+  ++launch_counter();
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+static cudaError_t launch_prep_short(const PrepArgs& a, cudaStream_t st) {
+  return a.K <= 4 ? launch_prep_short_k<T, D, 4>(a, st) : launch_prep_short_k<T, D, PREP_KMAX>(a, st);
+}
+
 template <typename T, int D, int K>
 static cudaError_t launch_prep_k(const PrepArgs& a, cudaStream_t st) {
   constexpr int HPB = PREP_THREADS / (3 * D / 4);
@@ -226,6 +372,7 @@ static cudaError_t launch_prep_k(const PrepArgs& a, cudaStream_t st) {
 
 template <typename T, int D>
 static cudaError_t launch_prep_t(const PrepArgs& a, cudaStream_t st) {
+  if (a.short_tb > 0) return launch_prep_short<T, D>(a, st);
   switch (a.K) {
     case 1: return launch_prep_k<T, D, 1>(a, st);
     case 2: return launch_prep_k<T, D, 2>(a, st);

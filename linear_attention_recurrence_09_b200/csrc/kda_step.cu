@@ -19,6 +19,8 @@
 // (head, sequence) keeps its whole state in registers (16 float4 per thread
 // at 256 threads) with 16-byte coalesced loads and stores, and the two column
 // reductions go through shared memory across the 8 row groups.
+#include <type_traits>
+
 #include "kda_common.cuh"
 #include "kda_launch.h"
 
@@ -43,49 +45,12 @@ struct StepShape {
 // ~1e-7); 1 / (1 + inf) = 0 keeps the saturated end exact
 __device__ __forceinline__ float fsig(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
 
-// A thread's state tile is held as pairs of its rows: S2[p][c] = (S[r][c], S[r'][c]) for
-// r = rg + 2p RG, r' = r + RG and its four columns c.  The per-row factors of a step (a, k,
-// q) then come in pairs straight from a vector load of the (permuted) staged d-vector, and
-// every multiply and
-// fused multiply-add runs on sm_100's paired fp32 instructions: two lanes per
-// instruction, each rounded to nearest like a scalar fmul / fma, so every state element
-// gets the same value bit for bit as with scalar arithmetic.
-template <int PAIRS>
-struct PairTile {
-  float2 v[PAIRS][4];
-};
-
-// The state arrives as plain rows (every load issued before any of them is used), and is
-// regrouped into row pairs once it is needed
+// The state arrives as plain rows (every load issued before any of them is used)
 template <int D, int ROWS>
 __device__ __forceinline__ void rows_ld(float4 (&raw)[ROWS], const float* base, int rg, int c0) {
   constexpr int RG = D / ROWS;
 #pragma unroll
   for (int i = 0; i < ROWS; ++i) raw[i] = ld4(base + (size_t)(rg + i * RG) * D + c0);
-}
-
-template <int PAIRS>
-__device__ __forceinline__ void tile_from_rows(PairTile<PAIRS>& S, const float4 (&raw)[2 * PAIRS]) {
-#pragma unroll
-  for (int p = 0; p < PAIRS; ++p) {
-    const float4 x = raw[2 * p], y = raw[2 * p + 1];
-    S.v[p][0] = make_float2(x.x, y.x);
-    S.v[p][1] = make_float2(x.y, y.y);
-    S.v[p][2] = make_float2(x.z, y.z);
-    S.v[p][3] = make_float2(x.w, y.w);
-  }
-}
-
-template <int D, int PAIRS>
-__device__ __forceinline__ void tile_st(const PairTile<PAIRS>& S, float* base, int rg, int c0) {
-  constexpr int RG = D / (2 * PAIRS);
-#pragma unroll
-  for (int p = 0; p < PAIRS; ++p) {
-    st4(base + (size_t)(rg + 2 * p * RG) * D + c0,
-        make_float4(S.v[p][0].x, S.v[p][1].x, S.v[p][2].x, S.v[p][3].x));
-    st4(base + (size_t)(rg + (2 * p + 1) * RG) * D + c0,
-        make_float4(S.v[p][0].y, S.v[p][1].y, S.v[p][2].y, S.v[p][3].y));
-  }
 }
 
 // RV consecutive entries of a staged d-vector in shared memory as RV / 2 row pairs
@@ -100,6 +65,14 @@ __device__ __forceinline__ void pairs_ld(const float* p, float2 (&v)[RV / 2]) {
   }
 }
 
+__device__ __forceinline__ float4 f4_scale(float4 a, float s) {
+  return make_float4(a.x * s, a.y * s, a.z * s, a.w * s);
+}
+__device__ __forceinline__ float4 f4_fma(float s, float4 a, float4 acc) {
+  return make_float4(fmaf(s, a.x, acc.x), fmaf(s, a.y, acc.y), fmaf(s, a.z, acc.z),
+                     fmaf(s, a.w, acc.w));
+}
+
 // four columns of a staged d-vector, each duplicated into both lanes of a pair
 __device__ __forceinline__ void cols_dup(const float* p, float2 (&v)[4]) {
   const float4 w = *reinterpret_cast<const float4*>(p);
@@ -108,6 +81,134 @@ __device__ __forceinline__ void cols_dup(const float* p, float2 (&v)[4]) {
   v[2] = make_float2(w.z, w.z);
   v[3] = make_float2(w.w, w.w);
 }
+
+// The two ways a thread holds its state tile, behind one interface.  Both accumulate a
+// column's partial sums S^T k and S^T q in two chains (the thread's even-numbered rows,
+// then its odd-numbered rows, added at the end) and update each element with the same
+// two roundings (S a, then fma(k, u, .)), so the two give the same state and y bit for bit.
+//  * PairedTile: pairs of rows, (S[r][c], S[r + RG][c]), for sm_100's paired fp32 multiply
+//    and fused multiply-add (two lanes per instruction, each rounded to nearest like the
+//    scalar instruction); the per-row factors of a pair come straight from one vector load
+//    of the permuted staged vectors.  Fewest instructions: the verify blocks, whose steps
+//    run back to back on chip.
+//  * RowTile: rows as float4 with scalar arithmetic (fewest registers and moves; decode,
+//    where a CTA runs one step and the state stream dominates).
+template <int D>
+struct PairedTile {
+  using SH = StepShape<D>;
+  static constexpr int ROWS = SH::ROWS, PAIRS = SH::PAIRS, RV = SH::RV, RG = SH::RG;
+  float2 v[PAIRS][4];
+  __device__ __forceinline__ void from_rows(const float4 (&raw)[ROWS]) {
+#pragma unroll
+    for (int p = 0; p < PAIRS; ++p) {
+      const float4 x = raw[2 * p], y = raw[2 * p + 1];
+      v[p][0] = make_float2(x.x, y.x);
+      v[p][1] = make_float2(x.y, y.y);
+      v[p][2] = make_float2(x.z, y.z);
+      v[p][3] = make_float2(x.w, y.w);
+    }
+  }
+  // S <- Diag(a) S on the thread's rows; returns the partial column sums of k^T S, q^T S
+  __device__ __forceinline__ void decay_reduce(const float* k, const float* q, const float* a,
+                                               float4& rk, float4& rq) {
+    float2 pk[4], pq[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) pk[c] = pq[c] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int i0 = 0; i0 < ROWS; i0 += RV) {
+      float2 k2[RV / 2], q2[RV / 2], a2[RV / 2];
+      pairs_ld<RV>(k + i0, k2);
+      pairs_ld<RV>(q + i0, q2);
+      pairs_ld<RV>(a + i0, a2);
+#pragma unroll
+      for (int j = 0; j < RV / 2; ++j)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float2& x = v[i0 / 2 + j][c];
+          x = __fmul2_rn(x, a2[j]);
+          pk[c] = __ffma2_rn(k2[j], x, pk[c]);
+          pq[c] = __ffma2_rn(q2[j], x, pq[c]);
+        }
+    }
+    rk = make_float4(pk[0].x + pk[0].y, pk[1].x + pk[1].y, pk[2].x + pk[2].y, pk[3].x + pk[3].y);
+    rq = make_float4(pq[0].x + pq[0].y, pq[1].x + pq[1].y, pq[2].x + pq[2].y, pq[3].x + pq[3].y);
+  }
+  // S <- S + k u^T on the thread's rows and columns
+  __device__ __forceinline__ void rank1(const float* k, float4 u) {
+    const float2 u2[4] = {make_float2(u.x, u.x), make_float2(u.y, u.y), make_float2(u.z, u.z),
+                          make_float2(u.w, u.w)};
+#pragma unroll
+    for (int i0 = 0; i0 < ROWS; i0 += RV) {
+      float2 k2[RV / 2];
+      pairs_ld<RV>(k + i0, k2);
+#pragma unroll
+      for (int j = 0; j < RV / 2; ++j)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) v[i0 / 2 + j][c] = __ffma2_rn(k2[j], u2[c], v[i0 / 2 + j][c]);
+    }
+  }
+  __device__ __forceinline__ void store(float* base, int rg, int c0) const {
+#pragma unroll
+    for (int p = 0; p < PAIRS; ++p) {
+      st4(base + (size_t)(rg + 2 * p * RG) * D + c0,
+          make_float4(v[p][0].x, v[p][1].x, v[p][2].x, v[p][3].x));
+      st4(base + (size_t)(rg + (2 * p + 1) * RG) * D + c0,
+          make_float4(v[p][0].y, v[p][1].y, v[p][2].y, v[p][3].y));
+    }
+  }
+};
+
+template <int D>
+struct RowTile {
+  using SH = StepShape<D>;
+  static constexpr int ROWS = SH::ROWS, RV = SH::RV, RG = SH::RG;
+  float4 v[ROWS];
+  __device__ __forceinline__ void from_rows(const float4 (&raw)[ROWS]) {
+#pragma unroll
+    for (int i = 0; i < ROWS; ++i) v[i] = raw[i];
+  }
+  __device__ __forceinline__ void decay_reduce(const float* k, const float* q, const float* a,
+                                               float4& rk, float4& rq) {
+    float4 pk[2], pq[2];          // [0]: even-numbered rows, [1]: odd-numbered rows
+    pk[0] = pk[1] = pq[0] = pq[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i0 = 0; i0 < ROWS; i0 += RV) {
+      float2 k2[RV / 2], q2[RV / 2], a2[RV / 2];
+      pairs_ld<RV>(k + i0, k2);
+      pairs_ld<RV>(q + i0, q2);
+      pairs_ld<RV>(a + i0, a2);
+#pragma unroll
+      for (int j = 0; j < RV / 2; ++j) {
+        float4& x = v[i0 + 2 * j];
+        float4& y = v[i0 + 2 * j + 1];
+        x = f4_scale(x, a2[j].x);
+        y = f4_scale(y, a2[j].y);
+        pk[0] = f4_fma(k2[j].x, x, pk[0]);
+        pk[1] = f4_fma(k2[j].y, y, pk[1]);
+        pq[0] = f4_fma(q2[j].x, x, pq[0]);
+        pq[1] = f4_fma(q2[j].y, y, pq[1]);
+      }
+    }
+    rk = make_float4(pk[0].x + pk[1].x, pk[0].y + pk[1].y, pk[0].z + pk[1].z, pk[0].w + pk[1].w);
+    rq = make_float4(pq[0].x + pq[1].x, pq[0].y + pq[1].y, pq[0].z + pq[1].z, pq[0].w + pq[1].w);
+  }
+  __device__ __forceinline__ void rank1(const float* k, float4 u) {
+#pragma unroll
+    for (int i0 = 0; i0 < ROWS; i0 += RV) {
+      float2 k2[RV / 2];
+      pairs_ld<RV>(k + i0, k2);
+#pragma unroll
+      for (int j = 0; j < RV / 2; ++j) {
+        v[i0 + 2 * j] = f4_fma(k2[j].x, u, v[i0 + 2 * j]);
+        v[i0 + 2 * j + 1] = f4_fma(k2[j].y, u, v[i0 + 2 * j + 1]);
+      }
+    }
+  }
+  __device__ __forceinline__ void store(float* base, int rg, int c0) const {
+#pragma unroll
+    for (int i = 0; i < ROWS; ++i) st4(base + (size_t)(rg + i * RG) * D + c0, v[i]);
+  }
+};
 
 // The T tokens' inputs are independent of the state, so they are made ready for every
 // step first, in shared memory: loaded (kda_verify / kda_decode), or with the fused prep
@@ -226,11 +327,12 @@ __device__ __forceinline__ void commit_conv(const StepArgs& a, int h, int row, c
 
 // One CTA per (head, sequence), any d: the inputs of every step staged first, then the
 // recurrence runs T steps on the state in registers with two block barriers per step.
-template <typename T, int D, bool PREP>
+template <typename T, int D, bool PREP, bool PAIRED>
 __global__ void __launch_bounds__(StepShape<D>::THREADS, 2)
 step_kernel(const StepArgs a) {
   using SH = StepShape<D>;
-  constexpr int CG = SH::CG, RG = SH::RG, ROWS = SH::ROWS, PAIRS = SH::PAIRS, RV = SH::RV;
+  using Tile = std::conditional_t<PAIRED, PairedTile<D>, RowTile<D>>;
+  constexpr int CG = SH::CG, RG = SH::RG, ROWS = SH::ROWS;
   constexpr int THREADS = SH::THREADS, NW = SH::NW, TMAX = 16;
   extern __shared__ __align__(16) float dsm[];
   const int Tn = a.T;
@@ -260,43 +362,22 @@ step_kernel(const StepArgs a) {
   // covers RG consecutive rows.  s0: the first of the thread's staged positions.
   const int s0 = rg * ROWS, c0 = 4 * cg;
   const float* Sg = a.state_in + ((size_t)row * H + h) * D * D;
-  PairTile<PAIRS> S;
+  Tile S;
   {
     float4 raw[ROWS];
     rows_ld<D>(raw, Sg, rg, c0);
     if (a.early_state) grid_dep_wait();    // the other inputs may come from the kernel before
     stage_inputs<T, D, PREP, THREADS>(a, b, h, row, qs, ks, vs, as_, gs, xwin, kq_s, beta_s);
-    tile_from_rows(S, raw);
+    S.from_rows(raw);
   }
   const float nw = tid < D ? __ldg(a.norm_w + tid) : 0.f;
   for (int t = 0; t < Tn; ++t) {
     const size_t tok = (size_t)b * Tn + t;
-    // decay along the key axis, then both column reductions in one pass; each column's
-    // partial sums run in two lanes (even and odd rows), added at the end
-    float2 pk[4], pq[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) pk[c] = pq[c] = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int i0 = 0; i0 < ROWS; i0 += RV) {
-      float2 k2[RV / 2], q2[RV / 2], a2[RV / 2];
-      pairs_ld<RV>(ks + t * D + s0 + i0, k2);
-      pairs_ld<RV>(qs + t * D + s0 + i0, q2);
-      pairs_ld<RV>(as_ + t * D + s0 + i0, a2);
-#pragma unroll
-      for (int j = 0; j < RV / 2; ++j) {
-        const int p = i0 / 2 + j;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          S.v[p][c] = __fmul2_rn(S.v[p][c], a2[j]);
-          pk[c] = __ffma2_rn(k2[j], S.v[p][c], pk[c]);
-          pq[c] = __ffma2_rn(q2[j], S.v[p][c], pq[c]);
-        }
-      }
-    }
-    *reinterpret_cast<float4*>(&redk[rg][c0]) =
-        make_float4(pk[0].x + pk[0].y, pk[1].x + pk[1].y, pk[2].x + pk[2].y, pk[3].x + pk[3].y);
-    *reinterpret_cast<float4*>(&redq[rg][c0]) =
-        make_float4(pq[0].x + pq[0].y, pq[1].x + pq[1].y, pq[2].x + pq[2].y, pq[3].x + pq[3].y);
+    // decay along the key axis, then both column reductions in one pass
+    float4 pk, pq;
+    S.decay_reduce(ks + t * D + s0, qs + t * D + s0, as_ + t * D + s0, pk, pq);
+    *reinterpret_cast<float4*>(&redk[rg][c0]) = pk;
+    *reinterpret_cast<float4*>(&redq[rg][c0]) = pq;
     __syncthreads();                                       // (A) partial reductions
 
     // per value column: u = b (v - S^T k), o = S^T q + u (k.q), RMSNorm partials
@@ -325,18 +406,7 @@ step_kernel(const StepArgs a) {
 
     // rank-1 write and the gated RMSNorm epilogue.  The next step rewrites redk/redq, us
     // and ssq only after its barrier (A), which every thread reaches after these reads.
-    float2 u2[4];
-    cols_dup(&us[c0], u2);
-#pragma unroll
-    for (int i0 = 0; i0 < ROWS; i0 += RV) {
-      float2 k2[RV / 2];
-      pairs_ld<RV>(ks + t * D + s0 + i0, k2);
-#pragma unroll
-      for (int j = 0; j < RV / 2; ++j)
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          S.v[i0 / 2 + j][c] = __ffma2_rn(k2[j], u2[c], S.v[i0 / 2 + j][c]);
-    }
+    S.rank1(ks + t * D + s0, *reinterpret_cast<const float4*>(&us[c0]));
     if (tid < D) {
       float ss = 0.f;
 #pragma unroll
@@ -344,15 +414,15 @@ step_kernel(const StepArgs a) {
       const float rstd = rsqrtf(ss / (float)D + a.norm_eps);
       st1(static_cast<T*>(a.y) + (tok * H + h) * D + tid, o * rstd * nw * gs[t * D + tid]);
     }
-    if (a.tape != nullptr) tile_st<D>(S, a.tape + (tok * H + h) * D * D, rg, c0);
+    if (a.tape != nullptr) S.store(a.tape + (tok * H + h) * D * D, rg, c0);
   }
 
   if (PREP && a.conv_state != nullptr && a.window == nullptr)
     commit_conv<T, D, THREADS>(a, h, row, xwin);
-  if (a.state_out != nullptr) tile_st<D>(S, a.state_out + ((size_t)row * H + h) * D * D, rg, c0);
+  if (a.state_out != nullptr) S.store(a.state_out + ((size_t)row * H + h) * D * D, rg, c0);
 }
 
-template <typename T, bool PREP>
+template <typename T, bool PREP, bool PAIRED>
 static cudaError_t launch_step_p(const StepArgs& a, cudaStream_t st) {
   dim3 grid(a.H, a.B);
   const size_t smem =
@@ -361,11 +431,11 @@ static cudaError_t launch_step_p(const StepArgs& a, cudaStream_t st) {
   switch (a.D) {
 #define KDA_STEP_CASE(DD)                                                                     \
   case DD:                                                                                    \
-    e = cudaFuncSetAttribute(step_kernel<T, DD, PREP>,                                        \
+    e = cudaFuncSetAttribute(step_kernel<T, DD, PREP, PAIRED>,                                \
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);         \
     if (e != cudaSuccess) return e;                                                           \
-    e = launch_dependent(step_kernel<T, DD, PREP>, grid, dim3(StepShape<DD>::THREADS), smem,  \
-                         st, a);                                                              \
+    e = launch_dependent(step_kernel<T, DD, PREP, PAIRED>, grid,                              \
+                         dim3(StepShape<DD>::THREADS), smem, st, a);                          \
     break;
     KDA_STEP_CASE(16)
     KDA_STEP_CASE(32)
@@ -382,7 +452,10 @@ static cudaError_t launch_step_p(const StepArgs& a, cudaStream_t st) {
 template <typename T>
 static cudaError_t launch_step_t(const StepArgs& a, cudaStream_t st) {
   if (a.x != nullptr && (a.K < 1 || a.K > 8)) return cudaErrorInvalidValue;
-  return a.x ? launch_step_p<T, true>(a, st) : launch_step_p<T, false>(a, st);
+  // one token (decode): the state tile in rows; a block (verify): in row pairs
+  if (a.T == 1)
+    return a.x ? launch_step_p<T, true, false>(a, st) : launch_step_p<T, false, false>(a, st);
+  return a.x ? launch_step_p<T, true, true>(a, st) : launch_step_p<T, false, true>(a, st);
 }
 
 cudaError_t launch_step(const StepArgs& a, cudaStream_t st) {
@@ -424,7 +497,7 @@ __global__ void __launch_bounds__(256) rollback_kernel(const RollbackArgs a) {
 template <typename E, int D>
 __global__ void __launch_bounds__(StepShape<D>::THREADS) rollback_replay_kernel(const RollbackArgs a) {
   using SH = StepShape<D>;
-  constexpr int CG = SH::CG, ROWS = SH::ROWS, PAIRS = SH::PAIRS, RV = SH::RV;
+  constexpr int CG = SH::CG, ROWS = SH::ROWS, RV = SH::RV;
   constexpr int THREADS = SH::THREADS, TMAX = 16;
   __shared__ __align__(16) float kua[TMAX][3][D];
   const int h = blockIdx.x, b = blockIdx.y;
@@ -436,7 +509,7 @@ __global__ void __launch_bounds__(StepShape<D>::THREADS) rollback_replay_kernel(
   const int s0 = rg * ROWS, c0 = 4 * cg;
   float* Sg = a.state + ((size_t)row * H + h) * D * D;
   int L = 0;
-  PairTile<PAIRS> S;
+  PairedTile<D> S;
   {
     float4 raw[ROWS];
     if (a.early_state) {         // the state streams in while the kernel before finishes
@@ -455,7 +528,7 @@ __global__ void __launch_bounds__(StepShape<D>::THREADS) rollback_replay_kernel(
           __ldg(a.tape_kua + (((size_t)b * a.T + j) * H + h) * 3 * D + w);
     }
     __syncthreads();
-    tile_from_rows(S, raw);
+    S.from_rows(raw);
   }
   for (int j = 0; j < L; ++j) {
     float2 u2[4];
@@ -474,7 +547,7 @@ __global__ void __launch_bounds__(StepShape<D>::THREADS) rollback_replay_kernel(
         }
     }
   }
-  tile_st<D>(S, Sg, rg, c0);
+  S.store(Sg, rg, c0);
   if (a.conv_state != nullptr && a.window != nullptr) {
     const int Km1 = a.K - 1, C3 = 3 * D;
     const E* win = static_cast<const E*>(a.window);
