@@ -159,6 +159,8 @@ PROFILED = {
                    'linear_attention_recurrence_09_b200/csrc/kda_step.cu'),
     'kda_verify_compact': ('profiles/step_verify_compact_b16.md',
                            'linear_attention_recurrence_09_b200/csrc/kda_step.cu'),
+    'prep_short': ('profiles/prep_short_decode_b64.md',
+                   'linear_attention_recurrence_09_b200/csrc/kda_prep.cu'),
 }
 
 
