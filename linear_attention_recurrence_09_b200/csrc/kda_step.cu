@@ -73,15 +73,6 @@ __device__ __forceinline__ float4 f4_fma(float s, float4 a, float4 acc) {
                      fmaf(s, a.w, acc.w));
 }
 
-// four columns of a staged d-vector, each duplicated into both lanes of a pair
-__device__ __forceinline__ void cols_dup(const float* p, float2 (&v)[4]) {
-  const float4 w = *reinterpret_cast<const float4*>(p);
-  v[0] = make_float2(w.x, w.x);
-  v[1] = make_float2(w.y, w.y);
-  v[2] = make_float2(w.z, w.z);
-  v[3] = make_float2(w.w, w.w);
-}
-
 // The two ways a thread holds its state tile, behind one interface.  Both accumulate a
 // column's partial sums S^T k and S^T q in two chains (the thread's even-numbered rows,
 // then its odd-numbered rows, added at the end) and update each element with the same
@@ -490,65 +481,74 @@ __global__ void __launch_bounds__(256) rollback_kernel(const RollbackArgs a) {
 
 // ---------------------------------------------------------------------------
 // rollback by replay: state <- the accepted steps of the compact tape applied to the
-// live state, S <- Diag(a_j) S, then S <- S + k_j u_j^T, element by element exactly as
-// step_kernel does it (same layout, same two operations), so the result equals the
-// full tape's entry bit for bit; conv state as in rollback_kernel
+// live state, S <- Diag(a_j) S, then S <- S + k_j u_j^T, element by element with the
+// step kernel's two roundings (S a, then fma(k, u, .)), so the result equals the full
+// tape's entry bit for bit; conv state as in rollback_kernel.  Every element replays on
+// its own, so a (head, sequence) state is split over CTAs of RPC key rows each, for
+// more loads in flight than one CTA per state gives.
 // ---------------------------------------------------------------------------
+template <int D>
+struct ReplayShape {
+  static constexpr int RPC = D < 32 ? D : 32;                     // key rows per CTA
+  static constexpr int SLICES = D / RPC;
+  static constexpr int CG = D / 4;                                // column groups of 4
+  static constexpr int RG = (256 / CG < RPC) ? 256 / CG : RPC;    // row groups
+  static constexpr int ROWS = RPC / RG;                           // rows per thread
+  static constexpr int THREADS = CG * RG;
+};
+
 template <typename E, int D>
-__global__ void __launch_bounds__(StepShape<D>::THREADS) rollback_replay_kernel(const RollbackArgs a) {
-  using SH = StepShape<D>;
-  constexpr int CG = SH::CG, ROWS = SH::ROWS, RV = SH::RV;
-  constexpr int THREADS = SH::THREADS, TMAX = 16;
-  __shared__ __align__(16) float kua[TMAX][3][D];
-  const int h = blockIdx.x, b = blockIdx.y;
+__global__ void __launch_bounds__(ReplayShape<D>::THREADS) rollback_replay_kernel(const RollbackArgs a) {
+  using RS = ReplayShape<D>;
+  constexpr int CG = RS::CG, RG = RS::RG, ROWS = RS::ROWS, RPC = RS::RPC;
+  constexpr int THREADS = RS::THREADS, TMAX = 16, PER = 2 * RPC + D;
+  __shared__ __align__(16) float ks[TMAX][RPC];
+  __shared__ __align__(16) float as_[TMAX][RPC];
+  __shared__ __align__(16) float us[TMAX][D];
+  const int h = blockIdx.x, b = blockIdx.y, r0 = blockIdx.z * RPC;
   grid_dep_trigger();
   if (!a.early_state) grid_dep_wait();
   const int row = pool_row(a.slots, b, a.pool_size);
   if (row < 0) return;
-  const int H = a.H, tid = threadIdx.x, cg = tid % CG, rg = tid / CG;
-  const int s0 = rg * ROWS, c0 = 4 * cg;
+  const int H = a.H, tid = threadIdx.x, cg = tid % CG, rg = tid / CG, c0 = 4 * cg;
   float* Sg = a.state + ((size_t)row * H + h) * D * D;
-  int L = 0;
-  PairedTile<D> S;
-  {
-    float4 raw[ROWS];
-    if (a.early_state) {         // the state streams in while the kernel before finishes
-      rows_ld<D>(raw, Sg, rg, c0);
-      grid_dep_wait();
-      L = clampi(__ldg(a.accepted + b), 0, a.T);
-      if (L == 0) return;
-    } else {
-      L = clampi(__ldg(a.accepted + b), 0, a.T);
-      if (L == 0) return;
-      rows_ld<D>(raw, Sg, rg, c0);
-    }
-    for (int e = tid; e < L * 3 * D; e += THREADS) {   // k and a staged permuted
-      const int j = e / (3 * D), w = e - j * 3 * D, part = w / D, c = w - part * D;
-      kua[j][part][part == 1 ? c : SH::pos(c)] =
-          __ldg(a.tape_kua + (((size_t)b * a.T + j) * H + h) * 3 * D + w);
-    }
-    __syncthreads();
-    S.from_rows(raw);
+  float4 S[ROWS];                  // key rows r0 + rg + i RG, columns c0..c0+3
+  auto load_state = [&]() {
+#pragma unroll
+    for (int i = 0; i < ROWS; ++i) S[i] = ld4(Sg + (size_t)(r0 + rg + i * RG) * D + c0);
+  };
+  int L;
+  if (a.early_state) {             // the state streams in while the kernel before finishes
+    load_state();
+    grid_dep_wait();
+    L = clampi(__ldg(a.accepted + b), 0, a.T);
+    if (L == 0) return;
+  } else {
+    L = clampi(__ldg(a.accepted + b), 0, a.T);
+    if (L == 0) return;
+    load_state();
   }
+  // this CTA's k and a rows and every u column of the L accepted steps
+  const float* tk = a.tape_kua + ((size_t)b * a.T * H + h) * 3 * D;   // + j H 3d: step j
+  for (int e = tid; e < L * PER; e += THREADS) {
+    const int j = e / PER, w = e - j * PER;
+    const float* src = tk + (size_t)j * H * 3 * D;
+    if (w < RPC) ks[j][w] = __ldg(src + r0 + w);
+    else if (w < RPC + D) us[j][w - RPC] = __ldg(src + D + (w - RPC));
+    else as_[j][w - RPC - D] = __ldg(src + 2 * D + r0 + (w - RPC - D));
+  }
+  __syncthreads();
   for (int j = 0; j < L; ++j) {
-    float2 u2[4];
-    cols_dup(&kua[j][1][c0], u2);
+    const float4 u = *reinterpret_cast<const float4*>(&us[j][c0]);
 #pragma unroll
-    for (int i0 = 0; i0 < ROWS; i0 += RV) {
-      float2 k2[RV / 2], a2[RV / 2];
-      pairs_ld<RV>(&kua[j][0][s0 + i0], k2);
-      pairs_ld<RV>(&kua[j][2][s0 + i0], a2);
-#pragma unroll
-      for (int q = 0; q < RV / 2; ++q)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float2& x = S.v[i0 / 2 + q][c];
-          x = __ffma2_rn(k2[q], u2[c], __fmul2_rn(x, a2[q]));
-        }
+    for (int i = 0; i < ROWS; ++i) {
+      const int r = rg + i * RG;
+      S[i] = f4_fma(ks[j][r], u, f4_scale(S[i], as_[j][r]));
     }
   }
-  S.store(Sg, rg, c0);
-  if (a.conv_state != nullptr && a.window != nullptr) {
+#pragma unroll
+  for (int i = 0; i < ROWS; ++i) st4(Sg + (size_t)(r0 + rg + i * RG) * D + c0, S[i]);
+  if (blockIdx.z == 0 && a.conv_state != nullptr && a.window != nullptr) {
     const int Km1 = a.K - 1, C3 = 3 * D;
     const E* win = static_cast<const E*>(a.window);
     E* cs = static_cast<E*>(a.conv_state);
@@ -562,12 +562,12 @@ __global__ void __launch_bounds__(StepShape<D>::THREADS) rollback_replay_kernel(
 
 template <typename E>
 static cudaError_t launch_replay_e(const RollbackArgs& a, cudaStream_t st) {
-  dim3 grid(a.H, a.B);
   switch (a.D) {
 #define KDA_REPLAY_CASE(DD)                                                                   \
   case DD:                                                                                    \
-    return launch_dependent(rollback_replay_kernel<E, DD>, grid, dim3(StepShape<DD>::THREADS), \
-                            0, st, a);
+    return launch_dependent(rollback_replay_kernel<E, DD>,                                    \
+                            dim3(a.H, a.B, ReplayShape<DD>::SLICES),                          \
+                            dim3(ReplayShape<DD>::THREADS), 0, st, a);
     KDA_REPLAY_CASE(16)
     KDA_REPLAY_CASE(32)
     KDA_REPLAY_CASE(64)
