@@ -237,10 +237,18 @@ __global__ void __launch_bounds__(D) prep_short_kernel(const PrepArgs a) {
     // taps by distance m from the token: wa[m] = w[K-1-m] for m < K, else 0
     float wa[KM][4];
     const float* wr = a.conv_w + ((size_t)h * C3 + ch) * K;
+    if (KM == 4 && K == 4) {                               // one 16-byte load per channel
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 4; ++c) {
+        const float4 w4 = __ldg(reinterpret_cast<const float4*>(wr + 4 * c));
+        wa[0][c] = w4.w; wa[1][c] = w4.z; wa[2][c] = w4.y; wa[3][c] = w4.x;
+      }
+    } else {
 #pragma unroll
-      for (int m = 0; m < KM; ++m) wa[m][c] = m < K ? __ldg(wr + (size_t)c * K + (K - 1 - m)) : 0.f;
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int m = 0; m < KM; ++m) wa[m][c] = m < K ? __ldg(wr + (size_t)c * K + (K - 1 - m)) : 0.f;
+    }
     // win[m] = the row m back from the next token (m = 1..KM-1); history rows first
     float win[KM][4];
 #pragma unroll
@@ -277,7 +285,7 @@ __global__ void __launch_bounds__(D) prep_short_kernel(const PrepArgs a) {
           float acc = fmaf(wa[0][c], xin[i][c], 0.f);
 #pragma unroll
           for (int m = 1; m < KM; ++m) acc = fmaf(wa[m][c], win[m][c], acc);
-          y[c] = acc * sigmoid(acc);
+          y[c] = acc * __fdividef(1.f, 1.f + __expf(-acc));   // SiLU, approximate exp / divide
           ss = fmaf(y[c], y[c], ss);
         }
 #pragma unroll

@@ -759,3 +759,39 @@ def test_early_state_launch_bit_exact(dtype, d):
     torch.cuda.synchronize()
     assert torch.equal(g_y, ref_y) and torch.equal(g_st, ref_st) and torch.equal(g_cs, ref_cs)
     del g
+
+
+# ---------------------------------------------------------------------------
+# kda_prep with max_seqlen <= 16: the kernel for short sequences
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize('dtype', [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize('d,K,hint', [(128, 4, 1), (128, 4, 16), (64, 2, 8), (32, 8, 16),
+                                      (16, 4, 8)])
+def test_prep_short_matches_oracle(dtype, d, K, hint):
+    """The short-sequence prep (one CTA per sequence and head) against the oracle's prep:
+    q, k, v, log a, beta to 1e-5 of max, the committed conv state and the TAPE window bit
+    for bit.  One sequence is longer than the hint (taken in blocks, still exact)."""
+    seqlens = [0, 1, hint, 3, hint + 21]
+    cfg, P, A, _, hist = make_case(47, seqlens, 3, d, K, dtype, conv_hist=True)
+    dev = 'cuda'
+    Pd = {k: v.to(dev) for k, v in P.items()}
+    args = (A['cu_seqlens'].to(dev), A['x'].to(dev), A['f'].to(dev), A['beta_logit'].to(dev),
+            Pd['conv_w'], Pd['A_log'], Pd['dt_bias'])
+    cs = hist.to(dev)
+    p = kda.kda_prep(cfg, *args, conv_state=cs, max_seqlen=hint)
+    cs_t = hist.to(dev)
+    pt = kda.kda_prep(cfg, *args, conv_state=cs_t, conv_mode=kda.KDA_CONV_TAPE,
+                      max_seqlen=hint)
+    torch.cuda.synchronize()
+    ref = oracle_layer(cfg, P, A, None, hist)
+    for name, rname in [('q', 'q'), ('k', 'k'), ('v', 'v'), ('log_a', 'loga'), ('beta', 'beta')]:
+        assert rel_err(np64(p[name]), ref[rname]) <= 1e-5, name
+        assert torch.equal(p[name], pt[name]), name          # TAPE mode: the same outputs
+    assert np.array_equal(np64(cs), ref['conv_hist'])
+    assert torch.equal(cs_t, hist.to(dev))                   # TAPE never writes the state
+    Km1, cu = K - 1, A['cu_seqlens'].tolist()
+    win = pt['window'].cpu()
+    for s, T in enumerate(seqlens):
+        base = cu[s] + s * Km1
+        assert torch.equal(win[base:base + Km1], hist[s])
+        assert torch.equal(win[base + Km1:base + Km1 + T], A['x'][cu[s]:cu[s + 1]])
