@@ -11,7 +11,9 @@
 //   E1     U = U~ - W S  (fp32, rows past the sequence end forced to 0) -> bf16 U^T in smem
 //   MMA2   D2[128 x 32]  = K'^T (128 x 64) . U               (state increment, key rows;
 //                                                               K' stored token-major, read MN-major)
-//   MMA3   D1[64:128]   += M (64 x 64) . U                   (O = Q~ S + M U; A = [0 ; M])
+//   MMA3   D1[64:128]   += M (64 x 64) . U                   (O = Q~ S + M U; A = [X ; M],
+//                                                               X the 8 KB before M: its rows
+//                                                               land in D1[0:64], already read)
 //   E2     S <- Diag(e^{G_C}) S + D2 in fp32 registers (one key row per thread) -> bf16 S^T
 //   E3     O rows of D1 -> y = O / rms(O) * w * sigmoid(g) (FUSE_NORM), else o (fp32,
 //          workspace) for the separate gated RMSNorm pass
@@ -20,12 +22,14 @@
 // columns is assembled from the 4 slices' partials, which each CTA sends into every
 // peer's shared memory with asynchronous remote stores that complete on the peer's
 // mbarrier (a 2-slot ring indexed by chunk parity).
-// Warp roles: warp 0 issues TMA (two smem stages, so chunk n+1 loads while n
-// computes; the U~ slice comes with them), warp 1 allocates TMEM and issues the
-// MMAs from one thread with precomputed descriptors, warps 2-9 run the
-// epilogues, two warps per TMEM lane quarter (quarter = warp % 4), each owning
-// 16 of the 32 value columns.  E1 and E2 are on the serial chain; E3 waits for
-// MMA3 after the state is handed back, off the chain.  Every MMA operand uses the
+// Warp roles: warp 0 issues TMA (three smem stages, so chunks n+1 and n+2 load while n
+// computes: one chunk's tiles take longer than a chunk period to arrive; the U~ slice
+// comes with them), warp 1 allocates TMEM and issues the MMAs from one thread, warps
+// 2-9 run the epilogues, two warps per TMEM lane quarter (quarter = warp % 4), each
+// owning 16 of the 32 value columns.  E1 and E2 are on the serial chain.  With the fused
+// norm, MMA3 of chunk n is issued after MMA1 of chunk n+1, off the chain (U is
+// double-buffered for it); without it, MMA3 follows MMA2 and the epilogue warps of lane
+// quarters 2-3 read O (E3) once it has retired.  Every MMA operand uses the
 // 128-byte swizzle: TMA writes the workspace tiles (K-major; K' read MN-major) and the
 // epilogue threads write S and U MN-major, 16 bytes at a time.
 //
@@ -53,22 +57,25 @@ constexpr uint32_t TMEM_COLS = 128;
 // shared memory carve-up (offsets from a 1024-byte aligned base)
 constexpr uint32_t A1_BYTES = 2 * 128 * 128;     // [W;Q~]: 2 K-blocks x 128 rows x 128 B
 constexpr uint32_t A2_BYTES = 128 * 128;         // K'   : 64 tokens x 128 key channels, read MN-major
-constexpr uint32_t A3_BYTES = 128 * 128;         // [0;M]: 128 rows x 64 (rows 0-63 zero)
+constexpr uint32_t M_BYTES = 64 * 128;           // M: 64 rows x 64 (the lower half of A3)
 constexpr uint32_t UT_BYTES = C * J * 2;         // U~ slice: 64 rows x 32 cols bf16, row-major
-constexpr uint32_t STAGE_BYTES = A1_BYTES + A2_BYTES + A3_BYTES + UT_BYTES;
-constexpr uint32_t NSTAGE = 2;
+constexpr uint32_t STAGE_BYTES = A1_BYTES + A2_BYTES + M_BYTES + UT_BYTES;
+constexpr uint32_t NSTAGE = 3;
 constexpr uint32_t TX_BYTES = 4 * 8192 + 2 * 8192 + 8192 + UT_BYTES;   // W x2, Q~ x2, K' x2, M, U~
 // S (128 key rows) and U (64 token rows) as MN-major B operands: one 128-byte swizzled
 // row per key / token with the slice's 32 value columns in its first 64 bytes (the MMAs
 // have N = 32 and never read the rest), so a thread writes its 16 columns as 2 x 16 bytes
 constexpr uint32_t OFF_S = NSTAGE * STAGE_BYTES;          // S: 128 rows x 128 B
-constexpr uint32_t OFF_U = OFF_S + 128 * 128;             // U:  64 rows x 128 B
-constexpr uint32_t OFF_BAR = OFF_U + 64 * 128;
+constexpr uint32_t OFF_U = OFF_S + 128 * 128;             // U:  2 buffers of 64 rows x 128 B
+constexpr uint32_t U_BYTES = 64 * 128;
+constexpr uint32_t OFF_BAR = OFF_U + 2 * U_BYTES;
 constexpr uint32_t OFF_SSQ = OFF_BAR + 256;   // fused norm: [2 parities][4 slices][64 tokens] fp32
 constexpr uint32_t SMEM_BYTES = OFF_SSQ + 2 * NSLICE * C * 4 + 1024;   // + alignment slack
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of one CTA");
 
 // barrier slots (8 bytes each)
-enum { BAR_FULL0 = 0, BAR_FULL1, BAR_EMPTY0, BAR_EMPTY1, BAR_MMA1, BAR_MMA2, BAR_SREADY,
+enum { BAR_FULL0 = 0, BAR_FULL1, BAR_FULL2, BAR_EMPTY0, BAR_EMPTY1, BAR_EMPTY2, BAR_MMA1,
+       BAR_MMA2, BAR_SREADY,
        BAR_UREADY, BAR_NFULL0, BAR_NFULL1, BAR_OFREE0, BAR_OFREE1, BAR_OFREE2, BAR_ODONE0,
        BAR_ODONE1, BAR_ODONE2, BAR_COUNT };
 static_assert(BAR_COUNT * 8 <= 256, "barrier slots");
@@ -121,10 +128,10 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    mbar_init(bar(BAR_FULL0), 1);
-    mbar_init(bar(BAR_FULL1), 1);
-    mbar_init(bar(BAR_EMPTY0), 1);
-    mbar_init(bar(BAR_EMPTY1), 1);
+    for (int st = 0; st < (int)NSTAGE; ++st) {
+      mbar_init(bar(BAR_FULL0 + st), 1);
+      mbar_init(bar(BAR_EMPTY0 + st), 1);
+    }
     mbar_init(bar(BAR_MMA1), 1);
     mbar_init(bar(BAR_MMA2), 1);
     mbar_init(bar(BAR_SREADY), 32 * NEPI);
@@ -139,12 +146,6 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
     mbar_init(bar(BAR_ODONE2), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // rows 0-63 of every A3 tile are the zero half of [0 ; M]
-  for (uint32_t st = 0; st < NSTAGE; ++st) {
-    uint4* z = reinterpret_cast<uint4*>(sm + st * STAGE_BYTES + A1_BYTES + A2_BYTES);
-    for (int i = threadIdx.x; i < 8192 / 16; i += threads_of<FUSE_NORM>()) z[i] = make_uint4(0, 0, 0, 0);
-  }
-  fence_proxy_async();
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&tmem_holder)),
@@ -170,11 +171,13 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
     if (lane == 0) {
       int issued = 0;
       for (int n = 0; n < nch && !abort_flag; ++n) {
-        const int st = n & 1;
-        if (n >= 2 && !mbar_wait(bar(BAR_EMPTY0 + st), ((n >> 1) - 1) & 1, &abort_flag)) break;
+        const int st = n % NSTAGE;
+        if (n >= (int)NSTAGE &&
+            !mbar_wait(bar(BAR_EMPTY0 + st), ((n / NSTAGE) - 1) & 1, &abort_flag))
+          break;
         const int tile = (start / C + s + n) * H + h;
-        const uint32_t A1 = sbase + st * STAGE_BYTES, A2 = A1 + A1_BYTES, A3 = A2 + A2_BYTES;
-        const uint32_t UTs = A3 + A3_BYTES;
+        const uint32_t A1 = sbase + st * STAGE_BYTES, A2 = A1 + A1_BYTES, Ms = A2 + A2_BYTES;
+        const uint32_t UTs = Ms + M_BYTES;
         mbar_expect_tx(bar(BAR_FULL0 + st), TX_BYTES);
         tma_load_2d(A1, &maps.W, 0, tile * C, bar(BAR_FULL0 + st));
         tma_load_2d(A1 + 16384, &maps.W, 64, tile * C, bar(BAR_FULL0 + st));
@@ -182,14 +185,14 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
         tma_load_2d(A1 + 16384 + 8192, &maps.Q, 64, tile * C, bar(BAR_FULL0 + st));
         tma_load_2d(A2, &maps.KT, 0, tile * C, bar(BAR_FULL0 + st));
         tma_load_2d(A2 + 8192, &maps.KT, 64, tile * C, bar(BAR_FULL0 + st));
-        tma_load_2d(A3 + 8192, &maps.M, 0, tile * C, bar(BAR_FULL0 + st));
+        tma_load_2d(Ms, &maps.M, 0, tile * C, bar(BAR_FULL0 + st));
         tma_load_2d(UTs, &maps.Ut, j0, tile * C, bar(BAR_FULL0 + st));
         issued = n + 1;
       }
       if (abort_flag) {  // let the copies this thread started land before the CTA exits
-        for (int n = (issued >= 2 ? issued - 2 : 0); n < issued; ++n) {
+        for (int n = (issued >= (int)NSTAGE ? issued - (int)NSTAGE : 0); n < issued; ++n) {
           const long long t0 = clock64();
-          while (!mbar_try(bar(BAR_FULL0 + (n & 1)), (n >> 1) & 1) &&
+          while (!mbar_try(bar(BAR_FULL0 + n % NSTAGE), (n / NSTAGE) & 1) &&
                  clock64() - t0 < WAIT_LIMIT_CYCLES) {
           }
         }
@@ -200,12 +203,27 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
     if (lane == 0) {
       const uint32_t id = idesc_bf16(128, J) | (1u << 16);      // B (S or U) MN-major
       const uint32_t id_amn = id | (1u << 15);                   // K' is read MN-major too
-      const uint64_t dA1s0 = sw128_desc(sbase), dA1s1 = sw128_desc(sbase + STAGE_BYTES);
-      const uint32_t sS = sbase + OFF_S, sU = sbase + OFF_U;   // K steps of 16 rows = 2 KB
-      int last = -1;
+      const uint32_t sS = sbase + OFF_S, sU0 = sbase + OFF_U;   // K steps of 16 rows = 2 KB
+      // MMA3 of chunk m: O rows (64-127) of D1 buffer m % 3 += M U.  A is the 64 rows before
+      // M in shared memory, then M: the upper half of the product lands in the W S rows of
+      // that buffer, which E1 has already read and nothing reads again before the buffer's
+      // next MMA1 overwrites them.
+      auto issue_mma3 = [&](int m) {
+        const int stm = m % NSTAGE;
+        const uint64_t a3 = sw128_desc(sbase + stm * STAGE_BYTES + A1_BYTES + A2_BYTES - M_BYTES);
+        const uint32_t uB = sU0 + (m & 1) * U_BYTES;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma(d1_of(m), desc_add(a3, k * 32), sw128_mn_desc(uB + k * 2048, 8192), id, 1);
+        umma_commit(bar(BAR_EMPTY0 + stm));
+        // O of chunk m complete in D1 buffer m % 3 (its own barrier: the O warps may lag
+        // behind the stage barrier by more than one phase, never behind this one)
+        if (FUSE_NORM) umma_commit(bar(BAR_ODONE0 + m % 3));
+      };
+      int committed = 0;   // commits on BAR_MMA1 so far (one per chunk)
       for (int n = 0; n < nch; ++n) {
-        const int st = n & 1;
-        if (!mbar_wait(bar(BAR_FULL0 + st), (n >> 1) & 1, &abort_flag)) break;
+        const int st = n % NSTAGE;
+        if (!mbar_wait(bar(BAR_FULL0 + st), (n / NSTAGE) & 1, &abort_flag)) break;
         if (!mbar_wait(bar(BAR_SREADY), n & 1, &abort_flag)) break;
         const int db = n % 3;
         // fused norm: the O warps have copied chunk n-3's O out of this D1 buffer
@@ -213,34 +231,34 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
             !mbar_wait(bar(BAR_OFREE0 + db), ((n / 3) - 1) & 1, &abort_flag))
           break;
         tc_fence_after();
-        const uint64_t a1 = st ? dA1s1 : dA1s0;
+        const uint64_t a1 = sw128_desc(sbase + st * STAGE_BYTES);
         const uint32_t a2s = sbase + st * STAGE_BYTES + A1_BYTES;
-        const uint64_t a3 = desc_add(a1, A1_BYTES + A2_BYTES);
-        const uint32_t d1 = d1_of(n);
+        const uint32_t d1 = d1_of(n), uB = sU0 + (n & 1) * U_BYTES;
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           umma(d1, desc_add(a1, (k >> 2) * 16384 + (k & 3) * 32),
                sw128_mn_desc(sS + k * 2048, 8192), id, k > 0);
         umma_commit(bar(BAR_MMA1));
-        last = n;
+        ++committed;
+        // fused norm: the previous chunk's output product, off the chain (its U buffer is
+        // rewritten only by chunk n+1's E1, which waits for chunk n+1's MMA1, issued after
+        // this).  Without it, the epilogue warps read O themselves right after E2, so MMA3
+        // follows MMA2 at once (below).
+        if (FUSE_NORM && n > 0) issue_mma3(n - 1);
         if (!mbar_wait(bar(BAR_UREADY), n & 1, &abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          umma(d2_tmem, sw128_mn_desc(a2s + k * 2048, 8192), sw128_mn_desc(sU + k * 2048, 8192),
+          umma(d2_tmem, sw128_mn_desc(a2s + k * 2048, 8192), sw128_mn_desc(uB + k * 2048, 8192),
                id_amn, k > 0);
         umma_commit(bar(BAR_MMA2));
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma(d1, desc_add(a3, k * 32), sw128_mn_desc(sU + k * 2048, 8192), id, 1);
-        umma_commit(bar(BAR_EMPTY0 + st));
-        // O of chunk n complete in D1 buffer n % 3 (its own barrier: the O warps may lag
-        // behind the stage barrier by more than one phase, never behind this one)
-        if (FUSE_NORM) umma_commit(bar(BAR_ODONE0 + db));
+        if (!FUSE_NORM) issue_mma3(n);
       }
-      if (abort_flag && last >= 0) {  // let the issued MMAs retire before TMEM is freed
+      if (FUSE_NORM && !abort_flag && nch > 0) issue_mma3(nch - 1);
+      if (abort_flag) {  // let every issued MMA retire before TMEM is freed
+        umma_commit(bar(BAR_MMA1));
         const long long t0 = clock64();
-        while (!mbar_try(bar(BAR_MMA1), last & 1) && clock64() - t0 < WAIT_LIMIT_CYCLES) {
+        while (!mbar_try(bar(BAR_MMA1), committed & 1) && clock64() - t0 < WAIT_LIMIT_CYCLES) {
         }
       }
     }
@@ -327,7 +345,7 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
     const int cb = JH * half;               // first column of this thread
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     unsigned char* SB = sm + OFF_S;
-    unsigned char* UB = sm + OFF_U;
+    unsigned char* UB0 = sm + OFF_U;
     const float* gCg = reinterpret_cast<const float*>(a.ws + a.L.gC);
     float* og = reinterpret_cast<float*>(a.ws + a.L.o);
     const size_t sg = (((size_t)row * H + h) * D + i) * D + j0 + cb;
@@ -353,7 +371,8 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
     write_state();
 
     for (int n = 0; n < nch; ++n) {
-      const int st = n & 1;
+      const int st = n % NSTAGE;
+      unsigned char* UB = UB0 + (n & 1) * U_BYTES;
       const int tile = (start / C + s + n) * H + h;
       const int t0 = start + n * C;
       const int L = min(C, end - t0);
@@ -366,7 +385,7 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
         tmem_ld16(d1_of(n) + lane_off + cb, ws);
         const __nv_bfloat16* ut =
             reinterpret_cast<const __nv_bfloat16*>(sm + st * STAGE_BYTES + A1_BYTES + A2_BYTES +
-                                                   A3_BYTES) + i * J + cb;
+                                                   M_BYTES) + i * J + cb;
 #pragma unroll
         for (int m = 0; m < JH; m += 8) {   // token row i, columns cb+m..cb+m+7
           const uint4 raw = *reinterpret_cast<const uint4*>(ut + m);
@@ -396,7 +415,7 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
       write_state();
       if (!FUSE_NORM && q >= 2) {
         // E3 (off the chain): O rows (TMEM lanes 64-127) once MMA3 has retired
-        if (!mbar_wait_warp(bar(BAR_EMPTY0 + st), (n >> 1) & 1, &abort_flag)) break;
+        if (!mbar_wait_warp(bar(BAR_EMPTY0 + st), (n / NSTAGE) & 1, &abort_flag)) break;
         tc_fence_after();
         float o[JH];
         tmem_ld16(d1_of(n) + lane_off + cb, o);
