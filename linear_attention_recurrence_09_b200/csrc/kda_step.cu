@@ -489,7 +489,7 @@ __global__ void __launch_bounds__(256) rollback_kernel(const RollbackArgs a) {
 // ---------------------------------------------------------------------------
 template <int D>
 struct ReplayShape {
-  static constexpr int RPC = D < 32 ? D : 32;                     // key rows per CTA
+  static constexpr int RPC = D < 64 ? D : 64;                     // key rows per CTA
   static constexpr int SLICES = D / RPC;
   static constexpr int CG = D / 4;                                // column groups of 4
   static constexpr int RG = (256 / CG < RPC) ? 256 / CG : RPC;    // row groups
