@@ -378,27 +378,59 @@ def run_prefill(args, dist, torch, kda, synth, dev):
     T, H, d = W['T'], W['H'], W['d']
     value = dist.world * T / (ms_step / 1e3)
 
-    # end to end through the same entry points with host buffers (pinned)
+    # end to end through the same entry point with host buffers (pinned).  Steps are
+    # pipelined the way a serving loop runs them: step i+1's inputs are copied in on one
+    # copy stream while step i computes, and step i's y and final state are copied out on
+    # another while step i+1 computes (inputs and outputs double-buffered; the workspace is
+    # shared, the compute being serial).  Every step's own copies are inside the region.
     hx = {k: W['A_cpu'][k].pin_memory() for k in ('x', 'f', 'beta_logit', 'g')}
     hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
     hs = torch.empty(state.shape, dtype=state.dtype).pin_memory()
     n_e2e = max(3, min(20, args.steps))
+    bufs = [{'A': {k: A[k] for k in hx}, 'y': y, 'state': state},
+            {'A': {k: torch.empty_like(A[k]) for k in hx}, 'y': torch.empty_like(y),
+             'state': torch.empty_like(state)}]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    in_done = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
+    for e in in_done + comp_done + out_done:
+        e.record(stream)
 
-    def e2e_step():
-        for k, h in hx.items():
-            A[k].copy_(h, non_blocking=True)
-        step()
-        hy.copy_(y, non_blocking=True)
-        hs.copy_(state, non_blocking=True)
+    def e2e_step(i):
+        b, j = bufs[i & 1], i & 1
+        s_in.wait_event(comp_done[j])        # step i-2 has read this input buffer
+        with torch.cuda.stream(s_in):
+            for k, h in hx.items():
+                b['A'][k].copy_(h, non_blocking=True)
+        in_done[j].record(s_in)
+        stream.wait_event(in_done[j])
+        stream.wait_event(out_done[j])       # step i-2's outputs have left this buffer
+        kda.kda_layer_prefill(cfg, A['cu_seqlens'], b['A']['x'], b['A']['f'],
+                              b['A']['beta_logit'], b['A']['g'], P['conv_w'], P['A_log'],
+                              P['dt_bias'], P['norm_w'], state_out=b['state'], y=b['y'],
+                              workspace=ws, max_seqlen=W['T'], stream=stream)
+        comp_done[j].record(stream)
+        s_out.wait_event(comp_done[j])
+        with torch.cuda.stream(s_out):
+            hy.copy_(b['y'], non_blocking=True)
+            hs.copy_(b['state'], non_blocking=True)
+        out_done[j].record(s_out)
 
-    for _ in range(2):
-        e2e_step()
+    def e2e_run(n):
+        s_in.wait_stream(stream)
+        s_out.wait_stream(stream)
+        for i in range(n):
+            e2e_step(i)
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
+
+    e2e_run(2)
     torch.cuda.synchronize()
     dist.barrier()
     e0, e1 = ev(), ev()
     e0.record(stream)
-    for _ in range(n_e2e):
-        e2e_step()
+    e2e_run(n_e2e)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = dist.max(e0.elapsed_time(e1)) / n_e2e
@@ -419,7 +451,10 @@ def run_prefill(args, dist, torch, kda, synth, dev):
         'config': prefill_config(T, H, d, dist.world),
         'e2e': {'value': dist.world * T / (e2e_ms / 1e3), 'unit': 'tokens/s',
                 'h2d_bytes_per_step': h2d, 'd2h_bytes_per_step': d2h,
-                'ms_per_step': e2e_ms},
+                'ms_per_step': e2e_ms,
+                'pipelining': 'copies in / compute / copies out on three streams, inputs '
+                              'and outputs double-buffered; every step copies its own '
+                              'inputs in and its y and final state out'},
         'gpu_launches': launches,
         # the method's bytes (x, f, g, beta logit in; y, final state out) over the step, i.e.
         # over the one kda_layer_prefill call whose two launches are the dominant work
