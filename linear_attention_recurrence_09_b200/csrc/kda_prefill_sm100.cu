@@ -223,17 +223,18 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
       int committed = 0;   // commits on BAR_MMA1 so far (one per chunk)
       for (int n = 0; n < nch; ++n) {
         const int st = n % NSTAGE;
-        if (!mbar_wait(bar(BAR_FULL0 + st), (n / NSTAGE) & 1, &abort_flag)) break;
-        if (!mbar_wait(bar(BAR_SREADY), n & 1, &abort_flag)) break;
-        const int db = n % 3;
-        // fused norm: the O warps have copied chunk n-3's O out of this D1 buffer
-        if (FUSE_NORM && n >= 3 &&
-            !mbar_wait(bar(BAR_OFREE0 + db), ((n / 3) - 1) & 1, &abort_flag))
-          break;
-        tc_fence_after();
         const uint64_t a1 = sw128_desc(sbase + st * STAGE_BYTES);
         const uint32_t a2s = sbase + st * STAGE_BYTES + A1_BYTES;
         const uint32_t d1 = d1_of(n), uB = sU0 + (n & 1) * U_BYTES;
+        // the waits that are normally long satisfied first, the chain's own (S ready) last:
+        // this chunk's tiles, and (fused norm) the O warps done with chunk n-3's O in this
+        // D1 buffer
+        if (!mbar_wait(bar(BAR_FULL0 + st), (n / NSTAGE) & 1, &abort_flag)) break;
+        if (FUSE_NORM && n >= 3 &&
+            !mbar_wait(bar(BAR_OFREE0 + n % 3), ((n / 3) - 1) & 1, &abort_flag))
+          break;
+        if (!mbar_wait(bar(BAR_SREADY), n & 1, &abort_flag)) break;
+        tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           umma(d1, desc_add(a1, (k >> 2) * 16384 + (k & 3) * 32),
