@@ -379,25 +379,33 @@ interchunk_sm100_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps map
       const int L = min(C, end - t0);
       const float gc = __ldg(gCg + (size_t)tile * D + i);
       if (q < 2) {
-        // E1: U = U~ - W S for token row r = i (0..63), columns cb..cb+15
+        // E1: U = U~ - W S for token row r = i (0..63), columns cb..cb+15.  The U~ row is
+        // read (its stage has landed: this warp waits for it too) before MMA1 is waited for.
+        if (!mbar_wait_warp(bar(BAR_FULL0 + st), (n / NSTAGE) & 1, &abort_flag)) break;
+        const __nv_bfloat16* ut =
+            reinterpret_cast<const __nv_bfloat16*>(sm + st * STAGE_BYTES + A1_BYTES + A2_BYTES +
+                                                   M_BYTES) + i * J + cb;
+        float uf[JH];
+#pragma unroll
+        for (int m = 0; m < JH; m += 8) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(ut + m);
+          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(p2[e]);
+            uf[m + 2 * e] = f.x;
+            uf[m + 2 * e + 1] = f.y;
+          }
+        }
         if (!mbar_wait_warp(bar(BAR_MMA1), n & 1, &abort_flag)) break;
         tc_fence_after();
         float ws[JH];
         tmem_ld16(d1_of(n) + lane_off + cb, ws);
-        const __nv_bfloat16* ut =
-            reinterpret_cast<const __nv_bfloat16*>(sm + st * STAGE_BYTES + A1_BYTES + A2_BYTES +
-                                                   M_BYTES) + i * J + cb;
 #pragma unroll
         for (int m = 0; m < JH; m += 8) {   // token row i, columns cb+m..cb+m+7
-          const uint4 raw = *reinterpret_cast<const uint4*>(ut + m);
-          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
           float u[8];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(p2[e]);
-            u[2 * e] = (i < L) ? f.x - ws[m + 2 * e] : 0.f;
-            u[2 * e + 1] = (i < L) ? f.y - ws[m + 2 * e + 1] : 0.f;
-          }
+          for (int e = 0; e < 8; ++e) u[e] = (i < L) ? uf[m + e] - ws[m + e] : 0.f;
           *reinterpret_cast<uint4*>(UB + mn_row_chunk(i, (cb + m) / 8)) = pack8_bf16(u);
         }
         fence_proxy_async();
