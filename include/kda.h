@@ -127,8 +127,8 @@ typedef struct kda_config {
   float l2_eps;           /* q/k L2 eps, 1e-6 ("a literal 1e-6", PR #27754) */
   float norm_eps;         /* output RMSNorm eps, 1e-5 (rms_norm_eps, glm53-flash-mlx README) */
   float q_scale;          /* multiplies o = S^T q; 1.0 */
-  int32_t gate_kind;      /* enum kda_gate: which decay-gate function (see below) */
-  int32_t launch_flags;   /* bitwise OR of enum kda_launch_flag (see below); 0 by default */
+  int32_t gate_kind;      /* enum kda_gate: which decay-gate function (see above) */
+  int32_t launch_flags;   /* bitwise OR of enum kda_launch_flag (see above); 0 by default */
 } kda_config;
 
 /* Human-readable name of a kda_status code (static string, never NULL). */
