@@ -88,7 +88,7 @@ enum kda_conv_mode {
 /*
  * Decay gate (per key channel, A = exp(A_log[h])).  PR #27754, "Metadata and tensor
  * loading" commit: the bounded-sigmoid branch is selected by the gate_lower_bound key
- * and, when the key is absent, a softplus branch, "a different function":
+ * and, when the key is absent, a softplus branch (a separate function):
  *   KDA_GATE_BOUNDED_SIGMOID  log a = lb * sigmoid(A (f + dt_bias)),  lb in [-5, 0)
  *   KDA_GATE_SOFTPLUS         log a = -A * softplus(f + dt_bias)      (lb ignored)
  * The softplus gate has no lower bound, so a chunk's cumulative decay can span far
@@ -124,7 +124,7 @@ typedef struct kda_config {
   int32_t chunk_size;     /* prefill chunk length in {16, 32, 64} */
   float gate_lower_bound; /* lb of the bounded-sigmoid decay, in [-5, 0) (GLM-5.3-Flash:
                              -5); ignored by the softplus gate */
-  float l2_eps;           /* q/k L2 eps, 1e-6 ("a literal 1e-6", PR #27754) */
+  float l2_eps;           /* q/k L2 eps, 1e-6 (a constant in PR #27754) */
   float norm_eps;         /* output RMSNorm eps, 1e-5 (rms_norm_eps, glm53-flash-mlx README) */
   float q_scale;          /* multiplies o = S^T q; 1.0 */
   int32_t gate_kind;      /* enum kda_gate: which decay-gate function (see above) */
@@ -140,7 +140,7 @@ KDA_API int kda_abi_version(void);
 /*
  * kda_prep - fused short conv + SiLU + q/k L2 norm + decay gate + beta.
  * PR #27754, KDA commit: q|k|v convolved as ONE depthwise kernel, SiLU after
- * the conv, L2 eps a literal 1e-6 with max(sqrt(sum), eps), bounded-sigmoid
+ * the conv, L2 eps exactly 1e-6 with max(sqrt(sum), eps), bounded-sigmoid
  * decay with dt_bias per channel and per-head A broadcast; f and beta come
  * from the pre-conv hidden states (separate inputs here).
  *
@@ -188,7 +188,7 @@ KDA_API size_t kda_prefill_workspace_size(const kda_config* cfg, int32_t n_seqs,
 /*
  * kda_prefill - chunkwise-parallel prefill of packed sequences (chunk length
  * cfg->chunk_size).  llama.cpp PR #27754, KDA commit: prefill on backends without
- * the fused delta-net operator runs the layer as a "chunked fallback" graph; this
+ * the fused delta-net operator runs the layer as a chunked fallback graph; this
  * is that algorithm class, written for sm_100a.  An intra-chunk pass, parallel
  * over (sequence, head, chunk), builds the UT/WY form of each chunk with a
  * triangular solve; a
@@ -242,7 +242,7 @@ KDA_API int kda_layer_prefill(const kda_config* cfg, int32_t n_seqs, int32_t tot
                               kda_stream_t stream);
 
 /*
- * kda_decode - one token for each of `batch` sequences (the "fused operator"
+ * kda_decode - one token for each of `batch` sequences (the fused operator
  * path of PR #27754: no chunking).  Streams each head's d x d fp32 state once:
  * decay, both column reductions S^T k and S^T q in one pass, rank-1 update,
  * one store, gated RMSNorm.

@@ -1,6 +1,6 @@
 // kda_prefill: chunkwise-parallel prefill.
 //
-// Chunkwise form of the KDA recurrence (the "chunked fallback" class of
+// Chunkwise form of the KDA recurrence (the chunked fallback class of
 // llama.cpp PR #27754, written here from the delta-rule UT/WY transform of
 // DeltaNet's chunkwise algorithm with the per-channel decay of gated linear
 // attention).  For a chunk of C tokens starting from state S, with

@@ -2,7 +2,7 @@
 //
 // llama.cpp PR #27754 "model: add GLM-5-Next", KDA commit: q|k|v are convolved as
 // ONE depthwise kernel so the conv state is one contiguous block; SiLU follows
-// the conv; q/k use max(sqrt(sum), eps) with the literal eps 1e-6; the decay is
+// the conv; q/k use max(sqrt(sum), eps) with eps exactly 1e-6; the decay is
 // the bounded sigmoid with dt_bias per channel and per-head A broadcast (or, when the
 // gate has no lower bound, the softplus branch of the "Metadata and tensor loading"
 // commit).

@@ -1,7 +1,7 @@
 // kda_decode / kda_verify / kda_rollback (and kda_layer_decode / kda_layer_verify, which
 // run the prep of each token in the same kernel): the token-at-a-time path.
 //
-// The "fused operator" for the delta net of llama.cpp PR #27754 (backends that
+// The fused delta-net operator of llama.cpp PR #27754 (backends that
 // have it skip the chunked graph for generation): per (sequence, head) the
 // d x d fp32 state is read once, decayed along the key axis, reduced twice in
 // the same pass (S^T k and S^T q), updated by a rank-1 write and stored once.

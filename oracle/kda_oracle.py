@@ -182,7 +182,7 @@ def recurrence(q, k, v, loga, beta, S0=None, q_scale=1.0, return_states=False):
         S <- S + k_t u^T                       (rank-1 write)
         o_t = q_scale * S^T q_t                (read after the write)
     which equals S_t = (I - b k k^T) Diag(a_t) S_{t-1} + b k v^T.  The order
-    decay -> update -> read is the "recurrence ordering" of PR #27754.
+    decay -> update -> read is the ordering PR #27754's KDA commit settles.
 
     q, k: [T, ..., d_k]; v: [T, ..., d_v]; loga: [T, ..., d_k]; beta: [T, ...];
     S0: [..., d_k, d_v] or None (zeros).  Returns (o [T, ..., d_v], S_T) or,
@@ -216,7 +216,8 @@ def recurrence(q, k, v, loga, beta, S0=None, q_scale=1.0, return_states=False):
 def gated_rmsnorm(o, g, w, eps=NORM_EPS):
     """y = o / sqrt(mean(o^2) + eps) * w * sigmoid(g) over the last (d_v) axis.
 
-    PR #27754, KDA commit: gated output RMSNorm with a plain weight;
+    PR #27754, KDA commit: the output goes through an RMSNorm gated by sigmoid(g), with a
+    plain per-channel weight;
     glm53-flash-mlx README: rms_norm_eps = 1e-5.
     """
     o = np.asarray(o, np.float64)

@@ -4,9 +4,9 @@ Each check compares the oracle with something it does not contain: textbook
 constants, hand-derived values (tests/golden/), closed forms, a brute-force
 product of explicit transition matrices, invariants, and NumPy library
 routines.  The mutation controls at the bottom plant a plausible mistake in
-the oracle and require at least one pin to catch it (the negative control of
-the glm53-flash-mlx README's test list: "control: unclamped SwiGLU -> logits
-move").
+the oracle and require at least one pin to catch it (in the manner of the
+negative control in the glm53-flash-mlx README's test list, where a deliberately
+broken activation is shown to move the logits).
 """
 import math
 import os
