@@ -795,3 +795,58 @@ def test_prep_short_matches_oracle(dtype, d, K, hint):
         base = cu[s] + s * Km1
         assert torch.equal(win[base:base + Km1], hist[s])
         assert torch.equal(win[base + Km1:base + Km1 + T], A['x'][cu[s]:cu[s + 1]])
+
+
+def test_pool_slots_short_prep_and_early_state():
+    """Decode and verify rounds through a state pool (slots, including a skipped -1) with
+    the short prep (conv state in the pool too) and KDA_LAUNCH_EARLY_STATE: the mapped
+    rows equal a run on the rows alone, bit for bit, and the other rows are untouched."""
+    B, H, d, Tb, pool = 3, 2, 128, 8, 6
+    cfg, P, _, _, _ = make_case(48, [1] * B, H, d, 4, torch.bfloat16, chunk=16)
+    early = dataclasses.replace(cfg, launch_flags=kda.KDA_LAUNCH_EARLY_STATE)
+    dev = 'cuda'
+    Pd = {k: v.to(dev) for k, v in P.items()}
+    pool_state = synth.initial_state(48, pool, H, d, 0.01).to(dev)
+    pool_conv = synth.conv_history(48, pool, H, d, 4, torch.bfloat16).to(dev)
+    st0, cs0 = pool_state.clone(), pool_conv.clone()
+    slots_l = [4, -1, 1]
+    slots = torch.tensor(slots_l, dtype=torch.int32, device=dev)
+    step = {k: v.to(dev) for k, v in synth.layer_activations(48, [1] * B, H, d, torch.bfloat16,
+                                                              tag='pool_step').items()}
+    blk = {k: v.to(dev) for k, v in synth.layer_activations(48, [Tb] * B, H, d, torch.bfloat16,
+                                                             tag='pool_blk').items()}
+    acc = torch.tensor([5, 0, 8], dtype=torch.int32, device=dev)
+
+    def run(c, st, cs, sl, a_step, a_blk, acc_):
+        p = kda.kda_prep(c, a_step['cu_seqlens'], a_step['x'], a_step['f'], a_step['beta_logit'],
+                         Pd['conv_w'], Pd['A_log'], Pd['dt_bias'], conv_state=cs, state_slots=sl,
+                         max_seqlen=1)
+        y = kda.kda_decode(c, p['q'], p['k'], p['v'], p['log_a'], p['beta'], a_step['g'],
+                           Pd['norm_w'], st, state_slots=sl)
+        nb = a_step['x'].shape[0]
+        shp = lambda t, *tail: t.view(nb, Tb, *tail)
+        p = kda.kda_prep(c, a_blk['cu_seqlens'], a_blk['x'], a_blk['f'], a_blk['beta_logit'],
+                         Pd['conv_w'], Pd['A_log'], Pd['dt_bias'], conv_state=cs, state_slots=sl,
+                         conv_mode=kda.KDA_CONV_TAPE, max_seqlen=Tb)
+        yv, kua = kda.kda_verify_compact(c, shp(p['q'], H, d), shp(p['k'], H, d),
+                                         shp(p['v'], H, d), shp(p['log_a'], H, d),
+                                         shp(p['beta'], H), shp(a_blk['g'], H, d), Pd['norm_w'],
+                                         st, state_slots=sl)
+        kda.kda_rollback_replay(c, acc_, kua, st, conv_window=p['window'], conv_state=cs,
+                                state_slots=sl)
+        return y, yv
+
+    y, yv = run(early, pool_state, pool_conv, slots, step, blk, acc)
+    torch.cuda.synchronize()
+    for r in (0, 2, 3, 5):
+        assert torch.equal(pool_state[r], st0[r]) and torch.equal(pool_conv[r], cs0[r]), r
+    for b, r in enumerate(slots_l):
+        if r < 0:
+            continue
+        st, cs = st0[r:r + 1].clone(), cs0[r:r + 1].clone()
+        one = lambda a, T: {'cu_seqlens': torch.tensor([0, T], dtype=torch.int32, device=dev),
+                            **{k: a[k][b * T:(b + 1) * T].clone() for k in ('x', 'f', 'beta_logit', 'g')}}
+        y1, yv1 = run(cfg, st, cs, None, one(step, 1), one(blk, Tb), acc[b:b + 1].clone())
+        torch.cuda.synchronize()
+        assert torch.equal(st[0], pool_state[r]) and torch.equal(cs[0], pool_conv[r]), b
+        assert torch.equal(y1[0], y[b]) and torch.equal(yv1[0], yv[b]), b
