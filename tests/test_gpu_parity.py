@@ -765,14 +765,18 @@ def test_early_state_launch_bit_exact(dtype, d):
 # kda_prep with max_seqlen <= 16: the kernel for short sequences
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize('dtype', [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize('d,K,hint', [(128, 4, 1), (128, 4, 16), (64, 2, 8), (32, 8, 16),
-                                      (16, 4, 8)])
-def test_prep_short_matches_oracle(dtype, d, K, hint):
+@pytest.mark.parametrize('d,K,hint,softplus', [(128, 4, 1, False), (128, 4, 16, False),
+                                               (64, 2, 8, False), (32, 8, 16, False),
+                                               (16, 4, 8, False), (128, 4, 8, True)])
+def test_prep_short_matches_oracle(dtype, d, K, hint, softplus):
     """The short-sequence prep (one CTA per sequence and head) against the oracle's prep:
     q, k, v, log a, beta to 1e-5 of max, the committed conv state and the TAPE window bit
-    for bit.  One sequence is longer than the hint (taken in blocks, still exact)."""
+    for bit.  One sequence is longer than the hint (taken in blocks, still exact); one case
+    takes the softplus gate."""
     seqlens = [0, 1, hint, 3, hint + 21]
     cfg, P, A, _, hist = make_case(47, seqlens, 3, d, K, dtype, conv_hist=True)
+    if softplus:
+        cfg = dataclasses.replace(cfg, gate_lower_bound=None)
     dev = 'cuda'
     Pd = {k: v.to(dev) for k, v in P.items()}
     args = (A['cu_seqlens'].to(dev), A['x'].to(dev), A['f'].to(dev), A['beta_logit'].to(dev),
