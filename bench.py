@@ -149,6 +149,9 @@ def measured_peaks():
 # capture time, and the sha256 of its code (comments and blank lines removed), and counts
 # only while that code is unchanged.
 PROFILED = {
+    'prefill_cosched': ('profiles/prefill_cosched_sm100_8k.md',
+                        ('linear_attention_recurrence_09_b200/csrc/kda_intra_sm100.cu',
+                         'linear_attention_recurrence_09_b200/csrc/kda_chain_sm100.cuh')),
     'intra_chunk': ('profiles/intra_chunk_sm100_prefill_8k.md',
                     'linear_attention_recurrence_09_b200/csrc/kda_intra_sm100.cu'),
     'inter_chunk': ('profiles/interchunk_sm100_prefill_8k.md',
@@ -190,16 +193,24 @@ def code_text(src):
 
 
 def code_sha256(path):
+    """sha256 of the code of one source file, or of several joined by newlines."""
     import hashlib
-    with open(path, encoding='utf-8') as fh:
-        return hashlib.sha256(code_text(fh.read()).encode()).hexdigest()
+    paths = [path] if isinstance(path, str) else list(path)
+    texts = []
+    for p in paths:
+        with open(p, encoding='utf-8') as fh:
+            texts.append(code_text(fh.read()))
+    return hashlib.sha256('\n'.join(texts).encode()).hexdigest()
 
 
 def profiled_traffic(kernel):
     import re
     if kernel not in PROFILED:
         return None
-    summary, source = (os.path.join(ROOT, f) for f in PROFILED[kernel])
+    summary, source = PROFILED[kernel]
+    summary = os.path.join(ROOT, summary)
+    source = (os.path.join(ROOT, source) if isinstance(source, str)
+              else [os.path.join(ROOT, f) for f in source])
     try:
         text = open(summary).read()
         digest = code_sha256(source)
@@ -254,7 +265,8 @@ def prefill_bytes(T, H, d, C=64, K=4, fused_norm=True):
     layer = th * (3 * d * 2 + d * 2 + 2 + d * 2 + d * 2) + H * d * d * 4
     if fused_norm:
         inter = tiles + th * d * 2 + d * 4 + th * d * 2 + H * d * d * 4   # + g, norm_w in; y out
-        return {'intra_chunk': intra, 'inter_chunk': inter, 'layer': layer}
+        return {'intra_chunk': intra, 'inter_chunk': inter, 'layer': layer,
+                'prefill_cosched': intra + inter}
     inter = tiles + th * d * 4 + H * d * d * 4                  # tiles in, o and state out
     norm = th * d * 4 + th * d * 2 + d * 4 + th * d * 2         # o, g, norm_w in; y out
     return {'intra_chunk': intra, 'inter_chunk': inter, 'gated_norm': norm, 'layer': layer}
@@ -295,7 +307,8 @@ def prefill_mma_flops(T, H, d, C=64):
     intra_bf16 = tiles * 5 * 2 * d * C * C
     inter_bf16 = tiles * (2 * (2 * C) * d * d + 2 * d * d * C + 2 * (2 * C) * d * C)
     return {'intra_chunk': {'tf32': intra_tf32, 'bf16': intra_bf16},
-            'inter_chunk': {'tf32': 0, 'bf16': inter_bf16}}
+            'inter_chunk': {'tf32': 0, 'bf16': inter_bf16},
+            'prefill_cosched': {'tf32': intra_tf32, 'bf16': intra_bf16 + inter_bf16}}
 
 
 def issued_mma_view(flops, ms_phase, bf16_tflops):
@@ -332,12 +345,16 @@ def run_prefill(args, dist, torch, kda, synth, dev):
         e.record(stream)            # torch creates the CUDA event on first record
         return e
 
-    def step(e=None):
-        # one pass of the layer: fused prep + intra-chunk, inter-chunk, gated norm
+    # beside the headline: the same layer with the two passes as separate launches
+    cfg_sep = dataclasses.replace(cfg, launch_flags=kda.KDA_LAUNCH_SEPARATE_PASSES)
+
+    def step(e=None, c=cfg):
+        # one pass of the layer: fused prep + intra-chunk, inter-chunk, gated norm (one
+        # co-scheduled launch, or separate launches)
         if e:
             e[0].record(stream)
             kda.kda_set_phase_events(e[1:])
-        kda.kda_layer_prefill(cfg, A['cu_seqlens'], A['x'], A['f'], A['beta_logit'], A['g'],
+        kda.kda_layer_prefill(c, A['cu_seqlens'], A['x'], A['f'], A['beta_logit'], A['g'],
                               P['conv_w'], P['A_log'], P['dt_bias'], P['norm_w'],
                               state_out=state, y=y, workspace=ws, max_seqlen=W['T'])
         if e:
@@ -366,13 +383,27 @@ def run_prefill(args, dist, torch, kda, synth, dev):
         step()
         torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
-    fused_norm = launches == 2 * args.steps      # intra + inter (norm inside the inter pass)
-    phases = PHASES[:2] if fused_norm else PHASES
+    one_launch = launches == args.steps          # both passes (and the norm) co-scheduled
+    fused_norm = one_launch or launches == 2 * args.steps   # norm inside the inter pass
+    phases = (('prefill_cosched',) if one_launch else PHASES[:2] if fused_norm else PHASES)
     # per-step statistic: the median of the K per-step event durations (the timed region's
     # mean is kept beside it); per pass likewise
-    step_ms = [p[0].elapsed_time(p[len(phases)]) for p in per]
+    step_ms = [p[0].elapsed_time(p[3]) for p in per]
     ms_phase = {ph: statistics.median(p[i].elapsed_time(p[i + 1]) for p in per)
                 for i, ph in enumerate(phases)}
+    # the separate launches, timed the same way (untimed warm-up first)
+    for _ in range(args.warmup):
+        step(c=cfg_sep)
+    per_sep = [[ev() for _ in range(4)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        step(per_sep[i], c=cfg_sep)
+    torch.cuda.synchronize()
+    separate = {'ms_per_step': dist.max(statistics.median(p[0].elapsed_time(p[3])
+                                                          for p in per_sep)),
+                'breakdown_ms': {ph: statistics.median(p[i].elapsed_time(p[i + 1])
+                                                       for p in per_sep)
+                                 for i, ph in enumerate(PHASES[:2])},
+                'launches_per_step': 2}
     ms_step = dist.max(statistics.median(step_ms))
     ms_mean = dist.max(ms) / args.steps
     T, H, d = W['T'], W['H'], W['d']
@@ -458,14 +489,17 @@ def run_prefill(args, dist, torch, kda, synth, dev):
         'gpu_launches': launches,
         # the method's bytes (x, f, g, beta logit in; y, final state out) over the step, i.e.
         # over the one kda_layer_prefill call whose two launches are the dominant work
-        'roofline': {'bound': 'hbm', 'kernel': 'kda_layer_prefill (intra-chunk + inter-chunk '
-                     'launches)', 'achieved': achieved, 'peak': hbm, 'unit': 'GB/s',
+        'roofline': {'bound': 'hbm', 'kernel': ('kda_layer_prefill (one co-scheduled launch: '
+                     'the intra-chunk pass beside the inter-chunk chains)' if one_launch else
+                     'kda_layer_prefill (intra-chunk + inter-chunk launches)'),
+                     'achieved': achieved, 'peak': hbm, 'unit': 'GB/s',
                      'frac': achieved / hbm,
                      'traffic': (sum(pass_traffic) if all(t is not None for t in pass_traffic)
                                  else None),
                      'peak_kind': peak_kind, 'algorithmic_bytes_per_launch': method,
                      'per_unit': '1,538 B per (token, head) + 64 KB state per head'},
         'breakdown_ms': ms_phase,
+        'separate_passes': separate,
         # bytes this design moves per pass (incl. the chunk tiles handed from pass 1 to pass
         # 2, which the method itself does not need), with ncu DRAM traffic where profiled
         'design_traffic': {ph: {'bytes': nb[ph],
@@ -582,11 +616,11 @@ def run_long(torch, kda, synth, dev, steps=5, warmup=3):
 
         evs = [[ev() for _ in range(4)] for _ in range(steps)]
 
-        def step(e=None):
+        def step(e=None, c=cfg):
             if e:
                 e[0].record(stream)
                 kda.kda_set_phase_events(e[1:])
-            kda.kda_layer_prefill(cfg, cu, x, f, bl, g, P['conv_w'], P['A_log'], P['dt_bias'],
+            kda.kda_layer_prefill(c, cu, x, f, bl, g, P['conv_w'], P['A_log'], P['dt_bias'],
                                   P['norm_w'], state_in=s0, state_out=state, y=y, workspace=ws,
                                   max_seqlen=max(lens))
             if e:
@@ -601,21 +635,42 @@ def run_long(torch, kda, synth, dev, steps=5, warmup=3):
         launches = (kda.kda_launch_count() - n0) // steps
         torch.cuda.synchronize()
         ms = statistics.median(e[0].elapsed_time(e[3]) for e in evs)
-        ms_inter = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
         method = layer_method_bytes(T, N, H, d)
         ach = method / (ms / 1e3) / 1e9
+
+        def breakdown(ev_list, n_launch):
+            if n_launch == 1:
+                return {'prefill_cosched': statistics.median(e[0].elapsed_time(e[1])
+                                                             for e in ev_list)}
+            return {'intra_chunk': statistics.median(e[0].elapsed_time(e[1]) for e in ev_list),
+                    'inter_chunk': statistics.median(e[1].elapsed_time(e[2]) for e in ev_list)}
+
         rec = {'value': T / (ms / 1e3), 'unit': 'tokens/s', 'tokens': T, 'n_seqs': N,
                'max_seqlen': max(lens), 'ms_per_step': ms,
-               'breakdown_ms': {'intra_chunk': statistics.median(e[0].elapsed_time(e[1])
-                                                                  for e in evs),
-                                'inter_chunk': ms_inter},
+               'breakdown_ms': breakdown(evs, launches),
                'launches_per_step': launches,
                'roofline': {'bound': 'hbm', 'achieved': ach, 'peak': hbm, 'unit': 'GB/s',
                             'frac': ach / hbm, 'peak_kind': peak_kind,
                             'algorithmic_bytes_per_launch': method}}
-        if N == 1:
-            # one wave of 128 chain CTAs: the inter-chunk pass time over the serial chunks
-            rec['chain_us_per_chunk'] = ms_inter * 1e3 / (-(-T // 64))
+        if launches == 1:
+            # beside it: the two passes as separate launches, whose inter-chunk pass gives
+            # the chain period (one wave of 128 four-slice chain CTAs)
+            c_sep = dataclasses.replace(cfg, launch_flags=kda.KDA_LAUNCH_SEPARATE_PASSES)
+            for _ in range(warmup):
+                step(c=c_sep)
+            evs2 = [[ev() for _ in range(4)] for _ in range(steps)]
+            for i in range(steps):
+                step(evs2[i], c=c_sep)
+            torch.cuda.synchronize()
+            bd = breakdown(evs2, 2)
+            rec['separate_passes'] = {
+                'ms_per_step': statistics.median(e[0].elapsed_time(e[3]) for e in evs2),
+                'breakdown_ms': bd,
+                'chain_us_per_chunk': bd['inter_chunk'] * 1e3 / (-(-T // 64))}
+            # the co-scheduled chains run one CTA per head, all value columns; the step is
+            # bound by the intra-chunk pass on the remaining SMs, not by the chain
+        elif N == 1:
+            rec['chain_us_per_chunk'] = rec['breakdown_ms']['inter_chunk'] * 1e3 / (-(-T // 64))
         out[name] = rec
         del x, f, bl, g, y, ws, state, s0
         torch.cuda.empty_cache()

@@ -30,7 +30,8 @@ int check_cfg(const kda_config* c) {
   if (!(c->l2_eps > 0.0f) || !std::isfinite(c->l2_eps)) return KDA_ERR_INVALID_ARG;
   if (!(c->norm_eps >= 0.0f) || !std::isfinite(c->norm_eps)) return KDA_ERR_INVALID_ARG;
   if (!std::isfinite(c->q_scale)) return KDA_ERR_INVALID_ARG;
-  if ((c->launch_flags & ~KDA_LAUNCH_EARLY_STATE) != 0) return KDA_ERR_INVALID_ARG;
+  if ((c->launch_flags & ~(KDA_LAUNCH_EARLY_STATE | KDA_LAUNCH_SEPARATE_PASSES)) != 0)
+    return KDA_ERR_INVALID_ARG;
   return KDA_OK;
 }
 
@@ -166,8 +167,9 @@ int kda_prefill(const kda_config* cfg, int32_t n_seqs, int32_t total_tokens,
   a.y = y; a.ws = static_cast<char*>(workspace); a.L = L;
   a.norm_eps = cfg->norm_eps; a.q_scale = cfg->q_scale; a.lb = cfg->gate_lower_bound;
   a.gate_softplus = cfg->gate_kind == KDA_GATE_SOFTPLUS;
+  a.separate_passes = (cfg->launch_flags & KDA_LAUNCH_SEPARATE_PASSES) != 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(a.ws + L.status, 0, 256, s) != cudaSuccess) return KDA_ERR_CUDA;
+  if (cudaMemsetAsync(a.ws + L.status, 0, L.zeroed - L.status, s) != cudaSuccess) return KDA_ERR_CUDA;
   return cuda_status(kda::launch_prefill(a, s));
 }
 
@@ -243,7 +245,8 @@ int kda_layer_prefill(const kda_config* cfg, int32_t n_seqs, int32_t total_token
   a.norm_eps = cfg->norm_eps; a.q_scale = cfg->q_scale; a.lb = cfg->gate_lower_bound;
   a.l2_eps = cfg->l2_eps; a.K = cfg->conv_size;
   a.gate_softplus = cfg->gate_kind == KDA_GATE_SOFTPLUS;
-  if (cudaMemsetAsync(a.ws + L.status, 0, 256, s) != cudaSuccess) return KDA_ERR_CUDA;
+  a.separate_passes = (cfg->launch_flags & KDA_LAUNCH_SEPARATE_PASSES) != 0;
+  if (cudaMemsetAsync(a.ws + L.status, 0, L.zeroed - L.status, s) != cudaSuccess) return KDA_ERR_CUDA;
 
   if (layer_fused(cfg)) {
     // prep runs inside the intra-chunk pass; the conv state is committed afterwards

@@ -40,6 +40,7 @@
 // once; warps 12-15 then read the query gram M out of TMEM, off the tail's critical path.
 #include <type_traits>
 
+#include "kda_chain_sm100.cuh"
 #include "kda_common.cuh"
 #include "kda_launch.h"
 #include "kda_sm100.cuh"
@@ -202,8 +203,13 @@ __device__ __forceinline__ f2x ld_shared_f2x(uint32_t saddr) {
 }
 
 
-template <bool FUSED>
-__global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const PrefillArgs a) {
+// The pass on CTA `cta` of `ncta` working CTAs.  Tile n is (head n / slots, slot n % slots)
+// when it runs alone; when it shares the launch with the inter-chunk chains (COSCHED) the
+// tiles go slot by slot (slot n / H, head n % H), so that every head's chunks are done in
+// order, and each tile's word in `flags` is set once all of it has been written.
+template <bool FUSED, bool COSCHED>
+__device__ __forceinline__ void intra_body(const PrefillArgs& a, const int cta, const int ncta,
+                                           int* flags) {
   extern __shared__ __align__(1024) unsigned char smraw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~(uintptr_t)1023);
@@ -217,6 +223,8 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
 
   const int H = a.H, nslots = a.L.nslots;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  auto head_of = [&](int n) { return COSCHED ? n % H : n / nslots; };
+  auto slot_of = [&](int n) { return COSCHED ? n / H : n % nslots; };
   int* status = reinterpret_cast<int*>(a.ws + a.L.status);
 
   // once per CTA: the MMA barrier and 128 TMEM columns, kept across tiles
@@ -238,7 +246,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   const uint32_t tmem = tmem_holder;
   int issued = 0;   // MMA batches committed by thread 0 (two per tile)
 
-  // Persistent: tile index = head x slots + slot, strided over the grid.  Each iteration
+  // Persistent: tiles strided over the working CTAs.  Each iteration
   // runs the row pass of the tile in flight on all 16 warps; then warps 0-7 take its serial
   // tail (key gram readout, solve, W/U~) while warps 8-15 look up this CTA's next tile and run
   // its gate pass, whose G and beta the next row pass and tail read, and warps 12-15 read M.
@@ -250,7 +258,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   // and beta, by warps 8-15 (256 threads: channels gp, gp+1 of rows 16 gq .. 16 gq + 15) ----
   auto gate_pass = [&](int n, const TileRange& nt, int nbuf) {
     const int gt = tid - 256, gp = 2 * (gt & 63), gq = gt >> 6;
-    const int nh = n / nslots, ns = n % nslots;
+    const int nh = head_of(n), ns = slot_of(n);
     using GRawT = typename std::conditional<FUSED, uint32_t, float2>::type;   // 2 channels as loaded
     GRawT graw[16];
 #pragma unroll
@@ -271,9 +279,9 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
     // while the loads are in flight: pull into L2 the inputs of the tile after this one,
     // 128-byte lines spread over the threads
     {
-      const int nid = n + gridDim.x;
+      const int nid = n + ncta;
       if (nid < ntiles) {
-        const int nnh = nid / nslots, nns = nid % nslots;
+        const int nnh = head_of(nid), nns = slot_of(nid);
         // same sequence (slots of a sequence are consecutive): no search
         const int nc = nt.chunk + (nns - ns);
         TileRange ft;
@@ -363,7 +371,7 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   int prow = -1;
 #pragma unroll 1
   while (true) {
-  const int h = tl >= 0 ? tl / nslots : 0, slot = tl >= 0 ? tl % nslots : 0;
+  const int h = tl >= 0 ? head_of(tl) : 0, slot = tl >= 0 ? slot_of(tl) : 0;
   const size_t tile = (size_t)slot * H + h;
   __nv_bfloat16* Wo = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.W) + tile * C * D;
   __nv_bfloat16* Uo = reinterpret_cast<__nv_bfloat16*>(a.ws + a.L.Ut) + tile * C * D;
@@ -791,11 +799,11 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   } else {
     // the next tile with work: one thread walks this CTA's tiles, the group reads the result
     if (warp == THREADS / 32 - 1 && lane == 0) {
-      int n = tl < 0 ? (int)blockIdx.x : tl + (int)gridDim.x;
+      int n = tl < 0 ? cta : tl + ncta;
       TileRange nt{};
       int np = -1;
-      for (; n < ntiles; n += gridDim.x) {
-        nt = slot_to_tile(a.cu, a.n_seqs, a.total, C, n % nslots);
+      for (; n < ntiles; n += ncta) {
+        nt = slot_to_tile(a.cu, a.n_seqs, a.total, C, slot_of(n));
         np = nt.len ? pool_row(a.slots, nt.seq, a.pool_size) : -1;
         if (nt.len > 0 && np >= 0) break;
       }
@@ -839,6 +847,11 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
 
   tc_fence_before();
   __syncthreads();   // the tile's shared memory and TMEM are free; the next tile's G and beta are in place
+  if (COSCHED && tid == 0 && tl >= 0 && !abort_flag) {
+    // every write of the tile precedes the barrier: release them with its ready word
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(flags + tile), "r"(1) : "memory");
+  }
   if (abort_flag) break;
   tl = next_meta[0];
   if (tl < 0) break;
@@ -869,6 +882,59 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
 
 
 template <bool FUSED>
+__global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const PrefillArgs a) {
+  intra_body<FUSED, false>(a, blockIdx.x, gridDim.x, nullptr);
+}
+
+// One launch, two roles: CTAs 0 .. nchain-1 carry the inter-chunk chains (one per head and
+// sequence, all value columns), the others run the intra-chunk pass tile by tile and set
+// each tile's ready word, which the chains wait for (bounded).  The intra-chunk role never
+// waits for a chain, and the launch is cooperative (every CTA resident), so each wait ends.
+template <bool FUSED>
+__global__ void __launch_bounds__(THREADS, 1)
+prefill_cosched_sm100_kernel(const PrefillArgs a, const __grid_constant__ ChainMaps maps,
+                             const int nchain) {
+  int* flags = reinterpret_cast<int*>(a.ws + a.L.flags);
+  if ((int)blockIdx.x < nchain) chain::chain_body(a, maps, blockIdx.x, flags);
+  else intra_body<FUSED, true>(a, (int)blockIdx.x - nchain, (int)gridDim.x - nchain, flags);
+}
+
+template <bool FUSED>
+cudaError_t launch_cosched_t(const PrefillArgs& a, cudaStream_t st, bool* launched) {
+  constexpr size_t smem = SMEM_BYTES > chain::SMEM_BYTES ? SMEM_BYTES : chain::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(prefill_cosched_sm100_kernel<FUSED>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, nsm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  const int nchain = a.n_seqs * a.H;
+  if (nchain < 1 || 4 * nchain > nsm) return cudaSuccess;   // chains would starve the pass
+  ChainMaps maps;
+  if (!make_chain_maps(a, &maps)) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)nsm, 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, prefill_cosched_sm100_kernel<FUSED>, a, maps, nchain);
+  if (e == cudaErrorCooperativeLaunchTooLarge) {   // not every CTA fits at once: two passes
+    cudaGetLastError();
+    return cudaSuccess;
+  }
+  if (e != cudaSuccess) return e;
+  *launched = true;
+  ++launch_counter();
+  return cudaSuccess;
+}
+
+template <bool FUSED>
 cudaError_t launch_intra_t(const PrefillArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(intra_chunk_sm100_kernel<FUSED>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
@@ -896,6 +962,12 @@ bool sm100_fused_supported(const PrefillArgs& a) { return sm100_intra_supported(
 
 cudaError_t launch_intra_sm100(const PrefillArgs& a, cudaStream_t st) {
   return a.x ? launch_intra_t<true>(a, st) : launch_intra_t<false>(a, st);
+}
+
+cudaError_t launch_cosched_sm100(const PrefillArgs& a, cudaStream_t st, bool* launched) {
+  *launched = false;
+  if (!sm100_intra_supported(a) || a.y == nullptr || a.total == 0) return cudaSuccess;
+  return a.x ? launch_cosched_t<true>(a, st, launched) : launch_cosched_t<false>(a, st, launched);
 }
 
 }  // namespace kda

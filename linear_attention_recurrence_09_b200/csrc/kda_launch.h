@@ -82,7 +82,7 @@ struct RollbackArgs {
 
 // Workspace of the chunked prefill (byte offsets from its base, 256-aligned).
 struct PrefillLayout {
-  size_t status, W, Ut, Qt, Kp, o, M, gC, total;
+  size_t status, flags, zeroed, W, Ut, Qt, Kp, o, M, gC, total;
   int nslots;
   size_t wsize;  // bytes per workspace element (4 fp32 / 2 bf16)
 };
@@ -117,6 +117,7 @@ struct PrefillArgs {
   const void* conv_state;   // [pool, K-1, H, 3d] history, or nullptr for zeros
   int K;
   int gate_softplus;        // unbounded decay: the SIMT passes with exact diagonal gram blocks
+  bool separate_passes;     // never the co-scheduled single launch
 };
 
 // One output range of the projection GEMM: columns [col_begin, col_end) of C = A B^T go
@@ -152,6 +153,8 @@ bool sm100_intra_supported(const PrefillArgs& a);
 bool sm100_fused_supported(const PrefillArgs& a);
 cudaError_t launch_conv_commit(const PrepArgs& a, cudaStream_t st);
 cudaError_t launch_intra_sm100(const PrefillArgs& a, cudaStream_t st);
+// both tensor-core passes in one cooperative launch; `launched` false = not applicable
+cudaError_t launch_cosched_sm100(const PrefillArgs& a, cudaStream_t st, bool* launched);
 // fused_norm: set when the pass also applied the gated RMSNorm and wrote y
 cudaError_t launch_interchunk_sm100(const PrefillArgs& a, cudaStream_t st, bool* fused_norm);
 cudaError_t launch_wait_timeout_selftest(void* workspace, cudaStream_t st);

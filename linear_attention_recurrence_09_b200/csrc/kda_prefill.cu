@@ -46,6 +46,8 @@ PrefillLayout prefill_layout(int n_seqs, int total, int H, int D, int C, bool bf
   const size_t per_slot = (size_t)L.nslots * H * C * D;   // C x D tile per (slot, head)
   size_t off = 0;
   L.status = off; off += 256;
+  L.flags = off; off += align256((size_t)L.nslots * H * 4);  // per-tile ready flags
+  L.zeroed = off;                                            // status + flags, cleared per call
   L.W = off; off += align256(per_slot * L.wsize);
   L.Ut = off; off += align256(per_slot * L.wsize);
   L.Qt = off; off += align256(per_slot * L.wsize);
@@ -372,6 +374,15 @@ static cudaError_t launch_prefill_dc(const PrefillArgs& a, cudaStream_t st) {
   // with each other, and raw (pre-conv) inputs are only read by the tcgen05 pass
   if (sm100_intra_supported(a) != sm100_interchunk_supported(a)) return cudaErrorInvalidValue;
   if (a.x != nullptr && !sm100_fused_supported(a)) return cudaErrorInvalidValue;
+  if (sm100_intra_supported(a) && !a.separate_passes) {
+    bool one = false;
+    if ((e = launch_cosched_sm100(a, st, &one)) != cudaSuccess) return e;
+    if (one) {   // both passes and the norm in one launch
+      for (int i = 0; i < 3; ++i)
+        if (pe.ev[i] && (e = cudaEventRecord(pe.ev[i], st)) != cudaSuccess) return e;
+      return cudaSuccess;
+    }
+  }
   if (sm100_intra_supported(a)) {
     e = launch_intra_sm100(a, st);
     if (e != cudaSuccess) return e;

@@ -511,6 +511,17 @@ bool make_map(EncodeTiledFn enc, CUtensorMap* m, void* base, uint64_t rows, uint
 
 }  // namespace
 
+bool make_chain_maps(const PrefillArgs& a, ChainMaps* m) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const uint64_t tiles = (uint64_t)a.L.nslots * a.H;
+  return make_map(enc, &m->W, a.ws + a.L.W, tiles * C, D, 64) &&
+         make_map(enc, &m->Q, a.ws + a.L.Qt, tiles * C, D, 64) &&
+         make_map(enc, &m->KT, a.ws + a.L.Kp, tiles * C, D, 64) &&
+         make_map(enc, &m->M, a.ws + a.L.M, tiles * C, C, 64) &&
+         make_map(enc, &m->Ut, a.ws + a.L.Ut, tiles * C, D, 64);
+}
+
 cudaError_t launch_wait_timeout_selftest(void* workspace, cudaStream_t st) {
   wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(static_cast<int*>(workspace),
                                                  WAIT_LIMIT_CYCLES / 4);

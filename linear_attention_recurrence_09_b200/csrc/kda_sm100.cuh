@@ -254,4 +254,12 @@ __device__ __forceinline__ float to_tf32(float x) {
   return __uint_as_float(r);
 }
 
+// Tensor maps of the inter-chunk chain over the workspace tiles (bf16, 128B swizzle,
+// 64-column boxes): W, Q~, K' and U~ [tiles x 64 rows, 128], M [tiles x 64 rows, 64].
+struct ChainMaps {
+  CUtensorMap W, Q, KT, M, Ut;
+};
+struct PrefillArgs;
+bool make_chain_maps(const PrefillArgs& a, ChainMaps* m);   // false if a map is rejected
+
 }  // namespace kda

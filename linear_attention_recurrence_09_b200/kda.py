@@ -34,6 +34,7 @@ KDA_CONV_TAPE = 1
 KDA_GATE_BOUNDED_SIGMOID = 0
 KDA_GATE_SOFTPLUS = 1
 KDA_LAUNCH_EARLY_STATE = 1
+KDA_LAUNCH_SEPARATE_PASSES = 2
 ABI_VERSION = 2
 
 ENTRY_POINTS = ('kda_status_string', 'kda_abi_version', 'kda_prep',
@@ -70,7 +71,9 @@ class Config:
     ``launch_flags``: KDA_LAUNCH_EARLY_STATE lets the token-step calls and the replay
     rollback stream the recurrent state before the kernel ahead of them on the stream
     has finished; set it only when that kernel writes neither the state nor the slots
-    (kda_prep, or kda_verify_compact before kda_rollback_replay)."""
+    (kda_prep, or kda_verify_compact before kda_rollback_replay).
+    KDA_LAUNCH_SEPARATE_PASSES keeps the tensor-core prefill's two passes in separate
+    launches where one co-scheduled launch would otherwise carry both."""
     num_heads: int
     head_dim: int
     conv_size: int = 4

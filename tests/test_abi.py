@@ -80,7 +80,7 @@ def test_prep_rejects_bad_arguments(L):
     bad.gate_kind = 2
     assert _prep(L, bad) == kda.KDA_ERR_INVALID_ARG
     bad = _cfg()
-    bad.launch_flags = 2                              # only KDA_LAUNCH_EARLY_STATE is defined
+    bad.launch_flags = 4                              # bits 0 and 1 are the defined flags
     assert _prep(L, bad) == kda.KDA_ERR_INVALID_ARG
     ok = _cfg()
     ok.launch_flags = kda.KDA_LAUNCH_EARLY_STATE

@@ -35,7 +35,8 @@ def test_profile_summaries_name_their_source_and_traffic():
         text = open(os.path.join(ROOT, summary)).read()
         assert re.search(r'code_sha256:\s*[0-9a-f]{64}', text), summary
         assert re.search(r'traffic_bytes_per_launch:\s*[0-9]+', text), summary
-        assert os.path.exists(os.path.join(ROOT, source)), source
+        for src in ([source] if isinstance(source, str) else source):
+            assert os.path.exists(os.path.join(ROOT, src)), src
         assert '--clock-control none' in text, summary
 
 

@@ -73,6 +73,30 @@ def test_prefill_varlen_ragged_bf16(d, chunk, fused):
     _assert(compare_layer(cfg, P, A, S0, hist, fused=fused), 1e-2)
 
 
+@pytest.mark.parametrize('fused', [True, False])
+@pytest.mark.parametrize('seqlens,H', [([1000], 8), ([0, 130, 1, 64, 257], 6), ([8192], 32)])
+def test_cosched_launch_equals_separate_passes(seqlens, H, fused):
+    """The tensor-core prefill as one co-scheduled launch (a full-width inter-chunk chain per
+    (sequence, head) beside the intra-chunk pass, handing over through per-tile ready words)
+    equals the two separate launches bit for bit: the chain takes each state element and
+    each token's norm through the same operations in the same order.  Both meet the oracle
+    bar (checked on the smaller cases; the 8,192-token one is the headline shape)."""
+    cfg, P, A, S0, hist = make_case(23, seqlens, H, 128, 4, torch.bfloat16, state_var=0.01,
+                                    conv_hist=True, chunk=64)
+    sep = dataclasses.replace(cfg, launch_flags=kda.KDA_LAUNCH_SEPARATE_PASSES)
+    n0 = kda.kda_launch_count()
+    y1, s1, c1, _ = gpu_layer(cfg, P, A, S0, hist, fused=fused)
+    n1 = kda.kda_launch_count()
+    y2, s2, c2, _ = gpu_layer(sep, P, A, S0, hist, fused=fused)
+    n2 = kda.kda_launch_count()
+    assert n2 - n1 == (n1 - n0) + 1          # the co-scheduled form is one launch fewer
+    assert torch.equal(y1, y2)
+    assert torch.equal(s1, s2)
+    assert torch.equal(c1, c2)
+    if sum(seqlens) <= 2048:
+        _assert(compare_layer(cfg, P, A, S0, hist, fused=fused), 1e-2)
+
+
 @pytest.mark.parametrize('K', [2, 4])
 def test_layer_prefill_conv_sizes(K):
     """Fused (K = 4) and fallback (K = 2) layer prefill, conv history carried."""
@@ -313,18 +337,21 @@ def test_bounded_wait_times_out_and_context_survives():
 
 def test_layer_prefill_launches_and_fused_norm():
     """bf16, d = 128, chunk 64, conv 4: prep runs inside the intra-chunk pass and the gated
-    norm inside the inter-chunk pass, so one layer call is two kernels (plus the conv-state
-    commit when a conv state is given); the result is the oracle's either way."""
+    norm inside the inter-chunk pass.  With few (sequence, head) chains both passes share
+    one co-scheduled launch; with KDA_LAUNCH_SEPARATE_PASSES they are two kernels.  The
+    conv-state commit adds one launch when a conv state is given."""
     cfg, P, A, S0, hist = make_case(21, [300, 64], 4, 128, 4, torch.bfloat16, state_var=0.01,
                                     conv_hist=True, chunk=64)
+    sep = dataclasses.replace(cfg, launch_flags=kda.KDA_LAUNCH_SEPARATE_PASSES)
     Pd = {k: v.cuda() for k, v in P.items()}
     Ad = {k: v.cuda() for k, v in A.items()}
-    n0 = kda.kda_launch_count()
-    kda.layer_prefill(cfg, Pd, Ad, state_out=torch.empty(2, 4, 128, 128, device='cuda'))
-    assert kda.kda_launch_count() - n0 == 2
+    for c, n_pass in ((cfg, 1), (sep, 2)):
+        n0 = kda.kda_launch_count()
+        kda.layer_prefill(c, Pd, Ad, state_out=torch.empty(2, 4, 128, 128, device='cuda'))
+        assert kda.kda_launch_count() - n0 == n_pass
     n0 = kda.kda_launch_count()
     y, s_out, cs, _ = gpu_layer(cfg, P, A, S0, hist, fused=True)
-    assert kda.kda_launch_count() - n0 == 3
+    assert kda.kda_launch_count() - n0 == 2
     ref = oracle_layer(cfg, P, A, S0, hist)
     assert rel_err(np64(y), ref['y']) <= 1e-2
     assert rel_err(np64(s_out), ref['state']) <= 1e-2
