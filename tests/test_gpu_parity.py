@@ -881,3 +881,71 @@ def test_pool_slots_short_prep_and_early_state():
         torch.cuda.synchronize()
         assert torch.equal(st[0], pool_state[r]) and torch.equal(cs[0], pool_conv[r]), b
         assert torch.equal(y1[0], y[b]) and torch.equal(yv1[0], yv[b]), b
+
+
+def test_cosched_pool_slots_with_a_skipped_sequence():
+    """The co-scheduled launch with a state pool: a sequence mapped to slot -1 is skipped
+    (its chain CTA returns, the intra-chunk role skips its tiles) and the pool rows no
+    sequence maps to stay as they were; everything equals the separate launches bit for bit."""
+    seqlens, H, d, pool = [200, 70, 131], 4, 128, 6
+    cfg, P, A, _, _ = make_case(31, seqlens, H, d, 4, torch.bfloat16, chunk=64)
+    sep = dataclasses.replace(cfg, launch_flags=kda.KDA_LAUNCH_SEPARATE_PASSES)
+    dev = 'cuda'
+    Pd = {k: v.to(dev) for k, v in P.items()}
+    Ad = {k: v.to(dev) for k, v in A.items()}
+    slots = torch.tensor([4, -1, 1], dtype=torch.int32, device=dev)
+    s0 = synth.initial_state(31, pool, H, d, 0.01).to(dev)
+    c0 = (torch.randn(pool, 3, H, 3 * d, generator=torch.Generator().manual_seed(31)) * 0.5
+          ).to(cfg.dtype).to(dev)
+    outs = []
+    for c in (cfg, sep):
+        st, cs = s0.clone(), c0.clone()
+        y = torch.full((sum(seqlens), H, d), 7.0, dtype=cfg.dtype, device=dev)
+        kda.kda_layer_prefill(c, Ad['cu_seqlens'], Ad['x'], Ad['f'], Ad['beta_logit'], Ad['g'],
+                              Pd['conv_w'], Pd['A_log'], Pd['dt_bias'], Pd['norm_w'],
+                              conv_state=cs, state_in=st, state_out=st, state_slots=slots,
+                              pool_size=pool, y=y, max_seqlen=max(seqlens))
+        torch.cuda.synchronize()
+        outs.append((y.clone(), st.clone(), cs.clone()))
+    (y1, s1, c1), (y2, s2, c2) = outs
+    assert torch.equal(y1, y2) and torch.equal(s1, s2) and torch.equal(c1, c2)
+    skipped = slice(seqlens[0], seqlens[0] + seqlens[1])
+    assert torch.all(y1[skipped] == 7.0)
+    for r in (0, 2, 3, 5):
+        assert torch.equal(s1[r], s0[r]) and torch.equal(c1[r], c0[r])
+    assert not torch.equal(s1[4], s0[4]) and not torch.equal(s1[1], s0[1])
+
+
+def test_cosched_launch_in_a_cuda_graph():
+    """The co-scheduled (cooperative) launch captured in a CUDA graph with the call's
+    workspace clear: two replays give the eager result bit for bit."""
+    seqlens, H = [1000], 8
+    cfg, P, A, S0, hist = make_case(33, seqlens, H, 128, 4, torch.bfloat16, state_var=0.01,
+                                    chunk=64)
+    dev = 'cuda'
+    Pd = {k: v.to(dev) for k, v in P.items()}
+    Ad = {k: v.to(dev) for k, v in A.items()}
+    s_in = S0.to(dev)
+    ws = torch.empty(kda.kda_layer_prefill_workspace_size(cfg, 1, sum(seqlens)),
+                     dtype=torch.uint8, device=dev)
+    y_ref = torch.empty(sum(seqlens), H, 128, dtype=cfg.dtype, device=dev)
+    st_ref = torch.empty_like(s_in)
+    kda.layer_prefill(cfg, Pd, Ad, state_in=s_in, state_out=st_ref, workspace=ws, y=y_ref)
+    torch.cuda.synchronize()
+    y = torch.empty_like(y_ref)
+    st = torch.empty_like(st_ref)
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        kda.layer_prefill(cfg, Pd, Ad, state_in=s_in, state_out=st, workspace=ws, y=y)
+    torch.cuda.current_stream().wait_stream(side)
+    with torch.cuda.graph(g):
+        kda.layer_prefill(cfg, Pd, Ad, state_in=s_in, state_out=st, workspace=ws, y=y)
+    for _ in range(2):
+        y.zero_()
+        st.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, y_ref) and torch.equal(st, st_ref)
+    del g
