@@ -653,8 +653,8 @@ def run_long(torch, kda, synth, dev, steps=5, warmup=3):
                             'frac': ach / hbm, 'peak_kind': peak_kind,
                             'algorithmic_bytes_per_launch': method}}
         if launches == 1:
-            # beside it: the two passes as separate launches, whose inter-chunk pass gives
-            # the chain period (one wave of 128 four-slice chain CTAs)
+            # beside it: the two passes as separate launches (for one sequence, the inter-chunk
+            # pass over the serial chunks gives the 4-slice chain period)
             c_sep = dataclasses.replace(cfg, launch_flags=kda.KDA_LAUNCH_SEPARATE_PASSES)
             for _ in range(warmup):
                 step(c=c_sep)
@@ -665,8 +665,9 @@ def run_long(torch, kda, synth, dev, steps=5, warmup=3):
             bd = breakdown(evs2, 2)
             rec['separate_passes'] = {
                 'ms_per_step': statistics.median(e[0].elapsed_time(e[3]) for e in evs2),
-                'breakdown_ms': bd,
-                'chain_us_per_chunk': bd['inter_chunk'] * 1e3 / (-(-T // 64))}
+                'breakdown_ms': bd}
+            if N == 1:
+                rec['separate_passes']['chain_us_per_chunk'] = bd['inter_chunk'] * 1e3 / (-(-T // 64))
             # the co-scheduled chains run one CTA per head, all value columns; the step is
             # bound by the intra-chunk pass on the remaining SMs, not by the chain
         elif N == 1:

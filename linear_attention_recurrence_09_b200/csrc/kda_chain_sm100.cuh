@@ -61,8 +61,14 @@ static_assert(BAR_COUNT * 8 <= 256, "barrier slots");
 constexpr int NE = 12;        // E1/E2 warps (4..15)
 constexpr int NOUT = 8;       // warps of E3: 2, 3 and the E2 warps of lane quarters 2-3
 
-// sigmoid on the special-function unit (bf16 output: approximate exp and divide suffice)
-__device__ __forceinline__ float sigmoid_fast(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
+// sigmoid(z) = (1 + tanh(z / 2)) / 2 with one special-function op (tanh.approx, absolute
+// error about 2^-11): the outputs are bf16 and the output gate's error stays far inside
+// the parity budget; the two inter-chunk kernels share the form, so their outputs agree
+__device__ __forceinline__ float sigmoid_fast(float z) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
+  return fmaf(0.5f, t, 0.5f);
+}
 
 // byte offset of element (row k, 16-byte chunk) of an MN-major, 128B-swizzled tile
 __device__ __forceinline__ uint32_t mn_chunk(int k, int chunk) {
@@ -107,9 +113,35 @@ __device__ __forceinline__ bool wait_ready(const int* flag, volatile int* abort_
   }
 }
 
-// The chain of (head, sequence) c = s * H + h.  `flags` holds one word per workspace
-// tile, set once the intra-chunk pass has written all of that tile.
-__device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps& maps, int c,
+// A head's chain walks the batch sequence by sequence, chunk by chunk: the order in which
+// the intra-chunk role completes the tiles.  Position: sequence s (pool row `row`, tokens
+// [start, end), nch chunks), chunk n.
+struct ChainPos {
+  int s, row, start, end, nch, n;
+};
+// the first sequence >= s0 that has a pool row and at least one token; false past the end
+__device__ __forceinline__ bool chain_seq_from(const PrefillArgs& a, int s0, ChainPos& k) {
+  for (int s = s0; s < a.n_seqs; ++s) {
+    const int row = pool_row(a.slots, s, a.pool_size);
+    if (row < 0) continue;
+    int st, en;
+    seq_range(a.cu, a.total, s, st, en);
+    if (en > st) {
+      k.s = s; k.row = row; k.start = st; k.end = en; k.nch = (en - st + C - 1) / C; k.n = 0;
+      return true;
+    }
+  }
+  return false;
+}
+// the next chunk of the walk; false past the end
+__device__ __forceinline__ bool chain_next(const PrefillArgs& a, ChainPos& k) {
+  if (++k.n < k.nch) return true;
+  return chain_seq_from(a, k.s + 1, k);
+}
+
+// The chain of head h over every sequence of the batch.  `flags` holds one word per
+// workspace tile, set once the intra-chunk pass has written all of that tile.
+__device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps& maps, int h,
                                            const int* flags) {
   extern __shared__ __align__(1024) unsigned char smraw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
@@ -120,12 +152,7 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
   __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int H = a.H, h = c % H, s = c / H;
-  const int row = pool_row(a.slots, s, a.pool_size);
-  if (row < 0) return;
-  int start, end;
-  seq_range(a.cu, a.total, s, start, end);
-  const int nch = (end - start + C - 1) / C;
+  const int H = a.H;
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   if (threadIdx.x == 0) {
@@ -161,12 +188,12 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
   auto d1_of = [&](int n) -> uint32_t { return tmem + 128u * (uint32_t)(n % 3); };
   const uint32_t d2_tmem = tmem + 384;
   int* status = reinterpret_cast<int*>(a.ws + a.L.status);
-  auto tile_of = [&](int n) { return (start / C + s + n) * H + h; };
+  auto tile_of = [&](const ChainPos& k) { return (k.start / C + k.s + k.n) * H + h; };
   // E3 of chunk m for the 32 tokens of TMEM lane quarter q (2 or 3) and value columns
   // 32 j .. 32 j + 31 (slice j), by one warp: the four warps of a quarter each take a slice,
   // sum their squares, exchange the partials through shared memory (a bounded mbarrier wait)
   // and add them in slice order.  `gb` holds the slice's gate row.
-  auto o_slice = [&](int m, int q, int j, const uint4 (&gb)[4]) -> bool {
+  auto o_slice = [&](int m, int t0, int L, int q, int j, const uint4 (&gb)[4]) -> bool {
     if (!mbar_wait_warp(bar(BAR_ODONE0 + m % 3), (m / 3) & 1, &abort_flag)) return false;
     tc_fence_after();
     const int lane = threadIdx.x & 31;
@@ -197,8 +224,7 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
     tot += pp.z;
     tot += pp.w;
     const float rstd = rsqrtf(tot * (1.0f / D) + a.norm_eps);
-    const int t0 = start + m * C;
-    if (r < min(C, end - t0)) {
+    if (r < L) {
       const float* nw = reinterpret_cast<const float*>(sm + OFF_NW) + 32 * j;
       uint4* yp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.y) +
                                            ((size_t)(t0 + r) * H + h) * D + 32 * j);
@@ -222,10 +248,10 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
     }
     return true;
   };
-  // the gate row of token 32 (q - 2) + lane of chunk m, columns 32 j .. 32 j + 31
-  auto load_gate = [&](int m, int q, int j, uint4 (&gb)[4]) {
-    const int t0 = start + m * C, r = 32 * (q - 2) + (threadIdx.x & 31);
-    const bool live = m < nch && r < min(C, end - t0);
+  // the gate row of token t0 + 32 (q - 2) + lane of a chunk of L tokens, columns 32 j .. +31
+  auto load_gate = [&](int t0, int L, int q, int j, uint4 (&gb)[4]) {
+    const int r = 32 * (q - 2) + (threadIdx.x & 31);
+    const bool live = r < L;
     const uint4* gp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.g) +
                                                      ((size_t)(t0 + r) * H + h) * D + 32 * j);
 #pragma unroll
@@ -240,12 +266,14 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
     // ---------------- ready flags + TMA producer ----------------
     if (lane == 0) {
       int issued = 0;
-      for (int n = 0; n < nch && !abort_flag; ++n) {
+      ChainPos k;
+      bool more = chain_seq_from(a, 0, k);
+      for (int n = 0; more && !abort_flag; ++n, more = chain_next(a, k)) {
         const int st = n % NSTAGE;
         if (n >= (int)NSTAGE &&
             !mbar_wait(bar(BAR_EMPTY0 + st), ((n / NSTAGE) - 1) & 1, &abort_flag))
           break;
-        const int tile = tile_of(n);
+        const int tile = tile_of(k);
         if (!wait_ready(flags + tile, &abort_flag)) break;
         // the tile was written through the generic proxy by other SMs; TMA reads it
         // through the async proxy
@@ -290,6 +318,12 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
         umma_commit(bar(BAR_EMPTY0 + stm));
         umma_commit(bar(BAR_ODONE0 + m % 3));
       };
+      int nch = 0;   // chunks of the whole walk
+      {
+        ChainPos k;
+        for (bool more = chain_seq_from(a, 0, k); more; more = chain_seq_from(a, k.s + 1, k))
+          nch += k.nch;
+      }
       int committed = 0;
       for (int n = 0; n < nch; ++n) {
         const int st = n % NSTAGE;
@@ -329,14 +363,22 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
   } else if (warp < 4) {
     // ---------------- E3, slice 0 (warps 2, 3), off the serial chain ----------------
     const int q = warp & 3;
+    ChainPos k, kn;
+    bool more = chain_seq_from(a, 0, k);
     uint4 gb[4];
-    load_gate(0, q, 0, gb);
-    for (int m = 0; m < nch; ++m) {
+    if (more) load_gate(k.start, min(C, k.end - k.start), q, 0, gb);
+    for (int m = 0; more; ++m) {
+      const int t0 = k.start + k.n * C, L = min(C, k.end - t0);
+      kn = k;
+      const bool next = chain_next(a, kn);
       uint4 gn[4];
-      load_gate(m + 1, q, 0, gn);   // one chunk ahead
-      if (!o_slice(m, q, 0, gb)) break;
+      const int tn = kn.start + kn.n * C;
+      load_gate(tn, next ? min(C, kn.end - tn) : 0, q, 0, gn);   // one chunk ahead
+      if (!o_slice(m, t0, L, q, 0, gb)) break;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) gb[k] = gn[k];
+      for (int e = 0; e < 4; ++e) gb[e] = gn[e];
+      k = kn;
+      more = next;
     }
   } else {
     // ---------------- E1 / E2 warps 4..15 ----------------
@@ -349,16 +391,39 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
     unsigned char* SB = sm + OFF_S;
     unsigned char* UB0 = sm + OFF_U;
     const float* gCg = reinterpret_cast<const float*>(a.ws + a.L.gC);
-    const size_t sg = (((size_t)row * H + h) * D + i) * D + cb;
-
+    // this thread's part of a state: key row i, value columns cb + 16 g .. (ng groups)
+    auto state_at = [&](int row) { return (((size_t)row * H + h) * D + i) * D + cb; };
     float S[3][16];
+    auto load_state = [&](int row) {
 #pragma unroll
-    for (int g = 0; g < 3; ++g)
+      for (int g = 0; g < 3; ++g)
 #pragma unroll
-      for (int e = 0; e < 16; e += 4) {
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (g < ng && a.state_in) v = *reinterpret_cast<const float4*>(a.state_in + sg + 16 * g + e);
-        S[g][e] = v.x; S[g][e + 1] = v.y; S[g][e + 2] = v.z; S[g][e + 3] = v.w;
+        for (int e = 0; e < 16; e += 4) {
+          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (g < ng && a.state_in)
+            v = *reinterpret_cast<const float4*>(a.state_in + state_at(row) + 16 * g + e);
+          S[g][e] = v.x; S[g][e + 1] = v.y; S[g][e + 2] = v.z; S[g][e + 3] = v.w;
+        }
+    };
+    auto store_state = [&](int row) {
+      if (!a.state_out) return;
+#pragma unroll
+      for (int g = 0; g < 3; ++g)
+        if (g < ng)
+#pragma unroll
+          for (int e = 0; e < 16; e += 4)
+            *reinterpret_cast<float4*>(a.state_out + state_at(row) + 16 * g + e) =
+                make_float4(S[g][e], S[g][e + 1], S[g][e + 2], S[g][e + 3]);
+    };
+    // sequences without tokens keep their state (state_in, or zeros, to state_out)
+    if (a.state_out)
+      for (int sq = 0; sq < a.n_seqs; ++sq) {
+        const int row = pool_row(a.slots, sq, a.pool_size);
+        int st, en;
+        seq_range(a.cu, a.total, sq, st, en);
+        if (row < 0 || en > st) continue;
+        load_state(row);
+        store_state(row);
       }
     auto write_state = [&]() {   // key row i, 16 columns per group: two 16-byte chunks each
 #pragma unroll
@@ -374,22 +439,35 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
       tc_fence_before();
       mbar_arrive(bar(BAR_SREADY));
     };
+    ChainPos k;
+    bool more = chain_seq_from(a, 0, k);
+    if (more) load_state(k.row);
     write_state();
     uint4 gb[4];   // quarters 2-3: the gate row of the output slice of the previous chunk
+    int pt0 = 0, pL = 0, n = 0;   // the previous chunk's first token and length
 
-    for (int n = 0; n < nch; ++n) {
+    for (; more; ++n) {
       const int st = n % NSTAGE;
       unsigned char* UB = UB0 + (n & 1) * U_BYTES;
-      const int t0 = start + n * C;
-      const int L = min(C, end - t0);
+      const int t0 = k.start + k.n * C;
+      const int L = min(C, k.end - t0);
       // the stage has landed, so the producer saw the tile's ready flag: e^{G_C} is readable
       if (!mbar_wait_warp(bar(BAR_FULL0 + st), (n / NSTAGE) & 1, &abort_flag)) break;
-      const float gc = __ldcg(gCg + (size_t)tile_of(n) * D + i);
+      const float gc = __ldcg(gCg + (size_t)tile_of(k) * D + i);
       if (q >= 2 && n > 0) {   // the gate slice of the previous chunk's output, into L2
-        const int r = 32 * (q - 2) + lane, tp = start + (n - 1) * C;
-        if (r < min(C, end - tp))
+        const int r = 32 * (q - 2) + lane;
+        if (r < pL)
           asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const __nv_bfloat16*>(a.g) +
-                                                         ((size_t)(tp + r) * H + h) * D + 32 * (part + 1)));
+                                                         ((size_t)(pt0 + r) * H + h) * D + 32 * (part + 1)));
+      }
+      const bool last = k.n + 1 == k.nch;
+      if (last && a.state_in) {   // the next sequence's initial state, into L2
+        ChainPos kn;
+        if (chain_seq_from(a, k.s + 1, kn)) {
+          const char* sp = reinterpret_cast<const char*>(a.state_in + state_at(kn.row));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(sp));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(sp + 128));
+        }
       }
       if (q < 2) {
         // E1: U = U~ - W S for token row i (0..63), this thread's columns: groups 0-1, then 2
@@ -455,25 +533,25 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
 #pragma unroll
         for (int e = 0; e < 16; ++e) S[2][e] = fmaf(gc, S[2][e], __uint_as_float(d2v[e]));
       }
+      if (last) {   // the sequence's final state out, the next one's initial state in
+        store_state(k.row);
+        more = chain_seq_from(a, k.s + 1, k);
+        if (more) load_state(k.row);
+      } else {
+        ++k.n;
+      }
       write_state();
       // E3 of the previous chunk (its output product retired before this chunk's MMA2)
       if (q >= 2 && n > 0) {
-        load_gate(n - 1, q, part + 1, gb);
-        if (!o_slice(n - 1, q, part + 1, gb)) break;
+        load_gate(pt0, pL, q, part + 1, gb);
+        if (!o_slice(n - 1, pt0, pL, q, part + 1, gb)) break;
       }
+      pt0 = t0;
+      pL = L;
     }
-    if (q >= 2 && nch > 0 && !abort_flag) {
-      load_gate(nch - 1, q, part + 1, gb);
-      o_slice(nch - 1, q, part + 1, gb);
-    }
-    if (!abort_flag && a.state_out) {
-#pragma unroll
-      for (int g = 0; g < 3; ++g)
-        if (g < ng)
-#pragma unroll
-          for (int e = 0; e < 16; e += 4)
-            *reinterpret_cast<float4*>(a.state_out + sg + 16 * g + e) =
-                make_float4(S[g][e], S[g][e + 1], S[g][e + 2], S[g][e + 3]);
+    if (q >= 2 && n > 0 && !abort_flag) {
+      load_gate(pt0, pL, q, part + 1, gb);
+      o_slice(n - 1, pt0, pL, q, part + 1, gb);
     }
   }
 

@@ -886,10 +886,11 @@ __global__ void __launch_bounds__(THREADS, 1) intra_chunk_sm100_kernel(const Pre
   intra_body<FUSED, false>(a, blockIdx.x, gridDim.x, nullptr);
 }
 
-// One launch, two roles: CTAs 0 .. nchain-1 carry the inter-chunk chains (one per head and
-// sequence, all value columns), the others run the intra-chunk pass tile by tile and set
-// each tile's ready word, which the chains wait for (bounded).  The intra-chunk role never
-// waits for a chain, and the launch is cooperative (every CTA resident), so each wait ends.
+// One launch, two roles: CTAs 0 .. H-1 carry the inter-chunk chains (one per head, all
+// value columns, walking the sequences of the batch in order), the others run the
+// intra-chunk pass tile by tile in the same order and set each tile's ready word, which the
+// chains wait for (bounded).  The intra-chunk role never waits for a chain, and the launch
+// is cooperative (every CTA resident), so each wait ends.
 template <bool FUSED>
 __global__ void __launch_bounds__(THREADS, 1)
 prefill_cosched_sm100_kernel(const PrefillArgs a, const __grid_constant__ ChainMaps maps,
@@ -909,8 +910,12 @@ cudaError_t launch_cosched_t(const PrefillArgs& a, cudaStream_t st, bool* launch
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return e;
-  const int nchain = a.n_seqs * a.H;
-  if (nchain < 1 || 4 * nchain > nsm) return cudaSuccess;   // chains would starve the pass
+  // A chain completes a chunk in about 0.27 of the intra-chunk pass's time per tile, so
+  // the chains keep pace with the other SMs' production when H >= about a fifth of the
+  // SMs; with fewer heads they would set the pace, with more than a quarter the pass
+  // would lose too many SMs: the separate launches are faster in both cases.
+  const int nchain = a.H;
+  if (4 * nchain > nsm || 5 * nchain < nsm) return cudaSuccess;
   ChainMaps maps;
   if (!make_chain_maps(a, &maps)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};

@@ -86,8 +86,14 @@ struct TmaMaps {
   CUtensorMap W, Q, KT, M, Ut;
 };
 
-// sigmoid on the special-function unit (bf16 output: approximate exp and divide suffice)
-__device__ __forceinline__ float fast_sigmoid(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
+// sigmoid(z) = (1 + tanh(z / 2)) / 2 with one special-function op (tanh.approx, absolute
+// error about 2^-11): the outputs are bf16 and the output gate's error stays far inside
+// the parity budget; the two inter-chunk kernels share the form, so their outputs agree
+__device__ __forceinline__ float fast_sigmoid(float z) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
+  return fmaf(0.5f, t, 0.5f);
+}
 
 // byte offset of element (row k, column n < 64) of an MN-major, 128B-swizzled bf16 tile
 // (rows of 128 bytes, 8-row groups of 1024 bytes, 16-byte chunks XOR-ed with k mod 8)
