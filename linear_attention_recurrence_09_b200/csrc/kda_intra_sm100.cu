@@ -645,16 +645,17 @@ __device__ __forceinline__ void intra_body(const PrefillArgs& a, const int cta, 
   // column), then the blocks below (X_ab = -X_aa sum_{k=b}^{a-1} A_ak X_kb for a > b),
   // organised as two levels of 32 x 32 doubling
   if (tid < 64) {
+    // right-looking: once x_i is final it goes into every later row's sum, so the chain
+    // from one row to the next is one FMA; each x_r still sums its terms in order of i
     const int b = tid >> 4, jj = tid & 15;
     const float* Ab = Af + (16 * b) * AF_LD + 16 * b;
     float xc[16];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      float acc = (r == jj) ? 1.f : 0.f;
+    for (int r = 0; r < 16; ++r) xc[r] = (r == jj) ? 1.f : 0.f;
 #pragma unroll
-      for (int i = 0; i < r; ++i) acc = fmaf(-Ab[r * AF_LD + i], xc[i], acc);
-      xc[r] = acc;
-    }
+    for (int i = 0; i < 15; ++i)
+#pragma unroll
+      for (int r = i + 1; r < 16; ++r) xc[r] = fmaf(-Ab[r * AF_LD + i], xc[i], xc[r]);
 #pragma unroll
     for (int r = 0; r < 16; ++r) Xs[(16 * b + r) * AF_LD + 16 * b + jj] = xc[r];
   }
