@@ -115,11 +115,11 @@ enum kda_gate { KDA_GATE_BOUNDED_SIGMOID = 0, KDA_GATE_SOFTPLUS = 1 };
  *
  * The tensor-core prefill (bf16, d = 128, chunk 64, bounded gate) runs as ONE
  * cooperative launch when the head count lies between a fifth and a quarter of the SMs
- * (32 heads on a B200): H CTAs carry the inter-chunk chains, one per head over every
- * sequence of the batch, while the others run the intra-chunk pass, and each chain waits
- * (bounded) for its chunk's tiles through ready words in the workspace.
- * KDA_LAUNCH_SEPARATE_PASSES runs the two passes as separate launches instead (the form
- * used for other head counts); the results agree bit for bit.
+ * (32 heads on a B200) and the sequences average at least 4 chunks: H CTAs carry the
+ * inter-chunk chains, one per head over every sequence of the batch, while the others
+ * run the intra-chunk pass, and each chain waits (bounded) for its chunk's tiles through
+ * ready words in the workspace.  KDA_LAUNCH_SEPARATE_PASSES runs the two passes as
+ * separate launches instead (the form used otherwise); the results agree bit for bit.
  */
 enum kda_launch_flag { KDA_LAUNCH_EARLY_STATE = 1, KDA_LAUNCH_SEPARATE_PASSES = 2 };
 

@@ -150,11 +150,31 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   __shared__ uint32_t tmem_holder;
   __shared__ volatile int abort_flag;
+  constexpr int MAX_EMPTY = 64;
+  __shared__ int walk_chunks, n_empty, empty_seq[MAX_EMPTY];   // set up by all threads at once
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = a.H;
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
+  if (threadIdx.x == 0) {
+    walk_chunks = 0;
+    n_empty = 0;
+  }
+  __syncthreads();
+  // the walk's length, and the sequences with a pool row but no tokens (their state passes
+  // through): every thread looks at a strided share of the batch
+  for (int sq = threadIdx.x; sq < a.n_seqs; sq += blockDim.x) {
+    if (pool_row(a.slots, sq, a.pool_size) < 0) continue;
+    int st, en;
+    seq_range(a.cu, a.total, sq, st, en);
+    if (en > st) {
+      atomicAdd(&walk_chunks, (en - st + C - 1) / C);
+    } else {
+      const int e = atomicAdd(&n_empty, 1);
+      if (e < MAX_EMPTY) empty_seq[e] = sq;
+    }
+  }
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int st = 0; st < (int)NSTAGE; ++st) {
@@ -318,12 +338,7 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
         umma_commit(bar(BAR_EMPTY0 + stm));
         umma_commit(bar(BAR_ODONE0 + m % 3));
       };
-      int nch = 0;   // chunks of the whole walk
-      {
-        ChainPos k;
-        for (bool more = chain_seq_from(a, 0, k); more; more = chain_seq_from(a, k.s + 1, k))
-          nch += k.nch;
-      }
+      const int nch = walk_chunks;   // chunks of the whole walk
       int committed = 0;
       for (int n = 0; n < nch; ++n) {
         const int st = n % NSTAGE;
@@ -415,16 +430,26 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
             *reinterpret_cast<float4*>(a.state_out + state_at(row) + 16 * g + e) =
                 make_float4(S[g][e], S[g][e + 1], S[g][e + 2], S[g][e + 3]);
     };
-    // sequences without tokens keep their state (state_in, or zeros, to state_out)
-    if (a.state_out)
-      for (int sq = 0; sq < a.n_seqs; ++sq) {
-        const int row = pool_row(a.slots, sq, a.pool_size);
-        int st, en;
-        seq_range(a.cu, a.total, sq, st, en);
-        if (row < 0 || en > st) continue;
-        load_state(row);
-        store_state(row);
+    // sequences without tokens keep their state (state_in, or zeros, to state_out); past
+    // MAX_EMPTY of them the list is incomplete and the batch is walked instead
+    if (a.state_out) {
+      if (n_empty <= MAX_EMPTY) {
+        for (int e = 0; e < n_empty; ++e) {
+          const int row = pool_row(a.slots, empty_seq[e], a.pool_size);
+          load_state(row);
+          store_state(row);
+        }
+      } else {
+        for (int sq = 0; sq < a.n_seqs; ++sq) {
+          const int row = pool_row(a.slots, sq, a.pool_size);
+          int st, en;
+          seq_range(a.cu, a.total, sq, st, en);
+          if (row < 0 || en > st) continue;
+          load_state(row);
+          store_state(row);
+        }
       }
+    }
     auto write_state = [&]() {   // key row i, 16 columns per group: two 16-byte chunks each
 #pragma unroll
       for (int g = 0; g < 3; ++g)

@@ -917,6 +917,10 @@ cudaError_t launch_cosched_t(const PrefillArgs& a, cudaStream_t st, bool* launch
   // would lose too many SMs: the separate launches are faster in both cases.
   const int nchain = a.H;
   if (4 * nchain > nsm || 5 * nchain < nsm) return cudaSuccess;
+  // a chain walks the batch's sequences one after another, paying a state read and write
+  // at each boundary: with sequences of fewer than 4 chunks on average the chains would
+  // set the pace, and the separate launches run them side by side instead
+  if ((long long)a.total < 4LL * C * a.n_seqs) return cudaSuccess;
   ChainMaps maps;
   if (!make_chain_maps(a, &maps)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};

@@ -74,7 +74,7 @@ def test_prefill_varlen_ragged_bf16(d, chunk, fused):
 
 
 @pytest.mark.parametrize('fused', [True, False])
-@pytest.mark.parametrize('seqlens', [[1000], [0, 130, 1, 64, 257, 0, 65], [8192],
+@pytest.mark.parametrize('seqlens', [[1000], [0, 700, 1, 64, 1500, 0, 65], [8192],
                                      [3000, 17, 1500, 64, 2100]])
 def test_cosched_launch_equals_separate_passes(seqlens, fused):
     """The tensor-core prefill as one co-scheduled launch (a full-width inter-chunk chain per
@@ -96,7 +96,7 @@ def test_cosched_launch_equals_separate_passes(seqlens, fused):
     assert torch.equal(y1, y2)
     assert torch.equal(s1, s2)
     assert torch.equal(c1, c2)
-    if sum(seqlens) <= 2048:
+    if sum(seqlens) <= 2400:
         _assert(compare_layer(cfg, P, A, S0, hist, heads=[0, 21], fused=fused), 1e-2)
 
 
@@ -338,22 +338,24 @@ def test_bounded_wait_times_out_and_context_survives():
     assert kda.kda_workspace_status(w2) == kda.KDA_OK
 
 
-@pytest.mark.parametrize('H', [4, 32])
-def test_layer_prefill_launches_and_fused_norm(H):
+@pytest.mark.parametrize('H,seqlens,one_launch', [(4, [300, 264], False), (32, [300, 264], True),
+                                                  (32, [100, 64, 30], False)])
+def test_layer_prefill_launches_and_fused_norm(H, seqlens, one_launch):
     """bf16, d = 128, chunk 64, conv 4: prep runs inside the intra-chunk pass and the gated
-    norm inside the inter-chunk pass.  With H near a fifth to a quarter of the SMs (32 on a
-    B200) both passes share one co-scheduled launch, otherwise (and with
-    KDA_LAUNCH_SEPARATE_PASSES) they are two kernels.  The conv-state commit adds one launch
-    when a conv state is given."""
-    cfg, P, A, S0, hist = make_case(21, [300, 64], H, 128, 4, torch.bfloat16, state_var=0.01,
+    norm inside the inter-chunk pass.  With H between a fifth and a quarter of the SMs (32 on
+    a B200) and sequences of 4 chunks or more on average, both passes share one co-scheduled
+    launch; otherwise (and with KDA_LAUNCH_SEPARATE_PASSES) they are two kernels.  The
+    conv-state commit adds one launch when a conv state is given."""
+    cfg, P, A, S0, hist = make_case(21, seqlens, H, 128, 4, torch.bfloat16, state_var=0.01,
                                     conv_hist=True, chunk=64)
+    N = len(seqlens)
     sep = dataclasses.replace(cfg, launch_flags=kda.KDA_LAUNCH_SEPARATE_PASSES)
     Pd = {k: v.cuda() for k, v in P.items()}
     Ad = {k: v.cuda() for k, v in A.items()}
-    one = 1 if H == 32 else 2
+    one = 1 if one_launch else 2
     for c, n_pass in ((cfg, one), (sep, 2)):
         n0 = kda.kda_launch_count()
-        kda.layer_prefill(c, Pd, Ad, state_out=torch.empty(2, H, 128, 128, device='cuda'))
+        kda.layer_prefill(c, Pd, Ad, state_out=torch.empty(N, H, 128, 128, device='cuda'))
         assert kda.kda_launch_count() - n0 == n_pass
     n0 = kda.kda_launch_count()
     y, s_out, cs, _ = gpu_layer(cfg, P, A, S0, hist, fused=True)
@@ -894,7 +896,7 @@ def test_cosched_pool_slots_with_a_skipped_sequence():
     """The co-scheduled launch with a state pool: a sequence mapped to slot -1 is skipped
     (its chain CTA returns, the intra-chunk role skips its tiles) and the pool rows no
     sequence maps to stay as they were; everything equals the separate launches bit for bit."""
-    seqlens, H, d, pool = [200, 70, 131], 32, 128, 6
+    seqlens, H, d, pool = [600, 70, 331], 32, 128, 6
     cfg, P, A, _, _ = make_case(31, seqlens, H, d, 4, torch.bfloat16, chunk=64)
     sep = dataclasses.replace(cfg, launch_flags=kda.KDA_LAUNCH_SEPARATE_PASSES)
     dev = 'cuda'
