@@ -1,25 +1,28 @@
-// The inter-chunk chain of the co-scheduled prefill (sm_100a): one CTA carries one
-// (head, sequence) through its chunks with all 128 value columns of the state, so the
-// 32 heads of a sequence need 32 SMs and the rest of the GPU runs the intra-chunk pass
-// in the same launch.  Per chunk (C = 64 tokens), with S the bf16 copy of the state
-// (128 keys x 128 values) and the chunk's tiles from the intra-chunk pass:
+// The inter-chunk chain of the co-scheduled prefill (sm_100a): one CTA carries one head
+// through every sequence of the batch, chunk by chunk, with all 128 value columns of the
+// state, so H heads need H SMs and the rest of the GPU runs the intra-chunk pass in the
+// same launch.  Per chunk (C = 64 tokens), with S the bf16 copy of the state (128 keys x
+// 128 values) and the chunk's tiles from the intra-chunk pass:
 //   MMA1   D1[128 x 128] = [W ; Q~] (128 x 128) . S      rows 0-63: W S, rows 64-127: Q~ S
 //   E1     U = U~ - W S (fp32, rows past the sequence end forced to 0) -> bf16 U in smem
 //   MMA2   D2[128 x 128] = K'^T (128 x 64) . U           state increment (key rows)
 //   MMA3   D1[64:128]   += M (64 x 64) . U               O = Q~ S + M U (A = [X ; M], X the
 //                                                         8 KB before M: its rows land in
 //                                                         D1[0:64], already read)
-//   E2     S <- Diag(e^{G_C}) S + D2 in fp32 registers -> bf16 S in smem
-//   E3     y = O / rms(O) * w * sigmoid(g), a token's 128 columns in one thread
+//   E2     S <- Diag(e^{G_C}) S + D2 in fp32 registers -> bf16 S in smem (at a sequence's
+//          end the state goes out and the next sequence's comes in instead)
+//   E3     y = O / rms(O) * w * sigmoid(g), by four warps per TMEM lane quarter 2-3, one
+//          32-column slice each, the sums of squares exchanged through shared memory
 // This is the arithmetic of the 4-slice inter-chunk pass with the slices side by side:
 // each state element takes the same operations in the same order, and E3 sums a
 // token's squares in four 32-column partials, added in slice order, as that pass does.
 // Warp roles: warp 0 waits for each tile's ready flag (written by the intra-chunk
 // CTAs) and loads the chunk with TMA into two stages; warp 1 allocates all 512 TMEM
 // columns (D1 three times, D2) and issues the MMAs from one thread (MMA3 of chunk n
-// after MMA1 of chunk n+1, off the chain; U double-buffered for it); warps 2-3 run E3
-// on TMEM lanes 64-127; warps 4-15 run E1/E2, three per TMEM lane quarter (quarter =
-// warp % 4), owning value columns 0-47, 48-95 and 96-127.  Every wait is bounded.
+// after MMA1 of chunk n+1, off the chain; U double-buffered for it); warps 4-15 run E1/E2,
+// three per TMEM lane quarter (quarter = warp % 4), owning value columns 0-47, 48-95 and
+// 96-127; E3 runs on warps 2-3 (slice 0) and on the E2 warps of quarters 2-3 (slices 1-3,
+// the previous chunk's, after their E2).  Every wait is bounded.
 #pragma once
 
 #include "kda_common.cuh"
