@@ -958,3 +958,33 @@ def test_cosched_launch_in_a_cuda_graph():
         torch.cuda.synchronize()
         assert torch.equal(y, y_ref) and torch.equal(st, st_ref)
     del g
+
+
+def test_cosched_many_empty_sequences_pass_their_state_through():
+    """The co-scheduled launch with more empty sequences than the chain's list holds (they
+    are then found by walking the batch): every empty sequence's state row is copied from
+    state_in to state_out, and the states equal the separate launches' bit for bit.  With
+    2,304 (sequence, head) chains the separate form runs the gated norm as its own kernel
+    (exact sigmoid, another sum order), so y agrees to rounding there."""
+    n_empty, H, d = 70, 32, 128
+    seqlens = [9300] + [0] * n_empty + [9250]
+    N, T = len(seqlens), sum(seqlens)
+    assert T >= 4 * 64 * N                      # long enough on average for one launch
+    cfg = kda.Config(num_heads=H, head_dim=d, conv_size=4, dtype=torch.bfloat16, chunk_size=64)
+    sep = dataclasses.replace(cfg, launch_flags=kda.KDA_LAUNCH_SEPARATE_PASSES)
+    dev = 'cuda'
+    P = {k: v.to(dev) for k, v in synth.layer_params(41, H, d, 4).items()}
+    A = {k: v.to(dev) for k, v in synth.layer_activations(41, seqlens, H, d, torch.bfloat16).items()}
+    s0 = synth.initial_state(41, N, H, d, 0.01).to(dev)
+    outs = []
+    for c in (cfg, sep):
+        st = torch.full_like(s0, float('nan'))
+        n0 = kda.kda_launch_count()
+        y = kda.layer_prefill(c, P, A, state_in=s0, state_out=st)
+        torch.cuda.synchronize()
+        outs.append((y, st, kda.kda_launch_count() - n0))
+    (y1, s1, n1), (y2, s2, n2) = outs
+    assert n1 == 1 and n2 == 3
+    assert torch.equal(s1, s2)
+    assert rel_err(np64(y1), np64(y2)) <= 5e-3
+    assert torch.equal(s1[1:1 + n_empty], s0[1:1 + n_empty])
