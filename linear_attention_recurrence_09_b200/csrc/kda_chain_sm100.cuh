@@ -11,8 +11,8 @@
 //                                                         D1[0:64], already read)
 //   E2     S <- Diag(e^{G_C}) S + D2 in fp32 registers -> bf16 S in smem (at a sequence's
 //          end the state goes out and the next sequence's comes in instead)
-//   E3     y = O / rms(O) * w * sigmoid(g), by four warps per TMEM lane quarter 2-3, one
-//          32-column slice each, the sums of squares exchanged through shared memory
+//   E3     y = O / rms(O) * w * sigmoid(g) on TMEM lane quarters 2-3 in four 32-column
+//          slices, the sums of squares exchanged through shared memory
 // This is the arithmetic of the 4-slice inter-chunk pass with the slices side by side:
 // each state element takes the same operations in the same order, and E3 sums a
 // token's squares in four 32-column partials, added in slice order, as that pass does.
@@ -21,8 +21,9 @@
 // columns (D1 three times, D2) and issues the MMAs from one thread (MMA3 of chunk n
 // after MMA1 of chunk n+1, off the chain; U double-buffered for it); warps 4-15 run E1/E2,
 // three per TMEM lane quarter (quarter = warp % 4), owning value columns 0-47, 48-95 and
-// 96-127; E3 runs on warps 2-3 (slice 0) and on the E2 warps of quarters 2-3 (slices 1-3,
-// the previous chunk's, after their E2).  Every wait is bounded.
+// 96-127; E3 runs on warps 2-3 (slices 0-2) and on the narrowest E2 warps of quarters 2-3
+// (slice 3 of the previous chunk, after their E2), so the other E2 warps of those quarters
+// carry nothing but the chain.  Every wait is bounded.
 #pragma once
 
 #include "kda_common.cuh"
@@ -62,7 +63,7 @@ enum { BAR_FULL0 = 0, BAR_FULL1, BAR_EMPTY0, BAR_EMPTY1, BAR_MMA1, BAR_MMA2, BAR
        BAR_SSQ0, BAR_SSQ1, BAR_SSQ2, BAR_SSQ3, BAR_COUNT };
 static_assert(BAR_COUNT * 8 <= 256, "barrier slots");
 constexpr int NE = 12;        // E1/E2 warps (4..15)
-constexpr int NOUT = 8;       // warps of E3: 2, 3 and the E2 warps of lane quarters 2-3
+constexpr int NOUT = 4;       // warps of E3: 2, 3 and the narrowest E2 warps of quarters 2-3
 
 // sigmoid(z) = (1 + tanh(z / 2)) / 2 with one special-function op (tanh.approx, absolute
 // error about 2^-11): the outputs are bf16 and the output gate's error stays far inside
@@ -192,7 +193,7 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
       mbar_init(bar(BAR_OFREE0 + b), NOUT);
       mbar_init(bar(BAR_ODONE0 + b), 1);
     }
-    for (int b = 0; b < 4; ++b) mbar_init(bar(BAR_SSQ0 + b), 4);   // [quarter 2-3][parity]
+    for (int b = 0; b < 4; ++b) mbar_init(bar(BAR_SSQ0 + b), 2);   // [quarter 2-3][parity]
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (threadIdx.x < D) reinterpret_cast<float*>(sm + OFF_NW)[threadIdx.x] = __ldg(a.norm_w + threadIdx.x);
@@ -379,24 +380,84 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
       }
     }
   } else if (warp < 4) {
-    // ---------------- E3, slice 0 (warps 2, 3), off the serial chain ----------------
+    // ---------------- E3, slices 0-2 (warps 2, 3), off the serial chain ----------------
+    // Per chunk: the three slices' sums of squares into the exchange, then, once the fourth
+    // (from the narrowest E2 warp of the quarter) is in, y for the three slices.
     const int q = warp & 3;
-    ChainPos k, kn;
+    const int r = 32 * (q - 2) + lane;
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    const float* nwb = reinterpret_cast<const float*>(sm + OFF_NW);
+    ChainPos k;
     bool more = chain_seq_from(a, 0, k);
-    uint4 gb[4];
-    if (more) load_gate(k.start, min(C, k.end - k.start), q, 0, gb);
     for (int m = 0; more; ++m) {
       const int t0 = k.start + k.n * C, L = min(C, k.end - t0);
-      kn = k;
-      const bool next = chain_next(a, kn);
-      uint4 gn[4];
-      const int tn = kn.start + kn.n * C;
-      load_gate(tn, next ? min(C, kn.end - tn) : 0, q, 0, gn);   // one chunk ahead
-      if (!o_slice(m, t0, L, q, 0, gb)) break;
+      uint4 gcur[4];    // the gate row's slice 0, in flight through the waits below
+      load_gate(t0, L, q, 0, gcur);
+      if (r < L)        // slices 1-2 (and 3) into L2
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const __nv_bfloat16*>(a.g) +
+                                                       ((size_t)(t0 + r) * H + h) * D + 64));
+      if (!mbar_wait_warp(bar(BAR_ODONE0 + m % 3), (m / 3) & 1, &abort_flag)) break;
+      tc_fence_after();
+      const uint32_t ob = d1_of(m) + lane_off;
+      float* ssq = reinterpret_cast<float*>(sm + OFF_SSQ) + (m & 1) * (C * 4);
+#pragma unroll 1
+      for (int j = 0; j < 3; ++j) {
+        float part = 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) gb[e] = gn[e];
-      k = kn;
-      more = next;
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t o[16];
+          tmem_ld16_issue(ob + 32 * j + 16 * hf, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) part = fmaf(__uint_as_float(o[e]), __uint_as_float(o[e]), part);
+        }
+        ssq[r * 4 + j] = part;
+      }
+      __syncwarp();
+      const uint32_t xb = bar(BAR_SSQ0 + 2 * (q - 2) + (m & 1));
+      if (lane == 0) mbar_arrive(xb);
+      if (!mbar_wait_warp(xb, (m >> 1) & 1, &abort_flag)) break;
+      const float4 pp = *reinterpret_cast<const float4*>(ssq + r * 4);
+      float tot = 0.f;
+      tot += pp.x;
+      tot += pp.y;
+      tot += pp.z;
+      tot += pp.w;
+      const float rstd = rsqrtf(tot * (1.0f / D) + a.norm_eps);
+      uint4* yp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.y) +
+                                           ((size_t)(t0 + r) * H + h) * D);
+#pragma unroll 1
+      for (int j = 0; j < 3; ++j) {
+        uint4 gnext[4];   // the next slice's gate, in flight through this one
+        load_gate(t0, j < 2 ? L : 0, q, j < 2 ? j + 1 : 0, gnext);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t o[16];
+          tmem_ld16_issue(ob + 32 * j + 16 * hf, o);
+          tmem_ld_wait();
+          const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gcur[2 * hf]);
+          uint4 out[2];
+          __nv_bfloat162* y2 = reinterpret_cast<__nv_bfloat162*>(out);
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            const int col = 32 * j + 16 * hf + e;
+            const float2 gf = __bfloat1622float2(g2[e / 2]);
+            y2[e / 2] = __floats2bfloat162_rn(
+                __uint_as_float(o[e]) * rstd * nwb[col] * sigmoid_fast(gf.x),
+                __uint_as_float(o[e + 1]) * rstd * nwb[col + 1] * sigmoid_fast(gf.y));
+          }
+          if (r < L) {
+            yp[4 * j + 2 * hf] = out[0];
+            yp[4 * j + 2 * hf + 1] = out[1];
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) gcur[e] = gnext[e];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_OFREE0 + m % 3));
+      more = chain_next(a, k);
     }
   } else {
     // ---------------- E1 / E2 warps 4..15 ----------------
@@ -482,11 +543,11 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
       // the stage has landed, so the producer saw the tile's ready flag: e^{G_C} is readable
       if (!mbar_wait_warp(bar(BAR_FULL0 + st), (n / NSTAGE) & 1, &abort_flag)) break;
       const float gc = __ldcg(gCg + (size_t)tile_of(k) * D + i);
-      if (q >= 2 && n > 0) {   // the gate slice of the previous chunk's output, into L2
+      if (q >= 2 && part == 2 && n > 0) {   // the previous chunk's gate slice 3, into L2
         const int r = 32 * (q - 2) + lane;
         if (r < pL)
           asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const __nv_bfloat16*>(a.g) +
-                                                         ((size_t)(pt0 + r) * H + h) * D + 32 * (part + 1)));
+                                                         ((size_t)(pt0 + r) * H + h) * D + 96));
       }
       const bool last = k.n + 1 == k.nch;
       if (last && a.state_in) {   // the next sequence's initial state, into L2
@@ -569,17 +630,18 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
         ++k.n;
       }
       write_state();
-      // E3 of the previous chunk (its output product retired before this chunk's MMA2)
-      if (q >= 2 && n > 0) {
-        load_gate(pt0, pL, q, part + 1, gb);
-        if (!o_slice(n - 1, pt0, pL, q, part + 1, gb)) break;
+      // E3 slice 3 of the previous chunk (its output product retired before this chunk's
+      // MMA2), on the narrowest E2 warp of the quarter
+      if (q >= 2 && part == 2 && n > 0) {
+        load_gate(pt0, pL, q, 3, gb);
+        if (!o_slice(n - 1, pt0, pL, q, 3, gb)) break;
       }
       pt0 = t0;
       pL = L;
     }
-    if (q >= 2 && n > 0 && !abort_flag) {
-      load_gate(pt0, pL, q, part + 1, gb);
-      o_slice(n - 1, pt0, pL, q, part + 1, gb);
+    if (q >= 2 && part == 2 && n > 0 && !abort_flag) {
+      load_gate(pt0, pL, q, 3, gb);
+      o_slice(n - 1, pt0, pL, q, 3, gb);
     }
   }
 
