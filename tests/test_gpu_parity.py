@@ -988,3 +988,25 @@ def test_cosched_many_empty_sequences_pass_their_state_through():
     assert torch.equal(s1, s2)
     assert rel_err(np64(y1), np64(y2)) <= 5e-3
     assert torch.equal(s1[1:1 + n_empty], s0[1:1 + n_empty])
+
+
+def test_cosched_without_initial_or_final_state():
+    """The co-scheduled launch with no state_in (zeros) and with no state_out (only y):
+    the same y as the separate launches, bit for bit."""
+    seqlens, H = [700, 900], 32
+    cfg, P, A, _, _ = make_case(43, seqlens, H, 128, 4, torch.bfloat16, chunk=64)
+    sep = dataclasses.replace(cfg, launch_flags=kda.KDA_LAUNCH_SEPARATE_PASSES)
+    Pd = {k: v.cuda() for k, v in P.items()}
+    Ad = {k: v.cuda() for k, v in A.items()}
+    for with_out in (True, False):
+        ys, states = [], []
+        for c in (cfg, sep):
+            st = torch.empty(len(seqlens), H, 128, 128, device='cuda') if with_out else None
+            n0 = kda.kda_launch_count()
+            ys.append(kda.layer_prefill(c, Pd, Ad, state_out=st))
+            torch.cuda.synchronize()
+            assert kda.kda_launch_count() - n0 == (1 if c is cfg else 2)
+            states.append(st)
+        assert torch.equal(ys[0], ys[1])
+        if with_out:
+            assert torch.equal(states[0], states[1])
