@@ -203,10 +203,11 @@ __device__ __forceinline__ f2x ld_shared_f2x(uint32_t saddr) {
 }
 
 
-// The pass on CTA `cta` of `ncta` working CTAs.  Tile n is (head n / slots, slot n % slots)
-// when it runs alone; when it shares the launch with the inter-chunk chains (COSCHED) the
-// tiles go slot by slot (slot n / H, head n % H), so that every head's chunks are done in
-// order, and each tile's word in `flags` is set once all of it has been written.
+// The pass on CTA `cta` of `ncta` working CTAs.  Tile n is (slot n / H, head n % H): the
+// tiles in flight at once cover the same tokens of all heads (neighbouring rows of x in
+// HBM), and every head's chunks complete in order.  When the pass shares the launch with
+// the inter-chunk chains (COSCHED), each tile's word in `flags` is set once all of it has
+// been written.
 template <bool FUSED, bool COSCHED>
 __device__ __forceinline__ void intra_body(const PrefillArgs& a, const int cta, const int ncta,
                                            int* flags) {
@@ -223,8 +224,8 @@ __device__ __forceinline__ void intra_body(const PrefillArgs& a, const int cta, 
 
   const int H = a.H, nslots = a.L.nslots;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  auto head_of = [&](int n) { return COSCHED ? n % H : n / nslots; };
-  auto slot_of = [&](int n) { return COSCHED ? n / H : n % nslots; };
+  auto head_of = [&](int n) { return n % H; };
+  auto slot_of = [&](int n) { return n / H; };
   int* status = reinterpret_cast<int*>(a.ws + a.L.status);
 
   // once per CTA: the MMA barrier and 128 TMEM columns, kept across tiles
