@@ -214,9 +214,9 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const ChainMaps
   int* status = reinterpret_cast<int*>(a.ws + a.L.status);
   auto tile_of = [&](const ChainPos& k) { return (k.start / C + k.s + k.n) * H + h; };
   // E3 of chunk m for the 32 tokens of TMEM lane quarter q (2 or 3) and value columns
-  // 32 j .. 32 j + 31 (slice j), by one warp: the four warps of a quarter each take a slice,
-  // sum their squares, exchange the partials through shared memory (a bounded mbarrier wait)
-  // and add them in slice order.  `gb` holds the slice's gate row.
+  // 32 j .. 32 j + 31 (slice j) by one warp: its squares' partial sum goes into the
+  // exchange beside the other three slices' (from the quarter's dedicated E3 warp), the four
+  // are added in slice order after a bounded mbarrier wait.  `gb` holds the slice's gate row.
   auto o_slice = [&](int m, int t0, int L, int q, int j, const uint4 (&gb)[4]) -> bool {
     if (!mbar_wait_warp(bar(BAR_ODONE0 + m % 3), (m / 3) & 1, &abort_flag)) return false;
     tc_fence_after();
