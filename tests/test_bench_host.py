@@ -70,3 +70,14 @@ def test_dense_tile_flops_and_method_bytes_by_hand():
     assert bench.layer_method_bytes(8192, 1, 32, 128) == 8192 * 32 * 1538 + 32 * 128 * 128 * 4
     r = bench.tensor_roofline(2.25e9, 2.0, 2250.0, 1125.0)
     assert abs(r['frac'] - 5e-4) < 1e-12 and abs(r['frac_sustained'] - 1e-3) < 1e-12
+
+
+def test_cosched_launch_counts_both_passes():
+    # the one co-scheduled launch moves both passes' design bytes and issues both passes' MMAs
+    nb = bench.prefill_bytes(8192, 32, 128)
+    assert nb['prefill_cosched'] == nb['intra_chunk'] + nb['inter_chunk']
+    f = bench.prefill_mma_flops(8192, 32, 128)
+    for kind in ('tf32', 'bf16'):
+        assert f['prefill_cosched'][kind] == f['intra_chunk'][kind] + f['inter_chunk'][kind]
+    # the two-launch form's keys are still there for the separate-passes line
+    assert set(nb) >= {'intra_chunk', 'inter_chunk', 'layer'}
