@@ -1010,3 +1010,27 @@ def test_cosched_without_initial_or_final_state():
         assert torch.equal(ys[0], ys[1])
         if with_out:
             assert torch.equal(states[0], states[1])
+
+
+@pytest.mark.parametrize('fused', [True, False])
+def test_l2_eps_edge_rows_cosched(fused):
+    """The zero / below-eps q and k rows at 32 heads, where both passes run in one
+    co-scheduled launch: heads 0-3 (the edge rows) against the oracle, on the whole output
+    of those heads and on each edge region by itself."""
+    T, H, d = 300, 32, 128
+    cfg, P, A, S0, _ = make_case(35, [T], H, d, 4, torch.bfloat16, state_var=0.01, chunk=64)
+    x = A['x'].clone()
+    for h, seg, t0, t1, sc in EDGE_ROWS:
+        x[t0:t1, h, seg * d:(seg + 1) * d] *= sc
+    A['x'] = x
+    n0 = kda.kda_launch_count()
+    y, s_out, _, _ = gpu_layer(cfg, P, A, S0, None, fused=fused)
+    # one co-scheduled launch, plus the conv-state commit (and, unfused, the prep itself)
+    assert kda.kda_launch_count() - n0 == (2 if fused else 3)
+    heads = [0, 1, 2, 3]
+    ref = oracle_layer(cfg, P, A, S0, None, heads)
+    yg = np64(y)[:, heads]
+    assert rel_err(yg, ref['y']) <= 1e-2
+    assert rel_err(np64(s_out)[:, heads], ref['state']) <= 1e-2
+    for h, rows in _edge_regions():
+        assert rel_err(yg[rows, h], ref['y'][rows, h]) <= 1e-2, (h, rows)
