@@ -1034,3 +1034,18 @@ def test_l2_eps_edge_rows_cosched(fused):
     assert rel_err(np64(s_out)[:, heads], ref['state']) <= 1e-2
     for h, rows in _edge_regions():
         assert rel_err(yg[rows, h], ref['y'][rows, h]) <= 1e-2, (h, rows)
+
+
+@pytest.mark.parametrize('q_scale', [128 ** -0.5, 2.0])
+def test_q_scale_cosched(q_scale):
+    """q_scale != 1 at 32 heads, through the co-scheduled launch, with the RMSNorm eps at
+    1e3 so that y is proportional to o (a lost or doubled q_scale moves y by its factor);
+    two heads against the oracle."""
+    cfg, P, A, S0, hist = make_case(17, [300, 270], 32, 128, 4, torch.bfloat16, state_var=0.01,
+                                    conv_hist=True, chunk=64)
+    cfg.q_scale = q_scale
+    cfg.norm_eps = 1e3
+    n0 = kda.kda_launch_count()
+    errs = compare_layer(cfg, P, A, S0, hist, heads=[5, 30], fused=True)
+    assert kda.kda_launch_count() - n0 == 2        # one co-scheduled launch + conv commit
+    _assert(errs, 1e-2)
