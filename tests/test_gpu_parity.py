@@ -1049,3 +1049,17 @@ def test_q_scale_cosched(q_scale):
     errs = compare_layer(cfg, P, A, S0, hist, heads=[5, 30], fused=True)
     assert kda.kda_launch_count() - n0 == 2        # one co-scheduled launch + conv commit
     _assert(errs, 1e-2)
+
+
+def test_maximal_decay_gate_cosched():
+    """Every gate at its lower bound (log a = -5 per token and channel) at 32 heads, through
+    the co-scheduled launch: the widest exponent range inside a chunk; two heads against
+    the oracle, and the same bits as the separate launches."""
+    cfg, P, A, S0, hist = make_case(15, [300, 130], 32, 128, 4, torch.bfloat16, state_var=0.01,
+                                    conv_hist=True, chunk=64)
+    A['f'] = torch.full_like(A['f'], 30.0)
+    sep = dataclasses.replace(cfg, launch_flags=kda.KDA_LAUNCH_SEPARATE_PASSES)
+    y1, s1, c1, _ = gpu_layer(cfg, P, A, S0, hist)
+    y2, s2, c2, _ = gpu_layer(sep, P, A, S0, hist)
+    assert torch.equal(y1, y2) and torch.equal(s1, s2) and torch.equal(c1, c2)
+    _assert(compare_layer(cfg, P, A, S0, hist, heads=[0, 17]), 1e-2)
